@@ -1,0 +1,143 @@
+"""float64 CPU oracle for the Gated DeltaNet recurrence (test infrastructure).
+
+Only the tests, ``__graft_entry__.smoke()`` and the CPU-baseline leg of
+``bench.py`` may import this package.  The product path (the CUDA library and
+its Python binding) never imports, links or runs it, and it imports nothing
+from the product package: callers hand it numpy arrays.
+
+The arithmetic lives in ``gdn_oracle.c`` (plain C, float64, one token at a
+time).  This module compiles it with gcc on first use and wraps the two entry
+points with ctypes.  See ``gdn_oracle.c`` for the pages each step follows.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "gdn_oracle.c")
+_LIB = os.path.join(_HERE, "liboracle.so")
+_lib = None
+
+
+def build(force: bool = False) -> str:
+    """Compile ``liboracle.so`` next to its source (gcc, -O2, OpenMP)."""
+    if force or not os.path.exists(_LIB) or os.path.getmtime(_LIB) < os.path.getmtime(_SRC):
+        tmp = _LIB + f".tmp{os.getpid()}"
+        subprocess.check_call(
+            ["gcc", "-O2", "-std=c11", "-fopenmp", "-fPIC", "-shared", _SRC, "-o", tmp, "-lm"]
+        )
+        os.replace(tmp, _LIB)
+    return _LIB
+
+
+def _load():
+    global _lib
+    if _lib is None:
+        lib = ctypes.CDLL(build())
+        D = ctypes.POINTER(ctypes.c_double)
+        I32 = ctypes.POINTER(ctypes.c_int32)
+        lib.oracle_prefill.restype = None
+        lib.oracle_prefill.argtypes = [
+            D, D, D, D, D, I32, D, D, D,
+            ctypes.c_int, ctypes.c_int64, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int,
+            ctypes.c_double, ctypes.c_int, ctypes.c_int,
+        ]
+        lib.oracle_decode.restype = None
+        lib.oracle_decode.argtypes = [
+            D, D, D, D, D, ctypes.c_int, I32, I32, I32,
+            D, D, D, D, ctypes.c_double, D,
+            ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int,
+            ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int,
+        ]
+        lib.oracle_max_threads.restype = ctypes.c_int
+        lib.oracle_max_threads.argtypes = []
+        _lib = lib
+    return _lib
+
+
+def max_threads() -> int:
+    return int(_load().oracle_max_threads())
+
+
+def _f64(x):
+    return np.ascontiguousarray(np.asarray(x, dtype=np.float64))
+
+
+def _i32(x):
+    return np.ascontiguousarray(np.asarray(x, dtype=np.int32))
+
+
+def _dp(a):
+    return None if a is None else a.ctypes.data_as(ctypes.POINTER(ctypes.c_double))
+
+
+def _ip(a):
+    return None if a is None else a.ctypes.data_as(ctypes.POINTER(ctypes.c_int32))
+
+
+def prefill(q, k, v, g, beta, cu_seqlens=None, initial_state=None, *, B=None,
+            scale=1.0, qk_l2norm=False, out=None, threads=None):
+    """Sequential recurrence of the log-space form, float64.
+
+    q, k: [N, Hq, Dk]; v: [N, Hv, Dv]; g, beta: [N, Hv];
+    cu_seqlens: [B+1] int32 or None (uniform packing, needs ``B``);
+    initial_state: [B, Hv, Dv, Dk] or None.
+    ``out`` (optional, [N, Hv, Dv] float64) supplies the values kept for
+    tokens that no request covers.
+    Returns (out [N, Hv, Dv], final_state [B, Hv, Dv, Dk]) as float64.
+    """
+    q, k, v, g, beta = map(_f64, (q, k, v, g, beta))
+    N, Hq, Dk = q.shape
+    Hv, Dv = v.shape[1], v.shape[2]
+    if cu_seqlens is not None:
+        cu = _i32(cu_seqlens)
+        B = cu.shape[0] - 1
+    else:
+        cu = None
+        assert B is not None and N % B == 0
+    s0 = None if initial_state is None else _f64(initial_state)
+    fs = np.zeros((B, Hv, Dv, Dk), np.float64)
+    o = np.zeros((N, Hv, Dv), np.float64) if out is None else _f64(out).copy()
+    nt = threads if threads is not None else max_threads()
+    _load().oracle_prefill(_dp(q), _dp(k), _dp(v), _dp(g), _dp(beta), _ip(cu), _dp(s0),
+                           _dp(fs), _dp(o), B, N, Hq, Hv, Dk, Dv, float(scale),
+                           int(bool(qk_l2norm)), int(nt))
+    return o, fs
+
+
+def decode(q, k, v, pool, read_idx, A_log, a, dt_bias, b, *, write_idx=None,
+           scatter_idx=None, scale=None, use_qk_l2norm=True, disable_state_update=False,
+           out=None, threads=None):
+    """Decode / MTP over a slot pool, float64.
+
+    q: [B, T, H, Dk]; k: [B, T, nh, H, Dk]; v: [B, T, nh, HV, Dv];
+    pool: [P, HV, Dv, Dk]; read_idx, write_idx: [B]; scatter_idx: [B, T];
+    A_log, dt_bias: [HV]; a: [B, T, HV]; b: [B, T, nh, HV].
+    ``scale`` None means 1/sqrt(Dk).  ``out`` supplies the values kept in
+    padding rows (zeros when None).
+    Returns (out [B, T, HV, Dv], new pool [P, HV, Dv, Dk]) as float64.
+    """
+    q, k, v = map(_f64, (q, k, v))
+    Bn, T, H, Dk = q.shape
+    nh = k.shape[2]
+    HV, Dv = v.shape[3], v.shape[4]
+    pin = _f64(pool)
+    pout = pin.copy()
+    P = pin.shape[0]
+    if scale is None:
+        scale = 1.0 / np.sqrt(Dk)
+    o = np.zeros((Bn, T, HV, Dv), np.float64) if out is None else _f64(out).copy()
+    ri = _i32(read_idx)
+    wi = None if write_idx is None else _i32(write_idx)
+    si = None if scatter_idx is None else _i32(scatter_idx)
+    Al, ab, dtb, bb = map(_f64, (A_log, a, dt_bias, b))
+    nt = threads if threads is not None else max_threads()
+    _load().oracle_decode(_dp(q), _dp(k), _dp(v), _dp(pin), _dp(pout), P, _ip(ri), _ip(wi),
+                          _ip(si), _dp(Al), _dp(ab), _dp(dtb), _dp(bb), float(scale), _dp(o),
+                          Bn, T, nh, H, HV, Dk, Dv, int(bool(use_qk_l2norm)),
+                          int(bool(disable_state_update)), int(nt))
+    return o, pout

@@ -1,0 +1,293 @@
+/*
+ * gdn_oracle.c -- float64 CPU oracle for the Gated DeltaNet recurrence.
+ *
+ * TEST INFRASTRUCTURE ONLY.  Nothing on the product path may call, link or
+ * load this file: only the tests, the smoke check and the benchmark's CPU
+ * baseline leg use it.  It shares no code with the CUDA library.
+ *
+ * It is written to be read against the pages, not to be fast: one
+ * (request, value head) or (batch row, head) unit at a time, one token at a
+ * time, every sum in float64, no blocking and no reordering.  OpenMP only
+ * spreads independent units over host threads.
+ *
+ * Sources (pages, by title and section):
+ *  - "com.microsoft.GatedDeltaNet" (ONNX Runtime contrib op), Description:
+ *      S_t = exp(g_t) S_{t-1} + k_t (beta_t (v_t - exp(g_t) S_{t-1}^T k_t))^T,
+ *      o_t = scale * S_t^T q_t, per value head; value head h reads query/key
+ *      head h*Hq/Hv; Inputs table: cu_seqlens clamping, V-major float32
+ *      initial/final state, empty requests copy their state through;
+ *      Attributes table: qk_l2_norm with epsilon 1e-12, scale.
+ *  - "Gated DeltaNet State Update" (tensortonic), statement: the same
+ *      recurrence in the gamma form S_t = gamma_t (I - beta_t k_t k_t^T)
+ *      S_{t-1} + beta_t k_t v_t^T with y_t = q_t^T S_t (gamma_t = exp(g_t)).
+ *  - "flashinfer.cake_gdp.cake_gated_delta_product_mtp", description and
+ *      Parameters: the decode/MTP pool update with the fused gate
+ *      alpha = exp(-exp(A_log) softplus(a + dt_bias)) (softplus threshold 20),
+ *      beta = sigmoid(b) per Householder sub-step, L2 norm x*rsqrt(sum x^2 +
+ *      1e-6), padding rows, write-slot override and per-token scatter.
+ *
+ * Readings where the pages are silent (each one listed in the design notes):
+ *  - the prefill L2 norm is x * (sum x^2 + 1e-12)^(-1/2);
+ *  - h*Hq/Hv is integer floor division;
+ *  - decode reads every row's slot from the pool as it was before the call
+ *    (pool_in) and writes into a separate copy (pool_out); under the
+ *    precondition that no row writes a slot another row reads, this is the
+ *    in-place result;
+ *  - a slot index >= pool_size is treated like a negative one (skipped).
+ *
+ * Parity pins: tests/test_oracle_pins.py checks this file against the worked
+ * examples of "Gated DeltaNet State Update", a brute-force product of the
+ * gamma form, closed forms and invariants.
+ */
+#include <math.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+
+#ifdef _OPENMP
+#include <omp.h>
+#endif
+
+static int64_t clamp_i64(int64_t x, int64_t lo, int64_t hi)
+{
+    return x < lo ? lo : (x > hi ? hi : x);
+}
+
+int oracle_max_threads(void)
+{
+#ifdef _OPENMP
+    return omp_get_max_threads();
+#else
+    return 1;
+#endif
+}
+
+/* ------------------------------------------------------------------------
+ * Prefill.
+ *   q, k          [N, Hq, Dk]
+ *   v, out        [N, Hv, Dv]
+ *   g, beta       [N, Hv]            (log-space decay, update rate)
+ *   cu_seqlens    [B+1] or NULL      (NULL: uniform packing, N = B*S)
+ *   initial_state [B, Hv, Dv, Dk] or NULL (NULL: zero)
+ *   final_state   [B, Hv, Dv, Dk]
+ * The state is held here K-major, S[i][j] with i over Dk and j over Dv, as in
+ * the gamma-form statement; the V-major inputs/outputs are transposed on the
+ * way in and out.
+ * ---------------------------------------------------------------------- */
+void oracle_prefill(const double *q, const double *k, const double *v,
+                    const double *g, const double *beta,
+                    const int32_t *cu_seqlens,
+                    const double *initial_state, double *final_state,
+                    double *out,
+                    int B, int64_t N, int Hq, int Hv, int Dk, int Dv,
+                    double scale, int qk_l2norm, int nthreads)
+{
+    int nunits = B * Hv;
+    if (nthreads <= 0) nthreads = 1;
+
+#pragma omp parallel for schedule(dynamic, 1) num_threads(nthreads)
+    for (int unit = 0; unit < nunits; ++unit) {
+        int b = unit / Hv;
+        int h = unit % Hv;
+        int qh = (int)(((int64_t)h * Hq) / Hv);   /* floor(h * Hq / Hv) */
+
+        int64_t start, end;
+        if (cu_seqlens) {
+            start = clamp_i64(cu_seqlens[b], 0, N);
+            end = clamp_i64(cu_seqlens[b + 1], 0, N);
+        } else {
+            int64_t S = N / B;
+            start = (int64_t)b * S;
+            end = start + S;
+        }
+
+        double *S = (double *)calloc((size_t)Dk * Dv, sizeof(double));
+        double *xq = (double *)malloc(sizeof(double) * Dk);
+        double *xk = (double *)malloc(sizeof(double) * Dk);
+        double *p = (double *)malloc(sizeof(double) * Dv);
+
+        /* S_0 = initial_state[b, h]^T, or zero. */
+        if (initial_state) {
+            const double *s0 = initial_state + ((int64_t)b * Hv + h) * Dv * Dk;
+            for (int i = 0; i < Dk; ++i)
+                for (int j = 0; j < Dv; ++j)
+                    S[(int64_t)i * Dv + j] = s0[(int64_t)j * Dk + i];
+        }
+
+        for (int64_t t = start; t < end; ++t) {
+            const double *qt = q + (t * Hq + qh) * Dk;
+            const double *kt = k + (t * Hq + qh) * Dk;
+            const double *vt = v + (t * Hv + h) * Dv;
+            for (int i = 0; i < Dk; ++i) {
+                xq[i] = qt[i];
+                xk[i] = kt[i];
+            }
+            if (qk_l2norm) {
+                double sq = 0.0, sk = 0.0;
+                for (int i = 0; i < Dk; ++i) {
+                    sq += xq[i] * xq[i];
+                    sk += xk[i] * xk[i];
+                }
+                double rq = 1.0 / sqrt(sq + 1e-12);
+                double rk = 1.0 / sqrt(sk + 1e-12);
+                for (int i = 0; i < Dk; ++i) {
+                    xq[i] *= rq;
+                    xk[i] *= rk;
+                }
+            }
+            double gamma = exp(g[t * Hv + h]);
+            double bt = beta[t * Hv + h];
+
+            /* p = S_{t-1}^T k_t */
+            for (int j = 0; j < Dv; ++j) {
+                double acc = 0.0;
+                for (int i = 0; i < Dk; ++i) acc += S[(int64_t)i * Dv + j] * xk[i];
+                p[j] = acc;
+            }
+            /* S_t = gamma S_{t-1} + k_t (beta (v_t - gamma p))^T */
+            for (int i = 0; i < Dk; ++i)
+                for (int j = 0; j < Dv; ++j) {
+                    double u = bt * (vt[j] - gamma * p[j]);
+                    S[(int64_t)i * Dv + j] = gamma * S[(int64_t)i * Dv + j] + xk[i] * u;
+                }
+            /* o_t = scale * S_t^T q_t */
+            double *ot = out + (t * Hv + h) * Dv;
+            for (int j = 0; j < Dv; ++j) {
+                double acc = 0.0;
+                for (int i = 0; i < Dk; ++i) acc += S[(int64_t)i * Dv + j] * xq[i];
+                ot[j] = scale * acc;
+            }
+        }
+
+        /* final_state[b, h] = S^T (V-major). */
+        double *sf = final_state + ((int64_t)b * Hv + h) * Dv * Dk;
+        for (int j = 0; j < Dv; ++j)
+            for (int i = 0; i < Dk; ++i)
+                sf[(int64_t)j * Dk + i] = S[(int64_t)i * Dv + j];
+
+        free(S);
+        free(xq);
+        free(xk);
+        free(p);
+    }
+}
+
+/* ------------------------------------------------------------------------
+ * Decode / MTP (Gated DeltaProduct with num_householder = nh sub-steps).
+ *   q        [B, T, H, Dk]
+ *   k        [B, T, nh, H, Dk]
+ *   v        [B, T, nh, HV, Dv]
+ *   pool_in  [P, HV, Dv, Dk]   slots as they were before the call
+ *   pool_out [P, HV, Dv, Dk]   receives write-backs / scatters (the caller
+ *                              starts it as a copy of pool_in)
+ *   read_idx [B]; write_idx [B] or NULL (= read_idx); scatter_idx [B, T] or NULL
+ *   A_log, dt_bias [HV]; a [B, T, HV]; bgate [B, T, nh, HV]
+ *   out      [B, T, HV, Dv]    rows whose read slot is skipped are not written
+ * H must equal HV (no grouping on this path); head h reads q/k head h.
+ * ---------------------------------------------------------------------- */
+static double softplus_thr20(double x)
+{
+    return x > 20.0 ? x : log1p(exp(x));
+}
+
+void oracle_decode(const double *q, const double *k, const double *v,
+                   const double *pool_in, double *pool_out, int pool_size,
+                   const int32_t *read_idx, const int32_t *write_idx,
+                   const int32_t *scatter_idx,
+                   const double *A_log, const double *a, const double *dt_bias,
+                   const double *bgate, double scale, double *out,
+                   int B, int T, int nh, int H, int HV, int Dk, int Dv,
+                   int use_qk_l2norm, int disable_state_update, int nthreads)
+{
+    int nunits = B * HV;
+    int64_t slot_elems = (int64_t)HV * Dv * Dk;
+    (void)H;
+    if (nthreads <= 0) nthreads = 1;
+
+#pragma omp parallel for schedule(dynamic, 1) num_threads(nthreads)
+    for (int unit = 0; unit < nunits; ++unit) {
+        int b = unit / HV;
+        int h = unit % HV;
+        int r = read_idx[b];
+        if (r < 0 || r >= pool_size) continue;   /* padding row: nothing at all */
+
+        double *S = (double *)malloc(sizeof(double) * Dk * Dv);
+        double *xq = (double *)malloc(sizeof(double) * Dk);
+        double *xk = (double *)malloc(sizeof(double) * Dk);
+        double *p = (double *)malloc(sizeof(double) * Dv);
+
+        const double *s0 = pool_in + r * slot_elems + (int64_t)h * Dv * Dk;
+        for (int i = 0; i < Dk; ++i)
+            for (int j = 0; j < Dv; ++j)
+                S[(int64_t)i * Dv + j] = s0[(int64_t)j * Dk + i];
+
+        for (int t = 0; t < T; ++t) {
+            int64_t bt = (int64_t)b * T + t;
+            /* alpha_t = exp(-exp(A_log) * softplus(a_t + dt_bias)) */
+            double alpha = exp(-exp(A_log[h]) * softplus_thr20(a[bt * HV + h] + dt_bias[h]));
+            for (int64_t e = 0; e < (int64_t)Dk * Dv; ++e) S[e] *= alpha;
+
+            for (int j = 0; j < nh; ++j) {
+                const double *kt = k + ((bt * nh + j) * H + h) * Dk;
+                const double *vt = v + ((bt * nh + j) * HV + h) * Dv;
+                double bta = 1.0 / (1.0 + exp(-bgate[(bt * nh + j) * HV + h]));
+                for (int i = 0; i < Dk; ++i) xk[i] = kt[i];
+                if (use_qk_l2norm) {
+                    double s = 0.0;
+                    for (int i = 0; i < Dk; ++i) s += xk[i] * xk[i];
+                    double rn = 1.0 / sqrt(s + 1e-6);
+                    for (int i = 0; i < Dk; ++i) xk[i] *= rn;
+                }
+                /* one Householder-style delta sub-step: S += k (beta (v - S^T k))^T */
+                for (int jv = 0; jv < Dv; ++jv) {
+                    double acc = 0.0;
+                    for (int i = 0; i < Dk; ++i) acc += S[(int64_t)i * Dv + jv] * xk[i];
+                    p[jv] = acc;
+                }
+                for (int i = 0; i < Dk; ++i)
+                    for (int jv = 0; jv < Dv; ++jv)
+                        S[(int64_t)i * Dv + jv] += xk[i] * (bta * (vt[jv] - p[jv]));
+            }
+
+            const double *qt = q + (bt * H + h) * Dk;
+            for (int i = 0; i < Dk; ++i) xq[i] = qt[i];
+            if (use_qk_l2norm) {
+                double s = 0.0;
+                for (int i = 0; i < Dk; ++i) s += xq[i] * xq[i];
+                double rn = 1.0 / sqrt(s + 1e-6);
+                for (int i = 0; i < Dk; ++i) xq[i] *= rn;
+            }
+            double *ot = out + (bt * HV + h) * Dv;
+            for (int jv = 0; jv < Dv; ++jv) {
+                double acc = 0.0;
+                for (int i = 0; i < Dk; ++i) acc += S[(int64_t)i * Dv + jv] * xq[i];
+                ot[jv] = scale * acc;
+            }
+
+            if (scatter_idx && !disable_state_update) {
+                int s = scatter_idx[bt];
+                if (s >= 0 && s < pool_size) {
+                    double *dst = pool_out + s * slot_elems + (int64_t)h * Dv * Dk;
+                    for (int jv = 0; jv < Dv; ++jv)
+                        for (int i = 0; i < Dk; ++i)
+                            dst[(int64_t)jv * Dk + i] = S[(int64_t)i * Dv + jv];
+                }
+            }
+        }
+
+        if (!scatter_idx && !disable_state_update) {
+            int w = write_idx ? write_idx[b] : r;
+            if (w >= 0 && w < pool_size) {
+                double *dst = pool_out + w * slot_elems + (int64_t)h * Dv * Dk;
+                for (int jv = 0; jv < Dv; ++jv)
+                    for (int i = 0; i < Dk; ++i)
+                        dst[(int64_t)jv * Dk + i] = S[(int64_t)i * Dv + jv];
+            }
+        }
+
+        free(S);
+        free(xq);
+        free(xk);
+        free(p);
+    }
+}

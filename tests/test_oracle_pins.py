@@ -1,0 +1,350 @@
+"""Pins for the float64 oracle, against things other than the oracle itself.
+
+* the worked examples printed on "Gated DeltaNet State Update" (tests/golden);
+* a brute-force restatement of that page's gamma form,
+  S_t = gamma_t (I - beta_t k_t k_t^T) S_{t-1} + beta_t k_t v_t^T, written as
+  literal Dk x Dk matrix products in numpy (the oracle uses the log-space
+  rank-1 form of "com.microsoft.GatedDeltaNet", so a dropped term, a wrong
+  sign, a transposed state or a wrong GQA index disagrees here);
+* closed forms and invariants (beta = 0, unit keys, orthonormal keys);
+* the cu_seqlens clamping and empty-request rules of the op's Inputs table;
+* for decode, a brute-force DeltaProduct step with the fused gate restated in
+  numpy from "flashinfer.cake_gdp.cake_gated_delta_product_mtp".
+No test here needs a GPU.
+"""
+import json
+import os
+
+import numpy as np
+import pytest
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden", "p1_worked_examples.json")
+
+
+# ---------------------------------------------------------------- brute force
+def brute_prefill(q, k, v, g, beta, lengths, init, scale, l2norm, Hq, Hv):
+    """gamma form with explicit (I - beta k k^T) products; K-major state."""
+    N = q.shape[0]
+    Dk, Dv = q.shape[2], v.shape[2]
+    B = len(lengths)
+    out = np.zeros((N, Hv, Dv))
+    final = np.zeros((B, Hv, Dv, Dk))
+    off = 0
+    for b, L in enumerate(lengths):
+        for h in range(Hv):
+            qh = (h * Hq) // Hv
+            S = np.zeros((Dk, Dv)) if init is None else init[b, h].T.copy()
+            for t in range(off, off + L):
+                kt = k[t, qh].astype(np.float64)
+                qt = q[t, qh].astype(np.float64)
+                if l2norm:
+                    kt = kt / np.sqrt(kt @ kt + 1e-12)
+                    qt = qt / np.sqrt(qt @ qt + 1e-12)
+                gam = np.exp(g[t, h])
+                bt = beta[t, h]
+                S = gam * (np.eye(Dk) - bt * np.outer(kt, kt)) @ S + bt * np.outer(kt, v[t, h])
+                out[t, h] = scale * (qt @ S)
+            final[b, h] = S.T
+        off += L
+    return out, final
+
+
+def np_softplus20(x):
+    x = np.asarray(x, np.float64)
+    return np.where(x > 20.0, x, np.log1p(np.exp(np.minimum(x, 20.0))))
+
+
+def brute_decode_row(S0_vmajor, qs, ks, vs, a, bgate, A_log, dt_bias, scale, l2):
+    """One (row, head): returns per-token outputs and per-token states (V-major)."""
+    S = S0_vmajor.T.copy()  # K-major
+    Dk = S.shape[0]
+    outs, states = [], []
+    for t in range(qs.shape[0]):
+        alpha = np.exp(-np.exp(A_log) * np_softplus20(a[t] + dt_bias))
+        S = alpha * S
+        for j in range(ks.shape[1]):
+            kj = ks[t, j].astype(np.float64)
+            if l2:
+                kj = kj / np.sqrt(kj @ kj + 1e-6)
+            bj = 1.0 / (1.0 + np.exp(-bgate[t, j]))
+            S = (np.eye(Dk) - bj * np.outer(kj, kj)) @ S + bj * np.outer(kj, vs[t, j])
+        qt = qs[t].astype(np.float64)
+        if l2:
+            qt = qt / np.sqrt(qt @ qt + 1e-6)
+        outs.append(scale * (qt @ S))
+        states.append(S.T.copy())
+    return np.array(outs), states
+
+
+# ------------------------------------------------------------ golden examples
+def test_worked_examples(oracle_mod):
+    ex = json.load(open(GOLDEN))["examples"]
+    assert len(ex) == 3
+    for e in ex:
+        q = np.array(e["q"], np.float64)
+        k = np.array(e["k"], np.float64)
+        v = np.array(e["v"], np.float64)
+        gamma = np.array(e["gamma"], np.float64)
+        beta = np.array(e["beta"], np.float64)
+        B, S, Dk = q.shape
+        Dv = v.shape[2]
+        out, fs = oracle_mod.prefill(q.reshape(B * S, 1, Dk), k.reshape(B * S, 1, Dk),
+                                     v.reshape(B * S, 1, Dv), np.log(gamma).reshape(B * S, 1),
+                                     beta.reshape(B * S, 1), None, None, B=B, scale=1.0)
+        np.testing.assert_allclose(out.reshape(B, S, Dv), np.array(e["outputs"]), atol=1e-12)
+        # V-major [B, 1, Dv, Dk] -> the page's K-major (B, Dk, Dv)
+        np.testing.assert_allclose(fs[:, 0].transpose(0, 2, 1), np.array(e["final_state"]),
+                                   atol=1e-12)
+
+
+# ---------------------------------------------------------------- brute force
+@pytest.mark.parametrize("l2norm", [False, True])
+@pytest.mark.parametrize("Hq,Hv", [(1, 1), (1, 2), (2, 4), (3, 6)])
+def test_prefill_matches_gamma_form(oracle_mod, l2norm, Hq, Hv):
+    rng = np.random.default_rng(100 + Hq * 10 + Hv + int(l2norm))
+    lengths = [5, 1, 9, 4]
+    N, Dk, Dv = sum(lengths), 6, 4
+    q = rng.standard_normal((N, Hq, Dk))
+    k = rng.standard_normal((N, Hq, Dk))
+    if not l2norm:
+        k /= np.linalg.norm(k, axis=-1, keepdims=True)
+    v = rng.standard_normal((N, Hv, Dv))
+    g = -rng.uniform(0.0, 1.5, (N, Hv))
+    beta = rng.uniform(0.0, 1.0, (N, Hv))
+    init = rng.standard_normal((len(lengths), Hv, Dv, Dk))
+    cu = np.concatenate([[0], np.cumsum(lengths)]).astype(np.int32)
+    scale = 0.7
+    out, fs = oracle_mod.prefill(q, k, v, g, beta, cu, init, scale=scale, qk_l2norm=l2norm)
+    bo, bf = brute_prefill(q, k, v, g, beta, lengths, init, scale, l2norm, Hq, Hv)
+    np.testing.assert_allclose(out, bo, rtol=1e-10, atol=1e-12)
+    np.testing.assert_allclose(fs, bf, rtol=1e-10, atol=1e-12)
+
+
+def test_uniform_packing_equals_cu_seqlens(oracle_mod):
+    rng = np.random.default_rng(7)
+    B, S, H, D = 3, 6, 2, 4
+    q, k = rng.standard_normal((2, B * S, H, D))
+    v = rng.standard_normal((B * S, H, D))
+    g = -rng.uniform(0, 1, (B * S, H))
+    beta = rng.uniform(0, 1, (B * S, H))
+    cu = np.arange(0, B * S + 1, S, dtype=np.int32)
+    o1, f1 = oracle_mod.prefill(q, k, v, g, beta, None, None, B=B, qk_l2norm=True)
+    bo, bf = brute_prefill(q, k, v, g, beta, [S] * B, None, 1.0, True, H, H)
+    np.testing.assert_allclose(o1, bo, rtol=1e-10, atol=1e-12)
+    np.testing.assert_allclose(f1, bf, rtol=1e-10, atol=1e-12)
+
+
+# ---------------------------------------------------------------- invariants
+def test_beta0_gamma1_keeps_state(oracle_mod):
+    rng = np.random.default_rng(11)
+    N, Dk, Dv = 7, 5, 3
+    q, k = rng.standard_normal((2, N, 1, Dk))
+    v = rng.standard_normal((N, 1, Dv))
+    init = rng.standard_normal((1, 1, Dv, Dk))
+    out, fs = oracle_mod.prefill(q, k, v, np.zeros((N, 1)), np.zeros((N, 1)), None, init,
+                                 B=1, scale=0.5)
+    np.testing.assert_allclose(fs, init, atol=0, rtol=0)
+    np.testing.assert_allclose(out[:, 0], 0.5 * q[:, 0] @ init[0, 0].T, rtol=1e-13, atol=1e-13)
+
+
+def test_beta0_closed_form_decay(oracle_mod):
+    rng = np.random.default_rng(12)
+    N, Dk, Dv = 9, 4, 4
+    q, k = rng.standard_normal((2, N, 1, Dk))
+    v = rng.standard_normal((N, 1, Dv))
+    g = -rng.uniform(0, 0.5, (N, 1))
+    init = rng.standard_normal((1, 1, Dv, Dk))
+    out, fs = oracle_mod.prefill(q, k, v, g, np.zeros((N, 1)), None, init, B=1, scale=1.0)
+    np.testing.assert_allclose(fs, np.exp(g.sum()) * init, rtol=1e-12)
+    cum = np.cumsum(g[:, 0])
+    np.testing.assert_allclose(out[:, 0], np.exp(cum)[:, None] * (q[:, 0] @ init[0, 0].T),
+                               rtol=1e-12, atol=1e-14)
+
+
+def test_unit_key_beta1_retrieves_value(oracle_mod):
+    """beta = 1 with a unit key makes S_t^T k_t = v_t for any gamma; with q = k the output is v."""
+    rng = np.random.default_rng(13)
+    N, Dk, Dv = 12, 8, 5
+    k = rng.standard_normal((N, 1, Dk))
+    k /= np.linalg.norm(k, axis=-1, keepdims=True)
+    v = rng.standard_normal((N, 1, Dv))
+    g = -rng.uniform(0, 2, (N, 1))
+    init = rng.standard_normal((1, 1, Dv, Dk))
+    out, _ = oracle_mod.prefill(k, k, v, g, np.ones((N, 1)), None, init, B=1, scale=1.0)
+    np.testing.assert_allclose(out, v, rtol=1e-11, atol=1e-12)
+
+
+def test_orthonormal_keys_lookup(oracle_mod):
+    Dk, Dv = 6, 3
+    rng = np.random.default_rng(14)
+    E = np.eye(Dk)
+    v = rng.standard_normal((Dk, 1, Dv))
+    k = E[:, None, :]
+    out, fs = oracle_mod.prefill(k, k, v, np.zeros((Dk, 1)), np.ones((Dk, 1)), None, None,
+                                 B=1, scale=1.0)
+    np.testing.assert_allclose(out, v, atol=1e-15)
+    np.testing.assert_allclose(fs[0, 0], v[:, 0, :].T, atol=1e-15)  # V-major: [Dv, Dk]
+
+
+# ---------------------------------------------------------- cu_seqlens rules
+def test_cu_seqlens_clamp_and_empty(oracle_mod):
+    rng = np.random.default_rng(15)
+    N, H, D = 10, 1, 3
+    q, k = rng.standard_normal((2, N, H, D))
+    v = rng.standard_normal((N, H, D))
+    g = -rng.uniform(0, 1, (N, H))
+    beta = rng.uniform(0, 1, (N, H))
+    init = rng.standard_normal((4, H, D, D))
+    sentinel = np.full((N, H, D), 123.0)
+    # request 0: [0,4); request 1: decreasing -> empty; request 2: [2, 10) clamped from 99;
+    # request 3: [-5 -> 0, 0) empty
+    cu = np.array([0, 4, 2, 99, -5], np.int32)
+    out, fs = oracle_mod.prefill(q, k, v, g, beta, cu, init, out=sentinel, qk_l2norm=True)
+    o0, f0 = brute_prefill(q[:4], k[:4], v[:4], g[:4], beta[:4], [4], init[0:1], 1.0, True, 1, 1)
+    o2, f2 = brute_prefill(q[2:], k[2:], v[2:], g[2:], beta[2:], [8], init[2:3], 1.0, True, 1, 1)
+    np.testing.assert_allclose(fs[0], f0[0], rtol=1e-12)
+    np.testing.assert_array_equal(fs[1], init[1])       # empty request copies its state
+    np.testing.assert_allclose(fs[2], f2[0], rtol=1e-12)
+    np.testing.assert_array_equal(fs[3], init[3])
+    np.testing.assert_allclose(out[4:], o2[2:], rtol=1e-12)
+
+
+def test_split_and_resume(oracle_mod):
+    rng = np.random.default_rng(16)
+    N, Hq, Hv, D = 20, 1, 2, 4
+    q, k = rng.standard_normal((2, N, Hq, D))
+    v = rng.standard_normal((N, Hv, D))
+    g = -rng.uniform(0, 1, (N, Hv))
+    beta = rng.uniform(0, 1, (N, Hv))
+    init = rng.standard_normal((1, Hv, D, D))
+    o, f = oracle_mod.prefill(q, k, v, g, beta, None, init, B=1, qk_l2norm=True)
+    n = 7
+    oa, fa = oracle_mod.prefill(q[:n], k[:n], v[:n], g[:n], beta[:n], None, init, B=1,
+                                qk_l2norm=True)
+    ob, fb = oracle_mod.prefill(q[n:], k[n:], v[n:], g[n:], beta[n:], None, fa, B=1,
+                                qk_l2norm=True)
+    np.testing.assert_allclose(np.concatenate([oa, ob]), o, rtol=1e-12, atol=1e-14)
+    np.testing.assert_allclose(fb, f, rtol=1e-12, atol=1e-14)
+
+
+# -------------------------------------------------------------------- decode
+def _decode_inputs(rng, B, T, nh, H, Dk, Dv, P):
+    q = rng.standard_normal((B, T, H, Dk))
+    k = rng.standard_normal((B, T, nh, H, Dk))
+    v = rng.standard_normal((B, T, nh, H, Dv))
+    pool = rng.standard_normal((P, H, Dv, Dk)) * 0.3
+    A_log = rng.uniform(-2, 1, H)
+    dt_bias = rng.standard_normal(H) * 0.5
+    a = rng.standard_normal((B, T, H))
+    b = rng.standard_normal((B, T, nh, H))
+    return q, k, v, pool, A_log, dt_bias, a, b
+
+
+@pytest.mark.parametrize("nh", [1, 2, 3])
+def test_decode_matches_bruteforce(oracle_mod, nh):
+    rng = np.random.default_rng(20 + nh)
+    B, T, H, Dk, Dv, P = 4, 3, 2, 8, 4, 12
+    q, k, v, pool, A_log, dt_bias, a, b = _decode_inputs(rng, B, T, nh, H, Dk, Dv, P)
+    a[0, 1, 0] = 25.0  # softplus threshold branch
+    read = np.array([3, -1, 7, 0], np.int32)
+    write = np.array([5, 9, -1, 0], np.int32)
+    sentinel = np.full((B, T, H, Dv), -7.0)
+    out, newpool = oracle_mod.decode(q, k, v, pool, read, A_log, a, dt_bias, b, write_idx=write,
+                                     scale=0.4, out=sentinel)
+    expect_pool = pool.copy()
+    for row in range(B):
+        if read[row] < 0:
+            np.testing.assert_array_equal(out[row], sentinel[row])  # padding row untouched
+            continue
+        for h in range(H):
+            o, states = brute_decode_row(pool[read[row], h], q[row, :, h], k[row, :, :, h],
+                                         v[row, :, :, h], a[row, :, h], b[row, :, :, h],
+                                         A_log[h], dt_bias[h], 0.4, True)
+            np.testing.assert_allclose(out[row, :, h], o, rtol=1e-10, atol=1e-12)
+            if write[row] >= 0:
+                expect_pool[write[row], h] = states[-1]
+    np.testing.assert_allclose(newpool, expect_pool, rtol=1e-10, atol=1e-12)
+    # slot 9 is written by padding row 1, which must skip everything
+    np.testing.assert_array_equal(newpool[9], pool[9])
+
+
+def test_decode_softplus_threshold_exact(oracle_mod):
+    """x > 20 takes softplus(x) = x: alpha = exp(-exp(A_log) * x) exactly."""
+    B, T, nh, H, Dk, Dv = 1, 1, 1, 1, 4, 2
+    q = np.zeros((B, T, H, Dk)); q[..., 0] = 1
+    k = np.zeros((B, T, nh, H, Dk)); k[..., 1] = 1
+    v = np.zeros((B, T, nh, H, Dv))
+    pool = np.zeros((1, H, Dv, Dk)); pool[0, 0, :, 0] = [1.0, 2.0]
+    b = np.full((B, T, nh, H), -1e4)    # sigmoid -> 0: no write
+    out, newpool = oracle_mod.decode(q, k, v, pool, np.array([0], np.int32), np.array([0.0]),
+                                     np.full((B, T, H), 20.5), np.array([0.0]), b, scale=1.0,
+                                     use_qk_l2norm=False)
+    alpha = np.exp(-20.5)
+    np.testing.assert_allclose(out[0, 0, 0], alpha * np.array([1.0, 2.0]), rtol=1e-14)
+
+
+def test_decode_deltaproduct_reductions(oracle_mod):
+    rng = np.random.default_rng(30)
+    B, T, H, Dk, Dv, P = 2, 2, 2, 8, 4, 4
+    q, k, v, pool, A_log, dt_bias, a, b = _decode_inputs(rng, B, T, 2, H, Dk, Dv, P)
+    read = np.array([0, 1], np.int32)
+    # nh=2 with beta_1 = sigmoid(-1e4) = 0 equals nh=1
+    b2 = b.copy()
+    b2[:, :, 1] = -1e4
+    o2, p2 = oracle_mod.decode(q, k, v, pool, read, A_log, a, dt_bias, b2)
+    o1, p1 = oracle_mod.decode(q, k[:, :, :1], v[:, :, :1], pool, read, A_log, a, dt_bias,
+                               b[:, :, :1])
+    np.testing.assert_allclose(o2, o1, rtol=1e-12, atol=1e-14)
+    np.testing.assert_allclose(p2, p1, rtol=1e-12, atol=1e-14)
+    # nh=2 with k_1 = k_0, beta = 1: the second value overwrites; with q = k the readout is v_1
+    # (unit keys supplied directly: the in-kernel norm's 1e-6 epsilon would leave |k| < 1)
+    k3 = k / np.linalg.norm(k, axis=-1, keepdims=True)
+    k3[:, :, 1] = k3[:, :, 0]
+    q3 = k3[:, :, 0].copy()
+    b3 = np.full_like(b, 1e4)
+    o3, _ = oracle_mod.decode(q3, k3, v, pool, read, A_log, a, dt_bias, b3, scale=1.0,
+                              use_qk_l2norm=False)
+    np.testing.assert_allclose(o3, v[:, :, 1], rtol=1e-9, atol=1e-11)
+
+
+def test_decode_scatter_and_disable(oracle_mod):
+    rng = np.random.default_rng(31)
+    B, T, nh, H, Dk, Dv, P = 2, 3, 2, 1, 8, 4, 10
+    q, k, v, pool, A_log, dt_bias, a, b = _decode_inputs(rng, B, T, nh, H, Dk, Dv, P)
+    read = np.array([0, 1], np.int32)
+    write = np.array([2, 3], np.int32)
+    sc = np.array([[4, -1, 5], [6, 7, 8]], np.int32)
+    out, newpool = oracle_mod.decode(q, k, v, pool, read, A_log, a, dt_bias, b, write_idx=write,
+                                     scatter_idx=sc)
+    expect = pool.copy()
+    for row in range(B):
+        o, states = brute_decode_row(pool[read[row], 0], q[row, :, 0], k[row, :, :, 0],
+                                     v[row, :, :, 0], a[row, :, 0], b[row, :, :, 0], A_log[0],
+                                     dt_bias[0], 1 / np.sqrt(Dk), True)
+        np.testing.assert_allclose(out[row, :, 0], o, rtol=1e-10, atol=1e-12)
+        for t in range(T):
+            if sc[row, t] >= 0:
+                expect[sc[row, t], 0] = states[t]
+    # scatter given: the end write-back to write_idx is skipped
+    np.testing.assert_allclose(newpool, expect, rtol=1e-10, atol=1e-12)
+    np.testing.assert_array_equal(newpool[2], pool[2])
+    out_d, pool_d = oracle_mod.decode(q, k, v, pool, read, A_log, a, dt_bias, b, write_idx=write,
+                                      disable_state_update=True)
+    np.testing.assert_array_equal(pool_d, pool)
+    np.testing.assert_allclose(out_d, out, rtol=1e-12)
+
+
+def test_decode_equals_prefill_with_restated_gate(oracle_mod):
+    """nh = 1 decode over T tokens equals prefill with g = log(alpha), beta = sigmoid(b)."""
+    rng = np.random.default_rng(32)
+    B, T, H, Dk, Dv = 1, 6, 2, 8, 5
+    q, k, v, pool, A_log, dt_bias, a, b = _decode_inputs(rng, B, T, 1, H, Dk, Dv, 1)
+    q /= np.linalg.norm(q, axis=-1, keepdims=True)
+    k /= np.linalg.norm(k, axis=-1, keepdims=True)
+    od, pd = oracle_mod.decode(q, k, v, pool, np.array([0], np.int32), A_log, a, dt_bias, b,
+                               use_qk_l2norm=False, scale=0.3)
+    g = -np.exp(A_log)[None, :] * np_softplus20(a[0] + dt_bias[None, :])
+    beta = 1.0 / (1.0 + np.exp(-b[0, :, 0]))
+    op, fp = oracle_mod.prefill(q[0], k[0, :, 0], v[0, :, 0], g, beta, None, pool, B=1, scale=0.3)
+    np.testing.assert_allclose(od[0], op, rtol=1e-10, atol=1e-13)
+    np.testing.assert_allclose(pd, fp, rtol=1e-10, atol=1e-13)
