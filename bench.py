@@ -1,0 +1,461 @@
+"""Benchmark of the Gated DeltaNet hot path on B200 (one JSON line on rank 0).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl gdn|reference]
+                    [--workload ragged|long]
+
+One step = one gdn_prefill call over the whole prefill workload (default: 8
+ragged requests with lengths U[1,4096], Hq=16, Hv=32, Dk=Dv=128, bf16), inputs
+resident in HBM.  `value` is prefill tokens/s over all ranks.  The same run
+then times gdn_decode over the state-pool workload (pool [1024,32,128,128]
+fp32, 256 rows with 13 padding rows) for K steps and reports its state-pool
+GB/s under "decode".
+
+Multi-GPU (torchrun): every rank runs an independent replica of the workload
+(weak scaling, no collective on the data path); times are the max over ranks.
+
+--impl reference times the float64 CPU oracle on a bounded sample of the same
+workload on this host's cores (rank 0 only).
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "GDN prefill tokens/s (tensor-pipe %); decode state-pool GB/s vs HBM peak"
+CHUNK = 64
+
+
+# ----------------------------------------------------------------- helpers
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return {"hbm_gbs": float(d["hbm_gbs"]), "bf16_tflops": float(d["bf16_tflops"]),
+                "bf16_tflops_sustained": float(d.get("bf16_tflops_sustained", d["bf16_tflops"])),
+                "source": "measured"}
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0,
+            "source": "fallback"}
+
+
+def prefill_flops_per_token_head(Dk, Dv, C=CHUNK):
+    """Tensor-core FLOPs of the chunked form per token and value head:
+    Gram K K^T and Q K^T (2 * 2 C Dk), W = T diag(b G) K (2 C Dk), U~ = T diag(b) V (2 C Dv),
+    W S and Q S (2 * 2 Dk Dv), (Q K^T . M) U (2 C Dv), K~^T U (2 Dk Dv)."""
+    return 6 * Dk * Dv + 2 * C * (3 * Dk + 2 * Dv)
+
+
+def prefill_bytes(case):
+    N = case.N
+    Hq, Hv, Dk, Dv = case.dims
+    esz = case.q.element_size()
+    b = N * (2 * Hq * Dk + 2 * Hv * Dv) * esz + N * Hv * 8  # q, k, v, out, g, beta
+    st = case.B * Hv * Dv * Dk * 4
+    b += st * (2 if case.initial_state is not None else 1)
+    if case.cu_seqlens is not None:
+        b += (case.B + 1) * 4
+    return b
+
+
+def decode_bytes(case):
+    """HBM bytes the method must move: per live (row, head) the state read once and written
+    once per store, plus q, k, v, a, b, out."""
+    B, T, H, Dk = case.q.shape
+    nh = case.k.shape[2]
+    HV, Dv = case.v.shape[3], case.v.shape[4]
+    live = int((case.read_idx >= 0).sum())
+    state = Dv * Dk * 4
+    if case.scatter_idx is not None:
+        sc = case.scatter_idx[case.read_idx >= 0]
+        stores = int((sc >= 0).sum())
+    elif case.disable_state_update:
+        stores = 0
+    else:
+        w = case.read_idx if case.write_idx is None else case.write_idx
+        stores = int(((case.read_idx >= 0) & (w >= 0)).sum())
+    act = live * T * (H * Dk + nh * H * Dk + nh * HV * Dv + HV * Dv) * 2 + live * T * (HV + nh * HV) * 2
+    return live * HV * state + stores * HV * state + act
+
+
+class ClockSampler:
+    """nvidia-smi clocks/throttle sampling in the background during timed regions."""
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index):
+        self.gpu_index = gpu_index
+        self.rows = []
+        self.proc = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.gpu_index}", f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.thread = threading.Thread(target=self._read, daemon=True)
+            self.thread.start()
+        except (OSError, FileNotFoundError):
+            self.proc = None
+
+    def _read(self):
+        for line in self.proc.stdout:
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) >= 9:
+                self.rows.append(parts)
+
+    def stop(self):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+
+    def summary(self):
+        if not self.rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"], "samples": 0}
+        sm = [float(r[1]) for r in self.rows if r[1].replace(".", "").isdigit()]
+        smax = [float(r[2]) for r in self.rows if r[2].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = set()
+        for r in self.rows:
+            for n, v in zip(names, r[5:9]):
+                if v.strip().lower().startswith("active"):
+                    reasons.add(n)
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(smax) if smax else None,
+                "reasons": sorted(reasons), "samples": len(self.rows)}
+
+
+def dist_setup():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    return world, rank, local
+
+
+def max_over_ranks(x: float, world: int) -> float:
+    if world == 1:
+        return x
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+# ---------------------------------------------------------------- GPU arms
+def to_dev(t):
+    return None if t is None else t.cuda(non_blocking=False)
+
+
+def time_prefill(gdn, case, steps, warmup, world):
+    q, k, v, g, beta = map(to_dev, (case.q, case.k, case.v, case.g, case.beta))
+    cu, init = to_dev(case.cu_seqlens), to_dev(case.initial_state)
+    Hq, Hv, Dk, Dv = case.dims
+    out = torch.empty((case.N, Hv, Dv), dtype=case.q.dtype, device="cuda")
+    fs = torch.empty((case.B, Hv, Dv, Dk), dtype=torch.float32, device="cuda")
+
+    def step():
+        gdn.gdn_prefill(q, k, v, g, beta, cu, init, fs, out, num_requests=case.B,
+                        scale=case.scale, qk_l2norm=case.qk_l2norm)
+
+    for _ in range(warmup):
+        step()
+    stream = torch.cuda.current_stream()
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(steps)]
+    barrier(world)
+    torch.cuda.synchronize()
+    t0 = torch.cuda.Event(enable_timing=True)
+    t1 = torch.cuda.Event(enable_timing=True)
+    t0.record(stream)
+    for s, e in ev:
+        s.record(stream)
+        step()
+        e.record(stream)
+    t1.record(stream)
+    torch.cuda.synchronize()
+    barrier(world)
+    total_ms = t0.elapsed_time(t1)
+    launch_ms = [s.elapsed_time(e) for s, e in ev]
+    return total_ms, launch_ms
+
+
+def time_prefill_e2e(gdn, case, steps, warmup, world):
+    """Through the public call, from pinned host buffers, with host<->device copies inside."""
+    hq, hk, hv, hg, hb = (t.pin_memory() for t in (case.q, case.k, case.v, case.g, case.beta))
+    hcu = None if case.cu_seqlens is None else case.cu_seqlens.pin_memory()
+    hinit = None if case.initial_state is None else case.initial_state.pin_memory()
+    Hq, Hv, Dk, Dv = case.dims
+    dq, dk, dv, dg, db = (torch.empty_like(t, device="cuda") for t in (hq, hk, hv, hg, hb))
+    dcu = None if hcu is None else torch.empty_like(hcu, device="cuda")
+    dinit = None if hinit is None else torch.empty_like(hinit, device="cuda")
+    out = torch.empty((case.N, Hv, Dv), dtype=case.q.dtype, device="cuda")
+    fs = torch.empty((case.B, Hv, Dv, Dk), dtype=torch.float32, device="cuda")
+    hout = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+    hfs = torch.empty(fs.shape, dtype=fs.dtype).pin_memory()
+    h2d = sum(t.numel() * t.element_size() for t in (hq, hk, hv, hg, hb, hcu, hinit)
+              if t is not None)
+    d2h = hout.numel() * hout.element_size() + hfs.numel() * hfs.element_size()
+
+    def step():
+        for d, h in ((dq, hq), (dk, hk), (dv, hv), (dg, hg), (db, hb), (dcu, hcu),
+                     (dinit, hinit)):
+            if d is not None:
+                d.copy_(h, non_blocking=True)
+        gdn.gdn_prefill(dq, dk, dv, dg, db, dcu, dinit, fs, out, num_requests=case.B,
+                        scale=case.scale, qk_l2norm=case.qk_l2norm)
+        hout.copy_(out, non_blocking=True)
+        hfs.copy_(fs, non_blocking=True)
+
+    for _ in range(warmup):
+        step()
+    stream = torch.cuda.current_stream()
+    barrier(world)
+    torch.cuda.synchronize()
+    t0 = torch.cuda.Event(enable_timing=True)
+    t1 = torch.cuda.Event(enable_timing=True)
+    t0.record(stream)
+    for _ in range(steps):
+        step()
+    t1.record(stream)
+    torch.cuda.synchronize()
+    barrier(world)
+    return t0.elapsed_time(t1), h2d, d2h
+
+
+def time_decode(gdn, case, steps, warmup, world):
+    q, k, v, a, b = map(to_dev, (case.q, case.k, case.v, case.a, case.b))
+    A_log, dt_bias = to_dev(case.A_log), to_dev(case.dt_bias)
+    ri, wi, si = to_dev(case.read_idx), to_dev(case.write_idx), to_dev(case.scatter_idx)
+    pool = to_dev(case.pool)
+    B, T, H, Dk = case.q.shape
+    HV, Dv = case.v.shape[3], case.v.shape[4]
+    out = torch.zeros((B, T, HV, Dv), dtype=torch.bfloat16, device="cuda")
+
+    def step():
+        gdn.gdn_decode(q, k, v, pool, ri, A_log, a, dt_bias, b, scale=case.scale, out=out,
+                       scatter_idx=si, use_qk_l2norm=case.use_qk_l2norm, write_idx=wi)
+
+    for _ in range(warmup):
+        step()
+    stream = torch.cuda.current_stream()
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(steps)]
+    barrier(world)
+    torch.cuda.synchronize()
+    for s, e in ev:
+        s.record(stream)
+        step()
+        e.record(stream)
+    torch.cuda.synchronize()
+    barrier(world)
+    del pool
+    return [s.elapsed_time(e) for s, e in ev]
+
+
+# ---------------------------------------------------------------- CPU oracle
+def cpu_oracle_sample(case, target_s=10.0):
+    """Time the float64 oracle on a bounded sample of the prefill workload: the first L
+    tokens of request 0 with every head; L is grown until one run takes ~target_s/4, then
+    scaled so the whole measurement is ~target_s."""
+    import oracle
+    oracle.build()
+    threads = oracle.max_threads()
+    Hq, Hv, Dk, Dv = case.dims
+    start = 0 if case.cu_seqlens is None else int(case.cu_seqlens[0])
+    total = case.N - start
+
+    def run(L):
+        sl = slice(start, start + L)
+        q = case.q[sl].to(torch.float64).numpy()
+        k = case.k[sl].to(torch.float64).numpy()
+        v = case.v[sl].to(torch.float64).numpy()
+        g = case.g[sl].to(torch.float64).numpy()
+        b = case.beta[sl].to(torch.float64).numpy()
+        init = None if case.initial_state is None else \
+            case.initial_state[:1].to(torch.float64).numpy()
+        t = time.perf_counter()
+        oracle.prefill(q, k, v, g, b, None, init, B=1, scale=case.scale,
+                       qk_l2norm=case.qk_l2norm, threads=threads)
+        return time.perf_counter() - t
+
+    L = 16
+    dt = run(L)
+    while dt < target_s / 8 and L * 2 <= total:
+        L *= 2
+        dt = run(L)
+    L_final = max(1, min(total, int(L * (target_s / max(dt, 1e-6)))))
+    dt = run(L_final)
+    return {"value": L_final / dt, "unit": "tokens/s", "cores": threads, "kind": "oracle",
+            "sample": f"first {L_final} tokens of the packed stream run as one request, "
+                      f"all {Hv} value heads ({Hq} query/key heads), float64, {dt:.1f} s"}
+
+
+# ---------------------------------------------------------------------- main
+def make_case(name):
+    from gated_deltanet_state_gdn_b200 import workloads
+    if name == "ragged":
+        return workloads.ragged_prefill_case()
+    if name == "long":
+        return workloads.long_prefill_case()
+    raise ValueError(name)
+
+
+def workload_config(case, name):
+    Hq, Hv, Dk, Dv = case.dims
+    return {"workload": case.name, "requests": case.B, "tokens": case.N,
+            "lengths": "U[1,4096] seeded" if name == "ragged" else str(case.N),
+            "Hq": Hq, "Hv": Hv, "Dk": Dk, "Dv": Dv, "chunk": CHUNK,
+            "l2": "inputs larger than L2 (q+k+v+out > 126 MB), no flush"}
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="gdn", choices=["gdn", "reference"])
+    ap.add_argument("--workload", default="ragged", choices=["ragged", "long"])
+    ap.add_argument("--no-decode", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=10.0)
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+
+    if args.impl == "reference":
+        if rank != 0:
+            return 0
+        case = make_case(args.workload)
+        per = []
+        base = None
+        for _ in range(args.steps):
+            base = cpu_oracle_sample(case, target_s=max(2.0, args.cpu_seconds / 4))
+            per.append(base["value"])
+        val = statistics.median(per)
+        base["value"] = val
+        print(json.dumps({
+            "impl": "reference", "metric": METRIC, "value": val, "unit": "tokens/s",
+            "n_gpus": args.gpus, "steps": args.steps, "warmup": 0,
+            "ms_per_step": case.N / val * 1e3, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": workload_config(case, args.workload), "cpu_baseline": base,
+            "e2e": {"value": val, "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}), flush=True)
+        return 0
+
+    world, rank, local = dist_setup()
+    torch.cuda.set_device(local)
+    import gated_deltanet_state_gdn_b200 as gdn
+    from gated_deltanet_state_gdn_b200 import workloads
+    gdn.lib()
+    peaks = load_peaks()
+
+    case = make_case(args.workload)
+    Hq, Hv, Dk, Dv = case.dims
+    clocks = ClockSampler(int(os.environ.get("CUDA_VISIBLE_DEVICES", str(local)).split(",")[0])
+                          if os.environ.get("CUDA_VISIBLE_DEVICES", "").split(",")[0].isdigit()
+                          else local)
+    clocks.start()
+    total_ms, launch_ms = time_prefill(gdn, case, args.steps, args.warmup, world)
+    max_ms = max_over_ranks(total_ms, world)
+    ms_per_step = max_ms / args.steps
+    tokens = case.N * world
+    value = tokens / (ms_per_step / 1e3)
+    launches = args.steps
+
+    chunked = gdn.prefill_uses_chunked(case.q.dtype, Dk, Dv)
+    avg_launch_s = statistics.mean(launch_ms) / 1e3
+    if chunked:
+        flops = case.N * Hv * prefill_flops_per_token_head(Dk, Dv)
+        ach = flops / avg_launch_s / 1e12
+        roof = {"kernel": "gdn_prefill_chunk", "bound": "tensor", "achieved": ach,
+                "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
+                "frac": ach / peaks["bf16_tflops"], "traffic": None,
+                "peak_source": peaks["source"] + " (burst bf16)"}
+    else:
+        byts = prefill_bytes(case)
+        ach = byts / avg_launch_s / 1e9
+        roof = {"kernel": "gdn_prefill_seq", "bound": "hbm", "achieved": ach,
+                "peak": peaks["hbm_gbs"], "unit": "GB/s", "frac": ach / peaks["hbm_gbs"],
+                "traffic": None, "peak_source": peaks["source"]}
+
+    decode = None
+    if not args.no_decode:
+        dcase = workloads.decode_pool_case()
+        dms = time_decode(gdn, dcase, args.steps, args.warmup, world)
+        dmax = max_over_ranks(sum(dms), world) / args.steps
+        dbytes = decode_bytes(dcase)
+        gbs = dbytes * world / (dmax / 1e3) / 1e9
+        per_gpu = dbytes / (statistics.mean(dms) / 1e3) / 1e9
+        decode = {"workload": dcase.name, "value": gbs, "unit": "GB/s",
+                  "bytes_per_step": dbytes, "ms_per_step": dmax,
+                  "frac": per_gpu / peaks["hbm_gbs"], "peak": peaks["hbm_gbs"],
+                  "peak_source": peaks["source"]}
+        launches += args.steps
+        del dcase
+    clocks.stop()
+
+    e2e = None
+    if not args.no_e2e:
+        e_ms, h2d, d2h = time_prefill_e2e(gdn, case, max(3, args.steps // 4), args.warmup, world)
+        e_steps = max(3, args.steps // 4)
+        e_max = max_over_ranks(e_ms, world) / e_steps
+        e2e = {"value": tokens / (e_max / 1e3), "unit": "tokens/s",
+               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e_max}
+        launches += e_steps
+
+    cpu = None
+    if rank == 0 and world == 1:
+        cpu = cpu_oracle_sample(case, target_s=args.cpu_seconds)
+
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_per_step,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "data": "synthetic", "config": dict(workload_config(case, args.workload),
+                                                parallelism=f"replicas{world}"),
+            "roofline": roof, "decode": decode, "e2e": e2e, "cpu_baseline": cpu,
+            "clocks": clocks.summary(), "gpu_launches": launches,
+        }
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

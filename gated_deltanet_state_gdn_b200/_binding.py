@@ -1,0 +1,227 @@
+"""ctypes binding of libgdn (argument marshalling only).
+
+Each function takes torch CUDA tensors, checks dtypes and shapes, makes
+inputs contiguous, allocates outputs the caller did not pass (torch is the
+allocator), and calls the C entry point of the same name on torch's current
+stream.  Every step of the recurrence runs in libgdn's kernels; there is no
+other path.  If libgdn.so cannot be loaded, every call raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import math
+import os
+from typing import Optional
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libgdn.so")
+
+GDN_OK = 0
+GDN_ERR_NULL = 1
+GDN_ERR_SHAPE = 2
+GDN_ERR_DTYPE = 3
+GDN_ERR_ALIGN = 4
+GDN_ERR_ALIAS = 5
+GDN_ERR_UNSUPPORTED = 6
+GDN_ERR_CUDA = 7
+
+GDN_F32 = 0
+GDN_BF16 = 1
+
+GDN_PREFILL_SEQUENTIAL = 1
+GDN_DISABLE_STATE_UPDATE = 2
+GDN_DECODE_QK_L2NORM = 4
+
+GDN_DEV_BAD_SLOT = 1
+
+EXPORTED = ("gdn_prefill", "gdn_decode", "gdn_status_string", "gdn_last_error",
+            "gdn_abi_version", "gdn_prefill_uses_chunked")
+
+_lib = None
+
+
+class GdnError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        name = status_string(status)
+        detail = ""
+        if status == GDN_ERR_CUDA:
+            detail = ": " + lib().gdn_last_error().decode()
+        super().__init__(f"{where} failed with {name}{detail}")
+
+
+def lib():
+    """Load libgdn.so (built in-tree); raise if it is missing."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(
+                f"libgdn.so not found at {LIB_PATH}: build it with "
+                "`python -m gated_deltanet_state_gdn_b200.build` (there is no fallback path)")
+        L = ctypes.CDLL(LIB_PATH)
+        vp, i32, i64, u32, f32 = (ctypes.c_void_p, ctypes.c_int32, ctypes.c_int64,
+                                  ctypes.c_uint32, ctypes.c_float)
+        L.gdn_prefill.restype = ctypes.c_int
+        L.gdn_prefill.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp,
+                                  i32, i64, i32, i32, i32, i32, ctypes.c_int, f32, i32, u32,
+                                  vp, vp]
+        L.gdn_decode.restype = ctypes.c_int
+        L.gdn_decode.argtypes = [vp, vp, vp, vp, i32, i64, i64, vp, vp, vp,
+                                 vp, vp, vp, vp, f32, vp,
+                                 i32, i32, i32, i32, i32, i32, i32, u32, vp, vp]
+        L.gdn_status_string.restype = ctypes.c_char_p
+        L.gdn_status_string.argtypes = [i32]
+        L.gdn_last_error.restype = ctypes.c_char_p
+        L.gdn_last_error.argtypes = []
+        L.gdn_abi_version.restype = i32
+        L.gdn_abi_version.argtypes = []
+        L.gdn_prefill_uses_chunked.restype = i32
+        L.gdn_prefill_uses_chunked.argtypes = [ctypes.c_int, i32, i32, u32]
+        _lib = L
+    return _lib
+
+
+def prefill_uses_chunked(dtype: torch.dtype, Dk: int, Dv: int, sequential: bool = False) -> bool:
+    code = GDN_BF16 if dtype == torch.bfloat16 else GDN_F32
+    return bool(lib().gdn_prefill_uses_chunked(code, Dk, Dv,
+                                               GDN_PREFILL_SEQUENTIAL if sequential else 0))
+
+
+def status_string(status: int) -> str:
+    return lib().gdn_status_string(int(status)).decode()
+
+
+def _ptr(t: Optional[torch.Tensor]):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream) -> ctypes.c_void_p:
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def _check_cuda(name, t, dtype=None):
+    if t is None:
+        return None
+    if not isinstance(t, torch.Tensor) or not t.is_cuda:
+        raise TypeError(f"{name} must be a CUDA tensor")
+    if dtype is not None and t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    return t.contiguous()
+
+
+def gdn_prefill(q, k, v, g, beta, cu_seqlens=None, initial_state=None, final_state=None,
+                out=None, *, num_requests: Optional[int] = None, scale: Optional[float] = None,
+                qk_l2norm: bool = False, sequential: bool = False, dev_status=None, stream=None):
+    """Gated DeltaNet prefill (log-space form) over ragged requests.
+
+    q, k: [N, Hq, Dk] or [B, S, Hq, Dk]; v: [N, Hv, Dv] (same leading axes);
+    g, beta: [N, Hv] fp32; cu_seqlens: [B+1] int32 (rank-3 form) or None;
+    initial_state: [B, Hv, Dv, Dk] fp32 or None.  ``scale`` None or 0 selects
+    1/sqrt(Dk).  Returns (out, final_state).
+    """
+    if q.dim() == 4:
+        Bq, S = q.shape[0], q.shape[1]
+        if cu_seqlens is not None:
+            raise ValueError("cu_seqlens requires the rank-3 (total_tokens, heads, dim) form")
+        num_requests = Bq
+        q = q.reshape(Bq * S, *q.shape[2:])
+        k = k.reshape(Bq * S, *k.shape[2:])
+        v = v.reshape(Bq * S, *v.shape[2:])
+        g = g.reshape(Bq * S, -1)
+        beta = beta.reshape(Bq * S, -1)
+        if out is not None:
+            out = out.view(Bq * S, *out.shape[2:])
+    if q.dtype == torch.bfloat16:
+        dt = GDN_BF16
+    elif q.dtype == torch.float32:
+        dt = GDN_F32
+    else:
+        raise TypeError(f"unsupported activation dtype {q.dtype}")
+    q = _check_cuda("q", q, q.dtype)
+    k = _check_cuda("k", k, q.dtype)
+    v = _check_cuda("v", v, q.dtype)
+    g = _check_cuda("g", g, torch.float32)
+    beta = _check_cuda("beta", beta, torch.float32)
+    cu_seqlens = _check_cuda("cu_seqlens", cu_seqlens, torch.int32)
+    initial_state = _check_cuda("initial_state", initial_state, torch.float32)
+    N, Hq, Dk = q.shape
+    Hv, Dv = v.shape[1], v.shape[2]
+    if k.shape != q.shape or v.shape[0] != N or g.shape != (N, Hv) or beta.shape != (N, Hv):
+        raise ValueError("inconsistent q/k/v/g/beta shapes")
+    if cu_seqlens is not None:
+        B = cu_seqlens.shape[0] - 1
+    else:
+        if num_requests is None:
+            raise ValueError("num_requests is required without cu_seqlens")
+        B = int(num_requests)
+    if out is None:
+        out = torch.empty((N, Hv, Dv), dtype=q.dtype, device=q.device)
+    elif not out.is_contiguous() or out.dtype != q.dtype or tuple(out.shape) != (N, Hv, Dv):
+        raise ValueError("out must be a contiguous [N, Hv, Dv] tensor of q's dtype")
+    if final_state is None:
+        final_state = torch.empty((B, Hv, Dv, Dk), dtype=torch.float32, device=q.device)
+    elif not final_state.is_contiguous() or final_state.dtype != torch.float32:
+        raise ValueError("final_state must be a contiguous fp32 tensor")
+    if initial_state is not None and tuple(initial_state.shape) != (B, Hv, Dv, Dk):
+        raise ValueError("initial_state must be [B, Hv, Dv, Dk]")
+    if scale is None or scale == 0.0:
+        scale = 1.0 / math.sqrt(Dk)
+    flags = GDN_PREFILL_SEQUENTIAL if sequential else 0
+    st = lib().gdn_prefill(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(cu_seqlens),
+                           _ptr(initial_state), _ptr(final_state), _ptr(out), B, N, Hq, Hv, Dk,
+                           Dv, dt, float(scale), int(bool(qk_l2norm)), flags, _ptr(dev_status),
+                           _stream(stream))
+    if st != GDN_OK:
+        raise GdnError(st, "gdn_prefill")
+    return out, final_state
+
+
+def gdn_decode(q, k, v, state_pool, read_idx, A_log, a, dt_bias, b, *, scale=None, out=None,
+               scatter_idx=None, disable_state_update: bool = False, use_qk_l2norm: bool = True,
+               write_idx=None, dev_status=None, stream=None):
+    """Gated DeltaProduct decode / MTP over an fp32 pool (updated in place).
+
+    q: [B, T, H, Dk]; k: [B, T, nh, H, Dk]; v: [B, T, nh, HV, Dv] (bf16);
+    state_pool: [P, HV, Dv, Dk] fp32 with dense rows (slot/head padding allowed);
+    read_idx, write_idx: [B] int32; scatter_idx: [B, T] int32;
+    A_log, dt_bias: [HV] fp32; a: [B, T, HV]; b: [B, T, nh, HV] (bf16).
+    Returns (out, state_pool).
+    """
+    q = _check_cuda("q", q, torch.bfloat16)
+    k = _check_cuda("k", k, torch.bfloat16)
+    v = _check_cuda("v", v, torch.bfloat16)
+    a = _check_cuda("a", a, torch.bfloat16)
+    b = _check_cuda("b", b, torch.bfloat16)
+    A_log = _check_cuda("A_log", A_log, torch.float32)
+    dt_bias = _check_cuda("dt_bias", dt_bias, torch.float32)
+    read_idx = _check_cuda("read_idx", read_idx, torch.int32)
+    write_idx = _check_cuda("write_idx", write_idx, torch.int32)
+    scatter_idx = _check_cuda("scatter_idx", scatter_idx, torch.int32)
+    if not state_pool.is_cuda or state_pool.dtype != torch.float32 or state_pool.dim() != 4:
+        raise TypeError("state_pool must be a 4-d fp32 CUDA tensor")
+    P, HV, Dv, Dk = state_pool.shape
+    if state_pool.stride(3) != 1 or state_pool.stride(2) != Dk:
+        raise ValueError("state_pool rows must be dense")
+    B, T, H, _ = q.shape
+    nh = k.shape[2]
+    if out is None:
+        out = torch.zeros((B, T, HV, Dv), dtype=torch.bfloat16, device=q.device)
+    elif (not out.is_contiguous() or out.dtype != torch.bfloat16
+          or tuple(out.shape) != (B, T, HV, Dv)):
+        raise ValueError("out must be a contiguous bf16 [B, T, HV, Dv] tensor")
+    if scale is None:
+        scale = 1.0 / math.sqrt(Dk)
+    flags = (GDN_DISABLE_STATE_UPDATE if disable_state_update else 0) | \
+        (GDN_DECODE_QK_L2NORM if use_qk_l2norm else 0)
+    st = lib().gdn_decode(_ptr(q), _ptr(k), _ptr(v), _ptr(state_pool), P, state_pool.stride(0),
+                          state_pool.stride(1), _ptr(read_idx), _ptr(write_idx),
+                          _ptr(scatter_idx), _ptr(A_log), _ptr(a), _ptr(dt_bias), _ptr(b),
+                          float(scale), _ptr(out), B, T, nh, H, HV, Dk, Dv, flags,
+                          _ptr(dev_status), _stream(stream))
+    if st != GDN_OK:
+        raise GdnError(st, "gdn_decode")
+    return out, state_pool

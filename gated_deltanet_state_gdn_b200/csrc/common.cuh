@@ -1,0 +1,107 @@
+// common.cuh -- small device helpers shared by the libgdn kernels.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "gdn.h"
+
+namespace gdn {
+
+__device__ __forceinline__ float bf16_to_f32(__nv_bfloat16 x) { return __bfloat162float(x); }
+
+// 4 consecutive bf16 (8 bytes) -> float4
+__device__ __forceinline__ float4 ld_bf16x4(const __nv_bfloat16 *p)
+{
+    uint2 raw = __ldg(reinterpret_cast<const uint2 *>(p));
+    __nv_bfloat162 lo = *reinterpret_cast<__nv_bfloat162 *>(&raw.x);
+    __nv_bfloat162 hi = *reinterpret_cast<__nv_bfloat162 *>(&raw.y);
+    float2 a = __bfloat1622float2(lo);
+    float2 b = __bfloat1622float2(hi);
+    return make_float4(a.x, a.y, b.x, b.y);
+}
+
+__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi)
+{
+    __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
+    return *reinterpret_cast<uint32_t *>(&v);
+}
+
+// streaming (evict-first) 16-byte global load / store
+__device__ __forceinline__ float4 ld_stream(const float *p)
+{
+    return __ldcs(reinterpret_cast<const float4 *>(p));
+}
+__device__ __forceinline__ void st_stream(float *p, float4 v)
+{
+    __stcs(reinterpret_cast<float4 *>(p), v);
+}
+
+__device__ __forceinline__ float dot4(float4 a, float4 b)
+{
+    return a.x * b.x + a.y * b.y + a.z * b.z + a.w * b.w;
+}
+
+template <int WIDTH>
+__device__ __forceinline__ float group_sum(float x)
+{
+#pragma unroll
+    for (int m = 1; m < WIDTH; m <<= 1) x += __shfl_xor_sync(0xffffffffu, x, m);
+    return x;
+}
+
+__device__ __forceinline__ float warp_sum(float x) { return group_sum<32>(x); }
+
+__device__ __forceinline__ int64_t clamp_i64(int64_t x, int64_t lo, int64_t hi)
+{
+    return x < lo ? lo : (x > hi ? hi : x);
+}
+
+// softplus with the threshold-20 rule of the decode gate
+__device__ __forceinline__ float softplus20(float x)
+{
+    return x > 20.f ? x : log1pf(expf(x));
+}
+
+}  // namespace gdn
+
+// Launchers implemented by the kernel translation units.
+struct GdnPrefillArgs {
+    const void *q, *k, *v;
+    const float *g, *beta;
+    const int32_t *cu_seqlens;
+    const float *initial_state;
+    float *final_state;
+    void *out;
+    int32_t B;
+    int64_t N;
+    int32_t Hq, Hv, Dk, Dv;
+    gdn_dtype dtype;
+    float scale;
+    int32_t qk_l2norm;
+    int32_t *dev_status;
+};
+
+struct GdnDecodeArgs {
+    const void *q, *k, *v;
+    float *pool;
+    int32_t pool_size;
+    int64_t slot_stride, head_stride;
+    const int32_t *read_idx, *write_idx, *scatter_idx;
+    const float *A_log;
+    const void *a;
+    const float *dt_bias;
+    const void *b;
+    float scale;
+    void *out;
+    int32_t B, T, nh, H, HV, Dk, Dv;
+    int32_t disable_state_update;
+    int32_t use_qk_l2norm;
+    int32_t *dev_status;
+};
+
+cudaError_t launch_decode(const GdnDecodeArgs &a, cudaStream_t stream);
+cudaError_t launch_prefill_sequential(const GdnPrefillArgs &a, cudaStream_t stream);
+cudaError_t launch_prefill_chunked(const GdnPrefillArgs &a, cudaStream_t stream);
+bool prefill_chunked_supported(const GdnPrefillArgs &a);

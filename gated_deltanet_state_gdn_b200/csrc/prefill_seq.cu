@@ -1,0 +1,168 @@
+// prefill_seq.cu -- per-token Gated DeltaNet prefill for any head size <= 256.
+//
+// Operation ("com.microsoft.GatedDeltaNet", Description; "Gated DeltaNet
+// State Update", statement): per request and value head, for every token
+//   p   = S_{t-1}^T k_t
+//   S_t = exp(g_t) S_{t-1} + k_t (beta_t (v_t - exp(g_t) p))^T
+//   o_t = scale * S_t^T q_t
+// The state stays in fp32 registers for the whole request.
+//
+// This is the general path: fp32 or bf16 activations, any Dk, Dv in
+// [1, 256], any Hq | Hv.  It is also the sequential counterpart the chunked
+// tensor-core kernel is checked against.  Layout: grid (B * Hv, Dv tiles of
+// 32 rows); a warp owns 4 V-rows of S (V-major, one row = Dk floats), lane l
+// owns elements l + 32 j of each row; row dot products are warp reductions.
+#include "common.cuh"
+
+namespace gdn {
+
+constexpr int kSeqWarps = 8;
+constexpr int kSeqRows = 4;  // V-rows per warp
+
+template <typename Tin>
+__device__ __forceinline__ float load_act(const Tin *p);
+template <>
+__device__ __forceinline__ float load_act<float>(const float *p) { return __ldg(p); }
+template <>
+__device__ __forceinline__ float load_act<__nv_bfloat16>(const __nv_bfloat16 *p)
+{
+    return __bfloat162float(p[0]);
+}
+
+template <typename Tout>
+__device__ __forceinline__ void store_act(Tout *p, float x);
+template <>
+__device__ __forceinline__ void store_act<float>(float *p, float x) { *p = x; }
+template <>
+__device__ __forceinline__ void store_act<__nv_bfloat16>(__nv_bfloat16 *p, float x)
+{
+    *p = __float2bfloat16_rn(x);
+}
+
+template <typename Tin, int EPL>
+__global__ void __launch_bounds__(kSeqWarps * 32)
+prefill_seq_kernel(const GdnPrefillArgs p)
+{
+    constexpr int R = kSeqRows;
+    const int lane = threadIdx.x & 31;
+    const int warp = threadIdx.x >> 5;
+    const int Hv = p.Hv, Hq = p.Hq, Dk = p.Dk, Dv = p.Dv;
+    const int b = blockIdx.x / Hv;
+    const int h = blockIdx.x - b * Hv;
+    const int qh = (int)(((int64_t)h * Hq) / Hv);
+    const int row_base = blockIdx.y * (kSeqWarps * R) + warp * R;
+    if (row_base >= Dv) return;  // whole warp idle (uniform)
+
+    int64_t start, end;
+    if (p.cu_seqlens) {
+        start = clamp_i64(p.cu_seqlens[b], 0, p.N);
+        end = clamp_i64(p.cu_seqlens[b + 1], 0, p.N);
+    } else {
+        const int64_t S = p.N / p.B;
+        start = (int64_t)b * S;
+        end = start + S;
+    }
+
+    const Tin *qg = static_cast<const Tin *>(p.q);
+    const Tin *kg = static_cast<const Tin *>(p.k);
+    const Tin *vg = static_cast<const Tin *>(p.v);
+    Tin *og = static_cast<Tin *>(p.out);
+
+    float S[R][EPL];
+    const int64_t state_off = ((int64_t)b * Hv + h) * Dv * (int64_t)Dk;
+#pragma unroll
+    for (int i = 0; i < R; ++i)
+#pragma unroll
+        for (int j = 0; j < EPL; ++j) {
+            const int e = lane + 32 * j;
+            const int row = row_base + i;
+            S[i][j] = (p.initial_state && e < Dk && row < Dv)
+                          ? p.initial_state[state_off + (int64_t)row * Dk + e]
+                          : 0.f;
+        }
+
+    for (int64_t t = start; t < end; ++t) {
+        float kx[EPL], qx[EPL];
+        const int64_t qk_off = (t * Hq + qh) * (int64_t)Dk;
+#pragma unroll
+        for (int j = 0; j < EPL; ++j) {
+            const int e = lane + 32 * j;
+            kx[j] = e < Dk ? load_act<Tin>(kg + qk_off + e) : 0.f;
+            qx[j] = e < Dk ? load_act<Tin>(qg + qk_off + e) : 0.f;
+        }
+        if (p.qk_l2norm) {
+            float sk = 0.f, sq = 0.f;
+#pragma unroll
+            for (int j = 0; j < EPL; ++j) {
+                sk += kx[j] * kx[j];
+                sq += qx[j] * qx[j];
+            }
+            sk = warp_sum(sk);
+            sq = warp_sum(sq);
+            const float rk = 1.0f / sqrtf(sk + 1e-12f);
+            const float rq = 1.0f / sqrtf(sq + 1e-12f);
+#pragma unroll
+            for (int j = 0; j < EPL; ++j) {
+                kx[j] *= rk;
+                qx[j] *= rq;
+            }
+        }
+        const float gamma = expf(__ldg(p.g + t * Hv + h));
+        const float bt = __ldg(p.beta + t * Hv + h);
+        const int64_t vo = (t * Hv + h) * (int64_t)Dv;
+#pragma unroll
+        for (int i = 0; i < R; ++i) {
+            const int row = row_base + i;
+            if (row >= Dv) break;  // uniform across the warp
+            const float vi = load_act<Tin>(vg + vo + row);
+            float pd = 0.f;
+#pragma unroll
+            for (int j = 0; j < EPL; ++j) pd += S[i][j] * kx[j];
+            pd = warp_sum(pd);
+            const float u = bt * (vi - gamma * pd);
+            float o = 0.f;
+#pragma unroll
+            for (int j = 0; j < EPL; ++j) {
+                S[i][j] = fmaf(kx[j], u, gamma * S[i][j]);
+                o += S[i][j] * qx[j];
+            }
+            o = warp_sum(o);
+            if (lane == 0) store_act<Tin>(og + vo + row, p.scale * o);
+        }
+    }
+
+#pragma unroll
+    for (int i = 0; i < R; ++i)
+#pragma unroll
+        for (int j = 0; j < EPL; ++j) {
+            const int e = lane + 32 * j;
+            const int row = row_base + i;
+            if (e < Dk && row < Dv) p.final_state[state_off + (int64_t)row * Dk + e] = S[i][j];
+        }
+}
+
+template <typename Tin>
+static cudaError_t launch_seq_t(const GdnPrefillArgs &a, cudaStream_t stream)
+{
+    dim3 grid((unsigned)a.B * (unsigned)a.Hv, (unsigned)((a.Dv + kSeqWarps * kSeqRows - 1) /
+                                                         (kSeqWarps * kSeqRows)));
+    dim3 block(kSeqWarps * 32);
+    if (a.Dk <= 32)
+        prefill_seq_kernel<Tin, 1><<<grid, block, 0, stream>>>(a);
+    else if (a.Dk <= 64)
+        prefill_seq_kernel<Tin, 2><<<grid, block, 0, stream>>>(a);
+    else if (a.Dk <= 128)
+        prefill_seq_kernel<Tin, 4><<<grid, block, 0, stream>>>(a);
+    else
+        prefill_seq_kernel<Tin, 8><<<grid, block, 0, stream>>>(a);
+    return cudaGetLastError();
+}
+
+}  // namespace gdn
+
+cudaError_t launch_prefill_sequential(const GdnPrefillArgs &a, cudaStream_t stream)
+{
+    if (a.B == 0 || a.Hv == 0) return cudaSuccess;
+    if (a.dtype == GDN_F32) return gdn::launch_seq_t<float>(a, stream);
+    return gdn::launch_seq_t<__nv_bfloat16>(a, stream);
+}

@@ -1,0 +1,183 @@
+/*
+ * gdn.h -- C ABI of libgdn: the Gated DeltaNet recurrence on NVIDIA B200
+ * (sm_100a).
+ *
+ * Two entry points:
+ *   gdn_prefill  chunked / sequential scan over ragged requests;
+ *   gdn_decode   decode / MTP update of an fp32 slot-indexed state pool.
+ *
+ * Conventions shared by every call
+ *   - Every tensor argument is a DEVICE pointer owned by the caller.  The
+ *     library allocates no device memory and keeps no pointer after the call
+ *     returns (device-side it only holds read-only constant tables).
+ *   - Calls are asynchronous on `stream` (a cudaStream_t; NULL means the
+ *     legacy default stream).  The library never reads tensor contents on the
+ *     host and never synchronises, so a call may be captured in a CUDA graph.
+ *   - Inputs are never modified.  The only buffers written are `out`,
+ *     `final_state` (prefill) and `state_pool`, `out` (decode), plus the
+ *     optional `dev_status` word.
+ *   - Errors the host can see (null pointers, shapes, alignment, aliasing,
+ *     unsupported sizes) are returned as a gdn_status before anything is
+ *     launched.  Errors only the device can see (a slot index >= pool_size)
+ *     skip the affected unit and OR a GDN_DEV_* bit into *dev_status when
+ *     `dev_status` is non-NULL.  No kernel traps or asserts.
+ *   - Layouts are dense, row-major, with the strides implied by the shapes
+ *     below (decode's pool alone takes explicit strides).
+ */
+#ifndef GDN_H
+#define GDN_H
+
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define GDN_API __attribute__((visibility("default")))
+#else
+#define GDN_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    GDN_OK = 0,
+    GDN_ERR_NULL = 1,        /* a required pointer is NULL */
+    GDN_ERR_SHAPE = 2,       /* inconsistent sizes (e.g. Hv % Hq != 0, H != HV) */
+    GDN_ERR_DTYPE = 3,       /* unknown dtype code */
+    GDN_ERR_ALIGN = 4,       /* a pointer or stride breaks the alignment rule */
+    GDN_ERR_ALIAS = 5,       /* an output overlaps an input it must not overlap */
+    GDN_ERR_UNSUPPORTED = 6, /* valid, but outside what the kernels implement */
+    GDN_ERR_CUDA = 7         /* a CUDA runtime call failed; see gdn_last_error() */
+} gdn_status;
+
+typedef enum {
+    GDN_F32 = 0,   /* float32 activations */
+    GDN_BF16 = 1   /* bfloat16 activations */
+} gdn_dtype;
+
+/* flags */
+enum {
+    GDN_PREFILL_SEQUENTIAL = 1u << 0,   /* prefill: force the per-token kernel */
+    GDN_DISABLE_STATE_UPDATE = 1u << 1, /* decode: leave the pool unchanged */
+    GDN_DECODE_QK_L2NORM = 1u << 2      /* decode: L2-normalise q and k in the kernel */
+};
+
+/* bits OR-ed into *dev_status by the kernels */
+enum {
+    GDN_DEV_BAD_SLOT = 1   /* decode: a read/write/scatter slot >= pool_size was skipped */
+};
+
+/*
+ * gdn_prefill -- the log-space Gated DeltaNet recurrence over ragged requests.
+ *
+ * Defined by "com.microsoft.GatedDeltaNet" (ONNX Runtime contrib operator),
+ * Description and Inputs/Outputs/Attributes tables: per value head h,
+ *     S_t = exp(g_t) S_{t-1} + k_t (beta_t (v_t - exp(g_t) S_{t-1}^T k_t))^T
+ *     o_t = scale * S_t^T q_t
+ * with value head h reading query/key head floor(h * Hq / Hv).  This is the
+ * gamma form of "Gated DeltaNet State Update" (statement) with gamma = exp(g).
+ *
+ * Arguments (N = total tokens, B = requests):
+ *   q, k           [N, Hq, Dk]  `dtype`
+ *   v              [N, Hv, Dv]  `dtype`
+ *   g              [N, Hv] float32, log-space decay (g <= 0; -inf allowed)
+ *   beta           [N, Hv] float32, update rate
+ *   cu_seqlens     [B+1] int32 exclusive prefix sums, or NULL for uniform
+ *                  packing (then N % B == 0 and request b is tokens
+ *                  [b*N/B, (b+1)*N/B)).  Entries are clamped on the device to
+ *                  [0, N]; a request whose end <= start is empty.
+ *   initial_state  [B, Hv, Dv, Dk] float32 (V-major), or NULL for zero
+ *   final_state    [B, Hv, Dv, Dk] float32, written; must not overlap
+ *                  initial_state.  An empty request copies its initial state.
+ *   out            [N, Hv, Dv] `dtype`, written for every token that a
+ *                  request covers (others keep the caller's values).
+ *   scale          applied as given (the Python binding maps 0/None to
+ *                  1/sqrt(Dk), the op's default).
+ *   qk_l2norm      non-zero: q and k vectors are scaled by
+ *                  (sum x^2 + 1e-12)^(-1/2) before use.
+ *   flags          GDN_PREFILL_SEQUENTIAL or 0.
+ *   dev_status     optional device int32 (unused by prefill today).
+ * Requirements: 1 <= Dk, Dv <= 256; Hv % Hq == 0; q, k, v, out,
+ * initial_state and final_state 16-byte aligned; out must not overlap any
+ * input.  bf16 with Dk = Dv = 128 runs the chunked tensor-core kernel (unless
+ * GDN_PREFILL_SEQUENTIAL); everything else runs the per-token fp32 kernel.
+ * Overlapping request ranges are not supported (their outputs are undefined).
+ */
+GDN_API gdn_status gdn_prefill(const void *q, const void *k, const void *v,
+                       const float *g, const float *beta,
+                       const int32_t *cu_seqlens,
+                       const float *initial_state, float *final_state,
+                       void *out,
+                       int32_t B, int64_t N, int32_t Hq, int32_t Hv,
+                       int32_t Dk, int32_t Dv, gdn_dtype dtype,
+                       float scale, int32_t qk_l2norm, uint32_t flags,
+                       int32_t *dev_status, void *stream);
+
+/*
+ * gdn_decode -- Gated DeltaProduct decode / MTP over an fp32 state pool.
+ *
+ * Defined by "flashinfer.cake_gdp.cake_gated_delta_product_mtp" (description,
+ * Parameters): for every batch row b and head h with r = read_idx[b] >= 0,
+ * S = pool[r, h]; for each token t:
+ *     S <- alpha_t S,  alpha_t = exp(-exp(A_log[h]) softplus(a[b,t,h] + dt_bias[h]))
+ *                      (softplus(x) = x for x > 20)
+ *     for j < nh:  S <- S + k_tj (beta_tj (v_tj - S^T k_tj))^T,  beta_tj = sigmoid(b[b,t,j,h])
+ *     out[b,t,h] = scale * S^T q_t
+ *     if scatter_idx: pool[scatter_idx[b,t], h] <- S   (negative entry: skipped)
+ * and after the last token, unless scatter_idx or GDN_DISABLE_STATE_UPDATE:
+ *     pool[w, h] <- S with w = write_idx ? write_idx[b] : r (negative: skipped).
+ * With GDN_DECODE_QK_L2NORM, q_t and every k_tj are first scaled by
+ * (sum x^2 + 1e-6)^(-1/2).  A row with read_idx < 0 is padding: nothing is
+ * read, computed or stored and its `out` rows keep the caller's values.
+ *
+ * Arguments:
+ *   q      [B, T, H, Dk] bf16            k  [B, T, nh, H, Dk] bf16
+ *   v      [B, T, nh, HV, Dv] bf16       out [B, T, HV, Dv] bf16 (written)
+ *   state_pool  fp32, slot s head h row j at
+ *               state_pool + s*slot_stride + h*head_stride + j*Dk (rows dense);
+ *               read and written in place.  pool_size slots.
+ *   read_idx [B], write_idx [B] or NULL (= read_idx), scatter_idx [B, T] or NULL: int32
+ *   A_log, dt_bias [HV] float32;  a [B, T, HV] bf16;  b [B, T, nh, HV] bf16
+ *   scale  applied as given (the Python binding maps None to 1/sqrt(Dk))
+ *   flags  GDN_DISABLE_STATE_UPDATE | GDN_DECODE_QK_L2NORM, or 0
+ *   dev_status  optional device int32; GDN_DEV_BAD_SLOT is OR-ed in when a
+ *               slot index >= pool_size is met (that read/write is skipped).
+ * Requirements: H == HV; Dk == 128; Dv in {64, 128}; 1 <= T <= 16;
+ * 1 <= nh <= 4; scatter_idx requires the update enabled; state_pool 16-byte
+ * aligned with slot_stride and head_stride multiples of 4 elements,
+ * head_stride >= Dv*Dk, slot_stride >= HV*head_stride; q, k, v, out 8-byte
+ * aligned.  Rows must not write a slot that another row reads (a row's own
+ * write slot may equal its read slot).
+ */
+GDN_API gdn_status gdn_decode(const void *q, const void *k, const void *v,
+                      float *state_pool, int32_t pool_size,
+                      int64_t slot_stride, int64_t head_stride,
+                      const int32_t *read_idx, const int32_t *write_idx,
+                      const int32_t *scatter_idx,
+                      const float *A_log, const void *a, const float *dt_bias,
+                      const void *b, float scale, void *out,
+                      int32_t B, int32_t T, int32_t nh, int32_t H, int32_t HV,
+                      int32_t Dk, int32_t Dv, uint32_t flags,
+                      int32_t *dev_status, void *stream);
+
+/* 1 when gdn_prefill with these arguments runs the chunked tensor-core
+ * kernel, 0 when it runs the per-token kernel (host-only query, no launch). */
+GDN_API int32_t gdn_prefill_uses_chunked(gdn_dtype dtype, int32_t Dk, int32_t Dv,
+                                         uint32_t flags);
+
+/* Name of a gdn_status code (static string). */
+GDN_API const char *gdn_status_string(int32_t status);
+
+/* Text of the last GDN_ERR_CUDA on the calling thread (static per thread). */
+GDN_API const char *gdn_last_error(void);
+
+/* ABI version of this header: increments on any incompatible change. */
+GDN_API int32_t gdn_abi_version(void);
+
+#define GDN_ABI_VERSION 1
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* GDN_H */

@@ -1,0 +1,127 @@
+"""Host-side checks of libgdn that need no GPU.
+
+* the library loads and exports every entry point include/gdn.h declares;
+* every argument check the C ABI documents returns its status code before
+  anything is launched (the pointers used here are never dereferenced:
+  each call is rejected by a scalar or pointer-value rule first).
+"""
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "gdn.h")
+
+
+@pytest.fixture(scope="module")
+def L():
+    from gated_deltanet_state_gdn_b200 import build
+    build.build()
+    import gated_deltanet_state_gdn_b200 as g
+    return g.lib()
+
+
+def declared_symbols():
+    text = open(HEADER).read()
+    return sorted(set(re.findall(r"GDN_API\s+[\w\s\*]*?\b(gdn_\w+)\s*\(", text)))
+
+
+def test_header_declares_entry_points():
+    syms = declared_symbols()
+    assert {"gdn_prefill", "gdn_decode", "gdn_status_string"} <= set(syms)
+
+
+def test_library_exports_every_declared_symbol(L):
+    for name in declared_symbols():
+        assert hasattr(L, name), name
+    import gated_deltanet_state_gdn_b200 as g
+    assert set(g.EXPORTED) == set(declared_symbols())
+
+
+def test_abi_version_and_status_strings(L):
+    assert L.gdn_abi_version() == 1
+    import gated_deltanet_state_gdn_b200 as g
+    for code, name in [(0, "GDN_OK"), (1, "GDN_ERR_NULL"), (2, "GDN_ERR_SHAPE"),
+                       (3, "GDN_ERR_DTYPE"), (4, "GDN_ERR_ALIGN"), (5, "GDN_ERR_ALIAS"),
+                       (6, "GDN_ERR_UNSUPPORTED"), (7, "GDN_ERR_CUDA")]:
+        assert g.status_string(code) == name
+    assert g.status_string(99) == "GDN_ERR_UNKNOWN"
+
+
+# fake, never-dereferenced device addresses (distinct 256-byte aligned regions)
+def P(i, off=0):
+    return ctypes.c_void_p(0x7f0000000000 + i * (1 << 32) + off)
+
+
+def prefill(L, **kw):
+    args = dict(q=P(1), k=P(2), v=P(3), g=P(4), beta=P(5), cu=None, init=None, final=P(7),
+                out=P(8), B=2, N=64, Hq=1, Hv=1, Dk=16, Dv=16, dtype=0, scale=1.0, l2=0,
+                flags=0, status=None, stream=None)
+    args.update(kw)
+    return L.gdn_prefill(args["q"], args["k"], args["v"], args["g"], args["beta"], args["cu"],
+                         args["init"], args["final"], args["out"], args["B"], args["N"],
+                         args["Hq"], args["Hv"], args["Dk"], args["Dv"], args["dtype"],
+                         args["scale"], args["l2"], args["flags"], args["status"],
+                         args["stream"])
+
+
+def test_prefill_host_validation(L):
+    assert prefill(L, dtype=5) == 3                       # GDN_ERR_DTYPE
+    assert prefill(L, Hq=3, Hv=4) == 2                    # Hv % Hq != 0
+    assert prefill(L, Dk=0) == 2
+    assert prefill(L, Dk=300) == 6                        # beyond 256
+    assert prefill(L, N=63) == 2                          # uniform packing needs N % B == 0
+    assert prefill(L, q=None) == 1
+    assert prefill(L, final=None) == 1
+    assert prefill(L, beta=None) == 1
+    assert prefill(L, v=P(3, 8)) == 4                     # 16-byte alignment
+    assert prefill(L, g=P(4, 2)) == 4
+    assert prefill(L, flags=1 << 9) == 6                  # unknown flag
+    assert prefill(L, init=P(7, 256), final=P(7)) == 5    # initial/final overlap
+    assert prefill(L, out=P(1, 64)) == 5                  # out overlaps q
+    assert prefill(L, final=P(3, 16)) == 5                # final_state overlaps v
+    assert prefill(L, B=0, N=0) == 0                      # nothing to do, nothing launched
+    assert prefill(L, B=0, N=4) == 2
+
+
+def decode(L, **kw):
+    args = dict(q=P(1), k=P(2), v=P(3), pool=P(4), P=16, ss=32 * 128 * 128, hs=128 * 128,
+                ri=P(5), wi=None, si=None, A=P(6), a=P(7), dtb=P(8), b=P(9), scale=0.1,
+                out=P(10), B=4, T=1, nh=1, H=32, HV=32, Dk=128, Dv=128, flags=0, status=None,
+                stream=None)
+    args.update(kw)
+    return L.gdn_decode(args["q"], args["k"], args["v"], args["pool"], args["P"], args["ss"],
+                        args["hs"], args["ri"], args["wi"], args["si"], args["A"], args["a"],
+                        args["dtb"], args["b"], args["scale"], args["out"], args["B"],
+                        args["T"], args["nh"], args["H"], args["HV"], args["Dk"], args["Dv"],
+                        args["flags"], args["status"], args["stream"])
+
+
+def test_decode_host_validation(L):
+    assert decode(L, H=16) == 2                           # H != HV
+    assert decode(L, T=17) == 6
+    assert decode(L, nh=5) == 6
+    assert decode(L, Dk=64) == 6
+    assert decode(L, Dv=96) == 6
+    assert decode(L, si=P(11), flags=2) == 2              # scatter + disable
+    assert decode(L, hs=100) == 2                         # head stride below Dv*Dk
+    assert decode(L, ss=16 * 128 * 128) == 2              # slot stride below HV*head_stride
+    assert decode(L, ss=32 * 128 * 128 + 2) == 4          # stride not a multiple of 4 elements
+    assert decode(L, pool=P(4, 8)) == 4                   # pool not 16-byte aligned
+    assert decode(L, q=P(1, 4)) == 4
+    assert decode(L, ri=None) == 1
+    assert decode(L, b=None) == 1
+    assert decode(L, out=P(4, 1024)) == 5                 # out inside the pool
+    assert decode(L, flags=1 << 7) == 6
+    assert decode(L, P=0) == 2
+    assert decode(L, B=0) == 0
+
+
+def test_binding_fails_loudly_without_library(monkeypatch, tmp_path):
+    import gated_deltanet_state_gdn_b200._binding as b
+    monkeypatch.setattr(b, "_lib", None)
+    monkeypatch.setattr(b, "LIB_PATH", str(tmp_path / "missing.so"))
+    with pytest.raises(RuntimeError, match="no fallback"):
+        b.lib()

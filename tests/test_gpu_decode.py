@@ -1,0 +1,212 @@
+"""GPU parity of gdn_decode against the float64 oracle (through the C ABI).
+
+Tolerance: relative L2 <= 2e-2 (bf16 activations, fp32 state) on outputs and on
+every written pool slot; pool slots nobody writes must stay bit-identical.
+"""
+import numpy as np
+import pytest
+import torch
+
+from _util import TOL_BF16, dev, f64, rel_l2
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def gdn():
+    import gated_deltanet_state_gdn_b200 as g
+    g.lib()
+    return g
+
+
+@pytest.fixture(scope="module")
+def W():
+    from gated_deltanet_state_gdn_b200 import workloads
+    return workloads
+
+
+def run_gpu(gdn, c, pool_dev=None, out=None, dev_status=None, disable=None):
+    pool = dev(c.pool) if pool_dev is None else pool_dev
+    o, _ = gdn.gdn_decode(dev(c.q), dev(c.k), dev(c.v), pool, dev(c.read_idx), dev(c.A_log),
+                          dev(c.a), dev(c.dt_bias), dev(c.b), scale=c.scale,
+                          out=None if out is None else dev(out),
+                          scatter_idx=dev(c.scatter_idx),
+                          disable_state_update=c.disable_state_update if disable is None
+                          else disable,
+                          use_qk_l2norm=c.use_qk_l2norm, write_idx=dev(c.write_idx),
+                          dev_status=dev_status)
+    torch.cuda.synchronize()
+    return o, pool
+
+
+def run_oracle(oracle_mod, c, rows=None, out=None):
+    """Oracle on all rows, or on a subset `rows` through a compact pool holding only their
+    read slots (returns outputs of those rows and the final per-row states)."""
+    if rows is None:
+        return oracle_mod.decode(f64(c.q), f64(c.k), f64(c.v), f64(c.pool), c.read_idx.numpy(),
+                                 f64(c.A_log), f64(c.a), f64(c.dt_bias), f64(c.b),
+                                 write_idx=None if c.write_idx is None else c.write_idx.numpy(),
+                                 scatter_idx=None if c.scatter_idx is None
+                                 else c.scatter_idx.numpy(),
+                                 scale=c.scale, use_qk_l2norm=c.use_qk_l2norm,
+                                 disable_state_update=c.disable_state_update,
+                                 out=None if out is None else f64(out))
+    rows = np.asarray(rows)
+    reads = c.read_idx.numpy()[rows]
+    assert (reads >= 0).all()
+    small = f64(c.pool[torch.from_numpy(reads.astype(np.int64))])
+    return oracle_mod.decode(f64(c.q[rows]), f64(c.k[rows]), f64(c.v[rows]), small,
+                             np.arange(len(rows), dtype=np.int32), f64(c.A_log),
+                             f64(c.a[rows]), f64(c.dt_bias), f64(c.b[rows]), scale=c.scale,
+                             use_qk_l2norm=c.use_qk_l2norm)
+
+
+def small_case(W, seed, **kw):
+    base = dict(P=64, B=12, T=1, nh=1, H=4, Dv=128, pad_frac=0.25)
+    base.update(kw)
+    return W.make_decode(seed, **base)
+
+
+@pytest.mark.parametrize("Dv", [64, 128])
+@pytest.mark.parametrize("write_mode", ["distinct", "same", "none"])
+def test_small_decode(gdn, W, oracle_mod, Dv, write_mode):
+    c = small_case(W, 100 + Dv, Dv=Dv, write_mode=write_mode)
+    sentinel = torch.full((12, 1, 4, Dv), -2.0, dtype=torch.bfloat16)
+    o, pool = run_gpu(gdn, c, out=sentinel)
+    ro, rp = run_oracle(oracle_mod, c, out=sentinel)
+    assert rel_l2(f64(o), ro) <= TOL_BF16
+    pad = (c.read_idx < 0).numpy()
+    assert pad.any()
+    assert torch.equal(o.cpu()[torch.from_numpy(pad)], sentinel[torch.from_numpy(pad)])
+    written = set(c.read_idx[~torch.from_numpy(pad)].tolist()) if c.write_idx is None else \
+        set(w for w in c.write_idx.tolist() if w >= 0)
+    pc = pool.cpu()
+    for s in range(c.pool.shape[0]):
+        if s in written:
+            assert rel_l2(f64(pc[s]), rp[s]) <= TOL_BF16, s
+        else:
+            assert torch.equal(pc[s], c.pool[s]), s
+
+
+@pytest.mark.parametrize("T,nh", [(2, 1), (4, 2), (3, 3), (16, 4), (1, 4)])
+def test_multi_token_and_householder(gdn, W, oracle_mod, T, nh):
+    c = small_case(W, 200 + 10 * T + nh, T=T, nh=nh, Dv=64, pad_frac=0.1)
+    o, pool = run_gpu(gdn, c)
+    ro, rp = run_oracle(oracle_mod, c)
+    assert rel_l2(f64(o), ro) <= TOL_BF16
+    assert rel_l2(f64(pool.cpu()), rp) <= TOL_BF16
+
+
+def test_scatter_with_negative_entries(gdn, W, oracle_mod):
+    c = small_case(W, 300, T=4, nh=2, Dv=64, write_mode="distinct", scatter=True, P=128)
+    c.scatter_idx[0, 1] = -1
+    c.scatter_idx[3, 0] = -5
+    o, pool = run_gpu(gdn, c)
+    ro, rp = run_oracle(oracle_mod, c)
+    assert rel_l2(f64(o), ro) <= TOL_BF16
+    pc = pool.cpu()
+    sc = set(int(x) for x, r in zip(c.scatter_idx.flatten().tolist(),
+                                    np.repeat(c.read_idx.numpy(), 4)) if x >= 0 and r >= 0)
+    for s in range(128):
+        if s in sc:
+            assert rel_l2(f64(pc[s]), rp[s]) <= TOL_BF16
+        else:  # includes the write slots: scatter skips the end write-back
+            assert torch.equal(pc[s], c.pool[s]), s
+
+
+def test_disable_state_update(gdn, W, oracle_mod):
+    c = small_case(W, 400, T=3, nh=2, Dv=128)
+    c.disable_state_update = True
+    o, pool = run_gpu(gdn, c)
+    ro, _ = run_oracle(oracle_mod, c)
+    assert rel_l2(f64(o), ro) <= TOL_BF16
+    assert torch.equal(pool.cpu(), c.pool)
+
+
+def test_bad_slot_sets_status_and_skips(gdn, W, oracle_mod):
+    c = small_case(W, 500, pad_frac=0.0, write_mode="distinct")
+    c.read_idx[2] = 1000        # beyond the pool: row skipped, flagged
+    c.write_idx[5] = 64         # beyond the pool: write-back skipped, flagged
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    sentinel = torch.full((12, 1, 4, 128), 5.0, dtype=torch.bfloat16)
+    o, pool = run_gpu(gdn, c, out=sentinel, dev_status=status)
+    assert int(status.item()) == 1
+    assert torch.equal(o[2].cpu(), sentinel[2])
+    ok_rows = [r for r in range(12) if r != 2]
+    ro, rp = run_oracle(oracle_mod, c, rows=ok_rows)
+    assert rel_l2(f64(o.cpu()[ok_rows]), ro) <= TOL_BF16
+    pc = pool.cpu()
+    for i, r in enumerate(ok_rows):
+        w = int(c.write_idx[r])
+        if w < 64:
+            assert rel_l2(f64(pc[w]), rp[i]) <= TOL_BF16
+    untouched = set(range(64)) - set(int(w) for w in c.write_idx.tolist() if w < 64)
+    for s in untouched:
+        if s != int(c.write_idx[2]):
+            assert torch.equal(pc[s], c.pool[s])
+
+
+def test_padded_pool_strides(gdn, W, oracle_mod):
+    """A pool with padding between heads and slots (dense rows) is used in place."""
+    c = small_case(W, 600, Dv=64, write_mode="same")
+    P, HV, Dv, Dk = c.pool.shape
+    big = torch.full((P, HV + 1, Dv + 4, Dk), 9.0, dtype=torch.float32, device="cuda")
+    view = big[:, :HV, :Dv, :]
+    view.copy_(dev(c.pool))
+    assert not view.is_contiguous()
+    o, _ = run_gpu(gdn, c, pool_dev=view)
+    ro, rp = run_oracle(oracle_mod, c)
+    assert rel_l2(f64(o), ro) <= TOL_BF16
+    assert rel_l2(f64(view.cpu()), rp) <= TOL_BF16
+    assert (big[:, HV] == 9.0).all() and (big[:, :, Dv:] == 9.0).all()
+
+
+def test_deterministic(gdn, W):
+    c = small_case(W, 700, T=4, nh=2, Dv=128, write_mode="distinct")
+    outs = []
+    for _ in range(3):
+        o, pool = run_gpu(gdn, c)
+        outs.append((o.clone(), pool.clone()))
+    for o, p in outs[1:]:
+        assert torch.equal(o, outs[0][0]) and torch.equal(p, outs[0][1])
+
+
+# ---------------------------------------------------------------- full sizes
+def test_full_decode_pool(gdn, W, oracle_mod):
+    """Pool [1024, 32, 128, 128] (2 GiB), B=256 with 13 padding rows: 24 sampled rows against
+    the oracle, every padding row and every slot outside the write set bit-identical."""
+    c = W.decode_pool_case()
+    pool = dev(c.pool)
+    o, _ = run_gpu(gdn, c, pool_dev=pool)
+    reads = c.read_idx.numpy()
+    live = np.nonzero(reads >= 0)[0]
+    rng = np.random.default_rng(0)
+    rows = np.sort(rng.choice(live, 24, replace=False))
+    ro, rp = run_oracle(oracle_mod, c, rows=rows)
+    oc = o.cpu()
+    assert rel_l2(f64(oc[torch.from_numpy(rows)]), ro) <= TOL_BF16
+    for i, r in enumerate(rows):
+        w = int(c.write_idx[r])
+        assert rel_l2(f64(pool[w].cpu()), rp[i]) <= TOL_BF16
+    pad = np.nonzero(reads < 0)[0]
+    assert len(pad) == 13
+    assert (oc[torch.from_numpy(pad)] == 0).all()
+    written = set(int(w) for w in c.write_idx.tolist() if w >= 0)
+    untouched = [s for s in range(1024) if s not in written]
+    idx = torch.tensor(untouched, device="cuda")
+    assert torch.equal(pool.index_select(0, idx).cpu(), c.pool[torch.tensor(untouched)])
+    assert torch.isfinite(o.float()).all()
+
+
+def test_full_mtp(gdn, W, oracle_mod):
+    """B=64, T=4, nh=2, H=16, Dv=64, per-token scatter into 256 distinct slots: every output
+    and every scattered slot against the oracle."""
+    c = W.mtp_case()
+    o, pool = run_gpu(gdn, c)
+    ro, rp = run_oracle(oracle_mod, c)
+    assert rel_l2(f64(o), ro) <= TOL_BF16
+    pc = pool.cpu()
+    sc = c.scatter_idx.flatten().tolist()
+    assert rel_l2(f64(pc[sc]), rp[sc]) <= TOL_BF16
+    others = [s for s in range(512) if s not in set(sc)]
+    assert torch.equal(pc[others], c.pool[others])

@@ -1,0 +1,206 @@
+"""GPU parity of gdn_prefill against the float64 oracle (through the C ABI).
+
+Tolerances (relative L2 over the whole tensor): 1e-4 for fp32 activations,
+2e-2 for bf16 activations with the fp32 state.
+"""
+import json
+import os
+
+import numpy as np
+import pytest
+import torch
+
+from _util import (TOL_BF16, TOL_F32, dev, f64, oracle_prefill_case, rel_l2, run_gpu_prefill,
+                   sub_case_head)
+
+pytestmark = pytest.mark.gpu
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden", "p1_worked_examples.json")
+
+
+@pytest.fixture(scope="module")
+def gdn():
+    import gated_deltanet_state_gdn_b200 as g
+    g.lib()
+    return g
+
+
+@pytest.fixture(scope="module")
+def W():
+    from gated_deltanet_state_gdn_b200 import workloads
+    return workloads
+
+
+@pytest.mark.parametrize("sequential", [True, False])
+def test_worked_examples(gdn, sequential):
+    for e in json.load(open(GOLDEN))["examples"]:
+        q = torch.tensor(e["q"], dtype=torch.float32)
+        B, S, Dk = q.shape
+        k = torch.tensor(e["k"], dtype=torch.float32)
+        v = torch.tensor(e["v"], dtype=torch.float32)
+        Dv = v.shape[2]
+        g = torch.log(torch.tensor(e["gamma"], dtype=torch.float32)).reshape(B * S, 1)
+        beta = torch.tensor(e["beta"], dtype=torch.float32).reshape(B * S, 1)
+        out, fs = gdn.gdn_prefill(dev(q.reshape(B * S, 1, Dk)), dev(k.reshape(B * S, 1, Dk)),
+                                  dev(v.reshape(B * S, 1, Dv)), dev(g), dev(beta),
+                                  num_requests=B, scale=1.0, sequential=sequential)
+        torch.cuda.synchronize()
+        np.testing.assert_allclose(f64(out).reshape(B, S, Dv), np.array(e["outputs"]),
+                                   atol=1e-5)
+        np.testing.assert_allclose(f64(fs)[:, 0].transpose(0, 2, 1),
+                                   np.array(e["final_state"]), atol=1e-5)
+
+
+def test_tiny_oracle_case_fp32(gdn, W, oracle_mod):
+    c = W.tiny_oracle_case()
+    out, fs = run_gpu_prefill(c)
+    ro, rf = oracle_prefill_case(oracle_mod, c)
+    assert rel_l2(f64(out), ro) <= TOL_F32
+    assert rel_l2(f64(fs), rf) <= TOL_F32
+
+
+@pytest.mark.parametrize("dtype,tol", [(torch.float32, TOL_F32), (torch.bfloat16, TOL_BF16)])
+def test_odd_head_sizes_gqa(gdn, W, oracle_mod, dtype, tol):
+    """The op page's example call shape: T=4, Hq=1, Hv=2, Dk=12, Dv=9, with an initial state."""
+    c = W.make_prefill(11, [4], 1, 2, 12, 9, dtype=dtype, uniform=True, init_std=0.5,
+                       qk_l2norm=True)
+    out, fs = run_gpu_prefill(c)
+    ro, rf = oracle_prefill_case(oracle_mod, c)
+    assert rel_l2(f64(out), ro) <= tol
+    assert rel_l2(f64(fs), rf) <= tol
+
+
+@pytest.mark.parametrize("Dk,Dv", [(1, 1), (33, 7), (256, 256), (128, 40)])
+def test_head_size_range_fp32(gdn, W, oracle_mod, Dk, Dv):
+    c = W.make_prefill(12 + Dk, [3, 17, 0, 9], 2, 4, Dk, Dv, dtype=torch.float32, init_std=0.3,
+                       qk_l2norm=True)
+    out, fs = run_gpu_prefill(c)
+    ro, rf = oracle_prefill_case(oracle_mod, c)
+    assert rel_l2(f64(out), ro) <= TOL_F32
+    assert rel_l2(f64(fs), rf) <= TOL_F32
+
+
+RAGGED = [1, 64, 65, 130, 0, 200, 63, 128]
+
+
+@pytest.mark.parametrize("sequential", [True, False])
+@pytest.mark.parametrize("l2norm", [True, False])
+def test_ragged_bf16_d128(gdn, W, oracle_mod, sequential, l2norm):
+    """Several 64-token chunks per request, ragged tails, an empty request, GQA 2 -> 4."""
+    c = W.make_prefill(21 + int(l2norm), RAGGED, 2, 4, 128, 128, init_std=0.02,
+                       qk_l2norm=l2norm, host_norm_qk=not l2norm)
+    out, fs = run_gpu_prefill(c, sequential=sequential)
+    ro, rf = oracle_prefill_case(oracle_mod, c)
+    assert rel_l2(f64(out), ro) <= TOL_BF16
+    assert rel_l2(f64(fs), rf) <= TOL_BF16
+    # the empty request copies its initial state through bit for bit
+    assert torch.equal(fs[4].cpu(), c.initial_state[4])
+
+
+@pytest.mark.parametrize("sequential", [True, False])
+def test_cu_seqlens_clamp_and_uncovered_tokens(gdn, W, oracle_mod, sequential):
+    c = W.make_prefill(31, [40, 30, 40, 20, 10], 1, 2, 128, 128, init_std=0.1, qk_l2norm=True)
+    N = c.N  # 140
+    sentinel = torch.full((N, 2, 128), 3.0, dtype=torch.bfloat16)
+    # (a) tokens 0..9 and N-20..N-1 belong to no request and keep the caller's values;
+    #     request 1 is empty, request 4 is decreasing (empty)
+    c.cu_seqlens = torch.tensor([10, 40, 40, 60, N - 20, 3], dtype=torch.int32)
+    out, fs = run_gpu_prefill(c, sequential=sequential, out=sentinel)
+    ro, rf = oracle_prefill_case(oracle_mod, c, out=f64(sentinel))
+    assert rel_l2(f64(out), ro) <= TOL_BF16
+    assert torch.equal(out[:10].cpu(), sentinel[:10])
+    assert torch.equal(out[N - 20:].cpu(), sentinel[N - 20:])
+    assert rel_l2(f64(fs), rf) <= TOL_BF16
+    assert torch.equal(fs[1].cpu(), c.initial_state[1])
+    assert torch.equal(fs[4].cpu(), c.initial_state[4])
+    # (b) out-of-range entries clamp to [0, N]; request 1 decreasing -> empty
+    c.cu_seqlens = torch.tensor([-9, 40, 30, N + 500], dtype=torch.int32)
+    c.initial_state = c.initial_state[:3].contiguous()
+    c.B = 3
+    out, fs = run_gpu_prefill(c, sequential=sequential, out=sentinel)
+    ro, rf = oracle_prefill_case(oracle_mod, c, out=f64(sentinel))
+    keep = np.r_[0:30, 40:N]  # tokens 30..39 lie in two requests: undefined outputs
+    assert rel_l2(f64(out)[keep], ro[keep]) <= TOL_BF16
+    assert rel_l2(f64(fs), rf) <= TOL_BF16
+    assert torch.equal(fs[1].cpu(), c.initial_state[1])
+
+
+@pytest.mark.parametrize("sequential", [True, False])
+def test_zero_gate_and_zero_initial_state(gdn, W, oracle_mod, sequential):
+    """gamma = 0 (g = -inf) wipes the state; no initial state means zero."""
+    c = W.make_prefill(41, [70, 130], 1, 1, 128, 128, init_std=None, qk_l2norm=True)
+    c.g[5] = float("-inf")
+    c.g[100] = float("-inf")
+    c.g[101:110] = 0.0
+    out, fs = run_gpu_prefill(c, sequential=sequential)
+    ro, rf = oracle_prefill_case(oracle_mod, c)
+    assert np.isfinite(f64(out)).all() and np.isfinite(f64(fs)).all()
+    assert rel_l2(f64(out), ro) <= TOL_BF16
+    assert rel_l2(f64(fs), rf) <= TOL_BF16
+
+
+def test_noncontiguous_inputs_and_inputs_unchanged(gdn, W, oracle_mod):
+    c = W.make_prefill(51, [33, 70], 2, 4, 128, 128, init_std=0.1, qk_l2norm=True)
+    qd = dev(c.q).transpose(0, 1).contiguous().transpose(0, 1)   # same values, other strides
+    assert not qd.is_contiguous()
+    kd, vd, gd, bd = dev(c.k), dev(c.v), dev(c.g), dev(c.beta)
+    init = dev(c.initial_state)
+    snap = [t.clone() for t in (qd, kd, vd, gd, bd, init)]
+    out, fs = gdn.gdn_prefill(qd, kd, vd, gd, bd, dev(c.cu_seqlens), init, scale=c.scale,
+                              qk_l2norm=True)
+    torch.cuda.synchronize()
+    for a, b in zip(snap, (qd, kd, vd, gd, bd, init)):
+        assert torch.equal(a, b)
+    ro, rf = oracle_prefill_case(oracle_mod, c)
+    assert rel_l2(f64(out), ro) <= TOL_BF16
+
+
+@pytest.mark.parametrize("sequential", [True, False])
+def test_deterministic(gdn, W, sequential):
+    c = W.make_prefill(61, [300, 77], 2, 4, 128, 128, init_std=0.02, qk_l2norm=True)
+    runs = [run_gpu_prefill(c, sequential=sequential) for _ in range(3)]
+    for o, f in runs[1:]:
+        assert torch.equal(o, runs[0][0]) and torch.equal(f, runs[0][1])
+
+
+def test_rank4_spelling(gdn, W, oracle_mod):
+    c = W.make_prefill(71, [50, 50], 1, 2, 128, 128, uniform=True, init_std=0.1,
+                       qk_l2norm=True)
+    q4 = dev(c.q).reshape(2, 50, 1, 128)
+    k4 = dev(c.k).reshape(2, 50, 1, 128)
+    v4 = dev(c.v).reshape(2, 50, 2, 128)
+    out, fs = gdn.gdn_prefill(q4, k4, v4, dev(c.g).reshape(2, 50, 2),
+                              dev(c.beta).reshape(2, 50, 2), None, dev(c.initial_state),
+                              scale=c.scale, qk_l2norm=True)
+    torch.cuda.synchronize()
+    ro, rf = oracle_prefill_case(oracle_mod, c)
+    assert rel_l2(f64(out), ro) <= TOL_BF16
+    assert rel_l2(f64(fs), rf) <= TOL_BF16
+
+
+# ---------------------------------------------------------------- full sizes
+def _sampled_heads_parity(oracle_mod, c, out, fs, heads):
+    o = f64(out)
+    f = f64(fs)
+    for h in heads:
+        s = sub_case_head(c, h)
+        ro, rf = oracle_prefill_case(oracle_mod, s)
+        assert rel_l2(o[:, h:h + 1], ro) <= TOL_BF16, h
+        assert rel_l2(f[:, h:h + 1], rf) <= TOL_BF16, h
+
+
+def test_full_ragged_prefill_sampled_heads(gdn, W, oracle_mod):
+    """8 requests U[1,4096], Hq=16, Hv=32, D=128: every output of heads 0, 13 (GQA pair of 12)
+    and 31 against the oracle, and finiteness everywhere."""
+    c = W.ragged_prefill_case()
+    out, fs = run_gpu_prefill(c)
+    assert torch.isfinite(out.float()).all() and torch.isfinite(fs).all()
+    _sampled_heads_parity(oracle_mod, c, out, fs, [0, 13, 31])
+
+
+def test_full_long_prefill_sampled_heads(gdn, W, oracle_mod):
+    """B=1, S=32768: all 32768 outputs of heads 0 and 31 and their final states."""
+    c = W.long_prefill_case()
+    out, fs = run_gpu_prefill(c)
+    assert torch.isfinite(out.float()).all() and torch.isfinite(fs).all()
+    _sampled_heads_parity(oracle_mod, c, out, fs, [0, 31])
