@@ -395,7 +395,7 @@ def main():
     value = tokens / (ms_per_step / 1e3)
     launches = args.steps
 
-    chunked = gdn.prefill_uses_chunked(case.q.dtype, Dk, Dv)
+    chunked = gdn.prefill_uses_chunked(case.q.dtype, Hv, Dk, Dv)
     avg_launch_s = statistics.mean(launch_ms) / 1e3
     if chunked:
         flops = case.N * Hv * prefill_flops_per_token_head(Dk, Dv)

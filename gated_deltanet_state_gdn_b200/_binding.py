@@ -35,6 +35,8 @@ GDN_DISABLE_STATE_UPDATE = 2
 GDN_DECODE_QK_L2NORM = 4
 
 GDN_DEV_BAD_SLOT = 1
+GDN_DEV_TIMEOUT = 2
+GDN_DEV_INTERNAL = 4
 
 EXPORTED = ("gdn_prefill", "gdn_decode", "gdn_status_string", "gdn_last_error",
             "gdn_abi_version", "gdn_prefill_uses_chunked")
@@ -78,14 +80,16 @@ def lib():
         L.gdn_abi_version.restype = i32
         L.gdn_abi_version.argtypes = []
         L.gdn_prefill_uses_chunked.restype = i32
-        L.gdn_prefill_uses_chunked.argtypes = [ctypes.c_int, i32, i32, u32]
+        L.gdn_prefill_uses_chunked.argtypes = [ctypes.c_int, i32, i32, i32, u32]
         _lib = L
     return _lib
 
 
-def prefill_uses_chunked(dtype: torch.dtype, Dk: int, Dv: int, sequential: bool = False) -> bool:
+def prefill_uses_chunked(dtype: torch.dtype, Hv: int, Dk: int, Dv: int,
+                         sequential: bool = False) -> bool:
+    """True when gdn_prefill would run the chunked tensor-core kernel for these sizes."""
     code = GDN_BF16 if dtype == torch.bfloat16 else GDN_F32
-    return bool(lib().gdn_prefill_uses_chunked(code, Dk, Dv,
+    return bool(lib().gdn_prefill_uses_chunked(code, Hv, Dk, Dv,
                                                GDN_PREFILL_SEQUENTIAL if sequential else 0))
 
 

@@ -53,12 +53,13 @@ const char *gdn_status_string(int32_t s)
     }
 }
 
-int32_t gdn_prefill_uses_chunked(gdn_dtype dtype, int32_t Dk, int32_t Dv, uint32_t flags)
+int32_t gdn_prefill_uses_chunked(gdn_dtype dtype, int32_t Hv, int32_t Dk, int32_t Dv,
+                                 uint32_t flags)
 {
     if (flags & GDN_PREFILL_SEQUENTIAL) return 0;
     GdnPrefillArgs a;
     memset(&a, 0, sizeof(a));
-    a.dtype = dtype; a.Dk = Dk; a.Dv = Dv; a.Hq = 1; a.Hv = 1;
+    a.dtype = dtype; a.Dk = Dk; a.Dv = Dv; a.Hq = 1; a.Hv = Hv;
     return prefill_chunked_supported(a) ? 1 : 0;
 }
 

@@ -1,9 +1,1105 @@
-// prefill_chunk.cu -- chunked tensor-core Gated DeltaNet prefill (sm_100a).
+// prefill_chunk.cu -- chunked Gated DeltaNet prefill on sm_100a tensor cores.
+//
+// Operation: the recurrence of "com.microsoft.GatedDeltaNet" (Description),
+//   S_t = exp(g_t) S_{t-1} + k_t (beta_t (v_t - exp(g_t) S_{t-1}^T k_t))^T,
+//   o_t = scale * S_t^T q_t,
+// for bf16 q/k/v with Dk = Dv = 128, computed 64 tokens at a time.  The
+// chunk form (derived from the recurrence; the op page names a chunk-parallel
+// prefill with chunk_size 64 and states that the chunk size does not change
+// the result) is, for a chunk with incoming state S0 (Dk x Dv), cumulative
+// log-decay G_i = sum_{l<=i} g_l, Gamma_i = exp(G_i):
+//   A_ij = beta_i (k_i . k_j) exp(G_i - G_j)   (j < i),   T = (I + A)^-1
+//   W    = T diag(beta Gamma) K,   U~ = T diag(beta) V
+//   U    = U~ - W S0
+//   O    = scale (diag(Gamma) Q S0 + P U),  P_ij = (q_i . k_j) exp(G_i - G_j) (j <= i)
+//   S_C  = Gamma_C S0 + (diag(exp(G_C - G)) K)^T U
+// All state-dependent products are evaluated transposed (rows = value index
+// dv), so every tcgen05 MMA here has M = 128:
+//   (G)  [K; Q] K^T                         -> TMEM  (Gram, 128 x 64)
+//   (W)  W^T  = K^T . Tbg^T                 -> TMEM  (Tbg = T diag(beta Gamma))
+//   (U~) U^T  = V^T . Tb^T                  -> TMEM  (Tb  = T diag(beta))
+//   (1a) U^T += S^T . (-W)^T                 (bf16 copy of S^T from SMEM)
+//   (1b) Y    = S^T . Q^T
+//   (2)  S^T += (U^T diag(exp(G_C - G))) . K (fp32 accumulator stays in TMEM)
+//   (3)  Z    = U^T . P^T
+//   O^T = scale (Y diag(Gamma) + Z)
+// TMEM (512 columns): S^T [0,128) | U^T x2 [128,256) | Y x2 [256,384) |
+// Z [384,448) | Gram/W^T [448,512).
+//
+// CTA = 10 warps, one (request, value head) unit at a time, persistent over a
+// longest-first unit list:
+//   warps 0-3  state warpgroup: TMEM <-> bf16 operand tiles, outputs, state I/O
+//   warps 4-7  prep warpgroup: L2 norm, gates, Gram -> A and P, the 64x64
+//              unit-triangular solve, T/W tiles (runs one chunk ahead)
+//   warp  8    TMA producer (q/k/v/g/beta tiles, two stages)
+//   warp  9    TMEM owner and single-thread UMMA issuer
+// Every wait on an mbarrier is bounded; on timeout the kernel sets
+// GDN_DEV_TIMEOUT in the status word, drains and exits.
+#include <cudaTypedefs.h>
+#include <stdio.h>
+#include <string.h>
+
 #include "common.cuh"
+#include "sm100.cuh"
 
-bool prefill_chunked_supported(const GdnPrefillArgs &) { return false; }
+using namespace sm100;
 
-cudaError_t launch_prefill_chunked(const GdnPrefillArgs &, cudaStream_t)
+namespace gdn_chunk {
+
+constexpr int C = 64;       // chunk length (tokens)
+constexpr int D = 128;      // Dk = Dv
+constexpr int NTHREADS = 320;
+constexpr int MAX_UNITS = 128;     // per CTA per batch of the unit list
+constexpr float G_FLOOR = -30.f;   // per-token log-decay floor (exp(-30) ~ 9e-14)
+constexpr float LOG2E = 1.4426950408889634f;
+
+// ---- shared-memory map (bytes from a 1024-aligned base) ----
+constexpr uint32_t OFF_KQ0 = 0;          // [kb][128 rows: K 0-63, Q 64-127][128 B], 32 KB
+constexpr uint32_t OFF_KQ1 = 32768;
+constexpr uint32_t KQ_KB = 16384;        // k-block (64 dk) stride inside a KQ stage
+constexpr uint32_t OFF_V = 65536;        // [dv half][64 rows j][128 B], 16 KB
+constexpr uint32_t V_HALF = 8192;
+constexpr uint32_t OFF_SBF = 81920;      // [dk half][128 rows dv][128 B], 32 KB
+constexpr uint32_t SBF_KB = 16384;
+constexpr uint32_t OFF_WNEG = 114688;    // [128 rows dk][64 i], 16 KB (MN-major B)
+constexpr uint32_t OFF_P0 = 131072;      // [64 rows i][64 j], 8 KB
+constexpr uint32_t OFF_P1 = 139264;
+constexpr uint32_t OFF_TB = 147456;      // [64 rows i][64 j], 8 KB
+constexpr uint32_t OFF_TBG = 155648;
+constexpr uint32_t OFF_UBF = 163840;     // [128 rows dv][64 i], 16 KB
+constexpr uint32_t OFF_UBFD = 180224;
+constexpr uint32_t OFF_SOLVE = 196608;   // 16 blocks of 16 x 20 fp32
+constexpr uint32_t SOLVE_LD = 20;        // padded row stride (floats)
+constexpr uint32_t SOLVE_BLK = 16 * SOLVE_LD;  // floats per block
+constexpr uint32_t OFF_GB0 = OFF_SOLVE + 16 * SOLVE_BLK * 4;   // g tile 1 KB + beta tile 1 KB
+constexpr uint32_t OFF_GB1 = OFF_GB0 + 2048;
+constexpr uint32_t OFF_GATE0 = OFF_GB1 + 2048;                 // processed gates, 2 KB
+constexpr uint32_t OFF_GATE1 = OFF_GATE0 + 2048;
+constexpr uint32_t OFF_UNITS = OFF_GATE1 + 2048;               // int4 x MAX_UNITS
+constexpr uint32_t OFF_BARS = OFF_UNITS + MAX_UNITS * 16;
+constexpr uint32_t NUM_BARS = 19;
+constexpr uint32_t OFF_MISC = OFF_BARS + 256;                  // tmem base, abort flag, count
+constexpr uint32_t SMEM_USED = OFF_MISC + 64;
+constexpr uint32_t SMEM_BYTES = SMEM_USED + 1024;              // + alignment slack
+static_assert(SMEM_BYTES <= 232448, "shared memory budget");
+static_assert(OFF_GB0 % 1024 == 0, "alignment");
+
+// gate-array offsets (floats) inside a GATE stage
+constexpr int GA_G2 = 0;       // G_i * log2(e)
+constexpr int GA_CF = 64;      // exp(Gend_J(i) - G_i): column factor to the end of i's 16-block
+constexpr int GA_BETA = 128;   // beta_i (0 beyond the request)
+constexpr int GA_BGAM = 192;   // beta_i exp(G_i)
+constexpr int GA_GAM = 256;    // exp(G_i)
+constexpr int GA_DEC = 320;    // exp(G_C - G_i)
+constexpr int GA_GEND = 384;   // G_end of each 16-block * log2(e)  [4]
+constexpr int GA_GC = 388;     // exp(G_C)
+
+// barrier indices
+enum {
+    B_KQ_FULL = 0, B_KQ_EMPTY = 2, B_V_FULL = 4, B_V_EMPTY = 5, B_GATE_FULL = 6,
+    B_GATE_EMPTY = 8, B_NORM = 10, B_G_DONE = 11, B_T_READY = 12, B_WU_DONE = 13,
+    B_WNEG = 14, B_S_READY = 15, B_U_DONE = 16, B_E1 = 17, B_SZ_DONE = 18
+};
+
+// TMEM columns
+constexpr uint32_t TM_S = 0, TM_U = 128, TM_Y = 256, TM_Z = 384, TM_GW = 448;
+
+struct __align__(64) Params {
+    CUtensorMap tm_q;     // (128, Hq, N) bf16, box (64, 1, 64), 128B swizzle
+    CUtensorMap tm_k;
+    CUtensorMap tm_v;     // (128, Hv, N)
+    CUtensorMap tm_g;     // (Hv, N) fp32, box (4, 64)
+    CUtensorMap tm_beta;
+    const int32_t *cu_seqlens;
+    const float *initial_state;
+    float *final_state;
+    __nv_bfloat16 *out;
+    int32_t *dev_status;
+    int64_t N;
+    int32_t B, Hq, Hv;
+    float scale;
+    int32_t qk_l2norm;
+};
+
+// --------------------------------------------------------------------------
+struct Ctx {
+    uint8_t *smem;
+    uint32_t sbase;        // shared address of smem
+    volatile int *abort_flag;
+    int32_t *dev_status;
+
+    __device__ uint32_t bar(int i) const { return sbase + OFF_BARS + 8u * i; }
+
+    // bounded wait; returns false on timeout or when another role aborted
+    __device__ bool wait(int b, uint32_t parity) const
+    {
+        if (mbar_try_wait(bar(b), parity)) return true;
+        const long long t0 = clock64();
+        while (true) {
+            if (mbar_try_wait(bar(b), parity)) return true;
+            if (*abort_flag) return false;
+            if (clock64() - t0 > (1ll << 31)) {
+                *abort_flag = 1;
+                if (dev_status) atomicOr(dev_status, GDN_DEV_TIMEOUT);
+                return false;
+            }
+        }
+    }
+    __device__ bool aborted() const { return *abort_flag != 0; }
+};
+
+struct Unit {
+    int b, h, start, len;
+};
+
+__device__ __forceinline__ Unit load_unit(const uint8_t *smem, int k)
 {
-    return cudaErrorNotSupported;
+    const int4 u = reinterpret_cast<const int4 *>(smem + OFF_UNITS)[k];
+    return Unit{u.x, u.y, u.z, u.w};
+}
+
+__device__ __forceinline__ int64_t clampi(int64_t x, int64_t lo, int64_t hi)
+{
+    return x < lo ? lo : (x > hi ? hi : x);
+}
+
+// 16-byte chunk `c` of row `r` in a 128B-swizzled tile whose base is 1024-aligned
+__device__ __forceinline__ uint32_t sw128(uint32_t row, uint32_t c)
+{
+    return row * 128u + ((c ^ (row & 7u)) << 4);
+}
+
+__device__ __forceinline__ uint4 pack8_bf16(const float *x)
+{
+    uint4 r;
+    r.x = gdn::pack_bf16x2(x[0], x[1]);
+    r.y = gdn::pack_bf16x2(x[2], x[3]);
+    r.z = gdn::pack_bf16x2(x[4], x[5]);
+    r.w = gdn::pack_bf16x2(x[6], x[7]);
+    return r;
+}
+
+__device__ __forceinline__ void unpack8_bf16(uint4 r, float *x)
+{
+    const uint32_t w[4] = {r.x, r.y, r.z, r.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        __nv_bfloat162 h = *reinterpret_cast<const __nv_bfloat162 *>(&w[i]);
+        float2 f = __bfloat1622float2(h);
+        x[2 * i] = f.x;
+        x[2 * i + 1] = f.y;
+    }
+}
+
+// --------------------------------------------------------------------------
+// Unit list: requests sorted by length (longest first), heads fastest; unit u
+// goes to CTA (u mod G) on even waves and G-1-(u mod G) on odd waves.
+__device__ void build_unit_list(const Params &p, uint8_t *smem, int batch0, int *count_out)
+{
+    int *ord = reinterpret_cast<int *>(smem + OFF_UBF);   // scratch: up to 8192 ints
+    const int B = p.B;
+    const int tid = threadIdx.x;
+    const bool sorted = B <= 8192;
+    auto req_range = [&](int b, int &s, int &l) {
+        int64_t st, en;
+        if (p.cu_seqlens) {
+            st = clampi(p.cu_seqlens[b], 0, p.N);
+            en = clampi(p.cu_seqlens[b + 1], 0, p.N);
+        } else {
+            const int64_t S = p.N / B;
+            st = (int64_t)b * S;
+            en = st + S;
+        }
+        s = (int)st;
+        l = en > st ? (int)(en - st) : 0;
+    };
+    if (sorted) {
+        for (int b = tid; b < B; b += NTHREADS) {
+            int sb, lb;
+            req_range(b, sb, lb);
+            int rank = 0;
+            for (int o = 0; o < B; ++o) {
+                int so, lo;
+                req_range(o, so, lo);
+                rank += (lo > lb) || (lo == lb && o < b);
+            }
+            ord[rank] = b;
+        }
+    }
+    __syncthreads();
+    const int G = gridDim.x;
+    const int U = B * p.Hv;
+    const int c = blockIdx.x;
+    int4 *list = reinterpret_cast<int4 *>(smem + OFF_UNITS);
+    // number of units of this CTA from wave batch0 on
+    int total = 0;
+    {
+        const int waves = (U + G - 1) / G;
+        for (int w = batch0; w < waves && total < MAX_UNITS; ++w) {
+            const int u = w * G + ((w & 1) ? (G - 1 - c) : c);
+            if (u < U) {
+                if (tid == 0) {
+                    const int r = u / p.Hv;
+                    const int h = u - r * p.Hv;
+                    const int b = sorted ? ord[r] : r;
+                    int s, l;
+                    req_range(b, s, l);
+                    list[total] = make_int4(b, h, s, l);
+                }
+                ++total;
+            }
+        }
+    }
+    *count_out = total;
+}
+
+// --------------------------------------------------------------------------
+// warp-level 16x16x16 tf32 products on padded fp32 blocks (row stride SOLVE_LD)
+// acc[nh][.] += X(16x16) * Y(16x16), fragments of mma.m16n8k8
+__device__ __forceinline__ void blk_mma(float (&acc)[2][4], const float *X, const float *Y)
+{
+    const int lane = threadIdx.x & 31;
+    const int g = lane >> 2, t = lane & 3;
+#pragma unroll
+    for (int kh = 0; kh < 2; ++kh) {
+        uint32_t a[4];
+        a[0] = to_tf32(X[g * SOLVE_LD + 8 * kh + t]);
+        a[1] = to_tf32(X[(g + 8) * SOLVE_LD + 8 * kh + t]);
+        a[2] = to_tf32(X[g * SOLVE_LD + 8 * kh + t + 4]);
+        a[3] = to_tf32(X[(g + 8) * SOLVE_LD + 8 * kh + t + 4]);
+#pragma unroll
+        for (int nh = 0; nh < 2; ++nh) {
+            uint32_t b[2];
+            b[0] = to_tf32(Y[(8 * kh + t) * SOLVE_LD + 8 * nh + g]);
+            b[1] = to_tf32(Y[(8 * kh + t + 4) * SOLVE_LD + 8 * nh + g]);
+            mma_tf32_16x8x8(acc[nh], a, b);
+        }
+    }
+}
+
+__device__ __forceinline__ void blk_store(float *Z, const float (&acc)[2][4], float sgn)
+{
+    const int lane = threadIdx.x & 31;
+    const int g = lane >> 2, t = lane & 3;
+#pragma unroll
+    for (int nh = 0; nh < 2; ++nh) {
+        Z[g * SOLVE_LD + 8 * nh + 2 * t] = sgn * acc[nh][0];
+        Z[g * SOLVE_LD + 8 * nh + 2 * t + 1] = sgn * acc[nh][1];
+        Z[(g + 8) * SOLVE_LD + 8 * nh + 2 * t] = sgn * acc[nh][2];
+        Z[(g + 8) * SOLVE_LD + 8 * nh + 2 * t + 1] = sgn * acc[nh][3];
+    }
+}
+
+// SOLVE slots: 0-3 A_II (strictly lower), 4 A_10, 5 A_32, 6-9 A_20 A_21 A_30 A_31
+// (later X, later T_20 T_21 T_30 T_31), 10-13 D_I = (I + A_II)^-1, 14 T_10, 15 T_32.
+__device__ __forceinline__ int a_slot(int I, int J)
+{
+    // J < I
+    if (I == 1) return 4;                      // (1,0)
+    if (I == 2) return 6 + J;                  // (2,0) (2,1)
+    return J == 2 ? 5 : 8 + J;                 // (3,2) -> 5, (3,0) (3,1) -> 8, 9
+}
+
+__device__ __forceinline__ int t_slot(int I, int J)
+{
+    // J <= I
+    if (I == J) return 10 + I;
+    if (I == 1) return 14;
+    if (I == 3 && J == 2) return 15;
+    if (I == 2) return 6 + J;
+    return 8 + J;
+}
+
+// ========================================================================== kernel
+__global__ void __launch_bounds__(NTHREADS, 1) gdn_prefill_chunk_kernel(const __grid_constant__ Params p)
+{
+    extern __shared__ uint8_t smem_raw[];
+    // align the shared-window offset (not the generic address) to 1024 bytes: the
+    // 128-byte swizzle of TMA and UMMA is a function of shared-address bits [4, 10)
+    const uint32_t raw_base = smem_u32(smem_raw);
+    uint8_t *smem = smem_raw + ((1024u - (raw_base & 1023u)) & 1023u);
+    const uint32_t sbase = smem_u32(smem);
+    const int tid = threadIdx.x;
+    const int warp = tid >> 5;
+    const int lane = tid & 31;
+
+    // layout self-check: swizzled tiles need a 1024-aligned base, tensor maps 64 bytes
+    if ((sbase & 1023u) != 0 || (reinterpret_cast<uintptr_t>(&p.tm_q) & 63) != 0) {
+        if (tid == 0 && p.dev_status) atomicOr(p.dev_status, GDN_DEV_INTERNAL);
+        return;
+    }
+
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + OFF_MISC + 4);
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + OFF_MISC);
+    int *count_slot = reinterpret_cast<int *>(smem + OFF_MISC + 8);
+    Ctx cx{smem, sbase, abort_flag, p.dev_status};
+
+    if (tid == 0) {
+        *abort_flag = 0;
+        const uint32_t counts[NUM_BARS] = {1, 1, 1, 1, 1, 1, 1, 1, 1, 1, 1, 1, 1, 1, 1, 1, 1, 1, 1};
+        for (int i = 0; i < (int)NUM_BARS; ++i) mbar_init(cx.bar(i), counts[i]);
+        fence_mbar_init();
+    }
+    if (warp == 8 && lane == 0) {
+        prefetch_tmap(&p.tm_q);
+        prefetch_tmap(&p.tm_k);
+        prefetch_tmap(&p.tm_v);
+        prefetch_tmap(&p.tm_g);
+        prefetch_tmap(&p.tm_beta);
+    }
+    if (warp == 9) {
+        tmem_alloc(sbase + OFF_MISC, 512);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+
+    // per-role pipeline counters (persist across units and batches)
+    uint32_t kq_use[2] = {0, 0}, v_use = 0;                       // TMA
+    uint32_t m_norm = 0, m_t = 0, m_wneg = 0, m_s = 0, m_e1 = 0;  // MMA
+    uint32_t m_kq[2] = {0, 0}, m_v = 0;
+    uint32_t p_kq[2] = {0, 0}, p_gate_empty[2] = {0, 0}, p_g = 0, p_wu = 0;   // prep
+    uint32_t s_u = 0, s_sz = 0, s_gate[2] = {0, 0};                // state
+    uint32_t gc = 0;   // global chunk counter (same sequence in every role)
+
+    const int G = gridDim.x;
+    const int U = p.B * p.Hv;
+    const int waves = (U + G - 1) / G;
+
+    for (int batch0 = 0; batch0 < waves;) {
+        build_unit_list(p, smem, batch0, count_slot);
+        __syncthreads();
+        const int nunits = *count_slot;
+        // waves covered by this batch: count units until MAX_UNITS
+        int wcover = 0;
+        {
+            int cnt = 0;
+            for (int w = batch0; w < waves; ++w) {
+                const int u = w * G + ((w & 1) ? (G - 1 - (int)blockIdx.x) : (int)blockIdx.x);
+                if (u < U) {
+                    if (cnt == MAX_UNITS) break;
+                    ++cnt;
+                }
+                ++wcover;
+            }
+        }
+
+        if (warp == 8) {
+            // ------------------------------------------------------------ TMA producer
+            if (lane == 0) {
+                for (int k = 0; k < nunits && !cx.aborted(); ++k) {
+                    const Unit un = load_unit(smem, k);
+                    const int qh = (int)(((int64_t)un.h * p.Hq) / p.Hv);
+                    const int nc = (un.len + C - 1) / C;
+                    for (int n = 0; n < nc; ++n) {
+                        const uint32_t s = (gc + n) & 1;
+                        if (kq_use[s] > 0 && !cx.wait(B_KQ_EMPTY + s, (kq_use[s] - 1) & 1)) break;
+                        ++kq_use[s];
+                        const uint32_t kq = sbase + (s ? OFF_KQ1 : OFF_KQ0);
+                        const uint32_t gb = sbase + (s ? OFF_GB1 : OFF_GB0);
+                        const int t0 = un.start + n * C;
+                        mbar_arrive_expect_tx(cx.bar(B_KQ_FULL + s), 32768 + 2048);
+                        tma_load_3d(kq, &p.tm_k, cx.bar(B_KQ_FULL + s), 0, qh, t0);
+                        tma_load_3d(kq + KQ_KB, &p.tm_k, cx.bar(B_KQ_FULL + s), 64, qh, t0);
+                        tma_load_3d(kq + 8192, &p.tm_q, cx.bar(B_KQ_FULL + s), 0, qh, t0);
+                        tma_load_3d(kq + KQ_KB + 8192, &p.tm_q, cx.bar(B_KQ_FULL + s), 64, qh, t0);
+                        tma_load_2d(gb, &p.tm_g, cx.bar(B_KQ_FULL + s), un.h & ~3, t0);
+                        tma_load_2d(gb + 1024, &p.tm_beta, cx.bar(B_KQ_FULL + s), un.h & ~3, t0);
+                        if (v_use > 0 && !cx.wait(B_V_EMPTY, (v_use - 1) & 1)) break;
+                        ++v_use;
+                        mbar_arrive_expect_tx(cx.bar(B_V_FULL), 16384);
+                        tma_load_3d(sbase + OFF_V, &p.tm_v, cx.bar(B_V_FULL), 0, un.h, t0);
+                        tma_load_3d(sbase + OFF_V + V_HALF, &p.tm_v, cx.bar(B_V_FULL), 64, un.h, t0);
+                    }
+                    gc += nc;
+                }
+            }
+        } else if (warp == 9) {
+            // ------------------------------------------------------------ UMMA issuer
+            if (lane == 0) {
+                constexpr uint32_t ID_G = idesc_bf16(128, 64, 0, 0);
+                constexpr uint32_t ID_W = idesc_bf16(128, 64, 1, 0);
+                constexpr uint32_t ID_U = idesc_bf16(128, 64, 1, 0);
+                constexpr uint32_t ID_1A = idesc_bf16(128, 64, 0, 1);
+                constexpr uint32_t ID_1B = idesc_bf16(128, 64, 0, 0);
+                constexpr uint32_t ID_2 = idesc_bf16(128, 128, 0, 1);
+                constexpr uint32_t ID_3 = idesc_bf16(128, 64, 0, 0);
+                bool ok = true;
+                auto issue_gram = [&](uint32_t s) {
+                    // (G): [K;Q] (128 x 128, K-major) x K^T
+                    const uint32_t kq = sbase + (s ? OFF_KQ1 : OFF_KQ0);
+                    for (int kk = 0; kk < 8; ++kk) {
+                        const uint32_t off = (kk >> 2) * KQ_KB + (kk & 3) * 32;
+                        umma_bf16(tmem + TM_GW, sdesc_sw128(kq + off, 16, 1024),
+                                  sdesc_sw128(kq + off, 16, 1024), ID_G, kk > 0);
+                    }
+                    umma_commit(cx.bar(B_G_DONE));
+                };
+                auto issue_wu = [&](uint32_t s) {
+                    const uint32_t kq = sbase + (s ? OFF_KQ1 : OFF_KQ0);
+                    // (W): W^T[dk][i] = sum_j K[j][dk] Tbg[i][j]; A = K (MN-major), B = Tbg (K-major)
+                    for (int kk = 0; kk < 4; ++kk)
+                        umma_bf16(tmem + TM_GW, sdesc_sw128(kq + kk * 2048, KQ_KB, 1024),
+                                  sdesc_sw128(sbase + OFF_TBG + kk * 32, 16, 1024), ID_W, kk > 0);
+                    // (U~): U^T[dv][i] = sum_j V[j][dv] Tb[i][j]; A = V (MN-major), B = Tb
+                    for (int kk = 0; kk < 4; ++kk)
+                        umma_bf16(tmem + TM_U + 64 * s, sdesc_sw128(sbase + OFF_V + kk * 2048, V_HALF, 1024),
+                                  sdesc_sw128(sbase + OFF_TB + kk * 32, 16, 1024), ID_U, kk > 0);
+                    umma_commit(cx.bar(B_WU_DONE));
+                    umma_commit(cx.bar(B_V_EMPTY));
+                };
+                for (int k = 0; k < nunits && ok; ++k) {
+                    const Unit un = load_unit(smem, k);
+                    const int nc = (un.len + C - 1) / C;
+                    if (nc == 0) continue;
+                    // prologue: prep MMAs of chunk 0
+                    {
+                        const uint32_t s = gc & 1;
+                        ok = ok && cx.wait(B_KQ_FULL + s, m_kq[s] & 1);
+                        ++m_kq[s];
+                        ok = ok && cx.wait(B_NORM, m_norm & 1);
+                        ++m_norm;
+                        if (!ok) break;
+                        tc_fence_after();
+                        issue_gram(s);
+                        ok = ok && cx.wait(B_T_READY, m_t & 1);
+                        ++m_t;
+                        ok = ok && cx.wait(B_V_FULL, m_v & 1);
+                        ++m_v;
+                        if (!ok) break;
+                        tc_fence_after();
+                        issue_wu(s);
+                    }
+                    for (int n = 0; n < nc && ok; ++n) {
+                        const uint32_t s = (gc + n) & 1;
+                        const uint32_t s1 = (gc + n + 1) & 1;
+                        const uint32_t kq = sbase + (s ? OFF_KQ1 : OFF_KQ0);
+                        const bool more = n + 1 < nc;
+                        if (more) {
+                            ok = ok && cx.wait(B_KQ_FULL + s1, m_kq[s1] & 1);
+                            ++m_kq[s1];
+                            ok = ok && cx.wait(B_NORM, m_norm & 1);
+                            ++m_norm;
+                            if (!ok) break;
+                            tc_fence_after();
+                            issue_gram(s1);
+                        }
+                        // chain 1: U^T += S^T (-W)^T ; Y = S^T Q^T
+                        ok = ok && cx.wait(B_S_READY, m_s & 1);
+                        ++m_s;
+                        ok = ok && cx.wait(B_WNEG, m_wneg & 1);
+                        ++m_wneg;
+                        if (!ok) break;
+                        tc_fence_after();
+                        for (int kk = 0; kk < 8; ++kk) {
+                            const uint32_t aoff = (kk >> 2) * SBF_KB + (kk & 3) * 32;
+                            umma_bf16(tmem + TM_U + 64 * s, sdesc_sw128(sbase + OFF_SBF + aoff, 16, 1024),
+                                      sdesc_sw128(sbase + OFF_WNEG + kk * 2048, 8192, 1024), ID_1A, 1);
+                        }
+                        for (int kk = 0; kk < 8; ++kk) {
+                            const uint32_t aoff = (kk >> 2) * SBF_KB + (kk & 3) * 32;
+                            const uint32_t boff = (kk >> 2) * KQ_KB + 8192 + (kk & 3) * 32;
+                            umma_bf16(tmem + TM_Y + 64 * s, sdesc_sw128(sbase + OFF_SBF + aoff, 16, 1024),
+                                      sdesc_sw128(kq + boff, 16, 1024), ID_1B, kk > 0);
+                        }
+                        umma_commit(cx.bar(B_U_DONE));
+                        // chain 2: S^T += Ud K ; Z = U^T P^T
+                        ok = ok && cx.wait(B_E1, m_e1 & 1);
+                        ++m_e1;
+                        if (!ok) break;
+                        tc_fence_after();
+                        for (int kk = 0; kk < 4; ++kk)
+                            umma_bf16(tmem + TM_S, sdesc_sw128(sbase + OFF_UBFD + kk * 32, 16, 1024),
+                                      sdesc_sw128(kq + kk * 2048, KQ_KB, 1024), ID_2, 1);
+                        const uint32_t pb = sbase + (s ? OFF_P1 : OFF_P0);
+                        for (int kk = 0; kk < 4; ++kk)
+                            umma_bf16(tmem + TM_Z, sdesc_sw128(sbase + OFF_UBF + kk * 32, 16, 1024),
+                                      sdesc_sw128(pb + kk * 32, 16, 1024), ID_3, kk > 0);
+                        umma_commit(cx.bar(B_SZ_DONE));
+                        umma_commit(cx.bar(B_KQ_EMPTY + s));
+                        // prep MMAs of the next chunk
+                        if (more) {
+                            ok = ok && cx.wait(B_T_READY, m_t & 1);
+                            ++m_t;
+                            ok = ok && cx.wait(B_V_FULL, m_v & 1);
+                            ++m_v;
+                            if (!ok) break;
+                            tc_fence_after();
+                            issue_wu(s1);
+                        }
+                    }
+                    gc += nc;
+                }
+            }
+        } else if (warp >= 4) {
+            // ------------------------------------------------------------ prep warpgroup
+            const int tp = tid - 128;           // 0..127 == TMEM lane
+            const int pw = tp >> 5;             // 0..3
+            const uint32_t tl = tmem + ((uint32_t)(32 * pw) << 16);
+            float *solve = reinterpret_cast<float *>(smem + OFF_SOLVE);
+            for (int k = 0; k < nunits; ++k) {
+                const Unit un = load_unit(smem, k);
+                const int nc = (un.len + C - 1) / C;
+                bool ok = true;
+                for (int n = 0; n < nc && ok; ++n) {
+                    const uint32_t s = (gc + n) & 1;
+                    const int len_n = min(C, un.len - n * C);
+                    uint8_t *kq = smem + (s ? OFF_KQ1 : OFF_KQ0);
+                    const float *gtile = reinterpret_cast<const float *>(smem + (s ? OFF_GB1 : OFF_GB0));
+                    float *ga = reinterpret_cast<float *>(smem + (s ? OFF_GATE1 : OFF_GATE0));
+                    ok = cx.wait(B_KQ_FULL + s, p_kq[s] & 1);
+                    ++p_kq[s];
+                    if (p_gate_empty[s] > 0) ok = ok && cx.wait(B_GATE_EMPTY + s, (p_gate_empty[s] - 1) & 1);
+                    ++p_gate_empty[s];
+                    // --- gates: inclusive scan of the floored, masked log-decay (threads 0..63)
+                    float Gi = 0.f;
+                    if (tp < 64) {
+                        const int i = tp;
+                        const int hc = un.h & 3;
+                        float gi = 0.f, bi = 0.f;
+                        if (i < len_n) {
+                            gi = fmaxf(gtile[i * 4 + hc], G_FLOOR);
+                            bi = gtile[256 + i * 4 + hc];
+                        }
+                        float x = gi;
+#pragma unroll
+                        for (int o = 1; o < 32; o <<= 1) {
+                            const float y = __shfl_up_sync(0xffffffffu, x, o);
+                            if (lane >= o) x += y;
+                        }
+                        Gi = x;
+                        ga[GA_BETA + i] = bi;
+                        ga[GA_G2 + i] = Gi;   // raw scan for now (warp-local)
+                    }
+                    // --- L2 norm of K and Q rows in place (thread tp owns row tp)
+                    if (p.qk_l2norm) {
+                        uint4 *r0 = reinterpret_cast<uint4 *>(kq + tp * 128);
+                        uint4 *r1 = reinterpret_cast<uint4 *>(kq + KQ_KB + tp * 128);
+                        float ss = 0.f;
+                        uint4 v0[8], v1[8];
+#pragma unroll
+                        for (int c = 0; c < 8; ++c) {
+                            v0[c] = r0[c];
+                            v1[c] = r1[c];
+                            float x[8];
+                            unpack8_bf16(v0[c], x);
+#pragma unroll
+                            for (int e = 0; e < 8; ++e) ss += x[e] * x[e];
+                            unpack8_bf16(v1[c], x);
+#pragma unroll
+                            for (int e = 0; e < 8; ++e) ss += x[e] * x[e];
+                        }
+                        const float rn = 1.0f / sqrtf(ss + 1e-12f);
+#pragma unroll
+                        for (int c = 0; c < 8; ++c) {
+                            float x[8];
+                            unpack8_bf16(v0[c], x);
+#pragma unroll
+                            for (int e = 0; e < 8; ++e) x[e] *= rn;
+                            r0[c] = pack8_bf16(x);
+                            unpack8_bf16(v1[c], x);
+#pragma unroll
+                            for (int e = 0; e < 8; ++e) x[e] *= rn;
+                            r1[c] = pack8_bf16(x);
+                        }
+                        fence_proxy_async_smem();
+                    }
+                    named_sync(1, 128);
+                    if (tp < 64) {
+                        // finish the 64-wide scan: add warp 0's total to warp 1
+                        if (tp >= 32) Gi += ga[GA_G2 + 31];
+                    }
+                    named_sync(1, 128);
+                    if (tp < 64) {
+                        const int i = tp;
+                        const float G2 = Gi * LOG2E;
+                        ga[GA_G2 + i] = G2;
+                        ga[GA_GAM + i] = exp2f(G2);
+                        ga[GA_BGAM + i] = ga[GA_BETA + i] * exp2f(G2);
+                        if ((i & 15) == 15) ga[GA_GEND + (i >> 4)] = G2;
+                        if (i == 63) ga[GA_GC] = exp2f(G2);
+                    }
+                    named_sync(1, 128);
+                    if (tp < 64) {
+                        const int i = tp;
+                        const float G2 = ga[GA_G2 + i];
+                        ga[GA_CF + i] = exp2f(ga[GA_GEND + (i >> 4)] - G2);
+                        ga[GA_DEC + i] = exp2f(ga[GA_G2 + 63] - G2);
+                    }
+                    named_sync(1, 128);
+                    if (tp == 0) {
+                        mbar_arrive(cx.bar(B_GATE_FULL + s));
+                        mbar_arrive(cx.bar(B_NORM));
+                    }
+                    // --- Gram -> A (rows 0..63) and P (rows 64..127)
+                    ok = ok && cx.wait(B_G_DONE, p_g & 1);
+                    ++p_g;
+                    tc_fence_after();
+                    float gr[64];
+                    {
+                        float t32[32];
+                        tmem_ld32(tl + TM_GW, t32);
+                        tmem_wait_ld();
+#pragma unroll
+                        for (int j = 0; j < 32; ++j) gr[j] = t32[j];
+                        tmem_ld32(tl + TM_GW + 32, t32);
+                        tmem_wait_ld();
+#pragma unroll
+                        for (int j = 0; j < 32; ++j) gr[32 + j] = t32[j];
+                    }
+                    {
+                        const int i = tp & 63;
+                        const int I = i >> 4;
+                        const float G2i = ga[GA_G2 + i];
+                        float rJ[4];
+#pragma unroll
+                        for (int J = 0; J < 4; ++J)
+                            rJ[J] = (J < I) ? exp2f(G2i - ga[GA_GEND + J]) : 0.f;
+                        if (tp < 64) {
+                            const float bi = ga[GA_BETA + i];
+                            // off-diagonal blocks J < I
+#pragma unroll
+                            for (int J = 0; J < 3; ++J) {
+                                if (J < I) {
+                                    float *blk = solve + a_slot(I, J) * SOLVE_BLK + (i & 15) * SOLVE_LD;
+#pragma unroll
+                                    for (int jj = 0; jj < 16; ++jj) {
+                                        const int j = 16 * J + jj;
+                                        blk[jj] = bi * gr[j] * rJ[J] * ga[GA_CF + j];
+                                    }
+                                }
+                            }
+                            // diagonal block: strictly lower
+                            {
+                                float *blk = solve + I * SOLVE_BLK + (i & 15) * SOLVE_LD;
+#pragma unroll
+                                for (int jj = 0; jj < 16; ++jj) {
+                                    const int j = 16 * I + jj;
+                                    float a = 0.f;
+#pragma unroll
+                                    for (int JJ = 0; JJ < 4; ++JJ)
+                                        if (JJ == I && jj < (i & 15))
+                                            a = bi * gr[16 * JJ + jj] * exp2f(G2i - ga[GA_G2 + j]);
+                                    blk[jj] = a;
+                                }
+                            }
+                        } else {
+                            // P row i (inclusive lower, unscaled by beta)
+                            uint8_t *prow = smem + (s ? OFF_P1 : OFF_P0);
+#pragma unroll
+                            for (int c = 0; c < 8; ++c) {
+                                float x[8];
+#pragma unroll
+                                for (int e = 0; e < 8; ++e) {
+                                    const int j = 8 * c + e;
+                                    const int J = j >> 4;
+                                    float f = 0.f;
+                                    if (j <= i) {
+                                        if (J < I) f = rJ[J] * ga[GA_CF + j];
+                                        else f = exp2f(G2i - ga[GA_G2 + j]);
+                                    }
+                                    x[e] = gr[j] * f;
+                                }
+                                *reinterpret_cast<uint4 *>(prow + sw128(i, c)) = pack8_bf16(x);
+                            }
+                            fence_proxy_async_smem();
+                        }
+                    }
+                    tc_fence_before();
+                    named_sync(1, 128);
+                    // --- diagonal 16x16 inverses D_I = (I + A_II)^-1 (threads 0..63, one column each)
+                    if (tp < 64) {
+                        const int I = tp >> 4, c = tp & 15;
+                        const float *Ab = solve + I * SOLVE_BLK;
+                        float x[16];
+#pragma unroll
+                        for (int r = 0; r < 16; ++r) {
+                            float acc = (r == c) ? 1.f : 0.f;
+#pragma unroll
+                            for (int m = 0; m < r; ++m) acc -= Ab[r * SOLVE_LD + m] * x[m];
+                            x[r] = acc;
+                        }
+                        float *Db = solve + (10 + I) * SOLVE_BLK;
+#pragma unroll
+                        for (int r = 0; r < 16; ++r) Db[r * SOLVE_LD + c] = x[r];
+                    }
+                    named_sync(1, 128);
+                    // --- level 1: T_10 = -D_1 A_10 D_0 (warp 0), T_32 = -D_3 A_32 D_2 (warp 1)
+                    if (pw < 2) {
+                        const int lo = pw ? 2 : 0;   // block pair (lo+1, lo)
+                        float acc[2][4] = {};
+                        blk_mma(acc, solve + (pw ? 5 : 4) * SOLVE_BLK, solve + (10 + lo) * SOLVE_BLK);
+                        float *tmp = solve + (pw ? 15 : 14) * SOLVE_BLK;
+                        blk_store(tmp, acc, 1.f);
+                        __syncwarp();
+                        float acc2[2][4] = {};
+                        blk_mma(acc2, solve + (10 + lo + 1) * SOLVE_BLK, tmp);
+                        __syncwarp();
+                        blk_store(tmp, acc2, -1.f);
+                    }
+                    named_sync(1, 128);
+                    // --- X = A_BA T_AA (warp w: block (p = w>>1, q = w&1))
+                    {
+                        const int pp = pw >> 1, q = pw & 1;
+                        float acc[2][4] = {};
+                        if (q == 0) {
+                            blk_mma(acc, solve + a_slot(2 + pp, 0) * SOLVE_BLK, solve + 10 * SOLVE_BLK);
+                            blk_mma(acc, solve + a_slot(2 + pp, 1) * SOLVE_BLK, solve + 14 * SOLVE_BLK);
+                        } else {
+                            blk_mma(acc, solve + a_slot(2 + pp, 1) * SOLVE_BLK, solve + 11 * SOLVE_BLK);
+                        }
+                        named_sync(1, 128);
+                        blk_store(solve + (6 + 2 * pp + q) * SOLVE_BLK, acc, 1.f);   // X_pq
+                        named_sync(1, 128);
+                        // --- T_BA = -T_BB X
+                        float acc2[2][4] = {};
+                        if (pp == 0) {
+                            blk_mma(acc2, solve + 12 * SOLVE_BLK, solve + (6 + q) * SOLVE_BLK);
+                        } else {
+                            blk_mma(acc2, solve + 15 * SOLVE_BLK, solve + (6 + q) * SOLVE_BLK);
+                            blk_mma(acc2, solve + 13 * SOLVE_BLK, solve + (8 + q) * SOLVE_BLK);
+                        }
+                        named_sync(1, 128);
+                        blk_store(solve + (6 + 2 * pp + q) * SOLVE_BLK, acc2, -1.f);  // T_{2+p, q}
+                        named_sync(1, 128);
+                    }
+                    // --- Tb = T diag(beta), Tbg = T diag(beta Gamma) (bf16, K-major, swizzled)
+                    {
+                        const int i = tp >> 1, jh = tp & 1;
+                        const int I = i >> 4;
+#pragma unroll
+                        for (int cc = 0; cc < 4; ++cc) {
+                            const int c = 4 * jh + cc;   // 16-byte chunk: j = 8c .. 8c+7
+                            const int J = c >> 1;
+                            float tv[8];
+                            if (J <= I) {
+                                const float *row = solve + t_slot(I, J) * SOLVE_BLK + (i & 15) * SOLVE_LD + 8 * (c & 1);
+                                const float4 a = *reinterpret_cast<const float4 *>(row);
+                                const float4 b = *reinterpret_cast<const float4 *>(row + 4);
+                                tv[0] = a.x; tv[1] = a.y; tv[2] = a.z; tv[3] = a.w;
+                                tv[4] = b.x; tv[5] = b.y; tv[6] = b.z; tv[7] = b.w;
+                                if (J == I) {
+#pragma unroll
+                                    for (int e = 0; e < 8; ++e) {
+                                        const int j = 8 * c + e;
+                                        if (j > i) tv[e] = 0.f;
+                                        if (j == i) tv[e] = 1.f;
+                                    }
+                                }
+                            } else {
+#pragma unroll
+                                for (int e = 0; e < 8; ++e) tv[e] = 0.f;
+                            }
+                            float xb[8], xg[8];
+#pragma unroll
+                            for (int e = 0; e < 8; ++e) {
+                                xb[e] = tv[e] * ga[GA_BETA + 8 * c + e];
+                                xg[e] = tv[e] * ga[GA_BGAM + 8 * c + e];
+                            }
+                            *reinterpret_cast<uint4 *>(smem + OFF_TB + sw128(i, c)) = pack8_bf16(xb);
+                            *reinterpret_cast<uint4 *>(smem + OFF_TBG + sw128(i, c)) = pack8_bf16(xg);
+                        }
+                        fence_proxy_async_smem();
+                    }
+                    named_sync(1, 128);
+                    if (tp == 0) mbar_arrive(cx.bar(B_T_READY));
+                    // --- W^T from TMEM -> (-W) as the MN-major B tile (row dk = tp)
+                    ok = ok && cx.wait(B_WU_DONE, p_wu & 1);
+                    ++p_wu;
+                    tc_fence_after();
+                    {
+                        float t32[32];
+                        tmem_ld32(tl + TM_GW, t32);
+                        tmem_wait_ld();
+#pragma unroll
+                        for (int c = 0; c < 4; ++c) {
+                            float x[8];
+#pragma unroll
+                            for (int e = 0; e < 8; ++e) x[e] = -t32[8 * c + e];
+                            *reinterpret_cast<uint4 *>(smem + OFF_WNEG + sw128(tp, c)) = pack8_bf16(x);
+                        }
+                        tmem_ld32(tl + TM_GW + 32, t32);
+                        tmem_wait_ld();
+#pragma unroll
+                        for (int c = 0; c < 4; ++c) {
+                            float x[8];
+#pragma unroll
+                            for (int e = 0; e < 8; ++e) x[e] = -t32[8 * c + e];
+                            *reinterpret_cast<uint4 *>(smem + OFF_WNEG + sw128(tp, 4 + c)) = pack8_bf16(x);
+                        }
+                        fence_proxy_async_smem();
+                    }
+                    tc_fence_before();
+                    named_sync(1, 128);
+                    if (tp == 0) mbar_arrive(cx.bar(B_WNEG));
+                    ok = !named_sync_or(1, 128, !ok || cx.aborted());
+                }
+                gc += nc;
+                if (!ok) break;
+            }
+        } else {
+            // ------------------------------------------------------------ state warpgroup
+            const int dv = tid;                 // 0..127 == TMEM lane
+            const uint32_t tl = tmem + ((uint32_t)(32 * warp) << 16);
+            for (int k = 0; k < nunits; ++k) {
+                const Unit un = load_unit(smem, k);
+                const int nc = (un.len + C - 1) / C;
+                const int64_t st_off = (((int64_t)un.b * p.Hv + un.h) * D + dv) * D;
+                const float *init = p.initial_state ? p.initial_state + st_off : nullptr;
+                float *fin = p.final_state + st_off;
+                if (nc == 0) {
+                    for (int c = 0; c < D; c += 4) {
+                        float4 v = init ? *reinterpret_cast<const float4 *>(init + c) : make_float4(0.f, 0.f, 0.f, 0.f);
+                        *reinterpret_cast<float4 *>(fin + c) = v;
+                    }
+                    continue;
+                }
+                bool ok = true;
+                // unit start: S0 -> bf16 tile and gC(0) * S0 -> TMEM
+                {
+                    const uint32_t s = gc & 1;
+                    ok = cx.wait(B_GATE_FULL + s, s_gate[s] & 1);
+                    ++s_gate[s];
+                    const float *ga = reinterpret_cast<const float *>(smem + (s ? OFF_GATE1 : OFF_GATE0));
+                    const float gC = ga[GA_GC];
+                    for (int half = 0; half < 2; ++half) {
+                        float x[64];
+#pragma unroll
+                        for (int c = 0; c < 64; c += 4) {
+                            float4 v = init ? *reinterpret_cast<const float4 *>(init + 64 * half + c) : make_float4(0.f, 0.f, 0.f, 0.f);
+                            x[c] = v.x; x[c + 1] = v.y; x[c + 2] = v.z; x[c + 3] = v.w;
+                        }
+#pragma unroll
+                        for (int c = 0; c < 8; ++c)
+                            *reinterpret_cast<uint4 *>(smem + OFF_SBF + half * SBF_KB + sw128(dv, c)) = pack8_bf16(x + 8 * c);
+                        float t32[32];
+#pragma unroll
+                        for (int q = 0; q < 2; ++q) {
+#pragma unroll
+                            for (int e = 0; e < 32; ++e) t32[e] = gC * x[32 * q + e];
+                            tmem_st32(tl + TM_S + 64 * half + 32 * q, t32);
+                        }
+                    }
+                    tmem_wait_st();
+                    fence_proxy_async_smem();
+                    tc_fence_before();
+                    ok = !named_sync_or(2, 128, !ok || cx.aborted());
+                    if (dv == 0 && ok) mbar_arrive(cx.bar(B_S_READY));
+                }
+                for (int n = 0; n < nc && ok; ++n) {
+                    const uint32_t s = (gc + n) & 1;
+                    const uint32_t s1 = (gc + n + 1) & 1;
+                    const int len_n = min(C, un.len - n * C);
+                    const float *ga = reinterpret_cast<const float *>(smem + (s ? OFF_GATE1 : OFF_GATE0));
+                    // ---- E1: U^T -> bf16 tiles (plain and decayed)
+                    ok = cx.wait(B_U_DONE, s_u & 1);
+                    ++s_u;
+                    tc_fence_after();
+#pragma unroll
+                    for (int q = 0; q < 2; ++q) {
+                        float u[32];
+                        tmem_ld32(tl + TM_U + 64 * s + 32 * q, u);
+                        tmem_wait_ld();
+#pragma unroll
+                        for (int c = 0; c < 4; ++c) {
+                            float xd[8];
+#pragma unroll
+                            for (int e = 0; e < 8; ++e) xd[e] = u[8 * c + e] * ga[GA_DEC + 32 * q + 8 * c + e];
+                            *reinterpret_cast<uint4 *>(smem + OFF_UBF + sw128(dv, 4 * q + c)) = pack8_bf16(u + 8 * c);
+                            *reinterpret_cast<uint4 *>(smem + OFF_UBFD + sw128(dv, 4 * q + c)) = pack8_bf16(xd);
+                        }
+                    }
+                    fence_proxy_async_smem();
+                    tc_fence_before();
+                    named_sync(2, 128);
+                    if (dv == 0) mbar_arrive(cx.bar(B_E1));
+                    // ---- E2: new state -> bf16 tile (+ decay of the next chunk) or final state
+                    ok = ok && cx.wait(B_SZ_DONE, s_sz & 1);
+                    ++s_sz;
+                    tc_fence_after();
+                    const bool more = n + 1 < nc;
+                    float gC1 = 1.f;
+                    if (more) {
+                        ok = ok && cx.wait(B_GATE_FULL + s1, s_gate[s1] & 1);
+                        ++s_gate[s1];
+                        gC1 = reinterpret_cast<const float *>(smem + (s1 ? OFF_GATE1 : OFF_GATE0))[GA_GC];
+                    }
+#pragma unroll
+                    for (int q = 0; q < 4; ++q) {
+                        float x[32];
+                        tmem_ld32(tl + TM_S + 32 * q, x);
+                        tmem_wait_ld();
+                        if (more) {
+#pragma unroll
+                            for (int c = 0; c < 4; ++c)
+                                *reinterpret_cast<uint4 *>(smem + OFF_SBF + (q >> 1) * SBF_KB + sw128(dv, 4 * (q & 1) + c)) = pack8_bf16(x + 8 * c);
+#pragma unroll
+                            for (int e = 0; e < 32; ++e) x[e] *= gC1;
+                            tmem_st32(tl + TM_S + 32 * q, x);
+                        } else {
+#pragma unroll
+                            for (int c = 0; c < 32; c += 4)
+                                *reinterpret_cast<float4 *>(fin + 32 * q + c) = make_float4(x[c], x[c + 1], x[c + 2], x[c + 3]);
+                        }
+                    }
+                    if (more) {
+                        tmem_wait_st();
+                        fence_proxy_async_smem();
+                        tc_fence_before();
+                        named_sync(2, 128);
+                        if (dv == 0) mbar_arrive(cx.bar(B_S_READY));
+                    }
+                    // ---- outputs O^T = scale (Y diag(Gamma) + Z)
+                    {
+                        __nv_bfloat16 *orow = p.out + ((int64_t)(un.start + n * C) * p.Hv + un.h) * D + dv;
+                        const int64_t ostride = (int64_t)p.Hv * D;
+#pragma unroll
+                        for (int q = 0; q < 2; ++q) {
+                            float y[32], z[32];
+                            tmem_ld32(tl + TM_Y + 64 * s + 32 * q, y);
+                            tmem_ld32(tl + TM_Z + 32 * q, z);
+                            tmem_wait_ld();
+#pragma unroll
+                            for (int e = 0; e < 32; ++e) {
+                                const int i = 32 * q + e;
+                                if (i < len_n) {
+                                    const float o = p.scale * (ga[GA_GAM + i] * y[e] + z[e]);
+                                    orow[i * ostride] = __float2bfloat16_rn(o);
+                                }
+                            }
+                        }
+                    }
+                    tc_fence_before();
+                    named_sync(2, 128);
+                    if (dv == 0) mbar_arrive(cx.bar(B_GATE_EMPTY + s));
+                    ok = !named_sync_or(2, 128, !ok || cx.aborted());
+                }
+                gc += nc;
+                if (!ok) break;
+            }
+        }
+        __syncthreads();
+        if (cx.aborted()) break;
+        batch0 += wcover;
+    }
+
+    // teardown: drain outstanding TMA stages on abort, then free TMEM
+    if (cx.aborted() && warp == 8 && lane == 0) {
+        // every armed stage either completed or will complete; wait (bounded) for each
+        for (int s = 0; s < 2; ++s) {
+            const long long t0 = clock64();
+            while (kq_use[s] > 0 && !mbar_try_wait(cx.bar(B_KQ_FULL + s), (kq_use[s] - 1) & 1))
+                if (clock64() - t0 > (1ll << 31)) break;
+        }
+        const long long t0 = clock64();
+        while (v_use > 0 && !mbar_try_wait(cx.bar(B_V_FULL), (v_use - 1) & 1))
+            if (clock64() - t0 > (1ll << 31)) break;
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    if (warp == 9) tmem_dealloc(tmem, 512);
+}
+
+}  // namespace gdn_chunk
+
+// ============================================================================ host side
+namespace {
+
+PFN_cuTensorMapEncodeTiled_v12000 get_encode()
+{
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    if (!fn) {
+        cudaDriverEntryPointQueryResult q;
+        void *ptr = nullptr;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) ==
+                cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
+    }
+    return fn;
+}
+
+bool make_map_3d_bf16(CUtensorMap *m, const void *base, uint64_t d0, uint64_t d1, uint64_t d2)
+{
+    auto enc = get_encode();
+    if (!enc) return false;
+    cuuint64_t dims[3] = {d0, d1, d2};
+    cuuint64_t strides[2] = {d0 * 2, d0 * d1 * 2};
+    cuuint32_t box[3] = {64, 1, 64};
+    cuuint32_t estr[3] = {1, 1, 1};
+    return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(base), dims, strides,
+               box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+bool make_map_2d_f32(CUtensorMap *m, const void *base, uint64_t d0, uint64_t d1)
+{
+    auto enc = get_encode();
+    if (!enc) return false;
+    cuuint64_t dims[2] = {d0, d1};
+    cuuint64_t strides[1] = {d0 * 4};
+    cuuint32_t box[2] = {4, 64};
+    cuuint32_t estr[2] = {1, 1};
+    return enc(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, const_cast<void *>(base), dims, strides, box,
+               estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+               CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+int num_sms()
+{
+    int dev = 0, n = 0;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+    return n > 0 ? n : 148;
+}
+
+}  // namespace
+
+bool prefill_chunked_supported(const GdnPrefillArgs &a)
+{
+    return a.dtype == GDN_BF16 && a.Dk == 128 && a.Dv == 128 && (a.Hv % 4) == 0 &&
+           get_encode() != nullptr;
+}
+
+cudaError_t launch_prefill_chunked(const GdnPrefillArgs &a, cudaStream_t stream)
+{
+    using namespace gdn_chunk;
+    if (a.B == 0) return cudaSuccess;
+    static bool attr_set = false;
+    if (!attr_set) {
+        cudaError_t e = cudaFuncSetAttribute(gdn_prefill_chunk_kernel,
+                                             cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             (int)SMEM_BYTES);
+        if (e != cudaSuccess) return e;
+        attr_set = true;
+    }
+    Params p;
+    memset(&p, 0, sizeof(p));
+    const uint64_t N = (uint64_t)(a.N > 0 ? a.N : 1);
+    // TMA maps need a valid base even when N == 0 (no chunk is loaded then)
+    if (a.N > 0) {
+        if (!make_map_3d_bf16(&p.tm_q, a.q, 128, a.Hq, N) ||
+            !make_map_3d_bf16(&p.tm_k, a.k, 128, a.Hq, N) ||
+            !make_map_3d_bf16(&p.tm_v, a.v, 128, a.Hv, N) ||
+            !make_map_2d_f32(&p.tm_g, a.g, a.Hv, N) || !make_map_2d_f32(&p.tm_beta, a.beta, a.Hv, N))
+            return cudaErrorInvalidValue;
+    }
+    p.cu_seqlens = a.cu_seqlens;
+    p.initial_state = a.initial_state;
+    p.final_state = a.final_state;
+    p.out = static_cast<__nv_bfloat16 *>(a.out);
+    p.dev_status = a.dev_status;
+    p.N = a.N;
+    p.B = a.B;
+    p.Hq = a.Hq;
+    p.Hv = a.Hv;
+    p.scale = a.scale;
+    p.qk_l2norm = a.qk_l2norm;
+    const int units = a.B * a.Hv;
+    const int grid = units < num_sms() ? units : num_sms();
+    gdn_prefill_chunk_kernel<<<grid, NTHREADS, SMEM_BYTES, stream>>>(p);
+    return cudaGetLastError();
 }

@@ -64,7 +64,9 @@ enum {
 
 /* bits OR-ed into *dev_status by the kernels */
 enum {
-    GDN_DEV_BAD_SLOT = 1   /* decode: a read/write/scatter slot >= pool_size was skipped */
+    GDN_DEV_BAD_SLOT = 1,  /* decode: a read/write/scatter slot >= pool_size was skipped */
+    GDN_DEV_TIMEOUT = 2,   /* a kernel-internal wait exceeded its bound; outputs invalid */
+    GDN_DEV_INTERNAL = 4   /* a kernel's layout self-check failed; nothing was computed */
 };
 
 /*
@@ -96,11 +98,15 @@ enum {
  *   qk_l2norm      non-zero: q and k vectors are scaled by
  *                  (sum x^2 + 1e-12)^(-1/2) before use.
  *   flags          GDN_PREFILL_SEQUENTIAL or 0.
- *   dev_status     optional device int32 (unused by prefill today).
+ *   dev_status     optional device int32; GDN_DEV_TIMEOUT is OR-ed in if an
+ *                  internal pipeline wait of the chunked kernel exceeds its
+ *                  bound (the call's outputs are then invalid).
  * Requirements: 1 <= Dk, Dv <= 256; Hv % Hq == 0; q, k, v, out,
  * initial_state and final_state 16-byte aligned; out must not overlap any
- * input.  bf16 with Dk = Dv = 128 runs the chunked tensor-core kernel (unless
- * GDN_PREFILL_SEQUENTIAL); everything else runs the per-token fp32 kernel.
+ * input.  bf16 with Dk = Dv = 128 and Hv % 4 == 0 runs the chunked
+ * tensor-core kernel (unless GDN_PREFILL_SEQUENTIAL); everything else runs the
+ * per-token fp32 kernel.  The chunked kernel floors each g at -30
+ * (exp(-30) ~ 9e-14) so that in-chunk decay differences stay finite.
  * Overlapping request ranges are not supported (their outputs are undefined).
  */
 GDN_API gdn_status gdn_prefill(const void *q, const void *k, const void *v,
@@ -161,8 +167,9 @@ GDN_API gdn_status gdn_decode(const void *q, const void *k, const void *v,
                       int32_t *dev_status, void *stream);
 
 /* 1 when gdn_prefill with these arguments runs the chunked tensor-core
- * kernel, 0 when it runs the per-token kernel (host-only query, no launch). */
-GDN_API int32_t gdn_prefill_uses_chunked(gdn_dtype dtype, int32_t Dk, int32_t Dv,
+ * kernel, 0 when it runs the per-token kernel (host-only query, no launch).
+ * The chunked kernel takes bf16 with Dk = Dv = 128 and Hv % 4 == 0. */
+GDN_API int32_t gdn_prefill_uses_chunked(gdn_dtype dtype, int32_t Hv, int32_t Dk, int32_t Dv,
                                          uint32_t flags);
 
 /* Name of a gdn_status code (static string). */

@@ -99,9 +99,9 @@ def test_ragged_bf16_d128(gdn, W, oracle_mod, sequential, l2norm):
 
 @pytest.mark.parametrize("sequential", [True, False])
 def test_cu_seqlens_clamp_and_uncovered_tokens(gdn, W, oracle_mod, sequential):
-    c = W.make_prefill(31, [40, 30, 40, 20, 10], 1, 2, 128, 128, init_std=0.1, qk_l2norm=True)
+    c = W.make_prefill(31, [40, 30, 40, 20, 10], 1, 4, 128, 128, init_std=0.1, qk_l2norm=True)
     N = c.N  # 140
-    sentinel = torch.full((N, 2, 128), 3.0, dtype=torch.bfloat16)
+    sentinel = torch.full((N, 4, 128), 3.0, dtype=torch.bfloat16)
     # (a) tokens 0..9 and N-20..N-1 belong to no request and keep the caller's values;
     #     request 1 is empty, request 4 is decreasing (empty)
     c.cu_seqlens = torch.tensor([10, 40, 40, 60, N - 20, 3], dtype=torch.int32)
@@ -128,7 +128,7 @@ def test_cu_seqlens_clamp_and_uncovered_tokens(gdn, W, oracle_mod, sequential):
 @pytest.mark.parametrize("sequential", [True, False])
 def test_zero_gate_and_zero_initial_state(gdn, W, oracle_mod, sequential):
     """gamma = 0 (g = -inf) wipes the state; no initial state means zero."""
-    c = W.make_prefill(41, [70, 130], 1, 1, 128, 128, init_std=None, qk_l2norm=True)
+    c = W.make_prefill(41, [70, 130], 1, 4, 128, 128, init_std=None, qk_l2norm=True)
     c.g[5] = float("-inf")
     c.g[100] = float("-inf")
     c.g[101:110] = 0.0
@@ -164,18 +164,43 @@ def test_deterministic(gdn, W, sequential):
 
 
 def test_rank4_spelling(gdn, W, oracle_mod):
-    c = W.make_prefill(71, [50, 50], 1, 2, 128, 128, uniform=True, init_std=0.1,
+    c = W.make_prefill(71, [50, 50], 1, 4, 128, 128, uniform=True, init_std=0.1,
                        qk_l2norm=True)
     q4 = dev(c.q).reshape(2, 50, 1, 128)
     k4 = dev(c.k).reshape(2, 50, 1, 128)
-    v4 = dev(c.v).reshape(2, 50, 2, 128)
-    out, fs = gdn.gdn_prefill(q4, k4, v4, dev(c.g).reshape(2, 50, 2),
-                              dev(c.beta).reshape(2, 50, 2), None, dev(c.initial_state),
+    v4 = dev(c.v).reshape(2, 50, 4, 128)
+    out, fs = gdn.gdn_prefill(q4, k4, v4, dev(c.g).reshape(2, 50, 4),
+                              dev(c.beta).reshape(2, 50, 4), None, dev(c.initial_state),
                               scale=c.scale, qk_l2norm=True)
     torch.cuda.synchronize()
     ro, rf = oracle_prefill_case(oracle_mod, c)
     assert rel_l2(f64(out), ro) <= TOL_BF16
     assert rel_l2(f64(fs), rf) <= TOL_BF16
+
+
+def test_chunked_path_is_selected(gdn):
+    assert gdn.prefill_uses_chunked(torch.bfloat16, 4, 128, 128)
+    assert gdn.prefill_uses_chunked(torch.bfloat16, 32, 128, 128)
+    assert not gdn.prefill_uses_chunked(torch.bfloat16, 32, 128, 128, sequential=True)
+    assert not gdn.prefill_uses_chunked(torch.float32, 32, 128, 128)
+    assert not gdn.prefill_uses_chunked(torch.bfloat16, 2, 128, 128)
+    assert not gdn.prefill_uses_chunked(torch.bfloat16, 32, 64, 128)
+
+
+@pytest.mark.parametrize("lengths", [[1], [64], [65], [4096, 3, 700], [129, 0, 1, 191, 64]])
+def test_chunked_equals_sequential(gdn, W, lengths):
+    """The chunk form equals the token recurrence (same inputs, both GPU paths), and no
+    pipeline wait of the chunked kernel ran out."""
+    c = W.make_prefill(81 + len(lengths), lengths, 2, 8, 128, 128, init_std=0.05, qk_l2norm=True)
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    oc, fc = gdn.gdn_prefill(dev(c.q), dev(c.k), dev(c.v), dev(c.g), dev(c.beta),
+                             dev(c.cu_seqlens), dev(c.initial_state), scale=c.scale,
+                             qk_l2norm=True, dev_status=status)
+    os_, fs_ = run_gpu_prefill(c, sequential=True)
+    torch.cuda.synchronize()
+    assert int(status.item()) == 0
+    assert rel_l2(f64(oc), f64(os_)) <= TOL_BF16
+    assert rel_l2(f64(fc), f64(fs_)) <= TOL_BF16
 
 
 # ---------------------------------------------------------------- full sizes
