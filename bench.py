@@ -319,6 +319,21 @@ def cpu_oracle_sample(case, target_s=10.0):
                       f"all {Hv} value heads ({Hq} query/key heads), float64, {dt:.1f} s"}
 
 
+def profile_phase(gdn, workloads, args):
+    """Run one phase for `--steps` steps after `--warmup` (under a profiler); prints timings."""
+    if args.phase == "prefill":
+        case = make_case(args.workload)
+        total_ms, launch_ms = time_prefill(gdn, case, args.steps, args.warmup, 1)
+        print(json.dumps({"phase": "prefill", "workload": case.name,
+                          "ms_per_launch": statistics.mean(launch_ms)}), flush=True)
+    else:
+        dcase = workloads.decode_pool_case()
+        dms = time_decode(gdn, dcase, args.steps, args.warmup, 1)
+        print(json.dumps({"phase": "decode", "workload": dcase.name,
+                          "ms_per_launch": statistics.mean(dms)}), flush=True)
+    return 0
+
+
 # ---------------------------------------------------------------------- main
 def make_case(name):
     from gated_deltanet_state_gdn_b200 import workloads
@@ -346,6 +361,9 @@ def main():
     ap.add_argument("--workload", default="ragged", choices=["ragged", "long"])
     ap.add_argument("--no-decode", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu", action="store_true", help="skip the CPU oracle baseline")
+    ap.add_argument("--phase", default="all", choices=["all", "prefill", "decode"],
+                    help="prefill or decode alone (for profiling); 'all' for the JSON line")
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     args = ap.parse_args()
     if args.warmup < 3:
@@ -381,6 +399,9 @@ def main():
     from gated_deltanet_state_gdn_b200 import workloads
     gdn.lib()
     peaks = load_peaks()
+
+    if args.phase != "all":
+        return profile_phase(gdn, workloads, args)
 
     case = make_case(args.workload)
     Hq, Hv, Dk, Dv = case.dims
@@ -437,7 +458,7 @@ def main():
         launches += e_steps
 
     cpu = None
-    if rank == 0 and world == 1:
+    if rank == 0 and world == 1 and not args.no_cpu:
         cpu = cpu_oracle_sample(case, target_s=args.cpu_seconds)
 
     if rank == 0:

@@ -7,29 +7,33 @@
 // chunk form (derived from the recurrence; the op page names a chunk-parallel
 // prefill with chunk_size 64 and states that the chunk size does not change
 // the result) is, for a chunk with incoming state S0 (Dk x Dv), cumulative
-// log-decay G_i = sum_{l<=i} g_l, Gamma_i = exp(G_i):
-//   A_ij = beta_i (k_i . k_j) exp(G_i - G_j)   (j < i),   T = (I + A)^-1
-//   W    = T diag(beta Gamma) K,   U~ = T diag(beta) V
+// log-decay G_i = sum_{l<=i} g_l, Gamma_i = exp(G_i), and (optionally) the
+// L2-normalised rows k^_i = rk_i k_i, q^_i = rq_i q_i:
+//   A_ij = beta_i (k^_i . k^_j) exp(G_i - G_j)   (j < i),   T = (I + A)^-1
+//   W    = T diag(beta Gamma) K^,   U~ = T diag(beta) V
 //   U    = U~ - W S0
-//   O    = scale (diag(Gamma) Q S0 + P U),  P_ij = (q_i . k_j) exp(G_i - G_j) (j <= i)
-//   S_C  = Gamma_C S0 + (diag(exp(G_C - G)) K)^T U
+//   O    = scale (diag(Gamma) Q^ S0 + P U),  P_ij = (q^_i . k^_j) exp(G_i - G_j) (j <= i)
+//   S_C  = Gamma_C S0 + (diag(exp(G_C - G)) K^)^T U
+// The norms rk, rq are never applied to the bf16 tiles: they fold into A, P,
+// the columns of T (for W), the decayed copy of U (for S_C) and the output
+// scale, so the tensor cores always read the caller's q/k bytes.
 // All state-dependent products are evaluated transposed (rows = value index
 // dv), so every tcgen05 MMA here has M = 128:
 //   (G)  [K; Q] K^T                         -> TMEM  (Gram, 128 x 64)
-//   (W)  W^T  = K^T . Tbg^T                 -> TMEM  (Tbg = T diag(beta Gamma))
+//   (W)  W^T  = K^T . Tbg^T                 -> TMEM  (Tbg = T diag(beta Gamma rk))
 //   (U~) U^T  = V^T . Tb^T                  -> TMEM  (Tb  = T diag(beta))
 //   (1a) U^T += S^T . (-W)^T                 (bf16 copy of S^T from SMEM)
 //   (1b) Y    = S^T . Q^T
-//   (2)  S^T += (U^T diag(exp(G_C - G))) . K (fp32 accumulator stays in TMEM)
+//   (2)  S^T += (U^T diag(exp(G_C - G) rk)) . K   (fp32 accumulator stays in TMEM)
 //   (3)  Z    = U^T . P^T
-//   O^T = scale (Y diag(Gamma) + Z)
+//   O^T = scale (Y diag(Gamma rq) + Z)
 // TMEM (512 columns): S^T [0,128) | U^T x2 [128,256) | Y x2 [256,384) |
 // Z [384,448) | Gram/W^T [448,512).
 //
 // CTA = 10 warps, one (request, value head) unit at a time, persistent over a
 // longest-first unit list:
 //   warps 0-3  state warpgroup: TMEM <-> bf16 operand tiles, outputs, state I/O
-//   warps 4-7  prep warpgroup: L2 norm, gates, Gram -> A and P, the 64x64
+//   warps 4-7  prep warpgroup: row norms, gates, Gram -> A and P, the 64x64
 //              unit-triangular solve, T/W tiles (runs one chunk ahead)
 //   warp  8    TMA producer (q/k/v/g/beta tiles, two stages)
 //   warp  9    TMEM owner and single-thread UMMA issuer
@@ -66,16 +70,17 @@ constexpr uint32_t OFF_P0 = 131072;      // [64 rows i][64 j], 8 KB
 constexpr uint32_t OFF_P1 = 139264;
 constexpr uint32_t OFF_TB = 147456;      // [64 rows i][64 j], 8 KB
 constexpr uint32_t OFF_TBG = 155648;
-constexpr uint32_t OFF_UBF = 163840;     // [128 rows dv][64 i], 16 KB
+constexpr uint32_t OFF_UBF = 163840;     // [128 rows dv][64 i], 16 KB; also the output staging tile
 constexpr uint32_t OFF_UBFD = 180224;
 constexpr uint32_t OFF_SOLVE = 196608;   // 16 blocks of 16 x 20 fp32
 constexpr uint32_t SOLVE_LD = 20;        // padded row stride (floats)
 constexpr uint32_t SOLVE_BLK = 16 * SOLVE_LD;  // floats per block
 constexpr uint32_t OFF_GB0 = OFF_SOLVE + 16 * SOLVE_BLK * 4;   // g tile 1 KB + beta tile 1 KB
 constexpr uint32_t OFF_GB1 = OFF_GB0 + 2048;
-constexpr uint32_t OFF_GATE0 = OFF_GB1 + 2048;                 // processed gates, 2 KB
-constexpr uint32_t OFF_GATE1 = OFF_GATE0 + 2048;
-constexpr uint32_t OFF_UNITS = OFF_GATE1 + 2048;               // int4 x MAX_UNITS
+constexpr uint32_t GATE_BYTES = 2560;
+constexpr uint32_t OFF_GATE0 = OFF_GB1 + 2048;                 // processed gates
+constexpr uint32_t OFF_GATE1 = OFF_GATE0 + GATE_BYTES;
+constexpr uint32_t OFF_UNITS = OFF_GATE1 + GATE_BYTES;         // int4 x MAX_UNITS
 constexpr uint32_t OFF_BARS = OFF_UNITS + MAX_UNITS * 16;
 constexpr uint32_t NUM_BARS = 19;
 constexpr uint32_t OFF_MISC = OFF_BARS + 256;                  // tmem base, abort flag, count
@@ -86,19 +91,21 @@ static_assert(OFF_GB0 % 1024 == 0, "alignment");
 
 // gate-array offsets (floats) inside a GATE stage
 constexpr int GA_G2 = 0;       // G_i * log2(e)
-constexpr int GA_CF = 64;      // exp(Gend_J(i) - G_i): column factor to the end of i's 16-block
+constexpr int GA_CF = 64;      // exp(Gend_J(i) - G_i): factor to the end of i's 16-block
 constexpr int GA_BETA = 128;   // beta_i (0 beyond the request)
-constexpr int GA_BGAM = 192;   // beta_i exp(G_i)
-constexpr int GA_GAM = 256;    // exp(G_i)
-constexpr int GA_DEC = 320;    // exp(G_C - G_i)
-constexpr int GA_GEND = 384;   // G_end of each 16-block * log2(e)  [4]
-constexpr int GA_GC = 388;     // exp(G_C)
+constexpr int GA_GAM = 192;    // exp(G_i)
+constexpr int GA_DEC = 256;    // exp(G_C - G_i)
+constexpr int GA_RK = 320;     // key norm factor rk_i (1 without qk_l2norm)
+constexpr int GA_RQ = 384;     // query norm factor rq_i
+constexpr int GA_GEND = 448;   // G_end of each 16-block * log2(e)  [4]
+constexpr int GA_GC = 452;     // exp(G_C)
+static_assert((GA_GC + 1) * 4 <= (int)GATE_BYTES, "gate stage size");
 
 // barrier indices
 enum {
     B_KQ_FULL = 0, B_KQ_EMPTY = 2, B_V_FULL = 4, B_V_EMPTY = 5, B_GATE_FULL = 6,
-    B_GATE_EMPTY = 8, B_NORM = 10, B_G_DONE = 11, B_T_READY = 12, B_WU_DONE = 13,
-    B_WNEG = 14, B_S_READY = 15, B_U_DONE = 16, B_E1 = 17, B_SZ_DONE = 18
+    B_GATE_EMPTY = 8, B_G_DONE = 10, B_T_READY = 11, B_WU_DONE = 12, B_WNEG = 13,
+    B_S_READY = 14, B_U_DONE = 15, B_E1 = 16, B_S_DONE = 17, B_Z_DONE = 18
 };
 
 // TMEM columns
@@ -179,16 +186,24 @@ __device__ __forceinline__ uint4 pack8_bf16(const float *x)
     return r;
 }
 
-__device__ __forceinline__ void unpack8_bf16(uint4 r, float *x)
+__device__ __forceinline__ float sumsq8_bf16(uint4 r)
 {
     const uint32_t w[4] = {r.x, r.y, r.z, r.w};
+    float s = 0.f;
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
-        __nv_bfloat162 h = *reinterpret_cast<const __nv_bfloat162 *>(&w[i]);
-        float2 f = __bfloat1622float2(h);
-        x[2 * i] = f.x;
-        x[2 * i + 1] = f.y;
+        const float lo = __uint_as_float(w[i] << 16);
+        const float hi = __uint_as_float(w[i] & 0xffff0000u);
+        s = fmaf(lo, lo, s);
+        s = fmaf(hi, hi, s);
     }
+    return s;
+}
+
+__device__ __forceinline__ float4 ld4(const float *p) { return *reinterpret_cast<const float4 *>(p); }
+__device__ __forceinline__ void st4(float *p, float a, float b, float c, float d)
+{
+    *reinterpret_cast<float4 *>(p) = make_float4(a, b, c, d);
 }
 
 // --------------------------------------------------------------------------
@@ -231,30 +246,28 @@ __device__ void build_unit_list(const Params &p, uint8_t *smem, int batch0, int 
     const int U = B * p.Hv;
     const int c = blockIdx.x;
     int4 *list = reinterpret_cast<int4 *>(smem + OFF_UNITS);
-    // number of units of this CTA from wave batch0 on
     int total = 0;
-    {
-        const int waves = (U + G - 1) / G;
-        for (int w = batch0; w < waves && total < MAX_UNITS; ++w) {
-            const int u = w * G + ((w & 1) ? (G - 1 - c) : c);
-            if (u < U) {
-                if (tid == 0) {
-                    const int r = u / p.Hv;
-                    const int h = u - r * p.Hv;
-                    const int b = sorted ? ord[r] : r;
-                    int s, l;
-                    req_range(b, s, l);
-                    list[total] = make_int4(b, h, s, l);
-                }
-                ++total;
+    const int waves = (U + G - 1) / G;
+    for (int w = batch0; w < waves && total < MAX_UNITS; ++w) {
+        const int u = w * G + ((w & 1) ? (G - 1 - c) : c);
+        if (u < U) {
+            if (tid == 0) {
+                const int r = u / p.Hv;
+                const int h = u - r * p.Hv;
+                const int b = sorted ? ord[r] : r;
+                int s, l;
+                req_range(b, s, l);
+                list[total] = make_int4(b, h, s, l);
             }
+            ++total;
         }
     }
     *count_out = total;
 }
 
 // --------------------------------------------------------------------------
-// warp-level 16x16x16 tf32 products on padded fp32 blocks (row stride SOLVE_LD)
+// warp-level 16x16x16 tf32 products on padded fp32 blocks (row stride SOLVE_LD); the
+// fp32 bits are passed as they are and the tensor core reads them as tf32
 // acc[nh][.] += X(16x16) * Y(16x16), fragments of mma.m16n8k8
 __device__ __forceinline__ void blk_mma(float (&acc)[2][4], const float *X, const float *Y)
 {
@@ -263,15 +276,15 @@ __device__ __forceinline__ void blk_mma(float (&acc)[2][4], const float *X, cons
 #pragma unroll
     for (int kh = 0; kh < 2; ++kh) {
         uint32_t a[4];
-        a[0] = to_tf32(X[g * SOLVE_LD + 8 * kh + t]);
-        a[1] = to_tf32(X[(g + 8) * SOLVE_LD + 8 * kh + t]);
-        a[2] = to_tf32(X[g * SOLVE_LD + 8 * kh + t + 4]);
-        a[3] = to_tf32(X[(g + 8) * SOLVE_LD + 8 * kh + t + 4]);
+        a[0] = __float_as_uint(X[g * SOLVE_LD + 8 * kh + t]);
+        a[1] = __float_as_uint(X[(g + 8) * SOLVE_LD + 8 * kh + t]);
+        a[2] = __float_as_uint(X[g * SOLVE_LD + 8 * kh + t + 4]);
+        a[3] = __float_as_uint(X[(g + 8) * SOLVE_LD + 8 * kh + t + 4]);
 #pragma unroll
         for (int nh = 0; nh < 2; ++nh) {
             uint32_t b[2];
-            b[0] = to_tf32(Y[(8 * kh + t) * SOLVE_LD + 8 * nh + g]);
-            b[1] = to_tf32(Y[(8 * kh + t + 4) * SOLVE_LD + 8 * nh + g]);
+            b[0] = __float_as_uint(Y[(8 * kh + t) * SOLVE_LD + 8 * nh + g]);
+            b[1] = __float_as_uint(Y[(8 * kh + t + 4) * SOLVE_LD + 8 * nh + g]);
             mma_tf32_16x8x8(acc[nh], a, b);
         }
     }
@@ -283,21 +296,18 @@ __device__ __forceinline__ void blk_store(float *Z, const float (&acc)[2][4], fl
     const int g = lane >> 2, t = lane & 3;
 #pragma unroll
     for (int nh = 0; nh < 2; ++nh) {
-        Z[g * SOLVE_LD + 8 * nh + 2 * t] = sgn * acc[nh][0];
-        Z[g * SOLVE_LD + 8 * nh + 2 * t + 1] = sgn * acc[nh][1];
-        Z[(g + 8) * SOLVE_LD + 8 * nh + 2 * t] = sgn * acc[nh][2];
-        Z[(g + 8) * SOLVE_LD + 8 * nh + 2 * t + 1] = sgn * acc[nh][3];
+        *reinterpret_cast<float2 *>(Z + g * SOLVE_LD + 8 * nh + 2 * t) =
+            make_float2(sgn * acc[nh][0], sgn * acc[nh][1]);
+        *reinterpret_cast<float2 *>(Z + (g + 8) * SOLVE_LD + 8 * nh + 2 * t) =
+            make_float2(sgn * acc[nh][2], sgn * acc[nh][3]);
     }
 }
 
 // SOLVE slots: 0-3 A_II (strictly lower), 4 A_10, 5 A_32, 6-9 A_20 A_21 A_30 A_31
 // (later X, later T_20 T_21 T_30 T_31), 10-13 D_I = (I + A_II)^-1, 14 T_10, 15 T_32.
-__device__ __forceinline__ int a_slot(int I, int J)
+__host__ __device__ constexpr int a_slot(int I, int J)
 {
-    // J < I
-    if (I == 1) return 4;                      // (1,0)
-    if (I == 2) return 6 + J;                  // (2,0) (2,1)
-    return J == 2 ? 5 : 8 + J;                 // (3,2) -> 5, (3,0) (3,1) -> 8, 9
+    return I == 1 ? 4 : (I == 2 ? 6 + J : (J == 2 ? 5 : 8 + J));
 }
 
 __device__ __forceinline__ int t_slot(int I, int J)
@@ -308,6 +318,67 @@ __device__ __forceinline__ int t_slot(int I, int J)
     if (I == 3 && J == 2) return 15;
     if (I == 2) return 6 + J;
     return 8 + J;
+}
+
+// Row i of A (prep warps 0-1: beta_i (k^_i . k^_j) exp(G_i - G_j) for j < i, fp32
+// into the solve blocks) or of P (prep warps 2-3: (q^_i . k^_j) exp(G_i - G_j) for
+// j <= i, bf16 tile), read 16 Gram columns at a time from TMEM.  The exponent of an
+// earlier block J is split as exp(G_i - Gend_J) exp(Gend_J - G_j), both <= 1.
+__device__ __forceinline__ void build_row(uint32_t tl_gram, int pw, const float *ga, float *solve,
+                                          uint8_t *ptile)
+{
+    const int lane = threadIdx.x & 31;
+    const bool isP = pw >= 2;
+    const int r = lane & 15;
+    const int I = 2 * (pw & 1) + (lane >> 4);
+    const int i = 16 * I + r;
+    const float G2i = ga[GA_G2 + i];
+    const float rowscale = isP ? ga[GA_RQ + i] : ga[GA_BETA + i] * ga[GA_RK + i];
+    float gend[3];
+#pragma unroll
+    for (int J = 0; J < 3; ++J) gend[J] = ga[GA_GEND + J];
+#pragma unroll 1
+    for (int J = 0; J < 4; ++J) {
+        // ---- loads (TMEM Gram columns, gate factors) before any store of this block
+        float x[16], cf[16], g2[16], rk[16];
+        tmem_ld16(tl_gram + 16 * J, x);
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+            const float4 a = ld4(ga + GA_CF + 16 * J + 4 * q);
+            const float4 b = ld4(ga + GA_G2 + 16 * J + 4 * q);
+            const float4 c = ld4(ga + GA_RK + 16 * J + 4 * q);
+            cf[4 * q] = a.x; cf[4 * q + 1] = a.y; cf[4 * q + 2] = a.z; cf[4 * q + 3] = a.w;
+            g2[4 * q] = b.x; g2[4 * q + 1] = b.y; g2[4 * q + 2] = b.z; g2[4 * q + 3] = b.w;
+            rk[4 * q] = c.x; rk[4 * q + 1] = c.y; rk[4 * q + 2] = c.z; rk[4 * q + 3] = c.w;
+        }
+        tmem_wait_ld();
+        // ---- compute
+        if (J < I) {
+            const float f = ex2_approx(G2i - (J == 0 ? gend[0] : (J == 1 ? gend[1] : gend[2]))) * rowscale;
+#pragma unroll
+            for (int jj = 0; jj < 16; ++jj) x[jj] *= f * cf[jj] * rk[jj];
+        } else if (J == I) {
+            // branch-free: every lane evaluates all 16 factors, then masks
+            const int lim = isP ? r + 1 : r;
+#pragma unroll
+            for (int jj = 0; jj < 16; ++jj) {
+                const float e = ex2_approx(fminf(G2i - g2[jj], 0.f)) * rk[jj] * rowscale;
+                x[jj] = (jj < lim) ? x[jj] * e : 0.f;
+            }
+        } else {
+#pragma unroll
+            for (int jj = 0; jj < 16; ++jj) x[jj] = 0.f;
+        }
+        // ---- stores
+        if (isP) {
+            *reinterpret_cast<uint4 *>(ptile + sw128(i, 2 * J)) = pack8_bf16(x);
+            *reinterpret_cast<uint4 *>(ptile + sw128(i, 2 * J + 1)) = pack8_bf16(x + 8);
+        } else if (J <= I) {
+            float *row = solve + (J == I ? I : a_slot(I, J)) * SOLVE_BLK + r * SOLVE_LD;
+#pragma unroll
+            for (int q = 0; q < 4; ++q) st4(row + 4 * q, x[4 * q], x[4 * q + 1], x[4 * q + 2], x[4 * q + 3]);
+        }
+    }
 }
 
 // ========================================================================== kernel
@@ -336,8 +407,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) gdn_prefill_chunk_kernel(const __
 
     if (tid == 0) {
         *abort_flag = 0;
-        const uint32_t counts[NUM_BARS] = {1, 1, 1, 1, 1, 1, 1, 1, 1, 1, 1, 1, 1, 1, 1, 1, 1, 1, 1};
-        for (int i = 0; i < (int)NUM_BARS; ++i) mbar_init(cx.bar(i), counts[i]);
+        for (int i = 0; i < (int)NUM_BARS; ++i) mbar_init(cx.bar(i), 1);
         fence_mbar_init();
     }
     if (warp == 8 && lane == 0) {
@@ -357,11 +427,11 @@ __global__ void __launch_bounds__(NTHREADS, 1) gdn_prefill_chunk_kernel(const __
     const uint32_t tmem = *tmem_slot;
 
     // per-role pipeline counters (persist across units and batches)
-    uint32_t kq_use[2] = {0, 0}, v_use = 0;                       // TMA
-    uint32_t m_norm = 0, m_t = 0, m_wneg = 0, m_s = 0, m_e1 = 0;  // MMA
-    uint32_t m_kq[2] = {0, 0}, m_v = 0;
+    uint32_t kq_use[2] = {0, 0}, v_use = 0;                          // TMA
+    uint32_t m_t = 0, m_wneg = 0, m_s = 0, m_e1 = 0, m_v = 0;        // MMA
+    uint32_t m_kq[2] = {0, 0};
     uint32_t p_kq[2] = {0, 0}, p_gate_empty[2] = {0, 0}, p_g = 0, p_wu = 0;   // prep
-    uint32_t s_u = 0, s_sz = 0, s_gate[2] = {0, 0};                // state
+    uint32_t s_u = 0, s_sd = 0, s_zd = 0, s_gate[2] = {0, 0};         // state
     uint32_t gc = 0;   // global chunk counter (same sequence in every role)
 
     const int G = gridDim.x;
@@ -372,7 +442,6 @@ __global__ void __launch_bounds__(NTHREADS, 1) gdn_prefill_chunk_kernel(const __
         build_unit_list(p, smem, batch0, count_slot);
         __syncthreads();
         const int nunits = *count_slot;
-        // waves covered by this batch: count units until MAX_UNITS
         int wcover = 0;
         {
             int cnt = 0;
@@ -426,27 +495,39 @@ __global__ void __launch_bounds__(NTHREADS, 1) gdn_prefill_chunk_kernel(const __
                 constexpr uint32_t ID_1B = idesc_bf16(128, 64, 0, 0);
                 constexpr uint32_t ID_2 = idesc_bf16(128, 128, 0, 1);
                 constexpr uint32_t ID_3 = idesc_bf16(128, 64, 0, 0);
+                // descriptor bases; a byte offset `o` inside a tile is added as (o >> 4)
+                const uint64_t dKQk0 = sdesc_sw128(sbase + OFF_KQ0, 16, 1024);      // K-major
+                const uint64_t dKQk1 = sdesc_sw128(sbase + OFF_KQ1, 16, 1024);
+                const uint64_t dKQm0 = sdesc_sw128(sbase + OFF_KQ0, KQ_KB, 1024);   // MN-major K
+                const uint64_t dKQm1 = sdesc_sw128(sbase + OFF_KQ1, KQ_KB, 1024);
+                const uint64_t dV = sdesc_sw128(sbase + OFF_V, V_HALF, 1024);
+                const uint64_t dTB = sdesc_sw128(sbase + OFF_TB, 16, 1024);
+                const uint64_t dTBG = sdesc_sw128(sbase + OFF_TBG, 16, 1024);
+                const uint64_t dSBF = sdesc_sw128(sbase + OFF_SBF, 16, 1024);
+                const uint64_t dWNEG = sdesc_sw128(sbase + OFF_WNEG, 8192, 1024);
+                const uint64_t dUBF = sdesc_sw128(sbase + OFF_UBF, 16, 1024);
+                const uint64_t dUBFD = sdesc_sw128(sbase + OFF_UBFD, 16, 1024);
+                const uint64_t dP0 = sdesc_sw128(sbase + OFF_P0, 16, 1024);
+                const uint64_t dP1 = sdesc_sw128(sbase + OFF_P1, 16, 1024);
                 bool ok = true;
                 auto issue_gram = [&](uint32_t s) {
                     // (G): [K;Q] (128 x 128, K-major) x K^T
-                    const uint32_t kq = sbase + (s ? OFF_KQ1 : OFF_KQ0);
+#pragma unroll 1
                     for (int kk = 0; kk < 8; ++kk) {
-                        const uint32_t off = (kk >> 2) * KQ_KB + (kk & 3) * 32;
-                        umma_bf16(tmem + TM_GW, sdesc_sw128(kq + off, 16, 1024),
-                                  sdesc_sw128(kq + off, 16, 1024), ID_G, kk > 0);
+                        const uint32_t o = ((kk >> 2) * KQ_KB + (kk & 3) * 32) >> 4;
+                        const uint64_t d = (s ? dKQk1 : dKQk0) + o;
+                        umma_bf16(tmem + TM_GW, d, d, ID_G, kk > 0);
                     }
                     umma_commit(cx.bar(B_G_DONE));
                 };
                 auto issue_wu = [&](uint32_t s) {
-                    const uint32_t kq = sbase + (s ? OFF_KQ1 : OFF_KQ0);
                     // (W): W^T[dk][i] = sum_j K[j][dk] Tbg[i][j]; A = K (MN-major), B = Tbg (K-major)
-                    for (int kk = 0; kk < 4; ++kk)
-                        umma_bf16(tmem + TM_GW, sdesc_sw128(kq + kk * 2048, KQ_KB, 1024),
-                                  sdesc_sw128(sbase + OFF_TBG + kk * 32, 16, 1024), ID_W, kk > 0);
                     // (U~): U^T[dv][i] = sum_j V[j][dv] Tb[i][j]; A = V (MN-major), B = Tb
-                    for (int kk = 0; kk < 4; ++kk)
-                        umma_bf16(tmem + TM_U + 64 * s, sdesc_sw128(sbase + OFF_V + kk * 2048, V_HALF, 1024),
-                                  sdesc_sw128(sbase + OFF_TB + kk * 32, 16, 1024), ID_U, kk > 0);
+#pragma unroll 1
+                    for (int kk = 0; kk < 4; ++kk) {
+                        umma_bf16(tmem + TM_GW, (s ? dKQm1 : dKQm0) + ((kk * 2048) >> 4), dTBG + ((kk * 32) >> 4), ID_W, kk > 0);
+                        umma_bf16(tmem + TM_U + 64 * s, dV + ((kk * 2048) >> 4), dTB + ((kk * 32) >> 4), ID_U, kk > 0);
+                    }
                     umma_commit(cx.bar(B_WU_DONE));
                     umma_commit(cx.bar(B_V_EMPTY));
                 };
@@ -459,8 +540,6 @@ __global__ void __launch_bounds__(NTHREADS, 1) gdn_prefill_chunk_kernel(const __
                         const uint32_t s = gc & 1;
                         ok = ok && cx.wait(B_KQ_FULL + s, m_kq[s] & 1);
                         ++m_kq[s];
-                        ok = ok && cx.wait(B_NORM, m_norm & 1);
-                        ++m_norm;
                         if (!ok) break;
                         tc_fence_after();
                         issue_gram(s);
@@ -475,49 +554,48 @@ __global__ void __launch_bounds__(NTHREADS, 1) gdn_prefill_chunk_kernel(const __
                     for (int n = 0; n < nc && ok; ++n) {
                         const uint32_t s = (gc + n) & 1;
                         const uint32_t s1 = (gc + n + 1) & 1;
-                        const uint32_t kq = sbase + (s ? OFF_KQ1 : OFF_KQ0);
                         const bool more = n + 1 < nc;
-                        if (more) {
-                            ok = ok && cx.wait(B_KQ_FULL + s1, m_kq[s1] & 1);
-                            ++m_kq[s1];
-                            ok = ok && cx.wait(B_NORM, m_norm & 1);
-                            ++m_norm;
-                            if (!ok) break;
-                            tc_fence_after();
-                            issue_gram(s1);
-                        }
-                        // chain 1: U^T += S^T (-W)^T ; Y = S^T Q^T
+                        // chain 1: U^T += S^T (-W)^T, then Y = S^T Q^T
                         ok = ok && cx.wait(B_S_READY, m_s & 1);
                         ++m_s;
                         ok = ok && cx.wait(B_WNEG, m_wneg & 1);
                         ++m_wneg;
                         if (!ok) break;
                         tc_fence_after();
+#pragma unroll 1
                         for (int kk = 0; kk < 8; ++kk) {
-                            const uint32_t aoff = (kk >> 2) * SBF_KB + (kk & 3) * 32;
-                            umma_bf16(tmem + TM_U + 64 * s, sdesc_sw128(sbase + OFF_SBF + aoff, 16, 1024),
-                                      sdesc_sw128(sbase + OFF_WNEG + kk * 2048, 8192, 1024), ID_1A, 1);
-                        }
-                        for (int kk = 0; kk < 8; ++kk) {
-                            const uint32_t aoff = (kk >> 2) * SBF_KB + (kk & 3) * 32;
-                            const uint32_t boff = (kk >> 2) * KQ_KB + 8192 + (kk & 3) * 32;
-                            umma_bf16(tmem + TM_Y + 64 * s, sdesc_sw128(sbase + OFF_SBF + aoff, 16, 1024),
-                                      sdesc_sw128(kq + boff, 16, 1024), ID_1B, kk > 0);
+                            const uint32_t ao = ((kk >> 2) * SBF_KB + (kk & 3) * 32) >> 4;
+                            umma_bf16(tmem + TM_U + 64 * s, dSBF + ao, dWNEG + ((kk * 2048) >> 4), ID_1A, 1);
                         }
                         umma_commit(cx.bar(B_U_DONE));
-                        // chain 2: S^T += Ud K ; Z = U^T P^T
+                        // Gram of the next chunk first: the prep warpgroup waits on it
+                        if (more) {
+                            ok = ok && cx.wait(B_KQ_FULL + s1, m_kq[s1] & 1);
+                            ++m_kq[s1];
+                            if (!ok) break;
+                            tc_fence_after();
+                            issue_gram(s1);
+                        }
+                        // Y = S^T Q^T (only needed for the outputs)
+#pragma unroll 1
+                        for (int kk = 0; kk < 8; ++kk) {
+                            const uint32_t ao = ((kk >> 2) * SBF_KB + (kk & 3) * 32) >> 4;
+                            const uint32_t bo = ((kk >> 2) * KQ_KB + 8192 + (kk & 3) * 32) >> 4;
+                            umma_bf16(tmem + TM_Y + 64 * s, dSBF + ao, (s ? dKQk1 : dKQk0) + bo, ID_1B, kk > 0);
+                        }
+                        // chain 2: S^T += Ud K, then Z = U^T P^T
                         ok = ok && cx.wait(B_E1, m_e1 & 1);
                         ++m_e1;
                         if (!ok) break;
                         tc_fence_after();
+#pragma unroll 1
                         for (int kk = 0; kk < 4; ++kk)
-                            umma_bf16(tmem + TM_S, sdesc_sw128(sbase + OFF_UBFD + kk * 32, 16, 1024),
-                                      sdesc_sw128(kq + kk * 2048, KQ_KB, 1024), ID_2, 1);
-                        const uint32_t pb = sbase + (s ? OFF_P1 : OFF_P0);
+                            umma_bf16(tmem + TM_S, dUBFD + ((kk * 32) >> 4), (s ? dKQm1 : dKQm0) + ((kk * 2048) >> 4), ID_2, 1);
+                        umma_commit(cx.bar(B_S_DONE));
+#pragma unroll 1
                         for (int kk = 0; kk < 4; ++kk)
-                            umma_bf16(tmem + TM_Z, sdesc_sw128(sbase + OFF_UBF + kk * 32, 16, 1024),
-                                      sdesc_sw128(pb + kk * 32, 16, 1024), ID_3, kk > 0);
-                        umma_commit(cx.bar(B_SZ_DONE));
+                            umma_bf16(tmem + TM_Z, dUBF + ((kk * 32) >> 4), (s ? dP1 : dP0) + ((kk * 32) >> 4), ID_3, kk > 0);
+                        umma_commit(cx.bar(B_Z_DONE));
                         umma_commit(cx.bar(B_KQ_EMPTY + s));
                         // prep MMAs of the next chunk
                         if (more) {
@@ -546,166 +624,68 @@ __global__ void __launch_bounds__(NTHREADS, 1) gdn_prefill_chunk_kernel(const __
                 for (int n = 0; n < nc && ok; ++n) {
                     const uint32_t s = (gc + n) & 1;
                     const int len_n = min(C, un.len - n * C);
-                    uint8_t *kq = smem + (s ? OFF_KQ1 : OFF_KQ0);
+                    const uint8_t *kq = smem + (s ? OFF_KQ1 : OFF_KQ0);
                     const float *gtile = reinterpret_cast<const float *>(smem + (s ? OFF_GB1 : OFF_GB0));
                     float *ga = reinterpret_cast<float *>(smem + (s ? OFF_GATE1 : OFF_GATE0));
                     ok = cx.wait(B_KQ_FULL + s, p_kq[s] & 1);
                     ++p_kq[s];
                     if (p_gate_empty[s] > 0) ok = ok && cx.wait(B_GATE_EMPTY + s, (p_gate_empty[s] - 1) & 1);
                     ++p_gate_empty[s];
-                    // --- gates: inclusive scan of the floored, masked log-decay (threads 0..63)
-                    float Gi = 0.f;
-                    if (tp < 64) {
-                        const int i = tp;
-                        const int hc = un.h & 3;
-                        float gi = 0.f, bi = 0.f;
-                        if (i < len_n) {
-                            gi = fmaxf(gtile[i * 4 + hc], G_FLOOR);
-                            bi = gtile[256 + i * 4 + hc];
+                    // --- row norms (K rows 0..63, Q rows 64..127), conflict-free chunk order
+                    {
+                        float rn = 1.f;
+                        if (p.qk_l2norm) {
+                            float ss = 0.f;
+#pragma unroll 2
+                            for (int c = 0; c < 8; ++c) {
+                                const uint32_t off = sw128(tp, c);
+                                const uint4 va = *reinterpret_cast<const uint4 *>(kq + off);
+                                const uint4 vb = *reinterpret_cast<const uint4 *>(kq + KQ_KB + off);
+                                ss += sumsq8_bf16(va) + sumsq8_bf16(vb);
+                            }
+                            rn = 1.0f / sqrtf(ss + 1e-12f);
                         }
-                        float x = gi;
+                        ga[GA_RK + tp] = rn;   // GA_RQ = GA_RK + 64
+                    }
+                    // --- gates (prep warp 0, tokens 2l and 2l+1 per lane): floored, masked
+                    //     log-decay, inclusive prefix sum, exponentials
+                    if (pw == 0) {
+                        const int i0 = 2 * lane, i1 = i0 + 1;
+                        const int hc = un.h & 3;
+                        const float g0 = i0 < len_n ? fmaxf(gtile[i0 * 4 + hc], G_FLOOR) : 0.f;
+                        const float g1 = i1 < len_n ? fmaxf(gtile[i1 * 4 + hc], G_FLOOR) : 0.f;
+                        const float b0 = i0 < len_n ? gtile[256 + i0 * 4 + hc] : 0.f;
+                        const float b1 = i1 < len_n ? gtile[256 + i1 * 4 + hc] : 0.f;
+                        float x = g0 + g1;
 #pragma unroll
                         for (int o = 1; o < 32; o <<= 1) {
                             const float y = __shfl_up_sync(0xffffffffu, x, o);
                             if (lane >= o) x += y;
                         }
-                        Gi = x;
-                        ga[GA_BETA + i] = bi;
-                        ga[GA_G2 + i] = Gi;   // raw scan for now (warp-local)
-                    }
-                    // --- L2 norm of K and Q rows in place (thread tp owns row tp)
-                    if (p.qk_l2norm) {
-                        uint4 *r0 = reinterpret_cast<uint4 *>(kq + tp * 128);
-                        uint4 *r1 = reinterpret_cast<uint4 *>(kq + KQ_KB + tp * 128);
-                        float ss = 0.f;
-                        uint4 v0[8], v1[8];
-#pragma unroll
-                        for (int c = 0; c < 8; ++c) {
-                            v0[c] = r0[c];
-                            v1[c] = r1[c];
-                            float x[8];
-                            unpack8_bf16(v0[c], x);
-#pragma unroll
-                            for (int e = 0; e < 8; ++e) ss += x[e] * x[e];
-                            unpack8_bf16(v1[c], x);
-#pragma unroll
-                            for (int e = 0; e < 8; ++e) ss += x[e] * x[e];
-                        }
-                        const float rn = 1.0f / sqrtf(ss + 1e-12f);
-#pragma unroll
-                        for (int c = 0; c < 8; ++c) {
-                            float x[8];
-                            unpack8_bf16(v0[c], x);
-#pragma unroll
-                            for (int e = 0; e < 8; ++e) x[e] *= rn;
-                            r0[c] = pack8_bf16(x);
-                            unpack8_bf16(v1[c], x);
-#pragma unroll
-                            for (int e = 0; e < 8; ++e) x[e] *= rn;
-                            r1[c] = pack8_bf16(x);
-                        }
-                        fence_proxy_async_smem();
+                        const float G2b = x * LOG2E;            // token i1
+                        const float G2a = (x - g1) * LOG2E;     // token i0
+                        const float gend = __shfl_sync(0xffffffffu, G2b, (lane & ~7) + 7);
+                        const float gcl = __shfl_sync(0xffffffffu, G2b, 31);
+                        *reinterpret_cast<float2 *>(ga + GA_G2 + i0) = make_float2(G2a, G2b);
+                        *reinterpret_cast<float2 *>(ga + GA_BETA + i0) = make_float2(b0, b1);
+                        *reinterpret_cast<float2 *>(ga + GA_CF + i0) =
+                            make_float2(ex2_approx(gend - G2a), ex2_approx(gend - G2b));
+                        *reinterpret_cast<float2 *>(ga + GA_GAM + i0) = make_float2(ex2_approx(G2a), ex2_approx(G2b));
+                        *reinterpret_cast<float2 *>(ga + GA_DEC + i0) =
+                            make_float2(ex2_approx(gcl - G2a), ex2_approx(gcl - G2b));
+                        if ((lane & 7) == 7) ga[GA_GEND + (lane >> 3)] = G2b;
+                        if (lane == 31) ga[GA_GC] = ex2_approx(G2b);
                     }
                     named_sync(1, 128);
-                    if (tp < 64) {
-                        // finish the 64-wide scan: add warp 0's total to warp 1
-                        if (tp >= 32) Gi += ga[GA_G2 + 31];
-                    }
-                    named_sync(1, 128);
-                    if (tp < 64) {
-                        const int i = tp;
-                        const float G2 = Gi * LOG2E;
-                        ga[GA_G2 + i] = G2;
-                        ga[GA_GAM + i] = exp2f(G2);
-                        ga[GA_BGAM + i] = ga[GA_BETA + i] * exp2f(G2);
-                        if ((i & 15) == 15) ga[GA_GEND + (i >> 4)] = G2;
-                        if (i == 63) ga[GA_GC] = exp2f(G2);
-                    }
-                    named_sync(1, 128);
-                    if (tp < 64) {
-                        const int i = tp;
-                        const float G2 = ga[GA_G2 + i];
-                        ga[GA_CF + i] = exp2f(ga[GA_GEND + (i >> 4)] - G2);
-                        ga[GA_DEC + i] = exp2f(ga[GA_G2 + 63] - G2);
-                    }
-                    named_sync(1, 128);
-                    if (tp == 0) {
-                        mbar_arrive(cx.bar(B_GATE_FULL + s));
-                        mbar_arrive(cx.bar(B_NORM));
-                    }
-                    // --- Gram -> A (rows 0..63) and P (rows 64..127)
+                    if (tp == 0) mbar_arrive(cx.bar(B_GATE_FULL + s));
+                    // --- Gram -> A (rows 0..63, fp32 blocks) and P (rows 64..127, bf16 tile)
                     ok = ok && cx.wait(B_G_DONE, p_g & 1);
                     ++p_g;
                     tc_fence_after();
-                    float gr[64];
                     {
-                        float t32[32];
-                        tmem_ld32(tl + TM_GW, t32);
-                        tmem_wait_ld();
-#pragma unroll
-                        for (int j = 0; j < 32; ++j) gr[j] = t32[j];
-                        tmem_ld32(tl + TM_GW + 32, t32);
-                        tmem_wait_ld();
-#pragma unroll
-                        for (int j = 0; j < 32; ++j) gr[32 + j] = t32[j];
-                    }
-                    {
-                        const int i = tp & 63;
-                        const int I = i >> 4;
-                        const float G2i = ga[GA_G2 + i];
-                        float rJ[4];
-#pragma unroll
-                        for (int J = 0; J < 4; ++J)
-                            rJ[J] = (J < I) ? exp2f(G2i - ga[GA_GEND + J]) : 0.f;
-                        if (tp < 64) {
-                            const float bi = ga[GA_BETA + i];
-                            // off-diagonal blocks J < I
-#pragma unroll
-                            for (int J = 0; J < 3; ++J) {
-                                if (J < I) {
-                                    float *blk = solve + a_slot(I, J) * SOLVE_BLK + (i & 15) * SOLVE_LD;
-#pragma unroll
-                                    for (int jj = 0; jj < 16; ++jj) {
-                                        const int j = 16 * J + jj;
-                                        blk[jj] = bi * gr[j] * rJ[J] * ga[GA_CF + j];
-                                    }
-                                }
-                            }
-                            // diagonal block: strictly lower
-                            {
-                                float *blk = solve + I * SOLVE_BLK + (i & 15) * SOLVE_LD;
-#pragma unroll
-                                for (int jj = 0; jj < 16; ++jj) {
-                                    const int j = 16 * I + jj;
-                                    float a = 0.f;
-#pragma unroll
-                                    for (int JJ = 0; JJ < 4; ++JJ)
-                                        if (JJ == I && jj < (i & 15))
-                                            a = bi * gr[16 * JJ + jj] * exp2f(G2i - ga[GA_G2 + j]);
-                                    blk[jj] = a;
-                                }
-                            }
-                        } else {
-                            // P row i (inclusive lower, unscaled by beta)
-                            uint8_t *prow = smem + (s ? OFF_P1 : OFF_P0);
-#pragma unroll
-                            for (int c = 0; c < 8; ++c) {
-                                float x[8];
-#pragma unroll
-                                for (int e = 0; e < 8; ++e) {
-                                    const int j = 8 * c + e;
-                                    const int J = j >> 4;
-                                    float f = 0.f;
-                                    if (j <= i) {
-                                        if (J < I) f = rJ[J] * ga[GA_CF + j];
-                                        else f = exp2f(G2i - ga[GA_G2 + j]);
-                                    }
-                                    x[e] = gr[j] * f;
-                                }
-                                *reinterpret_cast<uint4 *>(prow + sw128(i, c)) = pack8_bf16(x);
-                            }
-                            fence_proxy_async_smem();
-                        }
+                        uint8_t *ptile = smem + (s ? OFF_P1 : OFF_P0);
+                        build_row(tl + TM_GW, pw, ga, solve, ptile);
+                        if (pw >= 2) fence_proxy_async_smem();
                     }
                     tc_fence_before();
                     named_sync(1, 128);
@@ -716,90 +696,117 @@ __global__ void __launch_bounds__(NTHREADS, 1) gdn_prefill_chunk_kernel(const __
                         float x[16];
 #pragma unroll
                         for (int r = 0; r < 16; ++r) {
-                            float acc = (r == c) ? 1.f : 0.f;
+                            float a[16];
 #pragma unroll
-                            for (int m = 0; m < r; ++m) acc -= Ab[r * SOLVE_LD + m] * x[m];
-                            x[r] = acc;
+                            for (int q = 0; q < 4; ++q) {
+                                if (4 * q < r) {
+                                    const float4 v = ld4(Ab + r * SOLVE_LD + 4 * q);
+                                    a[4 * q] = v.x; a[4 * q + 1] = v.y; a[4 * q + 2] = v.z; a[4 * q + 3] = v.w;
+                                }
+                            }
+                            float acc0 = (r == c) ? 1.f : 0.f, acc1 = 0.f;
+#pragma unroll
+                            for (int m = 0; m < r; ++m) {
+                                if (m & 1) acc1 = fmaf(-a[m], x[m], acc1);
+                                else acc0 = fmaf(-a[m], x[m], acc0);
+                            }
+                            x[r] = acc0 + acc1;
                         }
                         float *Db = solve + (10 + I) * SOLVE_BLK;
 #pragma unroll
                         for (int r = 0; r < 16; ++r) Db[r * SOLVE_LD + c] = x[r];
                     }
                     named_sync(1, 128);
-                    // --- level 1: T_10 = -D_1 A_10 D_0 (warp 0), T_32 = -D_3 A_32 D_2 (warp 1)
+                    // --- block merges (warp-level tf32 products):
+                    //   L1: T_10 = -D_1 (A_10 D_0) (warp 0), T_32 = -D_3 (A_32 D_2) (warp 1)
+                    //   X : X_pq = (A_BA T_AA)_pq -> slot 2p+q (the dead A_II blocks)
+                    //   TB: T_{2+p,q} = -(T_BB X)_pq -> slot 6+2p+q (the dead A_BA blocks)
                     if (pw < 2) {
-                        const int lo = pw ? 2 : 0;   // block pair (lo+1, lo)
-                        float acc[2][4] = {};
-                        blk_mma(acc, solve + (pw ? 5 : 4) * SOLVE_BLK, solve + (10 + lo) * SOLVE_BLK);
                         float *tmp = solve + (pw ? 15 : 14) * SOLVE_BLK;
+                        float acc[2][4] = {};
+                        blk_mma(acc, solve + (pw ? 5 : 4) * SOLVE_BLK, solve + (pw ? 12 : 10) * SOLVE_BLK);
                         blk_store(tmp, acc, 1.f);
                         __syncwarp();
                         float acc2[2][4] = {};
-                        blk_mma(acc2, solve + (10 + lo + 1) * SOLVE_BLK, tmp);
+                        blk_mma(acc2, solve + (pw ? 13 : 11) * SOLVE_BLK, tmp);
                         __syncwarp();
                         blk_store(tmp, acc2, -1.f);
                     }
                     named_sync(1, 128);
-                    // --- X = A_BA T_AA (warp w: block (p = w>>1, q = w&1))
-                    {
+#pragma unroll 1
+                    for (int ph = 0; ph < 2; ++ph) {
                         const int pp = pw >> 1, q = pw & 1;
+                        const float *X0, *Y0, *X1 = nullptr, *Y1 = nullptr;
+                        int dst;
+                        float sgn;
+                        if (ph == 0) {
+                            if (q == 0) {
+                                X0 = solve + a_slot(2 + pp, 0) * SOLVE_BLK; Y0 = solve + 10 * SOLVE_BLK;
+                                X1 = solve + a_slot(2 + pp, 1) * SOLVE_BLK; Y1 = solve + 14 * SOLVE_BLK;
+                            } else {
+                                X0 = solve + a_slot(2 + pp, 1) * SOLVE_BLK; Y0 = solve + 11 * SOLVE_BLK;
+                            }
+                            dst = 2 * pp + q; sgn = 1.f;
+                        } else {
+                            if (pp == 0) {
+                                X0 = solve + 12 * SOLVE_BLK; Y0 = solve + q * SOLVE_BLK;
+                            } else {
+                                X0 = solve + 15 * SOLVE_BLK; Y0 = solve + q * SOLVE_BLK;
+                                X1 = solve + 13 * SOLVE_BLK; Y1 = solve + (2 + q) * SOLVE_BLK;
+                            }
+                            dst = 6 + 2 * pp + q; sgn = -1.f;
+                        }
                         float acc[2][4] = {};
-                        if (q == 0) {
-                            blk_mma(acc, solve + a_slot(2 + pp, 0) * SOLVE_BLK, solve + 10 * SOLVE_BLK);
-                            blk_mma(acc, solve + a_slot(2 + pp, 1) * SOLVE_BLK, solve + 14 * SOLVE_BLK);
-                        } else {
-                            blk_mma(acc, solve + a_slot(2 + pp, 1) * SOLVE_BLK, solve + 11 * SOLVE_BLK);
-                        }
-                        named_sync(1, 128);
-                        blk_store(solve + (6 + 2 * pp + q) * SOLVE_BLK, acc, 1.f);   // X_pq
-                        named_sync(1, 128);
-                        // --- T_BA = -T_BB X
-                        float acc2[2][4] = {};
-                        if (pp == 0) {
-                            blk_mma(acc2, solve + 12 * SOLVE_BLK, solve + (6 + q) * SOLVE_BLK);
-                        } else {
-                            blk_mma(acc2, solve + 15 * SOLVE_BLK, solve + (6 + q) * SOLVE_BLK);
-                            blk_mma(acc2, solve + 13 * SOLVE_BLK, solve + (8 + q) * SOLVE_BLK);
-                        }
-                        named_sync(1, 128);
-                        blk_store(solve + (6 + 2 * pp + q) * SOLVE_BLK, acc2, -1.f);  // T_{2+p, q}
+                        const int np = X1 ? 2 : 1;
+#pragma unroll 1
+                        for (int t = 0; t < np; ++t) blk_mma(acc, t ? X1 : X0, t ? Y1 : Y0);
+                        blk_store(solve + dst * SOLVE_BLK, acc, sgn);
                         named_sync(1, 128);
                     }
-                    // --- Tb = T diag(beta), Tbg = T diag(beta Gamma) (bf16, K-major, swizzled)
+                    // --- Tb = T diag(beta), Tbg = T diag(beta Gamma rk) (bf16, K-major, swizzled)
                     {
                         const int i = tp >> 1, jh = tp & 1;
                         const int I = i >> 4;
+#pragma unroll 1
+                        for (int cc = 0; cc < 4; cc += 2) {
+                            float tv[2][8], bb[2][8], bg[2][8];
 #pragma unroll
-                        for (int cc = 0; cc < 4; ++cc) {
-                            const int c = 4 * jh + cc;   // 16-byte chunk: j = 8c .. 8c+7
-                            const int J = c >> 1;
-                            float tv[8];
-                            if (J <= I) {
-                                const float *row = solve + t_slot(I, J) * SOLVE_BLK + (i & 15) * SOLVE_LD + 8 * (c & 1);
-                                const float4 a = *reinterpret_cast<const float4 *>(row);
-                                const float4 b = *reinterpret_cast<const float4 *>(row + 4);
-                                tv[0] = a.x; tv[1] = a.y; tv[2] = a.z; tv[3] = a.w;
-                                tv[4] = b.x; tv[5] = b.y; tv[6] = b.z; tv[7] = b.w;
-                                if (J == I) {
+                            for (int u = 0; u < 2; ++u) {
+                                const int c = 4 * jh + cc + u;   // 16-byte chunk: j = 8c .. 8c+7
+                                const int J = c >> 1;
+                                const float *row = solve + (J <= I ? t_slot(I, J) : 10) * SOLVE_BLK + (i & 15) * SOLVE_LD + 8 * (c & 1);
+                                const float4 a = ld4(row), b = ld4(row + 4);
+                                const float z = J <= I ? 1.f : 0.f;
+                                tv[u][0] = z * a.x; tv[u][1] = z * a.y; tv[u][2] = z * a.z; tv[u][3] = z * a.w;
+                                tv[u][4] = z * b.x; tv[u][5] = z * b.y; tv[u][6] = z * b.z; tv[u][7] = z * b.w;
+                                const float4 b0 = ld4(ga + GA_BETA + 8 * c), b1 = ld4(ga + GA_BETA + 8 * c + 4);
+                                const float4 g0 = ld4(ga + GA_GAM + 8 * c), g1 = ld4(ga + GA_GAM + 8 * c + 4);
+                                const float4 k0 = ld4(ga + GA_RK + 8 * c), k1 = ld4(ga + GA_RK + 8 * c + 4);
+                                bb[u][0] = b0.x; bb[u][1] = b0.y; bb[u][2] = b0.z; bb[u][3] = b0.w;
+                                bb[u][4] = b1.x; bb[u][5] = b1.y; bb[u][6] = b1.z; bb[u][7] = b1.w;
+                                bg[u][0] = b0.x * g0.x * k0.x; bg[u][1] = b0.y * g0.y * k0.y;
+                                bg[u][2] = b0.z * g0.z * k0.z; bg[u][3] = b0.w * g0.w * k0.w;
+                                bg[u][4] = b1.x * g1.x * k1.x; bg[u][5] = b1.y * g1.y * k1.y;
+                                bg[u][6] = b1.z * g1.z * k1.z; bg[u][7] = b1.w * g1.w * k1.w;
+                            }
+                            uint4 ob[2], og[2];
 #pragma unroll
-                                    for (int e = 0; e < 8; ++e) {
-                                        const int j = 8 * c + e;
-                                        if (j > i) tv[e] = 0.f;
-                                        if (j == i) tv[e] = 1.f;
-                                    }
+                            for (int u = 0; u < 2; ++u) {
+                                float xb[8], xg[8];
+#pragma unroll
+                                for (int e = 0; e < 8; ++e) {
+                                    xb[e] = tv[u][e] * bb[u][e];
+                                    xg[e] = tv[u][e] * bg[u][e];
                                 }
-                            } else {
-#pragma unroll
-                                for (int e = 0; e < 8; ++e) tv[e] = 0.f;
+                                ob[u] = pack8_bf16(xb);
+                                og[u] = pack8_bf16(xg);
                             }
-                            float xb[8], xg[8];
 #pragma unroll
-                            for (int e = 0; e < 8; ++e) {
-                                xb[e] = tv[e] * ga[GA_BETA + 8 * c + e];
-                                xg[e] = tv[e] * ga[GA_BGAM + 8 * c + e];
+                            for (int u = 0; u < 2; ++u) {
+                                const int c = 4 * jh + cc + u;
+                                *reinterpret_cast<uint4 *>(smem + OFF_TB + sw128(i, c)) = ob[u];
+                                *reinterpret_cast<uint4 *>(smem + OFF_TBG + sw128(i, c)) = og[u];
                             }
-                            *reinterpret_cast<uint4 *>(smem + OFF_TB + sw128(i, c)) = pack8_bf16(xb);
-                            *reinterpret_cast<uint4 *>(smem + OFF_TBG + sw128(i, c)) = pack8_bf16(xg);
                         }
                         fence_proxy_async_smem();
                     }
@@ -810,24 +817,15 @@ __global__ void __launch_bounds__(NTHREADS, 1) gdn_prefill_chunk_kernel(const __
                     ++p_wu;
                     tc_fence_after();
                     {
-                        float t32[32];
-                        tmem_ld32(tl + TM_GW, t32);
-                        tmem_wait_ld();
+#pragma unroll 1
+                        for (int q = 0; q < 4; ++q) {
+                            float t[16];
+                            tmem_ld16(tl + TM_GW + 16 * q, t);
+                            tmem_wait_ld();
 #pragma unroll
-                        for (int c = 0; c < 4; ++c) {
-                            float x[8];
-#pragma unroll
-                            for (int e = 0; e < 8; ++e) x[e] = -t32[8 * c + e];
-                            *reinterpret_cast<uint4 *>(smem + OFF_WNEG + sw128(tp, c)) = pack8_bf16(x);
-                        }
-                        tmem_ld32(tl + TM_GW + 32, t32);
-                        tmem_wait_ld();
-#pragma unroll
-                        for (int c = 0; c < 4; ++c) {
-                            float x[8];
-#pragma unroll
-                            for (int e = 0; e < 8; ++e) x[e] = -t32[8 * c + e];
-                            *reinterpret_cast<uint4 *>(smem + OFF_WNEG + sw128(tp, 4 + c)) = pack8_bf16(x);
+                            for (int e = 0; e < 16; ++e) t[e] = -t[e];
+                            *reinterpret_cast<uint4 *>(smem + OFF_WNEG + sw128(tp, 2 * q)) = pack8_bf16(t);
+                            *reinterpret_cast<uint4 *>(smem + OFF_WNEG + sw128(tp, 2 * q + 1)) = pack8_bf16(t + 8);
                         }
                         fence_proxy_async_smem();
                     }
@@ -851,7 +849,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) gdn_prefill_chunk_kernel(const __
                 float *fin = p.final_state + st_off;
                 if (nc == 0) {
                     for (int c = 0; c < D; c += 4) {
-                        float4 v = init ? *reinterpret_cast<const float4 *>(init + c) : make_float4(0.f, 0.f, 0.f, 0.f);
+                        float4 v = init ? ld4(init + c) : make_float4(0.f, 0.f, 0.f, 0.f);
                         *reinterpret_cast<float4 *>(fin + c) = v;
                     }
                     continue;
@@ -864,23 +862,20 @@ __global__ void __launch_bounds__(NTHREADS, 1) gdn_prefill_chunk_kernel(const __
                     ++s_gate[s];
                     const float *ga = reinterpret_cast<const float *>(smem + (s ? OFF_GATE1 : OFF_GATE0));
                     const float gC = ga[GA_GC];
-                    for (int half = 0; half < 2; ++half) {
-                        float x[64];
+#pragma unroll 1
+                    for (int q = 0; q < 8; ++q) {
+                        float x[16];
 #pragma unroll
-                        for (int c = 0; c < 64; c += 4) {
-                            float4 v = init ? *reinterpret_cast<const float4 *>(init + 64 * half + c) : make_float4(0.f, 0.f, 0.f, 0.f);
+                        for (int c = 0; c < 16; c += 4) {
+                            const float4 v = init ? ld4(init + 16 * q + c) : make_float4(0.f, 0.f, 0.f, 0.f);
                             x[c] = v.x; x[c + 1] = v.y; x[c + 2] = v.z; x[c + 3] = v.w;
                         }
+                        uint8_t *srow = smem + OFF_SBF + (q >> 2) * SBF_KB;
+                        *reinterpret_cast<uint4 *>(srow + sw128(dv, 2 * (q & 3))) = pack8_bf16(x);
+                        *reinterpret_cast<uint4 *>(srow + sw128(dv, 2 * (q & 3) + 1)) = pack8_bf16(x + 8);
 #pragma unroll
-                        for (int c = 0; c < 8; ++c)
-                            *reinterpret_cast<uint4 *>(smem + OFF_SBF + half * SBF_KB + sw128(dv, c)) = pack8_bf16(x + 8 * c);
-                        float t32[32];
-#pragma unroll
-                        for (int q = 0; q < 2; ++q) {
-#pragma unroll
-                            for (int e = 0; e < 32; ++e) t32[e] = gC * x[32 * q + e];
-                            tmem_st32(tl + TM_S + 64 * half + 32 * q, t32);
-                        }
+                        for (int e = 0; e < 16; ++e) x[e] *= gC;
+                        tmem_st16(tl + TM_S + 16 * q, x);
                     }
                     tmem_wait_st();
                     fence_proxy_async_smem();
@@ -893,31 +888,37 @@ __global__ void __launch_bounds__(NTHREADS, 1) gdn_prefill_chunk_kernel(const __
                     const uint32_t s1 = (gc + n + 1) & 1;
                     const int len_n = min(C, un.len - n * C);
                     const float *ga = reinterpret_cast<const float *>(smem + (s ? OFF_GATE1 : OFF_GATE0));
-                    // ---- E1: U^T -> bf16 tiles (plain and decayed)
+                    // ---- E1: U^T -> bf16 tiles (plain for Z, decayed and key-normed for S)
                     ok = cx.wait(B_U_DONE, s_u & 1);
                     ++s_u;
                     tc_fence_after();
+#pragma unroll 1
+                    for (int q = 0; q < 4; ++q) {
+                        float u[16], d[16];
+                        tmem_ld16(tl + TM_U + 64 * s + 16 * q, u);
 #pragma unroll
-                    for (int q = 0; q < 2; ++q) {
-                        float u[32];
-                        tmem_ld32(tl + TM_U + 64 * s + 32 * q, u);
-                        tmem_wait_ld();
-#pragma unroll
-                        for (int c = 0; c < 4; ++c) {
-                            float xd[8];
-#pragma unroll
-                            for (int e = 0; e < 8; ++e) xd[e] = u[8 * c + e] * ga[GA_DEC + 32 * q + 8 * c + e];
-                            *reinterpret_cast<uint4 *>(smem + OFF_UBF + sw128(dv, 4 * q + c)) = pack8_bf16(u + 8 * c);
-                            *reinterpret_cast<uint4 *>(smem + OFF_UBFD + sw128(dv, 4 * q + c)) = pack8_bf16(xd);
+                        for (int e = 0; e < 16; e += 4) {
+                            const float4 d4 = ld4(ga + GA_DEC + 16 * q + e);
+                            const float4 k4 = ld4(ga + GA_RK + 16 * q + e);
+                            d[e] = d4.x * k4.x; d[e + 1] = d4.y * k4.y; d[e + 2] = d4.z * k4.z; d[e + 3] = d4.w * k4.w;
                         }
+                        tmem_wait_ld();
+                        const uint4 p0 = pack8_bf16(u), p1 = pack8_bf16(u + 8);
+#pragma unroll
+                        for (int e = 0; e < 16; ++e) u[e] *= d[e];
+                        const uint4 p2 = pack8_bf16(u), p3 = pack8_bf16(u + 8);
+                        *reinterpret_cast<uint4 *>(smem + OFF_UBF + sw128(dv, 2 * q)) = p0;
+                        *reinterpret_cast<uint4 *>(smem + OFF_UBF + sw128(dv, 2 * q + 1)) = p1;
+                        *reinterpret_cast<uint4 *>(smem + OFF_UBFD + sw128(dv, 2 * q)) = p2;
+                        *reinterpret_cast<uint4 *>(smem + OFF_UBFD + sw128(dv, 2 * q + 1)) = p3;
                     }
                     fence_proxy_async_smem();
                     tc_fence_before();
                     named_sync(2, 128);
                     if (dv == 0) mbar_arrive(cx.bar(B_E1));
                     // ---- E2: new state -> bf16 tile (+ decay of the next chunk) or final state
-                    ok = ok && cx.wait(B_SZ_DONE, s_sz & 1);
-                    ++s_sz;
+                    ok = ok && cx.wait(B_S_DONE, s_sd & 1);
+                    ++s_sd;
                     tc_fence_after();
                     const bool more = n + 1 < nc;
                     float gC1 = 1.f;
@@ -926,22 +927,21 @@ __global__ void __launch_bounds__(NTHREADS, 1) gdn_prefill_chunk_kernel(const __
                         ++s_gate[s1];
                         gC1 = reinterpret_cast<const float *>(smem + (s1 ? OFF_GATE1 : OFF_GATE0))[GA_GC];
                     }
-#pragma unroll
-                    for (int q = 0; q < 4; ++q) {
-                        float x[32];
-                        tmem_ld32(tl + TM_S + 32 * q, x);
+#pragma unroll 1
+                    for (int q = 0; q < 8; ++q) {
+                        float x[16];
+                        tmem_ld16(tl + TM_S + 16 * q, x);
                         tmem_wait_ld();
                         if (more) {
+                            uint8_t *srow = smem + OFF_SBF + (q >> 2) * SBF_KB;
+                            *reinterpret_cast<uint4 *>(srow + sw128(dv, 2 * (q & 3))) = pack8_bf16(x);
+                            *reinterpret_cast<uint4 *>(srow + sw128(dv, 2 * (q & 3) + 1)) = pack8_bf16(x + 8);
 #pragma unroll
-                            for (int c = 0; c < 4; ++c)
-                                *reinterpret_cast<uint4 *>(smem + OFF_SBF + (q >> 1) * SBF_KB + sw128(dv, 4 * (q & 1) + c)) = pack8_bf16(x + 8 * c);
-#pragma unroll
-                            for (int e = 0; e < 32; ++e) x[e] *= gC1;
-                            tmem_st32(tl + TM_S + 32 * q, x);
+                            for (int e = 0; e < 16; ++e) x[e] *= gC1;
+                            tmem_st16(tl + TM_S + 16 * q, x);
                         } else {
 #pragma unroll
-                            for (int c = 0; c < 32; c += 4)
-                                *reinterpret_cast<float4 *>(fin + 32 * q + c) = make_float4(x[c], x[c + 1], x[c + 2], x[c + 3]);
+                            for (int c = 0; c < 16; c += 4) st4(fin + 16 * q + c, x[c], x[c + 1], x[c + 2], x[c + 3]);
                         }
                     }
                     if (more) {
@@ -951,24 +951,49 @@ __global__ void __launch_bounds__(NTHREADS, 1) gdn_prefill_chunk_kernel(const __
                         named_sync(2, 128);
                         if (dv == 0) mbar_arrive(cx.bar(B_S_READY));
                     }
-                    // ---- outputs O^T = scale (Y diag(Gamma) + Z)
+                    // ---- outputs O^T = scale (Y diag(Gamma rq) + Z): staged through the U tile
+                    ok = ok && cx.wait(B_Z_DONE, s_zd & 1);
+                    ++s_zd;
+                    tc_fence_after();
                     {
-                        __nv_bfloat16 *orow = p.out + ((int64_t)(un.start + n * C) * p.Hv + un.h) * D + dv;
-                        const int64_t ostride = (int64_t)p.Hv * D;
+                        uint8_t *ot = smem + OFF_UBF;   // [64 rows i][256 B], 16-byte chunks XOR (i & 15)
+                        const float sc = p.scale;
+#pragma unroll 1
+                        for (int q = 0; q < 4; ++q) {
+                            float y[16], z[16], gg[16];
+                            tmem_ld16(tl + TM_Y + 64 * s + 16 * q, y);
+                            tmem_ld16(tl + TM_Z + 16 * q, z);
 #pragma unroll
-                        for (int q = 0; q < 2; ++q) {
-                            float y[32], z[32];
-                            tmem_ld32(tl + TM_Y + 64 * s + 32 * q, y);
-                            tmem_ld32(tl + TM_Z + 32 * q, z);
-                            tmem_wait_ld();
-#pragma unroll
-                            for (int e = 0; e < 32; ++e) {
-                                const int i = 32 * q + e;
-                                if (i < len_n) {
-                                    const float o = p.scale * (ga[GA_GAM + i] * y[e] + z[e]);
-                                    orow[i * ostride] = __float2bfloat16_rn(o);
-                                }
+                            for (int e = 0; e < 16; e += 4) {
+                                const float4 g4 = ld4(ga + GA_GAM + 16 * q + e);
+                                const float4 q4 = ld4(ga + GA_RQ + 16 * q + e);
+                                gg[e] = g4.x * q4.x; gg[e + 1] = g4.y * q4.y; gg[e + 2] = g4.z * q4.z; gg[e + 3] = g4.w * q4.w;
                             }
+                            tmem_wait_ld();
+                            __nv_bfloat16 ob[16];
+#pragma unroll
+                            for (int e = 0; e < 16; ++e) ob[e] = __float2bfloat16_rn(sc * fmaf(gg[e], y[e], z[e]));
+#pragma unroll
+                            for (int e = 0; e < 16; ++e) {
+                                const uint32_t i = 16u * q + e;
+                                const uint32_t off = i * 256u + ((((uint32_t)dv >> 3) ^ (i & 15u)) << 4) +
+                                                     ((uint32_t)dv & 7u) * 2u;
+                                *reinterpret_cast<__nv_bfloat16 *>(ot + off) = ob[e];
+                            }
+                        }
+                        named_sync(2, 128);
+                        // coalesced 16-byte stores: thread -> (row i = dv >> 1, half = dv & 1)
+                        const int i = dv >> 1, hf = dv & 1;
+                        if (i < len_n) {
+                            __nv_bfloat16 *orow = p.out + ((int64_t)(un.start + n * C + i) * p.Hv + un.h) * D + 64 * hf;
+                            uint4 v[8];
+#pragma unroll
+                            for (int c = 0; c < 8; ++c) {
+                                const uint32_t ch = (uint32_t)(8 * hf + c);
+                                v[c] = *reinterpret_cast<const uint4 *>(ot + (uint32_t)i * 256u + ((ch ^ ((uint32_t)i & 15u)) << 4));
+                            }
+#pragma unroll
+                            for (int c = 0; c < 8; ++c) *reinterpret_cast<uint4 *>(orow + 8 * c) = v[c];
                         }
                     }
                     tc_fence_before();
@@ -987,7 +1012,6 @@ __global__ void __launch_bounds__(NTHREADS, 1) gdn_prefill_chunk_kernel(const __
 
     // teardown: drain outstanding TMA stages on abort, then free TMEM
     if (cx.aborted() && warp == 8 && lane == 0) {
-        // every armed stage either completed or will complete; wait (bounded) for each
         for (int s = 0; s < 2; ++s) {
             const long long t0 = clock64();
             while (kq_use[s] > 0 && !mbar_try_wait(cx.bar(B_KQ_FULL + s), (kq_use[s] - 1) & 1))
