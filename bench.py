@@ -51,6 +51,24 @@ def load_peaks():
             "source": "fallback"}
 
 
+def ncu_traffic(profile_name: str, source: str):
+    """DRAM bytes per launch recorded in profiles/<profile_name> by an ncu capture, or None when
+    the kernel source changed since (the summary stores the first 16 hex of its sha256)."""
+    import hashlib
+    import re
+    path = os.path.join(ROOT, "profiles", profile_name)
+    src = os.path.join(ROOT, "gated_deltanet_state_gdn_b200", "csrc", source)
+    if not (os.path.exists(path) and os.path.exists(src)):
+        return None
+    text = open(path).read()
+    m_t = re.search(r"^traffic_bytes_per_launch:\s*(\d+)", text, re.M)
+    m_h = re.search(r"^source_sha256_16:\s*([0-9a-f]+)", text, re.M)
+    if not (m_t and m_h):
+        return None
+    sha = hashlib.sha256(open(src, "rb").read()).hexdigest()[:16]
+    return int(m_t.group(1)) if sha == m_h.group(1) else None
+
+
 def prefill_flops_per_token_head(Dk, Dv, C=CHUNK):
     """Tensor-core FLOPs of the chunked form per token and value head:
     Gram K K^T and Q K^T (2 * 2 C Dk), W = T diag(b G) K (2 C Dk), U~ = T diag(b) V (2 C Dv),
@@ -155,13 +173,20 @@ def dist_setup():
     return world, rank, local
 
 
-def max_over_ranks(x: float, world: int) -> float:
+def max_over_ranks(x: float, world: int, device: str = "cuda") -> float:
+    """Max of a per-rank time over all ranks (replicas are timed independently; the job
+    takes as long as its slowest rank)."""
     if world == 1:
         return x
     import torch.distributed as dist
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    t = torch.tensor([x], dtype=torch.float64, device=device)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
+
+
+def job_throughput(units_per_rank: int, world: int, max_ms_per_step: float) -> float:
+    """Whole-job throughput of `world` weak-scaled replicas: all ranks' units / slowest rank."""
+    return units_per_rank * world / (max_ms_per_step / 1e3)
 
 
 def barrier(world):
@@ -413,7 +438,7 @@ def main():
     max_ms = max_over_ranks(total_ms, world)
     ms_per_step = max_ms / args.steps
     tokens = case.N * world
-    value = tokens / (ms_per_step / 1e3)
+    value = job_throughput(case.N, world, ms_per_step)
     launches = args.steps
 
     chunked = gdn.prefill_uses_chunked(case.q.dtype, Hv, Dk, Dv)
@@ -421,9 +446,13 @@ def main():
     if chunked:
         flops = case.N * Hv * prefill_flops_per_token_head(Dk, Dv)
         ach = flops / avg_launch_s / 1e12
+        traffic = ncu_traffic("prefill_chunk_ragged_prefill.md", "prefill_chunk.cu") \
+            if args.workload == "ragged" else None
         roof = {"kernel": "gdn_prefill_chunk", "bound": "tensor", "achieved": ach,
                 "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
-                "frac": ach / peaks["bf16_tflops"], "traffic": None,
+                "frac": ach / peaks["bf16_tflops"], "traffic": traffic,
+                "algorithmic_bytes": prefill_bytes(case),
+                "hbm_frac": prefill_bytes(case) / avg_launch_s / 1e9 / peaks["hbm_gbs"],
                 "peak_source": peaks["source"] + " (burst bf16)"}
     else:
         byts = prefill_bytes(case)
