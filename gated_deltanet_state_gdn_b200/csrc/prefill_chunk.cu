@@ -27,16 +27,18 @@
 //   (2)  S^T += (U^T diag(exp(G_C - G) rk)) . K   (fp32 accumulator stays in TMEM)
 //   (3)  Z    = U^T . P^T
 //   O^T = scale (Y diag(Gamma rq) + Z)
-// TMEM (512 columns): S^T [0,128) | U^T x2 [128,256) | Y x2 [256,384) |
-// Z [384,448) | Gram/W^T [448,512).
+// TMEM (512 columns allocated): S^T [0,128) | U^T [128,192) | Y [192,256) |
+// Z [256,320) | Gram [320,384) | W^T [384,448).
 //
-// CTA = 10 warps, one (request, value head) unit at a time, persistent over a
+// CTA = 15 warps, one (request, value head) unit at a time, persistent over a
 // longest-first unit list:
-//   warps 0-3  state warpgroup: TMEM <-> bf16 operand tiles, outputs, state I/O
-//   warps 4-7  prep warpgroup: row norms, gates, Gram -> A and P, the 64x64
-//              unit-triangular solve, T/W tiles (runs one chunk ahead)
-//   warp  8    TMA producer (q/k/v/g/beta tiles, two stages)
-//   warp  9    TMEM owner and single-thread UMMA issuer
+//   warps 0-3   state warpgroup: TMEM <-> bf16 operand tiles, outputs, state I/O
+//   warps 4-11  prep warpgroups (two threads per TMEM lane): row norms, gates,
+//               Gram -> A and P, the 64x64 unit-triangular solve, T/W tiles
+//               (runs one chunk ahead)
+//   warp  12    TMA producer (q/k/v/g/beta tiles, two stages)
+//   warp  13    TMEM owner; UMMA issuer of the state chain (1a, 1b, 2, 3)
+//   warp  14    UMMA issuer of the prep stream (G, W, U~)
 // Every wait on an mbarrier is bounded; on timeout the kernel sets
 // GDN_DEV_TIMEOUT in the status word, drains and exits.
 #include <cudaTypedefs.h>
@@ -52,8 +54,9 @@ namespace gdn_chunk {
 
 constexpr int C = 64;       // chunk length (tokens)
 constexpr int D = 128;      // Dk = Dv
-constexpr int NTHREADS = 320;
+constexpr int NTHREADS = 480;
 constexpr int MAX_UNITS = 128;     // per CTA per batch of the unit list
+constexpr int TMA_WARP = 12, MMA_WARP = 13, ISSUE_WARP = 14;   // warps 0-3 state, 4-11 prep
 constexpr float G_FLOOR = -30.f;   // per-token log-decay floor (exp(-30) ~ 9e-14)
 constexpr float LOG2E = 1.4426950408889634f;
 
@@ -82,7 +85,7 @@ constexpr uint32_t OFF_GATE0 = OFF_GB1 + 2048;                 // processed gate
 constexpr uint32_t OFF_GATE1 = OFF_GATE0 + GATE_BYTES;
 constexpr uint32_t OFF_UNITS = OFF_GATE1 + GATE_BYTES;         // int4 x MAX_UNITS
 constexpr uint32_t OFF_BARS = OFF_UNITS + MAX_UNITS * 16;
-constexpr uint32_t NUM_BARS = 19;
+constexpr uint32_t NUM_BARS = 20;
 constexpr uint32_t OFF_MISC = OFF_BARS + 256;                  // tmem base, abort flag, count
 constexpr uint32_t SMEM_USED = OFF_MISC + 64;
 constexpr uint32_t SMEM_BYTES = SMEM_USED + 1024;              // + alignment slack
@@ -105,11 +108,11 @@ static_assert((GA_GC + 1) * 4 <= (int)GATE_BYTES, "gate stage size");
 enum {
     B_KQ_FULL = 0, B_KQ_EMPTY = 2, B_V_FULL = 4, B_V_EMPTY = 5, B_GATE_FULL = 6,
     B_GATE_EMPTY = 8, B_G_DONE = 10, B_T_READY = 11, B_WU_DONE = 12, B_WNEG = 13,
-    B_S_READY = 14, B_U_DONE = 15, B_E1 = 16, B_S_DONE = 17, B_Z_DONE = 18
+    B_S_READY = 14, B_U_DONE = 15, B_E1 = 16, B_S_DONE = 17, B_Z_DONE = 18, B_Y_FREE = 19
 };
 
 // TMEM columns
-constexpr uint32_t TM_S = 0, TM_U = 128, TM_Y = 256, TM_Z = 384, TM_GW = 448;
+constexpr uint32_t TM_S = 0, TM_U = 128, TM_Y = 192, TM_Z = 256, TM_G = 320, TM_W = 384;
 
 struct __align__(64) Params {
     CUtensorMap tm_q;     // (128, Hq, N) bf16, box (64, 1, 64), 128B swizzle
@@ -117,6 +120,7 @@ struct __align__(64) Params {
     CUtensorMap tm_v;     // (128, Hv, N)
     CUtensorMap tm_g;     // (Hv, N) fp32, box (4, 64)
     CUtensorMap tm_beta;
+    CUtensorMap tm_out;   // (128, Hv, N) bf16, box (64, 1, 64), 128B swizzle (stores)
     const int32_t *cu_seqlens;
     const float *initial_state;
     float *final_state;
@@ -320,17 +324,18 @@ __device__ __forceinline__ int t_slot(int I, int J)
     return 8 + J;
 }
 
-// Row i of A (prep warps 0-1: beta_i (k^_i . k^_j) exp(G_i - G_j) for j < i, fp32
-// into the solve blocks) or of P (prep warps 2-3: (q^_i . k^_j) exp(G_i - G_j) for
-// j <= i, bf16 tile), read 16 Gram columns at a time from TMEM.  The exponent of an
+// Row i of A (TMEM quadrants 0-1: beta_i (k^_i . k^_j) exp(G_i - G_j) for j < i, fp32
+// into the solve blocks) or of P (quadrants 2-3: (q^_i . k^_j) exp(G_i - G_j) for
+// j <= i, bf16 tile), read 16 Gram columns at a time from TMEM; half hh of the
+// prep threads covers column blocks 2hh and 2hh+1.  The exponent of an
 // earlier block J is split as exp(G_i - Gend_J) exp(Gend_J - G_j), both <= 1.
-__device__ __forceinline__ void build_row(uint32_t tl_gram, int pw, const float *ga, float *solve,
-                                          uint8_t *ptile)
+__device__ __forceinline__ void build_row(uint32_t tl_gram, int qd, int hh, const float *ga,
+                                          float *solve, uint8_t *ptile)
 {
     const int lane = threadIdx.x & 31;
-    const bool isP = pw >= 2;
+    const bool isP = qd >= 2;
     const int r = lane & 15;
-    const int I = 2 * (pw & 1) + (lane >> 4);
+    const int I = 2 * (qd & 1) + (lane >> 4);
     const int i = 16 * I + r;
     const float G2i = ga[GA_G2 + i];
     const float rowscale = isP ? ga[GA_RQ + i] : ga[GA_BETA + i] * ga[GA_RK + i];
@@ -338,7 +343,7 @@ __device__ __forceinline__ void build_row(uint32_t tl_gram, int pw, const float 
 #pragma unroll
     for (int J = 0; J < 3; ++J) gend[J] = ga[GA_GEND + J];
 #pragma unroll 1
-    for (int J = 0; J < 4; ++J) {
+    for (int J = 2 * hh; J < 2 * hh + 2; ++J) {
         // ---- loads (TMEM Gram columns, gate factors) before any store of this block
         float x[16], cf[16], g2[16], rk[16];
         tmem_ld16(tl_gram + 16 * J, x);
@@ -410,14 +415,14 @@ __global__ void __launch_bounds__(NTHREADS, 1) gdn_prefill_chunk_kernel(const __
         for (int i = 0; i < (int)NUM_BARS; ++i) mbar_init(cx.bar(i), 1);
         fence_mbar_init();
     }
-    if (warp == 8 && lane == 0) {
+    if (warp == TMA_WARP && lane == 0) {
         prefetch_tmap(&p.tm_q);
         prefetch_tmap(&p.tm_k);
         prefetch_tmap(&p.tm_v);
         prefetch_tmap(&p.tm_g);
         prefetch_tmap(&p.tm_beta);
     }
-    if (warp == 9) {
+    if (warp == MMA_WARP) {
         tmem_alloc(sbase + OFF_MISC, 512);
         tmem_relinquish();
     }
@@ -428,8 +433,8 @@ __global__ void __launch_bounds__(NTHREADS, 1) gdn_prefill_chunk_kernel(const __
 
     // per-role pipeline counters (persist across units and batches)
     uint32_t kq_use[2] = {0, 0}, v_use = 0;                          // TMA
-    uint32_t m_t = 0, m_wneg = 0, m_s = 0, m_e1 = 0, m_v = 0;        // MMA
-    uint32_t m_kq[2] = {0, 0};
+    uint32_t c_wneg = 0, c_s = 0, c_y = 0, c_e1 = 0;                 // chain issuer
+    uint32_t q_kq[2] = {0, 0}, q_t = 0, q_v = 0, q_wu = 0;            // prep-stream issuer
     uint32_t p_kq[2] = {0, 0}, p_gate_empty[2] = {0, 0}, p_g = 0, p_wu = 0;   // prep
     uint32_t s_u = 0, s_sd = 0, s_zd = 0, s_gate[2] = {0, 0};         // state
     uint32_t gc = 0;   // global chunk counter (same sequence in every role)
@@ -455,7 +460,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) gdn_prefill_chunk_kernel(const __
             }
         }
 
-        if (warp == 8) {
+        if (warp == TMA_WARP) {
             // ------------------------------------------------------------ TMA producer
             if (lane == 0) {
                 for (int k = 0; k < nunits && !cx.aborted(); ++k) {
@@ -485,8 +490,19 @@ __global__ void __launch_bounds__(NTHREADS, 1) gdn_prefill_chunk_kernel(const __
                     gc += nc;
                 }
             }
-        } else if (warp == 9) {
-            // ------------------------------------------------------------ UMMA issuer
+        } else if (warp == MMA_WARP || warp == ISSUE_WARP) {
+            // ------------------------------------------------------------ UMMA issuers
+            // Two single-thread issuers, so that neither stream waits behind the other's
+            // (blocking) MMA issue: the chain issuer (warp MMA_WARP: C1, C2 of each chunk,
+            // in order) and the prep-stream issuer (warp ISSUE_WARP: Gram and W/U~ of each
+            // chunk, in order).  Each commit tracks only its own thread's MMAs; every
+            // cross-stream hazard is ordered by an mbarrier:
+            //   G(x):  KQ(x) loaded; the Gram columns are free because the prep issuer
+            //          waited T_READY(x-1) (A/P of x-1 built) before WU(x-1)
+            //   WU(x): T(x) ready, V(x) loaded, E1(x-1) (U columns read and updated),
+            //          WNEG(x-1) (W columns converted)
+            //   C1(x): WNEG(x) (so WU(x) completed), S_READY(x); Y part after Y_FREE(x-1)
+            //   C2(x): E1(x)
             if (lane == 0) {
                 constexpr uint32_t ID_G = idesc_bf16(128, 64, 0, 0);
                 constexpr uint32_t ID_W = idesc_bf16(128, 64, 1, 0);
@@ -500,127 +516,142 @@ __global__ void __launch_bounds__(NTHREADS, 1) gdn_prefill_chunk_kernel(const __
                 const uint64_t dKQk1 = sdesc_sw128(sbase + OFF_KQ1, 16, 1024);
                 const uint64_t dKQm0 = sdesc_sw128(sbase + OFF_KQ0, KQ_KB, 1024);   // MN-major K
                 const uint64_t dKQm1 = sdesc_sw128(sbase + OFF_KQ1, KQ_KB, 1024);
-                const uint64_t dV = sdesc_sw128(sbase + OFF_V, V_HALF, 1024);
-                const uint64_t dTB = sdesc_sw128(sbase + OFF_TB, 16, 1024);
-                const uint64_t dTBG = sdesc_sw128(sbase + OFF_TBG, 16, 1024);
-                const uint64_t dSBF = sdesc_sw128(sbase + OFF_SBF, 16, 1024);
-                const uint64_t dWNEG = sdesc_sw128(sbase + OFF_WNEG, 8192, 1024);
-                const uint64_t dUBF = sdesc_sw128(sbase + OFF_UBF, 16, 1024);
-                const uint64_t dUBFD = sdesc_sw128(sbase + OFF_UBFD, 16, 1024);
-                const uint64_t dP0 = sdesc_sw128(sbase + OFF_P0, 16, 1024);
-                const uint64_t dP1 = sdesc_sw128(sbase + OFF_P1, 16, 1024);
                 bool ok = true;
-                auto issue_gram = [&](uint32_t s) {
-                    // (G): [K;Q] (128 x 128, K-major) x K^T
-#pragma unroll 1
-                    for (int kk = 0; kk < 8; ++kk) {
-                        const uint32_t o = ((kk >> 2) * KQ_KB + (kk & 3) * 32) >> 4;
-                        const uint64_t d = (s ? dKQk1 : dKQk0) + o;
-                        umma_bf16(tmem + TM_GW, d, d, ID_G, kk > 0);
-                    }
-                    umma_commit(cx.bar(B_G_DONE));
-                };
-                auto issue_wu = [&](uint32_t s) {
-                    // (W): W^T[dk][i] = sum_j K[j][dk] Tbg[i][j]; A = K (MN-major), B = Tbg (K-major)
-                    // (U~): U^T[dv][i] = sum_j V[j][dv] Tb[i][j]; A = V (MN-major), B = Tb
-#pragma unroll 1
-                    for (int kk = 0; kk < 4; ++kk) {
-                        umma_bf16(tmem + TM_GW, (s ? dKQm1 : dKQm0) + ((kk * 2048) >> 4), dTBG + ((kk * 32) >> 4), ID_W, kk > 0);
-                        umma_bf16(tmem + TM_U + 64 * s, dV + ((kk * 2048) >> 4), dTB + ((kk * 32) >> 4), ID_U, kk > 0);
-                    }
-                    umma_commit(cx.bar(B_WU_DONE));
-                    umma_commit(cx.bar(B_V_EMPTY));
-                };
-                for (int k = 0; k < nunits && ok; ++k) {
-                    const Unit un = load_unit(smem, k);
-                    const int nc = (un.len + C - 1) / C;
-                    if (nc == 0) continue;
-                    // prologue: prep MMAs of chunk 0
-                    {
-                        const uint32_t s = gc & 1;
-                        ok = ok && cx.wait(B_KQ_FULL + s, m_kq[s] & 1);
-                        ++m_kq[s];
-                        if (!ok) break;
-                        tc_fence_after();
-                        issue_gram(s);
-                        ok = ok && cx.wait(B_T_READY, m_t & 1);
-                        ++m_t;
-                        ok = ok && cx.wait(B_V_FULL, m_v & 1);
-                        ++m_v;
-                        if (!ok) break;
-                        tc_fence_after();
-                        issue_wu(s);
-                    }
-                    for (int n = 0; n < nc && ok; ++n) {
-                        const uint32_t s = (gc + n) & 1;
-                        const uint32_t s1 = (gc + n + 1) & 1;
-                        const bool more = n + 1 < nc;
-                        // chain 1: U^T += S^T (-W)^T, then Y = S^T Q^T
-                        ok = ok && cx.wait(B_S_READY, m_s & 1);
-                        ++m_s;
-                        ok = ok && cx.wait(B_WNEG, m_wneg & 1);
-                        ++m_wneg;
-                        if (!ok) break;
-                        tc_fence_after();
-#pragma unroll 1
-                        for (int kk = 0; kk < 8; ++kk) {
-                            const uint32_t ao = ((kk >> 2) * SBF_KB + (kk & 3) * 32) >> 4;
-                            umma_bf16(tmem + TM_U + 64 * s, dSBF + ao, dWNEG + ((kk * 2048) >> 4), ID_1A, 1);
-                        }
-                        umma_commit(cx.bar(B_U_DONE));
-                        // Gram of the next chunk first: the prep warpgroup waits on it
-                        if (more) {
-                            ok = ok && cx.wait(B_KQ_FULL + s1, m_kq[s1] & 1);
-                            ++m_kq[s1];
+                if (warp == ISSUE_WARP) {
+                    const uint64_t dV = sdesc_sw128(sbase + OFF_V, V_HALF, 1024);
+                    const uint64_t dTB = sdesc_sw128(sbase + OFF_TB, 16, 1024);
+                    const uint64_t dTBG = sdesc_sw128(sbase + OFF_TBG, 16, 1024);
+                    for (int k = 0; k < nunits && ok; ++k) {
+                        const Unit un = load_unit(smem, k);
+                        const int nc = (un.len + C - 1) / C;
+                        for (int n = 0; n < nc && ok; ++n) {
+                            const uint32_t s = (gc + n) & 1;
+                            // (G): [K;Q] (128 x 128, K-major) x K^T
+                            ok = cx.wait(B_KQ_FULL + s, q_kq[s] & 1);
+                            ++q_kq[s];
                             if (!ok) break;
                             tc_fence_after();
-                            issue_gram(s1);
-                        }
-                        // Y = S^T Q^T (only needed for the outputs)
 #pragma unroll 1
-                        for (int kk = 0; kk < 8; ++kk) {
-                            const uint32_t ao = ((kk >> 2) * SBF_KB + (kk & 3) * 32) >> 4;
-                            const uint32_t bo = ((kk >> 2) * KQ_KB + 8192 + (kk & 3) * 32) >> 4;
-                            umma_bf16(tmem + TM_Y + 64 * s, dSBF + ao, (s ? dKQk1 : dKQk0) + bo, ID_1B, kk > 0);
-                        }
-                        // chain 2: S^T += Ud K, then Z = U^T P^T
-                        ok = ok && cx.wait(B_E1, m_e1 & 1);
-                        ++m_e1;
-                        if (!ok) break;
-                        tc_fence_after();
-#pragma unroll 1
-                        for (int kk = 0; kk < 4; ++kk)
-                            umma_bf16(tmem + TM_S, dUBFD + ((kk * 32) >> 4), (s ? dKQm1 : dKQm0) + ((kk * 2048) >> 4), ID_2, 1);
-                        umma_commit(cx.bar(B_S_DONE));
-#pragma unroll 1
-                        for (int kk = 0; kk < 4; ++kk)
-                            umma_bf16(tmem + TM_Z, dUBF + ((kk * 32) >> 4), (s ? dP1 : dP0) + ((kk * 32) >> 4), ID_3, kk > 0);
-                        umma_commit(cx.bar(B_Z_DONE));
-                        umma_commit(cx.bar(B_KQ_EMPTY + s));
-                        // prep MMAs of the next chunk
-                        if (more) {
-                            ok = ok && cx.wait(B_T_READY, m_t & 1);
-                            ++m_t;
-                            ok = ok && cx.wait(B_V_FULL, m_v & 1);
-                            ++m_v;
+                            for (int kk = 0; kk < 8; ++kk) {
+                                const uint32_t o = ((kk >> 2) * KQ_KB + (kk & 3) * 32) >> 4;
+                                const uint64_t d = (s ? dKQk1 : dKQk0) + o;
+                                umma_bf16(tmem + TM_G, d, d, ID_G, kk > 0);
+                            }
+                            umma_commit(cx.bar(B_G_DONE));
+                            // (W): W^T[dk][i] = sum_j K[j][dk] Tbg[i][j]; A = K (MN-major), B = Tbg
+                            // (U~): U^T[dv][i] = sum_j V[j][dv] Tb[i][j]; A = V (MN-major), B = Tb
+                            ok = cx.wait(B_T_READY, q_t & 1);
+                            ++q_t;
+                            ok = ok && cx.wait(B_V_FULL, q_v & 1);
+                            ++q_v;
+                            if (q_wu > 0) {
+                                ok = ok && cx.wait(B_E1, (q_wu - 1) & 1);
+                                ok = ok && cx.wait(B_WNEG, (q_wu - 1) & 1);
+                            }
+                            ++q_wu;
                             if (!ok) break;
                             tc_fence_after();
-                            issue_wu(s1);
+#pragma unroll 1
+                            for (int kk = 0; kk < 4; ++kk) {
+                                umma_bf16(tmem + TM_W, (s ? dKQm1 : dKQm0) + ((kk * 2048) >> 4), dTBG + ((kk * 32) >> 4), ID_W, kk > 0);
+                                umma_bf16(tmem + TM_U, dV + ((kk * 2048) >> 4), dTB + ((kk * 32) >> 4), ID_U, kk > 0);
+                            }
+                            umma_commit(cx.bar(B_WU_DONE));
+                            umma_commit(cx.bar(B_V_EMPTY));
                         }
+                        gc += nc;
                     }
-                    gc += nc;
+                } else {
+                    const uint64_t dSBF = sdesc_sw128(sbase + OFF_SBF, 16, 1024);
+                    const uint64_t dWNEG = sdesc_sw128(sbase + OFF_WNEG, 8192, 1024);
+                    const uint64_t dUBF = sdesc_sw128(sbase + OFF_UBF, 16, 1024);
+                    const uint64_t dUBFD = sdesc_sw128(sbase + OFF_UBFD, 16, 1024);
+                    const uint64_t dP0 = sdesc_sw128(sbase + OFF_P0, 16, 1024);
+                    const uint64_t dP1 = sdesc_sw128(sbase + OFF_P1, 16, 1024);
+                    for (int k = 0; k < nunits && ok; ++k) {
+                        const Unit un = load_unit(smem, k);
+                        const int nc = (un.len + C - 1) / C;
+                        for (int n = 0; n < nc && ok; ++n) {
+                            const uint32_t s = (gc + n) & 1;
+                            // (1a) U^T += S^T (-W)^T
+                            ok = cx.wait(B_WNEG, c_wneg & 1);
+                            ++c_wneg;
+                            ok = ok && cx.wait(B_S_READY, c_s & 1);
+                            ++c_s;
+                            if (!ok) break;
+                            tc_fence_after();
+#pragma unroll 1
+                            for (int kk = 0; kk < 8; ++kk) {
+                                const uint32_t ao = ((kk >> 2) * SBF_KB + (kk & 3) * 32) >> 4;
+                                umma_bf16(tmem + TM_U, dSBF + ao, dWNEG + ((kk * 2048) >> 4), ID_1A, 1);
+                            }
+                            umma_commit(cx.bar(B_U_DONE));
+                            // (1b) Y = S^T Q^T, once the outputs of the previous chunk have read Y
+                            if (c_y > 0) ok = cx.wait(B_Y_FREE, (c_y - 1) & 1);
+                            ++c_y;
+                            if (!ok) break;
+                            tc_fence_after();
+#pragma unroll 1
+                            for (int kk = 0; kk < 8; ++kk) {
+                                const uint32_t ao = ((kk >> 2) * SBF_KB + (kk & 3) * 32) >> 4;
+                                const uint32_t bo = ((kk >> 2) * KQ_KB + 8192 + (kk & 3) * 32) >> 4;
+                                umma_bf16(tmem + TM_Y, dSBF + ao, (s ? dKQk1 : dKQk0) + bo, ID_1B, kk > 0);
+                            }
+                            // (2) S^T += Ud K, then (3) Z = U^T P^T
+                            ok = cx.wait(B_E1, c_e1 & 1);
+                            ++c_e1;
+                            if (!ok) break;
+                            tc_fence_after();
+#pragma unroll 1
+                            for (int kk = 0; kk < 4; ++kk)
+                                umma_bf16(tmem + TM_S, dUBFD + ((kk * 32) >> 4), (s ? dKQm1 : dKQm0) + ((kk * 2048) >> 4), ID_2, 1);
+                            umma_commit(cx.bar(B_S_DONE));
+#pragma unroll 1
+                            for (int kk = 0; kk < 4; ++kk)
+                                umma_bf16(tmem + TM_Z, dUBF + ((kk * 32) >> 4), (s ? dP1 : dP0) + ((kk * 32) >> 4), ID_3, kk > 0);
+                            umma_commit(cx.bar(B_Z_DONE));
+                            umma_commit(cx.bar(B_KQ_EMPTY + s));
+                        }
+                        gc += nc;
+                    }
                 }
             }
         } else if (warp >= 4) {
             // ------------------------------------------------------------ prep warpgroup
-            const int tp = tid - 128;           // 0..127 == TMEM lane
-            const int pw = tp >> 5;             // 0..3
-            const uint32_t tl = tmem + ((uint32_t)(32 * pw) << 16);
+            const int pt = tid - 128;           // 0..255
+            const int pw = pt >> 5;             // prep warp 0..7
+            const int qd = pw & 3;              // TMEM lane quadrant
+            const int hh = pw >> 2;             // half: which columns / which sub-task
+            const int tp = 32 * qd + lane;      // TMEM lane == row handled by this thread
+            const uint32_t tl = tmem + ((uint32_t)(32 * qd) << 16);
             float *solve = reinterpret_cast<float *>(smem + OFF_SOLVE);
-            for (int k = 0; k < nunits; ++k) {
+            bool wneg_pending = false;   // W^T of the previous chunk still to be converted
+            // -W^T (TMEM, lane dk) -> MN-major B tile (row dk); run by prep half 1, which
+            // then releases the chain of that chunk and the Gram of the next
+            auto convert_wneg = [&]() -> bool {
+                const bool w_ok = cx.wait(B_WU_DONE, p_wu & 1);
+                ++p_wu;
+                tc_fence_after();
+#pragma unroll 1
+                for (int q = 0; q < 4; ++q) {
+                    float t[16];
+                    tmem_ld16(tl + TM_W + 16 * q, t);
+                    tmem_wait_ld();
+#pragma unroll
+                    for (int e = 0; e < 16; ++e) t[e] = -t[e];
+                    *reinterpret_cast<uint4 *>(smem + OFF_WNEG + sw128(tp, 2 * q)) = pack8_bf16(t);
+                    *reinterpret_cast<uint4 *>(smem + OFF_WNEG + sw128(tp, 2 * q + 1)) = pack8_bf16(t + 8);
+                }
+                fence_proxy_async_smem();
+                tc_fence_before();
+                named_sync(3, 128);
+                if (pt == 128) mbar_arrive(cx.bar(B_WNEG));
+                return w_ok;
+            };
+            bool ok = true;
+            for (int k = 0; k < nunits && ok; ++k) {
                 const Unit un = load_unit(smem, k);
                 const int nc = (un.len + C - 1) / C;
-                bool ok = true;
                 for (int n = 0; n < nc && ok; ++n) {
                     const uint32_t s = (gc + n) & 1;
                     const int len_n = min(C, un.len - n * C);
@@ -631,8 +662,10 @@ __global__ void __launch_bounds__(NTHREADS, 1) gdn_prefill_chunk_kernel(const __
                     ++p_kq[s];
                     if (p_gate_empty[s] > 0) ok = ok && cx.wait(B_GATE_EMPTY + s, (p_gate_empty[s] - 1) & 1);
                     ++p_gate_empty[s];
-                    // --- row norms (K rows 0..63, Q rows 64..127), conflict-free chunk order
-                    {
+                    // --- half 1: the previous chunk's -W tile (the chain of that chunk waits on it)
+                    if (hh == 1 && wneg_pending) ok = convert_wneg() && ok;
+                    // --- row norms (K rows 0..63, Q rows 64..127, prep half 0), conflict-free chunk order
+                    if (hh == 0) {
                         float rn = 1.f;
                         if (p.qk_l2norm) {
                             float ss = 0.f;
@@ -676,22 +709,23 @@ __global__ void __launch_bounds__(NTHREADS, 1) gdn_prefill_chunk_kernel(const __
                         if ((lane & 7) == 7) ga[GA_GEND + (lane >> 3)] = G2b;
                         if (lane == 31) ga[GA_GC] = ex2_approx(G2b);
                     }
-                    named_sync(1, 128);
-                    if (tp == 0) mbar_arrive(cx.bar(B_GATE_FULL + s));
+                    named_sync(1, 256);
+                    if (pt == 0) mbar_arrive(cx.bar(B_GATE_FULL + s));
+                    wneg_pending = false;
                     // --- Gram -> A (rows 0..63, fp32 blocks) and P (rows 64..127, bf16 tile)
                     ok = ok && cx.wait(B_G_DONE, p_g & 1);
                     ++p_g;
                     tc_fence_after();
                     {
                         uint8_t *ptile = smem + (s ? OFF_P1 : OFF_P0);
-                        build_row(tl + TM_GW, pw, ga, solve, ptile);
-                        if (pw >= 2) fence_proxy_async_smem();
+                        build_row(tl + TM_G, qd, hh, ga, solve, ptile);
+                        if (qd >= 2) fence_proxy_async_smem();
                     }
                     tc_fence_before();
-                    named_sync(1, 128);
+                    named_sync(1, 256);
                     // --- diagonal 16x16 inverses D_I = (I + A_II)^-1 (threads 0..63, one column each)
-                    if (tp < 64) {
-                        const int I = tp >> 4, c = tp & 15;
+                    if (pt < 64) {
+                        const int I = pt >> 4, c = pt & 15;
                         const float *Ab = solve + I * SOLVE_BLK;
                         float x[16];
 #pragma unroll
@@ -716,7 +750,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) gdn_prefill_chunk_kernel(const __
 #pragma unroll
                         for (int r = 0; r < 16; ++r) Db[r * SOLVE_LD + c] = x[r];
                     }
-                    named_sync(1, 128);
+                    named_sync(1, 256);
                     // --- block merges (warp-level tf32 products):
                     //   L1: T_10 = -D_1 (A_10 D_0) (warp 0), T_32 = -D_3 (A_32 D_2) (warp 1)
                     //   X : X_pq = (A_BA T_AA)_pq -> slot 2p+q (the dead A_II blocks)
@@ -732,10 +766,10 @@ __global__ void __launch_bounds__(NTHREADS, 1) gdn_prefill_chunk_kernel(const __
                         __syncwarp();
                         blk_store(tmp, acc2, -1.f);
                     }
-                    named_sync(1, 128);
+                    named_sync(1, 256);
 #pragma unroll 1
                     for (int ph = 0; ph < 2; ++ph) {
-                        const int pp = pw >> 1, q = pw & 1;
+                        const int pp = (pw >> 1) & 1, q = pw & 1;
                         const float *X0, *Y0, *X1 = nullptr, *Y1 = nullptr;
                         int dst;
                         float sgn;
@@ -756,23 +790,25 @@ __global__ void __launch_bounds__(NTHREADS, 1) gdn_prefill_chunk_kernel(const __
                             }
                             dst = 6 + 2 * pp + q; sgn = -1.f;
                         }
-                        float acc[2][4] = {};
-                        const int np = X1 ? 2 : 1;
+                        if (pw < 4) {
+                            float acc[2][4] = {};
+                            const int np = X1 ? 2 : 1;
 #pragma unroll 1
-                        for (int t = 0; t < np; ++t) blk_mma(acc, t ? X1 : X0, t ? Y1 : Y0);
-                        blk_store(solve + dst * SOLVE_BLK, acc, sgn);
-                        named_sync(1, 128);
+                            for (int t = 0; t < np; ++t) blk_mma(acc, t ? X1 : X0, t ? Y1 : Y0);
+                            blk_store(solve + dst * SOLVE_BLK, acc, sgn);
+                        }
+                        named_sync(1, 256);
                     }
                     // --- Tb = T diag(beta), Tbg = T diag(beta Gamma rk) (bf16, K-major, swizzled)
                     {
-                        const int i = tp >> 1, jh = tp & 1;
+                        const int i = pt >> 2, jh = pt & 3;   // row, pair of 16-byte chunks
                         const int I = i >> 4;
-#pragma unroll 1
-                        for (int cc = 0; cc < 4; cc += 2) {
+                        {
+                            const int cc = 0;
                             float tv[2][8], bb[2][8], bg[2][8];
 #pragma unroll
                             for (int u = 0; u < 2; ++u) {
-                                const int c = 4 * jh + cc + u;   // 16-byte chunk: j = 8c .. 8c+7
+                                const int c = 2 * jh + cc + u;   // 16-byte chunk: j = 8c .. 8c+7
                                 const int J = c >> 1;
                                 const float *row = solve + (J <= I ? t_slot(I, J) : 10) * SOLVE_BLK + (i & 15) * SOLVE_LD + 8 * (c & 1);
                                 const float4 a = ld4(row), b = ld4(row + 4);
@@ -803,44 +839,27 @@ __global__ void __launch_bounds__(NTHREADS, 1) gdn_prefill_chunk_kernel(const __
                             }
 #pragma unroll
                             for (int u = 0; u < 2; ++u) {
-                                const int c = 4 * jh + cc + u;
+                                const int c = 2 * jh + cc + u;
                                 *reinterpret_cast<uint4 *>(smem + OFF_TB + sw128(i, c)) = ob[u];
                                 *reinterpret_cast<uint4 *>(smem + OFF_TBG + sw128(i, c)) = og[u];
                             }
                         }
                         fence_proxy_async_smem();
                     }
-                    named_sync(1, 128);
-                    if (tp == 0) mbar_arrive(cx.bar(B_T_READY));
-                    // --- W^T from TMEM -> (-W) as the MN-major B tile (row dk = tp)
-                    ok = ok && cx.wait(B_WU_DONE, p_wu & 1);
-                    ++p_wu;
-                    tc_fence_after();
-                    {
-#pragma unroll 1
-                        for (int q = 0; q < 4; ++q) {
-                            float t[16];
-                            tmem_ld16(tl + TM_GW + 16 * q, t);
-                            tmem_wait_ld();
-#pragma unroll
-                            for (int e = 0; e < 16; ++e) t[e] = -t[e];
-                            *reinterpret_cast<uint4 *>(smem + OFF_WNEG + sw128(tp, 2 * q)) = pack8_bf16(t);
-                            *reinterpret_cast<uint4 *>(smem + OFF_WNEG + sw128(tp, 2 * q + 1)) = pack8_bf16(t + 8);
-                        }
-                        fence_proxy_async_smem();
-                    }
-                    tc_fence_before();
-                    named_sync(1, 128);
-                    if (tp == 0) mbar_arrive(cx.bar(B_WNEG));
-                    ok = !named_sync_or(1, 128, !ok || cx.aborted());
+                    named_sync(1, 256);
+                    if (pt == 0) mbar_arrive(cx.bar(B_T_READY));
+                    wneg_pending = true;
+                    ok = !named_sync_or(1, 256, !ok || cx.aborted());
                 }
                 gc += nc;
-                if (!ok) break;
             }
+            // the last chunk's -W tile
+            if (ok && wneg_pending && hh == 1) convert_wneg();
         } else {
             // ------------------------------------------------------------ state warpgroup
             const int dv = tid;                 // 0..127 == TMEM lane
             const uint32_t tl = tmem + ((uint32_t)(32 * warp) << 16);
+            bool store_pending = false;         // an output TMA store may still read OFF_UBF
             for (int k = 0; k < nunits; ++k) {
                 const Unit un = load_unit(smem, k);
                 const int nc = (un.len + C - 1) / C;
@@ -892,10 +911,16 @@ __global__ void __launch_bounds__(NTHREADS, 1) gdn_prefill_chunk_kernel(const __
                     ok = cx.wait(B_U_DONE, s_u & 1);
                     ++s_u;
                     tc_fence_after();
+                    if (store_pending) {
+                        // the previous chunk's output store still reads the staging tile
+                        if (dv == 0) bulk_wait_read();
+                        named_sync(2, 128);
+                        store_pending = false;
+                    }
 #pragma unroll 1
                     for (int q = 0; q < 4; ++q) {
                         float u[16], d[16];
-                        tmem_ld16(tl + TM_U + 64 * s + 16 * q, u);
+                        tmem_ld16(tl + TM_U + 16 * q, u);
 #pragma unroll
                         for (int e = 0; e < 16; e += 4) {
                             const float4 d4 = ld4(ga + GA_DEC + 16 * q + e);
@@ -951,17 +976,20 @@ __global__ void __launch_bounds__(NTHREADS, 1) gdn_prefill_chunk_kernel(const __
                         named_sync(2, 128);
                         if (dv == 0) mbar_arrive(cx.bar(B_S_READY));
                     }
-                    // ---- outputs O^T = scale (Y diag(Gamma rq) + Z): staged through the U tile
+                    // ---- outputs O^T = scale (Y diag(Gamma rq) + Z), staged through the U tile as
+                    //      two 128B-swizzled [64 rows i][64 dv] bf16 tiles (the layout of the TMA box)
                     ok = ok && cx.wait(B_Z_DONE, s_zd & 1);
                     ++s_zd;
                     tc_fence_after();
                     {
-                        uint8_t *ot = smem + OFF_UBF;   // [64 rows i][256 B], 16-byte chunks XOR (i & 15)
+                        uint8_t *ot = smem + OFF_UBF;
                         const float sc = p.scale;
+                        const uint32_t obase = ((uint32_t)dv >> 6) * 8192u + ((uint32_t)dv & 7u) * 2u;
+                        const uint32_t och = ((uint32_t)dv >> 3) & 7u;
 #pragma unroll 1
                         for (int q = 0; q < 4; ++q) {
                             float y[16], z[16], gg[16];
-                            tmem_ld16(tl + TM_Y + 64 * s + 16 * q, y);
+                            tmem_ld16(tl + TM_Y + 16 * q, y);
                             tmem_ld16(tl + TM_Z + 16 * q, z);
 #pragma unroll
                             for (int e = 0; e < 16; e += 4) {
@@ -970,30 +998,40 @@ __global__ void __launch_bounds__(NTHREADS, 1) gdn_prefill_chunk_kernel(const __
                                 gg[e] = g4.x * q4.x; gg[e + 1] = g4.y * q4.y; gg[e + 2] = g4.z * q4.z; gg[e + 3] = g4.w * q4.w;
                             }
                             tmem_wait_ld();
-                            __nv_bfloat16 ob[16];
-#pragma unroll
-                            for (int e = 0; e < 16; ++e) ob[e] = __float2bfloat16_rn(sc * fmaf(gg[e], y[e], z[e]));
 #pragma unroll
                             for (int e = 0; e < 16; ++e) {
                                 const uint32_t i = 16u * q + e;
-                                const uint32_t off = i * 256u + ((((uint32_t)dv >> 3) ^ (i & 15u)) << 4) +
-                                                     ((uint32_t)dv & 7u) * 2u;
-                                *reinterpret_cast<__nv_bfloat16 *>(ot + off) = ob[e];
+                                *reinterpret_cast<__nv_bfloat16 *>(ot + obase + i * 128u + ((och ^ (i & 7u)) << 4)) =
+                                    __float2bfloat16_rn(sc * fmaf(gg[e], y[e], z[e]));
                             }
                         }
+                        fence_proxy_async_smem();
+                        tc_fence_before();
                         named_sync(2, 128);
-                        // coalesced 16-byte stores: thread -> (row i = dv >> 1, half = dv & 1)
-                        const int i = dv >> 1, hf = dv & 1;
-                        if (i < len_n) {
-                            __nv_bfloat16 *orow = p.out + ((int64_t)(un.start + n * C + i) * p.Hv + un.h) * D + 64 * hf;
-                            uint4 v[8];
-#pragma unroll
-                            for (int c = 0; c < 8; ++c) {
-                                const uint32_t ch = (uint32_t)(8 * hf + c);
-                                v[c] = *reinterpret_cast<const uint4 *>(ot + (uint32_t)i * 256u + ((ch ^ ((uint32_t)i & 15u)) << 4));
+                        if (dv == 0) mbar_arrive(cx.bar(B_Y_FREE));
+                        if (len_n == C) {
+                            // full chunk: two TMA box stores, completion checked before the tile is reused
+                            if (dv == 0) {
+                                const int row = un.start + n * C;
+                                tma_store_3d(&p.tm_out, sbase + OFF_UBF, 0, un.h, row);
+                                tma_store_3d(&p.tm_out, sbase + OFF_UBF + 8192, 64, un.h, row);
+                                bulk_commit();
                             }
+                            store_pending = true;
+                        } else {
+                            // ragged tail: rows past len_n belong to the next request; coalesced
+                            // 16-byte stores, thread -> (row i = dv >> 1, half = dv & 1)
+                            const int i = dv >> 1, hf = dv & 1;
+                            if (i < len_n) {
+                                __nv_bfloat16 *orow = p.out + ((int64_t)(un.start + n * C + i) * p.Hv + un.h) * D + 64 * hf;
+                                const uint8_t *srow = ot + hf * 8192 + i * 128;
+                                uint4 v[8];
 #pragma unroll
-                            for (int c = 0; c < 8; ++c) *reinterpret_cast<uint4 *>(orow + 8 * c) = v[c];
+                                for (int c = 0; c < 8; ++c)
+                                    v[c] = *reinterpret_cast<const uint4 *>(srow + ((c ^ (i & 7)) << 4));
+#pragma unroll
+                                for (int c = 0; c < 8; ++c) *reinterpret_cast<uint4 *>(orow + 8 * c) = v[c];
+                            }
                         }
                     }
                     tc_fence_before();
@@ -1004,6 +1042,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) gdn_prefill_chunk_kernel(const __
                 gc += nc;
                 if (!ok) break;
             }
+            if (dv == 0) bulk_wait_all();   // the unit list is rebuilt in the staging tile
         }
         __syncthreads();
         if (cx.aborted()) break;
@@ -1011,7 +1050,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) gdn_prefill_chunk_kernel(const __
     }
 
     // teardown: drain outstanding TMA stages on abort, then free TMEM
-    if (cx.aborted() && warp == 8 && lane == 0) {
+    if (cx.aborted() && warp == TMA_WARP && lane == 0) {
         for (int s = 0; s < 2; ++s) {
             const long long t0 = clock64();
             while (kq_use[s] > 0 && !mbar_try_wait(cx.bar(B_KQ_FULL + s), (kq_use[s] - 1) & 1))
@@ -1024,7 +1063,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) gdn_prefill_chunk_kernel(const __
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
-    if (warp == 9) tmem_dealloc(tmem, 512);
+    if (warp == MMA_WARP) tmem_dealloc(tmem, 512);
 }
 
 }  // namespace gdn_chunk
@@ -1108,6 +1147,7 @@ cudaError_t launch_prefill_chunked(const GdnPrefillArgs &a, cudaStream_t stream)
         if (!make_map_3d_bf16(&p.tm_q, a.q, 128, a.Hq, N) ||
             !make_map_3d_bf16(&p.tm_k, a.k, 128, a.Hq, N) ||
             !make_map_3d_bf16(&p.tm_v, a.v, 128, a.Hv, N) ||
+            !make_map_3d_bf16(&p.tm_out, a.out, 128, a.Hv, N) ||
             !make_map_2d_f32(&p.tm_g, a.g, a.Hv, N) || !make_map_2d_f32(&p.tm_beta, a.beta, a.Hv, N))
             return cudaErrorInvalidValue;
     }
