@@ -102,7 +102,8 @@ constexpr int GA_RK = 320;     // key norm factor rk_i (1 without qk_l2norm)
 constexpr int GA_RQ = 384;     // query norm factor rq_i
 constexpr int GA_GEND = 448;   // G_end of each 16-block * log2(e)  [4]
 constexpr int GA_GC = 452;     // exp(G_C)
-static_assert((GA_GC + 1) * 4 <= (int)GATE_BYTES, "gate stage size");
+constexpr int GA_BG = 456;     // beta_i Gamma_i rk_i (column scale of Tbg)
+static_assert((GA_BG + 64) * 4 <= (int)GATE_BYTES, "gate stage size");
 
 // barrier indices
 enum {
@@ -307,6 +308,28 @@ __device__ __forceinline__ void blk_store(float *Z, const float (&acc)[2][4], fl
     }
 }
 
+// Block (I, J) of T from an mma fragment (times sgn), written to the bf16 operand
+// tiles Tb = T diag(beta) and Tbg = T diag(beta Gamma rk) (K-major, 128B-swizzled)
+__device__ __forceinline__ void blk_store_tiles(const float (&acc)[2][4], float sgn, int I, int J,
+                                                const float *ga, uint8_t *tb, uint8_t *tbg)
+{
+    const int lane = threadIdx.x & 31;
+    const int g = lane >> 2, t = lane & 3;
+#pragma unroll
+    for (int nh = 0; nh < 2; ++nh) {
+        const int j = 16 * J + 8 * nh + 2 * t;
+        const float2 b = *reinterpret_cast<const float2 *>(ga + GA_BETA + j);
+        const float2 bg = *reinterpret_cast<const float2 *>(ga + GA_BG + j);
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+            const float x0 = sgn * acc[nh][2 * h], x1 = sgn * acc[nh][2 * h + 1];
+            const uint32_t off = sw128(16 * I + g + 8 * h, j >> 3) + (uint32_t)(j & 7) * 2u;
+            *reinterpret_cast<uint32_t *>(tb + off) = gdn::pack_bf16x2(x0 * b.x, x1 * b.y);
+            *reinterpret_cast<uint32_t *>(tbg + off) = gdn::pack_bf16x2(x0 * bg.x, x1 * bg.y);
+        }
+    }
+}
+
 // SOLVE slots: 0-3 A_II (strictly lower), 4 A_10, 5 A_32, 6-9 A_20 A_21 A_30 A_31
 // (later X, later T_20 T_21 T_30 T_31), 10-13 D_I = (I + A_II)^-1, 14 T_10, 15 T_32.
 __host__ __device__ constexpr int a_slot(int I, int J)
@@ -426,6 +449,10 @@ __global__ void __launch_bounds__(NTHREADS, 1) gdn_prefill_chunk_kernel(const __
         tmem_alloc(sbase + OFF_MISC, 512);
         tmem_relinquish();
     }
+    // T tiles: only the blocks on and below the diagonal are ever written
+    for (int i = tid; i < 16384 / 16; i += NTHREADS)
+        reinterpret_cast<uint4 *>(smem + OFF_TB)[i] = make_uint4(0u, 0u, 0u, 0u);
+    fence_proxy_async_smem();
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
@@ -720,6 +747,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) gdn_prefill_chunk_kernel(const __
                         uint8_t *ptile = smem + (s ? OFF_P1 : OFF_P0);
                         build_row(tl + TM_G, qd, hh, ga, solve, ptile);
                         if (qd >= 2) fence_proxy_async_smem();
+                        if (pt < 64) ga[GA_BG + pt] = ga[GA_BETA + pt] * ga[GA_GAM + pt] * ga[GA_RK + pt];
                     }
                     tc_fence_before();
                     named_sync(1, 256);
@@ -749,6 +777,15 @@ __global__ void __launch_bounds__(NTHREADS, 1) gdn_prefill_chunk_kernel(const __
                         float *Db = solve + (10 + I) * SOLVE_BLK;
 #pragma unroll
                         for (int r = 0; r < 16; ++r) Db[r * SOLVE_LD + c] = x[r];
+                        const int j = 16 * I + c;
+                        const float bj = ga[GA_BETA + j], sj = ga[GA_BG + j];
+                        const uint32_t cw = (uint32_t)(j & 7) * 2u;
+#pragma unroll
+                        for (int r = 0; r < 16; ++r) {
+                            const uint32_t off = sw128(16 * I + r, j >> 3) + cw;
+                            *reinterpret_cast<__nv_bfloat16 *>(smem + OFF_TB + off) = __float2bfloat16_rn(x[r] * bj);
+                            *reinterpret_cast<__nv_bfloat16 *>(smem + OFF_TBG + off) = __float2bfloat16_rn(x[r] * sj);
+                        }
                     }
                     named_sync(1, 256);
                     // --- block merges (warp-level tf32 products):
@@ -765,6 +802,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) gdn_prefill_chunk_kernel(const __
                         blk_mma(acc2, solve + (pw ? 13 : 11) * SOLVE_BLK, tmp);
                         __syncwarp();
                         blk_store(tmp, acc2, -1.f);
+                        blk_store_tiles(acc2, -1.f, pw ? 3 : 1, pw ? 2 : 0, ga, smem + OFF_TB, smem + OFF_TBG);
                     }
                     named_sync(1, 256);
 #pragma unroll 1
@@ -795,58 +833,12 @@ __global__ void __launch_bounds__(NTHREADS, 1) gdn_prefill_chunk_kernel(const __
                             const int np = X1 ? 2 : 1;
 #pragma unroll 1
                             for (int t = 0; t < np; ++t) blk_mma(acc, t ? X1 : X0, t ? Y1 : Y0);
-                            blk_store(solve + dst * SOLVE_BLK, acc, sgn);
+                            if (ph == 0) blk_store(solve + dst * SOLVE_BLK, acc, sgn);
+                            else blk_store_tiles(acc, sgn, 2 + pp, q, ga, smem + OFF_TB, smem + OFF_TBG);
                         }
+                        if (ph == 1) fence_proxy_async_smem();   // T tiles -> UMMA operands
                         named_sync(1, 256);
                     }
-                    // --- Tb = T diag(beta), Tbg = T diag(beta Gamma rk) (bf16, K-major, swizzled)
-                    {
-                        const int i = pt >> 2, jh = pt & 3;   // row, pair of 16-byte chunks
-                        const int I = i >> 4;
-                        {
-                            const int cc = 0;
-                            float tv[2][8], bb[2][8], bg[2][8];
-#pragma unroll
-                            for (int u = 0; u < 2; ++u) {
-                                const int c = 2 * jh + cc + u;   // 16-byte chunk: j = 8c .. 8c+7
-                                const int J = c >> 1;
-                                const float *row = solve + (J <= I ? t_slot(I, J) : 10) * SOLVE_BLK + (i & 15) * SOLVE_LD + 8 * (c & 1);
-                                const float4 a = ld4(row), b = ld4(row + 4);
-                                const float z = J <= I ? 1.f : 0.f;
-                                tv[u][0] = z * a.x; tv[u][1] = z * a.y; tv[u][2] = z * a.z; tv[u][3] = z * a.w;
-                                tv[u][4] = z * b.x; tv[u][5] = z * b.y; tv[u][6] = z * b.z; tv[u][7] = z * b.w;
-                                const float4 b0 = ld4(ga + GA_BETA + 8 * c), b1 = ld4(ga + GA_BETA + 8 * c + 4);
-                                const float4 g0 = ld4(ga + GA_GAM + 8 * c), g1 = ld4(ga + GA_GAM + 8 * c + 4);
-                                const float4 k0 = ld4(ga + GA_RK + 8 * c), k1 = ld4(ga + GA_RK + 8 * c + 4);
-                                bb[u][0] = b0.x; bb[u][1] = b0.y; bb[u][2] = b0.z; bb[u][3] = b0.w;
-                                bb[u][4] = b1.x; bb[u][5] = b1.y; bb[u][6] = b1.z; bb[u][7] = b1.w;
-                                bg[u][0] = b0.x * g0.x * k0.x; bg[u][1] = b0.y * g0.y * k0.y;
-                                bg[u][2] = b0.z * g0.z * k0.z; bg[u][3] = b0.w * g0.w * k0.w;
-                                bg[u][4] = b1.x * g1.x * k1.x; bg[u][5] = b1.y * g1.y * k1.y;
-                                bg[u][6] = b1.z * g1.z * k1.z; bg[u][7] = b1.w * g1.w * k1.w;
-                            }
-                            uint4 ob[2], og[2];
-#pragma unroll
-                            for (int u = 0; u < 2; ++u) {
-                                float xb[8], xg[8];
-#pragma unroll
-                                for (int e = 0; e < 8; ++e) {
-                                    xb[e] = tv[u][e] * bb[u][e];
-                                    xg[e] = tv[u][e] * bg[u][e];
-                                }
-                                ob[u] = pack8_bf16(xb);
-                                og[u] = pack8_bf16(xg);
-                            }
-#pragma unroll
-                            for (int u = 0; u < 2; ++u) {
-                                const int c = 2 * jh + cc + u;
-                                *reinterpret_cast<uint4 *>(smem + OFF_TB + sw128(i, c)) = ob[u];
-                                *reinterpret_cast<uint4 *>(smem + OFF_TBG + sw128(i, c)) = og[u];
-                            }
-                        }
-                        fence_proxy_async_smem();
-                    }
-                    named_sync(1, 256);
                     if (pt == 0) mbar_arrive(cx.bar(B_T_READY));
                     wneg_pending = true;
                     ok = !named_sync_or(1, 256, !ok || cx.aborted());
