@@ -28,7 +28,9 @@
 //   (3)  Z    = U^T . P^T
 //   O^T = scale (Y diag(Gamma rq) + Z)
 // TMEM (512 columns allocated): S^T [0,128) | U^T [128,192) | Y [192,256) |
-// Z [256,320) | Gram [320,384) | W^T [384,448).
+// Z [256,320) | Gram [320,384) | W^T [384,448).  After U^T is read, its columns
+// hold the bf16 A operands of (2) and (3) (per 16 tokens: 8 columns of U, then 8
+// of the decayed U), so those products read A from TMEM.
 //
 // CTA = 15 warps, one (request, value head) unit at a time, persistent over a
 // longest-first unit list:
@@ -68,14 +70,12 @@ constexpr uint32_t OFF_V = 65536;        // [dv half][64 rows j][128 B], 16 KB
 constexpr uint32_t V_HALF = 8192;
 constexpr uint32_t OFF_SBF = 81920;      // [dk half][128 rows dv][128 B], 32 KB
 constexpr uint32_t SBF_KB = 16384;
-constexpr uint32_t OFF_WNEG = 114688;    // [128 rows dk][64 i], 16 KB (MN-major B)
+constexpr uint32_t OFF_WNEG = 114688;    // [128 rows dk][64 i], 16 KB (MN-major B); also the output staging tile
 constexpr uint32_t OFF_P0 = 131072;      // [64 rows i][64 j], 8 KB
 constexpr uint32_t OFF_P1 = 139264;
 constexpr uint32_t OFF_TB = 147456;      // [64 rows i][64 j], 8 KB
 constexpr uint32_t OFF_TBG = 155648;
-constexpr uint32_t OFF_UBF = 163840;     // [128 rows dv][64 i], 16 KB; also the output staging tile
-constexpr uint32_t OFF_UBFD = 180224;
-constexpr uint32_t OFF_SOLVE = 196608;   // 16 blocks of 16 x 20 fp32
+constexpr uint32_t OFF_SOLVE = 163840;   // 16 blocks of 16 x 20 fp32
 constexpr uint32_t SOLVE_LD = 20;        // padded row stride (floats)
 constexpr uint32_t SOLVE_BLK = 16 * SOLVE_LD;  // floats per block
 constexpr uint32_t OFF_GB0 = OFF_SOLVE + 16 * SOLVE_BLK * 4;   // g tile 1 KB + beta tile 1 KB
@@ -85,9 +85,10 @@ constexpr uint32_t OFF_GATE0 = OFF_GB1 + 2048;                 // processed gate
 constexpr uint32_t OFF_GATE1 = OFF_GATE0 + GATE_BYTES;
 constexpr uint32_t OFF_UNITS = OFF_GATE1 + GATE_BYTES;         // int4 x MAX_UNITS
 constexpr uint32_t OFF_BARS = OFF_UNITS + MAX_UNITS * 16;
-constexpr uint32_t NUM_BARS = 20;
+constexpr uint32_t NUM_BARS = 21;
 constexpr uint32_t OFF_MISC = OFF_BARS + 256;                  // tmem base, abort flag, count
-constexpr uint32_t SMEM_USED = OFF_MISC + 64;
+constexpr uint32_t OFF_OGR = OFF_MISC + 64;                    // Gamma_i rq_i for the outputs, 64 floats
+constexpr uint32_t SMEM_USED = OFF_OGR + 256;
 constexpr uint32_t SMEM_BYTES = SMEM_USED + 1024;              // + alignment slack
 static_assert(SMEM_BYTES <= 232448, "shared memory budget");
 static_assert(OFF_GB0 % 1024 == 0, "alignment");
@@ -109,7 +110,8 @@ static_assert((GA_BG + 64) * 4 <= (int)GATE_BYTES, "gate stage size");
 enum {
     B_KQ_FULL = 0, B_KQ_EMPTY = 2, B_V_FULL = 4, B_V_EMPTY = 5, B_GATE_FULL = 6,
     B_GATE_EMPTY = 8, B_G_DONE = 10, B_T_READY = 11, B_WU_DONE = 12, B_WNEG = 13,
-    B_S_READY = 14, B_U_DONE = 15, B_E1 = 16, B_S_DONE = 17, B_Z_DONE = 18, B_Y_FREE = 19
+    B_S_READY = 14, B_U_DONE = 15, B_E1 = 16, B_S_DONE = 17, B_Z_DONE = 18, B_Y_FREE = 19,
+    B_G_FREE = 20
 };
 
 // TMEM columns
@@ -216,7 +218,7 @@ __device__ __forceinline__ void st4(float *p, float a, float b, float c, float d
 // goes to CTA (u mod G) on even waves and G-1-(u mod G) on odd waves.
 __device__ void build_unit_list(const Params &p, uint8_t *smem, int batch0, int *count_out)
 {
-    int *ord = reinterpret_cast<int *>(smem + OFF_UBF);   // scratch: up to 8192 ints
+    int *ord = reinterpret_cast<int *>(smem + OFF_SBF);   // scratch: up to 8192 ints
     const int B = p.B;
     const int tid = threadIdx.x;
     const bool sorted = B <= 8192;
@@ -461,9 +463,9 @@ __global__ void __launch_bounds__(NTHREADS, 1) gdn_prefill_chunk_kernel(const __
     // per-role pipeline counters (persist across units and batches)
     uint32_t kq_use[2] = {0, 0}, v_use = 0;                          // TMA
     uint32_t c_wneg = 0, c_s = 0, c_y = 0, c_e1 = 0;                 // chain issuer
-    uint32_t q_kq[2] = {0, 0}, q_t = 0, q_v = 0, q_wu = 0;            // prep-stream issuer
+    uint32_t q_kq[2] = {0, 0}, q_t = 0, q_v = 0, q_wu = 0, q_g = 0;   // prep-stream issuer
     uint32_t p_kq[2] = {0, 0}, p_gate_empty[2] = {0, 0}, p_g = 0, p_wu = 0;   // prep
-    uint32_t s_u = 0, s_sd = 0, s_zd = 0, s_gate[2] = {0, 0};         // state
+    uint32_t s_u = 0, s_sd = 0, s_zd = 0, s_wu = 0, s_gate[2] = {0, 0};   // state
     uint32_t gc = 0;   // global chunk counter (same sequence in every role)
 
     const int G = gridDim.x;
@@ -513,6 +515,19 @@ __global__ void __launch_bounds__(NTHREADS, 1) gdn_prefill_chunk_kernel(const __
                         mbar_arrive_expect_tx(cx.bar(B_V_FULL), 16384);
                         tma_load_3d(sbase + OFF_V, &p.tm_v, cx.bar(B_V_FULL), 0, un.h, t0);
                         tma_load_3d(sbase + OFF_V + V_HALF, &p.tm_v, cx.bar(B_V_FULL), 64, un.h, t0);
+                        if (n + 2 < nc) {
+                            // the chunk after next into L2: its loads wait on buffers freed by
+                            // the state chain and would otherwise start cold
+                            const int t2 = t0 + 2 * C;
+                            tma_prefetch_3d(&p.tm_k, 0, qh, t2);
+                            tma_prefetch_3d(&p.tm_k, 64, qh, t2);
+                            tma_prefetch_3d(&p.tm_q, 0, qh, t2);
+                            tma_prefetch_3d(&p.tm_q, 64, qh, t2);
+                            tma_prefetch_3d(&p.tm_v, 0, un.h, t2);
+                            tma_prefetch_3d(&p.tm_v, 64, un.h, t2);
+                            tma_prefetch_2d(&p.tm_g, un.h & ~3, t2);
+                            tma_prefetch_2d(&p.tm_beta, un.h & ~3, t2);
+                        }
                     }
                     gc += nc;
                 }
@@ -524,10 +539,10 @@ __global__ void __launch_bounds__(NTHREADS, 1) gdn_prefill_chunk_kernel(const __
             // in order) and the prep-stream issuer (warp ISSUE_WARP: Gram and W/U~ of each
             // chunk, in order).  Each commit tracks only its own thread's MMAs; every
             // cross-stream hazard is ordered by an mbarrier:
-            //   G(x):  KQ(x) loaded; the Gram columns are free because the prep issuer
-            //          waited T_READY(x-1) (A/P of x-1 built) before WU(x-1)
-            //   WU(x): T(x) ready, V(x) loaded, E1(x-1) (U columns read and updated),
-            //          WNEG(x-1) (W columns converted)
+            //   G(x):  KQ(x) loaded, G_FREE(x-1) (A/P of x-1 built); up to one chunk
+            //          ahead of WU inside a unit
+            //   WU(x): T(x) ready, V(x) loaded, Z_DONE(x-1) (the U columns hold the bf16
+            //          operands of (2)/(3) until then), WNEG(x-1) (W columns converted)
             //   C1(x): WNEG(x) (so WU(x) completed), S_READY(x); Y part after Y_FREE(x-1)
             //   C2(x): E1(x)
             if (lane == 0) {
@@ -548,51 +563,78 @@ __global__ void __launch_bounds__(NTHREADS, 1) gdn_prefill_chunk_kernel(const __
                     const uint64_t dV = sdesc_sw128(sbase + OFF_V, V_HALF, 1024);
                     const uint64_t dTB = sdesc_sw128(sbase + OFF_TB, 16, 1024);
                     const uint64_t dTBG = sdesc_sw128(sbase + OFF_TBG, 16, 1024);
+                    // Two tasks per chunk x, each issued as soon as its inputs are ready
+                    // (non-blocking tests, so neither waits behind the other):
+                    //   G(x):  previous Gram read by the prep (G_FREE), KQ(x) loaded; at most
+                    //          one chunk ahead of WU
+                    //   WU(x): G(x) issued, T(x) ready, V(x) loaded, Z_DONE(x-1), WNEG(x-1)
+                    // Every barrier tested here can run at most one phase ahead of its counter:
+                    // its next phase depends on the task that consumes this one.
                     for (int k = 0; k < nunits && ok; ++k) {
                         const Unit un = load_unit(smem, k);
                         const int nc = (un.len + C - 1) / C;
-                        for (int n = 0; n < nc && ok; ++n) {
-                            const uint32_t s = (gc + n) & 1;
-                            // (G): [K;Q] (128 x 128, K-major) x K^T
-                            ok = cx.wait(B_KQ_FULL + s, q_kq[s] & 1);
-                            ++q_kq[s];
-                            if (!ok) break;
-                            tc_fence_after();
+                        int gi = 0, wi = 0;   // G / WU issued in this unit
+                        long long t_last = clock64();
+                        while (wi < nc) {
+                            bool did = false;
+                            if (gi < nc && gi <= wi + 1) {
+                                const uint32_t sg = (gc + gi) & 1;
+                                if ((q_g == 0 || mbar_test_wait(cx.bar(B_G_FREE), (q_g - 1) & 1)) &&
+                                    mbar_test_wait(cx.bar(B_KQ_FULL + sg), q_kq[sg] & 1)) {
+                                    ++q_g;
+                                    ++q_kq[sg];
+                                    tc_fence_after();
+                                    // (G): [K;Q] (128 x 128, K-major) x K^T
 #pragma unroll 1
-                            for (int kk = 0; kk < 8; ++kk) {
-                                const uint32_t o = ((kk >> 2) * KQ_KB + (kk & 3) * 32) >> 4;
-                                const uint64_t d = (s ? dKQk1 : dKQk0) + o;
-                                umma_bf16(tmem + TM_G, d, d, ID_G, kk > 0);
+                                    for (int kk = 0; kk < 8; ++kk) {
+                                        const uint32_t o = ((kk >> 2) * KQ_KB + (kk & 3) * 32) >> 4;
+                                        const uint64_t d = (sg ? dKQk1 : dKQk0) + o;
+                                        umma_bf16(tmem + TM_G, d, d, ID_G, kk > 0);
+                                    }
+                                    umma_commit(cx.bar(B_G_DONE));
+                                    ++gi;
+                                    did = true;
+                                }
                             }
-                            umma_commit(cx.bar(B_G_DONE));
-                            // (W): W^T[dk][i] = sum_j K[j][dk] Tbg[i][j]; A = K (MN-major), B = Tbg
-                            // (U~): U^T[dv][i] = sum_j V[j][dv] Tb[i][j]; A = V (MN-major), B = Tb
-                            ok = cx.wait(B_T_READY, q_t & 1);
-                            ++q_t;
-                            ok = ok && cx.wait(B_V_FULL, q_v & 1);
-                            ++q_v;
-                            if (q_wu > 0) {
-                                ok = ok && cx.wait(B_E1, (q_wu - 1) & 1);
-                                ok = ok && cx.wait(B_WNEG, (q_wu - 1) & 1);
-                            }
-                            ++q_wu;
-                            if (!ok) break;
-                            tc_fence_after();
+                            if (!did && wi < gi && mbar_test_wait(cx.bar(B_T_READY), q_t & 1) &&
+                                mbar_test_wait(cx.bar(B_V_FULL), q_v & 1) &&
+                                (q_wu == 0 || (mbar_test_wait(cx.bar(B_Z_DONE), (q_wu - 1) & 1) &&
+                                               mbar_test_wait(cx.bar(B_WNEG), (q_wu - 1) & 1)))) {
+                                ++q_t;
+                                ++q_v;
+                                ++q_wu;
+                                const uint32_t s = (gc + wi) & 1;
+                                tc_fence_after();
+                                // (W): W^T[dk][i] = sum_j K[j][dk] Tbg[i][j]; A = K (MN-major), B = Tbg
+                                // (U~): U^T[dv][i] = sum_j V[j][dv] Tb[i][j]; A = V (MN-major), B = Tb
 #pragma unroll 1
-                            for (int kk = 0; kk < 4; ++kk) {
-                                umma_bf16(tmem + TM_W, (s ? dKQm1 : dKQm0) + ((kk * 2048) >> 4), dTBG + ((kk * 32) >> 4), ID_W, kk > 0);
-                                umma_bf16(tmem + TM_U, dV + ((kk * 2048) >> 4), dTB + ((kk * 32) >> 4), ID_U, kk > 0);
+                                for (int kk = 0; kk < 4; ++kk) {
+                                    umma_bf16(tmem + TM_W, (s ? dKQm1 : dKQm0) + ((kk * 2048) >> 4), dTBG + ((kk * 32) >> 4), ID_W, kk > 0);
+                                    umma_bf16(tmem + TM_U, dV + ((kk * 2048) >> 4), dTB + ((kk * 32) >> 4), ID_U, kk > 0);
+                                }
+                                umma_commit(cx.bar(B_WU_DONE));
+                                umma_commit(cx.bar(B_V_EMPTY));
+                                ++wi;
+                                did = true;
                             }
-                            umma_commit(cx.bar(B_WU_DONE));
-                            umma_commit(cx.bar(B_V_EMPTY));
+                            if (did) {
+                                t_last = clock64();
+                            } else {
+                                if (cx.aborted()) { ok = false; break; }
+                                if (clock64() - t_last > (1ll << 31)) {
+                                    *cx.abort_flag = 1;
+                                    if (p.dev_status) atomicOr(p.dev_status, GDN_DEV_TIMEOUT);
+                                    ok = false;
+                                    break;
+                                }
+                                __nanosleep(32);
+                            }
                         }
                         gc += nc;
                     }
                 } else {
                     const uint64_t dSBF = sdesc_sw128(sbase + OFF_SBF, 16, 1024);
                     const uint64_t dWNEG = sdesc_sw128(sbase + OFF_WNEG, 8192, 1024);
-                    const uint64_t dUBF = sdesc_sw128(sbase + OFF_UBF, 16, 1024);
-                    const uint64_t dUBFD = sdesc_sw128(sbase + OFF_UBFD, 16, 1024);
                     const uint64_t dP0 = sdesc_sw128(sbase + OFF_P0, 16, 1024);
                     const uint64_t dP1 = sdesc_sw128(sbase + OFF_P1, 16, 1024);
                     for (int k = 0; k < nunits && ok; ++k) {
@@ -631,11 +673,11 @@ __global__ void __launch_bounds__(NTHREADS, 1) gdn_prefill_chunk_kernel(const __
                             tc_fence_after();
 #pragma unroll 1
                             for (int kk = 0; kk < 4; ++kk)
-                                umma_bf16(tmem + TM_S, dUBFD + ((kk * 32) >> 4), (s ? dKQm1 : dKQm0) + ((kk * 2048) >> 4), ID_2, 1);
+                                umma_bf16_ts(tmem + TM_S, tmem + TM_U + 16 * kk + 8, (s ? dKQm1 : dKQm0) + ((kk * 2048) >> 4), ID_2, 1);
                             umma_commit(cx.bar(B_S_DONE));
 #pragma unroll 1
                             for (int kk = 0; kk < 4; ++kk)
-                                umma_bf16(tmem + TM_Z, dUBF + ((kk * 32) >> 4), (s ? dP1 : dP0) + ((kk * 32) >> 4), ID_3, kk > 0);
+                                umma_bf16_ts(tmem + TM_Z, tmem + TM_U + 16 * kk, (s ? dP1 : dP0) + ((kk * 32) >> 4), ID_3, kk > 0);
                             umma_commit(cx.bar(B_Z_DONE));
                             umma_commit(cx.bar(B_KQ_EMPTY + s));
                         }
@@ -652,29 +694,6 @@ __global__ void __launch_bounds__(NTHREADS, 1) gdn_prefill_chunk_kernel(const __
             const int tp = 32 * qd + lane;      // TMEM lane == row handled by this thread
             const uint32_t tl = tmem + ((uint32_t)(32 * qd) << 16);
             float *solve = reinterpret_cast<float *>(smem + OFF_SOLVE);
-            bool wneg_pending = false;   // W^T of the previous chunk still to be converted
-            // -W^T (TMEM, lane dk) -> MN-major B tile (row dk); run by prep half 1, which
-            // then releases the chain of that chunk and the Gram of the next
-            auto convert_wneg = [&]() -> bool {
-                const bool w_ok = cx.wait(B_WU_DONE, p_wu & 1);
-                ++p_wu;
-                tc_fence_after();
-#pragma unroll 1
-                for (int q = 0; q < 4; ++q) {
-                    float t[16];
-                    tmem_ld16(tl + TM_W + 16 * q, t);
-                    tmem_wait_ld();
-#pragma unroll
-                    for (int e = 0; e < 16; ++e) t[e] = -t[e];
-                    *reinterpret_cast<uint4 *>(smem + OFF_WNEG + sw128(tp, 2 * q)) = pack8_bf16(t);
-                    *reinterpret_cast<uint4 *>(smem + OFF_WNEG + sw128(tp, 2 * q + 1)) = pack8_bf16(t + 8);
-                }
-                fence_proxy_async_smem();
-                tc_fence_before();
-                named_sync(3, 128);
-                if (pt == 128) mbar_arrive(cx.bar(B_WNEG));
-                return w_ok;
-            };
             bool ok = true;
             for (int k = 0; k < nunits && ok; ++k) {
                 const Unit un = load_unit(smem, k);
@@ -689,8 +708,6 @@ __global__ void __launch_bounds__(NTHREADS, 1) gdn_prefill_chunk_kernel(const __
                     ++p_kq[s];
                     if (p_gate_empty[s] > 0) ok = ok && cx.wait(B_GATE_EMPTY + s, (p_gate_empty[s] - 1) & 1);
                     ++p_gate_empty[s];
-                    // --- half 1: the previous chunk's -W tile (the chain of that chunk waits on it)
-                    if (hh == 1 && wneg_pending) ok = convert_wneg() && ok;
                     // --- row norms (K rows 0..63, Q rows 64..127, prep half 0), conflict-free chunk order
                     if (hh == 0) {
                         float rn = 1.f;
@@ -707,9 +724,9 @@ __global__ void __launch_bounds__(NTHREADS, 1) gdn_prefill_chunk_kernel(const __
                         }
                         ga[GA_RK + tp] = rn;   // GA_RQ = GA_RK + 64
                     }
-                    // --- gates (prep warp 0, tokens 2l and 2l+1 per lane): floored, masked
+                    // --- gates (prep warp 4, tokens 2l and 2l+1 per lane): floored, masked
                     //     log-decay, inclusive prefix sum, exponentials
-                    if (pw == 0) {
+                    if (pw == 4) {
                         const int i0 = 2 * lane, i1 = i0 + 1;
                         const int hc = un.h & 3;
                         const float g0 = i0 < len_n ? fmaxf(gtile[i0 * 4 + hc], G_FLOOR) : 0.f;
@@ -738,7 +755,6 @@ __global__ void __launch_bounds__(NTHREADS, 1) gdn_prefill_chunk_kernel(const __
                     }
                     named_sync(1, 256);
                     if (pt == 0) mbar_arrive(cx.bar(B_GATE_FULL + s));
-                    wneg_pending = false;
                     // --- Gram -> A (rows 0..63, fp32 blocks) and P (rows 64..127, bf16 tile)
                     ok = ok && cx.wait(B_G_DONE, p_g & 1);
                     ++p_g;
@@ -751,6 +767,10 @@ __global__ void __launch_bounds__(NTHREADS, 1) gdn_prefill_chunk_kernel(const __
                     }
                     tc_fence_before();
                     named_sync(1, 256);
+                    if (pt == 0) mbar_arrive(cx.bar(B_G_FREE));
+                    // the T tiles of the previous chunk are read by its WU products
+                    if (p_wu > 0) ok = ok && cx.wait(B_WU_DONE, (p_wu - 1) & 1);
+                    ++p_wu;
                     // --- diagonal 16x16 inverses D_I = (I + A_II)^-1 (threads 0..63, one column each)
                     if (pt < 64) {
                         const int I = pt >> 4, c = pt & 15;
@@ -840,18 +860,16 @@ __global__ void __launch_bounds__(NTHREADS, 1) gdn_prefill_chunk_kernel(const __
                         named_sync(1, 256);
                     }
                     if (pt == 0) mbar_arrive(cx.bar(B_T_READY));
-                    wneg_pending = true;
                     ok = !named_sync_or(1, 256, !ok || cx.aborted());
                 }
                 gc += nc;
             }
-            // the last chunk's -W tile
-            if (ok && wneg_pending && hh == 1) convert_wneg();
         } else {
             // ------------------------------------------------------------ state warpgroup
             const int dv = tid;                 // 0..127 == TMEM lane
             const uint32_t tl = tmem + ((uint32_t)(32 * warp) << 16);
-            bool store_pending = false;         // an output TMA store may still read OFF_UBF
+            bool store_pending = false;         // an output TMA store may still read OFF_WNEG
+            float *ogr = reinterpret_cast<float *>(smem + OFF_OGR);
             for (int k = 0; k < nunits; ++k) {
                 const Unit un = load_unit(smem, k);
                 const int nc = (un.len + C - 1) / C;
@@ -899,16 +917,34 @@ __global__ void __launch_bounds__(NTHREADS, 1) gdn_prefill_chunk_kernel(const __
                     const uint32_t s1 = (gc + n + 1) & 1;
                     const int len_n = min(C, un.len - n * C);
                     const float *ga = reinterpret_cast<const float *>(smem + (s ? OFF_GATE1 : OFF_GATE0));
-                    // ---- E1: U^T -> bf16 tiles (plain for Z, decayed and key-normed for S)
-                    ok = cx.wait(B_U_DONE, s_u & 1);
-                    ++s_u;
+                    // ---- W^T (TMEM, lane dk) -> -W as the MN-major B tile of (1a) (row dk)
+                    ok = cx.wait(B_WU_DONE, s_wu & 1);
+                    ++s_wu;
                     tc_fence_after();
                     if (store_pending) {
-                        // the previous chunk's output store still reads the staging tile
+                        // the previous chunk's output store still reads the tile
                         if (dv == 0) bulk_wait_read();
                         named_sync(2, 128);
                         store_pending = false;
                     }
+#pragma unroll 1
+                    for (int q = 0; q < 4; ++q) {
+                        float t[16];
+                        tmem_ld16(tl + TM_W + 16 * q, t);
+                        tmem_wait_ld();
+#pragma unroll
+                        for (int e = 0; e < 16; ++e) t[e] = -t[e];
+                        *reinterpret_cast<uint4 *>(smem + OFF_WNEG + sw128(dv, 2 * q)) = pack8_bf16(t);
+                        *reinterpret_cast<uint4 *>(smem + OFF_WNEG + sw128(dv, 2 * q + 1)) = pack8_bf16(t + 8);
+                    }
+                    fence_proxy_async_smem();
+                    tc_fence_before();
+                    named_sync(2, 128);
+                    if (dv == 0) mbar_arrive(cx.bar(B_WNEG));
+                    // ---- E1: U^T -> bf16 tiles (plain for Z, decayed and key-normed for S)
+                    ok = ok && cx.wait(B_U_DONE, s_u & 1);
+                    ++s_u;
+                    tc_fence_after();
 #pragma unroll 1
                     for (int q = 0; q < 4; ++q) {
                         float u[16], d[16];
@@ -920,19 +956,24 @@ __global__ void __launch_bounds__(NTHREADS, 1) gdn_prefill_chunk_kernel(const __
                             d[e] = d4.x * k4.x; d[e + 1] = d4.y * k4.y; d[e + 2] = d4.z * k4.z; d[e + 3] = d4.w * k4.w;
                         }
                         tmem_wait_ld();
-                        const uint4 p0 = pack8_bf16(u), p1 = pack8_bf16(u + 8);
+                        // columns [16q, 16q+8): bf16 U (A of (3)); [16q+8, 16q+16): decayed U (A of (2))
+                        uint32_t w[16];
 #pragma unroll
-                        for (int e = 0; e < 16; ++e) u[e] *= d[e];
-                        const uint4 p2 = pack8_bf16(u), p3 = pack8_bf16(u + 8);
-                        *reinterpret_cast<uint4 *>(smem + OFF_UBF + sw128(dv, 2 * q)) = p0;
-                        *reinterpret_cast<uint4 *>(smem + OFF_UBF + sw128(dv, 2 * q + 1)) = p1;
-                        *reinterpret_cast<uint4 *>(smem + OFF_UBFD + sw128(dv, 2 * q)) = p2;
-                        *reinterpret_cast<uint4 *>(smem + OFF_UBFD + sw128(dv, 2 * q + 1)) = p3;
+                        for (int e = 0; e < 8; ++e) {
+                            w[e] = gdn::pack_bf16x2(u[2 * e], u[2 * e + 1]);
+                            w[8 + e] = gdn::pack_bf16x2(u[2 * e] * d[2 * e], u[2 * e + 1] * d[2 * e + 1]);
+                        }
+                        tmem_st16u(tl + TM_U + 16 * q, w);
                     }
+                    tmem_wait_st();
+                    if (dv < 64) ogr[dv] = ga[GA_GAM + dv] * ga[GA_RQ + dv];
                     fence_proxy_async_smem();
                     tc_fence_before();
                     named_sync(2, 128);
-                    if (dv == 0) mbar_arrive(cx.bar(B_E1));
+                    if (dv == 0) {
+                        mbar_arrive(cx.bar(B_E1));
+                        mbar_arrive(cx.bar(B_GATE_EMPTY + s));   // the outputs read ogr from here on
+                    }
                     // ---- E2: new state -> bf16 tile (+ decay of the next chunk) or final state
                     ok = ok && cx.wait(B_S_DONE, s_sd & 1);
                     ++s_sd;
@@ -974,7 +1015,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) gdn_prefill_chunk_kernel(const __
                     ++s_zd;
                     tc_fence_after();
                     {
-                        uint8_t *ot = smem + OFF_UBF;
+                        uint8_t *ot = smem + OFF_WNEG;
                         const float sc = p.scale;
                         const uint32_t obase = ((uint32_t)dv >> 6) * 8192u + ((uint32_t)dv & 7u) * 2u;
                         const uint32_t och = ((uint32_t)dv >> 3) & 7u;
@@ -985,9 +1026,8 @@ __global__ void __launch_bounds__(NTHREADS, 1) gdn_prefill_chunk_kernel(const __
                             tmem_ld16(tl + TM_Z + 16 * q, z);
 #pragma unroll
                             for (int e = 0; e < 16; e += 4) {
-                                const float4 g4 = ld4(ga + GA_GAM + 16 * q + e);
-                                const float4 q4 = ld4(ga + GA_RQ + 16 * q + e);
-                                gg[e] = g4.x * q4.x; gg[e + 1] = g4.y * q4.y; gg[e + 2] = g4.z * q4.z; gg[e + 3] = g4.w * q4.w;
+                                const float4 g4 = ld4(ogr + 16 * q + e);
+                                gg[e] = g4.x; gg[e + 1] = g4.y; gg[e + 2] = g4.z; gg[e + 3] = g4.w;
                             }
                             tmem_wait_ld();
 #pragma unroll
@@ -1005,8 +1045,8 @@ __global__ void __launch_bounds__(NTHREADS, 1) gdn_prefill_chunk_kernel(const __
                             // full chunk: two TMA box stores, completion checked before the tile is reused
                             if (dv == 0) {
                                 const int row = un.start + n * C;
-                                tma_store_3d(&p.tm_out, sbase + OFF_UBF, 0, un.h, row);
-                                tma_store_3d(&p.tm_out, sbase + OFF_UBF + 8192, 64, un.h, row);
+                                tma_store_3d(&p.tm_out, sbase + OFF_WNEG, 0, un.h, row);
+                                tma_store_3d(&p.tm_out, sbase + OFF_WNEG + 8192, 64, un.h, row);
                                 bulk_commit();
                             }
                             store_pending = true;
@@ -1026,9 +1066,6 @@ __global__ void __launch_bounds__(NTHREADS, 1) gdn_prefill_chunk_kernel(const __
                             }
                         }
                     }
-                    tc_fence_before();
-                    named_sync(2, 128);
-                    if (dv == 0) mbar_arrive(cx.bar(B_GATE_EMPTY + s));
                     ok = !named_sync_or(2, 128, !ok || cx.aborted());
                 }
                 gc += nc;
