@@ -22,23 +22,23 @@
 //   (G)  [K; Q] K^T                         -> TMEM  (Gram, 128 x 64)
 //   (W)  W^T  = K^T . Tbg^T                 -> TMEM  (Tbg = T diag(beta Gamma rk))
 //   (U~) U^T  = V^T . Tb^T                  -> TMEM  (Tb  = T diag(beta))
-//   (1a) U^T += S^T . (-W)^T                 (bf16 copy of S^T from SMEM)
+//   (1a) U^T += S^T . (-W)^T                 (bf16 copy of S^T from TMEM)
 //   (1b) Y    = S^T . Q^T
 //   (2)  S^T += (U^T diag(exp(G_C - G) rk)) . K   (fp32 accumulator stays in TMEM)
 //   (3)  Z    = U^T . P^T
 //   O^T = scale (Y diag(Gamma rq) + Z)
-// TMEM (512 columns allocated): S^T [0,128) | U^T [128,192) | Y [192,256) |
-// Z [256,320) | Gram [320,384) | W^T [384,448).  After U^T is read, its columns
-// hold the bf16 A operands of (2) and (3) (per 16 tokens: 8 columns of U, then 8
-// of the decayed U), so those products read A from TMEM.
+// TMEM (512 columns): S^T [0,128) | U^T [128,192) | Y [192,256) | Z [256,320) |
+// Gram [320,384) | W^T [384,448) | bf16 S^T [448,512) (A of 1a/1b, 8 columns per
+// 16 dk).  After U^T is read, its columns hold the bf16 A operands of (2) and (3)
+// (per 16 tokens: 8 columns of U, then 8 of the decayed U).
 //
 // CTA = 15 warps, one (request, value head) unit at a time, persistent over a
 // longest-first unit list:
 //   warps 0-3   state warpgroup: TMEM <-> bf16 operand tiles, outputs, state I/O
-//   warps 4-11  prep warpgroups (two threads per TMEM lane): row norms, gates,
-//               Gram -> A and P, the 64x64 unit-triangular solve, T/W tiles
-//               (runs one chunk ahead)
-//   warp  12    TMA producer (q/k/v/g/beta tiles, two stages)
+//   warps 4-7   prep front: row norms, gates, Gram -> A and P
+//   warps 8-11  prep back: the 64x64 unit-triangular solve and the bf16 T tiles
+//               (front and back work on consecutive chunks, ahead of the state chain)
+//   warp  12    TMA producer (q/k/g/beta tiles in three stages, v tiles in one)
 //   warp  13    TMEM owner; UMMA issuer of the state chain (1a, 1b, 2, 3)
 //   warp  14    UMMA issuer of the prep stream (G, W, U~)
 // Every wait on an mbarrier is bounded; on timeout the kernel sets
@@ -63,35 +63,37 @@ constexpr float G_FLOOR = -30.f;   // per-token log-decay floor (exp(-30) ~ 9e-1
 constexpr float LOG2E = 1.4426950408889634f;
 
 // ---- shared-memory map (bytes from a 1024-aligned base) ----
-constexpr uint32_t OFF_KQ0 = 0;          // [kb][128 rows: K 0-63, Q 64-127][128 B], 32 KB
-constexpr uint32_t OFF_KQ1 = 32768;
+constexpr int KQ_STAGES = 3;
+constexpr uint32_t OFF_KQ0 = 0;          // KQ_STAGES x [kb][128 rows: K 0-63, Q 64-127][128 B]
+constexpr uint32_t KQ_STAGE = 32768;     // bytes per KQ stage
 constexpr uint32_t KQ_KB = 16384;        // k-block (64 dk) stride inside a KQ stage
-constexpr uint32_t OFF_V = 65536;        // [dv half][64 rows j][128 B], 16 KB
+constexpr uint32_t OFF_V = 98304;        // [dv half][64 rows j][128 B], 16 KB
 constexpr uint32_t V_HALF = 8192;
-constexpr uint32_t OFF_SBF = 81920;      // [dk half][128 rows dv][128 B], 32 KB
-constexpr uint32_t SBF_KB = 16384;
 constexpr uint32_t OFF_WNEG = 114688;    // [128 rows dk][64 i], 16 KB (MN-major B); also the output staging tile
 constexpr uint32_t OFF_P0 = 131072;      // [64 rows i][64 j], 8 KB
 constexpr uint32_t OFF_P1 = 139264;
 constexpr uint32_t OFF_TB = 147456;      // [64 rows i][64 j], 8 KB
 constexpr uint32_t OFF_TBG = 155648;
-constexpr uint32_t OFF_SOLVE = 163840;   // 16 blocks of 16 x 20 fp32
 constexpr uint32_t SOLVE_LD = 20;        // padded row stride (floats)
 constexpr uint32_t SOLVE_BLK = 16 * SOLVE_LD;  // floats per block
-constexpr uint32_t OFF_GB0 = OFF_SOLVE + 16 * SOLVE_BLK * 4;   // g tile 1 KB + beta tile 1 KB
-constexpr uint32_t OFF_GB1 = OFF_GB0 + 2048;
+constexpr uint32_t SOLVE_BYTES = 16 * SOLVE_BLK * 4;
+constexpr uint32_t OFF_SOLVE0 = 163840;  // two areas of 16 blocks of 16 x 20 fp32
+constexpr uint32_t OFF_SOLVE1 = OFF_SOLVE0 + SOLVE_BYTES;
+constexpr uint32_t OFF_GB0 = OFF_SOLVE1 + SOLVE_BYTES;         // KQ_STAGES x (g tile 1 KB + beta tile 1 KB)
 constexpr uint32_t GATE_BYTES = 2560;
-constexpr uint32_t OFF_GATE0 = OFF_GB1 + 2048;                 // processed gates
+constexpr uint32_t OFF_GATE0 = OFF_GB0 + KQ_STAGES * 2048;     // processed gates
 constexpr uint32_t OFF_GATE1 = OFF_GATE0 + GATE_BYTES;
 constexpr uint32_t OFF_UNITS = OFF_GATE1 + GATE_BYTES;         // int4 x MAX_UNITS
 constexpr uint32_t OFF_BARS = OFF_UNITS + MAX_UNITS * 16;
-constexpr uint32_t NUM_BARS = 21;
+constexpr uint32_t NUM_BARS = 29;
+static_assert(NUM_BARS * 8 <= 256, "barrier area");
 constexpr uint32_t OFF_MISC = OFF_BARS + 256;                  // tmem base, abort flag, count
 constexpr uint32_t OFF_OGR = OFF_MISC + 64;                    // Gamma_i rq_i for the outputs, 64 floats
 constexpr uint32_t SMEM_USED = OFF_OGR + 256;
 constexpr uint32_t SMEM_BYTES = SMEM_USED + 1024;              // + alignment slack
 static_assert(SMEM_BYTES <= 232448, "shared memory budget");
-static_assert(OFF_GB0 % 1024 == 0, "alignment");
+static_assert(OFF_GB0 % 1024 == 0 && OFF_V % 1024 == 0 && OFF_WNEG % 1024 == 0 &&
+              OFF_KQ0 + KQ_STAGES * KQ_STAGE <= OFF_V && OFF_V + 16384 <= OFF_WNEG, "alignment");
 
 // gate-array offsets (floats) inside a GATE stage
 constexpr int GA_G2 = 0;       // G_i * log2(e)
@@ -108,14 +110,15 @@ static_assert((GA_BG + 64) * 4 <= (int)GATE_BYTES, "gate stage size");
 
 // barrier indices
 enum {
-    B_KQ_FULL = 0, B_KQ_EMPTY = 2, B_V_FULL = 4, B_V_EMPTY = 5, B_GATE_FULL = 6,
-    B_GATE_EMPTY = 8, B_G_DONE = 10, B_T_READY = 11, B_WU_DONE = 12, B_WNEG = 13,
-    B_S_READY = 14, B_U_DONE = 15, B_E1 = 16, B_S_DONE = 17, B_Z_DONE = 18, B_Y_FREE = 19,
-    B_G_FREE = 20
+    B_KQ_FULL = 0, B_KQ_EMPTY = 3, B_V_FULL = 6, B_V_EMPTY = 7, B_GATE_FULL = 8,
+    B_GATE_EMPTY = 10, B_G_DONE = 12, B_T_READY = 13, B_WU_DONE = 14, B_WNEG = 15,
+    B_S_READY = 16, B_U_DONE = 17, B_E1 = 18, B_S_DONE = 19, B_Z_DONE = 20, B_Y_FREE = 21,
+    B_G_FREE = 22, B_A_READY = 23, B_SOLVE_FREE = 25, B_P_FREE = 27, B_COUNT = 29
 };
+static_assert(B_COUNT == (int)NUM_BARS, "barrier count");
 
 // TMEM columns
-constexpr uint32_t TM_S = 0, TM_U = 128, TM_Y = 192, TM_Z = 256, TM_G = 320, TM_W = 384;
+constexpr uint32_t TM_S = 0, TM_U = 128, TM_Y = 192, TM_Z = 256, TM_G = 320, TM_W = 384, TM_SB = 448;
 
 struct __align__(64) Params {
     CUtensorMap tm_q;     // (128, Hq, N) bf16, box (64, 1, 64), 128B swizzle
@@ -218,7 +221,10 @@ __device__ __forceinline__ void st4(float *p, float a, float b, float c, float d
 // goes to CTA (u mod G) on even waves and G-1-(u mod G) on odd waves.
 __device__ void build_unit_list(const Params &p, uint8_t *smem, int batch0, int *count_out)
 {
-    int *ord = reinterpret_cast<int *>(smem + OFF_SBF);   // scratch: up to 8192 ints
+    // scratch for up to 8192 ints: the two solve areas, idle between batches and written by
+    // generic stores only (a TMA destination here would need a proxy fence before its next load)
+    static_assert(2 * SOLVE_BYTES >= 8192 * 4 && OFF_SOLVE1 == OFF_SOLVE0 + SOLVE_BYTES, "unit scratch");
+    int *ord = reinterpret_cast<int *>(smem + OFF_SOLVE0);
     const int B = p.B;
     const int tid = threadIdx.x;
     const bool sorted = B <= 8192;
@@ -351,24 +357,26 @@ __device__ __forceinline__ int t_slot(int I, int J)
 
 // Row i of A (TMEM quadrants 0-1: beta_i (k^_i . k^_j) exp(G_i - G_j) for j < i, fp32
 // into the solve blocks) or of P (quadrants 2-3: (q^_i . k^_j) exp(G_i - G_j) for
-// j <= i, bf16 tile), read 16 Gram columns at a time from TMEM; half hh of the
-// prep threads covers column blocks 2hh and 2hh+1.  The exponent of an
-// earlier block J is split as exp(G_i - Gend_J) exp(Gend_J - G_j), both <= 1.
-__device__ __forceinline__ void build_row(uint32_t tl_gram, int qd, int hh, const float *ga,
-                                          float *solve, uint8_t *ptile)
+// j <= i, bf16 tile), read 16 Gram columns at a time from TMEM.  Blocks right of the
+// row's diagonal block are zero: never stored for A, zero from the start in P.  The
+// exponent of an earlier block J is split as exp(G_i - Gend_J) exp(Gend_J - G_j),
+// both <= 1.
+__device__ __forceinline__ void build_row(uint32_t tl_gram, int qd, const float *ga, float *solve,
+                                          uint8_t *ptile)
 {
     const int lane = threadIdx.x & 31;
     const bool isP = qd >= 2;
     const int r = lane & 15;
     const int I = 2 * (qd & 1) + (lane >> 4);
     const int i = 16 * I + r;
+    const int jmax = 2 * (qd & 1) + 1;   // last diagonal block among the warp's rows
     const float G2i = ga[GA_G2 + i];
     const float rowscale = isP ? ga[GA_RQ + i] : ga[GA_BETA + i] * ga[GA_RK + i];
     float gend[3];
 #pragma unroll
     for (int J = 0; J < 3; ++J) gend[J] = ga[GA_GEND + J];
 #pragma unroll 1
-    for (int J = 2 * hh; J < 2 * hh + 2; ++J) {
+    for (int J = 0; J <= jmax; ++J) {
         // ---- loads (TMEM Gram columns, gate factors) before any store of this block
         float x[16], cf[16], g2[16], rk[16];
         tmem_ld16(tl_gram + 16 * J, x);
@@ -382,12 +390,13 @@ __device__ __forceinline__ void build_row(uint32_t tl_gram, int qd, int hh, cons
             rk[4 * q] = c.x; rk[4 * q + 1] = c.y; rk[4 * q + 2] = c.z; rk[4 * q + 3] = c.w;
         }
         tmem_wait_ld();
+        if (J > I) continue;
         // ---- compute
         if (J < I) {
             const float f = ex2_approx(G2i - (J == 0 ? gend[0] : (J == 1 ? gend[1] : gend[2]))) * rowscale;
 #pragma unroll
             for (int jj = 0; jj < 16; ++jj) x[jj] *= f * cf[jj] * rk[jj];
-        } else if (J == I) {
+        } else {
             // branch-free: every lane evaluates all 16 factors, then masks
             const int lim = isP ? r + 1 : r;
 #pragma unroll
@@ -395,15 +404,12 @@ __device__ __forceinline__ void build_row(uint32_t tl_gram, int qd, int hh, cons
                 const float e = ex2_approx(fminf(G2i - g2[jj], 0.f)) * rk[jj] * rowscale;
                 x[jj] = (jj < lim) ? x[jj] * e : 0.f;
             }
-        } else {
-#pragma unroll
-            for (int jj = 0; jj < 16; ++jj) x[jj] = 0.f;
         }
         // ---- stores
         if (isP) {
             *reinterpret_cast<uint4 *>(ptile + sw128(i, 2 * J)) = pack8_bf16(x);
             *reinterpret_cast<uint4 *>(ptile + sw128(i, 2 * J + 1)) = pack8_bf16(x + 8);
-        } else if (J <= I) {
+        } else {
             float *row = solve + (J == I ? I : a_slot(I, J)) * SOLVE_BLK + r * SOLVE_LD;
 #pragma unroll
             for (int q = 0; q < 4; ++q) st4(row + 4 * q, x[4 * q], x[4 * q + 1], x[4 * q + 2], x[4 * q + 3]);
@@ -451,9 +457,10 @@ __global__ void __launch_bounds__(NTHREADS, 1) gdn_prefill_chunk_kernel(const __
         tmem_alloc(sbase + OFF_MISC, 512);
         tmem_relinquish();
     }
-    // T tiles: only the blocks on and below the diagonal are ever written
-    for (int i = tid; i < 16384 / 16; i += NTHREADS)
-        reinterpret_cast<uint4 *>(smem + OFF_TB)[i] = make_uint4(0u, 0u, 0u, 0u);
+    // P and T tiles: only the blocks on and below the diagonal are ever written
+    static_assert(OFF_P1 == OFF_P0 + 8192 && OFF_TB == OFF_P1 + 8192 && OFF_TBG == OFF_TB + 8192, "tile order");
+    for (int i = tid; i < 32768 / 16; i += NTHREADS)
+        reinterpret_cast<uint4 *>(smem + OFF_P0)[i] = make_uint4(0u, 0u, 0u, 0u);
     fence_proxy_async_smem();
     tc_fence_before();
     __syncthreads();
@@ -461,10 +468,12 @@ __global__ void __launch_bounds__(NTHREADS, 1) gdn_prefill_chunk_kernel(const __
     const uint32_t tmem = *tmem_slot;
 
     // per-role pipeline counters (persist across units and batches)
-    uint32_t kq_use[2] = {0, 0}, v_use = 0;                          // TMA
+    uint32_t kq_use[KQ_STAGES] = {}, v_use = 0;               // TMA
     uint32_t c_wneg = 0, c_s = 0, c_y = 0, c_e1 = 0;                 // chain issuer
-    uint32_t q_kq[2] = {0, 0}, q_t = 0, q_v = 0, q_wu = 0, q_g = 0;   // prep-stream issuer
-    uint32_t p_kq[2] = {0, 0}, p_gate_empty[2] = {0, 0}, p_g = 0, p_wu = 0;   // prep
+    uint32_t q_kq[KQ_STAGES] = {}, q_t = 0, q_v = 0, q_wu = 0, q_g = 0;   // prep-stream issuer
+    uint32_t p_kq[KQ_STAGES] = {}, p_gate_empty[2] = {0, 0}, p_g = 0, p_sf[2] = {0, 0};   // prep front
+    uint32_t p_pf[2] = {0, 0};
+    uint32_t p_ar[2] = {0, 0}, p_wu = 0;                              // prep back
     uint32_t s_u = 0, s_sd = 0, s_zd = 0, s_wu = 0, s_gate[2] = {0, 0};   // state
     uint32_t gc = 0;   // global chunk counter (same sequence in every role)
 
@@ -497,19 +506,20 @@ __global__ void __launch_bounds__(NTHREADS, 1) gdn_prefill_chunk_kernel(const __
                     const int qh = (int)(((int64_t)un.h * p.Hq) / p.Hv);
                     const int nc = (un.len + C - 1) / C;
                     for (int n = 0; n < nc; ++n) {
-                        const uint32_t s = (gc + n) & 1;
-                        if (kq_use[s] > 0 && !cx.wait(B_KQ_EMPTY + s, (kq_use[s] - 1) & 1)) break;
-                        ++kq_use[s];
-                        const uint32_t kq = sbase + (s ? OFF_KQ1 : OFF_KQ0);
-                        const uint32_t gb = sbase + (s ? OFF_GB1 : OFF_GB0);
+                        const uint32_t ks = (gc + n) % KQ_STAGES;
+                        if (kq_use[ks] > 0 && !cx.wait(B_KQ_EMPTY + ks, (kq_use[ks] - 1) & 1)) break;
+                        ++kq_use[ks];
+                        const uint32_t kq = sbase + OFF_KQ0 + ks * KQ_STAGE;
+                        const uint32_t gb = sbase + OFF_GB0 + ks * 2048;
                         const int t0 = un.start + n * C;
-                        mbar_arrive_expect_tx(cx.bar(B_KQ_FULL + s), 32768 + 2048);
-                        tma_load_3d(kq, &p.tm_k, cx.bar(B_KQ_FULL + s), 0, qh, t0);
-                        tma_load_3d(kq + KQ_KB, &p.tm_k, cx.bar(B_KQ_FULL + s), 64, qh, t0);
-                        tma_load_3d(kq + 8192, &p.tm_q, cx.bar(B_KQ_FULL + s), 0, qh, t0);
-                        tma_load_3d(kq + KQ_KB + 8192, &p.tm_q, cx.bar(B_KQ_FULL + s), 64, qh, t0);
-                        tma_load_2d(gb, &p.tm_g, cx.bar(B_KQ_FULL + s), un.h & ~3, t0);
-                        tma_load_2d(gb + 1024, &p.tm_beta, cx.bar(B_KQ_FULL + s), un.h & ~3, t0);
+                        const uint32_t kb = cx.bar(B_KQ_FULL + ks);
+                        mbar_arrive_expect_tx(kb, 32768 + 2048);
+                        tma_load_3d(kq, &p.tm_k, kb, 0, qh, t0);
+                        tma_load_3d(kq + KQ_KB, &p.tm_k, kb, 64, qh, t0);
+                        tma_load_3d(kq + 8192, &p.tm_q, kb, 0, qh, t0);
+                        tma_load_3d(kq + KQ_KB + 8192, &p.tm_q, kb, 64, qh, t0);
+                        tma_load_2d(gb, &p.tm_g, kb, un.h & ~3, t0);
+                        tma_load_2d(gb + 1024, &p.tm_beta, kb, un.h & ~3, t0);
                         if (v_use > 0 && !cx.wait(B_V_EMPTY, (v_use - 1) & 1)) break;
                         ++v_use;
                         mbar_arrive_expect_tx(cx.bar(B_V_FULL), 16384);
@@ -554,10 +564,9 @@ __global__ void __launch_bounds__(NTHREADS, 1) gdn_prefill_chunk_kernel(const __
                 constexpr uint32_t ID_2 = idesc_bf16(128, 128, 0, 1);
                 constexpr uint32_t ID_3 = idesc_bf16(128, 64, 0, 0);
                 // descriptor bases; a byte offset `o` inside a tile is added as (o >> 4)
-                const uint64_t dKQk0 = sdesc_sw128(sbase + OFF_KQ0, 16, 1024);      // K-major
-                const uint64_t dKQk1 = sdesc_sw128(sbase + OFF_KQ1, 16, 1024);
-                const uint64_t dKQm0 = sdesc_sw128(sbase + OFF_KQ0, KQ_KB, 1024);   // MN-major K
-                const uint64_t dKQm1 = sdesc_sw128(sbase + OFF_KQ1, KQ_KB, 1024);
+                // KQ stage ks starts (ks * KQ_STAGE) >> 4 descriptor units after stage 0
+                const uint64_t dKQk = sdesc_sw128(sbase + OFF_KQ0, 16, 1024);      // K-major
+                const uint64_t dKQm = sdesc_sw128(sbase + OFF_KQ0, KQ_KB, 1024);   // MN-major K
                 bool ok = true;
                 if (warp == ISSUE_WARP) {
                     const uint64_t dV = sdesc_sw128(sbase + OFF_V, V_HALF, 1024);
@@ -578,7 +587,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) gdn_prefill_chunk_kernel(const __
                         while (wi < nc) {
                             bool did = false;
                             if (gi < nc && gi <= wi + 1) {
-                                const uint32_t sg = (gc + gi) & 1;
+                                const uint32_t sg = (gc + gi) % KQ_STAGES;
                                 if ((q_g == 0 || mbar_test_wait(cx.bar(B_G_FREE), (q_g - 1) & 1)) &&
                                     mbar_test_wait(cx.bar(B_KQ_FULL + sg), q_kq[sg] & 1)) {
                                     ++q_g;
@@ -588,7 +597,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) gdn_prefill_chunk_kernel(const __
 #pragma unroll 1
                                     for (int kk = 0; kk < 8; ++kk) {
                                         const uint32_t o = ((kk >> 2) * KQ_KB + (kk & 3) * 32) >> 4;
-                                        const uint64_t d = (sg ? dKQk1 : dKQk0) + o;
+                                        const uint64_t d = dKQk + ((sg * KQ_STAGE) >> 4) + o;
                                         umma_bf16(tmem + TM_G, d, d, ID_G, kk > 0);
                                     }
                                     umma_commit(cx.bar(B_G_DONE));
@@ -603,13 +612,13 @@ __global__ void __launch_bounds__(NTHREADS, 1) gdn_prefill_chunk_kernel(const __
                                 ++q_t;
                                 ++q_v;
                                 ++q_wu;
-                                const uint32_t s = (gc + wi) & 1;
+                                const uint32_t ks = (gc + wi) % KQ_STAGES;
                                 tc_fence_after();
                                 // (W): W^T[dk][i] = sum_j K[j][dk] Tbg[i][j]; A = K (MN-major), B = Tbg
                                 // (U~): U^T[dv][i] = sum_j V[j][dv] Tb[i][j]; A = V (MN-major), B = Tb
 #pragma unroll 1
                                 for (int kk = 0; kk < 4; ++kk) {
-                                    umma_bf16(tmem + TM_W, (s ? dKQm1 : dKQm0) + ((kk * 2048) >> 4), dTBG + ((kk * 32) >> 4), ID_W, kk > 0);
+                                    umma_bf16(tmem + TM_W, dKQm + ((ks * KQ_STAGE + kk * 2048) >> 4), dTBG + ((kk * 32) >> 4), ID_W, kk > 0);
                                     umma_bf16(tmem + TM_U, dV + ((kk * 2048) >> 4), dTB + ((kk * 32) >> 4), ID_U, kk > 0);
                                 }
                                 umma_commit(cx.bar(B_WU_DONE));
@@ -633,7 +642,6 @@ __global__ void __launch_bounds__(NTHREADS, 1) gdn_prefill_chunk_kernel(const __
                         gc += nc;
                     }
                 } else {
-                    const uint64_t dSBF = sdesc_sw128(sbase + OFF_SBF, 16, 1024);
                     const uint64_t dWNEG = sdesc_sw128(sbase + OFF_WNEG, 8192, 1024);
                     const uint64_t dP0 = sdesc_sw128(sbase + OFF_P0, 16, 1024);
                     const uint64_t dP1 = sdesc_sw128(sbase + OFF_P1, 16, 1024);
@@ -642,7 +650,9 @@ __global__ void __launch_bounds__(NTHREADS, 1) gdn_prefill_chunk_kernel(const __
                         const int nc = (un.len + C - 1) / C;
                         for (int n = 0; n < nc && ok; ++n) {
                             const uint32_t s = (gc + n) & 1;
-                            // (1a) U^T += S^T (-W)^T
+                            const uint32_t ks = (gc + n) % KQ_STAGES;
+                            // (1a) U^T += S^T (-W)^T; the bf16 S^T is the TMEM A operand (8 columns
+                            //      per 16 dk)
                             ok = cx.wait(B_WNEG, c_wneg & 1);
                             ++c_wneg;
                             ok = ok && cx.wait(B_S_READY, c_s & 1);
@@ -650,10 +660,8 @@ __global__ void __launch_bounds__(NTHREADS, 1) gdn_prefill_chunk_kernel(const __
                             if (!ok) break;
                             tc_fence_after();
 #pragma unroll 1
-                            for (int kk = 0; kk < 8; ++kk) {
-                                const uint32_t ao = ((kk >> 2) * SBF_KB + (kk & 3) * 32) >> 4;
-                                umma_bf16(tmem + TM_U, dSBF + ao, dWNEG + ((kk * 2048) >> 4), ID_1A, 1);
-                            }
+                            for (int kk = 0; kk < 8; ++kk)
+                                umma_bf16_ts(tmem + TM_U, tmem + TM_SB + 8 * kk, dWNEG + ((kk * 2048) >> 4), ID_1A, 1);
                             umma_commit(cx.bar(B_U_DONE));
                             // (1b) Y = S^T Q^T, once the outputs of the previous chunk have read Y
                             if (c_y > 0) ok = cx.wait(B_Y_FREE, (c_y - 1) & 1);
@@ -662,9 +670,8 @@ __global__ void __launch_bounds__(NTHREADS, 1) gdn_prefill_chunk_kernel(const __
                             tc_fence_after();
 #pragma unroll 1
                             for (int kk = 0; kk < 8; ++kk) {
-                                const uint32_t ao = ((kk >> 2) * SBF_KB + (kk & 3) * 32) >> 4;
-                                const uint32_t bo = ((kk >> 2) * KQ_KB + 8192 + (kk & 3) * 32) >> 4;
-                                umma_bf16(tmem + TM_Y, dSBF + ao, (s ? dKQk1 : dKQk0) + bo, ID_1B, kk > 0);
+                                const uint32_t bo = (ks * KQ_STAGE + (kk >> 2) * KQ_KB + 8192 + (kk & 3) * 32) >> 4;
+                                umma_bf16_ts(tmem + TM_Y, tmem + TM_SB + 8 * kk, dKQk + bo, ID_1B, kk > 0);
                             }
                             // (2) S^T += Ud K, then (3) Z = U^T P^T
                             ok = cx.wait(B_E1, c_e1 & 1);
@@ -673,194 +680,213 @@ __global__ void __launch_bounds__(NTHREADS, 1) gdn_prefill_chunk_kernel(const __
                             tc_fence_after();
 #pragma unroll 1
                             for (int kk = 0; kk < 4; ++kk)
-                                umma_bf16_ts(tmem + TM_S, tmem + TM_U + 16 * kk + 8, (s ? dKQm1 : dKQm0) + ((kk * 2048) >> 4), ID_2, 1);
+                                umma_bf16_ts(tmem + TM_S, tmem + TM_U + 16 * kk + 8, dKQm + ((ks * KQ_STAGE + kk * 2048) >> 4), ID_2, 1);
                             umma_commit(cx.bar(B_S_DONE));
 #pragma unroll 1
                             for (int kk = 0; kk < 4; ++kk)
                                 umma_bf16_ts(tmem + TM_Z, tmem + TM_U + 16 * kk, (s ? dP1 : dP0) + ((kk * 32) >> 4), ID_3, kk > 0);
                             umma_commit(cx.bar(B_Z_DONE));
-                            umma_commit(cx.bar(B_KQ_EMPTY + s));
+                            umma_commit(cx.bar(B_P_FREE + s));
+                            umma_commit(cx.bar(B_KQ_EMPTY + ks));
                         }
                         gc += nc;
                     }
                 }
             }
         } else if (warp >= 4) {
-            // ------------------------------------------------------------ prep warpgroup
-            const int pt = tid - 128;           // 0..255
-            const int pw = pt >> 5;             // prep warp 0..7
-            const int qd = pw & 3;              // TMEM lane quadrant
-            const int hh = pw >> 2;             // half: which columns / which sub-task
-            const int tp = 32 * qd + lane;      // TMEM lane == row handled by this thread
-            const uint32_t tl = tmem + ((uint32_t)(32 * qd) << 16);
-            float *solve = reinterpret_cast<float *>(smem + OFF_SOLVE);
+            // ------------------------------------------------------------ prep warpgroups
+            // Two groups of four warps form a two-stage pipeline over consecutive chunks:
+            //   front (warps 4-7):  row norms, gates, A and P from the Gram (TMEM)
+            //   back  (warps 8-11): 16x16 diagonal inverses, block merges, bf16 T tiles
+            // A crosses in one of two solve areas (A_READY / SOLVE_FREE per area).
+            const int pg = (warp - 4) >> 2;          // 0 front, 1 back
+            const int lt = tid - 128 - 128 * pg;     // thread in the group, 0..127
+            const int pw = lt >> 5;                  // warp in the group == TMEM lane quadrant
+            const int tp = 32 * pw + lane;           // TMEM lane == row handled by this thread
+            const uint32_t tl = tmem + ((uint32_t)(32 * pw) << 16);
+            const int nbar = pg ? 3 : 1;             // the group's named barrier
             bool ok = true;
             for (int k = 0; k < nunits && ok; ++k) {
                 const Unit un = load_unit(smem, k);
                 const int nc = (un.len + C - 1) / C;
                 for (int n = 0; n < nc && ok; ++n) {
                     const uint32_t s = (gc + n) & 1;
-                    const int len_n = min(C, un.len - n * C);
-                    const uint8_t *kq = smem + (s ? OFF_KQ1 : OFF_KQ0);
-                    const float *gtile = reinterpret_cast<const float *>(smem + (s ? OFF_GB1 : OFF_GB0));
+                    float *solve = reinterpret_cast<float *>(smem + (s ? OFF_SOLVE1 : OFF_SOLVE0));
                     float *ga = reinterpret_cast<float *>(smem + (s ? OFF_GATE1 : OFF_GATE0));
-                    ok = cx.wait(B_KQ_FULL + s, p_kq[s] & 1);
-                    ++p_kq[s];
-                    if (p_gate_empty[s] > 0) ok = ok && cx.wait(B_GATE_EMPTY + s, (p_gate_empty[s] - 1) & 1);
-                    ++p_gate_empty[s];
-                    // --- row norms (K rows 0..63, Q rows 64..127, prep half 0), conflict-free chunk order
-                    if (hh == 0) {
-                        float rn = 1.f;
-                        if (p.qk_l2norm) {
-                            float ss = 0.f;
-#pragma unroll 2
-                            for (int c = 0; c < 8; ++c) {
-                                const uint32_t off = sw128(tp, c);
-                                const uint4 va = *reinterpret_cast<const uint4 *>(kq + off);
-                                const uint4 vb = *reinterpret_cast<const uint4 *>(kq + KQ_KB + off);
-                                ss += sumsq8_bf16(va) + sumsq8_bf16(vb);
-                            }
-                            rn = 1.0f / sqrtf(ss + 1e-12f);
-                        }
-                        ga[GA_RK + tp] = rn;   // GA_RQ = GA_RK + 64
-                    }
-                    // --- gates (prep warp 4, tokens 2l and 2l+1 per lane): floored, masked
-                    //     log-decay, inclusive prefix sum, exponentials
-                    if (pw == 4) {
-                        const int i0 = 2 * lane, i1 = i0 + 1;
-                        const int hc = un.h & 3;
-                        const float g0 = i0 < len_n ? fmaxf(gtile[i0 * 4 + hc], G_FLOOR) : 0.f;
-                        const float g1 = i1 < len_n ? fmaxf(gtile[i1 * 4 + hc], G_FLOOR) : 0.f;
-                        const float b0 = i0 < len_n ? gtile[256 + i0 * 4 + hc] : 0.f;
-                        const float b1 = i1 < len_n ? gtile[256 + i1 * 4 + hc] : 0.f;
-                        float x = g0 + g1;
+                    if (pg == 0) {
+                        const int len_n = min(C, un.len - n * C);
+                        const uint32_t ks = (gc + n) % KQ_STAGES;
+                        const uint8_t *kq = smem + OFF_KQ0 + ks * KQ_STAGE;
+                        const float *gtile = reinterpret_cast<const float *>(smem + OFF_GB0 + ks * 2048);
+                        ok = cx.wait(B_KQ_FULL + ks, p_kq[ks] & 1);
+                        ++p_kq[ks];
+                        if (p_gate_empty[s] > 0) ok = ok && cx.wait(B_GATE_EMPTY + s, (p_gate_empty[s] - 1) & 1);
+                        ++p_gate_empty[s];
+                        if (p_sf[s] > 0) ok = ok && cx.wait(B_SOLVE_FREE + s, (p_sf[s] - 1) & 1);
+                        ++p_sf[s];
+                        // --- row norms (K rows 0..63, Q rows 64..127), conflict-free chunk order
+                        {
+                            float rn = 1.f;
+                            if (p.qk_l2norm) {
+                                float ss = 0.f;
 #pragma unroll
-                        for (int o = 1; o < 32; o <<= 1) {
-                            const float y = __shfl_up_sync(0xffffffffu, x, o);
-                            if (lane >= o) x += y;
-                        }
-                        const float G2b = x * LOG2E;            // token i1
-                        const float G2a = (x - g1) * LOG2E;     // token i0
-                        const float gend = __shfl_sync(0xffffffffu, G2b, (lane & ~7) + 7);
-                        const float gcl = __shfl_sync(0xffffffffu, G2b, 31);
-                        *reinterpret_cast<float2 *>(ga + GA_G2 + i0) = make_float2(G2a, G2b);
-                        *reinterpret_cast<float2 *>(ga + GA_BETA + i0) = make_float2(b0, b1);
-                        *reinterpret_cast<float2 *>(ga + GA_CF + i0) =
-                            make_float2(ex2_approx(gend - G2a), ex2_approx(gend - G2b));
-                        *reinterpret_cast<float2 *>(ga + GA_GAM + i0) = make_float2(ex2_approx(G2a), ex2_approx(G2b));
-                        *reinterpret_cast<float2 *>(ga + GA_DEC + i0) =
-                            make_float2(ex2_approx(gcl - G2a), ex2_approx(gcl - G2b));
-                        if ((lane & 7) == 7) ga[GA_GEND + (lane >> 3)] = G2b;
-                        if (lane == 31) ga[GA_GC] = ex2_approx(G2b);
-                    }
-                    named_sync(1, 256);
-                    if (pt == 0) mbar_arrive(cx.bar(B_GATE_FULL + s));
-                    // --- Gram -> A (rows 0..63, fp32 blocks) and P (rows 64..127, bf16 tile)
-                    ok = ok && cx.wait(B_G_DONE, p_g & 1);
-                    ++p_g;
-                    tc_fence_after();
-                    {
-                        uint8_t *ptile = smem + (s ? OFF_P1 : OFF_P0);
-                        build_row(tl + TM_G, qd, hh, ga, solve, ptile);
-                        if (qd >= 2) fence_proxy_async_smem();
-                        if (pt < 64) ga[GA_BG + pt] = ga[GA_BETA + pt] * ga[GA_GAM + pt] * ga[GA_RK + pt];
-                    }
-                    tc_fence_before();
-                    named_sync(1, 256);
-                    if (pt == 0) mbar_arrive(cx.bar(B_G_FREE));
-                    // the T tiles of the previous chunk are read by its WU products
-                    if (p_wu > 0) ok = ok && cx.wait(B_WU_DONE, (p_wu - 1) & 1);
-                    ++p_wu;
-                    // --- diagonal 16x16 inverses D_I = (I + A_II)^-1 (threads 0..63, one column each)
-                    if (pt < 64) {
-                        const int I = pt >> 4, c = pt & 15;
-                        const float *Ab = solve + I * SOLVE_BLK;
-                        float x[16];
-#pragma unroll
-                        for (int r = 0; r < 16; ++r) {
-                            float a[16];
-#pragma unroll
-                            for (int q = 0; q < 4; ++q) {
-                                if (4 * q < r) {
-                                    const float4 v = ld4(Ab + r * SOLVE_LD + 4 * q);
-                                    a[4 * q] = v.x; a[4 * q + 1] = v.y; a[4 * q + 2] = v.z; a[4 * q + 3] = v.w;
+                                for (int c = 0; c < 8; ++c) {
+                                    const uint32_t off = sw128(tp, c);
+                                    const uint4 va = *reinterpret_cast<const uint4 *>(kq + off);
+                                    const uint4 vb = *reinterpret_cast<const uint4 *>(kq + KQ_KB + off);
+                                    ss += sumsq8_bf16(va) + sumsq8_bf16(vb);
                                 }
+                                rn = 1.0f / sqrtf(ss + 1e-12f);
                             }
-                            float acc0 = (r == c) ? 1.f : 0.f, acc1 = 0.f;
-#pragma unroll
-                            for (int m = 0; m < r; ++m) {
-                                if (m & 1) acc1 = fmaf(-a[m], x[m], acc1);
-                                else acc0 = fmaf(-a[m], x[m], acc0);
-                            }
-                            x[r] = acc0 + acc1;
+                            ga[GA_RK + tp] = rn;   // GA_RQ = GA_RK + 64
                         }
-                        float *Db = solve + (10 + I) * SOLVE_BLK;
+                        // --- gates (front warp 0, tokens 2l and 2l+1 per lane): floored, masked
+                        //     log-decay, inclusive prefix sum, exponentials
+                        if (pw == 0) {
+                            const int i0 = 2 * lane, i1 = i0 + 1;
+                            const int hc = un.h & 3;
+                            const float g0 = i0 < len_n ? fmaxf(gtile[i0 * 4 + hc], G_FLOOR) : 0.f;
+                            const float g1 = i1 < len_n ? fmaxf(gtile[i1 * 4 + hc], G_FLOOR) : 0.f;
+                            const float b0 = i0 < len_n ? gtile[256 + i0 * 4 + hc] : 0.f;
+                            const float b1 = i1 < len_n ? gtile[256 + i1 * 4 + hc] : 0.f;
+                            float x = g0 + g1;
 #pragma unroll
-                        for (int r = 0; r < 16; ++r) Db[r * SOLVE_LD + c] = x[r];
-                        const int j = 16 * I + c;
-                        const float bj = ga[GA_BETA + j], sj = ga[GA_BG + j];
-                        const uint32_t cw = (uint32_t)(j & 7) * 2u;
+                            for (int o = 1; o < 32; o <<= 1) {
+                                const float y = __shfl_up_sync(0xffffffffu, x, o);
+                                if (lane >= o) x += y;
+                            }
+                            const float G2b = x * LOG2E;            // token i1
+                            const float G2a = (x - g1) * LOG2E;     // token i0
+                            const float gend = __shfl_sync(0xffffffffu, G2b, (lane & ~7) + 7);
+                            const float gcl = __shfl_sync(0xffffffffu, G2b, 31);
+                            *reinterpret_cast<float2 *>(ga + GA_G2 + i0) = make_float2(G2a, G2b);
+                            *reinterpret_cast<float2 *>(ga + GA_BETA + i0) = make_float2(b0, b1);
+                            *reinterpret_cast<float2 *>(ga + GA_CF + i0) =
+                                make_float2(ex2_approx(gend - G2a), ex2_approx(gend - G2b));
+                            *reinterpret_cast<float2 *>(ga + GA_GAM + i0) = make_float2(ex2_approx(G2a), ex2_approx(G2b));
+                            *reinterpret_cast<float2 *>(ga + GA_DEC + i0) =
+                                make_float2(ex2_approx(gcl - G2a), ex2_approx(gcl - G2b));
+                            if ((lane & 7) == 7) ga[GA_GEND + (lane >> 3)] = G2b;
+                            if (lane == 31) ga[GA_GC] = ex2_approx(G2b);
+                        }
+                        named_sync(1, 128);
+                        if (lt == 0) mbar_arrive(cx.bar(B_GATE_FULL + s));
+                        // --- Gram -> A (rows 0..63, fp32 blocks) and P (rows 64..127, bf16 tile); the
+                        //     P tile of this parity is read by (3) of the chunk before last
+                        if (p_pf[s] > 0) ok = ok && cx.wait(B_P_FREE + s, (p_pf[s] - 1) & 1);
+                        ++p_pf[s];
+                        ok = ok && cx.wait(B_G_DONE, p_g & 1);
+                        ++p_g;
+                        tc_fence_after();
+                        build_row(tl + TM_G, pw, ga, solve, smem + (s ? OFF_P1 : OFF_P0));
+                        if (pw >= 2) fence_proxy_async_smem();
+                        if (lt < 64) ga[GA_BG + lt] = ga[GA_BETA + lt] * ga[GA_GAM + lt] * ga[GA_RK + lt];
+                        tc_fence_before();
+                        named_sync(1, 128);
+                        if (lt == 0) {
+                            mbar_arrive(cx.bar(B_G_FREE));
+                            mbar_arrive(cx.bar(B_A_READY + s));
+                        }
+                    } else {
+                        ok = cx.wait(B_A_READY + s, p_ar[s] & 1);
+                        ++p_ar[s];
+                        // the T tiles of the previous chunk are read by its WU products
+                        if (p_wu > 0) ok = ok && cx.wait(B_WU_DONE, (p_wu - 1) & 1);
+                        ++p_wu;
+                        // --- diagonal 16x16 inverses D_I = (I + A_II)^-1 (back threads 0..63, one column each)
+                        if (lt < 64) {
+                            const int I = lt >> 4, c = lt & 15;
+                            const float *Ab = solve + I * SOLVE_BLK;
+                            float x[16];
 #pragma unroll
-                        for (int r = 0; r < 16; ++r) {
-                            const uint32_t off = sw128(16 * I + r, j >> 3) + cw;
-                            *reinterpret_cast<__nv_bfloat16 *>(smem + OFF_TB + off) = __float2bfloat16_rn(x[r] * bj);
-                            *reinterpret_cast<__nv_bfloat16 *>(smem + OFF_TBG + off) = __float2bfloat16_rn(x[r] * sj);
-                        }
-                    }
-                    named_sync(1, 256);
-                    // --- block merges (warp-level tf32 products):
-                    //   L1: T_10 = -D_1 (A_10 D_0) (warp 0), T_32 = -D_3 (A_32 D_2) (warp 1)
-                    //   X : X_pq = (A_BA T_AA)_pq -> slot 2p+q (the dead A_II blocks)
-                    //   TB: T_{2+p,q} = -(T_BB X)_pq -> slot 6+2p+q (the dead A_BA blocks)
-                    if (pw < 2) {
-                        float *tmp = solve + (pw ? 15 : 14) * SOLVE_BLK;
-                        float acc[2][4] = {};
-                        blk_mma(acc, solve + (pw ? 5 : 4) * SOLVE_BLK, solve + (pw ? 12 : 10) * SOLVE_BLK);
-                        blk_store(tmp, acc, 1.f);
-                        __syncwarp();
-                        float acc2[2][4] = {};
-                        blk_mma(acc2, solve + (pw ? 13 : 11) * SOLVE_BLK, tmp);
-                        __syncwarp();
-                        blk_store(tmp, acc2, -1.f);
-                        blk_store_tiles(acc2, -1.f, pw ? 3 : 1, pw ? 2 : 0, ga, smem + OFF_TB, smem + OFF_TBG);
-                    }
-                    named_sync(1, 256);
-#pragma unroll 1
-                    for (int ph = 0; ph < 2; ++ph) {
-                        const int pp = (pw >> 1) & 1, q = pw & 1;
-                        const float *X0, *Y0, *X1 = nullptr, *Y1 = nullptr;
-                        int dst;
-                        float sgn;
-                        if (ph == 0) {
-                            if (q == 0) {
-                                X0 = solve + a_slot(2 + pp, 0) * SOLVE_BLK; Y0 = solve + 10 * SOLVE_BLK;
-                                X1 = solve + a_slot(2 + pp, 1) * SOLVE_BLK; Y1 = solve + 14 * SOLVE_BLK;
-                            } else {
-                                X0 = solve + a_slot(2 + pp, 1) * SOLVE_BLK; Y0 = solve + 11 * SOLVE_BLK;
+                            for (int r = 0; r < 16; ++r) {
+                                float a[16];
+#pragma unroll
+                                for (int q = 0; q < 4; ++q) {
+                                    if (4 * q < r) {
+                                        const float4 v = ld4(Ab + r * SOLVE_LD + 4 * q);
+                                        a[4 * q] = v.x; a[4 * q + 1] = v.y; a[4 * q + 2] = v.z; a[4 * q + 3] = v.w;
+                                    }
+                                }
+                                float acc0 = (r == c) ? 1.f : 0.f, acc1 = 0.f;
+#pragma unroll
+                                for (int m = 0; m < r; ++m) {
+                                    if (m & 1) acc1 = fmaf(-a[m], x[m], acc1);
+                                    else acc0 = fmaf(-a[m], x[m], acc0);
+                                }
+                                x[r] = acc0 + acc1;
                             }
-                            dst = 2 * pp + q; sgn = 1.f;
-                        } else {
-                            if (pp == 0) {
-                                X0 = solve + 12 * SOLVE_BLK; Y0 = solve + q * SOLVE_BLK;
-                            } else {
-                                X0 = solve + 15 * SOLVE_BLK; Y0 = solve + q * SOLVE_BLK;
-                                X1 = solve + 13 * SOLVE_BLK; Y1 = solve + (2 + q) * SOLVE_BLK;
+                            float *Db = solve + (10 + I) * SOLVE_BLK;
+#pragma unroll
+                            for (int r = 0; r < 16; ++r) Db[r * SOLVE_LD + c] = x[r];
+                            const int j = 16 * I + c;
+                            const float bj = ga[GA_BETA + j], sj = ga[GA_BG + j];
+                            const uint32_t cw = (uint32_t)(j & 7) * 2u;
+#pragma unroll
+                            for (int r = 0; r < 16; ++r) {
+                                const uint32_t off = sw128(16 * I + r, j >> 3) + cw;
+                                *reinterpret_cast<__nv_bfloat16 *>(smem + OFF_TB + off) = __float2bfloat16_rn(x[r] * bj);
+                                *reinterpret_cast<__nv_bfloat16 *>(smem + OFF_TBG + off) = __float2bfloat16_rn(x[r] * sj);
                             }
-                            dst = 6 + 2 * pp + q; sgn = -1.f;
                         }
-                        if (pw < 4) {
+                        named_sync(3, 128);
+                        // --- block merges (warp-level tf32 products):
+                        //   L1: T_10 = -D_1 (A_10 D_0) (warp 0), T_32 = -D_3 (A_32 D_2) (warp 1)
+                        //   X : X_pq = (A_BA T_AA)_pq -> slot 2p+q (the dead A_II blocks)
+                        //   TB: T_{2+p,q} = -(T_BB X)_pq -> slot 6+2p+q (the dead A_BA blocks)
+                        if (pw < 2) {
+                            float *tmp = solve + (pw ? 15 : 14) * SOLVE_BLK;
                             float acc[2][4] = {};
-                            const int np = X1 ? 2 : 1;
-#pragma unroll 1
-                            for (int t = 0; t < np; ++t) blk_mma(acc, t ? X1 : X0, t ? Y1 : Y0);
-                            if (ph == 0) blk_store(solve + dst * SOLVE_BLK, acc, sgn);
-                            else blk_store_tiles(acc, sgn, 2 + pp, q, ga, smem + OFF_TB, smem + OFF_TBG);
+                            blk_mma(acc, solve + (pw ? 5 : 4) * SOLVE_BLK, solve + (pw ? 12 : 10) * SOLVE_BLK);
+                            blk_store(tmp, acc, 1.f);
+                            __syncwarp();
+                            float acc2[2][4] = {};
+                            blk_mma(acc2, solve + (pw ? 13 : 11) * SOLVE_BLK, tmp);
+                            __syncwarp();
+                            blk_store(tmp, acc2, -1.f);
+                            blk_store_tiles(acc2, -1.f, pw ? 3 : 1, pw ? 2 : 0, ga, smem + OFF_TB, smem + OFF_TBG);
                         }
-                        if (ph == 1) fence_proxy_async_smem();   // T tiles -> UMMA operands
-                        named_sync(1, 256);
+                        named_sync(3, 128);
+#pragma unroll 1
+                        for (int ph = 0; ph < 2; ++ph) {
+                            const int pp = (pw >> 1) & 1, q = pw & 1;
+                            const float *X0, *Y0, *X1 = nullptr, *Y1 = nullptr;
+                            int dst;
+                            float sgn;
+                            if (ph == 0) {
+                                if (q == 0) {
+                                    X0 = solve + a_slot(2 + pp, 0) * SOLVE_BLK; Y0 = solve + 10 * SOLVE_BLK;
+                                    X1 = solve + a_slot(2 + pp, 1) * SOLVE_BLK; Y1 = solve + 14 * SOLVE_BLK;
+                                } else {
+                                    X0 = solve + a_slot(2 + pp, 1) * SOLVE_BLK; Y0 = solve + 11 * SOLVE_BLK;
+                                }
+                                dst = 2 * pp + q; sgn = 1.f;
+                            } else {
+                                if (pp == 0) {
+                                    X0 = solve + 12 * SOLVE_BLK; Y0 = solve + q * SOLVE_BLK;
+                                } else {
+                                    X0 = solve + 15 * SOLVE_BLK; Y0 = solve + q * SOLVE_BLK;
+                                    X1 = solve + 13 * SOLVE_BLK; Y1 = solve + (2 + q) * SOLVE_BLK;
+                                }
+                                dst = 6 + 2 * pp + q; sgn = -1.f;
+                            }
+                            {
+                                float acc[2][4] = {};
+                                const int np = X1 ? 2 : 1;
+#pragma unroll 1
+                                for (int t = 0; t < np; ++t) blk_mma(acc, t ? X1 : X0, t ? Y1 : Y0);
+                                if (ph == 0) blk_store(solve + dst * SOLVE_BLK, acc, sgn);
+                                else blk_store_tiles(acc, sgn, 2 + pp, q, ga, smem + OFF_TB, smem + OFF_TBG);
+                            }
+                            if (ph == 1) fence_proxy_async_smem();   // T tiles -> UMMA operands
+                            named_sync(3, 128);
+                        }
+                        if (lt == 0) {
+                            mbar_arrive(cx.bar(B_T_READY));
+                            mbar_arrive(cx.bar(B_SOLVE_FREE + s));
+                        }
                     }
-                    if (pt == 0) mbar_arrive(cx.bar(B_T_READY));
-                    ok = !named_sync_or(1, 256, !ok || cx.aborted());
+                    ok = !named_sync_or(nbar, 128, !ok || cx.aborted());
                 }
                 gc += nc;
             }
@@ -884,7 +910,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) gdn_prefill_chunk_kernel(const __
                     continue;
                 }
                 bool ok = true;
-                // unit start: S0 -> bf16 tile and gC(0) * S0 -> TMEM
+                // unit start: S0 -> bf16 operand columns and gC(0) * S0 -> TMEM
                 {
                     const uint32_t s = gc & 1;
                     ok = cx.wait(B_GATE_FULL + s, s_gate[s] & 1);
@@ -899,15 +925,15 @@ __global__ void __launch_bounds__(NTHREADS, 1) gdn_prefill_chunk_kernel(const __
                             const float4 v = init ? ld4(init + 16 * q + c) : make_float4(0.f, 0.f, 0.f, 0.f);
                             x[c] = v.x; x[c + 1] = v.y; x[c + 2] = v.z; x[c + 3] = v.w;
                         }
-                        uint8_t *srow = smem + OFF_SBF + (q >> 2) * SBF_KB;
-                        *reinterpret_cast<uint4 *>(srow + sw128(dv, 2 * (q & 3))) = pack8_bf16(x);
-                        *reinterpret_cast<uint4 *>(srow + sw128(dv, 2 * (q & 3) + 1)) = pack8_bf16(x + 8);
+                        uint32_t w[8];
+#pragma unroll
+                        for (int e = 0; e < 8; ++e) w[e] = gdn::pack_bf16x2(x[2 * e], x[2 * e + 1]);
+                        tmem_st8u(tl + TM_SB + 8 * q, w);
 #pragma unroll
                         for (int e = 0; e < 16; ++e) x[e] *= gC;
                         tmem_st16(tl + TM_S + 16 * q, x);
                     }
                     tmem_wait_st();
-                    fence_proxy_async_smem();
                     tc_fence_before();
                     ok = !named_sync_or(2, 128, !ok || cx.aborted());
                     if (dv == 0 && ok) mbar_arrive(cx.bar(B_S_READY));
@@ -974,7 +1000,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) gdn_prefill_chunk_kernel(const __
                         mbar_arrive(cx.bar(B_E1));
                         mbar_arrive(cx.bar(B_GATE_EMPTY + s));   // the outputs read ogr from here on
                     }
-                    // ---- E2: new state -> bf16 tile (+ decay of the next chunk) or final state
+                    // ---- E2: new state -> bf16 operand columns (+ decay of the next chunk) or final state
                     ok = ok && cx.wait(B_S_DONE, s_sd & 1);
                     ++s_sd;
                     tc_fence_after();
@@ -991,9 +1017,10 @@ __global__ void __launch_bounds__(NTHREADS, 1) gdn_prefill_chunk_kernel(const __
                         tmem_ld16(tl + TM_S + 16 * q, x);
                         tmem_wait_ld();
                         if (more) {
-                            uint8_t *srow = smem + OFF_SBF + (q >> 2) * SBF_KB;
-                            *reinterpret_cast<uint4 *>(srow + sw128(dv, 2 * (q & 3))) = pack8_bf16(x);
-                            *reinterpret_cast<uint4 *>(srow + sw128(dv, 2 * (q & 3) + 1)) = pack8_bf16(x + 8);
+                            uint32_t w[8];
+#pragma unroll
+                            for (int e = 0; e < 8; ++e) w[e] = gdn::pack_bf16x2(x[2 * e], x[2 * e + 1]);
+                            tmem_st8u(tl + TM_SB + 8 * q, w);
 #pragma unroll
                             for (int e = 0; e < 16; ++e) x[e] *= gC1;
                             tmem_st16(tl + TM_S + 16 * q, x);
@@ -1004,7 +1031,6 @@ __global__ void __launch_bounds__(NTHREADS, 1) gdn_prefill_chunk_kernel(const __
                     }
                     if (more) {
                         tmem_wait_st();
-                        fence_proxy_async_smem();
                         tc_fence_before();
                         named_sync(2, 128);
                         if (dv == 0) mbar_arrive(cx.bar(B_S_READY));
@@ -1080,7 +1106,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) gdn_prefill_chunk_kernel(const __
 
     // teardown: drain outstanding TMA stages on abort, then free TMEM
     if (cx.aborted() && warp == TMA_WARP && lane == 0) {
-        for (int s = 0; s < 2; ++s) {
+        for (int s = 0; s < KQ_STAGES; ++s) {
             const long long t0 = clock64();
             while (kq_use[s] > 0 && !mbar_try_wait(cx.bar(B_KQ_FULL + s), (kq_use[s] - 1) & 1))
                 if (clock64() - t0 > (1ll << 31)) break;
