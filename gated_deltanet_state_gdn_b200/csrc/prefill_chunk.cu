@@ -38,7 +38,7 @@
 //   warps 4-7   prep front: row norms, gates, Gram -> A and P
 //   warps 8-11  prep back: the 64x64 unit-triangular solve and the bf16 T tiles
 //               (front and back work on consecutive chunks, ahead of the state chain)
-//   warp  12    TMA producer (q/k/g/beta tiles in three stages, v tiles in one)
+//   warp  12    TMA producers (lane 0: q/k/g/beta tiles in three stages; lane 1: v tiles)
 //   warp  13    TMEM owner; UMMA issuer of the state chain (1a, 1b, 2, 3)
 //   warp  14    UMMA issuer of the prep stream (G, W, U~)
 // Every wait on an mbarrier is bounded; on timeout the kernel sets
@@ -57,7 +57,7 @@ namespace gdn_chunk {
 constexpr int C = 64;       // chunk length (tokens)
 constexpr int D = 128;      // Dk = Dv
 constexpr int NTHREADS = 480;
-constexpr int MAX_UNITS = 128;     // per CTA per batch of the unit list
+constexpr int MAX_UNITS = 64;      // per CTA per batch of the unit list
 constexpr int TMA_WARP = 12, MMA_WARP = 13, ISSUE_WARP = 14;   // warps 0-3 state, 4-11 prep
 constexpr float G_FLOOR = -30.f;   // per-token log-decay floor (exp(-30) ~ 9e-14)
 constexpr float LOG2E = 1.4426950408889634f;
@@ -69,30 +69,30 @@ constexpr uint32_t KQ_STAGE = 32768;     // bytes per KQ stage
 constexpr uint32_t KQ_KB = 16384;        // k-block (64 dk) stride inside a KQ stage
 constexpr uint32_t OFF_V = 98304;        // [dv half][64 rows j][128 B], 16 KB
 constexpr uint32_t V_HALF = 8192;
-constexpr uint32_t OFF_WNEG = 114688;    // [128 rows dk][64 i], 16 KB (MN-major B); also the output staging tile
-constexpr uint32_t OFF_P0 = 131072;      // [64 rows i][64 j], 8 KB
-constexpr uint32_t OFF_P1 = 139264;
-constexpr uint32_t OFF_TB = 147456;      // [64 rows i][64 j], 8 KB
-constexpr uint32_t OFF_TBG = 155648;
+constexpr uint32_t OFF_WNEG = 114688;    // [128 rows dk][64 i], 16 KB (MN-major B)
+constexpr uint32_t OFF_P = 131072;       // KQ_STAGES x [64 rows i][64 j], 8 KB (stage = KQ stage)
+constexpr uint32_t P_STAGE = 8192;
+constexpr uint32_t OFF_TB = OFF_P + KQ_STAGES * P_STAGE;   // [64 rows i][64 j], 8 KB
+constexpr uint32_t OFF_TBG = OFF_TB + 8192;
 constexpr uint32_t SOLVE_LD = 20;        // padded row stride (floats)
 constexpr uint32_t SOLVE_BLK = 16 * SOLVE_LD;  // floats per block
 constexpr uint32_t SOLVE_BYTES = 16 * SOLVE_BLK * 4;
-constexpr uint32_t OFF_SOLVE0 = 163840;  // two areas of 16 blocks of 16 x 20 fp32
+constexpr uint32_t OFF_SOLVE0 = OFF_TBG + 8192;   // two areas of 16 blocks of 16 x 20 fp32
 constexpr uint32_t OFF_SOLVE1 = OFF_SOLVE0 + SOLVE_BYTES;
 constexpr uint32_t OFF_GB0 = OFF_SOLVE1 + SOLVE_BYTES;         // KQ_STAGES x (g tile 1 KB + beta tile 1 KB)
 constexpr uint32_t GATE_BYTES = 2560;
-constexpr uint32_t OFF_GATE0 = OFF_GB0 + KQ_STAGES * 2048;     // processed gates
-constexpr uint32_t OFF_GATE1 = OFF_GATE0 + GATE_BYTES;
-constexpr uint32_t OFF_UNITS = OFF_GATE1 + GATE_BYTES;         // int4 x MAX_UNITS
+constexpr uint32_t OFF_GATE = OFF_GB0 + KQ_STAGES * 2048;      // KQ_STAGES x processed gates
+constexpr uint32_t OFF_UNITS = OFF_GATE + KQ_STAGES * GATE_BYTES;   // int4 x MAX_UNITS
 constexpr uint32_t OFF_BARS = OFF_UNITS + MAX_UNITS * 16;
-constexpr uint32_t NUM_BARS = 29;
+constexpr uint32_t NUM_BARS = 30;
 static_assert(NUM_BARS * 8 <= 256, "barrier area");
 constexpr uint32_t OFF_MISC = OFF_BARS + 256;                  // tmem base, abort flag, count
 constexpr uint32_t OFF_OGR = OFF_MISC + 64;                    // Gamma_i rq_i for the outputs, 64 floats
-constexpr uint32_t SMEM_USED = OFF_OGR + 256;
+constexpr uint32_t OFF_OST = OFF_OGR + 256;                    // output transpose, 512 B per state warp
+constexpr uint32_t SMEM_USED = OFF_OST + 4 * 512;
 constexpr uint32_t SMEM_BYTES = SMEM_USED + 1024;              // + alignment slack
 static_assert(SMEM_BYTES <= 232448, "shared memory budget");
-static_assert(OFF_GB0 % 1024 == 0 && OFF_V % 1024 == 0 && OFF_WNEG % 1024 == 0 &&
+static_assert(OFF_GB0 % 1024 == 0 && OFF_V % 1024 == 0 && OFF_WNEG % 1024 == 0 && OFF_TB % 1024 == 0 &&
               OFF_KQ0 + KQ_STAGES * KQ_STAGE <= OFF_V && OFF_V + 16384 <= OFF_WNEG, "alignment");
 
 // gate-array offsets (floats) inside a GATE stage
@@ -111,9 +111,9 @@ static_assert((GA_BG + 64) * 4 <= (int)GATE_BYTES, "gate stage size");
 // barrier indices
 enum {
     B_KQ_FULL = 0, B_KQ_EMPTY = 3, B_V_FULL = 6, B_V_EMPTY = 7, B_GATE_FULL = 8,
-    B_GATE_EMPTY = 10, B_G_DONE = 12, B_T_READY = 13, B_WU_DONE = 14, B_WNEG = 15,
-    B_S_READY = 16, B_U_DONE = 17, B_E1 = 18, B_S_DONE = 19, B_Z_DONE = 20, B_Y_FREE = 21,
-    B_G_FREE = 22, B_A_READY = 23, B_SOLVE_FREE = 25, B_P_FREE = 27, B_COUNT = 29
+    B_GATE_EMPTY = 11, B_G_DONE = 14, B_T_READY = 15, B_W_DONE = 16, B_WNEG = 17,
+    B_S_READY = 18, B_U_DONE = 19, B_E1 = 20, B_S_DONE = 21, B_Z_DONE = 22, B_Y_FREE = 23,
+    B_G_FREE = 24, B_A_READY = 25, B_SOLVE_FREE = 27, B_UT_DONE = 29, B_COUNT = 30
 };
 static_assert(B_COUNT == (int)NUM_BARS, "barrier count");
 
@@ -126,7 +126,6 @@ struct __align__(64) Params {
     CUtensorMap tm_v;     // (128, Hv, N)
     CUtensorMap tm_g;     // (Hv, N) fp32, box (4, 64)
     CUtensorMap tm_beta;
-    CUtensorMap tm_out;   // (128, Hv, N) bf16, box (64, 1, 64), 128B swizzle (stores)
     const int32_t *cu_seqlens;
     const float *initial_state;
     float *final_state;
@@ -458,9 +457,9 @@ __global__ void __launch_bounds__(NTHREADS, 1) gdn_prefill_chunk_kernel(const __
         tmem_relinquish();
     }
     // P and T tiles: only the blocks on and below the diagonal are ever written
-    static_assert(OFF_P1 == OFF_P0 + 8192 && OFF_TB == OFF_P1 + 8192 && OFF_TBG == OFF_TB + 8192, "tile order");
-    for (int i = tid; i < 32768 / 16; i += NTHREADS)
-        reinterpret_cast<uint4 *>(smem + OFF_P0)[i] = make_uint4(0u, 0u, 0u, 0u);
+    static_assert(OFF_TB == OFF_P + KQ_STAGES * P_STAGE && OFF_TBG == OFF_TB + 8192, "tile order");
+    for (int i = tid; i < (int)((OFF_TBG + 8192 - OFF_P) / 16); i += NTHREADS)
+        reinterpret_cast<uint4 *>(smem + OFF_P)[i] = make_uint4(0u, 0u, 0u, 0u);
     fence_proxy_async_smem();
     tc_fence_before();
     __syncthreads();
@@ -469,12 +468,11 @@ __global__ void __launch_bounds__(NTHREADS, 1) gdn_prefill_chunk_kernel(const __
 
     // per-role pipeline counters (persist across units and batches)
     uint32_t kq_use[KQ_STAGES] = {}, v_use = 0;               // TMA
-    uint32_t c_wneg = 0, c_s = 0, c_y = 0, c_e1 = 0;                 // chain issuer
-    uint32_t q_kq[KQ_STAGES] = {}, q_t = 0, q_v = 0, q_wu = 0, q_g = 0;   // prep-stream issuer
-    uint32_t p_kq[KQ_STAGES] = {}, p_gate_empty[2] = {0, 0}, p_g = 0, p_sf[2] = {0, 0};   // prep front
-    uint32_t p_pf[2] = {0, 0};
+    uint32_t c_wneg = 0, c_s = 0, c_y = 0, c_e1 = 0, c_ut = 0;       // chain issuer
+    uint32_t q_kq[KQ_STAGES] = {}, q_t = 0, q_v = 0, q_w = 0, q_u = 0, q_g = 0;   // prep-stream issuer
+    uint32_t p_kq[KQ_STAGES] = {}, p_gate_empty[KQ_STAGES] = {}, p_g = 0, p_sf[2] = {0, 0};   // prep front
     uint32_t p_ar[2] = {0, 0}, p_wu = 0;                              // prep back
-    uint32_t s_u = 0, s_sd = 0, s_zd = 0, s_wu = 0, s_gate[2] = {0, 0};   // state
+    uint32_t s_u = 0, s_sd = 0, s_zd = 0, s_w = 0, s_gate[KQ_STAGES] = {};   // state
     uint32_t gc = 0;   // global chunk counter (same sequence in every role)
 
     const int G = gridDim.x;
@@ -499,7 +497,11 @@ __global__ void __launch_bounds__(NTHREADS, 1) gdn_prefill_chunk_kernel(const __
         }
 
         if (warp == TMA_WARP) {
-            // ------------------------------------------------------------ TMA producer
+            // ------------------------------------------------------------ TMA producers
+            // lane 0: q/k/g/beta tiles (KQ_STAGES stages); lane 1: v tiles (one stage).  The
+            // two streams are released by different consumers (the state chain, the W/U~
+            // products), so neither waits behind the other.  Each also pulls a later chunk
+            // of its stream into L2, so that a reload does not start cold.
             if (lane == 0) {
                 for (int k = 0; k < nunits && !cx.aborted(); ++k) {
                     const Unit un = load_unit(smem, k);
@@ -520,23 +522,32 @@ __global__ void __launch_bounds__(NTHREADS, 1) gdn_prefill_chunk_kernel(const __
                         tma_load_3d(kq + KQ_KB + 8192, &p.tm_q, kb, 64, qh, t0);
                         tma_load_2d(gb, &p.tm_g, kb, un.h & ~3, t0);
                         tma_load_2d(gb + 1024, &p.tm_beta, kb, un.h & ~3, t0);
+                        if (n + KQ_STAGES < nc) {
+                            const int t2 = t0 + KQ_STAGES * C;
+                            tma_prefetch_3d(&p.tm_k, 0, qh, t2);
+                            tma_prefetch_3d(&p.tm_k, 64, qh, t2);
+                            tma_prefetch_3d(&p.tm_q, 0, qh, t2);
+                            tma_prefetch_3d(&p.tm_q, 64, qh, t2);
+                            tma_prefetch_2d(&p.tm_g, un.h & ~3, t2);
+                            tma_prefetch_2d(&p.tm_beta, un.h & ~3, t2);
+                        }
+                    }
+                    gc += nc;
+                }
+            } else if (lane == 1) {
+                for (int k = 0; k < nunits && !cx.aborted(); ++k) {
+                    const Unit un = load_unit(smem, k);
+                    const int nc = (un.len + C - 1) / C;
+                    for (int n = 0; n < nc; ++n) {
+                        const int t0 = un.start + n * C;
                         if (v_use > 0 && !cx.wait(B_V_EMPTY, (v_use - 1) & 1)) break;
                         ++v_use;
                         mbar_arrive_expect_tx(cx.bar(B_V_FULL), 16384);
                         tma_load_3d(sbase + OFF_V, &p.tm_v, cx.bar(B_V_FULL), 0, un.h, t0);
                         tma_load_3d(sbase + OFF_V + V_HALF, &p.tm_v, cx.bar(B_V_FULL), 64, un.h, t0);
                         if (n + 2 < nc) {
-                            // the chunk after next into L2: its loads wait on buffers freed by
-                            // the state chain and would otherwise start cold
-                            const int t2 = t0 + 2 * C;
-                            tma_prefetch_3d(&p.tm_k, 0, qh, t2);
-                            tma_prefetch_3d(&p.tm_k, 64, qh, t2);
-                            tma_prefetch_3d(&p.tm_q, 0, qh, t2);
-                            tma_prefetch_3d(&p.tm_q, 64, qh, t2);
-                            tma_prefetch_3d(&p.tm_v, 0, un.h, t2);
-                            tma_prefetch_3d(&p.tm_v, 64, un.h, t2);
-                            tma_prefetch_2d(&p.tm_g, un.h & ~3, t2);
-                            tma_prefetch_2d(&p.tm_beta, un.h & ~3, t2);
+                            tma_prefetch_3d(&p.tm_v, 0, un.h, t0 + 2 * C);
+                            tma_prefetch_3d(&p.tm_v, 64, un.h, t0 + 2 * C);
                         }
                     }
                     gc += nc;
@@ -551,9 +562,12 @@ __global__ void __launch_bounds__(NTHREADS, 1) gdn_prefill_chunk_kernel(const __
             // cross-stream hazard is ordered by an mbarrier:
             //   G(x):  KQ(x) loaded, G_FREE(x-1) (A/P of x-1 built); up to one chunk
             //          ahead of WU inside a unit
-            //   WU(x): T(x) ready, V(x) loaded, Z_DONE(x-1) (the U columns hold the bf16
-            //          operands of (2)/(3) until then), WNEG(x-1) (W columns converted)
-            //   C1(x): WNEG(x) (so WU(x) completed), S_READY(x); Y part after Y_FREE(x-1)
+            //   W(x):  T(x) ready, WNEG(x-1) (W columns converted)
+            //   U~(x): V(x) loaded, Z_DONE(x-1) (the U columns hold the bf16 operands of
+            //          (2)/(3) until then)
+            //   C1(x): WNEG(x) (W(x) converted; the state warpgroup converts only after it
+            //          saw U_DONE(x-1), so (1a) of x-1 no longer reads the -W tile),
+            //          UT_DONE(x), S_READY(x); the Y part after Y_FREE(x-1)
             //   C2(x): E1(x)
             if (lane == 0) {
                 constexpr uint32_t ID_G = idesc_bf16(128, 64, 0, 0);
@@ -572,19 +586,22 @@ __global__ void __launch_bounds__(NTHREADS, 1) gdn_prefill_chunk_kernel(const __
                     const uint64_t dV = sdesc_sw128(sbase + OFF_V, V_HALF, 1024);
                     const uint64_t dTB = sdesc_sw128(sbase + OFF_TB, 16, 1024);
                     const uint64_t dTBG = sdesc_sw128(sbase + OFF_TBG, 16, 1024);
-                    // Two tasks per chunk x, each issued as soon as its inputs are ready
-                    // (non-blocking tests, so neither waits behind the other):
+                    // Three tasks per chunk x, each issued as soon as its inputs are ready
+                    // (non-blocking tests, so none waits behind another):
                     //   G(x):  previous Gram read by the prep (G_FREE), KQ(x) loaded; at most
-                    //          one chunk ahead of WU
-                    //   WU(x): G(x) issued, T(x) ready, V(x) loaded, Z_DONE(x-1), WNEG(x-1)
+                    //          one chunk ahead of W
+                    //   W(x):  G(x) issued, T(x) ready, WNEG(x-1) (W columns converted)
+                    //   U~(x): W(x) issued, V(x) loaded, Z_DONE(x-1) (the U columns hold the bf16
+                    //          operands of (2)/(3) of x-1 until then); its commit (UT_DONE)
+                    //          therefore also covers W(x)
                     // Every barrier tested here can run at most one phase ahead of its counter:
                     // its next phase depends on the task that consumes this one.
                     for (int k = 0; k < nunits && ok; ++k) {
                         const Unit un = load_unit(smem, k);
                         const int nc = (un.len + C - 1) / C;
-                        int gi = 0, wi = 0;   // G / WU issued in this unit
+                        int gi = 0, wi = 0, ui = 0;   // G / W / U~ issued in this unit
                         long long t_last = clock64();
-                        while (wi < nc) {
+                        while (ui < nc) {
                             bool did = false;
                             if (gi < nc && gi <= wi + 1) {
                                 const uint32_t sg = (gc + gi) % KQ_STAGES;
@@ -606,24 +623,31 @@ __global__ void __launch_bounds__(NTHREADS, 1) gdn_prefill_chunk_kernel(const __
                                 }
                             }
                             if (!did && wi < gi && mbar_test_wait(cx.bar(B_T_READY), q_t & 1) &&
-                                mbar_test_wait(cx.bar(B_V_FULL), q_v & 1) &&
-                                (q_wu == 0 || (mbar_test_wait(cx.bar(B_Z_DONE), (q_wu - 1) & 1) &&
-                                               mbar_test_wait(cx.bar(B_WNEG), (q_wu - 1) & 1)))) {
+                                (q_w == 0 || mbar_test_wait(cx.bar(B_WNEG), (q_w - 1) & 1))) {
                                 ++q_t;
-                                ++q_v;
-                                ++q_wu;
+                                ++q_w;
                                 const uint32_t ks = (gc + wi) % KQ_STAGES;
                                 tc_fence_after();
                                 // (W): W^T[dk][i] = sum_j K[j][dk] Tbg[i][j]; A = K (MN-major), B = Tbg
+#pragma unroll 1
+                                for (int kk = 0; kk < 4; ++kk)
+                                    umma_bf16(tmem + TM_W, dKQm + ((ks * KQ_STAGE + kk * 2048) >> 4), dTBG + ((kk * 32) >> 4), ID_W, kk > 0);
+                                umma_commit(cx.bar(B_W_DONE));
+                                ++wi;
+                                did = true;
+                            }
+                            if (!did && ui < wi && mbar_test_wait(cx.bar(B_V_FULL), q_v & 1) &&
+                                (q_u == 0 || mbar_test_wait(cx.bar(B_Z_DONE), (q_u - 1) & 1))) {
+                                ++q_v;
+                                ++q_u;
+                                tc_fence_after();
                                 // (U~): U^T[dv][i] = sum_j V[j][dv] Tb[i][j]; A = V (MN-major), B = Tb
 #pragma unroll 1
-                                for (int kk = 0; kk < 4; ++kk) {
-                                    umma_bf16(tmem + TM_W, dKQm + ((ks * KQ_STAGE + kk * 2048) >> 4), dTBG + ((kk * 32) >> 4), ID_W, kk > 0);
+                                for (int kk = 0; kk < 4; ++kk)
                                     umma_bf16(tmem + TM_U, dV + ((kk * 2048) >> 4), dTB + ((kk * 32) >> 4), ID_U, kk > 0);
-                                }
-                                umma_commit(cx.bar(B_WU_DONE));
+                                umma_commit(cx.bar(B_UT_DONE));
                                 umma_commit(cx.bar(B_V_EMPTY));
-                                ++wi;
+                                ++ui;
                                 did = true;
                             }
                             if (did) {
@@ -643,18 +667,18 @@ __global__ void __launch_bounds__(NTHREADS, 1) gdn_prefill_chunk_kernel(const __
                     }
                 } else {
                     const uint64_t dWNEG = sdesc_sw128(sbase + OFF_WNEG, 8192, 1024);
-                    const uint64_t dP0 = sdesc_sw128(sbase + OFF_P0, 16, 1024);
-                    const uint64_t dP1 = sdesc_sw128(sbase + OFF_P1, 16, 1024);
+                    const uint64_t dP = sdesc_sw128(sbase + OFF_P, 16, 1024);
                     for (int k = 0; k < nunits && ok; ++k) {
                         const Unit un = load_unit(smem, k);
                         const int nc = (un.len + C - 1) / C;
                         for (int n = 0; n < nc && ok; ++n) {
-                            const uint32_t s = (gc + n) & 1;
                             const uint32_t ks = (gc + n) % KQ_STAGES;
                             // (1a) U^T += S^T (-W)^T; the bf16 S^T is the TMEM A operand (8 columns
                             //      per 16 dk)
                             ok = cx.wait(B_WNEG, c_wneg & 1);
                             ++c_wneg;
+                            ok = ok && cx.wait(B_UT_DONE, c_ut & 1);
+                            ++c_ut;
                             ok = ok && cx.wait(B_S_READY, c_s & 1);
                             ++c_s;
                             if (!ok) break;
@@ -684,10 +708,9 @@ __global__ void __launch_bounds__(NTHREADS, 1) gdn_prefill_chunk_kernel(const __
                             umma_commit(cx.bar(B_S_DONE));
 #pragma unroll 1
                             for (int kk = 0; kk < 4; ++kk)
-                                umma_bf16_ts(tmem + TM_Z, tmem + TM_U + 16 * kk, (s ? dP1 : dP0) + ((kk * 32) >> 4), ID_3, kk > 0);
+                                umma_bf16_ts(tmem + TM_Z, tmem + TM_U + 16 * kk, dP + ((ks * P_STAGE + kk * 32) >> 4), ID_3, kk > 0);
                             umma_commit(cx.bar(B_Z_DONE));
-                            umma_commit(cx.bar(B_P_FREE + s));
-                            umma_commit(cx.bar(B_KQ_EMPTY + ks));
+                            umma_commit(cx.bar(B_KQ_EMPTY + ks));   // also releases P stage ks
                         }
                         gc += nc;
                     }
@@ -712,16 +735,16 @@ __global__ void __launch_bounds__(NTHREADS, 1) gdn_prefill_chunk_kernel(const __
                 for (int n = 0; n < nc && ok; ++n) {
                     const uint32_t s = (gc + n) & 1;
                     float *solve = reinterpret_cast<float *>(smem + (s ? OFF_SOLVE1 : OFF_SOLVE0));
-                    float *ga = reinterpret_cast<float *>(smem + (s ? OFF_GATE1 : OFF_GATE0));
+                    const uint32_t ks = (gc + n) % KQ_STAGES;   // KQ and gate stage
+                    float *ga = reinterpret_cast<float *>(smem + OFF_GATE + ks * GATE_BYTES);
                     if (pg == 0) {
                         const int len_n = min(C, un.len - n * C);
-                        const uint32_t ks = (gc + n) % KQ_STAGES;
                         const uint8_t *kq = smem + OFF_KQ0 + ks * KQ_STAGE;
                         const float *gtile = reinterpret_cast<const float *>(smem + OFF_GB0 + ks * 2048);
                         ok = cx.wait(B_KQ_FULL + ks, p_kq[ks] & 1);
                         ++p_kq[ks];
-                        if (p_gate_empty[s] > 0) ok = ok && cx.wait(B_GATE_EMPTY + s, (p_gate_empty[s] - 1) & 1);
-                        ++p_gate_empty[s];
+                        if (p_gate_empty[ks] > 0) ok = ok && cx.wait(B_GATE_EMPTY + ks, (p_gate_empty[ks] - 1) & 1);
+                        ++p_gate_empty[ks];
                         if (p_sf[s] > 0) ok = ok && cx.wait(B_SOLVE_FREE + s, (p_sf[s] - 1) & 1);
                         ++p_sf[s];
                         // --- row norms (K rows 0..63, Q rows 64..127), conflict-free chunk order
@@ -770,15 +793,14 @@ __global__ void __launch_bounds__(NTHREADS, 1) gdn_prefill_chunk_kernel(const __
                             if (lane == 31) ga[GA_GC] = ex2_approx(G2b);
                         }
                         named_sync(1, 128);
-                        if (lt == 0) mbar_arrive(cx.bar(B_GATE_FULL + s));
-                        // --- Gram -> A (rows 0..63, fp32 blocks) and P (rows 64..127, bf16 tile); the
-                        //     P tile of this parity is read by (3) of the chunk before last
-                        if (p_pf[s] > 0) ok = ok && cx.wait(B_P_FREE + s, (p_pf[s] - 1) & 1);
-                        ++p_pf[s];
+                        if (lt == 0) mbar_arrive(cx.bar(B_GATE_FULL + ks));
+                        // --- Gram -> A (rows 0..63, fp32 blocks) and P (rows 64..127, bf16 tile); P
+                        //     shares the KQ stage, so the (3) product that last read it completed
+                        //     before this stage was reloaded (KQ_EMPTY is committed after it)
                         ok = ok && cx.wait(B_G_DONE, p_g & 1);
                         ++p_g;
                         tc_fence_after();
-                        build_row(tl + TM_G, pw, ga, solve, smem + (s ? OFF_P1 : OFF_P0));
+                        build_row(tl + TM_G, pw, ga, solve, smem + OFF_P + ks * P_STAGE);
                         if (pw >= 2) fence_proxy_async_smem();
                         if (lt < 64) ga[GA_BG + lt] = ga[GA_BETA + lt] * ga[GA_GAM + lt] * ga[GA_RK + lt];
                         tc_fence_before();
@@ -790,8 +812,8 @@ __global__ void __launch_bounds__(NTHREADS, 1) gdn_prefill_chunk_kernel(const __
                     } else {
                         ok = cx.wait(B_A_READY + s, p_ar[s] & 1);
                         ++p_ar[s];
-                        // the T tiles of the previous chunk are read by its WU products
-                        if (p_wu > 0) ok = ok && cx.wait(B_WU_DONE, (p_wu - 1) & 1);
+                        // the T tiles of the previous chunk are read by its W and U~ products
+                        if (p_wu > 0) ok = ok && cx.wait(B_UT_DONE, (p_wu - 1) & 1);
                         ++p_wu;
                         // --- diagonal 16x16 inverses D_I = (I + A_II)^-1 (back threads 0..63, one column each)
                         if (lt < 64) {
@@ -894,7 +916,29 @@ __global__ void __launch_bounds__(NTHREADS, 1) gdn_prefill_chunk_kernel(const __
             // ------------------------------------------------------------ state warpgroup
             const int dv = tid;                 // 0..127 == TMEM lane
             const uint32_t tl = tmem + ((uint32_t)(32 * warp) << 16);
-            bool store_pending = false;         // an output TMA store may still read OFF_WNEG
+            // W^T of the next chunk (TMEM, lane dk) -> -W as the MN-major B tile of (1a) (row
+            // dk).  The tile is free: this warpgroup already saw U_DONE of the chunk before,
+            // so (1a) of that chunk has read it.
+            auto convert_wneg = [&]() -> bool {
+                const bool w_ok = cx.wait(B_W_DONE, s_w & 1);
+                ++s_w;
+                tc_fence_after();
+#pragma unroll 1
+                for (int q = 0; q < 4; ++q) {
+                    float t[16];
+                    tmem_ld16(tl + TM_W + 16 * q, t);
+                    tmem_wait_ld();
+#pragma unroll
+                    for (int e = 0; e < 16; ++e) t[e] = -t[e];
+                    *reinterpret_cast<uint4 *>(smem + OFF_WNEG + sw128(dv, 2 * q)) = pack8_bf16(t);
+                    *reinterpret_cast<uint4 *>(smem + OFF_WNEG + sw128(dv, 2 * q + 1)) = pack8_bf16(t + 8);
+                }
+                fence_proxy_async_smem();
+                tc_fence_before();
+                named_sync(2, 128);
+                if (dv == 0) mbar_arrive(cx.bar(B_WNEG));
+                return w_ok;
+            };
             float *ogr = reinterpret_cast<float *>(smem + OFF_OGR);
             for (int k = 0; k < nunits; ++k) {
                 const Unit un = load_unit(smem, k);
@@ -912,10 +956,10 @@ __global__ void __launch_bounds__(NTHREADS, 1) gdn_prefill_chunk_kernel(const __
                 bool ok = true;
                 // unit start: S0 -> bf16 operand columns and gC(0) * S0 -> TMEM
                 {
-                    const uint32_t s = gc & 1;
-                    ok = cx.wait(B_GATE_FULL + s, s_gate[s] & 1);
-                    ++s_gate[s];
-                    const float *ga = reinterpret_cast<const float *>(smem + (s ? OFF_GATE1 : OFF_GATE0));
+                    const uint32_t gs = gc % KQ_STAGES;
+                    ok = cx.wait(B_GATE_FULL + gs, s_gate[gs] & 1);
+                    ++s_gate[gs];
+                    const float *ga = reinterpret_cast<const float *>(smem + OFF_GATE + gs * GATE_BYTES);
                     const float gC = ga[GA_GC];
 #pragma unroll 1
                     for (int q = 0; q < 8; ++q) {
@@ -939,34 +983,11 @@ __global__ void __launch_bounds__(NTHREADS, 1) gdn_prefill_chunk_kernel(const __
                     if (dv == 0 && ok) mbar_arrive(cx.bar(B_S_READY));
                 }
                 for (int n = 0; n < nc && ok; ++n) {
-                    const uint32_t s = (gc + n) & 1;
-                    const uint32_t s1 = (gc + n + 1) & 1;
+                    const uint32_t gs = (gc + n) % KQ_STAGES, gs1 = (gc + n + 1) % KQ_STAGES;
                     const int len_n = min(C, un.len - n * C);
-                    const float *ga = reinterpret_cast<const float *>(smem + (s ? OFF_GATE1 : OFF_GATE0));
-                    // ---- W^T (TMEM, lane dk) -> -W as the MN-major B tile of (1a) (row dk)
-                    ok = cx.wait(B_WU_DONE, s_wu & 1);
-                    ++s_wu;
-                    tc_fence_after();
-                    if (store_pending) {
-                        // the previous chunk's output store still reads the tile
-                        if (dv == 0) bulk_wait_read();
-                        named_sync(2, 128);
-                        store_pending = false;
-                    }
-#pragma unroll 1
-                    for (int q = 0; q < 4; ++q) {
-                        float t[16];
-                        tmem_ld16(tl + TM_W + 16 * q, t);
-                        tmem_wait_ld();
-#pragma unroll
-                        for (int e = 0; e < 16; ++e) t[e] = -t[e];
-                        *reinterpret_cast<uint4 *>(smem + OFF_WNEG + sw128(dv, 2 * q)) = pack8_bf16(t);
-                        *reinterpret_cast<uint4 *>(smem + OFF_WNEG + sw128(dv, 2 * q + 1)) = pack8_bf16(t + 8);
-                    }
-                    fence_proxy_async_smem();
-                    tc_fence_before();
-                    named_sync(2, 128);
-                    if (dv == 0) mbar_arrive(cx.bar(B_WNEG));
+                    const float *ga = reinterpret_cast<const float *>(smem + OFF_GATE + gs * GATE_BYTES);
+                    // the -W tile of a unit's first chunk (later ones are converted after E2)
+                    if (n == 0) ok = convert_wneg();
                     // ---- E1: U^T -> bf16 tiles (plain for Z, decayed and key-normed for S)
                     ok = ok && cx.wait(B_U_DONE, s_u & 1);
                     ++s_u;
@@ -993,12 +1014,11 @@ __global__ void __launch_bounds__(NTHREADS, 1) gdn_prefill_chunk_kernel(const __
                     }
                     tmem_wait_st();
                     if (dv < 64) ogr[dv] = ga[GA_GAM + dv] * ga[GA_RQ + dv];
-                    fence_proxy_async_smem();
                     tc_fence_before();
                     named_sync(2, 128);
                     if (dv == 0) {
                         mbar_arrive(cx.bar(B_E1));
-                        mbar_arrive(cx.bar(B_GATE_EMPTY + s));   // the outputs read ogr from here on
+                        mbar_arrive(cx.bar(B_GATE_EMPTY + gs));   // the outputs read ogr from here on
                     }
                     // ---- E2: new state -> bf16 operand columns (+ decay of the next chunk) or final state
                     ok = ok && cx.wait(B_S_DONE, s_sd & 1);
@@ -1007,9 +1027,9 @@ __global__ void __launch_bounds__(NTHREADS, 1) gdn_prefill_chunk_kernel(const __
                     const bool more = n + 1 < nc;
                     float gC1 = 1.f;
                     if (more) {
-                        ok = ok && cx.wait(B_GATE_FULL + s1, s_gate[s1] & 1);
-                        ++s_gate[s1];
-                        gC1 = reinterpret_cast<const float *>(smem + (s1 ? OFF_GATE1 : OFF_GATE0))[GA_GC];
+                        ok = ok && cx.wait(B_GATE_FULL + gs1, s_gate[gs1] & 1);
+                        ++s_gate[gs1];
+                        gC1 = reinterpret_cast<const float *>(smem + OFF_GATE + gs1 * GATE_BYTES)[GA_GC];
                     }
 #pragma unroll 1
                     for (int q = 0; q < 8; ++q) {
@@ -1034,17 +1054,23 @@ __global__ void __launch_bounds__(NTHREADS, 1) gdn_prefill_chunk_kernel(const __
                         tc_fence_before();
                         named_sync(2, 128);
                         if (dv == 0) mbar_arrive(cx.bar(B_S_READY));
+                        // the next chunk's (1a) waits on its -W tile: convert it before the outputs
+                        ok = convert_wneg() && ok;
                     }
-                    // ---- outputs O^T = scale (Y diag(Gamma rq) + Z), staged through the U tile as
-                    //      two 128B-swizzled [64 rows i][64 dv] bf16 tiles (the layout of the TMA box)
+                    // ---- outputs O^T = scale (Y diag(Gamma rq) + Z): 8 tokens at a time through a
+                    //      warp-private [8 tokens][32 dv] bf16 scratch, then one 16-byte store per
+                    //      lane (lanes 4t..4t+3 write token t's 64 bytes of this warp's dv); rows
+                    //      past len_n belong to the next request and are skipped
                     ok = ok && cx.wait(B_Z_DONE, s_zd & 1);
                     ++s_zd;
                     tc_fence_after();
                     {
-                        uint8_t *ot = smem + OFF_WNEG;
                         const float sc = p.scale;
-                        const uint32_t obase = ((uint32_t)dv >> 6) * 8192u + ((uint32_t)dv & 7u) * 2u;
-                        const uint32_t och = ((uint32_t)dv >> 3) & 7u;
+                        uint8_t *ost = smem + OFF_OST + 512 * warp;
+                        const int tt = lane >> 2;   // token of this lane's 16-byte store
+                        __nv_bfloat16 *obase = p.out + ((int64_t)(un.start + n * C + tt) * p.Hv + un.h) * D +
+                                               32 * warp + 8 * (lane & 3);
+                        const int64_t ostride8 = (int64_t)8 * p.Hv * D;
 #pragma unroll 1
                         for (int q = 0; q < 4; ++q) {
                             float y[16], z[16], gg[16];
@@ -1057,47 +1083,27 @@ __global__ void __launch_bounds__(NTHREADS, 1) gdn_prefill_chunk_kernel(const __
                             }
                             tmem_wait_ld();
 #pragma unroll
-                            for (int e = 0; e < 16; ++e) {
-                                const uint32_t i = 16u * q + e;
-                                *reinterpret_cast<__nv_bfloat16 *>(ot + obase + i * 128u + ((och ^ (i & 7u)) << 4)) =
-                                    __float2bfloat16_rn(sc * fmaf(gg[e], y[e], z[e]));
+                            for (int hb = 0; hb < 2; ++hb) {
+#pragma unroll
+                                for (int e = 0; e < 8; ++e)
+                                    *reinterpret_cast<__nv_bfloat16 *>(ost + e * 64 + lane * 2) =
+                                        __float2bfloat16_rn(sc * fmaf(gg[8 * hb + e], y[8 * hb + e], z[8 * hb + e]));
+                                __syncwarp();
+                                const uint4 v = *reinterpret_cast<const uint4 *>(ost + lane * 16);
+                                __syncwarp();
+                                const int i0 = 16 * q + 8 * hb;   // first token of this group
+                                if (i0 + tt < len_n) *reinterpret_cast<uint4 *>(obase + (i0 / 8) * ostride8) = v;
                             }
                         }
-                        fence_proxy_async_smem();
                         tc_fence_before();
                         named_sync(2, 128);
                         if (dv == 0) mbar_arrive(cx.bar(B_Y_FREE));
-                        if (len_n == C) {
-                            // full chunk: two TMA box stores, completion checked before the tile is reused
-                            if (dv == 0) {
-                                const int row = un.start + n * C;
-                                tma_store_3d(&p.tm_out, sbase + OFF_WNEG, 0, un.h, row);
-                                tma_store_3d(&p.tm_out, sbase + OFF_WNEG + 8192, 64, un.h, row);
-                                bulk_commit();
-                            }
-                            store_pending = true;
-                        } else {
-                            // ragged tail: rows past len_n belong to the next request; coalesced
-                            // 16-byte stores, thread -> (row i = dv >> 1, half = dv & 1)
-                            const int i = dv >> 1, hf = dv & 1;
-                            if (i < len_n) {
-                                __nv_bfloat16 *orow = p.out + ((int64_t)(un.start + n * C + i) * p.Hv + un.h) * D + 64 * hf;
-                                const uint8_t *srow = ot + hf * 8192 + i * 128;
-                                uint4 v[8];
-#pragma unroll
-                                for (int c = 0; c < 8; ++c)
-                                    v[c] = *reinterpret_cast<const uint4 *>(srow + ((c ^ (i & 7)) << 4));
-#pragma unroll
-                                for (int c = 0; c < 8; ++c) *reinterpret_cast<uint4 *>(orow + 8 * c) = v[c];
-                            }
-                        }
                     }
                     ok = !named_sync_or(2, 128, !ok || cx.aborted());
                 }
                 gc += nc;
                 if (!ok) break;
             }
-            if (dv == 0) bulk_wait_all();   // the unit list is rebuilt in the staging tile
         }
         __syncthreads();
         if (cx.aborted()) break;
@@ -1105,7 +1111,8 @@ __global__ void __launch_bounds__(NTHREADS, 1) gdn_prefill_chunk_kernel(const __
     }
 
     // teardown: drain outstanding TMA stages on abort, then free TMEM
-    if (cx.aborted() && warp == TMA_WARP && lane == 0) {
+    if (cx.aborted() && warp == TMA_WARP && lane < 2) {
+        // each producer lane waits for the copies it issued
         for (int s = 0; s < KQ_STAGES; ++s) {
             const long long t0 = clock64();
             while (kq_use[s] > 0 && !mbar_try_wait(cx.bar(B_KQ_FULL + s), (kq_use[s] - 1) & 1))
@@ -1202,7 +1209,6 @@ cudaError_t launch_prefill_chunked(const GdnPrefillArgs &a, cudaStream_t stream)
         if (!make_map_3d_bf16(&p.tm_q, a.q, 128, a.Hq, N) ||
             !make_map_3d_bf16(&p.tm_k, a.k, 128, a.Hq, N) ||
             !make_map_3d_bf16(&p.tm_v, a.v, 128, a.Hv, N) ||
-            !make_map_3d_bf16(&p.tm_out, a.out, 128, a.Hv, N) ||
             !make_map_2d_f32(&p.tm_g, a.g, a.Hv, N) || !make_map_2d_f32(&p.tm_beta, a.beta, a.Hv, N))
             return cudaErrorInvalidValue;
     }
