@@ -587,7 +587,9 @@ __global__ void __launch_bounds__(NTHREADS, 1) gdn_prefill_chunk_kernel(const __
                     const uint64_t dTB = sdesc_sw128(sbase + OFF_TB, 16, 1024);
                     const uint64_t dTBG = sdesc_sw128(sbase + OFF_TBG, 16, 1024);
                     // Three tasks per chunk x, each issued as soon as its inputs are ready
-                    // (non-blocking tests, so none waits behind another):
+                    // (non-blocking tests, so none waits behind another; an issue blocks while
+                    // the tensor pipe drains, so the state chain's inputs U~ and W go first and
+                    // the Gram look-ahead last):
                     //   G(x):  previous Gram read by the prep (G_FREE), KQ(x) loaded; at most
                     //          one chunk ahead of W
                     //   W(x):  G(x) issued, T(x) ready, WNEG(x-1) (W columns converted)
@@ -603,7 +605,35 @@ __global__ void __launch_bounds__(NTHREADS, 1) gdn_prefill_chunk_kernel(const __
                         long long t_last = clock64();
                         while (ui < nc) {
                             bool did = false;
-                            if (gi < nc && gi <= wi + 1) {
+                            if (ui < wi && mbar_test_wait(cx.bar(B_V_FULL), q_v & 1) &&
+                                (q_u == 0 || mbar_test_wait(cx.bar(B_Z_DONE), (q_u - 1) & 1))) {
+                                ++q_v;
+                                ++q_u;
+                                tc_fence_after();
+                                // (U~): U^T[dv][i] = sum_j V[j][dv] Tb[i][j]; A = V (MN-major), B = Tb
+#pragma unroll 1
+                                for (int kk = 0; kk < 4; ++kk)
+                                    umma_bf16(tmem + TM_U, dV + ((kk * 2048) >> 4), dTB + ((kk * 32) >> 4), ID_U, kk > 0);
+                                umma_commit(cx.bar(B_UT_DONE));
+                                umma_commit(cx.bar(B_V_EMPTY));
+                                ++ui;
+                                did = true;
+                            }
+                            if (!did && wi < gi && mbar_test_wait(cx.bar(B_T_READY), q_t & 1) &&
+                                (q_w == 0 || mbar_test_wait(cx.bar(B_WNEG), (q_w - 1) & 1))) {
+                                ++q_t;
+                                ++q_w;
+                                const uint32_t ks = (gc + wi) % KQ_STAGES;
+                                tc_fence_after();
+                                // (W): W^T[dk][i] = sum_j K[j][dk] Tbg[i][j]; A = K (MN-major), B = Tbg
+#pragma unroll 1
+                                for (int kk = 0; kk < 4; ++kk)
+                                    umma_bf16(tmem + TM_W, dKQm + ((ks * KQ_STAGE + kk * 2048) >> 4), dTBG + ((kk * 32) >> 4), ID_W, kk > 0);
+                                umma_commit(cx.bar(B_W_DONE));
+                                ++wi;
+                                did = true;
+                            }
+                            if (!did && gi < nc && gi <= wi + 1) {
                                 const uint32_t sg = (gc + gi) % KQ_STAGES;
                                 if ((q_g == 0 || mbar_test_wait(cx.bar(B_G_FREE), (q_g - 1) & 1)) &&
                                     mbar_test_wait(cx.bar(B_KQ_FULL + sg), q_kq[sg] & 1)) {
@@ -621,34 +651,6 @@ __global__ void __launch_bounds__(NTHREADS, 1) gdn_prefill_chunk_kernel(const __
                                     ++gi;
                                     did = true;
                                 }
-                            }
-                            if (!did && wi < gi && mbar_test_wait(cx.bar(B_T_READY), q_t & 1) &&
-                                (q_w == 0 || mbar_test_wait(cx.bar(B_WNEG), (q_w - 1) & 1))) {
-                                ++q_t;
-                                ++q_w;
-                                const uint32_t ks = (gc + wi) % KQ_STAGES;
-                                tc_fence_after();
-                                // (W): W^T[dk][i] = sum_j K[j][dk] Tbg[i][j]; A = K (MN-major), B = Tbg
-#pragma unroll 1
-                                for (int kk = 0; kk < 4; ++kk)
-                                    umma_bf16(tmem + TM_W, dKQm + ((ks * KQ_STAGE + kk * 2048) >> 4), dTBG + ((kk * 32) >> 4), ID_W, kk > 0);
-                                umma_commit(cx.bar(B_W_DONE));
-                                ++wi;
-                                did = true;
-                            }
-                            if (!did && ui < wi && mbar_test_wait(cx.bar(B_V_FULL), q_v & 1) &&
-                                (q_u == 0 || mbar_test_wait(cx.bar(B_Z_DONE), (q_u - 1) & 1))) {
-                                ++q_v;
-                                ++q_u;
-                                tc_fence_after();
-                                // (U~): U^T[dv][i] = sum_j V[j][dv] Tb[i][j]; A = V (MN-major), B = Tb
-#pragma unroll 1
-                                for (int kk = 0; kk < 4; ++kk)
-                                    umma_bf16(tmem + TM_U, dV + ((kk * 2048) >> 4), dTB + ((kk * 32) >> 4), ID_U, kk > 0);
-                                umma_commit(cx.bar(B_UT_DONE));
-                                umma_commit(cx.bar(B_V_EMPTY));
-                                ++ui;
-                                did = true;
                             }
                             if (did) {
                                 t_last = clock64();
@@ -924,14 +926,15 @@ __global__ void __launch_bounds__(NTHREADS, 1) gdn_prefill_chunk_kernel(const __
                 ++s_w;
                 tc_fence_after();
 #pragma unroll 1
-                for (int q = 0; q < 4; ++q) {
-                    float t[16];
-                    tmem_ld16(tl + TM_W + 16 * q, t);
+                for (int q = 0; q < 2; ++q) {
+                    float t[32];
+                    tmem_ld32(tl + TM_W + 32 * q, t);
                     tmem_wait_ld();
 #pragma unroll
-                    for (int e = 0; e < 16; ++e) t[e] = -t[e];
-                    *reinterpret_cast<uint4 *>(smem + OFF_WNEG + sw128(dv, 2 * q)) = pack8_bf16(t);
-                    *reinterpret_cast<uint4 *>(smem + OFF_WNEG + sw128(dv, 2 * q + 1)) = pack8_bf16(t + 8);
+                    for (int e = 0; e < 32; ++e) t[e] = -t[e];
+#pragma unroll
+                    for (int c = 0; c < 4; ++c)
+                        *reinterpret_cast<uint4 *>(smem + OFF_WNEG + sw128(dv, 4 * q + c)) = pack8_bf16(t + 8 * c);
                 }
                 fence_proxy_async_smem();
                 tc_fence_before();
@@ -993,24 +996,29 @@ __global__ void __launch_bounds__(NTHREADS, 1) gdn_prefill_chunk_kernel(const __
                     ++s_u;
                     tc_fence_after();
 #pragma unroll 1
-                    for (int q = 0; q < 4; ++q) {
-                        float u[16], d[16];
-                        tmem_ld16(tl + TM_U + 16 * q, u);
-#pragma unroll
-                        for (int e = 0; e < 16; e += 4) {
-                            const float4 d4 = ld4(ga + GA_DEC + 16 * q + e);
-                            const float4 k4 = ld4(ga + GA_RK + 16 * q + e);
-                            d[e] = d4.x * k4.x; d[e + 1] = d4.y * k4.y; d[e + 2] = d4.z * k4.z; d[e + 3] = d4.w * k4.w;
-                        }
+                    for (int q = 0; q < 2; ++q) {
+                        float u[32];
+                        tmem_ld32(tl + TM_U + 32 * q, u);
                         tmem_wait_ld();
-                        // columns [16q, 16q+8): bf16 U (A of (3)); [16q+8, 16q+16): decayed U (A of (2))
-                        uint32_t w[16];
+                        // per 16 tokens: 8 columns of bf16 U (A of (3)), then 8 of the decayed U (A of (2))
 #pragma unroll
-                        for (int e = 0; e < 8; ++e) {
-                            w[e] = gdn::pack_bf16x2(u[2 * e], u[2 * e + 1]);
-                            w[8 + e] = gdn::pack_bf16x2(u[2 * e] * d[2 * e], u[2 * e + 1] * d[2 * e + 1]);
+                        for (int h = 0; h < 2; ++h) {
+                            const int t0 = 32 * q + 16 * h;
+                            float d[16];
+#pragma unroll
+                            for (int e = 0; e < 16; e += 4) {
+                                const float4 d4 = ld4(ga + GA_DEC + t0 + e);
+                                const float4 k4 = ld4(ga + GA_RK + t0 + e);
+                                d[e] = d4.x * k4.x; d[e + 1] = d4.y * k4.y; d[e + 2] = d4.z * k4.z; d[e + 3] = d4.w * k4.w;
+                            }
+                            uint32_t w[16];
+#pragma unroll
+                            for (int e = 0; e < 8; ++e) {
+                                w[e] = gdn::pack_bf16x2(u[16 * h + 2 * e], u[16 * h + 2 * e + 1]);
+                                w[8 + e] = gdn::pack_bf16x2(u[16 * h + 2 * e] * d[2 * e], u[16 * h + 2 * e + 1] * d[2 * e + 1]);
+                            }
+                            tmem_st16u(tl + TM_U + t0, w);
                         }
-                        tmem_st16u(tl + TM_U + 16 * q, w);
                     }
                     tmem_wait_st();
                     if (dv < 64) ogr[dv] = ga[GA_GAM + dv] * ga[GA_RQ + dv];
@@ -1032,21 +1040,21 @@ __global__ void __launch_bounds__(NTHREADS, 1) gdn_prefill_chunk_kernel(const __
                         gC1 = reinterpret_cast<const float *>(smem + OFF_GATE + gs1 * GATE_BYTES)[GA_GC];
                     }
 #pragma unroll 1
-                    for (int q = 0; q < 8; ++q) {
-                        float x[16];
-                        tmem_ld16(tl + TM_S + 16 * q, x);
+                    for (int q = 0; q < 4; ++q) {
+                        float x[32];
+                        tmem_ld32(tl + TM_S + 32 * q, x);
                         tmem_wait_ld();
                         if (more) {
-                            uint32_t w[8];
+                            uint32_t w[16];
 #pragma unroll
-                            for (int e = 0; e < 8; ++e) w[e] = gdn::pack_bf16x2(x[2 * e], x[2 * e + 1]);
-                            tmem_st8u(tl + TM_SB + 8 * q, w);
+                            for (int e = 0; e < 16; ++e) w[e] = gdn::pack_bf16x2(x[2 * e], x[2 * e + 1]);
+                            tmem_st16u(tl + TM_SB + 16 * q, w);
 #pragma unroll
-                            for (int e = 0; e < 16; ++e) x[e] *= gC1;
-                            tmem_st16(tl + TM_S + 16 * q, x);
+                            for (int e = 0; e < 32; ++e) x[e] *= gC1;
+                            tmem_st32(tl + TM_S + 32 * q, x);
                         } else {
 #pragma unroll
-                            for (int c = 0; c < 16; c += 4) st4(fin + 16 * q + c, x[c], x[c + 1], x[c + 2], x[c + 3]);
+                            for (int c = 0; c < 32; c += 4) st4(fin + 32 * q + c, x[c], x[c + 1], x[c + 2], x[c + 3]);
                         }
                     }
                     if (more) {
@@ -1073,21 +1081,18 @@ __global__ void __launch_bounds__(NTHREADS, 1) gdn_prefill_chunk_kernel(const __
                         const int64_t ostride8 = (int64_t)8 * p.Hv * D;
 #pragma unroll 1
                         for (int q = 0; q < 4; ++q) {
-                            float y[16], z[16], gg[16];
+                            float y[16], z[16];
                             tmem_ld16(tl + TM_Y + 16 * q, y);
                             tmem_ld16(tl + TM_Z + 16 * q, z);
-#pragma unroll
-                            for (int e = 0; e < 16; e += 4) {
-                                const float4 g4 = ld4(ogr + 16 * q + e);
-                                gg[e] = g4.x; gg[e + 1] = g4.y; gg[e + 2] = g4.z; gg[e + 3] = g4.w;
-                            }
                             tmem_wait_ld();
 #pragma unroll
                             for (int hb = 0; hb < 2; ++hb) {
+                                const float4 g0 = ld4(ogr + 16 * q + 8 * hb), g1 = ld4(ogr + 16 * q + 8 * hb + 4);
+                                const float gg[8] = {g0.x, g0.y, g0.z, g0.w, g1.x, g1.y, g1.z, g1.w};
 #pragma unroll
                                 for (int e = 0; e < 8; ++e)
                                     *reinterpret_cast<__nv_bfloat16 *>(ost + e * 64 + lane * 2) =
-                                        __float2bfloat16_rn(sc * fmaf(gg[8 * hb + e], y[8 * hb + e], z[8 * hb + e]));
+                                        __float2bfloat16_rn(sc * fmaf(gg[e], y[8 * hb + e], z[8 * hb + e]));
                                 __syncwarp();
                                 const uint4 v = *reinterpret_cast<const uint4 *>(ost + lane * 16);
                                 __syncwarp();
