@@ -44,7 +44,7 @@ def _load():
         lib.oracle_prefill.argtypes = [
             D, D, D, D, D, I32, D, D, D,
             ctypes.c_int, ctypes.c_int64, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int,
-            ctypes.c_double, ctypes.c_int, ctypes.c_int,
+            ctypes.c_double, ctypes.c_int, ctypes.c_int, D, D, ctypes.c_int, ctypes.c_int,
         ]
         lib.oracle_decode.restype = None
         lib.oracle_decode.argtypes = [
@@ -79,18 +79,34 @@ def _ip(a):
     return None if a is None else a.ctypes.data_as(ctypes.POINTER(ctypes.c_int32))
 
 
+RULES = {"gated_delta": 0, "gated": 1, "delta": 2, "linear": 3}
+
+
 def prefill(q, k, v, g, beta, cu_seqlens=None, initial_state=None, *, B=None,
-            scale=1.0, qk_l2norm=False, out=None, threads=None):
+            scale=1.0, qk_l2norm=False, out=None, threads=None, update_rule="gated_delta",
+            gate_activation="none", a_log=None, dt_bias=None, beta_activation="none"):
     """Sequential recurrence of the log-space form, float64.
 
-    q, k: [N, Hq, Dk]; v: [N, Hv, Dv]; g, beta: [N, Hv];
-    cu_seqlens: [B+1] int32 or None (uniform packing, needs ``B``);
-    initial_state: [B, Hv, Dv, Dk] or None.
+    q, k: [N, Hq, Dk]; v: [N, Hv, Dv]; g, beta: [N, Hv] (None where the update
+    rule has no decay / no retrieval); cu_seqlens: [B+1] int32 or None (uniform
+    packing, needs ``B``); initial_state: [B, Hv, Dv, Dk] or None.
+    update_rule: gated_delta | gated | delta | linear; gate_activation: none |
+    qwen (needs a_log, dt_bias [Hv]); beta_activation: none | sigmoid.
     ``out`` (optional, [N, Hv, Dv] float64) supplies the values kept for
     tokens that no request covers.
     Returns (out [N, Hv, Dv], final_state [B, Hv, Dv, Dk]) as float64.
     """
-    q, k, v, g, beta = map(_f64, (q, k, v, g, beta))
+    rule = RULES[update_rule]
+    has_decay, has_retr = rule in (0, 1), rule in (0, 2)
+    assert (g is not None) == has_decay and (beta is not None) == has_retr
+    assert gate_activation in ("none", "qwen") and beta_activation in ("none", "sigmoid")
+    qwen = gate_activation == "qwen"
+    assert not qwen or (has_decay and a_log is not None and dt_bias is not None)
+    q, k, v = map(_f64, (q, k, v))
+    g = None if g is None else _f64(g)
+    beta = None if beta is None else _f64(beta)
+    al = _f64(a_log) if qwen else None
+    dtb = _f64(dt_bias) if qwen else None
     N, Hq, Dk = q.shape
     Hv, Dv = v.shape[1], v.shape[2]
     if cu_seqlens is not None:
@@ -105,7 +121,8 @@ def prefill(q, k, v, g, beta, cu_seqlens=None, initial_state=None, *, B=None,
     nt = threads if threads is not None else max_threads()
     _load().oracle_prefill(_dp(q), _dp(k), _dp(v), _dp(g), _dp(beta), _ip(cu), _dp(s0),
                            _dp(fs), _dp(o), B, N, Hq, Hv, Dk, Dv, float(scale),
-                           int(bool(qk_l2norm)), int(nt))
+                           int(bool(qk_l2norm)), rule, _dp(al), _dp(dtb),
+                           int(beta_activation == "sigmoid"), int(nt))
     return o, fs
 
 

@@ -16,7 +16,12 @@
  *      o_t = scale * S_t^T q_t, per value head; value head h reads query/key
  *      head h*Hq/Hv; Inputs table: cu_seqlens clamping, V-major float32
  *      initial/final state, empty requests copy their state through;
- *      Attributes table: qk_l2_norm with epsilon 1e-12, scale.
+ *      Attributes table: qk_l2_norm with epsilon 1e-12, scale; update_rule
+ *      (linear drops the decay and the delta retrieval, gated keeps only the
+ *      decay, delta only the retrieval, gated_delta both; decay is an input
+ *      exactly for gated / gated_delta, beta exactly for delta / gated_delta);
+ *      gate_activation qwen: g = -exp(a_log) * softplus(decay + dt_bias);
+ *      beta_activation sigmoid.
  *  - "Gated DeltaNet State Update" (tensortonic), statement: the same
  *      recurrence in the gamma form S_t = gamma_t (I - beta_t k_t k_t^T)
  *      S_{t-1} + beta_t k_t v_t^T with y_t = q_t^T S_t (gamma_t = exp(g_t)).
@@ -33,7 +38,11 @@
  *    (pool_in) and writes into a separate copy (pool_out); under the
  *    precondition that no row writes a slot another row reads, this is the
  *    in-place result;
- *  - a slot index >= pool_size is treated like a negative one (skipped).
+ *  - a slot index >= pool_size is treated like a negative one (skipped);
+ *  - an update rule without beta writes k_t v_t^T (beta = 1); one without
+ *    the retrieval drops the -exp(g_t) S_{t-1}^T k_t term; one without decay
+ *    uses g_t = 0;
+ *  - the prefill qwen gate uses the decode page's softplus threshold 20.
  *
  * Parity pins: tests/test_oracle_pins.py checks this file against the worked
  * examples of "Gated DeltaNet State Update", a brute-force product of the
@@ -62,11 +71,18 @@ int oracle_max_threads(void)
 #endif
 }
 
+static double softplus20(double x) { return x > 20.0 ? x : log1p(exp(x)); }
+
 /* ------------------------------------------------------------------------
  * Prefill.
  *   q, k          [N, Hq, Dk]
  *   v, out        [N, Hv, Dv]
- *   g, beta       [N, Hv]            (log-space decay, update rate)
+ *   g, beta       [N, Hv]            (log-space decay, update rate); g is NULL
+ *                                    for rules without decay, beta for rules
+ *                                    without retrieval
+ *   rule          0 gated_delta, 1 gated, 2 delta, 3 linear
+ *   a_log, dt_bias [Hv] or NULL      (non-NULL: qwen gate on g)
+ *   beta_sigmoid  non-zero: beta <- sigmoid(beta)
  *   cu_seqlens    [B+1] or NULL      (NULL: uniform packing, N = B*S)
  *   initial_state [B, Hv, Dv, Dk] or NULL (NULL: zero)
  *   final_state   [B, Hv, Dv, Dk]
@@ -80,9 +96,13 @@ void oracle_prefill(const double *q, const double *k, const double *v,
                     const double *initial_state, double *final_state,
                     double *out,
                     int B, int64_t N, int Hq, int Hv, int Dk, int Dv,
-                    double scale, int qk_l2norm, int nthreads)
+                    double scale, int qk_l2norm, int rule,
+                    const double *a_log, const double *dt_bias, int beta_sigmoid,
+                    int nthreads)
 {
     int nunits = B * Hv;
+    const int has_decay = rule == 0 || rule == 1;
+    const int has_retrieval = rule == 0 || rule == 2;
     if (nthreads <= 0) nthreads = 1;
 
 #pragma omp parallel for schedule(dynamic, 1) num_threads(nthreads)
@@ -135,8 +155,18 @@ void oracle_prefill(const double *q, const double *k, const double *v,
                     xk[i] *= rk;
                 }
             }
-            double gamma = exp(g[t * Hv + h]);
-            double bt = beta[t * Hv + h];
+            /* gate: log-space decay (qwen form if requested), update rate */
+            double lg = 0.0;
+            if (has_decay) {
+                lg = g[t * Hv + h];
+                if (a_log) lg = -exp(a_log[h]) * softplus20(lg + dt_bias[h]);
+            }
+            double gamma = exp(lg);
+            double bt = 1.0;
+            if (has_retrieval) {
+                bt = beta[t * Hv + h];
+                if (beta_sigmoid) bt = 1.0 / (1.0 + exp(-bt));
+            }
 
             /* p = S_{t-1}^T k_t */
             for (int j = 0; j < Dv; ++j) {
@@ -144,10 +174,11 @@ void oracle_prefill(const double *q, const double *k, const double *v,
                 for (int i = 0; i < Dk; ++i) acc += S[(int64_t)i * Dv + j] * xk[i];
                 p[j] = acc;
             }
-            /* S_t = gamma S_{t-1} + k_t (beta (v_t - gamma p))^T */
+            /* S_t = gamma S_{t-1} + k_t (beta (v_t - gamma p))^T; without the
+             * retrieval the written value is beta v_t */
             for (int i = 0; i < Dk; ++i)
                 for (int j = 0; j < Dv; ++j) {
-                    double u = bt * (vt[j] - gamma * p[j]);
+                    double u = bt * (vt[j] - (has_retrieval ? gamma * p[j] : 0.0));
                     S[(int64_t)i * Dv + j] = gamma * S[(int64_t)i * Dv + j] + xk[i] * u;
                 }
             /* o_t = scale * S_t^T q_t */

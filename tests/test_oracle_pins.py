@@ -348,3 +348,123 @@ def test_decode_equals_prefill_with_restated_gate(oracle_mod):
     op, fp = oracle_mod.prefill(q[0], k[0, :, 0], v[0, :, 0], g, beta, None, pool, B=1, scale=0.3)
     np.testing.assert_allclose(od[0], op, rtol=1e-10, atol=1e-13)
     np.testing.assert_allclose(pd, fp, rtol=1e-10, atol=1e-13)
+
+
+# ------------------------------------------- update rules, gate and beta activations
+# "com.microsoft.GatedDeltaNet", Attributes table: update_rule keeps or drops the decay and
+# the delta retrieval; gate_activation qwen maps the decay input to
+# -exp(a_log) * softplus(decay + dt_bias); beta_activation sigmoid.  Pinned here against
+# closed forms of the rules without retrieval (causal sums of decayed outer products),
+# the gamma-form brute force with gamma = 1, and special gate values.
+def _rand_case(seed, N, Dk, Dv, unit_keys=True):
+    rng = np.random.default_rng(seed)
+    q = rng.standard_normal((N, 1, Dk))
+    k = rng.standard_normal((N, 1, Dk))
+    if unit_keys:
+        k /= np.linalg.norm(k, axis=-1, keepdims=True)
+    v = rng.standard_normal((N, 1, Dv))
+    init = rng.standard_normal((1, 1, Dv, Dk))
+    return rng, q, k, v, init
+
+
+def _decayed_sum_closed_form(q, k, v, G, S0k, scale):
+    """out_t = scale (exp(G_t) S0^T q_t + sum_{j<=t} exp(G_t - G_j) (k_j . q_t) v_j) and the
+    final state exp(G_T) S0 + sum_j exp(G_T - G_j) k_j v_j^T (K-major), as masked products."""
+    N = q.shape[0]
+    Q, K, V = q[:, 0], k[:, 0], v[:, 0]
+    D = np.exp(G[:, None] - G[None, :]) * np.tril(np.ones((N, N)))
+    out = scale * (np.exp(G)[:, None] * (Q @ S0k) + (D * (Q @ K.T)) @ V)
+    fin = np.exp(G[-1]) * S0k + (np.exp(G[-1] - G)[:, None] * K).T @ V
+    return out, fin
+
+
+def test_rule_linear_is_causal_linear_attention(oracle_mod):
+    _, q, k, v, init = _rand_case(201, 11, 6, 4, unit_keys=False)
+    out, fs = oracle_mod.prefill(q, k, v, None, None, None, init, B=1, scale=0.7,
+                                 update_rule="linear")
+    ro, rf = _decayed_sum_closed_form(q, k, v, np.zeros(11), init[0, 0].T, 0.7)
+    np.testing.assert_allclose(out[:, 0], ro, rtol=1e-11, atol=1e-12)
+    np.testing.assert_allclose(fs[0, 0], rf.T, rtol=1e-11, atol=1e-12)
+
+
+def test_rule_gated_is_decayed_linear_attention(oracle_mod):
+    rng, q, k, v, init = _rand_case(202, 13, 5, 3, unit_keys=False)
+    g = -rng.uniform(0.0, 1.0, (13, 1))
+    out, fs = oracle_mod.prefill(q, k, v, g, None, None, init, B=1, scale=1.3,
+                                 update_rule="gated")
+    ro, rf = _decayed_sum_closed_form(q, k, v, np.cumsum(g[:, 0]), init[0, 0].T, 1.3)
+    np.testing.assert_allclose(out[:, 0], ro, rtol=1e-10, atol=1e-12)
+    np.testing.assert_allclose(fs[0, 0], rf.T, rtol=1e-10, atol=1e-12)
+
+
+@pytest.mark.parametrize("l2norm", [False, True])
+def test_rule_delta_is_gamma_form_with_gamma_one(oracle_mod, l2norm):
+    rng, q, k, v, init = _rand_case(203 + int(l2norm), 9, 6, 4, unit_keys=not l2norm)
+    beta = rng.uniform(0.0, 1.0, (9, 1))
+    out, fs = oracle_mod.prefill(q, k, v, None, beta, None, init, B=1, scale=0.5,
+                                 qk_l2norm=l2norm, update_rule="delta")
+    ro, rf = brute_prefill(q, k, v, np.zeros((9, 1)), beta, [9], init, 0.5, l2norm, 1, 1)
+    np.testing.assert_allclose(out, ro, rtol=1e-11, atol=1e-12)
+    np.testing.assert_allclose(fs, rf, rtol=1e-11, atol=1e-12)
+
+
+def test_qwen_gate_reproduces_worked_example_two(oracle_mod):
+    """a_log = 0, dt_bias = 0, decay = 0 gives g = -softplus(0) = -ln 2, i.e. gamma = 0.5 on
+    every token: the page's second worked example (4 stored, then halved to 2) with the first
+    token's gate replaced by the same 0.5 and beta_1 = 0."""
+    e = json.load(open(GOLDEN))["examples"][1]
+    q = np.array(e["q"], np.float64).reshape(2, 1, 2)
+    k = np.array(e["k"], np.float64).reshape(2, 1, 2)
+    v = np.array(e["v"], np.float64).reshape(2, 1, 2)
+    beta = np.array(e["beta"], np.float64).reshape(2, 1)
+    out, fs = oracle_mod.prefill(q, k, v, np.zeros((2, 1)), beta, None, None, B=1, scale=1.0,
+                                 gate_activation="qwen", a_log=np.zeros(1), dt_bias=np.zeros(1))
+    # token 0: S = 0.5*0 + k(1*(4 - 0)) -> 4; token 1: S = 0.5*4, beta = 0 -> 2
+    np.testing.assert_allclose(out[:, 0], np.array(e["outputs"])[0], atol=1e-12)
+    np.testing.assert_allclose(fs[0, 0].T, np.array(e["final_state"])[0], atol=1e-12)
+
+
+def test_qwen_gate_closed_form_decay(oracle_mod):
+    """beta = 0 leaves only the decay: exp(a_log) = 2 with decay + dt_bias = 0 gives
+    gamma = 2^-2 per token; decay + dt_bias = 30 lies above the softplus threshold, so with
+    exp(a_log) = ln(2)/30 the gate is again exactly 0.5."""
+    rng, q, k, v, init = _rand_case(205, 6, 4, 3)
+    for a_log, dec, dtb, gam in [(np.log(2.0), -0.75, 0.75, 0.25), (np.log(np.log(2.0) / 30.0),
+                                                                    29.0, 1.0, 0.5)]:
+        out, fs = oracle_mod.prefill(q, k, v, np.full((6, 1), dec), np.zeros((6, 1)), None, init,
+                                     B=1, scale=1.0, gate_activation="qwen",
+                                     a_log=np.array([a_log]), dt_bias=np.array([dtb]))
+        decay = gam ** np.arange(1, 7)
+        np.testing.assert_allclose(out[:, 0], decay[:, None] * (q[:, 0] @ init[0, 0].T),
+                                   rtol=1e-12, atol=1e-14)
+        np.testing.assert_allclose(fs[0, 0], gam ** 6 * init[0, 0], rtol=1e-12, atol=1e-14)
+
+
+def test_beta_sigmoid_special_values(oracle_mod):
+    """sigmoid(0) = 1/2 exactly (gamma-form brute force with beta = 0.5); a large positive
+    input saturates to 1 (unit key, q = k: the output is the value, the overwrite rule of the
+    first worked example); a large negative one to 0 (only the decay remains)."""
+    rng, q, k, v, init = _rand_case(206, 8, 5, 3)
+    g = -rng.uniform(0.0, 1.0, (8, 1))
+    out, fs = oracle_mod.prefill(q, k, v, g, np.zeros((8, 1)), None, init, B=1, scale=1.0,
+                                 beta_activation="sigmoid")
+    ro, rf = brute_prefill(q, k, v, g, np.full((8, 1), 0.5), [8], init, 1.0, False, 1, 1)
+    np.testing.assert_allclose(out, ro, rtol=1e-11, atol=1e-12)
+    np.testing.assert_allclose(fs, rf, rtol=1e-11, atol=1e-12)
+    out, _ = oracle_mod.prefill(k, k, v, g, np.full((8, 1), 60.0), None, init, B=1, scale=1.0,
+                                beta_activation="sigmoid")
+    np.testing.assert_allclose(out, v, rtol=1e-11, atol=1e-12)
+    out, fs = oracle_mod.prefill(q, k, v, g, np.full((8, 1), -60.0), None, init, B=1, scale=1.0,
+                                 beta_activation="sigmoid")
+    cum = np.cumsum(g[:, 0])
+    np.testing.assert_allclose(out[:, 0], np.exp(cum)[:, None] * (q[:, 0] @ init[0, 0].T),
+                               rtol=1e-11, atol=1e-13)
+
+
+def test_rule_inputs_are_checked(oracle_mod):
+    _, q, k, v, _ = _rand_case(207, 3, 2, 2)
+    z = np.zeros((3, 1))
+    with pytest.raises(AssertionError):
+        oracle_mod.prefill(q, k, v, z, z, None, None, B=1, update_rule="linear")
+    with pytest.raises(AssertionError):
+        oracle_mod.prefill(q, k, v, None, z, None, None, B=1, update_rule="gated_delta")
