@@ -29,10 +29,24 @@ GDN_ERR_CUDA = 7
 
 GDN_F32 = 0
 GDN_BF16 = 1
+GDN_F16 = 2
 
 GDN_PREFILL_SEQUENTIAL = 1
 GDN_DISABLE_STATE_UPDATE = 2
 GDN_DECODE_QK_L2NORM = 4
+GDN_RULE_GATED = 1 << 3
+GDN_RULE_DELTA = 2 << 3
+GDN_RULE_LINEAR = 3 << 3
+GDN_GATE_QWEN = 1 << 5
+GDN_BETA_SIGMOID = 1 << 6
+
+# update_rule of the op -> (flag bits, has decay input, has beta input)
+UPDATE_RULES = {
+    "gated_delta": (0, True, True),
+    "gated": (GDN_RULE_GATED, True, False),
+    "delta": (GDN_RULE_DELTA, False, True),
+    "linear": (GDN_RULE_LINEAR, False, False),
+}
 
 GDN_DEV_BAD_SLOT = 1
 GDN_DEV_TIMEOUT = 2
@@ -66,7 +80,7 @@ def lib():
         vp, i32, i64, u32, f32 = (ctypes.c_void_p, ctypes.c_int32, ctypes.c_int64,
                                   ctypes.c_uint32, ctypes.c_float)
         L.gdn_prefill.restype = ctypes.c_int
-        L.gdn_prefill.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp,
+        L.gdn_prefill.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp,
                                   i32, i64, i32, i32, i32, i32, ctypes.c_int, f32, i32, u32,
                                   vp, vp]
         L.gdn_decode.restype = ctypes.c_int
@@ -88,7 +102,7 @@ def lib():
 def prefill_uses_chunked(dtype: torch.dtype, Hv: int, Dk: int, Dv: int,
                          sequential: bool = False) -> bool:
     """True when gdn_prefill would run the chunked tensor-core kernel for these sizes."""
-    code = GDN_BF16 if dtype == torch.bfloat16 else GDN_F32
+    code = {torch.bfloat16: GDN_BF16, torch.float16: GDN_F16}.get(dtype, GDN_F32)
     return bool(lib().gdn_prefill_uses_chunked(code, Hv, Dk, Dv,
                                                GDN_PREFILL_SEQUENTIAL if sequential else 0))
 
@@ -119,14 +133,30 @@ def _check_cuda(name, t, dtype=None):
 
 def gdn_prefill(q, k, v, g, beta, cu_seqlens=None, initial_state=None, final_state=None,
                 out=None, *, num_requests: Optional[int] = None, scale: Optional[float] = None,
-                qk_l2norm: bool = False, sequential: bool = False, dev_status=None, stream=None):
+                qk_l2norm: bool = False, sequential: bool = False, update_rule: str = "gated_delta",
+                gate_activation: str = "none", a_log=None, dt_bias=None,
+                beta_activation: str = "none", dev_status=None, stream=None):
     """Gated DeltaNet prefill (log-space form) over ragged requests.
 
     q, k: [N, Hq, Dk] or [B, S, Hq, Dk]; v: [N, Hv, Dv] (same leading axes);
-    g, beta: [N, Hv] fp32; cu_seqlens: [B+1] int32 (rank-3 form) or None;
-    initial_state: [B, Hv, Dv, Dk] fp32 or None.  ``scale`` None or 0 selects
-    1/sqrt(Dk).  Returns (out, final_state).
+    activations fp32, bf16 or fp16; g, beta: [N, Hv] fp32 (g None for the rules
+    without decay, beta None for those without retrieval); cu_seqlens: [B+1]
+    int32 (rank-3 form) or None; initial_state: [B, Hv, Dv, Dk] fp32 or None.
+    update_rule: gated_delta | gated | delta | linear; gate_activation: none |
+    qwen (a_log, dt_bias: [Hv] fp32); beta_activation: none | sigmoid.
+    ``scale`` None or 0 selects 1/sqrt(Dk).  Returns (out, final_state).
     """
+    if update_rule not in UPDATE_RULES:
+        raise ValueError(f"unknown update_rule {update_rule!r}")
+    if gate_activation not in ("none", "qwen") or beta_activation not in ("none", "sigmoid"):
+        raise ValueError("gate_activation must be none|qwen and beta_activation none|sigmoid")
+    rule_flags, has_decay, has_beta = UPDATE_RULES[update_rule]
+    if (g is not None) != has_decay or (beta is not None) != has_beta:
+        raise ValueError(f"update_rule {update_rule!r} takes "
+                         f"{'a' if has_decay else 'no'} decay and {'a' if has_beta else 'no'} beta")
+    qwen = gate_activation == "qwen"
+    if qwen != (a_log is not None and dt_bias is not None):
+        raise ValueError("gate_activation 'qwen' requires a_log and dt_bias (and only it takes them)")
     if q.dim() == 4:
         Bq, S = q.shape[0], q.shape[1]
         if cu_seqlens is not None:
@@ -135,27 +165,29 @@ def gdn_prefill(q, k, v, g, beta, cu_seqlens=None, initial_state=None, final_sta
         q = q.reshape(Bq * S, *q.shape[2:])
         k = k.reshape(Bq * S, *k.shape[2:])
         v = v.reshape(Bq * S, *v.shape[2:])
-        g = g.reshape(Bq * S, -1)
-        beta = beta.reshape(Bq * S, -1)
+        g = None if g is None else g.reshape(Bq * S, -1)
+        beta = None if beta is None else beta.reshape(Bq * S, -1)
         if out is not None:
             out = out.view(Bq * S, *out.shape[2:])
-    if q.dtype == torch.bfloat16:
-        dt = GDN_BF16
-    elif q.dtype == torch.float32:
-        dt = GDN_F32
-    else:
+    dt = {torch.bfloat16: GDN_BF16, torch.float32: GDN_F32, torch.float16: GDN_F16}.get(q.dtype)
+    if dt is None:
         raise TypeError(f"unsupported activation dtype {q.dtype}")
     q = _check_cuda("q", q, q.dtype)
     k = _check_cuda("k", k, q.dtype)
     v = _check_cuda("v", v, q.dtype)
     g = _check_cuda("g", g, torch.float32)
     beta = _check_cuda("beta", beta, torch.float32)
+    a_log = _check_cuda("a_log", a_log, torch.float32)
+    dt_bias = _check_cuda("dt_bias", dt_bias, torch.float32)
     cu_seqlens = _check_cuda("cu_seqlens", cu_seqlens, torch.int32)
     initial_state = _check_cuda("initial_state", initial_state, torch.float32)
     N, Hq, Dk = q.shape
     Hv, Dv = v.shape[1], v.shape[2]
-    if k.shape != q.shape or v.shape[0] != N or g.shape != (N, Hv) or beta.shape != (N, Hv):
+    if k.shape != q.shape or v.shape[0] != N or (g is not None and g.shape != (N, Hv)) or \
+            (beta is not None and beta.shape != (N, Hv)):
         raise ValueError("inconsistent q/k/v/g/beta shapes")
+    if qwen and (a_log.shape != (Hv,) or dt_bias.shape != (Hv,)):
+        raise ValueError("a_log and dt_bias must be [Hv]")
     if cu_seqlens is not None:
         B = cu_seqlens.shape[0] - 1
     else:
@@ -174,8 +206,10 @@ def gdn_prefill(q, k, v, g, beta, cu_seqlens=None, initial_state=None, final_sta
         raise ValueError("initial_state must be [B, Hv, Dv, Dk]")
     if scale is None or scale == 0.0:
         scale = 1.0 / math.sqrt(Dk)
-    flags = GDN_PREFILL_SEQUENTIAL if sequential else 0
-    st = lib().gdn_prefill(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(cu_seqlens),
+    flags = (GDN_PREFILL_SEQUENTIAL if sequential else 0) | rule_flags
+    flags |= (GDN_GATE_QWEN if qwen else 0) | (GDN_BETA_SIGMOID if beta_activation == "sigmoid" else 0)
+    st = lib().gdn_prefill(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(a_log),
+                           _ptr(dt_bias), _ptr(cu_seqlens),
                            _ptr(initial_state), _ptr(final_state), _ptr(out), B, N, Hq, Hv, Dk,
                            Dv, dt, float(scale), int(bool(qk_l2norm)), flags, _ptr(dev_status),
                            _stream(stream))

@@ -64,6 +64,8 @@ __device__ __forceinline__ float softplus20(float x)
     return x > 20.f ? x : log1pf(expf(x));
 }
 
+__device__ __forceinline__ float sigmoidf_(float x) { return 1.0f / (1.0f + expf(-x)); }
+
 }  // namespace gdn
 
 // Launchers implemented by the kernel translation units.
@@ -81,6 +83,11 @@ struct GdnPrefillArgs {
     float scale;
     int32_t qk_l2norm;
     int32_t *dev_status;
+    // update_rule of the op: which of the decay and the delta retrieval survive; a rule
+    // without decay has g == NULL (g = 0), one without retrieval has beta == NULL (beta = 1)
+    int32_t has_decay, has_retrieval;
+    const float *a_log, *dt_bias;   // non-NULL: qwen gate on g
+    int32_t beta_sigmoid;
 };
 
 struct GdnDecodeArgs {

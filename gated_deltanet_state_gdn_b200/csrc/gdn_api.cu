@@ -64,21 +64,34 @@ int32_t gdn_prefill_uses_chunked(gdn_dtype dtype, int32_t Hv, int32_t Dk, int32_
 }
 
 gdn_status gdn_prefill(const void *q, const void *k, const void *v, const float *g,
-                       const float *beta, const int32_t *cu_seqlens, const float *initial_state,
+                       const float *beta, const float *a_log, const float *dt_bias,
+                       const int32_t *cu_seqlens, const float *initial_state,
                        float *final_state, void *out, int32_t B, int64_t N, int32_t Hq,
                        int32_t Hv, int32_t Dk, int32_t Dv, gdn_dtype dtype, float scale,
                        int32_t qk_l2norm, uint32_t flags, int32_t *dev_status, void *stream)
 {
-    if (dtype != GDN_F32 && dtype != GDN_BF16) return GDN_ERR_DTYPE;
+    if (dtype != GDN_F32 && dtype != GDN_BF16 && dtype != GDN_F16) return GDN_ERR_DTYPE;
     if (B < 0 || N < 0 || Hq < 1 || Hv < 1 || Dk < 1 || Dv < 1) return GDN_ERR_SHAPE;
     if (Hv % Hq != 0) return GDN_ERR_SHAPE;
     if (Dk > 256 || Dv > 256) return GDN_ERR_UNSUPPORTED;
-    if (flags & ~(uint32_t)GDN_PREFILL_SEQUENTIAL) return GDN_ERR_UNSUPPORTED;
+    const uint32_t known = GDN_PREFILL_SEQUENTIAL | GDN_RULE_MASK | GDN_GATE_QWEN | GDN_BETA_SIGMOID;
+    if (flags & ~known) return GDN_ERR_UNSUPPORTED;
+    // update_rule: decay input exactly for gated / gated_delta, beta exactly for delta /
+    // gated_delta, qwen parameters exactly with the qwen gate (which needs a decay)
+    const uint32_t rule = flags & GDN_RULE_MASK;
+    const bool has_decay = rule == 0 || rule == GDN_RULE_GATED;
+    const bool has_retrieval = rule == 0 || rule == GDN_RULE_DELTA;
+    const bool qwen = (flags & GDN_GATE_QWEN) != 0;
+    if (qwen && !has_decay) return GDN_ERR_SHAPE;
+    if ((flags & GDN_BETA_SIGMOID) && !has_retrieval) return GDN_ERR_SHAPE;
     if (B == 0) return N == 0 ? GDN_OK : GDN_ERR_SHAPE;
     if (!cu_seqlens && N % B != 0) return GDN_ERR_SHAPE;
     if (N > ((int64_t)1 << 31) - 1) return GDN_ERR_UNSUPPORTED;
     if (!final_state) return GDN_ERR_NULL;
-    if (N > 0 && (!q || !k || !v || !g || !beta || !out)) return GDN_ERR_NULL;
+    if (N > 0 && (!q || !k || !v || !out)) return GDN_ERR_NULL;
+    if (N > 0 && (has_decay != (g != nullptr) || has_retrieval != (beta != nullptr)))
+        return GDN_ERR_NULL;
+    if (qwen != (a_log != nullptr) || qwen != (dt_bias != nullptr)) return GDN_ERR_NULL;
 
     const size_t esz = dtype == GDN_F32 ? 4 : 2;
     const size_t qk_bytes = (size_t)N * Hq * Dk * esz;
@@ -87,7 +100,7 @@ gdn_status gdn_prefill(const void *q, const void *k, const void *v, const float 
     const size_t st_bytes = (size_t)B * Hv * Dv * Dk * 4;
     if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(out, 16) ||
         !aligned(initial_state, 16) || !aligned(final_state, 16) || !aligned(g, 4) ||
-        !aligned(beta, 4) || !aligned(cu_seqlens, 4))
+        !aligned(beta, 4) || !aligned(cu_seqlens, 4) || !aligned(a_log, 4) || !aligned(dt_bias, 4))
         return GDN_ERR_ALIGN;
     if (overlaps(initial_state, st_bytes, final_state, st_bytes)) return GDN_ERR_ALIAS;
     if (overlaps(out, v_bytes, q, qk_bytes) || overlaps(out, v_bytes, k, qk_bytes) ||
@@ -99,7 +112,10 @@ gdn_status gdn_prefill(const void *q, const void *k, const void *v, const float 
         overlaps(final_state, st_bytes, v, v_bytes) ||
         overlaps(final_state, st_bytes, g, gb_bytes) ||
         overlaps(final_state, st_bytes, beta, gb_bytes) ||
-        overlaps(final_state, st_bytes, cu_seqlens, (size_t)(B + 1) * 4))
+        overlaps(final_state, st_bytes, cu_seqlens, (size_t)(B + 1) * 4) ||
+        overlaps(out, v_bytes, a_log, (size_t)Hv * 4) || overlaps(out, v_bytes, dt_bias, (size_t)Hv * 4) ||
+        overlaps(final_state, st_bytes, a_log, (size_t)Hv * 4) ||
+        overlaps(final_state, st_bytes, dt_bias, (size_t)Hv * 4))
         return GDN_ERR_ALIAS;
 
     GdnPrefillArgs a;
@@ -107,6 +123,8 @@ gdn_status gdn_prefill(const void *q, const void *k, const void *v, const float 
     a.initial_state = initial_state; a.final_state = final_state; a.out = out;
     a.B = B; a.N = N; a.Hq = Hq; a.Hv = Hv; a.Dk = Dk; a.Dv = Dv; a.dtype = dtype;
     a.scale = scale; a.qk_l2norm = qk_l2norm ? 1 : 0; a.dev_status = dev_status;
+    a.has_decay = has_decay; a.has_retrieval = has_retrieval;
+    a.a_log = a_log; a.dt_bias = dt_bias; a.beta_sigmoid = (flags & GDN_BETA_SIGMOID) ? 1 : 0;
 
     cudaStream_t s = (cudaStream_t)stream;
     cudaError_t e;

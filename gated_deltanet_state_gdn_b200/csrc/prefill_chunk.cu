@@ -14,6 +14,10 @@
 //   U    = U~ - W S0
 //   O    = scale (diag(Gamma) Q^ S0 + P U),  P_ij = (q^_i . k^_j) exp(G_i - G_j) (j <= i)
 //   S_C  = Gamma_C S0 + (diag(exp(G_C - G)) K^)^T U
+// The op's update_rule variants reuse the same products: without decay g = 0;
+// without the delta retrieval A = 0 (T = I) and W = 0, so U = diag(beta) V with
+// beta = 1 (the rule has no beta input).  The qwen gate and the sigmoid beta
+// are applied to the per-token gate values before the prefix sum.
 // The norms rk, rq are never applied to the bf16 tiles: they fold into A, P,
 // the columns of T (for W), the decayed copy of U (for S_C) and the output
 // scale, so the tensor cores always read the caller's q/k bytes.
@@ -124,8 +128,8 @@ struct __align__(64) Params {
     CUtensorMap tm_q;     // (128, Hq, N) bf16, box (64, 1, 64), 128B swizzle
     CUtensorMap tm_k;
     CUtensorMap tm_v;     // (128, Hv, N)
-    CUtensorMap tm_g;     // (Hv, N) fp32, box (4, 64)
-    CUtensorMap tm_beta;
+    CUtensorMap tm_g;     // (Hv, N) fp32, box (4, 64); encoded only with a decay input
+    CUtensorMap tm_beta;  // encoded only with a beta input
     const int32_t *cu_seqlens;
     const float *initial_state;
     float *final_state;
@@ -135,6 +139,8 @@ struct __align__(64) Params {
     int32_t B, Hq, Hv;
     float scale;
     int32_t qk_l2norm;
+    int32_t has_decay, has_retrieval, beta_sigmoid;   // update rule and activations
+    const float *a_log, *dt_bias;                     // qwen gate when non-NULL
 };
 
 // --------------------------------------------------------------------------
@@ -361,7 +367,7 @@ __device__ __forceinline__ int t_slot(int I, int J)
 // exponent of an earlier block J is split as exp(G_i - Gend_J) exp(Gend_J - G_j),
 // both <= 1.
 __device__ __forceinline__ void build_row(uint32_t tl_gram, int qd, const float *ga, float *solve,
-                                          uint8_t *ptile)
+                                          uint8_t *ptile, bool retrieval)
 {
     const int lane = threadIdx.x & 31;
     const bool isP = qd >= 2;
@@ -370,7 +376,8 @@ __device__ __forceinline__ void build_row(uint32_t tl_gram, int qd, const float 
     const int i = 16 * I + r;
     const int jmax = 2 * (qd & 1) + 1;   // last diagonal block among the warp's rows
     const float G2i = ga[GA_G2 + i];
-    const float rowscale = isP ? ga[GA_RQ + i] : ga[GA_BETA + i] * ga[GA_RK + i];
+    // without the delta retrieval A = 0, so T = I
+    const float rowscale = isP ? ga[GA_RQ + i] : (retrieval ? ga[GA_BETA + i] * ga[GA_RK + i] : 0.f);
     float gend[3];
 #pragma unroll
     for (int J = 0; J < 3; ++J) gend[J] = ga[GA_GEND + J];
@@ -449,8 +456,8 @@ __global__ void __launch_bounds__(NTHREADS, 1) gdn_prefill_chunk_kernel(const __
         prefetch_tmap(&p.tm_q);
         prefetch_tmap(&p.tm_k);
         prefetch_tmap(&p.tm_v);
-        prefetch_tmap(&p.tm_g);
-        prefetch_tmap(&p.tm_beta);
+        if (p.has_decay) prefetch_tmap(&p.tm_g);
+        if (p.has_retrieval) prefetch_tmap(&p.tm_beta);
     }
     if (warp == MMA_WARP) {
         tmem_alloc(sbase + OFF_MISC, 512);
@@ -515,21 +522,21 @@ __global__ void __launch_bounds__(NTHREADS, 1) gdn_prefill_chunk_kernel(const __
                         const uint32_t gb = sbase + OFF_GB0 + ks * 2048;
                         const int t0 = un.start + n * C;
                         const uint32_t kb = cx.bar(B_KQ_FULL + ks);
-                        mbar_arrive_expect_tx(kb, 32768 + 2048);
+                        mbar_arrive_expect_tx(kb, 32768 + (p.has_decay ? 1024 : 0) + (p.has_retrieval ? 1024 : 0));
                         tma_load_3d(kq, &p.tm_k, kb, 0, qh, t0);
                         tma_load_3d(kq + KQ_KB, &p.tm_k, kb, 64, qh, t0);
                         tma_load_3d(kq + 8192, &p.tm_q, kb, 0, qh, t0);
                         tma_load_3d(kq + KQ_KB + 8192, &p.tm_q, kb, 64, qh, t0);
-                        tma_load_2d(gb, &p.tm_g, kb, un.h & ~3, t0);
-                        tma_load_2d(gb + 1024, &p.tm_beta, kb, un.h & ~3, t0);
+                        if (p.has_decay) tma_load_2d(gb, &p.tm_g, kb, un.h & ~3, t0);
+                        if (p.has_retrieval) tma_load_2d(gb + 1024, &p.tm_beta, kb, un.h & ~3, t0);
                         if (n + KQ_STAGES < nc) {
                             const int t2 = t0 + KQ_STAGES * C;
                             tma_prefetch_3d(&p.tm_k, 0, qh, t2);
                             tma_prefetch_3d(&p.tm_k, 64, qh, t2);
                             tma_prefetch_3d(&p.tm_q, 0, qh, t2);
                             tma_prefetch_3d(&p.tm_q, 64, qh, t2);
-                            tma_prefetch_2d(&p.tm_g, un.h & ~3, t2);
-                            tma_prefetch_2d(&p.tm_beta, un.h & ~3, t2);
+                            if (p.has_decay) tma_prefetch_2d(&p.tm_g, un.h & ~3, t2);
+                            if (p.has_retrieval) tma_prefetch_2d(&p.tm_beta, un.h & ~3, t2);
                         }
                     }
                     gc += nc;
@@ -770,10 +777,24 @@ __global__ void __launch_bounds__(NTHREADS, 1) gdn_prefill_chunk_kernel(const __
                         if (pw == 0) {
                             const int i0 = 2 * lane, i1 = i0 + 1;
                             const int hc = un.h & 3;
-                            const float g0 = i0 < len_n ? fmaxf(gtile[i0 * 4 + hc], G_FLOOR) : 0.f;
-                            const float g1 = i1 < len_n ? fmaxf(gtile[i1 * 4 + hc], G_FLOOR) : 0.f;
-                            const float b0 = i0 < len_n ? gtile[256 + i0 * 4 + hc] : 0.f;
-                            const float b1 = i1 < len_n ? gtile[256 + i1 * 4 + hc] : 0.f;
+                            // update rule: no decay -> g = 0; no retrieval -> beta = 1; qwen gate
+                            // -exp(a_log) softplus(decay + dt_bias) and sigmoid beta in fp32
+                            const float ea = p.a_log ? expf(__ldg(p.a_log + un.h)) : 0.f;
+                            const float dtb = p.a_log ? __ldg(p.dt_bias + un.h) : 0.f;
+                            auto gate = [&](int i) -> float {
+                                if (!p.has_decay || i >= len_n) return 0.f;
+                                float x = gtile[i * 4 + hc];
+                                if (p.a_log) x = -ea * gdn::softplus20(x + dtb);
+                                return fmaxf(x, G_FLOOR);
+                            };
+                            auto rate = [&](int i) -> float {
+                                if (i >= len_n) return 0.f;
+                                if (!p.has_retrieval) return 1.f;
+                                const float x = gtile[256 + i * 4 + hc];
+                                return p.beta_sigmoid ? gdn::sigmoidf_(x) : x;
+                            };
+                            const float g0 = gate(i0), g1 = gate(i1);
+                            const float b0 = rate(i0), b1 = rate(i1);
                             float x = g0 + g1;
 #pragma unroll
                             for (int o = 1; o < 32; o <<= 1) {
@@ -802,9 +823,11 @@ __global__ void __launch_bounds__(NTHREADS, 1) gdn_prefill_chunk_kernel(const __
                         ok = ok && cx.wait(B_G_DONE, p_g & 1);
                         ++p_g;
                         tc_fence_after();
-                        build_row(tl + TM_G, pw, ga, solve, smem + OFF_P + ks * P_STAGE);
+                        build_row(tl + TM_G, pw, ga, solve, smem + OFF_P + ks * P_STAGE, p.has_retrieval != 0);
                         if (pw >= 2) fence_proxy_async_smem();
-                        if (lt < 64) ga[GA_BG + lt] = ga[GA_BETA + lt] * ga[GA_GAM + lt] * ga[GA_RK + lt];
+                        // W = T diag(beta Gamma rk) K carries the retrieval term: zero without it
+                        if (lt < 64)
+                            ga[GA_BG + lt] = p.has_retrieval ? ga[GA_BETA + lt] * ga[GA_GAM + lt] * ga[GA_RK + lt] : 0.f;
                         tc_fence_before();
                         named_sync(1, 128);
                         if (lt == 0) {
@@ -1214,7 +1237,8 @@ cudaError_t launch_prefill_chunked(const GdnPrefillArgs &a, cudaStream_t stream)
         if (!make_map_3d_bf16(&p.tm_q, a.q, 128, a.Hq, N) ||
             !make_map_3d_bf16(&p.tm_k, a.k, 128, a.Hq, N) ||
             !make_map_3d_bf16(&p.tm_v, a.v, 128, a.Hv, N) ||
-            !make_map_2d_f32(&p.tm_g, a.g, a.Hv, N) || !make_map_2d_f32(&p.tm_beta, a.beta, a.Hv, N))
+            (a.has_decay && !make_map_2d_f32(&p.tm_g, a.g, a.Hv, N)) ||
+            (a.has_retrieval && !make_map_2d_f32(&p.tm_beta, a.beta, a.Hv, N)))
             return cudaErrorInvalidValue;
     }
     p.cu_seqlens = a.cu_seqlens;
@@ -1228,6 +1252,11 @@ cudaError_t launch_prefill_chunked(const GdnPrefillArgs &a, cudaStream_t stream)
     p.Hv = a.Hv;
     p.scale = a.scale;
     p.qk_l2norm = a.qk_l2norm;
+    p.has_decay = a.has_decay;
+    p.has_retrieval = a.has_retrieval;
+    p.beta_sigmoid = a.beta_sigmoid;
+    p.a_log = a.a_log;
+    p.dt_bias = a.dt_bias;
     const int units = a.B * a.Hv;
     const int grid = units < num_sms() ? units : num_sms();
     gdn_prefill_chunk_kernel<<<grid, NTHREADS, SMEM_BYTES, stream>>>(p);

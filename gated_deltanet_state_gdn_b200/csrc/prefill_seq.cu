@@ -7,11 +7,18 @@
 //   o_t = scale * S_t^T q_t
 // The state stays in fp32 registers for the whole request.
 //
-// This is the general path: fp32 or bf16 activations, any Dk, Dv in
+// The op's update_rule keeps or drops the decay (g = 0) and the delta
+// retrieval (the -exp(g_t) p term, with beta = 1 when the rule has no beta);
+// its qwen gate maps g to -exp(a_log[h]) softplus(g + dt_bias[h]) and its
+// sigmoid activation maps beta to sigmoid(beta), both in fp32.
+//
+// This is the general path: fp32, bf16 or fp16 activations, any Dk, Dv in
 // [1, 256], any Hq | Hv.  It is also the sequential counterpart the chunked
 // tensor-core kernel is checked against.  Layout: grid (B * Hv, Dv tiles of
 // 32 rows); a warp owns 4 V-rows of S (V-major, one row = Dk floats), lane l
 // owns elements l + 32 j of each row; row dot products are warp reductions.
+#include <cuda_fp16.h>
+
 #include "common.cuh"
 
 namespace gdn {
@@ -29,6 +36,12 @@ __device__ __forceinline__ float load_act<__nv_bfloat16>(const __nv_bfloat16 *p)
     return __bfloat162float(p[0]);
 }
 
+template <>
+__device__ __forceinline__ float load_act<__half>(const __half *p)
+{
+    return __half2float(p[0]);
+}
+
 template <typename Tout>
 __device__ __forceinline__ void store_act(Tout *p, float x);
 template <>
@@ -37,6 +50,11 @@ template <>
 __device__ __forceinline__ void store_act<__nv_bfloat16>(__nv_bfloat16 *p, float x)
 {
     *p = __float2bfloat16_rn(x);
+}
+template <>
+__device__ __forceinline__ void store_act<__half>(__half *p, float x)
+{
+    *p = __float2half_rn(x);
 }
 
 template <typename Tin, int EPL>
@@ -107,8 +125,17 @@ prefill_seq_kernel(const GdnPrefillArgs p)
                 qx[j] *= rq;
             }
         }
-        const float gamma = expf(__ldg(p.g + t * Hv + h));
-        const float bt = __ldg(p.beta + t * Hv + h);
+        float lg = 0.f, bt = 1.f;
+        if (p.has_decay) {
+            lg = __ldg(p.g + t * Hv + h);
+            if (p.a_log) lg = -expf(__ldg(p.a_log + h)) * softplus20(lg + __ldg(p.dt_bias + h));
+        }
+        if (p.has_retrieval) {
+            bt = __ldg(p.beta + t * Hv + h);
+            if (p.beta_sigmoid) bt = sigmoidf_(bt);
+        }
+        const float gamma = expf(lg);
+        const float rg = p.has_retrieval ? gamma : 0.f;   // weight of the retrieval term
         const int64_t vo = (t * Hv + h) * (int64_t)Dv;
 #pragma unroll
         for (int i = 0; i < R; ++i) {
@@ -119,7 +146,7 @@ prefill_seq_kernel(const GdnPrefillArgs p)
 #pragma unroll
             for (int j = 0; j < EPL; ++j) pd += S[i][j] * kx[j];
             pd = warp_sum(pd);
-            const float u = bt * (vi - gamma * pd);
+            const float u = bt * (vi - rg * pd);
             float o = 0.f;
 #pragma unroll
             for (int j = 0; j < EPL; ++j) {
@@ -164,5 +191,6 @@ cudaError_t launch_prefill_sequential(const GdnPrefillArgs &a, cudaStream_t stre
 {
     if (a.B == 0 || a.Hv == 0) return cudaSuccess;
     if (a.dtype == GDN_F32) return gdn::launch_seq_t<float>(a, stream);
+    if (a.dtype == GDN_F16) return gdn::launch_seq_t<__half>(a, stream);
     return gdn::launch_seq_t<__nv_bfloat16>(a, stream);
 }

@@ -27,6 +27,10 @@ def _f32(x: np.ndarray) -> torch.Tensor:
     return torch.from_numpy(np.ascontiguousarray(x, dtype=np.float32))
 
 
+def _f16(x: np.ndarray) -> torch.Tensor:
+    return torch.from_numpy(np.ascontiguousarray(x, dtype=np.float32)).to(torch.float16)
+
+
 def _unit_rows(x: np.ndarray) -> np.ndarray:
     """Scale each last-axis vector to unit L2 norm (input recipe, fp32)."""
     n = np.sqrt(np.sum(x.astype(np.float64) ** 2, axis=-1, keepdims=True))
@@ -125,7 +129,7 @@ def make_prefill(seed: int, lengths, Hq: int, Hv: int, Dk: int, Dv: int, *,
         cu = None
     else:
         cu = torch.from_numpy(np.concatenate([[0], np.cumsum(lengths)]).astype(np.int32))
-    conv = _bf16 if dtype == torch.bfloat16 else _f32
+    conv = {torch.bfloat16: _bf16, torch.float16: _f16}.get(dtype, _f32)
     return PrefillCase(name=name, q=conv(q), k=conv(k), v=conv(v), g=_f32(g), beta=_f32(beta),
                        cu_seqlens=cu, initial_state=init, B=B,
                        scale=(1.0 / np.sqrt(Dk)) if scale is None else float(scale),

@@ -52,14 +52,22 @@ typedef enum {
 
 typedef enum {
     GDN_F32 = 0,   /* float32 activations */
-    GDN_BF16 = 1   /* bfloat16 activations */
+    GDN_BF16 = 1,  /* bfloat16 activations */
+    GDN_F16 = 2    /* float16 activations (prefill, per-token kernel) */
 } gdn_dtype;
 
 /* flags */
 enum {
     GDN_PREFILL_SEQUENTIAL = 1u << 0,   /* prefill: force the per-token kernel */
     GDN_DISABLE_STATE_UPDATE = 1u << 1, /* decode: leave the pool unchanged */
-    GDN_DECODE_QK_L2NORM = 1u << 2      /* decode: L2-normalise q and k in the kernel */
+    GDN_DECODE_QK_L2NORM = 1u << 2,     /* decode: L2-normalise q and k in the kernel */
+    /* prefill update_rule (two bits; 0 = gated_delta, both terms) */
+    GDN_RULE_GATED = 1u << 3,           /* decay only: S_t = exp(g_t) S_{t-1} + k_t v_t^T */
+    GDN_RULE_DELTA = 2u << 3,           /* retrieval only: g = 0 */
+    GDN_RULE_LINEAR = 3u << 3,          /* neither: S_t = S_{t-1} + k_t v_t^T */
+    GDN_RULE_MASK = 3u << 3,
+    GDN_GATE_QWEN = 1u << 5,            /* prefill: g <- -exp(a_log[h]) softplus(g + dt_bias[h]) */
+    GDN_BETA_SIGMOID = 1u << 6          /* prefill: beta <- sigmoid(beta) */
 };
 
 /* bits OR-ed into *dev_status by the kernels */
@@ -82,8 +90,17 @@ enum {
  * Arguments (N = total tokens, B = requests):
  *   q, k           [N, Hq, Dk]  `dtype`
  *   v              [N, Hv, Dv]  `dtype`
- *   g              [N, Hv] float32, log-space decay (g <= 0; -inf allowed)
- *   beta           [N, Hv] float32, update rate
+ *   g              [N, Hv] float32, log-space decay (g <= 0; -inf allowed);
+ *                  required exactly for the rules with decay (gated_delta,
+ *                  gated), NULL otherwise.  With GDN_GATE_QWEN it is the raw
+ *                  `decay` input and the kernels use
+ *                  -exp(a_log[h]) * softplus(g + dt_bias[h]) (softplus(x) = x
+ *                  for x > 20), in float32.
+ *   beta           [N, Hv] float32, update rate; required exactly for the rules
+ *                  with the delta retrieval (gated_delta, delta), NULL
+ *                  otherwise (the write is then k_t v_t^T).  With
+ *                  GDN_BETA_SIGMOID the kernels use sigmoid(beta).
+ *   a_log, dt_bias [Hv] float32, required exactly with GDN_GATE_QWEN.
  *   cu_seqlens     [B+1] int32 exclusive prefix sums, or NULL for uniform
  *                  packing (then N % B == 0 and request b is tokens
  *                  [b*N/B, (b+1)*N/B)).  Entries are clamped on the device to
@@ -97,20 +114,23 @@ enum {
  *                  1/sqrt(Dk), the op's default).
  *   qk_l2norm      non-zero: q and k vectors are scaled by
  *                  (sum x^2 + 1e-12)^(-1/2) before use.
- *   flags          GDN_PREFILL_SEQUENTIAL or 0.
+ *   flags          GDN_PREFILL_SEQUENTIAL, one GDN_RULE_* (update_rule of the
+ *                  op's Attributes table: which of the decay and the delta
+ *                  retrieval survive), GDN_GATE_QWEN, GDN_BETA_SIGMOID.
  *   dev_status     optional device int32; GDN_DEV_TIMEOUT is OR-ed in if an
  *                  internal pipeline wait of the chunked kernel exceeds its
  *                  bound (the call's outputs are then invalid).
  * Requirements: 1 <= Dk, Dv <= 256; Hv % Hq == 0; q, k, v, out,
  * initial_state and final_state 16-byte aligned; out must not overlap any
  * input.  bf16 with Dk = Dv = 128 and Hv % 4 == 0 runs the chunked
- * tensor-core kernel (unless GDN_PREFILL_SEQUENTIAL); everything else runs the
- * per-token fp32 kernel.  The chunked kernel floors each g at -30
+ * tensor-core kernel (unless GDN_PREFILL_SEQUENTIAL); everything else (fp32,
+ * fp16, other head sizes) runs the per-token kernel, which computes in fp32.  The chunked kernel floors each g at -30
  * (exp(-30) ~ 9e-14) so that in-chunk decay differences stay finite.
  * Overlapping request ranges are not supported (their outputs are undefined).
  */
 GDN_API gdn_status gdn_prefill(const void *q, const void *k, const void *v,
                        const float *g, const float *beta,
+                       const float *a_log, const float *dt_bias,
                        const int32_t *cu_seqlens,
                        const float *initial_state, float *final_state,
                        void *out,
@@ -181,7 +201,7 @@ GDN_API const char *gdn_last_error(void);
 /* ABI version of this header: increments on any incompatible change. */
 GDN_API int32_t gdn_abi_version(void);
 
-#define GDN_ABI_VERSION 1
+#define GDN_ABI_VERSION 2
 
 #ifdef __cplusplus
 }

@@ -41,7 +41,7 @@ def test_library_exports_every_declared_symbol(L):
 
 
 def test_abi_version_and_status_strings(L):
-    assert L.gdn_abi_version() == 1
+    assert L.gdn_abi_version() == 2
     import gated_deltanet_state_gdn_b200 as g
     for code, name in [(0, "GDN_OK"), (1, "GDN_ERR_NULL"), (2, "GDN_ERR_SHAPE"),
                        (3, "GDN_ERR_DTYPE"), (4, "GDN_ERR_ALIGN"), (5, "GDN_ERR_ALIAS"),
@@ -56,11 +56,12 @@ def P(i, off=0):
 
 
 def prefill(L, **kw):
-    args = dict(q=P(1), k=P(2), v=P(3), g=P(4), beta=P(5), cu=None, init=None, final=P(7),
-                out=P(8), B=2, N=64, Hq=1, Hv=1, Dk=16, Dv=16, dtype=0, scale=1.0, l2=0,
-                flags=0, status=None, stream=None)
+    args = dict(q=P(1), k=P(2), v=P(3), g=P(4), beta=P(5), alog=None, dtb=None, cu=None,
+                init=None, final=P(7), out=P(8), B=2, N=64, Hq=1, Hv=1, Dk=16, Dv=16, dtype=0,
+                scale=1.0, l2=0, flags=0, status=None, stream=None)
     args.update(kw)
-    return L.gdn_prefill(args["q"], args["k"], args["v"], args["g"], args["beta"], args["cu"],
+    return L.gdn_prefill(args["q"], args["k"], args["v"], args["g"], args["beta"], args["alog"],
+                         args["dtb"], args["cu"],
                          args["init"], args["final"], args["out"], args["B"], args["N"],
                          args["Hq"], args["Hv"], args["Dk"], args["Dv"], args["dtype"],
                          args["scale"], args["l2"], args["flags"], args["status"],
@@ -84,6 +85,24 @@ def test_prefill_host_validation(L):
     assert prefill(L, final=P(3, 16)) == 5                # final_state overlaps v
     assert prefill(L, B=0, N=0) == 0                      # nothing to do, nothing launched
     assert prefill(L, B=0, N=4) == 2
+
+
+def test_prefill_rule_and_gate_validation(L):
+    GATED, DELTA, LINEAR, QWEN, SIG = 1 << 3, 2 << 3, 3 << 3, 1 << 5, 1 << 6
+    # decay input exactly for gated / gated_delta, beta exactly for delta / gated_delta
+    assert prefill(L, flags=GATED) == 1                   # gated takes no beta
+    assert prefill(L, flags=DELTA) == 1                   # delta takes no decay
+    assert prefill(L, flags=LINEAR, beta=None) == 1
+    assert prefill(L, g=None) == 1                        # gated_delta needs both
+    # qwen needs a decay and both per-head vectors; sigmoid needs a beta
+    assert prefill(L, flags=QWEN) == 1
+    assert prefill(L, flags=QWEN, alog=P(9)) == 1
+    assert prefill(L, flags=QWEN | DELTA, g=None, alog=P(9), dtb=P(10)) == 2
+    assert prefill(L, flags=SIG | GATED, beta=None) == 2
+    assert prefill(L, alog=P(9), dtb=P(10)) == 1          # vectors without the qwen gate
+    assert prefill(L, flags=QWEN, alog=P(9, 2), dtb=P(10)) == 4
+    assert prefill(L, flags=QWEN, alog=P(8, 4), dtb=P(10)) == 5   # out overlaps a_log
+    assert prefill(L, dtype=2, flags=1 << 7) == 6         # unknown flag bit
 
 
 def decode(L, **kw):

@@ -1,0 +1,102 @@
+"""GPU parity of the gdn_prefill variants against the float64 oracle (through the C ABI):
+the update rules of "com.microsoft.GatedDeltaNet" (Attributes table: linear, gated, delta,
+gated_delta), its qwen gate and sigmoid beta activations, and float16 activations.
+
+Tolerances (relative L2 over the whole tensor): 2e-2 for bf16 activations with the fp32
+state (as for the default rule); 2e-3 for fp16 activations, whose only rounding against the
+oracle is the fp16 cast of the outputs (unit roundoff 2^-11 ~ 4.9e-4) on top of the fp32
+state arithmetic.
+"""
+import numpy as np
+import pytest
+import torch
+
+from _util import TOL_BF16, dev, f64, rel_l2
+
+pytestmark = pytest.mark.gpu
+
+TOL_F16 = 2e-3
+RULES = {"gated_delta": (True, True), "gated": (True, False), "delta": (False, True),
+         "linear": (False, False)}
+LENGTHS = [1, 64, 65, 200, 0, 130]
+
+
+@pytest.fixture(scope="module")
+def gdn():
+    import gated_deltanet_state_gdn_b200 as g
+    g.lib()
+    return g
+
+
+@pytest.fixture(scope="module")
+def W():
+    from gated_deltanet_state_gdn_b200 import workloads
+    return workloads
+
+
+def _run_both(gdn, oracle_mod, c, g, beta, sequential, **kw):
+    o, f = gdn.gdn_prefill(dev(c.q), dev(c.k), dev(c.v), dev(g), dev(beta), dev(c.cu_seqlens),
+                           dev(c.initial_state), scale=c.scale, qk_l2norm=c.qk_l2norm,
+                           sequential=sequential,
+                           **{k: (dev(v) if torch.is_tensor(v) else v) for k, v in kw.items()})
+    torch.cuda.synchronize()
+    okw = {k: (f64(v) if torch.is_tensor(v) else v) for k, v in kw.items()}
+    ro, rf = oracle_mod.prefill(f64(c.q), f64(c.k), f64(c.v), None if g is None else f64(g),
+                                None if beta is None else f64(beta), c.cu_seqlens.numpy(),
+                                None if c.initial_state is None else f64(c.initial_state),
+                                scale=c.scale, qk_l2norm=c.qk_l2norm, **okw)
+    return f64(o), f64(f), ro, rf
+
+
+@pytest.mark.parametrize("sequential", [False, True])
+@pytest.mark.parametrize("rule", list(RULES))
+def test_update_rules(gdn, W, oracle_mod, rule, sequential):
+    c = W.make_prefill(31, LENGTHS, 2, 4, 128, 128, init_std=0.02, qk_l2norm=True)
+    has_decay, has_beta = RULES[rule]
+    o, f, ro, rf = _run_both(gdn, oracle_mod, c, c.g if has_decay else None,
+                             c.beta if has_beta else None, sequential, update_rule=rule)
+    assert rel_l2(o, ro) <= TOL_BF16, rule
+    assert rel_l2(f, rf) <= TOL_BF16, rule
+
+
+@pytest.mark.parametrize("sequential", [False, True])
+@pytest.mark.parametrize("rule", ["gated_delta", "gated", "delta"])
+def test_qwen_gate_and_sigmoid_beta(gdn, W, oracle_mod, rule, sequential):
+    """Raw decay N(0,1) through -exp(a_log) softplus(decay + dt_bias), a_log ~ U[-2,1],
+    dt_bias ~ N(0,0.5); raw beta N(0,1) through the sigmoid."""
+    c = W.make_prefill(32, LENGTHS, 2, 4, 128, 128, init_std=0.02, qk_l2norm=True)
+    rng = np.random.default_rng(33)
+    has_decay, has_beta = RULES[rule]
+    decay = torch.from_numpy(rng.standard_normal(c.g.shape).astype(np.float32))
+    braw = torch.from_numpy(rng.standard_normal(c.beta.shape).astype(np.float32))
+    kw = {"update_rule": rule}
+    if has_decay:
+        kw.update(gate_activation="qwen",
+                  a_log=torch.from_numpy(rng.uniform(-2, 1, 4).astype(np.float32)),
+                  dt_bias=torch.from_numpy((0.5 * rng.standard_normal(4)).astype(np.float32)))
+    if has_beta:
+        kw["beta_activation"] = "sigmoid"
+    o, f, ro, rf = _run_both(gdn, oracle_mod, c, decay if has_decay else None,
+                             braw if has_beta else None, sequential, **kw)
+    assert rel_l2(o, ro) <= TOL_BF16, rule
+    assert rel_l2(f, rf) <= TOL_BF16, rule
+
+
+@pytest.mark.parametrize("Dk,Dv", [(128, 128), (64, 32)])
+def test_fp16_activations(gdn, W, oracle_mod, Dk, Dv):
+    """float16 q/k/v/out run the per-token kernel (fp32 arithmetic); the oracle reads the same
+    fp16-rounded inputs."""
+    assert not gdn.prefill_uses_chunked(torch.float16, 4, Dk, Dv)
+    c = W.make_prefill(34, LENGTHS, 2, 4, Dk, Dv, dtype=torch.float16, init_std=0.02,
+                       qk_l2norm=True)
+    o, f, ro, rf = _run_both(gdn, oracle_mod, c, c.g, c.beta, False)
+    assert o.dtype == np.float64 and rel_l2(o, ro) <= TOL_F16
+    assert rel_l2(f, rf) <= TOL_F16
+
+
+def test_linear_rule_long_sequence_matches_oracle(gdn, W, oracle_mod):
+    """Without decay the state is a plain causal sum; a 1000-token request keeps growing it."""
+    c = W.make_prefill(35, [1000], 1, 4, 128, 128, init_std=None, qk_l2norm=True)
+    o, f, ro, rf = _run_both(gdn, oracle_mod, c, None, None, False, update_rule="linear")
+    assert rel_l2(o, ro) <= TOL_BF16
+    assert rel_l2(f, rf) <= TOL_BF16
