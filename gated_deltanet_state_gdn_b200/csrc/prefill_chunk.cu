@@ -424,8 +424,15 @@ __device__ __forceinline__ void build_row(uint32_t tl_gram, int qd, const float 
 }
 
 // ========================================================================== kernel
+// GENERAL = false: the default rule (gated_delta, no gate or beta activation), with the
+// variant switches folded at compile time; GENERAL = true reads them from p.
+template <bool GENERAL>
 __global__ void __launch_bounds__(NTHREADS, 1) gdn_prefill_chunk_kernel(const __grid_constant__ Params p)
 {
+    const bool has_decay = GENERAL ? p.has_decay != 0 : true;
+    const bool has_retrieval = GENERAL ? p.has_retrieval != 0 : true;
+    const bool beta_sigmoid = GENERAL ? p.beta_sigmoid != 0 : false;
+    const float *const a_log = GENERAL ? p.a_log : nullptr;
     extern __shared__ uint8_t smem_raw[];
     // align the shared-window offset (not the generic address) to 1024 bytes: the
     // 128-byte swizzle of TMA and UMMA is a function of shared-address bits [4, 10)
@@ -456,8 +463,8 @@ __global__ void __launch_bounds__(NTHREADS, 1) gdn_prefill_chunk_kernel(const __
         prefetch_tmap(&p.tm_q);
         prefetch_tmap(&p.tm_k);
         prefetch_tmap(&p.tm_v);
-        if (p.has_decay) prefetch_tmap(&p.tm_g);
-        if (p.has_retrieval) prefetch_tmap(&p.tm_beta);
+        if (has_decay) prefetch_tmap(&p.tm_g);
+        if (has_retrieval) prefetch_tmap(&p.tm_beta);
     }
     if (warp == MMA_WARP) {
         tmem_alloc(sbase + OFF_MISC, 512);
@@ -522,21 +529,21 @@ __global__ void __launch_bounds__(NTHREADS, 1) gdn_prefill_chunk_kernel(const __
                         const uint32_t gb = sbase + OFF_GB0 + ks * 2048;
                         const int t0 = un.start + n * C;
                         const uint32_t kb = cx.bar(B_KQ_FULL + ks);
-                        mbar_arrive_expect_tx(kb, 32768 + (p.has_decay ? 1024 : 0) + (p.has_retrieval ? 1024 : 0));
+                        mbar_arrive_expect_tx(kb, 32768 + (has_decay ? 1024 : 0) + (has_retrieval ? 1024 : 0));
                         tma_load_3d(kq, &p.tm_k, kb, 0, qh, t0);
                         tma_load_3d(kq + KQ_KB, &p.tm_k, kb, 64, qh, t0);
                         tma_load_3d(kq + 8192, &p.tm_q, kb, 0, qh, t0);
                         tma_load_3d(kq + KQ_KB + 8192, &p.tm_q, kb, 64, qh, t0);
-                        if (p.has_decay) tma_load_2d(gb, &p.tm_g, kb, un.h & ~3, t0);
-                        if (p.has_retrieval) tma_load_2d(gb + 1024, &p.tm_beta, kb, un.h & ~3, t0);
+                        if (has_decay) tma_load_2d(gb, &p.tm_g, kb, un.h & ~3, t0);
+                        if (has_retrieval) tma_load_2d(gb + 1024, &p.tm_beta, kb, un.h & ~3, t0);
                         if (n + KQ_STAGES < nc) {
                             const int t2 = t0 + KQ_STAGES * C;
                             tma_prefetch_3d(&p.tm_k, 0, qh, t2);
                             tma_prefetch_3d(&p.tm_k, 64, qh, t2);
                             tma_prefetch_3d(&p.tm_q, 0, qh, t2);
                             tma_prefetch_3d(&p.tm_q, 64, qh, t2);
-                            if (p.has_decay) tma_prefetch_2d(&p.tm_g, un.h & ~3, t2);
-                            if (p.has_retrieval) tma_prefetch_2d(&p.tm_beta, un.h & ~3, t2);
+                            if (has_decay) tma_prefetch_2d(&p.tm_g, un.h & ~3, t2);
+                            if (has_retrieval) tma_prefetch_2d(&p.tm_beta, un.h & ~3, t2);
                         }
                     }
                     gc += nc;
@@ -779,22 +786,32 @@ __global__ void __launch_bounds__(NTHREADS, 1) gdn_prefill_chunk_kernel(const __
                             const int hc = un.h & 3;
                             // update rule: no decay -> g = 0; no retrieval -> beta = 1; qwen gate
                             // -exp(a_log) softplus(decay + dt_bias) and sigmoid beta in fp32
-                            const float ea = p.a_log ? expf(__ldg(p.a_log + un.h)) : 0.f;
-                            const float dtb = p.a_log ? __ldg(p.dt_bias + un.h) : 0.f;
-                            auto gate = [&](int i) -> float {
-                                if (!p.has_decay || i >= len_n) return 0.f;
-                                float x = gtile[i * 4 + hc];
-                                if (p.a_log) x = -ea * gdn::softplus20(x + dtb);
-                                return fmaxf(x, G_FLOOR);
-                            };
-                            auto rate = [&](int i) -> float {
-                                if (i >= len_n) return 0.f;
-                                if (!p.has_retrieval) return 1.f;
-                                const float x = gtile[256 + i * 4 + hc];
-                                return p.beta_sigmoid ? gdn::sigmoidf_(x) : x;
-                            };
-                            const float g0 = gate(i0), g1 = gate(i1);
-                            const float b0 = rate(i0), b1 = rate(i1);
+                            const bool v0 = i0 < len_n, v1 = i1 < len_n;
+                            float g0 = 0.f, g1 = 0.f, b0 = 1.f, b1 = 1.f;
+                            if (has_decay) {
+                                g0 = gtile[i0 * 4 + hc];
+                                g1 = gtile[i1 * 4 + hc];
+                                if (a_log) {
+                                    const float ea = expf(__ldg(a_log + un.h));
+                                    const float dtb = __ldg(p.dt_bias + un.h);
+                                    g0 = -ea * gdn::softplus20(g0 + dtb);
+                                    g1 = -ea * gdn::softplus20(g1 + dtb);
+                                }
+                                g0 = fmaxf(g0, G_FLOOR);
+                                g1 = fmaxf(g1, G_FLOOR);
+                            }
+                            if (has_retrieval) {
+                                b0 = gtile[256 + i0 * 4 + hc];
+                                b1 = gtile[256 + i1 * 4 + hc];
+                                if (beta_sigmoid) {
+                                    b0 = gdn::sigmoidf_(b0);
+                                    b1 = gdn::sigmoidf_(b1);
+                                }
+                            }
+                            g0 = v0 ? g0 : 0.f;
+                            g1 = v1 ? g1 : 0.f;
+                            b0 = v0 ? b0 : 0.f;
+                            b1 = v1 ? b1 : 0.f;
                             float x = g0 + g1;
 #pragma unroll
                             for (int o = 1; o < 32; o <<= 1) {
@@ -823,11 +840,11 @@ __global__ void __launch_bounds__(NTHREADS, 1) gdn_prefill_chunk_kernel(const __
                         ok = ok && cx.wait(B_G_DONE, p_g & 1);
                         ++p_g;
                         tc_fence_after();
-                        build_row(tl + TM_G, pw, ga, solve, smem + OFF_P + ks * P_STAGE, p.has_retrieval != 0);
+                        build_row(tl + TM_G, pw, ga, solve, smem + OFF_P + ks * P_STAGE, has_retrieval);
                         if (pw >= 2) fence_proxy_async_smem();
                         // W = T diag(beta Gamma rk) K carries the retrieval term: zero without it
                         if (lt < 64)
-                            ga[GA_BG + lt] = p.has_retrieval ? ga[GA_BETA + lt] * ga[GA_GAM + lt] * ga[GA_RK + lt] : 0.f;
+                            ga[GA_BG + lt] = has_retrieval ? ga[GA_BETA + lt] * ga[GA_GAM + lt] * ga[GA_RK + lt] : 0.f;
                         tc_fence_before();
                         named_sync(1, 128);
                         if (lt == 0) {
@@ -1223,9 +1240,12 @@ cudaError_t launch_prefill_chunked(const GdnPrefillArgs &a, cudaStream_t stream)
     if (a.B == 0) return cudaSuccess;
     static bool attr_set = false;
     if (!attr_set) {
-        cudaError_t e = cudaFuncSetAttribute(gdn_prefill_chunk_kernel,
+        cudaError_t e = cudaFuncSetAttribute(gdn_prefill_chunk_kernel<false>,
                                              cudaFuncAttributeMaxDynamicSharedMemorySize,
                                              (int)SMEM_BYTES);
+        if (e == cudaSuccess)
+            e = cudaFuncSetAttribute(gdn_prefill_chunk_kernel<true>,
+                                     cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SMEM_BYTES);
         if (e != cudaSuccess) return e;
         attr_set = true;
     }
@@ -1259,6 +1279,10 @@ cudaError_t launch_prefill_chunked(const GdnPrefillArgs &a, cudaStream_t stream)
     p.dt_bias = a.dt_bias;
     const int units = a.B * a.Hv;
     const int grid = units < num_sms() ? units : num_sms();
-    gdn_prefill_chunk_kernel<<<grid, NTHREADS, SMEM_BYTES, stream>>>(p);
+    const bool general = !a.has_decay || !a.has_retrieval || a.beta_sigmoid || a.a_log != nullptr;
+    if (general)
+        gdn_prefill_chunk_kernel<true><<<grid, NTHREADS, SMEM_BYTES, stream>>>(p);
+    else
+        gdn_prefill_chunk_kernel<false><<<grid, NTHREADS, SMEM_BYTES, stream>>>(p);
     return cudaGetLastError();
 }
