@@ -6,8 +6,8 @@ its Python binding) never imports, links or runs it, and it imports nothing
 from the product package: callers hand it numpy arrays.
 
 The arithmetic lives in ``gdn_oracle.c`` (plain C, float64, one token at a
-time).  This module compiles it with gcc on first use and wraps the two entry
-points with ctypes.  See ``gdn_oracle.c`` for the pages each step follows.
+time).  This module compiles it with gcc on first use and wraps its entry
+points (prefill, decode, causal conv1d) with ctypes.  See ``gdn_oracle.c`` for the pages each step follows.
 """
 from __future__ import annotations
 
@@ -52,6 +52,12 @@ def _load():
             D, D, D, D, ctypes.c_double, D,
             ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int,
             ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int,
+        ]
+        U32 = ctypes.POINTER(ctypes.c_uint32)
+        lib.oracle_conv1d.restype = None
+        lib.oracle_conv1d.argtypes = [
+            D, D, D, D, U32, U32, D, ctypes.c_int, ctypes.c_int64, ctypes.c_int, ctypes.c_int,
+            ctypes.c_int, ctypes.c_int,
         ]
         lib.oracle_max_threads.restype = ctypes.c_int
         lib.oracle_max_threads.argtypes = []
@@ -158,3 +164,31 @@ def decode(q, k, v, pool, read_idx, A_log, a, dt_bias, b, *, write_idx=None,
                           Bn, T, nh, H, HV, Dk, Dv, int(bool(use_qk_l2norm)),
                           int(bool(disable_state_update)), int(nt))
     return o, pout
+
+
+def conv1d(x, weight, conv_state, slot_idx, row_offsets, *, write_state=True, out=None):
+    """Causal depthwise conv1d with a slot-indexed window pool, float64.
+
+    x: [N, conv_dim]; weight: [conv_dim, K]; conv_state: [max_slots, conv_dim, K-1];
+    slot_idx: [B] uint32; row_offsets: [B+1] uint32.  ``out`` supplies the values kept
+    in rows no request covers (zeros when None).
+    Returns (y [N, conv_dim], new conv_state) as float64; the input pool is not modified.
+    """
+    x = _f64(x)
+    w = _f64(weight)
+    pin = _f64(conv_state)
+    N, conv_dim = x.shape
+    K = w.shape[1]
+    assert w.shape == (conv_dim, K) and K >= 1
+    assert pin.ndim == 3 and pin.shape[1:] == (conv_dim, K - 1)
+    si = np.ascontiguousarray(np.asarray(slot_idx, dtype=np.uint32))
+    ro = np.ascontiguousarray(np.asarray(row_offsets, dtype=np.uint32))
+    B = si.shape[0]
+    assert ro.shape == (B + 1,)
+    pout = pin.copy()
+    y = np.zeros((N, conv_dim), np.float64) if out is None else _f64(out).copy()
+    U32 = ctypes.POINTER(ctypes.c_uint32)
+    _load().oracle_conv1d(_dp(x), _dp(w), _dp(pin), _dp(pout), si.ctypes.data_as(U32),
+                          ro.ctypes.data_as(U32), _dp(y), int(B), int(N), int(conv_dim), int(K),
+                          int(pin.shape[0]), int(bool(write_state)))
+    return y, pout

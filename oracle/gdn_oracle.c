@@ -30,6 +30,9 @@
  *      alpha = exp(-exp(A_log) softplus(a + dt_bias)) (softplus threshold 20),
  *      beta = sigmoid(b) per Householder sub-step, L2 norm x*rsqrt(sum x^2 +
  *      1e-6), padding rows, write-slot override and per-token scatter.
+ *  - "max.nn.legacy.state_space.gated_delta_conv1d_fwd", description,
+ *      Parameters and example: causal depthwise conv1d over ragged requests
+ *      with a slot-indexed window pool updated in place (oracle_conv1d).
  *
  * Readings where the pages are silent (each one listed in the design notes):
  *  - the prefill L2 norm is x * (sum x^2 + 1e-12)^(-1/2);
@@ -46,7 +49,9 @@
  *
  * Parity pins: tests/test_oracle_pins.py checks this file against the worked
  * examples of "Gated DeltaNet State Update", a brute-force product of the
- * gamma form, closed forms and invariants.
+ * gamma form, closed forms and invariants; tests/test_oracle_conv1d_pins.py
+ * checks the conv1d against its page's worked example, numpy's convolution,
+ * delta-weight closed forms and continuation over calls.
  */
 #include <math.h>
 #include <stdint.h>
@@ -320,5 +325,68 @@ void oracle_decode(const double *q, const double *k, const double *v,
         free(xq);
         free(xk);
         free(p);
+    }
+}
+
+/*
+ * Causal depthwise conv1d over a ragged token stream with a slot-indexed
+ * window pool.
+ *
+ * Source: "max.nn.legacy.state_space.gated_delta_conv1d_fwd" (description,
+ * Parameters and the worked example): input x [N, conv_dim], depthwise
+ * weights w [conv_dim, K], pool [max_slots, conv_dim, K-1] addressed by
+ * slot_idx[b], ragged offsets [B+1]; the pool is updated in place unless
+ * write_state is 0, and the untouched slots keep their values.
+ *
+ * For request b with tokens [s, e) and slot r, channel c sees the extended
+ * sequence
+ *     xe = (pool[r, c, 0], ..., pool[r, c, K-2], x[s, c], ..., x[e-1, c])
+ * and
+ *     y[s + i, c] = sum_{j=0}^{K-1} w[c, j] * xe[i + j]     (0 <= i < e - s)
+ * (w[c, K-1] weighs the current token, w[c, 0] the oldest); with write_state
+ * slot r receives the last K-1 entries of xe.
+ *
+ * Readings where the page is silent (listed in the design notes):
+ *  - the window is stored oldest first, and weight index K-1 meets the
+ *    current token (the causal-convolution convention the example's "last
+ *    three inputs" fits);
+ *  - a request shorter than K-1 keeps the newest old entries in front of its
+ *    inputs (the window slides; it is not zero-filled);
+ *  - no activation follows the convolution (the page names none);
+ *  - offsets are clamped to [0, N] and a request with e <= s is empty (its
+ *    slot is left as it was);
+ *  - a slot >= max_slots is skipped: no output row and no pool access;
+ *  - every request reads the pool as it was before the call (pool_in) and
+ *    writes pool_out; with distinct slots this is the in-place result.
+ */
+void oracle_conv1d(const double *x, const double *w, const double *pool_in,
+                   double *pool_out, const uint32_t *slot_idx,
+                   const uint32_t *offsets, double *y, int B, int64_t N,
+                   int conv_dim, int K, int max_slots, int write_state)
+{
+    const int W = K - 1;
+    for (int b = 0; b < B; ++b) {
+        const int64_t s = clamp_i64((int64_t)offsets[b], 0, N);
+        const int64_t e = clamp_i64((int64_t)offsets[b + 1], 0, N);
+        const uint32_t r = slot_idx[b];
+        if (r >= (uint32_t)max_slots) continue;
+        if (e <= s) continue;
+        const int64_t len = e - s;
+        double *xe = (double *)malloc(sizeof(double) * (size_t)(W + len));
+        for (int c = 0; c < conv_dim; ++c) {
+            const double *win = pool_in + ((int64_t)r * conv_dim + c) * W;
+            for (int j = 0; j < W; ++j) xe[j] = win[j];
+            for (int64_t i = 0; i < len; ++i) xe[W + i] = x[(s + i) * conv_dim + c];
+            for (int64_t i = 0; i < len; ++i) {
+                double acc = 0.0;
+                for (int j = 0; j < K; ++j) acc += w[(int64_t)c * K + j] * xe[i + j];
+                y[(s + i) * conv_dim + c] = acc;
+            }
+            if (write_state) {
+                double *wout = pool_out + ((int64_t)r * conv_dim + c) * W;
+                for (int j = 0; j < W; ++j) wout[j] = xe[len + j];
+            }
+        }
+        free(xe);
     }
 }
