@@ -52,7 +52,7 @@ GDN_DEV_BAD_SLOT = 1
 GDN_DEV_TIMEOUT = 2
 GDN_DEV_INTERNAL = 4
 
-EXPORTED = ("gdn_prefill", "gdn_decode", "gdn_status_string", "gdn_last_error",
+EXPORTED = ("gdn_prefill", "gdn_decode", "gdn_conv1d", "gdn_status_string", "gdn_last_error",
             "gdn_abi_version", "gdn_prefill_uses_chunked")
 
 _lib = None
@@ -87,6 +87,9 @@ def lib():
         L.gdn_decode.argtypes = [vp, vp, vp, vp, i32, i64, i64, vp, vp, vp,
                                  vp, vp, vp, vp, f32, vp,
                                  i32, i32, i32, i32, i32, i32, i32, u32, vp, vp]
+        L.gdn_conv1d.restype = ctypes.c_int
+        L.gdn_conv1d.argtypes = [vp, vp, vp, vp, vp, vp, i32, i64, i32, i32, i32, ctypes.c_int,
+                                 i32, vp, vp]
         L.gdn_status_string.restype = ctypes.c_char_p
         L.gdn_status_string.argtypes = [i32]
         L.gdn_last_error.restype = ctypes.c_char_p
@@ -263,3 +266,49 @@ def gdn_decode(q, k, v, state_pool, read_idx, A_log, a, dt_bias, b, *, scale=Non
     if st != GDN_OK:
         raise GdnError(st, "gdn_decode")
     return out, state_pool
+
+
+_CONV_DTYPES = {torch.float32: GDN_F32, torch.bfloat16: GDN_BF16, torch.float16: GDN_F16}
+
+
+def gdn_conv1d(x, weight, conv_state, slot_idx, row_offsets, out=None, *, write_state: bool = True,
+               dev_status=None, stream=None):
+    """Causal depthwise conv1d with a slot-indexed window pool (updated in place).
+
+    x: [N, conv_dim]; weight: [conv_dim, K]; conv_state: [max_slots, conv_dim, K-1], all of
+    one dtype (fp32, bf16 or fp16); slot_idx: [B] and row_offsets: [B+1], uint32 (int32
+    tensors with non-negative values are accepted and reinterpreted).  ``write_state=False``
+    only reads the pool.  Returns (out [N, conv_dim], conv_state).
+    """
+    if x.dtype not in _CONV_DTYPES:
+        raise TypeError(f"x must be fp32, bf16 or fp16, got {x.dtype}")
+    x = _check_cuda("x", x, x.dtype)
+    weight = _check_cuda("weight", weight, x.dtype)
+    if x.dim() != 2 or weight.dim() != 2 or weight.shape[0] != x.shape[1]:
+        raise ValueError("x must be [N, conv_dim] and weight [conv_dim, K]")
+    N, conv_dim = x.shape
+    K = weight.shape[1]
+    if (not isinstance(conv_state, torch.Tensor) or not conv_state.is_cuda
+            or conv_state.dtype != x.dtype or conv_state.dim() != 3
+            or tuple(conv_state.shape[1:]) != (conv_dim, K - 1) or not conv_state.is_contiguous()):
+        raise ValueError("conv_state must be a contiguous CUDA [max_slots, conv_dim, K-1] tensor "
+                         "of x's dtype")
+    idx_types = (torch.uint32, torch.int32)
+    if slot_idx.dtype not in idx_types or row_offsets.dtype not in idx_types:
+        raise TypeError("slot_idx and row_offsets must be uint32 (or int32)")
+    slot_idx = _check_cuda("slot_idx", slot_idx)
+    row_offsets = _check_cuda("row_offsets", row_offsets)
+    B = slot_idx.shape[0]
+    if row_offsets.shape != (B + 1,):
+        raise ValueError("row_offsets must have B + 1 entries")
+    if out is None:
+        out = torch.zeros_like(x)
+    elif not out.is_contiguous() or out.dtype != x.dtype or out.shape != x.shape:
+        raise ValueError("out must be a contiguous tensor shaped and typed like x")
+    st = lib().gdn_conv1d(_ptr(x), _ptr(weight), _ptr(conv_state), _ptr(slot_idx),
+                          _ptr(row_offsets), _ptr(out), B, N, conv_dim, K, conv_state.shape[0],
+                          _CONV_DTYPES[x.dtype], int(bool(write_state)), _ptr(dev_status),
+                          _stream(stream))
+    if st != GDN_OK:
+        raise GdnError(st, "gdn_conv1d")
+    return out, conv_state

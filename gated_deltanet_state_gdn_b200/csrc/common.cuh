@@ -108,7 +108,21 @@ struct GdnDecodeArgs {
     int32_t *dev_status;
 };
 
+struct GdnConv1dArgs {
+    const void *x;            // [N, conv_dim] dtype
+    const void *weight;       // [conv_dim, K] dtype
+    void *conv_state;         // [max_slots, conv_dim, K-1] dtype, in place (NULL when K == 1)
+    const uint32_t *slot_idx; // [B]
+    const uint32_t *offsets;  // [B+1]
+    void *out;                // [N, conv_dim] dtype
+    int32_t B, conv_dim, K, max_slots;
+    int64_t N;
+    int32_t dtype, write_state;
+    int32_t *dev_status;
+};
+
 cudaError_t launch_decode(const GdnDecodeArgs &a, cudaStream_t stream);
+cudaError_t launch_conv1d(const GdnConv1dArgs &a, cudaStream_t stream);
 cudaError_t launch_prefill_sequential(const GdnPrefillArgs &a, cudaStream_t stream);
 cudaError_t launch_prefill_chunked(const GdnPrefillArgs &a, cudaStream_t stream);
 bool prefill_chunked_supported(const GdnPrefillArgs &a);

@@ -1,0 +1,360 @@
+// conv1d.cu -- causal depthwise conv1d over ragged requests with a
+// slot-indexed pool of conv windows, updated in place.
+//
+// Operation ("max.nn.legacy.state_space.gated_delta_conv1d_fwd", description,
+// Parameters, example): request b covers tokens [s, e) of x [N, conv_dim] and
+// owns slot r = slot_idx[b] of the pool [max_slots, conv_dim, K-1].  Channel
+// c convolves xe = (pool[r, c, 0..K-2], x[s..e-1, c]) with weight[c, 0..K-1]
+// (index K-1 meets the current token); the slot then holds the last K-1
+// entries of xe.
+//
+// HBM-bound: every input row is read once (plus K-1 look-back rows per chunk,
+// mostly L2 hits), every output row written once, each request's window read
+// and written once.  Work layout:
+//   - a block is (request-aligned chunk of L tokens, channel tile), the tile
+//     index varying fastest along the 1-D grid; a thread owns V adjacent
+//     channels -- 16 bytes of a row, so a warp reads 512 contiguous bytes per
+//     token -- and walks its chunk in token order with the last K-1 inputs in
+//     registers, 8 rows loaded ahead when chunks are long (L >= 32);
+//   - L is the largest of 128, 64, ..., 8 that still gives about two waves of
+//     blocks, chosen on the host from N and conv_dim only;
+//   - chunks never straddle requests: block x finds its (request, chunk) by a
+//     block-wide prefix sum of ceil(len_b / L), so the host reads no device
+//     data and the launch can be captured in a graph;
+//   - only chunk 0 of a request touches its pool slot: it reads the old
+//     window for its look-back and, after that, writes the new one, so no
+//     block ever sees a half-updated slot.  Later chunks take their
+//     look-back from x (L >= K-1).
+#include <cuda_fp16.h>
+
+#include <type_traits>
+
+#include "common.cuh"
+
+namespace gdn_conv {
+
+constexpr int kThreads = 128;
+constexpr int kVecBytes = 16;  // bytes of a row per thread on the vector path
+constexpr int kBatchLong = 8;  // rows loaded ahead per thread (chunks >= 32 tokens)
+
+template <typename T>
+__device__ __forceinline__ float to_f(T x);
+template <>
+__device__ __forceinline__ float to_f<float>(float x) { return x; }
+template <>
+__device__ __forceinline__ float to_f<__nv_bfloat16>(__nv_bfloat16 x) { return __bfloat162float(x); }
+template <>
+__device__ __forceinline__ float to_f<__half>(__half x) { return __half2float(x); }
+
+template <typename T>
+__device__ __forceinline__ T from_f(float x);
+template <>
+__device__ __forceinline__ float from_f<float>(float x) { return x; }
+template <>
+__device__ __forceinline__ __nv_bfloat16 from_f<__nv_bfloat16>(float x) { return __float2bfloat16_rn(x); }
+template <>
+__device__ __forceinline__ __half from_f<__half>(float x) { return __float2half_rn(x); }
+
+// NE consecutive elements starting at p: kVecBytes-wide accesses on the vector
+// path (NE * sizeof(T) is then a multiple of kVecBytes and p aligned to it),
+// element accesses otherwise.  Raw words are kept so that loads can be issued ahead
+// of their conversion.
+template <typename T, int NE, bool VEC>
+struct Flat {
+    using Vw = typename std::conditional<kVecBytes == 16, uint4, uint2>::type;
+    static constexpr int kWords = VEC ? NE * (int)sizeof(T) / kVecBytes : NE;
+    using Word = typename std::conditional<VEC, Vw, T>::type;
+    Word w[kWords];
+
+    __device__ __forceinline__ void load(const T *p)
+    {
+        const Word *q = reinterpret_cast<const Word *>(p);
+#pragma unroll
+        for (int i = 0; i < kWords; ++i) w[i] = __ldg(q + i);
+    }
+    __device__ __forceinline__ void to_float(float (&f)[NE]) const
+    {
+        const T *e = reinterpret_cast<const T *>(w);
+#pragma unroll
+        for (int i = 0; i < NE; ++i) f[i] = to_f<T>(e[i]);
+    }
+    __device__ __forceinline__ void from_float(const float (&f)[NE])
+    {
+        T *e = reinterpret_cast<T *>(w);
+#pragma unroll
+        for (int i = 0; i < NE; ++i) e[i] = from_f<T>(f[i]);
+    }
+    __device__ __forceinline__ void store(T *p, bool streaming) const
+    {
+        Word *q = reinterpret_cast<Word *>(p);
+#pragma unroll
+        for (int i = 0; i < kWords; ++i) {
+            if (streaming)
+                __stcs(q + i, w[i]);
+            else
+                q[i] = w[i];
+        }
+    }
+};
+
+// inclusive block prefix sum of one int per thread; returns the block total in *total
+__device__ __forceinline__ int block_scan(int x, int *s_warp, int *total)
+{
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+#pragma unroll
+    for (int d = 1; d < 32; d <<= 1) {
+        const int y = __shfl_up_sync(0xffffffffu, x, d);
+        if (lane >= d) x += y;
+    }
+    if (lane == 31) s_warp[warp] = x;
+    __syncthreads();
+    int before = 0, all = 0;
+#pragma unroll
+    for (int w = 0; w < kThreads / 32; ++w) {
+        const int t = s_warp[w];
+        before += w < warp ? t : 0;
+        all += t;
+    }
+    __syncthreads();  // s_warp is reused by the next call
+    *total = all;
+    return x + before;
+}
+
+template <typename T, int K, bool VEC, int kBatch>
+__global__ void __launch_bounds__(kThreads) conv1d_kernel(const GdnConv1dArgs a, const int L, const int tiles)
+{
+    constexpr int V = VEC ? kVecBytes / (int)sizeof(T) : 1;
+    constexpr int W = K - 1;
+    __shared__ int s_warp[kThreads / 32];
+    __shared__ int s_req, s_chunk;
+
+    // ---- weights first (they do not depend on the request): V channels x K taps
+    // the channel tile varies fastest along the grid, so blocks resident together cover
+    // whole rows
+    const int tile = (int)(blockIdx.x % (unsigned)tiles);
+    const int chunk = (int)(blockIdx.x / (unsigned)tiles);
+    const int c0 = (tile * kThreads + threadIdx.x) * V;
+    const bool has_ch = c0 < a.conv_dim;
+    Flat<T, V * K, VEC> fw;
+    if (has_ch) fw.load(static_cast<const T *>(a.weight) + (int64_t)c0 * K);
+
+    // ---- which (request, chunk) this block covers
+    const int N32 = (int)a.N;
+    if (threadIdx.x == 0) s_req = -1;
+    int base = 0;
+    for (int b0 = 0; b0 < a.B; b0 += kThreads) {
+        const int b = b0 + threadIdx.x;
+        int cnt = 0;
+        if (b < a.B) {
+            const int s = (int)min(a.offsets[b], (uint32_t)N32);
+            const int e = (int)min(a.offsets[b + 1], (uint32_t)N32);
+            cnt = e > s ? (int)(((int64_t)(e - s) + L - 1) / L) : 0;
+        }
+        int total;
+        const int incl = block_scan(cnt, s_warp, &total);  // its barriers order s_req too
+        if (cnt > 0 && chunk >= base + incl - cnt && chunk < base + incl) {
+            s_req = b;
+            s_chunk = chunk - (base + incl - cnt);
+        }
+        base += total;
+        __syncthreads();
+        if (s_req >= 0 || chunk < base) break;
+    }
+    __syncthreads();
+    const int b = s_req;
+    if (b < 0) return;  // past the last chunk (the grid is an upper bound)
+    const int ci = s_chunk;
+    const int s = (int)min(a.offsets[b], (uint32_t)N32);
+    const int e = (int)min(a.offsets[b + 1], (uint32_t)N32);
+    const uint32_t r = a.slot_idx[b];
+    if (r >= (uint32_t)a.max_slots) {
+        if (ci == 0 && tile == 0 && threadIdx.x == 0 && a.dev_status)
+            atomicOr(a.dev_status, GDN_DEV_BAD_SLOT);
+        return;
+    }
+    if (!has_ch) return;
+
+    const T *__restrict__ x = static_cast<const T *>(a.x);
+    T *__restrict__ out = static_cast<T *>(a.out);
+    const int64_t ld = a.conv_dim;
+    const int t0 = s + ci * L;
+    const int t1 = min(e, t0 + L);
+
+    float wf[K][V];
+    {
+        float f[V * K];
+        fw.to_float(f);
+#pragma unroll
+        for (int v = 0; v < V; ++v)
+#pragma unroll
+            for (int j = 0; j < K; ++j) wf[j][v] = f[v * K + j];
+    }
+
+    // ---- look-back window, oldest first
+    float xw[W > 0 ? W : 1][V];
+    T *const slot = W > 0 ? static_cast<T *>(a.conv_state) + ((int64_t)r * a.conv_dim + c0) * W
+                          : nullptr;
+    if (W > 0) {
+        if (ci == 0) {
+            Flat<T, V * (W > 0 ? W : 1), VEC> fs;
+            fs.load(slot);
+            float f[V * (W > 0 ? W : 1)];
+            fs.to_float(f);
+#pragma unroll
+            for (int v = 0; v < V; ++v)
+#pragma unroll
+                for (int j = 0; j < W; ++j) xw[j][v] = f[v * W + j];
+        } else {
+#pragma unroll
+            for (int j = 0; j < W; ++j) {
+                Flat<T, V, VEC> fx;
+                fx.load(x + (int64_t)(t0 - W + j) * ld + c0);
+                float f[V];
+                fx.to_float(f);
+#pragma unroll
+                for (int v = 0; v < V; ++v) xw[j][v] = f[v];
+            }
+        }
+    }
+
+    // ---- the chunk's tokens: full batches of kBatch rows loaded ahead, then the rest
+    // one row at a time
+    const T *xp = x + (int64_t)t0 * ld + c0;
+    T *op = out + (int64_t)t0 * ld + c0;
+    auto step = [&](const Flat<T, V, VEC> &fx) {
+        float xn[V], y[V];
+        fx.to_float(xn);
+#pragma unroll
+        for (int v = 0; v < V; ++v) {
+            float acc = 0.f;
+#pragma unroll
+            for (int j = 0; j < W; ++j) acc = fmaf(wf[j][v], xw[j][v], acc);
+            y[v] = fmaf(wf[W][v], xn[v], acc);
+        }
+#pragma unroll
+        for (int j = 0; j + 1 < W; ++j)
+#pragma unroll
+            for (int v = 0; v < V; ++v) xw[j][v] = xw[j + 1][v];
+        if (W > 0) {
+#pragma unroll
+            for (int v = 0; v < V; ++v) xw[W > 0 ? W - 1 : 0][v] = xn[v];
+        }
+        Flat<T, V, VEC> fy;
+        fy.from_float(y);
+        fy.store(op, true);
+        op += ld;
+    };
+    int t = t0;
+    for (; t + kBatch <= t1; t += kBatch) {
+        Flat<T, V, VEC> fx[kBatch];
+#pragma unroll
+        for (int u = 0; u < kBatch; ++u) fx[u].load(xp + u * ld);
+        xp += kBatch * ld;
+#pragma unroll
+        for (int u = 0; u < kBatch; ++u) step(fx[u]);
+    }
+#pragma unroll 1
+    for (; t < t1; ++t) {
+        Flat<T, V, VEC> fx;
+        fx.load(xp);
+        xp += ld;
+        step(fx);
+    }
+
+    // ---- new window (chunk 0 only; it has read the old one above)
+    if (W > 0 && ci == 0 && a.write_state) {
+        if (t1 < e) {
+            // the request continues past this chunk, so it has >= L >= K-1 tokens: the
+            // window is its last K-1 inputs
+#pragma unroll
+            for (int j = 0; j < W; ++j) {
+                Flat<T, V, VEC> fx;
+                fx.load(x + (int64_t)(e - W + j) * ld + c0);
+                float f[V];
+                fx.to_float(f);
+#pragma unroll
+                for (int v = 0; v < V; ++v) xw[j][v] = f[v];
+            }
+        }
+        // else the sliding window after the last token already is the new one
+        float f[V * (W > 0 ? W : 1)];
+#pragma unroll
+        for (int v = 0; v < V; ++v)
+#pragma unroll
+            for (int j = 0; j < W; ++j) f[v * W + j] = xw[j][v];
+        Flat<T, V * (W > 0 ? W : 1), VEC> fs;
+        fs.from_float(f);
+        fs.store(slot, false);
+    }
+}
+
+int device_sms()
+{
+    int dev = 0, n = 0;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+    return n > 0 ? n : 148;
+}
+
+// tokens per chunk: the largest of 128, 64, ..., 8 that still gives about two
+// waves of blocks on the device (L >= 8 >= K-1 always holds)
+int chunk_tokens(int64_t N, int tiles)
+{
+    const int64_t target = (int64_t)device_sms() * 16;
+    int L = 128;
+    while (L > 8 && ((N + L - 1) / L) * tiles < target) L >>= 1;
+    return L;
+}
+
+template <typename T, bool VEC, int NB>
+cudaError_t launch_k(const GdnConv1dArgs &a, dim3 grid, int L, int tiles, cudaStream_t stream)
+{
+    switch (a.K) {
+    case 1: conv1d_kernel<T, 1, VEC, NB><<<grid, kThreads, 0, stream>>>(a, L, tiles); break;
+    case 2: conv1d_kernel<T, 2, VEC, NB><<<grid, kThreads, 0, stream>>>(a, L, tiles); break;
+    case 3: conv1d_kernel<T, 3, VEC, NB><<<grid, kThreads, 0, stream>>>(a, L, tiles); break;
+    case 4: conv1d_kernel<T, 4, VEC, NB><<<grid, kThreads, 0, stream>>>(a, L, tiles); break;
+    case 5: conv1d_kernel<T, 5, VEC, NB><<<grid, kThreads, 0, stream>>>(a, L, tiles); break;
+    case 6: conv1d_kernel<T, 6, VEC, NB><<<grid, kThreads, 0, stream>>>(a, L, tiles); break;
+    case 7: conv1d_kernel<T, 7, VEC, NB><<<grid, kThreads, 0, stream>>>(a, L, tiles); break;
+    case 8: conv1d_kernel<T, 8, VEC, NB><<<grid, kThreads, 0, stream>>>(a, L, tiles); break;
+    default: return cudaErrorInvalidValue;
+    }
+    return cudaGetLastError();
+}
+
+template <typename T, bool VEC>
+cudaError_t launch_t(const GdnConv1dArgs &a, cudaStream_t stream)
+{
+    constexpr int V = VEC ? kVecBytes / (int)sizeof(T) : 1;
+    const int tiles = (a.conv_dim + kThreads * V - 1) / (kThreads * V);
+    const int L = chunk_tokens(a.N, tiles);
+    const int64_t chunks = (a.N + L - 1) / L + a.B;  // request-aligned chunks, upper bound
+    if (chunks * tiles > 0x7fffffff) return cudaErrorInvalidConfiguration;
+    const dim3 grid((unsigned)(chunks * tiles));
+    // short chunks (few tokens per request) take the batch-1 body: fewer registers, more
+    // resident blocks to hide the per-block lookup latency
+    return L >= 32 ? launch_k<T, VEC, kBatchLong>(a, grid, L, tiles, stream)
+                   : launch_k<T, VEC, 1>(a, grid, L, tiles, stream);
+}
+
+template <typename T>
+cudaError_t launch_dtype(const GdnConv1dArgs &a, bool vec, cudaStream_t stream)
+{
+    return vec ? launch_t<T, true>(a, stream) : launch_t<T, false>(a, stream);
+}
+
+}  // namespace gdn_conv
+
+cudaError_t launch_conv1d(const GdnConv1dArgs &a, cudaStream_t stream)
+{
+    using namespace gdn_conv;
+    if (a.B == 0 || a.N == 0) return cudaSuccess;
+    const size_t esz = a.dtype == GDN_F32 ? 4 : 2;
+    auto alv = [](const void *p) { return ((uintptr_t)p & (kVecBytes - 1)) == 0; };
+    const bool vec = ((size_t)a.conv_dim * esz) % kVecBytes == 0 && alv(a.x) && alv(a.out) &&
+                     alv(a.weight) && (a.K == 1 || alv(a.conv_state));
+    if (a.dtype == GDN_F32) return launch_dtype<float>(a, vec, stream);
+    if (a.dtype == GDN_F16) return launch_dtype<__half>(a, vec, stream);
+    return launch_dtype<__nv_bfloat16>(a, vec, stream);
+}

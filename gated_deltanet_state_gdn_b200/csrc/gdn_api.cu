@@ -189,4 +189,43 @@ gdn_status gdn_decode(const void *q, const void *k, const void *v, float *state_
     return GDN_OK;
 }
 
+gdn_status gdn_conv1d(const void *x, const void *weight, void *conv_state,
+                      const uint32_t *slot_idx, const uint32_t *row_offsets, void *out,
+                      int32_t B, int64_t N, int32_t conv_dim, int32_t kernel_size,
+                      int32_t max_slots, gdn_dtype dtype, int32_t write_state,
+                      int32_t *dev_status, void *stream)
+{
+    if (dtype != GDN_F32 && dtype != GDN_BF16 && dtype != GDN_F16) return GDN_ERR_DTYPE;
+    if (B < 0 || N < 0 || conv_dim < 1 || kernel_size < 1 || max_slots < 1) return GDN_ERR_SHAPE;
+    if (kernel_size > 8) return GDN_ERR_UNSUPPORTED;
+    if (N > ((int64_t)1 << 31) - 1) return GDN_ERR_UNSUPPORTED;
+    if (B == 0) return GDN_OK;
+    if (!x || !weight || !out || !slot_idx || !row_offsets) return GDN_ERR_NULL;
+    if (kernel_size > 1 && !conv_state) return GDN_ERR_NULL;
+    const size_t esz = dtype == GDN_F32 ? 4 : 2;
+    if (!aligned(x, esz) || !aligned(weight, esz) || !aligned(out, esz) ||
+        !aligned(conv_state, esz) || !aligned(slot_idx, 4) || !aligned(row_offsets, 4))
+        return GDN_ERR_ALIGN;
+    const size_t x_bytes = (size_t)N * conv_dim * esz;
+    const size_t w_bytes = (size_t)conv_dim * kernel_size * esz;
+    const size_t st_bytes = (size_t)max_slots * conv_dim * (kernel_size - 1) * esz;
+    const size_t si_bytes = (size_t)B * 4, ro_bytes = (size_t)(B + 1) * 4;
+    if (overlaps(out, x_bytes, x, x_bytes) || overlaps(out, x_bytes, weight, w_bytes) ||
+        overlaps(out, x_bytes, conv_state, st_bytes) || overlaps(out, x_bytes, slot_idx, si_bytes) ||
+        overlaps(out, x_bytes, row_offsets, ro_bytes) ||
+        overlaps(conv_state, st_bytes, x, x_bytes) || overlaps(conv_state, st_bytes, weight, w_bytes) ||
+        overlaps(conv_state, st_bytes, slot_idx, si_bytes) ||
+        overlaps(conv_state, st_bytes, row_offsets, ro_bytes))
+        return GDN_ERR_ALIAS;
+
+    GdnConv1dArgs c;
+    c.x = x; c.weight = weight; c.conv_state = conv_state; c.slot_idx = slot_idx;
+    c.offsets = row_offsets; c.out = out; c.B = B; c.conv_dim = conv_dim; c.K = kernel_size;
+    c.max_slots = max_slots; c.N = N; c.dtype = dtype; c.write_state = write_state ? 1 : 0;
+    c.dev_status = dev_status;
+    cudaError_t e = launch_conv1d(c, (cudaStream_t)stream);
+    if (e != cudaSuccess) return cuda_fail(e, "gdn_conv1d launch");
+    return GDN_OK;
+}
+
 }  // extern "C"

@@ -234,3 +234,64 @@ def mtp_case(seed: int = 5) -> DecodeCase:
     and use_qk_l2norm on; per-token scatter into distinct slots."""
     return make_decode(seed, P=512, B=64, T=4, nh=2, H=16, Dv=64, write_mode="none", scatter=True,
                        host_norm_qk=True, name="mtp_P512_B64_T4_nh2_H16_Dv64")
+
+
+@dataclass
+class Conv1dCase:
+    """Inputs of one gdn_conv1d call (CPU tensors)."""
+    name: str
+    x: torch.Tensor            # [N, conv_dim]
+    weight: torch.Tensor       # [conv_dim, K]
+    conv_state: torch.Tensor   # [max_slots, conv_dim, K-1]
+    slot_idx: torch.Tensor     # [B] uint32
+    row_offsets: torch.Tensor  # [B+1] uint32
+    meta: dict = field(default_factory=dict)
+
+    @property
+    def B(self) -> int:
+        return int(self.slot_idx.shape[0])
+
+    @property
+    def N(self) -> int:
+        return int(self.x.shape[0])
+
+
+def make_conv1d(seed: int, lengths, conv_dim: int, K: int, max_slots: int, *,
+                dtype: torch.dtype = torch.bfloat16, N: Optional[int] = None, lead: int = 0,
+                name: str = "conv1d") -> Conv1dCase:
+    """Ragged conv1d case: x ~ N(0, 1) (the projected q/k/v rows), weights ~ U(-1/sqrt(K),
+    1/sqrt(K)) (the default init of a depthwise conv with K taps), pool ~ N(0, 1); the
+    requests take distinct slots from a seeded permutation.  Requests are packed from row
+    ``lead``; rows before it and after the last request (up to ``N``) belong to none."""
+    rng = np.random.default_rng(seed)
+    lengths = [int(L) for L in lengths]
+    total = lead + sum(lengths)
+    N = total if N is None else N
+    assert N >= total and len(lengths) <= max_slots
+    x = rng.standard_normal((N, conv_dim), dtype=np.float32)
+    bound = np.float32(1.0 / np.sqrt(K))
+    w = rng.uniform(-bound, bound, (conv_dim, K)).astype(np.float32)
+    pool = rng.standard_normal((max_slots, conv_dim, K - 1), dtype=np.float32)
+    slots = rng.permutation(max_slots)[:len(lengths)].astype(np.uint32)
+    off = (lead + np.concatenate([[0], np.cumsum(lengths)])).astype(np.uint32)
+    cast = {torch.bfloat16: _bf16, torch.float16: _f16, torch.float32: _f32}[dtype]
+    return Conv1dCase(name=name, x=cast(x), weight=cast(w), conv_state=cast(pool),
+                      slot_idx=torch.from_numpy(slots), row_offsets=torch.from_numpy(off),
+                      meta={"lengths": lengths})
+
+
+def conv_ragged_case(seed: int = 6, n_req: int = 8, max_len: int = 4096) -> Conv1dCase:
+    """The ragged prefill's token mix (lengths U[1, 4096], the same seed draw) through the
+    conv that feeds it: conv_dim = 2*16*128 + 32*128 = 8192 (q, k, v rows), K = 4, bf16,
+    a pool of 64 slots."""
+    rng = np.random.default_rng(2)
+    lengths = rng.integers(1, max_len + 1, n_req).tolist()
+    return make_conv1d(seed, lengths, 8192, 4, 64,
+                       name=f"conv1d_ragged_{n_req}req_U1-{max_len}_C8192_K4_bf16")
+
+
+def conv_decode_case(seed: int = 7, B: int = 256, max_slots: int = 1024) -> Conv1dCase:
+    """One token for each of 256 requests (a decode step) through the conv: conv_dim 8192,
+    K = 4, bf16, a pool of 1024 slots, distinct slots."""
+    return make_conv1d(seed, [1] * B, 8192, 4, max_slots,
+                       name=f"conv1d_decode_B{B}_P{max_slots}_C8192_K4_bf16")

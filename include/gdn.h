@@ -2,9 +2,11 @@
  * gdn.h -- C ABI of libgdn: the Gated DeltaNet recurrence on NVIDIA B200
  * (sm_100a).
  *
- * Two entry points:
+ * Three entry points:
  *   gdn_prefill  chunked / sequential scan over ragged requests;
- *   gdn_decode   decode / MTP update of an fp32 slot-indexed state pool.
+ *   gdn_decode   decode / MTP update of an fp32 slot-indexed state pool;
+ *   gdn_conv1d   the causal depthwise conv1d that feeds q, k, v, with a
+ *                slot-indexed pool of conv windows.
  *
  * Conventions shared by every call
  *   - Every tensor argument is a DEVICE pointer owned by the caller.  The
@@ -14,8 +16,8 @@
  *     legacy default stream).  The library never reads tensor contents on the
  *     host and never synchronises, so a call may be captured in a CUDA graph.
  *   - Inputs are never modified.  The only buffers written are `out`,
- *     `final_state` (prefill) and `state_pool`, `out` (decode), plus the
- *     optional `dev_status` word.
+ *     `final_state` (prefill), `state_pool`, `out` (decode) and `out`,
+ *     `conv_state` (conv1d), plus the optional `dev_status` word.
  *   - Errors the host can see (null pointers, shapes, alignment, aliasing,
  *     unsupported sizes) are returned as a gdn_status before anything is
  *     launched.  Errors only the device can see (a slot index >= pool_size)
@@ -53,7 +55,7 @@ typedef enum {
 typedef enum {
     GDN_F32 = 0,   /* float32 activations */
     GDN_BF16 = 1,  /* bfloat16 activations */
-    GDN_F16 = 2    /* float16 activations (prefill, per-token kernel) */
+    GDN_F16 = 2    /* float16 activations (prefill per-token kernel, conv1d) */
 } gdn_dtype;
 
 /* flags */
@@ -72,7 +74,7 @@ enum {
 
 /* bits OR-ed into *dev_status by the kernels */
 enum {
-    GDN_DEV_BAD_SLOT = 1,  /* decode: a read/write/scatter slot >= pool_size was skipped */
+    GDN_DEV_BAD_SLOT = 1,  /* a slot index >= the pool size was skipped (decode, conv1d) */
     GDN_DEV_TIMEOUT = 2,   /* a kernel-internal wait exceeded its bound; outputs invalid */
     GDN_DEV_INTERNAL = 4   /* a kernel's layout self-check failed; nothing was computed */
 };
@@ -185,6 +187,46 @@ GDN_API gdn_status gdn_decode(const void *q, const void *k, const void *v,
                       int32_t B, int32_t T, int32_t nh, int32_t H, int32_t HV,
                       int32_t Dk, int32_t Dv, uint32_t flags,
                       int32_t *dev_status, void *stream);
+
+/*
+ * gdn_conv1d -- causal depthwise conv1d over ragged requests with a
+ * slot-indexed pool of conv windows, updated in place.
+ *
+ * Defined by "max.nn.legacy.state_space.gated_delta_conv1d_fwd" (description,
+ * Parameters, example).  For request b with tokens [s, e) =
+ * [row_offsets[b], row_offsets[b+1]) (clamped to [0, N]; e <= s is empty) and
+ * slot r = slot_idx[b], channel c sees the sequence
+ *     xe = (conv_state[r, c, 0 .. K-2], x[s, c], ..., x[e-1, c])
+ * (the window is stored oldest first) and
+ *     out[s + i, c] = sum_{j=0}^{K-1} weight[c, j] * xe[i + j]
+ * accumulated in float32 and rounded to `dtype`; no activation follows.
+ * With write_state != 0, conv_state[r] receives the last K-1 entries of xe
+ * (a request shorter than K-1 keeps the newest old entries ahead of its
+ * inputs); with write_state == 0 the pool is only read.  Slots no request
+ * names keep their values; so does an empty request's slot.
+ *
+ * Arguments (N = total tokens, B = requests, K = kernel_size):
+ *   x            [N, conv_dim] `dtype` (the projected q/k/v rows)
+ *   weight       [conv_dim, K] `dtype`
+ *   conv_state   [max_slots, conv_dim, K-1] `dtype`, read and written in
+ *                place; may be NULL only when K == 1
+ *   slot_idx     [B] uint32;  row_offsets [B+1] uint32
+ *   out          [N, conv_dim] `dtype`, written for every token a request
+ *                with a valid slot covers (others keep the caller's values)
+ *   dev_status   optional device int32; GDN_DEV_BAD_SLOT is OR-ed in when a
+ *                slot >= max_slots is met (that request is skipped: no
+ *                output rows, no pool access).
+ * Requirements: 1 <= K <= 8; conv_dim >= 1; dtype F32, BF16 or F16; all
+ * tensors naturally aligned for `dtype` (16-byte alignment of every tensor
+ * and conv_dim * element size a multiple of 16 select the vector path);
+ * out and conv_state overlap no input and not each other.  Requests must
+ * name distinct slots when write_state != 0 (a shared slot is a race).
+ */
+GDN_API gdn_status gdn_conv1d(const void *x, const void *weight, void *conv_state,
+                              const uint32_t *slot_idx, const uint32_t *row_offsets,
+                              void *out, int32_t B, int64_t N, int32_t conv_dim,
+                              int32_t kernel_size, int32_t max_slots, gdn_dtype dtype,
+                              int32_t write_state, int32_t *dev_status, void *stream);
 
 /* 1 when gdn_prefill with these arguments runs the chunked tensor-core
  * kernel, 0 when it runs the per-token kernel (host-only query, no launch).

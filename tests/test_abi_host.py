@@ -30,7 +30,7 @@ def declared_symbols():
 
 def test_header_declares_entry_points():
     syms = declared_symbols()
-    assert {"gdn_prefill", "gdn_decode", "gdn_status_string"} <= set(syms)
+    assert {"gdn_prefill", "gdn_decode", "gdn_conv1d", "gdn_status_string"} <= set(syms)
 
 
 def test_library_exports_every_declared_symbol(L):
@@ -136,6 +136,38 @@ def test_decode_host_validation(L):
     assert decode(L, flags=1 << 7) == 6
     assert decode(L, P=0) == 2
     assert decode(L, B=0) == 0
+
+
+def conv1d(L, **kw):
+    args = dict(x=P(1), w=P(2), st=P(3), si=P(4), ro=P(5), out=P(6), B=2, N=64, C=64, K=4,
+                S=8, dtype=1, ws=1, status=None, stream=None)
+    args.update(kw)
+    return L.gdn_conv1d(args["x"], args["w"], args["st"], args["si"], args["ro"], args["out"],
+                        args["B"], args["N"], args["C"], args["K"], args["S"], args["dtype"],
+                        args["ws"], args["status"], args["stream"])
+
+
+def test_conv1d_host_validation(L):
+    assert conv1d(L, dtype=7) == 3                        # GDN_ERR_DTYPE
+    assert conv1d(L, K=0) == 2
+    assert conv1d(L, K=9) == 6                            # kernel_size beyond 8
+    assert conv1d(L, C=0) == 2
+    assert conv1d(L, S=0) == 2                            # no slots
+    assert conv1d(L, N=-1) == 2
+    assert conv1d(L, N=1 << 31) == 6
+    assert conv1d(L, x=None) == 1
+    assert conv1d(L, si=None) == 1
+    assert conv1d(L, ro=None) == 1
+    assert conv1d(L, st=None) == 1                        # a window pool is needed for K > 1
+    assert conv1d(L, x=P(1, 1)) == 4                      # bf16 elements need 2-byte alignment
+    assert conv1d(L, dtype=0, out=P(6, 2)) == 4           # fp32 elements need 4-byte alignment
+    assert conv1d(L, si=P(4, 2)) == 4
+    assert conv1d(L, out=P(1, 128)) == 5                  # out overlaps x
+    assert conv1d(L, st=P(6, 64)) == 5                    # pool overlaps out
+    assert conv1d(L, st=P(2, 16)) == 5                    # pool overlaps the weights
+    assert conv1d(L, B=0) == 0                            # nothing to do, nothing launched
+    # a 1-tap convolution has no window, so the pool may be NULL; N = 0 launches nothing
+    assert conv1d(L, K=1, st=None, N=0) == 0
 
 
 def test_binding_fails_loudly_without_library(monkeypatch, tmp_path):
