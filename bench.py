@@ -8,7 +8,9 @@ ragged requests with lengths U[1,4096], Hq=16, Hv=32, Dk=Dv=128, bf16), inputs
 resident in HBM.  `value` is prefill tokens/s over all ranks.  The same run
 then times gdn_decode over the state-pool workload (pool [1024,32,128,128]
 fp32, 256 rows with 13 padding rows) for K steps and reports its state-pool
-GB/s under "decode".
+GB/s under "decode", and gdn_conv1d (the causal conv feeding q, k, v: conv_dim
+8192, K = 4, bf16) over the ragged token mix ("conv1d") and over one decode
+step of 256 requests ("conv1d_decode"), in HBM GB/s.
 
 Multi-GPU (torchrun): every rank runs an independent replica of the workload
 (weak scaling, no collective on the data path); times are the max over ranks.
@@ -306,6 +308,63 @@ def time_decode(gdn, case, steps, warmup, world):
     return [s.elapsed_time(e) for s, e in ev]
 
 
+def conv_bytes(case):
+    """HBM bytes the conv must move: x read and out written once, each request's window read
+    and written once, the weights once."""
+    N, C = case.x.shape
+    K = case.weight.shape[1]
+    esz = case.x.element_size()
+    lens = (case.row_offsets[1:].to(torch.int64) - case.row_offsets[:-1].to(torch.int64))
+    live = int((lens > 0).sum())
+    return 2 * N * C * esz + 2 * live * C * (K - 1) * esz + C * K * esz
+
+
+def time_conv(gdn, case, steps, warmup, world, graph=False):
+    """Per-launch CUDA events around back-to-back launches; with graph=True the `steps`
+    launches are captured in one CUDA graph (host launch cost out of the way for small calls)
+    and the mean per launch is returned for every step."""
+    x, w, st, si, ro = map(to_dev, (case.x, case.weight, case.conv_state, case.slot_idx,
+                                    case.row_offsets))
+    out = torch.empty_like(x)
+
+    def step(stream=None):
+        gdn.gdn_conv1d(x, w, st, si, ro, out, stream=stream)
+
+    for _ in range(warmup):
+        step()
+    stream = torch.cuda.current_stream()
+    barrier(world)
+    torch.cuda.synchronize()
+    if graph:
+        side = torch.cuda.Stream()
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.stream(side):
+            with torch.cuda.graph(g, stream=side):
+                for _ in range(steps):
+                    step(side)
+        torch.cuda.synchronize()
+        g.replay()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        g.replay()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        barrier(world)
+        per = e0.elapsed_time(e1) / steps
+        del g
+        return [per] * steps
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(steps)]
+    for s, e in ev:
+        s.record(stream)
+        step()
+        e.record(stream)
+    torch.cuda.synchronize()
+    barrier(world)
+    return [s.elapsed_time(e) for s, e in ev]
+
+
 # ---------------------------------------------------------------- CPU oracle
 def cpu_oracle_sample(case, target_s=10.0):
     """Time the float64 oracle on a bounded sample of the prefill workload: the first L
@@ -351,6 +410,11 @@ def profile_phase(gdn, workloads, args):
         total_ms, launch_ms = time_prefill(gdn, case, args.steps, args.warmup, 1)
         print(json.dumps({"phase": "prefill", "workload": case.name,
                           "ms_per_launch": statistics.mean(launch_ms)}), flush=True)
+    elif args.phase == "conv":
+        for ccase in (workloads.conv_ragged_case(), workloads.conv_decode_case()):
+            cms = time_conv(gdn, ccase, args.steps, args.warmup, 1)
+            print(json.dumps({"phase": "conv", "workload": ccase.name,
+                              "ms_per_launch": statistics.mean(cms)}), flush=True)
     else:
         dcase = workloads.decode_pool_case()
         dms = time_decode(gdn, dcase, args.steps, args.warmup, 1)
@@ -385,9 +449,10 @@ def main():
     ap.add_argument("--impl", default="gdn", choices=["gdn", "reference"])
     ap.add_argument("--workload", default="ragged", choices=["ragged", "long"])
     ap.add_argument("--no-decode", action="store_true")
+    ap.add_argument("--no-conv", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu", action="store_true", help="skip the CPU oracle baseline")
-    ap.add_argument("--phase", default="all", choices=["all", "prefill", "decode"],
+    ap.add_argument("--phase", default="all", choices=["all", "prefill", "decode", "conv"],
                     help="prefill or decode alone (for profiling); 'all' for the JSON line")
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     args = ap.parse_args()
@@ -475,6 +540,29 @@ def main():
                   "peak_source": peaks["source"]}
         launches += args.steps
         del dcase
+
+    conv = conv_dec = None
+    if not args.no_conv:
+        for key, ccase, graph, note in (
+                ("conv1d", workloads.conv_ragged_case(), False,
+                 "back-to-back launches, working set > L2 (steady-state HBM traffic)"),
+                ("conv1d_decode", workloads.conv_decode_case(), True,
+                 "one CUDA graph of K launches; 33.6 MB working set stays in L2")):
+            cms = time_conv(gdn, ccase, args.steps, args.warmup, world, graph=graph)
+            cmax = max_over_ranks(sum(cms), world) / args.steps
+            cbytes = conv_bytes(ccase)
+            per_gpu = cbytes / (statistics.mean(cms) / 1e3) / 1e9
+            obj = {"workload": ccase.name, "value": cbytes * world / (cmax / 1e3) / 1e9,
+                   "unit": "GB/s", "bytes_per_step": cbytes, "ms_per_step": cmax,
+                   "frac": per_gpu / peaks["hbm_gbs"], "peak": peaks["hbm_gbs"],
+                   "peak_source": peaks["source"], "timing": note}
+            if key == "conv1d":
+                obj["traffic"] = ncu_traffic("conv1d_ragged.md", "conv1d.cu")
+                conv = obj
+            else:
+                conv_dec = obj
+            launches += args.steps
+            del ccase
     clocks.stop()
 
     e2e = None
@@ -497,7 +585,8 @@ def main():
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
             "data": "synthetic", "config": dict(workload_config(case, args.workload),
                                                 parallelism=f"replicas{world}"),
-            "roofline": roof, "decode": decode, "e2e": e2e, "cpu_baseline": cpu,
+            "roofline": roof, "decode": decode, "conv1d": conv, "conv1d_decode": conv_dec,
+            "e2e": e2e, "cpu_baseline": cpu,
             "clocks": clocks.summary(), "gpu_launches": launches,
         }
         print(json.dumps(line), flush=True)

@@ -30,8 +30,11 @@
 #include <type_traits>
 
 #include "common.cuh"
+#include "sm100.cuh"
 
 namespace gdn_conv {
+
+using namespace sm100;
 
 constexpr int kThreads = 128;
 constexpr int kVecBytes = 16;  // bytes of a row per thread on the vector path
@@ -120,13 +123,60 @@ __device__ __forceinline__ int block_scan(int x, int *s_warp, int *total)
     return x + before;
 }
 
+// Block-wide: the request b and chunk index ci of this block's chunk (b = -1 past the last
+// chunk; the grid is an upper bound).  Chunks are numbered request by request, request b
+// owning ceil(len_b / L) of them.  Every thread of the block must call it.
+__device__ __forceinline__ int2 find_chunk(const GdnConv1dArgs &a, int chunk, int L, int *s_warp,
+                                           int *s_ref)
+{
+    const int N32 = (int)a.N;
+    if (threadIdx.x == 0) s_ref[0] = -1;
+    int base = 0;
+    for (int b0 = 0; b0 < a.B; b0 += kThreads) {
+        const int b = b0 + threadIdx.x;
+        int cnt = 0;
+        if (b < a.B) {
+            const int s = (int)min(a.offsets[b], (uint32_t)N32);
+            const int e = (int)min(a.offsets[b + 1], (uint32_t)N32);
+            cnt = e > s ? (int)(((int64_t)(e - s) + L - 1) / L) : 0;
+        }
+        int total;
+        const int incl = block_scan(cnt, s_warp, &total);  // its barriers order s_ref too
+        if (cnt > 0 && chunk >= base + incl - cnt && chunk < base + incl) {
+            s_ref[0] = b;
+            s_ref[1] = chunk - (base + incl - cnt);
+        }
+        base += total;
+        __syncthreads();
+        if (s_ref[0] >= 0 || chunk < base) break;
+    }
+    __syncthreads();
+    return make_int2(s_ref[0], s_ref[1]);
+}
+
+// bounded wait for phase 0 of a copy barrier; false (and GDN_DEV_TIMEOUT) when it does not
+// complete within ~2^31 cycles
+__device__ __forceinline__ bool wait_copies(uint32_t bar, int32_t *dev_status)
+{
+    if (mbar_try_wait(bar, 0)) return true;
+    const long long start = clock64();
+    while (!mbar_try_wait(bar, 0)) {
+        if (clock64() - start > (1ll << 31)) {
+            if (dev_status) atomicOr(dev_status, GDN_DEV_TIMEOUT);
+            return false;
+        }
+    }
+    return true;
+}
+
+// Element path (rows not 16-byte aligned): every access goes through registers.
 template <typename T, int K, bool VEC, int kBatch>
 __global__ void __launch_bounds__(kThreads) conv1d_kernel(const GdnConv1dArgs a, const int L, const int tiles)
 {
     constexpr int V = VEC ? kVecBytes / (int)sizeof(T) : 1;
     constexpr int W = K - 1;
     __shared__ int s_warp[kThreads / 32];
-    __shared__ int s_req, s_chunk;
+    __shared__ int s_ref[2];
 
     // ---- weights first (they do not depend on the request): V channels x K taps
     // the channel tile varies fastest along the grid, so blocks resident together cover
@@ -140,30 +190,10 @@ __global__ void __launch_bounds__(kThreads) conv1d_kernel(const GdnConv1dArgs a,
 
     // ---- which (request, chunk) this block covers
     const int N32 = (int)a.N;
-    if (threadIdx.x == 0) s_req = -1;
-    int base = 0;
-    for (int b0 = 0; b0 < a.B; b0 += kThreads) {
-        const int b = b0 + threadIdx.x;
-        int cnt = 0;
-        if (b < a.B) {
-            const int s = (int)min(a.offsets[b], (uint32_t)N32);
-            const int e = (int)min(a.offsets[b + 1], (uint32_t)N32);
-            cnt = e > s ? (int)(((int64_t)(e - s) + L - 1) / L) : 0;
-        }
-        int total;
-        const int incl = block_scan(cnt, s_warp, &total);  // its barriers order s_req too
-        if (cnt > 0 && chunk >= base + incl - cnt && chunk < base + incl) {
-            s_req = b;
-            s_chunk = chunk - (base + incl - cnt);
-        }
-        base += total;
-        __syncthreads();
-        if (s_req >= 0 || chunk < base) break;
-    }
-    __syncthreads();
-    const int b = s_req;
+    const int2 ref = find_chunk(a, chunk, L, s_warp, s_ref);
+    const int b = ref.x;
     if (b < 0) return;  // past the last chunk (the grid is an upper bound)
-    const int ci = s_chunk;
+    const int ci = ref.y;
     const int s = (int)min(a.offsets[b], (uint32_t)N32);
     const int e = (int)min(a.offsets[b + 1], (uint32_t)N32);
     const uint32_t r = a.slot_idx[b];
@@ -288,6 +318,150 @@ __global__ void __launch_bounds__(kThreads) conv1d_kernel(const GdnConv1dArgs a,
     }
 }
 
+// Vector path (rows 16-byte aligned, conv_dim * sizeof(T) a multiple of 16).  The chunk's
+// rows of this channel tile -- plus the K-1 look-back rows when the chunk is not the
+// request's first -- are staged in shared memory by bulk async copies, one per row, all
+// completing on one mbarrier: up to (L + K-1) x 2 KB in flight per block, independent of
+// the register budget.  Threads then read their 16 bytes per row from shared memory.
+constexpr int kRowBytes = kThreads * 16;  // one row of a channel tile
+constexpr int kStagedMaxL = 32;
+
+template <typename T, int K>
+__global__ void __launch_bounds__(kThreads) conv1d_staged_kernel(const GdnConv1dArgs a,
+                                                                 const int L, const int tiles)
+{
+    constexpr int V = 16 / (int)sizeof(T);
+    constexpr int W = K - 1;
+    extern __shared__ __align__(128) uint8_t stage[];  // (L + W) rows of kRowBytes
+    __shared__ int s_warp[kThreads / 32];
+    __shared__ int s_ref[2];
+    __shared__ __align__(8) uint64_t s_bar;
+
+    const int tile = (int)(blockIdx.x % (unsigned)tiles);
+    const int chunk = (int)(blockIdx.x / (unsigned)tiles);
+    const int tc0 = tile * kThreads * V;  // first channel of the tile
+    const int c0 = tc0 + threadIdx.x * V;
+    const bool has_ch = c0 < a.conv_dim;
+    const uint32_t bar = smem_u32(&s_bar);
+    if (threadIdx.x == 0) {
+        mbar_init(bar, 1);
+        fence_mbar_init();
+    }
+    Flat<T, V * K, true> fw;
+    if (has_ch) fw.load(static_cast<const T *>(a.weight) + (int64_t)c0 * K);
+
+    const int2 ref = find_chunk(a, chunk, L, s_warp, s_ref);  // its barriers publish the init
+    const int b = ref.x;
+    if (b < 0) return;
+    const int ci = ref.y;
+    const int N32 = (int)a.N;
+    const int s = (int)min(a.offsets[b], (uint32_t)N32);
+    const int e = (int)min(a.offsets[b + 1], (uint32_t)N32);
+    const T *__restrict__ x = static_cast<const T *>(a.x);
+    const int64_t ld = a.conv_dim;
+    const int t0 = s + ci * L;
+    const int t1 = min(e, t0 + L);
+    const int r0 = ci > 0 ? t0 - W : t0;  // first staged row
+    const uint32_t row_bytes = (uint32_t)min(kThreads * V, a.conv_dim - tc0) * (uint32_t)sizeof(T);
+    const uint32_t r = __ldg(a.slot_idx + b);
+    if (r >= (uint32_t)a.max_slots) {
+        if (ci == 0 && tile == 0 && threadIdx.x == 0 && a.dev_status)
+            atomicOr(a.dev_status, GDN_DEV_BAD_SLOT);
+        return;
+    }
+    if (threadIdx.x == 0) {
+        const int nrows = t1 - r0;
+        mbar_arrive_expect_tx(bar, (uint32_t)nrows * row_bytes);
+        const T *src = x + (int64_t)r0 * ld + tc0;
+        const uint32_t dst = smem_u32(stage);
+        for (int i = 0; i < nrows; ++i)
+            bulk_load_1d(dst + (uint32_t)i * kRowBytes, src + (int64_t)i * ld, row_bytes, bar);
+    }
+    if (!has_ch) return;  // thread 0 always has channels, so the copies are waited for
+
+    float wf[K][V];
+    {
+        float f[V * K];
+        fw.to_float(f);
+#pragma unroll
+        for (int v = 0; v < V; ++v)
+#pragma unroll
+            for (int j = 0; j < K; ++j) wf[j][v] = f[v * K + j];
+    }
+    float xw[W > 0 ? W : 1][V];
+    T *const slot = W > 0 ? static_cast<T *>(a.conv_state) + ((int64_t)r * a.conv_dim + c0) * W
+                          : nullptr;
+    if (W > 0 && ci == 0) {
+        Flat<T, V * (W > 0 ? W : 1), true> fs;
+        fs.load(slot);
+        float f[V * (W > 0 ? W : 1)];
+        fs.to_float(f);
+#pragma unroll
+        for (int v = 0; v < V; ++v)
+#pragma unroll
+            for (int j = 0; j < W; ++j) xw[j][v] = f[v * W + j];
+    }
+    if (!wait_copies(bar, a.dev_status)) return;
+
+    const uint8_t *sp = stage + threadIdx.x * 16;
+    auto staged = [&](int row, float (&f)[V]) {
+        Flat<T, V, true> fx;
+        fx.w[0] = *reinterpret_cast<const uint4 *>(sp + row * kRowBytes);
+        fx.to_float(f);
+    };
+    if (W > 0 && ci > 0) {
+#pragma unroll
+        for (int j = 0; j < W; ++j) staged(j, xw[j]);
+    }
+    T *op = static_cast<T *>(a.out) + (int64_t)t0 * ld + c0;
+#pragma unroll 4
+    for (int t = t0; t < t1; ++t) {
+        float xn[V], y[V];
+        staged(t - r0, xn);
+#pragma unroll
+        for (int v = 0; v < V; ++v) {
+            float acc = 0.f;
+#pragma unroll
+            for (int j = 0; j < W; ++j) acc = fmaf(wf[j][v], xw[j][v], acc);
+            y[v] = fmaf(wf[W][v], xn[v], acc);
+        }
+#pragma unroll
+        for (int j = 0; j + 1 < W; ++j)
+#pragma unroll
+            for (int v = 0; v < V; ++v) xw[j][v] = xw[j + 1][v];
+        if (W > 0) {
+#pragma unroll
+            for (int v = 0; v < V; ++v) xw[W > 0 ? W - 1 : 0][v] = xn[v];
+        }
+        Flat<T, V, true> fy;
+        fy.from_float(y);
+        fy.store(op, true);
+        op += ld;
+    }
+
+    // new window (chunk 0 only; it read the old one above)
+    if (W > 0 && ci == 0 && a.write_state) {
+        if (t1 < e) {
+            // the request continues past this chunk (so it has >= L >= K-1 tokens): the
+            // window is its last K-1 inputs, read from x
+#pragma unroll
+            for (int j = 0; j < W; ++j) {
+                Flat<T, V, true> fx;
+                fx.load(x + (int64_t)(e - W + j) * ld + c0);
+                fx.to_float(xw[j]);
+            }
+        }
+        float f[V * (W > 0 ? W : 1)];
+#pragma unroll
+        for (int v = 0; v < V; ++v)
+#pragma unroll
+            for (int j = 0; j < W; ++j) f[v * W + j] = xw[j][v];
+        Flat<T, V * (W > 0 ? W : 1), true> fs;
+        fs.from_float(f);
+        fs.store(slot, false);
+    }
+}
+
 int device_sms()
 {
     int dev = 0, n = 0;
@@ -296,12 +470,12 @@ int device_sms()
     return n > 0 ? n : 148;
 }
 
-// tokens per chunk: the largest of 128, 64, ..., 8 that still gives about two
+// tokens per chunk: the largest of max_L, max_L / 2, ..., 8 that still gives about two
 // waves of blocks on the device (L >= 8 >= K-1 always holds)
-int chunk_tokens(int64_t N, int tiles)
+int chunk_tokens(int64_t N, int tiles, int max_L)
 {
     const int64_t target = (int64_t)device_sms() * 16;
-    int L = 128;
+    int L = max_L;
     while (L > 8 && ((N + L - 1) / L) * tiles < target) L >>= 1;
     return L;
 }
@@ -323,12 +497,50 @@ cudaError_t launch_k(const GdnConv1dArgs &a, dim3 grid, int L, int tiles, cudaSt
     return cudaGetLastError();
 }
 
+template <typename T, int K>
+cudaError_t launch_staged_k(const GdnConv1dArgs &a, int L, int tiles, int64_t chunks,
+                            cudaStream_t stream)
+{
+    const size_t smem = (size_t)(L + K - 1) * kRowBytes;
+    static bool attr = false;  // opt in once to the largest stage any call uses
+    if (!attr) {
+        const cudaError_t e = cudaFuncSetAttribute(conv1d_staged_kernel<T, K>,
+                                                   cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                                   (kStagedMaxL + K - 1) * kRowBytes);
+        if (e != cudaSuccess) return e;
+        attr = true;
+    }
+    conv1d_staged_kernel<T, K><<<(unsigned)(chunks * tiles), kThreads, smem, stream>>>(a, L, tiles);
+    return cudaGetLastError();
+}
+
+template <typename T>
+cudaError_t launch_staged(const GdnConv1dArgs &a, cudaStream_t stream)
+{
+    constexpr int V = 16 / (int)sizeof(T);
+    const int tiles = (a.conv_dim + kThreads * V - 1) / (kThreads * V);
+    const int L = chunk_tokens(a.N, tiles, kStagedMaxL);
+    const int64_t chunks = (a.N + L - 1) / L + a.B;  // request-aligned chunks, upper bound
+    if (chunks * tiles > 0x7fffffff) return cudaErrorInvalidConfiguration;
+    switch (a.K) {
+    case 1: return launch_staged_k<T, 1>(a, L, tiles, chunks, stream);
+    case 2: return launch_staged_k<T, 2>(a, L, tiles, chunks, stream);
+    case 3: return launch_staged_k<T, 3>(a, L, tiles, chunks, stream);
+    case 4: return launch_staged_k<T, 4>(a, L, tiles, chunks, stream);
+    case 5: return launch_staged_k<T, 5>(a, L, tiles, chunks, stream);
+    case 6: return launch_staged_k<T, 6>(a, L, tiles, chunks, stream);
+    case 7: return launch_staged_k<T, 7>(a, L, tiles, chunks, stream);
+    case 8: return launch_staged_k<T, 8>(a, L, tiles, chunks, stream);
+    default: return cudaErrorInvalidValue;
+    }
+}
+
 template <typename T, bool VEC>
 cudaError_t launch_t(const GdnConv1dArgs &a, cudaStream_t stream)
 {
     constexpr int V = VEC ? kVecBytes / (int)sizeof(T) : 1;
     const int tiles = (a.conv_dim + kThreads * V - 1) / (kThreads * V);
-    const int L = chunk_tokens(a.N, tiles);
+    const int L = chunk_tokens(a.N, tiles, 128);
     const int64_t chunks = (a.N + L - 1) / L + a.B;  // request-aligned chunks, upper bound
     if (chunks * tiles > 0x7fffffff) return cudaErrorInvalidConfiguration;
     const dim3 grid((unsigned)(chunks * tiles));
@@ -341,7 +553,7 @@ cudaError_t launch_t(const GdnConv1dArgs &a, cudaStream_t stream)
 template <typename T>
 cudaError_t launch_dtype(const GdnConv1dArgs &a, bool vec, cudaStream_t stream)
 {
-    return vec ? launch_t<T, true>(a, stream) : launch_t<T, false>(a, stream);
+    return vec ? launch_staged<T>(a, stream) : launch_t<T, false>(a, stream);
 }
 
 }  // namespace gdn_conv

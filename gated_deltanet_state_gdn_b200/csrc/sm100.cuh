@@ -77,6 +77,17 @@ __device__ __forceinline__ void tma_store_3d(const CUtensorMap *map, uint32_t sr
         : "memory");
 }
 
+// global -> shared bulk copy without a tensor map, completing on an mbarrier (no
+// multicast); dst, src and bytes must be multiples of 16
+__device__ __forceinline__ void bulk_load_1d(uint32_t dst, const void *src, uint32_t bytes,
+                                             uint32_t bar)
+{
+    asm volatile(
+        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(dst),
+        "l"(src), "r"(bytes), "r"(bar)
+        : "memory");
+}
+
 __device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
 
 // wait until every committed bulk store has finished reading shared memory
