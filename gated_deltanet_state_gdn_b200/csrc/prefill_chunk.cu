@@ -224,7 +224,44 @@ __device__ __forceinline__ void st4(float *p, float a, float b, float c, float d
 // --------------------------------------------------------------------------
 // Unit list: requests sorted by length (longest first), heads fastest; unit u
 // goes to CTA (u mod G) on even waves and G-1-(u mod G) on odd waves.
-__device__ void build_unit_list(const Params &p, uint8_t *smem, int batch0, int *count_out)
+// One TMEM lane's row of an initial state S0 (dv fixed, 128 dk; NULL: zero): its bf16 copy
+// into the (1a)/(1b) A-operand columns and gC * S0 into the fp32 state columns.  Runs once per
+// unit, out of line so that the per-chunk code stays compact.
+__device__ __noinline__ void load_state_tmem(const float *init, uint32_t tl, float gC)
+{
+#pragma unroll 1
+    for (int hq = 0; hq < 2; ++hq) {
+        float x[64];
+#pragma unroll
+        for (int c = 0; c < 64; c += 4) {
+            const float4 v = init ? ld4(init + 64 * hq + c) : make_float4(0.f, 0.f, 0.f, 0.f);
+            x[c] = v.x; x[c + 1] = v.y; x[c + 2] = v.z; x[c + 3] = v.w;
+        }
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+            uint32_t w[8];
+#pragma unroll
+            for (int e = 0; e < 8; ++e) w[e] = gdn::pack_bf16x2(x[16 * q + 2 * e], x[16 * q + 2 * e + 1]);
+            tmem_st8u(tl + TM_SB + 8 * (4 * hq + q), w);
+            float y[16];
+#pragma unroll
+            for (int e = 0; e < 16; ++e) y[e] = x[16 * q + e] * gC;
+            tmem_st16(tl + TM_S + 16 * (4 * hq + q), y);
+        }
+    }
+}
+
+// Few requests: every CTA runs the same greedy assignment (requests longest first; the Hv
+// heads of a request go to the Hv CTAs with the least work so far, counted in chunks plus one
+// per unit for the switch, ties to the lower index), so each CTA knows its own list.  Many
+// requests: units in length order dealt to the CTAs wave by wave, alternating direction.
+__device__ __forceinline__ bool greedy_schedule(const Params &p, int G)
+{
+    return p.B <= 32 && G <= 256 && p.B * ((p.Hv + G - 1) / G) <= MAX_UNITS;
+}
+
+__device__ __noinline__ void build_unit_list(const Params &p, uint8_t *smem, int batch0,
+                                             int *count_out)
 {
     // scratch for up to 8192 ints: the two solve areas, idle between batches and written by
     // generic stores only (a TMA destination here would need a proxy fence before its next load)
@@ -246,14 +283,29 @@ __device__ void build_unit_list(const Params &p, uint8_t *smem, int batch0, int 
         s = (int)st;
         l = en > st ? (int)(en - st) : 0;
     };
+    // few requests: ranges read once into shared memory (starts, lengths after ord)
+    const bool small = B <= 32;
+    int *rs = ord + 32, *rl = ord + 64;
+    if (small) {
+        if (tid < B) req_range(tid, rs[tid], rl[tid]);
+        __syncthreads();
+    }
     if (sorted) {
         for (int b = tid; b < B; b += NTHREADS) {
             int sb, lb;
-            req_range(b, sb, lb);
+            if (small) {
+                lb = rl[b];
+            } else {
+                req_range(b, sb, lb);
+            }
             int rank = 0;
             for (int o = 0; o < B; ++o) {
                 int so, lo;
-                req_range(o, so, lo);
+                if (small) {
+                    lo = rl[o];
+                } else {
+                    req_range(o, so, lo);
+                }
                 rank += (lo > lb) || (lo == lb && o < b);
             }
             ord[rank] = b;
@@ -264,6 +316,62 @@ __device__ void build_unit_list(const Params &p, uint8_t *smem, int batch0, int 
     const int U = B * p.Hv;
     const int c = blockIdx.x;
     int4 *list = reinterpret_cast<int4 *>(smem + OFF_UNITS);
+    if (greedy_schedule(p, G)) {
+        // CTAs kept in order of (work so far, index), as packed 64-bit keys: a request's heads
+        // go to the first Hv of the order; the order is then rebuilt by merging the untouched
+        // tail with the updated head (both stay sorted), each thread placing one CTA with a
+        // binary search.
+        long long *key = reinterpret_cast<long long *>(ord + 128);   // two buffers of G keys
+        for (int i = tid; i < G; i += NTHREADS) key[i] = i;
+        if (tid == 0) *count_out = 0;
+        __syncthreads();
+        int cur = 0;
+        for (int r = 0; r < B; ++r) {
+            const int b = ord[r];
+            const int sb = rs[b], lb = rl[b];
+            const long long cost = (long long)((lb + C - 1) / C + 1) << 32;
+            for (int h0 = 0; h0 < p.Hv; h0 += G) {
+                const int m = min(G, p.Hv - h0);   // CTAs taking one head of this request
+                const long long *od = key + cur * 256;
+                long long *nd = key + (cur ^ 1) * 256;
+                long long kx = 0;
+                int npos = 0;
+                if (tid < G) {
+                    kx = od[tid];
+                    int lo, hi;
+                    if (tid < m) {
+                        // updated head entry: count the tail entries below its new key
+                        kx += cost;
+                        lo = m;
+                        hi = G;
+                        while (lo < hi) {
+                            const int mid = (lo + hi) >> 1;
+                            if (od[mid] < kx) lo = mid + 1; else hi = mid;
+                        }
+                        npos = tid + (lo - m);
+                        if ((int)(kx & 0xffffffff) == c) {
+                            list[*count_out] = make_int4(b, h0 + tid, sb, lb);
+                            *count_out += 1;
+                        }
+                    } else {
+                        // untouched tail entry: count the updated head entries below it
+                        lo = 0;
+                        hi = m;
+                        while (lo < hi) {
+                            const int mid = (lo + hi) >> 1;
+                            if (od[mid] + cost < kx) lo = mid + 1; else hi = mid;
+                        }
+                        npos = (tid - m) + lo;
+                    }
+                }
+                __syncthreads();
+                if (tid < G) nd[npos] = kx;
+                __syncthreads();
+                cur ^= 1;
+            }
+        }
+        return;
+    }
     int total = 0;
     const int waves = (U + G - 1) / G;
     for (int w = batch0; w < waves && total < MAX_UNITS; ++w) {
@@ -498,7 +606,9 @@ __global__ void __launch_bounds__(NTHREADS, 1) gdn_prefill_chunk_kernel(const __
         __syncthreads();
         const int nunits = *count_slot;
         int wcover = 0;
-        {
+        if (greedy_schedule(p, G)) {
+            wcover = waves;   // one list holds every unit of this CTA
+        } else {
             int cnt = 0;
             for (int w = batch0; w < waves; ++w) {
                 const int u = w * G + ((w & 1) ? (G - 1 - (int)blockIdx.x) : (int)blockIdx.x);
@@ -983,6 +1093,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) gdn_prefill_chunk_kernel(const __
                 return w_ok;
             };
             float *ogr = reinterpret_cast<float *>(smem + OFF_OGR);
+            bool pre = false;   // this unit's state is already in TMEM
             for (int k = 0; k < nunits; ++k) {
                 const Unit un = load_unit(smem, k);
                 const int nc = (un.len + C - 1) / C;
@@ -997,40 +1108,39 @@ __global__ void __launch_bounds__(NTHREADS, 1) gdn_prefill_chunk_kernel(const __
                     continue;
                 }
                 bool ok = true;
-                // unit start: S0 -> bf16 operand columns and gC(0) * S0 -> TMEM
-                {
+                // unit start: S0 -> bf16 operand columns and gC(0) * S0 -> TMEM, unless the
+                // previous unit's last chunk already did it (pre)
+                if (!pre) {
                     const uint32_t gs = gc % KQ_STAGES;
                     ok = cx.wait(B_GATE_FULL + gs, s_gate[gs] & 1);
                     ++s_gate[gs];
-                    const float *ga = reinterpret_cast<const float *>(smem + OFF_GATE + gs * GATE_BYTES);
-                    const float gC = ga[GA_GC];
-#pragma unroll 1
-                    for (int q = 0; q < 8; ++q) {
-                        float x[16];
-#pragma unroll
-                        for (int c = 0; c < 16; c += 4) {
-                            const float4 v = init ? ld4(init + 16 * q + c) : make_float4(0.f, 0.f, 0.f, 0.f);
-                            x[c] = v.x; x[c + 1] = v.y; x[c + 2] = v.z; x[c + 3] = v.w;
-                        }
-                        uint32_t w[8];
-#pragma unroll
-                        for (int e = 0; e < 8; ++e) w[e] = gdn::pack_bf16x2(x[2 * e], x[2 * e + 1]);
-                        tmem_st8u(tl + TM_SB + 8 * q, w);
-#pragma unroll
-                        for (int e = 0; e < 16; ++e) x[e] *= gC;
-                        tmem_st16(tl + TM_S + 16 * q, x);
-                    }
+                    const float gC = reinterpret_cast<const float *>(smem + OFF_GATE + gs * GATE_BYTES)[GA_GC];
+                    load_state_tmem(init, tl, gC);
                     tmem_wait_st();
                     tc_fence_before();
                     ok = !named_sync_or(2, 128, !ok || cx.aborted());
                     if (dv == 0 && ok) mbar_arrive(cx.bar(B_S_READY));
                 }
+                // a non-empty next unit takes its state at this unit's last E2, before the last
+                // outputs, so that the chain does not wait for them at the switch; its row is
+                // pulled into L2 now
+                const Unit nx = load_unit(smem, min(k + 1, nunits - 1));
+                const bool has_next = k + 1 < nunits && nx.len > 0;
+                const float *next_init =
+                    has_next && p.initial_state
+                        ? p.initial_state + (((int64_t)nx.b * p.Hv + nx.h) * D + dv) * D
+                        : nullptr;
+                if (next_init) {
+#pragma unroll
+                    for (int c = 0; c < D; c += 32) prefetch_l2(next_init + c);
+                }
                 for (int n = 0; n < nc && ok; ++n) {
                     const uint32_t gs = (gc + n) % KQ_STAGES, gs1 = (gc + n + 1) % KQ_STAGES;
                     const int len_n = min(C, un.len - n * C);
                     const float *ga = reinterpret_cast<const float *>(smem + OFF_GATE + gs * GATE_BYTES);
-                    // the -W tile of a unit's first chunk (later ones are converted after E2)
-                    if (n == 0) ok = convert_wneg();
+                    // the -W tile of a unit's first chunk (later ones, and the first of a unit
+                    // that follows a non-empty one, are converted after E2)
+                    if (n == 0 && !pre) ok = convert_wneg();
                     // ---- E1: U^T -> bf16 tiles (plain for Z, decayed and key-normed for S)
                     ok = ok && cx.wait(B_U_DONE, s_u & 1);
                     ++s_u;
@@ -1073,8 +1183,9 @@ __global__ void __launch_bounds__(NTHREADS, 1) gdn_prefill_chunk_kernel(const __
                     ++s_sd;
                     tc_fence_after();
                     const bool more = n + 1 < nc;
+                    const bool chain = more || has_next;   // a state follows in TMEM
                     float gC1 = 1.f;
-                    if (more) {
+                    if (chain) {
                         ok = ok && cx.wait(B_GATE_FULL + gs1, s_gate[gs1] & 1);
                         ++s_gate[gs1];
                         gC1 = reinterpret_cast<const float *>(smem + OFF_GATE + gs1 * GATE_BYTES)[GA_GC];
@@ -1097,7 +1208,8 @@ __global__ void __launch_bounds__(NTHREADS, 1) gdn_prefill_chunk_kernel(const __
                             for (int c = 0; c < 32; c += 4) st4(fin + 32 * q + c, x[c], x[c + 1], x[c + 2], x[c + 3]);
                         }
                     }
-                    if (more) {
+                    if (!more && has_next) load_state_tmem(next_init, tl, gC1);
+                    if (chain) {
                         tmem_wait_st();
                         tc_fence_before();
                         named_sync(2, 128);
@@ -1147,6 +1259,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) gdn_prefill_chunk_kernel(const __
                     ok = !named_sync_or(2, 128, !ok || cx.aborted());
                 }
                 gc += nc;
+                pre = has_next;
                 if (!ok) break;
             }
         }

@@ -88,6 +88,12 @@ __device__ __forceinline__ void bulk_load_1d(uint32_t dst, const void *src, uint
         : "memory");
 }
 
+// pull the 128-byte line holding p into L2
+__device__ __forceinline__ void prefetch_l2(const void *p)
+{
+    asm volatile("prefetch.global.L2 [%0];" ::"l"(p));
+}
+
 __device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
 
 // wait until every committed bulk store has finished reading shared memory
