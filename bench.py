@@ -236,43 +236,77 @@ def time_prefill(gdn, case, steps, warmup, world):
 
 
 def time_prefill_e2e(gdn, case, steps, warmup, world):
-    """Through the public call, from pinned host buffers, with host<->device copies inside."""
-    hq, hk, hv, hg, hb = (t.pin_memory() for t in (case.q, case.k, case.v, case.g, case.beta))
-    hcu = None if case.cu_seqlens is None else case.cu_seqlens.pin_memory()
-    hinit = None if case.initial_state is None else case.initial_state.pin_memory()
+    """Through the public call, from pinned host buffers, with host<->device copies inside.
+
+    Every step copies that step's inputs (q, k, v, g, beta, cu_seqlens, initial state) from
+    pinned host memory, runs gdn_prefill and copies the outputs and final states back to
+    pinned host memory.  Steps are pipelined the way a serving loop would run them: two sets
+    of device buffers, the host-to-device copies on one stream, the call on a second and the
+    device-to-host copies on a third, ordered by events, so that step i+1's input copy
+    overlaps step i's kernel and output copy.  Nothing is skipped: every step moves all of
+    its bytes both ways.
+    """
+    hin = [case.q, case.k, case.v, case.g, case.beta, case.cu_seqlens, case.initial_state]
+    hin = [None if t is None else t.pin_memory() for t in hin]
     Hq, Hv, Dk, Dv = case.dims
-    dq, dk, dv, dg, db = (torch.empty_like(t, device="cuda") for t in (hq, hk, hv, hg, hb))
-    dcu = None if hcu is None else torch.empty_like(hcu, device="cuda")
-    dinit = None if hinit is None else torch.empty_like(hinit, device="cuda")
-    out = torch.empty((case.N, Hv, Dv), dtype=case.q.dtype, device="cuda")
-    fs = torch.empty((case.B, Hv, Dv, Dk), dtype=torch.float32, device="cuda")
-    hout = torch.empty(out.shape, dtype=out.dtype).pin_memory()
-    hfs = torch.empty(fs.shape, dtype=fs.dtype).pin_memory()
-    h2d = sum(t.numel() * t.element_size() for t in (hq, hk, hv, hg, hb, hcu, hinit)
-              if t is not None)
-    d2h = hout.numel() * hout.element_size() + hfs.numel() * hfs.element_size()
+    dins = [[None if t is None else torch.empty_like(t, device="cuda") for t in hin]
+            for _ in range(2)]
+    outs = [torch.empty((case.N, Hv, Dv), dtype=case.q.dtype, device="cuda") for _ in range(2)]
+    fss = [torch.empty((case.B, Hv, Dv, Dk), dtype=torch.float32, device="cuda") for _ in range(2)]
+    hout = [torch.empty(outs[0].shape, dtype=outs[0].dtype).pin_memory() for _ in range(2)]
+    hfs = [torch.empty(fss[0].shape, dtype=torch.float32).pin_memory() for _ in range(2)]
+    h2d = sum(t.numel() * t.element_size() for t in hin if t is not None)
+    d2h = hout[0].numel() * hout[0].element_size() + hfs[0].numel() * hfs[0].element_size()
+    s_in, s_run, s_out = torch.cuda.Stream(), torch.cuda.Stream(), torch.cuda.Stream()
+    copied = [torch.cuda.Event() for _ in range(2)]    # inputs of buffer set j on the device
+    consumed = [torch.cuda.Event() for _ in range(2)]  # the call has read buffer set j
+    done = [torch.cuda.Event() for _ in range(2)]      # outputs of set j written
+    drained = [torch.cuda.Event() for _ in range(2)]   # outputs of set j copied to the host
+    used = [False, False]
 
-    def step():
-        for d, h in ((dq, hq), (dk, hk), (dv, hv), (dg, hg), (db, hb), (dcu, hcu),
-                     (dinit, hinit)):
-            if d is not None:
-                d.copy_(h, non_blocking=True)
-        gdn.gdn_prefill(dq, dk, dv, dg, db, dcu, dinit, fs, out, num_requests=case.B,
-                        scale=case.scale, qk_l2norm=case.qk_l2norm)
-        hout.copy_(out, non_blocking=True)
-        hfs.copy_(fs, non_blocking=True)
+    def step(i):
+        j = i % 2
+        with torch.cuda.stream(s_in):
+            if used[j]:
+                s_in.wait_event(consumed[j])
+            for d, h in zip(dins[j], hin):
+                if d is not None:
+                    d.copy_(h, non_blocking=True)
+            copied[j].record(s_in)
+        with torch.cuda.stream(s_run):
+            s_run.wait_event(copied[j])
+            if used[j]:
+                s_run.wait_event(drained[j])
+            q, k, v, g, b, cu, init = dins[j]
+            gdn.gdn_prefill(q, k, v, g, b, cu, init, fss[j], outs[j], num_requests=case.B,
+                            scale=case.scale, qk_l2norm=case.qk_l2norm, stream=s_run)
+            consumed[j].record(s_run)
+            done[j].record(s_run)
+        with torch.cuda.stream(s_out):
+            s_out.wait_event(done[j])
+            hout[j].copy_(outs[j], non_blocking=True)
+            hfs[j].copy_(fss[j], non_blocking=True)
+            drained[j].record(s_out)
+        used[j] = True
 
-    for _ in range(warmup):
-        step()
-    stream = torch.cuda.current_stream()
+    main = torch.cuda.current_stream()
+    for i in range(warmup):
+        step(i)
+    torch.cuda.synchronize()
     barrier(world)
     torch.cuda.synchronize()
     t0 = torch.cuda.Event(enable_timing=True)
     t1 = torch.cuda.Event(enable_timing=True)
-    t0.record(stream)
-    for _ in range(steps):
-        step()
-    t1.record(stream)
+    t0.record(main)
+    for st in (s_in, s_run, s_out):
+        st.wait_event(t0)
+    for i in range(steps):
+        step(warmup + i)
+    for st in (s_in, s_run, s_out):
+        ev = torch.cuda.Event()
+        ev.record(st)
+        main.wait_event(ev)
+    t1.record(main)
     torch.cuda.synchronize()
     barrier(world)
     return t0.elapsed_time(t1), h2d, d2h
@@ -567,8 +601,8 @@ def main():
 
     e2e = None
     if not args.no_e2e:
-        e_ms, h2d, d2h = time_prefill_e2e(gdn, case, max(3, args.steps // 4), args.warmup, world)
-        e_steps = max(3, args.steps // 4)
+        e_steps = max(4, args.steps // 2)
+        e_ms, h2d, d2h = time_prefill_e2e(gdn, case, e_steps, args.warmup, world)
         e_max = max_over_ranks(e_ms, world) / e_steps
         e2e = {"value": tokens / (e_max / 1e3), "unit": "tokens/s",
                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e_max}
