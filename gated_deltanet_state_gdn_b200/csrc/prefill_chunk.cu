@@ -3,7 +3,9 @@
 // Operation: the recurrence of "com.microsoft.GatedDeltaNet" (Description),
 //   S_t = exp(g_t) S_{t-1} + k_t (beta_t (v_t - exp(g_t) S_{t-1}^T k_t))^T,
 //   o_t = scale * S_t^T q_t,
-// for bf16 q/k/v with Dk = Dv = 128, computed 64 tokens at a time.  The
+// for bf16 q/k/v with Dk, Dv <= 128 (multiples of 8; smaller heads are read as
+// 128-wide tiles zero-filled past their end by the TMA, which leaves every
+// product unchanged), computed 64 tokens at a time.  The
 // chunk form (derived from the recurrence; the op page names a chunk-parallel
 // prefill with chunk_size 64 and states that the chunk size does not change
 // the result) is, for a chunk with incoming state S0 (Dk x Dv), cumulative
@@ -140,6 +142,7 @@ struct __align__(64) Params {
     float scale;
     int32_t qk_l2norm;
     int32_t has_decay, has_retrieval, beta_sigmoid;   // update rule and activations
+    int32_t Dk, Dv;   // head sizes (multiples of 8, <= 128; the tiles are zero-padded to 128)
     const float *a_log, *dt_bias;                     // qwen gate when non-NULL
 };
 
@@ -224,17 +227,20 @@ __device__ __forceinline__ void st4(float *p, float a, float b, float c, float d
 // --------------------------------------------------------------------------
 // Unit list: requests sorted by length (longest first), heads fastest; unit u
 // goes to CTA (u mod G) on even waves and G-1-(u mod G) on odd waves.
-// One TMEM lane's row of an initial state S0 (dv fixed, 128 dk; NULL: zero): its bf16 copy
+// One TMEM lane's row of an initial state S0 (dv fixed, Dk entries, zero beyond; NULL: zero):
+// its bf16 copy
 // into the (1a)/(1b) A-operand columns and gC * S0 into the fp32 state columns.  Runs once per
 // unit, out of line so that the per-chunk code stays compact.
-__device__ __noinline__ void load_state_tmem(const float *init, uint32_t tl, float gC)
+template <bool GENERAL>
+__device__ __noinline__ void load_state_tmem(const float *init, int Dk, uint32_t tl, float gC)
 {
 #pragma unroll 1
     for (int hq = 0; hq < 2; ++hq) {
         float x[64];
 #pragma unroll
         for (int c = 0; c < 64; c += 4) {
-            const float4 v = init ? ld4(init + 64 * hq + c) : make_float4(0.f, 0.f, 0.f, 0.f);
+            const float4 v = init && (!GENERAL || 64 * hq + c < Dk) ? ld4(init + 64 * hq + c)
+                                                                    : make_float4(0.f, 0.f, 0.f, 0.f);
             x[c] = v.x; x[c + 1] = v.y; x[c + 2] = v.z; x[c + 3] = v.w;
         }
 #pragma unroll
@@ -541,6 +547,8 @@ __global__ void __launch_bounds__(NTHREADS, 1) gdn_prefill_chunk_kernel(const __
     const bool has_retrieval = GENERAL ? p.has_retrieval != 0 : true;
     const bool beta_sigmoid = GENERAL ? p.beta_sigmoid != 0 : false;
     const float *const a_log = GENERAL ? p.a_log : nullptr;
+    const int Dk = GENERAL ? p.Dk : D;
+    const int Dv = GENERAL ? p.Dv : D;
     extern __shared__ uint8_t smem_raw[];
     // align the shared-window offset (not the generic address) to 1024 bytes: the
     // 128-byte swizzle of TMA and UMMA is a function of shared-address bits [4, 10)
@@ -1097,13 +1105,17 @@ __global__ void __launch_bounds__(NTHREADS, 1) gdn_prefill_chunk_kernel(const __
             for (int k = 0; k < nunits; ++k) {
                 const Unit un = load_unit(smem, k);
                 const int nc = (un.len + C - 1) / C;
-                const int64_t st_off = (((int64_t)un.b * p.Hv + un.h) * D + dv) * D;
-                const float *init = p.initial_state ? p.initial_state + st_off : nullptr;
-                float *fin = p.final_state + st_off;
+                // this lane's state row (dv < Dv; lanes past Dv carry zero rows)
+                const int64_t st_off = (((int64_t)un.b * p.Hv + un.h) * Dv + dv) * Dk;
+                const bool row_ok = !GENERAL || dv < Dv;
+                const float *init = p.initial_state && row_ok ? p.initial_state + st_off : nullptr;
+                float *fin = row_ok ? p.final_state + st_off : nullptr;
                 if (nc == 0) {
-                    for (int c = 0; c < D; c += 4) {
-                        float4 v = init ? ld4(init + c) : make_float4(0.f, 0.f, 0.f, 0.f);
-                        *reinterpret_cast<float4 *>(fin + c) = v;
+                    if (row_ok) {
+                        for (int c = 0; c < Dk; c += 4) {
+                            float4 v = init ? ld4(init + c) : make_float4(0.f, 0.f, 0.f, 0.f);
+                            *reinterpret_cast<float4 *>(fin + c) = v;
+                        }
                     }
                     continue;
                 }
@@ -1115,7 +1127,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) gdn_prefill_chunk_kernel(const __
                     ok = cx.wait(B_GATE_FULL + gs, s_gate[gs] & 1);
                     ++s_gate[gs];
                     const float gC = reinterpret_cast<const float *>(smem + OFF_GATE + gs * GATE_BYTES)[GA_GC];
-                    load_state_tmem(init, tl, gC);
+                    load_state_tmem<GENERAL>(init, Dk, tl, gC);
                     tmem_wait_st();
                     tc_fence_before();
                     ok = !named_sync_or(2, 128, !ok || cx.aborted());
@@ -1127,12 +1139,11 @@ __global__ void __launch_bounds__(NTHREADS, 1) gdn_prefill_chunk_kernel(const __
                 const Unit nx = load_unit(smem, min(k + 1, nunits - 1));
                 const bool has_next = k + 1 < nunits && nx.len > 0;
                 const float *next_init =
-                    has_next && p.initial_state
-                        ? p.initial_state + (((int64_t)nx.b * p.Hv + nx.h) * D + dv) * D
+                    has_next && p.initial_state && row_ok
+                        ? p.initial_state + (((int64_t)nx.b * p.Hv + nx.h) * Dv + dv) * Dk
                         : nullptr;
                 if (next_init) {
-#pragma unroll
-                    for (int c = 0; c < D; c += 32) prefetch_l2(next_init + c);
+                    for (int c = 0; c < Dk; c += 32) prefetch_l2(next_init + c);
                 }
                 for (int n = 0; n < nc && ok; ++n) {
                     const uint32_t gs = (gc + n) % KQ_STAGES, gs1 = (gc + n + 1) % KQ_STAGES;
@@ -1204,11 +1215,16 @@ __global__ void __launch_bounds__(NTHREADS, 1) gdn_prefill_chunk_kernel(const __
                             for (int e = 0; e < 32; ++e) x[e] *= gC1;
                             tmem_st32(tl + TM_S + 32 * q, x);
                         } else {
+                            if (!GENERAL) {
 #pragma unroll
-                            for (int c = 0; c < 32; c += 4) st4(fin + 32 * q + c, x[c], x[c + 1], x[c + 2], x[c + 3]);
+                                for (int c = 0; c < 32; c += 4) st4(fin + 32 * q + c, x[c], x[c + 1], x[c + 2], x[c + 3]);
+                            } else if (row_ok) {
+                                for (int c = 0; c < 32 && 32 * q + c < Dk; c += 4)
+                                    st4(fin + 32 * q + c, x[c], x[c + 1], x[c + 2], x[c + 3]);
+                            }
                         }
                     }
-                    if (!more && has_next) load_state_tmem(next_init, tl, gC1);
+                    if (!more && has_next) load_state_tmem<GENERAL>(next_init, Dk, tl, gC1);
                     if (chain) {
                         tmem_wait_st();
                         tc_fence_before();
@@ -1228,9 +1244,9 @@ __global__ void __launch_bounds__(NTHREADS, 1) gdn_prefill_chunk_kernel(const __
                         const float sc = p.scale;
                         uint8_t *ost = smem + OFF_OST + 512 * warp;
                         const int tt = lane >> 2;   // token of this lane's 16-byte store
-                        __nv_bfloat16 *obase = p.out + ((int64_t)(un.start + n * C + tt) * p.Hv + un.h) * D +
-                                               32 * warp + 8 * (lane & 3);
-                        const int64_t ostride8 = (int64_t)8 * p.Hv * D;
+                        const int ocol = 32 * warp + 8 * (lane & 3);   // this lane's 8 dv
+                        __nv_bfloat16 *obase = p.out + ((int64_t)(un.start + n * C + tt) * p.Hv + un.h) * Dv + ocol;
+                        const int64_t ostride8 = (int64_t)8 * p.Hv * Dv;
 #pragma unroll 1
                         for (int q = 0; q < 4; ++q) {
                             float y[16], z[16];
@@ -1249,7 +1265,8 @@ __global__ void __launch_bounds__(NTHREADS, 1) gdn_prefill_chunk_kernel(const __
                                 const uint4 v = *reinterpret_cast<const uint4 *>(ost + lane * 16);
                                 __syncwarp();
                                 const int i0 = 16 * q + 8 * hb;   // first token of this group
-                                if (i0 + tt < len_n) *reinterpret_cast<uint4 *>(obase + (i0 / 8) * ostride8) = v;
+                                if (i0 + tt < len_n && (!GENERAL || ocol < Dv))
+                                    *reinterpret_cast<uint4 *>(obase + (i0 / 8) * ostride8) = v;
                             }
                         }
                         tc_fence_before();
@@ -1343,8 +1360,8 @@ int num_sms()
 
 bool prefill_chunked_supported(const GdnPrefillArgs &a)
 {
-    return a.dtype == GDN_BF16 && a.Dk == 128 && a.Dv == 128 && (a.Hv % 4) == 0 &&
-           get_encode() != nullptr;
+    return a.dtype == GDN_BF16 && a.Dk >= 8 && a.Dk <= 128 && a.Dk % 8 == 0 && a.Dv >= 8 &&
+           a.Dv <= 128 && a.Dv % 8 == 0 && (a.Hv % 4) == 0 && get_encode() != nullptr;
 }
 
 cudaError_t launch_prefill_chunked(const GdnPrefillArgs &a, cudaStream_t stream)
@@ -1367,9 +1384,11 @@ cudaError_t launch_prefill_chunked(const GdnPrefillArgs &a, cudaStream_t stream)
     const uint64_t N = (uint64_t)(a.N > 0 ? a.N : 1);
     // TMA maps need a valid base even when N == 0 (no chunk is loaded then)
     if (a.N > 0) {
-        if (!make_map_3d_bf16(&p.tm_q, a.q, 128, a.Hq, N) ||
-            !make_map_3d_bf16(&p.tm_k, a.k, 128, a.Hq, N) ||
-            !make_map_3d_bf16(&p.tm_v, a.v, 128, a.Hv, N) ||
+        // head dims below 128 read zeros past their end (TMA fill), so every tile is a
+        // zero-padded 128-wide tile and the products are unchanged
+        if (!make_map_3d_bf16(&p.tm_q, a.q, a.Dk, a.Hq, N) ||
+            !make_map_3d_bf16(&p.tm_k, a.k, a.Dk, a.Hq, N) ||
+            !make_map_3d_bf16(&p.tm_v, a.v, a.Dv, a.Hv, N) ||
             (a.has_decay && !make_map_2d_f32(&p.tm_g, a.g, a.Hv, N)) ||
             (a.has_retrieval && !make_map_2d_f32(&p.tm_beta, a.beta, a.Hv, N)))
             return cudaErrorInvalidValue;
@@ -1388,11 +1407,14 @@ cudaError_t launch_prefill_chunked(const GdnPrefillArgs &a, cudaStream_t stream)
     p.has_decay = a.has_decay;
     p.has_retrieval = a.has_retrieval;
     p.beta_sigmoid = a.beta_sigmoid;
+    p.Dk = a.Dk;
+    p.Dv = a.Dv;
     p.a_log = a.a_log;
     p.dt_bias = a.dt_bias;
     const int units = a.B * a.Hv;
     const int grid = units < num_sms() ? units : num_sms();
-    const bool general = !a.has_decay || !a.has_retrieval || a.beta_sigmoid || a.a_log != nullptr;
+    const bool general = !a.has_decay || !a.has_retrieval || a.beta_sigmoid || a.a_log != nullptr ||
+                         a.Dk != D || a.Dv != D;
     if (general)
         gdn_prefill_chunk_kernel<true><<<grid, NTHREADS, SMEM_BYTES, stream>>>(p);
     else

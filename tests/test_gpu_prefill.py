@@ -184,7 +184,34 @@ def test_chunked_path_is_selected(gdn):
     assert not gdn.prefill_uses_chunked(torch.bfloat16, 32, 128, 128, sequential=True)
     assert not gdn.prefill_uses_chunked(torch.float32, 32, 128, 128)
     assert not gdn.prefill_uses_chunked(torch.bfloat16, 2, 128, 128)
-    assert not gdn.prefill_uses_chunked(torch.bfloat16, 32, 64, 128)
+    assert gdn.prefill_uses_chunked(torch.bfloat16, 32, 64, 128)
+    assert gdn.prefill_uses_chunked(torch.bfloat16, 32, 8, 8)
+    assert not gdn.prefill_uses_chunked(torch.bfloat16, 32, 60, 128)   # not a multiple of 8
+    assert not gdn.prefill_uses_chunked(torch.bfloat16, 32, 128, 136)  # wider than 128
+    assert not gdn.prefill_uses_chunked(torch.bfloat16, 32, 256, 256)
+
+
+@pytest.mark.parametrize("Dk,Dv", [(64, 64), (128, 64), (64, 128), (96, 32), (8, 8), (120, 128)])
+def test_chunked_other_head_sizes(gdn, W, oracle_mod, Dk, Dv):
+    """Heads narrower than 128 on the tensor-core kernel (zero-padded tiles): ragged requests
+    with an empty one, initial states, the in-kernel norm; every output and final state against
+    the oracle, and no pipeline wait timed out."""
+    assert gdn.prefill_uses_chunked(torch.bfloat16, 4, Dk, Dv)
+    c = W.make_prefill(500 + Dk + Dv, [70, 0, 1, 130, 64], 2, 4, Dk, Dv, init_std=0.1,
+                       qk_l2norm=True)
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    keep = torch.full((c.N, 4, Dv), 7.0, dtype=torch.bfloat16)
+    out, fs = gdn.gdn_prefill(dev(c.q), dev(c.k), dev(c.v), dev(c.g), dev(c.beta),
+                              dev(c.cu_seqlens), dev(c.initial_state), None, dev(keep),
+                              scale=c.scale, qk_l2norm=True, dev_status=status)
+    torch.cuda.synchronize()
+    assert int(status.item()) == 0
+    ro, rf = oracle_prefill_case(oracle_mod, c)
+    assert rel_l2(f64(out), ro) <= TOL_BF16
+    assert rel_l2(f64(fs), rf) <= TOL_BF16
+    # the padded lanes and columns never reach memory: the final state of the empty request is
+    # its initial state, byte for byte
+    assert torch.equal(fs[1].cpu(), c.initial_state[1])
 
 
 @pytest.mark.parametrize("lengths", [[1], [64], [65], [4096, 3, 700], [129, 0, 1, 191, 64]])
