@@ -111,55 +111,98 @@ def decode_bytes(case):
 
 
 class ClockSampler:
-    """nvidia-smi clocks/throttle sampling in the background during timed regions."""
-    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
-              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
-              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    """SM clocks, power and clock-event (throttle) reasons sampled in the background.
+
+    NVML is polled every 5 ms from a thread (reads only; nothing is set); every sample carries
+    its host time, so the summary covers exactly the timed window it is asked about.  Without
+    NVML it falls back to `nvidia-smi -lms 100`.
+    """
+    NAMES = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
 
     def __init__(self, gpu_index):
         self.gpu_index = gpu_index
-        self.rows = []
+        self.rows = []            # (host time, sm MHz, max sm MHz, set of reason names)
         self.proc = None
+        self.stop_flag = threading.Event()
+        self.thread = None
 
     def start(self):
         try:
+            import pynvml
+            pynvml.nvmlInit()
+            self.nvml = pynvml
+            self.handle = pynvml.nvmlDeviceGetHandleByIndex(self.gpu_index)
+            self.max_sm = pynvml.nvmlDeviceGetMaxClockInfo(self.handle, pynvml.NVML_CLOCK_SM)
+            self.bits = {
+                "hw_slowdown": pynvml.nvmlClocksEventReasonHwSlowdown,
+                "hw_thermal_slowdown": pynvml.nvmlClocksEventReasonHwThermalSlowdown,
+                "sw_thermal_slowdown": pynvml.nvmlClocksEventReasonSwThermalSlowdown,
+                "sw_power_cap": pynvml.nvmlClocksEventReasonSwPowerCap,
+            }
+            self.thread = threading.Thread(target=self._poll_nvml, daemon=True)
+            self.thread.start()
+            return
+        except Exception:
+            self.nvml = None
+        try:
+            fields = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+                      "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+                      "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
             self.proc = subprocess.Popen(
-                ["nvidia-smi", f"--id={self.gpu_index}", f"--query-gpu={self.FIELDS}",
+                ["nvidia-smi", f"--id={self.gpu_index}", f"--query-gpu={fields}",
                  "--format=csv,noheader,nounits", "-lms", "100"],
                 stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
-            self.thread = threading.Thread(target=self._read, daemon=True)
+            self.thread = threading.Thread(target=self._read_smi, daemon=True)
             self.thread.start()
         except (OSError, FileNotFoundError):
             self.proc = None
 
-    def _read(self):
+    def _poll_nvml(self):
+        nv = self.nvml
+        while not self.stop_flag.is_set():
+            try:
+                sm = nv.nvmlDeviceGetClockInfo(self.handle, nv.NVML_CLOCK_SM)
+                mask = nv.nvmlDeviceGetCurrentClocksEventReasons(self.handle)
+                active = {n for n, bit in self.bits.items() if mask & bit}
+                self.rows.append((time.time(), float(sm), float(self.max_sm), active))
+            except Exception:
+                pass
+            time.sleep(0.005)
+
+    def _read_smi(self):
         for line in self.proc.stdout:
             parts = [p.strip() for p in line.split(",")]
-            if len(parts) >= 9:
-                self.rows.append(parts)
+            if len(parts) >= 9 and parts[1].replace(".", "").isdigit():
+                active = {n for n, v in zip(self.NAMES, parts[5:9])
+                          if v.strip().lower().startswith("active")}
+                smax = float(parts[2]) if parts[2].replace(".", "").isdigit() else None
+                self.rows.append((time.time(), float(parts[1]), smax, active))
 
     def stop(self):
+        self.stop_flag.set()
         if self.proc is not None:
             self.proc.terminate()
             try:
                 self.proc.wait(timeout=5)
             except subprocess.TimeoutExpired:
                 self.proc.kill()
+        if self.thread is not None:
+            self.thread.join(timeout=5)
 
-    def summary(self):
-        if not self.rows:
-            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"], "samples": 0}
-        sm = [float(r[1]) for r in self.rows if r[1].replace(".", "").isdigit()]
-        smax = [float(r[2]) for r in self.rows if r[2].replace(".", "").isdigit()]
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+    def summary(self, window=None, label="all timed phases"):
+        rows = self.rows if window is None else [r for r in self.rows
+                                                   if window[0] <= r[0] <= window[1]]
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"], "samples": 0,
+                    "window": label}
         reasons = set()
-        for r in self.rows:
-            for n, v in zip(names, r[5:9]):
-                if v.strip().lower().startswith("active"):
-                    reasons.add(n)
-        return {"sm_mhz": statistics.median(sm) if sm else None,
-                "sm_max_mhz": max(smax) if smax else None,
-                "reasons": sorted(reasons), "samples": len(self.rows)}
+        for r in rows:
+            reasons |= r[3]
+        smax = [r[2] for r in rows if r[2] is not None]
+        return {"sm_mhz": statistics.median(r[1] for r in rows),
+                "sm_max_mhz": max(smax) if smax else None, "reasons": sorted(reasons),
+                "samples": len(rows), "window": label,
+                "source": "nvml 5 ms" if self.nvml is not None else "nvidia-smi 100 ms"}
 
 
 def dist_setup():
@@ -222,6 +265,7 @@ def time_prefill(gdn, case, steps, warmup, world):
     torch.cuda.synchronize()
     t0 = torch.cuda.Event(enable_timing=True)
     t1 = torch.cuda.Event(enable_timing=True)
+    host0 = time.time()
     t0.record(stream)
     for s, e in ev:
         s.record(stream)
@@ -229,9 +273,11 @@ def time_prefill(gdn, case, steps, warmup, world):
         e.record(stream)
     t1.record(stream)
     torch.cuda.synchronize()
+    host1 = time.time()
     barrier(world)
     total_ms = t0.elapsed_time(t1)
     launch_ms = [s.elapsed_time(e) for s, e in ev]
+    time_prefill.window = (host0, host1)
     return total_ms, launch_ms
 
 
@@ -400,10 +446,11 @@ def time_conv(gdn, case, steps, warmup, world, graph=False):
 
 
 # ---------------------------------------------------------------- CPU oracle
-def cpu_oracle_sample(case, target_s=10.0):
+def cpu_oracle_sample(case, target_s=10.0, repeats=1):
     """Time the float64 oracle on a bounded sample of the prefill workload: the first L
-    tokens of request 0 with every head; L is grown until one run takes ~target_s/4, then
-    scaled so the whole measurement is ~target_s."""
+    tokens of the packed stream with every head; L is grown until one run takes ~target_s/8,
+    then scaled so that one run is ~target_s (at most the whole stream).  With repeats > 1
+    the calibrated sample is run that many times and the median rate is reported."""
     import oracle
     oracle.build()
     threads = oracle.max_threads()
@@ -431,10 +478,13 @@ def cpu_oracle_sample(case, target_s=10.0):
         L *= 2
         dt = run(L)
     L_final = max(1, min(total, int(L * (target_s / max(dt, 1e-6)))))
-    dt = run(L_final)
+    times = [run(L_final) for _ in range(max(1, repeats))]
+    dt = statistics.median(times)
     return {"value": L_final / dt, "unit": "tokens/s", "cores": threads, "kind": "oracle",
             "sample": f"first {L_final} tokens of the packed stream run as one request, "
-                      f"all {Hv} value heads ({Hq} query/key heads), float64, {dt:.1f} s"}
+                      f"all {Hv} value heads ({Hq} query/key heads), float64, {dt:.2f} s per run"
+                      + (f", median of {len(times)} runs" if len(times) > 1 else ""),
+            "runs": len(times)}
 
 
 def profile_phase(gdn, workloads, args):
@@ -478,7 +528,7 @@ def workload_config(case, name):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--steps", type=int, default=100)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="gdn", choices=["gdn", "reference"])
     ap.add_argument("--workload", default="ragged", choices=["ragged", "long"])
@@ -500,13 +550,10 @@ def main():
         if rank != 0:
             return 0
         case = make_case(args.workload)
-        per = []
-        base = None
-        for _ in range(args.steps):
-            base = cpu_oracle_sample(case, target_s=max(2.0, args.cpu_seconds / 4))
-            per.append(base["value"])
-        val = statistics.median(per)
-        base["value"] = val
+        # K steps of one calibrated sample each, sized so that the run stays near 90 s
+        per_step = min(2.5, max(0.2, 90.0 / max(1, args.steps)))
+        base = cpu_oracle_sample(case, target_s=per_step, repeats=args.steps)
+        val = base["value"]
         print(json.dumps({
             "impl": "reference", "metric": METRIC, "value": val, "unit": "tokens/s",
             "n_gpus": args.gpus, "steps": args.steps, "warmup": 0,
@@ -534,6 +581,7 @@ def main():
                           else local)
     clocks.start()
     total_ms, launch_ms = time_prefill(gdn, case, args.steps, args.warmup, world)
+    prefill_window = time_prefill.window
     max_ms = max_over_ranks(total_ms, world)
     ms_per_step = max_ms / args.steps
     tokens = case.N * world
@@ -621,7 +669,9 @@ def main():
                                                 parallelism=f"replicas{world}"),
             "roofline": roof, "decode": decode, "conv1d": conv, "conv1d_decode": conv_dec,
             "e2e": e2e, "cpu_baseline": cpu,
-            "clocks": clocks.summary(), "gpu_launches": launches,
+            "clocks": clocks.summary(prefill_window, "prefill timed region"),
+            "clocks_all_phases": clocks.summary(),
+            "gpu_launches": launches,
         }
         print(json.dumps(line), flush=True)
     if world > 1:
