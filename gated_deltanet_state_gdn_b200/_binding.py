@@ -34,6 +34,7 @@ GDN_F16 = 2
 GDN_PREFILL_SEQUENTIAL = 1
 GDN_DISABLE_STATE_UPDATE = 2
 GDN_DECODE_QK_L2NORM = 4
+GDN_DECODE_IDX64 = 1 << 7
 GDN_RULE_GATED = 1 << 3
 GDN_RULE_DELTA = 2 << 3
 GDN_RULE_LINEAR = 3 << 3
@@ -228,7 +229,7 @@ def gdn_decode(q, k, v, state_pool, read_idx, A_log, a, dt_bias, b, *, scale=Non
 
     q: [B, T, H, Dk]; k: [B, T, nh, H, Dk]; v: [B, T, nh, HV, Dv] (bf16);
     state_pool: [P, HV, Dv, Dk] fp32 with dense rows (slot/head padding allowed);
-    read_idx, write_idx: [B] int32; scatter_idx: [B, T] int32;
+    read_idx, write_idx: [B] int32 or int64 (the same for both); scatter_idx: [B, T] int32;
     A_log, dt_bias: [HV] fp32; a: [B, T, HV]; b: [B, T, nh, HV] (bf16).
     Returns (out, state_pool).
     """
@@ -239,8 +240,12 @@ def gdn_decode(q, k, v, state_pool, read_idx, A_log, a, dt_bias, b, *, scale=Non
     b = _check_cuda("b", b, torch.bfloat16)
     A_log = _check_cuda("A_log", A_log, torch.float32)
     dt_bias = _check_cuda("dt_bias", dt_bias, torch.float32)
-    read_idx = _check_cuda("read_idx", read_idx, torch.int32)
-    write_idx = _check_cuda("write_idx", write_idx, torch.int32)
+    # read/write slots: int32 or int64 (both the same); scatter slots: int32
+    idx_dtype = read_idx.dtype if isinstance(read_idx, torch.Tensor) else torch.int32
+    if idx_dtype not in (torch.int32, torch.int64):
+        raise TypeError(f"read_idx must be int32 or int64, got {idx_dtype}")
+    read_idx = _check_cuda("read_idx", read_idx, idx_dtype)
+    write_idx = _check_cuda("write_idx", write_idx, idx_dtype)
     scatter_idx = _check_cuda("scatter_idx", scatter_idx, torch.int32)
     if not state_pool.is_cuda or state_pool.dtype != torch.float32 or state_pool.dim() != 4:
         raise TypeError("state_pool must be a 4-d fp32 CUDA tensor")
@@ -257,7 +262,8 @@ def gdn_decode(q, k, v, state_pool, read_idx, A_log, a, dt_bias, b, *, scale=Non
     if scale is None:
         scale = 1.0 / math.sqrt(Dk)
     flags = (GDN_DISABLE_STATE_UPDATE if disable_state_update else 0) | \
-        (GDN_DECODE_QK_L2NORM if use_qk_l2norm else 0)
+        (GDN_DECODE_QK_L2NORM if use_qk_l2norm else 0) | \
+        (GDN_DECODE_IDX64 if idx_dtype == torch.int64 else 0)
     st = lib().gdn_decode(_ptr(q), _ptr(k), _ptr(v), _ptr(state_pool), P, state_pool.stride(0),
                           state_pool.stride(1), _ptr(read_idx), _ptr(write_idx),
                           _ptr(scatter_idx), _ptr(A_log), _ptr(a), _ptr(dt_bias), _ptr(b),

@@ -95,7 +95,9 @@ struct GdnDecodeArgs {
     float *pool;
     int32_t pool_size;
     int64_t slot_stride, head_stride;
-    const int32_t *read_idx, *write_idx, *scatter_idx;
+    const void *read_idx, *write_idx;   // int32, or int64 when idx64
+    const int32_t *scatter_idx;
+    int32_t idx64;
     const float *A_log;
     const void *a;
     const float *dt_bias;

@@ -20,6 +20,13 @@ namespace gdn {
 
 constexpr int kDecodeDk = 128;
 
+// slot index i of an int32 or int64 index array
+__device__ __forceinline__ int64_t slot_at(const void *idx, int i, bool wide)
+{
+    return wide ? (int64_t)__ldg(static_cast<const long long *>(idx) + i)
+                : (int64_t)__ldg(static_cast<const int *>(idx) + i);
+}
+
 template <int DV, int R>
 __global__ void __launch_bounds__(DV / (4 * R) * 32)
 decode_kernel(const GdnDecodeArgs p)
@@ -33,7 +40,7 @@ decode_kernel(const GdnDecodeArgs p)
     const int b = blockIdx.x / HV;
     const int h = blockIdx.x - b * HV;
 
-    const int r = __ldg(p.read_idx + b);
+    const int64_t r = slot_at(p.read_idx, b, p.idx64 != 0);
     if (r < 0) return;  // padding row: nothing is read, computed or stored
     if (r >= p.pool_size) {
         if (p.dev_status && threadIdx.x == 0) atomicOr(p.dev_status, GDN_DEV_BAD_SLOT);
@@ -181,7 +188,7 @@ decode_kernel(const GdnDecodeArgs p)
 
     // 6. end-of-sequence write-back
     if (!p.scatter_idx && !p.disable_state_update) {
-        const int w = p.write_idx ? __ldg(p.write_idx + b) : r;
+        const int64_t w = p.write_idx ? slot_at(p.write_idx, b, p.idx64 != 0) : r;
         if (w >= p.pool_size) {
             if (p.dev_status && threadIdx.x == 0) atomicOr(p.dev_status, GDN_DEV_BAD_SLOT);
         } else if (w >= 0) {

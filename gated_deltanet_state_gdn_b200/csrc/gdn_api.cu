@@ -138,13 +138,13 @@ gdn_status gdn_prefill(const void *q, const void *k, const void *v, const float 
 
 gdn_status gdn_decode(const void *q, const void *k, const void *v, float *state_pool,
                       int32_t pool_size, int64_t slot_stride, int64_t head_stride,
-                      const int32_t *read_idx, const int32_t *write_idx,
+                      const void *read_idx, const void *write_idx,
                       const int32_t *scatter_idx, const float *A_log, const void *a,
                       const float *dt_bias, const void *b, float scale, void *out, int32_t B,
                       int32_t T, int32_t nh, int32_t H, int32_t HV, int32_t Dk, int32_t Dv,
                       uint32_t flags, int32_t *dev_status, void *stream)
 {
-    const uint32_t known = GDN_DISABLE_STATE_UPDATE | GDN_DECODE_QK_L2NORM;
+    const uint32_t known = GDN_DISABLE_STATE_UPDATE | GDN_DECODE_QK_L2NORM | GDN_DECODE_IDX64;
     if (flags & ~known) return GDN_ERR_UNSUPPORTED;
     if (B < 0 || T < 1 || nh < 1 || H < 1 || HV < 1 || Dk < 1 || Dv < 1 || pool_size < 1)
         return GDN_ERR_SHAPE;
@@ -158,9 +158,10 @@ gdn_status gdn_decode(const void *q, const void *k, const void *v, float *state_
         return GDN_ERR_NULL;
     if (!aligned(state_pool, 16) || (slot_stride & 3) || (head_stride & 3))
         return GDN_ERR_ALIGN;
+    const uintptr_t idx_align = (flags & GDN_DECODE_IDX64) ? 8 : 4;
     if (!aligned(q, 8) || !aligned(k, 8) || !aligned(v, 8) || !aligned(out, 8) ||
         !aligned(a, 2) || !aligned(b, 2) || !aligned(A_log, 4) || !aligned(dt_bias, 4) ||
-        !aligned(read_idx, 4) || !aligned(write_idx, 4) || !aligned(scatter_idx, 4))
+        !aligned(read_idx, idx_align) || !aligned(write_idx, idx_align) || !aligned(scatter_idx, 4))
         return GDN_ERR_ALIGN;
     const size_t pool_bytes =
         ((size_t)(pool_size - 1) * slot_stride + (size_t)(HV - 1) * head_stride +
@@ -183,6 +184,7 @@ gdn_status gdn_decode(const void *q, const void *k, const void *v, float *state_
     d.B = B; d.T = T; d.nh = nh; d.H = H; d.HV = HV; d.Dk = Dk; d.Dv = Dv;
     d.disable_state_update = (flags & GDN_DISABLE_STATE_UPDATE) ? 1 : 0;
     d.use_qk_l2norm = (flags & GDN_DECODE_QK_L2NORM) ? 1 : 0;
+    d.idx64 = (flags & GDN_DECODE_IDX64) ? 1 : 0;
     d.dev_status = dev_status;
     cudaError_t e = launch_decode(d, (cudaStream_t)stream);
     if (e != cudaSuccess) return cuda_fail(e, "gdn_decode launch");

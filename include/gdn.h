@@ -63,6 +63,7 @@ enum {
     GDN_PREFILL_SEQUENTIAL = 1u << 0,   /* prefill: force the per-token kernel */
     GDN_DISABLE_STATE_UPDATE = 1u << 1, /* decode: leave the pool unchanged */
     GDN_DECODE_QK_L2NORM = 1u << 2,     /* decode: L2-normalise q and k in the kernel */
+    GDN_DECODE_IDX64 = 1u << 7,         /* decode: read_idx and write_idx are int64 */
     /* prefill update_rule (two bits; 0 = gated_delta, both terms) */
     GDN_RULE_GATED = 1u << 3,           /* decay only: S_t = exp(g_t) S_{t-1} + k_t v_t^T */
     GDN_RULE_DELTA = 2u << 3,           /* retrieval only: g = 0 */
@@ -165,23 +166,26 @@ GDN_API gdn_status gdn_prefill(const void *q, const void *k, const void *v,
  *   state_pool  fp32, slot s head h row j at
  *               state_pool + s*slot_stride + h*head_stride + j*Dk (rows dense);
  *               read and written in place.  pool_size slots.
- *   read_idx [B], write_idx [B] or NULL (= read_idx), scatter_idx [B, T] or NULL: int32
+ *   read_idx [B], write_idx [B] or NULL (= read_idx): int32, or int64 with
+ *          GDN_DECODE_IDX64 (the page allows either); scatter_idx [B, T] or NULL: int32
  *   A_log, dt_bias [HV] float32;  a [B, T, HV] bf16;  b [B, T, nh, HV] bf16
  *   scale  applied as given (the Python binding maps None to 1/sqrt(Dk))
- *   flags  GDN_DISABLE_STATE_UPDATE | GDN_DECODE_QK_L2NORM, or 0
+ *   flags  GDN_DISABLE_STATE_UPDATE | GDN_DECODE_QK_L2NORM | GDN_DECODE_IDX64, or 0
  *   dev_status  optional device int32; GDN_DEV_BAD_SLOT is OR-ed in when a
  *               slot index >= pool_size is met (that read/write is skipped).
  * Requirements: H == HV; Dk == 128; Dv in {64, 128}; 1 <= T <= 16;
  * 1 <= nh <= 4; scatter_idx requires the update enabled; state_pool 16-byte
  * aligned with slot_stride and head_stride multiples of 4 elements,
  * head_stride >= Dv*Dk, slot_stride >= HV*head_stride; q, k, v, out 8-byte
- * aligned.  Rows must not write a slot that another row reads (a row's own
+ * aligned; index arrays aligned to their element size.  A slot index beyond
+ * int32 range is >= pool_size (skipped and flagged).  Rows must not write a
+ * slot that another row reads (a row's own
  * write slot may equal its read slot).
  */
 GDN_API gdn_status gdn_decode(const void *q, const void *k, const void *v,
                       float *state_pool, int32_t pool_size,
                       int64_t slot_stride, int64_t head_stride,
-                      const int32_t *read_idx, const int32_t *write_idx,
+                      const void *read_idx, const void *write_idx,
                       const int32_t *scatter_idx,
                       const float *A_log, const void *a, const float *dt_bias,
                       const void *b, float scale, void *out,

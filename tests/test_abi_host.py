@@ -133,7 +133,9 @@ def test_decode_host_validation(L):
     assert decode(L, ri=None) == 1
     assert decode(L, b=None) == 1
     assert decode(L, out=P(4, 1024)) == 5                 # out inside the pool
-    assert decode(L, flags=1 << 7) == 6
+    assert decode(L, flags=1 << 8) == 6                   # unknown flag
+    assert decode(L, flags=1 << 7, ri=P(5, 4)) == 4       # int64 read slots need 8-byte alignment
+    assert decode(L, flags=1 << 7, wi=P(11, 4)) == 4
     assert decode(L, P=0) == 2
     assert decode(L, B=0) == 0
 

@@ -3,6 +3,8 @@
 Tolerance: relative L2 <= 2e-2 (bf16 activations, fp32 state) on outputs and on
 every written pool slot; pool slots nobody writes must stay bit-identical.
 """
+import copy
+
 import numpy as np
 import pytest
 import torch
@@ -210,3 +212,25 @@ def test_full_mtp(gdn, W, oracle_mod):
     assert rel_l2(f64(pc[sc]), rp[sc]) <= TOL_BF16
     others = [s for s in range(512) if s not in set(sc)]
     assert torch.equal(pc[others], c.pool[others])
+
+
+def test_int64_slot_indices(gdn, W):
+    """int64 read/write slots (the page allows int32 or int64) give the same bytes as int32,
+    padding rows included; an int64 slot beyond int32 range is out of the pool: skipped and
+    flagged."""
+    c = small_case(W, 800, T=2, nh=2, Dv=128, pad_frac=0.25, write_mode="distinct")
+    o32, p32 = run_gpu(gdn, c)
+    c64 = copy.copy(c)
+    c64.read_idx = c.read_idx.to(torch.int64)
+    c64.write_idx = c.write_idx.to(torch.int64)
+    o64, p64 = run_gpu(gdn, c64)
+    assert torch.equal(o32, o64) and torch.equal(p32, p64)
+    big = copy.copy(c64)
+    big.read_idx = c64.read_idx.clone()
+    live = int((c64.read_idx >= 0).nonzero()[0])
+    big.read_idx[live] = (1 << 33) + int(c64.read_idx[live])
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    ob, pb = run_gpu(gdn, big, dev_status=status)
+    assert int(status.item()) == gdn.GDN_DEV_BAD_SLOT
+    keep = [r for r in range(c.read_idx.shape[0]) if r != live]
+    assert torch.equal(ob[keep], o32[keep])
