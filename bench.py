@@ -358,7 +358,11 @@ def time_prefill_e2e(gdn, case, steps, warmup, world):
     return t0.elapsed_time(t1), h2d, d2h
 
 
-def time_decode(gdn, case, steps, warmup, world):
+def time_decode(gdn, case, steps, warmup, world, graph=False):
+    """Per-launch CUDA events around back-to-back launches; with graph=True the `steps` launches
+    are captured in one CUDA graph and replayed once (for launches short enough that the
+    Python call would otherwise show in the events), and the mean per launch is returned for
+    every step."""
     q, k, v, a, b = map(to_dev, (case.q, case.k, case.v, case.a, case.b))
     A_log, dt_bias = to_dev(case.A_log), to_dev(case.dt_bias)
     ri, wi, si = to_dev(case.read_idx), to_dev(case.write_idx), to_dev(case.scatter_idx)
@@ -367,17 +371,35 @@ def time_decode(gdn, case, steps, warmup, world):
     HV, Dv = case.v.shape[3], case.v.shape[4]
     out = torch.zeros((B, T, HV, Dv), dtype=torch.bfloat16, device="cuda")
 
-    def step():
+    def step(stream=None):
         gdn.gdn_decode(q, k, v, pool, ri, A_log, a, dt_bias, b, scale=case.scale, out=out,
-                       scatter_idx=si, use_qk_l2norm=case.use_qk_l2norm, write_idx=wi)
+                       scatter_idx=si, use_qk_l2norm=case.use_qk_l2norm, write_idx=wi,
+                       stream=stream)
 
     for _ in range(warmup):
         step()
     stream = torch.cuda.current_stream()
-    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-          for _ in range(steps)]
     barrier(world)
     torch.cuda.synchronize()
+    if graph:
+        side = torch.cuda.Stream()
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.stream(side):
+            with torch.cuda.graph(g, stream=side):
+                for _ in range(steps):
+                    step(side)
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        g.replay()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        barrier(world)
+        per = e0.elapsed_time(e1) / steps
+        del g, pool
+        return [per] * steps
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(steps)]
     for s, e in ev:
         s.record(stream)
         step()
@@ -608,7 +630,7 @@ def main():
                 "peak": peaks["hbm_gbs"], "unit": "GB/s", "frac": ach / peaks["hbm_gbs"],
                 "traffic": None, "peak_source": peaks["source"]}
 
-    decode = None
+    decode = decode_mtp = None
     if not args.no_decode:
         dcase = workloads.decode_pool_case()
         dms = time_decode(gdn, dcase, args.steps, args.warmup, world)
@@ -622,6 +644,18 @@ def main():
                   "peak_source": peaks["source"]}
         launches += args.steps
         del dcase
+        # MTP / Gated DeltaProduct: T = 4 tokens, 2 Householder sub-steps, per-token scatter
+        mcase = workloads.mtp_case()
+        mms = time_decode(gdn, mcase, args.steps, args.warmup, world, graph=True)
+        mmax = max_over_ranks(sum(mms), world) / args.steps
+        mbytes = decode_bytes(mcase)
+        decode_mtp = {"workload": mcase.name, "value": mbytes * world / (mmax / 1e3) / 1e9,
+                      "unit": "GB/s", "bytes_per_step": mbytes, "ms_per_step": mmax,
+                      "frac": mbytes / (statistics.mean(mms) / 1e3) / 1e9 / peaks["hbm_gbs"],
+                      "peak": peaks["hbm_gbs"], "peak_source": peaks["source"],
+                      "timing": "one CUDA graph of K launches (pool 256 MB)"}
+        launches += args.steps
+        del mcase
 
     conv = conv_dec = None
     if not args.no_conv:
@@ -667,7 +701,8 @@ def main():
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
             "data": "synthetic", "config": dict(workload_config(case, args.workload),
                                                 parallelism=f"replicas{world}"),
-            "roofline": roof, "decode": decode, "conv1d": conv, "conv1d_decode": conv_dec,
+            "roofline": roof, "decode": decode, "decode_mtp": decode_mtp, "conv1d": conv,
+            "conv1d_decode": conv_dec,
             "e2e": e2e, "cpu_baseline": cpu,
             "clocks": clocks.summary(prefill_window, "prefill timed region"),
             "clocks_all_phases": clocks.summary(),

@@ -22,6 +22,15 @@ __device__ __forceinline__ float4 ld_bf16x4(const __nv_bfloat16 *p)
     return make_float4(a.x, a.y, b.x, b.y);
 }
 
+// the same from shared memory (a plain load; the read-only global path does not apply)
+__device__ __forceinline__ float4 lds_bf16x4(const __nv_bfloat16 *p)
+{
+    const uint2 raw = *reinterpret_cast<const uint2 *>(p);
+    const float2 a = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&raw.x));
+    const float2 b = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&raw.y));
+    return make_float4(a.x, a.y, b.x, b.y);
+}
+
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi)
 {
     __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);

@@ -69,10 +69,51 @@ decode_kernel(const GdnDecodeArgs p)
     __nv_bfloat16 *og = static_cast<__nv_bfloat16 *>(p.out);
     const int T = p.T, nh = p.nh, H = p.H;
 
+    // 2. every token's k, q, v rows and gates for this (row, head) staged in shared memory by
+    //    the whole CTA while the state streams in, so that the token loop below waits on no
+    //    global load; alpha and beta are evaluated here once
+    extern __shared__ __align__(16) unsigned char stage_raw[];
+    __nv_bfloat16 *sk = reinterpret_cast<__nv_bfloat16 *>(stage_raw);   // [T][nh][DK]
+    __nv_bfloat16 *sq = sk + T * nh * DK;                                 // [T][DK]
+    __nv_bfloat16 *sv = sq + T * DK;                                      // [T][nh][DV]
+    float *salpha = reinterpret_cast<float *>(sv + T * nh * DV);          // [T]
+    float *sbeta = salpha + T;                                            // [T][nh]
+    {
+        constexpr int RW = DK / 4;   // 8-byte pieces of a k or q row
+        constexpr int VW = DV / 4;
+        const int nk = T * nh * RW, nq = T * RW, nv = T * nh * VW;
+        for (int i = threadIdx.x; i < nk + nq + nv; i += blockDim.x) {
+            if (i < nk) {
+                const int row = i / RW, c = i - row * RW;   // row = t * nh + j
+                const int64_t src = (((int64_t)b * T * nh + row) * H + h) * DK + 4 * c;
+                reinterpret_cast<uint2 *>(sk)[i] = __ldg(reinterpret_cast<const uint2 *>(kg + src));
+            } else if (i < nk + nq) {
+                const int e = i - nk, t = e / RW, c = e - t * RW;
+                const int64_t src = (((int64_t)b * T + t) * H + h) * DK + 4 * c;
+                reinterpret_cast<uint2 *>(sq)[e] = __ldg(reinterpret_cast<const uint2 *>(qg + src));
+            } else {
+                const int e = i - nk - nq, row = e / VW, c = e - row * VW;
+                const int64_t src = (((int64_t)b * T * nh + row) * HV + h) * DV + 4 * c;
+                reinterpret_cast<uint2 *>(sv)[e] = __ldg(reinterpret_cast<const uint2 *>(vg + src));
+            }
+        }
+        for (int i = threadIdx.x; i < T * (1 + nh); i += blockDim.x) {
+            if (i < T) {
+                // alpha = exp(-exp(A_log) * softplus20(a + dt_bias))
+                const int64_t bt = (int64_t)b * T + i;
+                salpha[i] = expf(neg_A * softplus20(bf16_to_f32(ag[bt * HV + h]) + dtb));
+            } else {
+                const int sj = i - T;   // t * nh + j
+                sbeta[sj] = 1.0f / (1.0f + expf(-bf16_to_f32(bg[((int64_t)b * T * nh + sj) * HV + h])));
+            }
+        }
+        __syncthreads();
+    }
+
     for (int t = 0; t < T; ++t) {
         const int64_t bt = (int64_t)b * T + t;
-        // 2. gate: alpha = exp(-exp(A_log) * softplus20(a + dt_bias))
-        const float alpha = expf(neg_A * softplus20(bf16_to_f32(ag[bt * HV + h]) + dtb));
+        // 3. decay by alpha_t
+        const float alpha = salpha[t];
 #pragma unroll
         for (int i = 0; i < R; ++i)
 #pragma unroll
@@ -80,13 +121,13 @@ decode_kernel(const GdnDecodeArgs p)
                 s[i][j].x *= alpha; s[i][j].y *= alpha; s[i][j].z *= alpha; s[i][j].w *= alpha;
             }
 
-        // 3. nh delta sub-steps
+        // 4. nh delta sub-steps
         for (int jh = 0; jh < nh; ++jh) {
-            const int64_t sj = bt * nh + jh;
-            const __nv_bfloat16 *kp = kg + (sj * H + h) * DK + 4 * sub;
+            const int tj = t * nh + jh;
+            const __nv_bfloat16 *kp = sk + tj * DK + 4 * sub;
             float4 kx[4];
 #pragma unroll
-            for (int j = 0; j < 4; ++j) kx[j] = ld_bf16x4(kp + 32 * j);
+            for (int j = 0; j < 4; ++j) kx[j] = lds_bf16x4(kp + 32 * j);
             if (p.use_qk_l2norm) {
                 float ss = 0.f;
 #pragma unroll
@@ -98,11 +139,11 @@ decode_kernel(const GdnDecodeArgs p)
                     kx[j].x *= rn; kx[j].y *= rn; kx[j].z *= rn; kx[j].w *= rn;
                 }
             }
-            const float beta = 1.0f / (1.0f + expf(-bf16_to_f32(bg[sj * HV + h])));
+            const float beta = sbeta[tj];
             float vr[R];
-            const __nv_bfloat16 *vp = vg + (sj * HV + h) * DV + row0;
+            const __nv_bfloat16 *vp = sv + tj * DV + row0;
             if constexpr (R == 4) {
-                float4 v4 = ld_bf16x4(vp);
+                float4 v4 = lds_bf16x4(vp);
                 vr[0] = v4.x; vr[1] = v4.y; vr[2] = v4.z; vr[3] = v4.w;
             } else {
 #pragma unroll
@@ -131,12 +172,12 @@ decode_kernel(const GdnDecodeArgs p)
             }
         }
 
-        // 4. readout o = scale * S q
+        // 5. readout o = scale * S q
         {
-            const __nv_bfloat16 *qp = qg + (bt * H + h) * DK + 4 * sub;
+            const __nv_bfloat16 *qp = sq + t * DK + 4 * sub;
             float4 qx[4];
 #pragma unroll
-            for (int j = 0; j < 4; ++j) qx[j] = ld_bf16x4(qp + 32 * j);
+            for (int j = 0; j < 4; ++j) qx[j] = lds_bf16x4(qp + 32 * j);
             float qs = p.scale;
             if (p.use_qk_l2norm) {
                 float ss = 0.f;
@@ -171,7 +212,7 @@ decode_kernel(const GdnDecodeArgs p)
             }
         }
 
-        // 5. per-token scatter
+        // 6. per-token scatter
         if (p.scatter_idx) {
             const int sidx = __ldg(p.scatter_idx + bt);
             if (sidx >= p.pool_size) {
@@ -186,7 +227,7 @@ decode_kernel(const GdnDecodeArgs p)
         }
     }
 
-    // 6. end-of-sequence write-back
+    // 7. end-of-sequence write-back
     if (!p.scatter_idx && !p.disable_state_update) {
         const int64_t w = p.write_idx ? slot_at(p.write_idx, b, p.idx64 != 0) : r;
         if (w >= p.pool_size) {
@@ -207,12 +248,15 @@ cudaError_t launch_decode(const GdnDecodeArgs &a, cudaStream_t stream)
 {
     const unsigned grid = (unsigned)a.B * (unsigned)a.HV;
     if (grid == 0) return cudaSuccess;
+    // staged k, q, v rows (bf16) and gates (fp32): at most 37 KB (T = 16, nh = 4, Dv = 128)
+    const size_t smem = (size_t)a.T * a.nh * gdn::kDecodeDk * 2 + (size_t)a.T * gdn::kDecodeDk * 2 +
+                        (size_t)a.T * a.nh * a.Dv * 2 + (size_t)a.T * (1 + a.nh) * 4;
     if (a.Dv == 128) {
         constexpr int R = 4;
-        gdn::decode_kernel<128, R><<<grid, 128 / (4 * R) * 32, 0, stream>>>(a);
+        gdn::decode_kernel<128, R><<<grid, 128 / (4 * R) * 32, smem, stream>>>(a);
     } else {
         constexpr int R = 4;
-        gdn::decode_kernel<64, R><<<grid, 64 / (4 * R) * 32, 0, stream>>>(a);
+        gdn::decode_kernel<64, R><<<grid, 64 / (4 * R) * 32, smem, stream>>>(a);
     }
     return cudaGetLastError();
 }

@@ -174,10 +174,12 @@ def test_deterministic(gdn, W):
 
 
 # ---------------------------------------------------------------- full sizes
-def test_full_decode_pool(gdn, W, oracle_mod):
-    """Pool [1024, 32, 128, 128] (2 GiB), B=256 with 13 padding rows: 24 sampled rows against
-    the oracle, every padding row and every slot outside the write set bit-identical."""
-    c = W.decode_pool_case()
+@pytest.mark.parametrize("write_mode", ["distinct", "same"])
+def test_full_decode_pool(gdn, W, oracle_mod, write_mode):
+    """Pool [1024, 32, 128, 128] (2 GiB), B=256 with 13 padding rows, write slots distinct from
+    the read slots or equal to them: 24 sampled rows against the oracle, every padding row and
+    every slot outside the write set bit-identical."""
+    c = W.decode_pool_case(write_mode=write_mode)
     pool = dev(c.pool)
     o, _ = run_gpu(gdn, c, pool_dev=pool)
     reads = c.read_idx.numpy()
