@@ -522,10 +522,10 @@ def profile_phase(gdn, workloads, args):
             print(json.dumps({"phase": "conv", "workload": ccase.name,
                               "ms_per_launch": statistics.mean(cms)}), flush=True)
     else:
-        dcase = workloads.decode_pool_case()
-        dms = time_decode(gdn, dcase, args.steps, args.warmup, 1)
-        print(json.dumps({"phase": "decode", "workload": dcase.name,
-                          "ms_per_launch": statistics.mean(dms)}), flush=True)
+        for dcase in (workloads.decode_pool_case(), workloads.mtp_case()):
+            dms = time_decode(gdn, dcase, args.steps, args.warmup, 1)
+            print(json.dumps({"phase": "decode", "workload": dcase.name,
+                              "ms_per_launch": statistics.mean(dms)}), flush=True)
     return 0
 
 
