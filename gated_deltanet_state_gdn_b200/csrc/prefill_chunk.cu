@@ -53,6 +53,8 @@
 #include <stdio.h>
 #include <string.h>
 
+#include <cuda_fp16.h>
+
 #include "common.cuh"
 #include "sm100.cuh"
 
@@ -127,7 +129,7 @@ static_assert(B_COUNT == (int)NUM_BARS, "barrier count");
 constexpr uint32_t TM_S = 0, TM_U = 128, TM_Y = 192, TM_Z = 256, TM_G = 320, TM_W = 384, TM_SB = 448;
 
 struct __align__(64) Params {
-    CUtensorMap tm_q;     // (128, Hq, N) bf16, box (64, 1, 64), 128B swizzle
+    CUtensorMap tm_q;     // (Dk, Hq, N) bf16 or fp16, box (64, 1, 64), 128B swizzle
     CUtensorMap tm_k;
     CUtensorMap tm_v;     // (128, Hv, N)
     CUtensorMap tm_g;     // (Hv, N) fp32, box (4, 64); encoded only with a decay input
@@ -135,7 +137,7 @@ struct __align__(64) Params {
     const int32_t *cu_seqlens;
     const float *initial_state;
     float *final_state;
-    __nv_bfloat16 *out;
+    uint16_t *out;   // bf16 or fp16 bits, as the activations
     int32_t *dev_status;
     int64_t N;
     int32_t B, Hq, Hv;
@@ -194,24 +196,58 @@ __device__ __forceinline__ uint32_t sw128(uint32_t row, uint32_t c)
     return row * 128u + ((c ^ (row & 7u)) << 4);
 }
 
+// 16-bit operand element: bf16, or fp16 (F16) for fp16 activations; every tile the tensor
+// cores read has the activations' type, since an MMA takes A and B of one type
+template <bool F16>
+__device__ __forceinline__ uint32_t pack2(float lo, float hi)
+{
+    if constexpr (F16) {
+        const __half2 v = __floats2half2_rn(lo, hi);
+        return *reinterpret_cast<const uint32_t *>(&v);
+    } else {
+        return gdn::pack_bf16x2(lo, hi);
+    }
+}
+
+template <bool F16>
+__device__ __forceinline__ uint16_t elem16(float x)
+{
+    if constexpr (F16) {
+        const __half v = __float2half_rn(x);
+        return *reinterpret_cast<const uint16_t *>(&v);
+    } else {
+        const __nv_bfloat16 v = __float2bfloat16_rn(x);
+        return *reinterpret_cast<const uint16_t *>(&v);
+    }
+}
+
+template <bool F16 = false>
 __device__ __forceinline__ uint4 pack8_bf16(const float *x)
 {
     uint4 r;
-    r.x = gdn::pack_bf16x2(x[0], x[1]);
-    r.y = gdn::pack_bf16x2(x[2], x[3]);
-    r.z = gdn::pack_bf16x2(x[4], x[5]);
-    r.w = gdn::pack_bf16x2(x[6], x[7]);
+    r.x = pack2<F16>(x[0], x[1]);
+    r.y = pack2<F16>(x[2], x[3]);
+    r.z = pack2<F16>(x[4], x[5]);
+    r.w = pack2<F16>(x[6], x[7]);
     return r;
 }
 
+template <bool F16 = false>
 __device__ __forceinline__ float sumsq8_bf16(uint4 r)
 {
     const uint32_t w[4] = {r.x, r.y, r.z, r.w};
     float s = 0.f;
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
-        const float lo = __uint_as_float(w[i] << 16);
-        const float hi = __uint_as_float(w[i] & 0xffff0000u);
+        float lo, hi;
+        if constexpr (F16) {
+            const float2 f = __half22float2(*reinterpret_cast<const __half2 *>(&w[i]));
+            lo = f.x;
+            hi = f.y;
+        } else {
+            lo = __uint_as_float(w[i] << 16);
+            hi = __uint_as_float(w[i] & 0xffff0000u);
+        }
         s = fmaf(lo, lo, s);
         s = fmaf(hi, hi, s);
     }
@@ -231,7 +267,7 @@ __device__ __forceinline__ void st4(float *p, float a, float b, float c, float d
 // its bf16 copy
 // into the (1a)/(1b) A-operand columns and gC * S0 into the fp32 state columns.  Runs once per
 // unit, out of line so that the per-chunk code stays compact.
-template <bool GENERAL>
+template <bool GENERAL, bool F16>
 __device__ __noinline__ void load_state_tmem(const float *init, int Dk, uint32_t tl, float gC)
 {
 #pragma unroll 1
@@ -247,7 +283,7 @@ __device__ __noinline__ void load_state_tmem(const float *init, int Dk, uint32_t
         for (int q = 0; q < 4; ++q) {
             uint32_t w[8];
 #pragma unroll
-            for (int e = 0; e < 8; ++e) w[e] = gdn::pack_bf16x2(x[16 * q + 2 * e], x[16 * q + 2 * e + 1]);
+            for (int e = 0; e < 8; ++e) w[e] = pack2<F16>(x[16 * q + 2 * e], x[16 * q + 2 * e + 1]);
             tmem_st8u(tl + TM_SB + 8 * (4 * hq + q), w);
             float y[16];
 #pragma unroll
@@ -437,6 +473,7 @@ __device__ __forceinline__ void blk_store(float *Z, const float (&acc)[2][4], fl
 
 // Block (I, J) of T from an mma fragment (times sgn), written to the bf16 operand
 // tiles Tb = T diag(beta) and Tbg = T diag(beta Gamma rk) (K-major, 128B-swizzled)
+template <bool F16>
 __device__ __forceinline__ void blk_store_tiles(const float (&acc)[2][4], float sgn, int I, int J,
                                                 const float *ga, uint8_t *tb, uint8_t *tbg)
 {
@@ -451,8 +488,8 @@ __device__ __forceinline__ void blk_store_tiles(const float (&acc)[2][4], float 
         for (int h = 0; h < 2; ++h) {
             const float x0 = sgn * acc[nh][2 * h], x1 = sgn * acc[nh][2 * h + 1];
             const uint32_t off = sw128(16 * I + g + 8 * h, j >> 3) + (uint32_t)(j & 7) * 2u;
-            *reinterpret_cast<uint32_t *>(tb + off) = gdn::pack_bf16x2(x0 * b.x, x1 * b.y);
-            *reinterpret_cast<uint32_t *>(tbg + off) = gdn::pack_bf16x2(x0 * bg.x, x1 * bg.y);
+            *reinterpret_cast<uint32_t *>(tb + off) = pack2<F16>(x0 * b.x, x1 * b.y);
+            *reinterpret_cast<uint32_t *>(tbg + off) = pack2<F16>(x0 * bg.x, x1 * bg.y);
         }
     }
 }
@@ -480,6 +517,7 @@ __device__ __forceinline__ int t_slot(int I, int J)
 // row's diagonal block are zero: never stored for A, zero from the start in P.  The
 // exponent of an earlier block J is split as exp(G_i - Gend_J) exp(Gend_J - G_j),
 // both <= 1.
+template <bool F16>
 __device__ __forceinline__ void build_row(uint32_t tl_gram, int qd, const float *ga, float *solve,
                                           uint8_t *ptile, bool retrieval)
 {
@@ -527,8 +565,8 @@ __device__ __forceinline__ void build_row(uint32_t tl_gram, int qd, const float 
         }
         // ---- stores
         if (isP) {
-            *reinterpret_cast<uint4 *>(ptile + sw128(i, 2 * J)) = pack8_bf16(x);
-            *reinterpret_cast<uint4 *>(ptile + sw128(i, 2 * J + 1)) = pack8_bf16(x + 8);
+            *reinterpret_cast<uint4 *>(ptile + sw128(i, 2 * J)) = pack8_bf16<F16>(x);
+            *reinterpret_cast<uint4 *>(ptile + sw128(i, 2 * J + 1)) = pack8_bf16<F16>(x + 8);
         } else {
             float *row = solve + (J == I ? I : a_slot(I, J)) * SOLVE_BLK + r * SOLVE_LD;
 #pragma unroll
@@ -540,7 +578,7 @@ __device__ __forceinline__ void build_row(uint32_t tl_gram, int qd, const float 
 // ========================================================================== kernel
 // GENERAL = false: the default rule (gated_delta, no gate or beta activation), with the
 // variant switches folded at compile time; GENERAL = true reads them from p.
-template <bool GENERAL>
+template <bool GENERAL, bool F16>
 __global__ void __launch_bounds__(NTHREADS, 1) gdn_prefill_chunk_kernel(const __grid_constant__ Params p)
 {
     const bool has_decay = GENERAL ? p.has_decay != 0 : true;
@@ -702,13 +740,13 @@ __global__ void __launch_bounds__(NTHREADS, 1) gdn_prefill_chunk_kernel(const __
             //          UT_DONE(x), S_READY(x); the Y part after Y_FREE(x-1)
             //   C2(x): E1(x)
             if (lane == 0) {
-                constexpr uint32_t ID_G = idesc_bf16(128, 64, 0, 0);
-                constexpr uint32_t ID_W = idesc_bf16(128, 64, 1, 0);
-                constexpr uint32_t ID_U = idesc_bf16(128, 64, 1, 0);
-                constexpr uint32_t ID_1A = idesc_bf16(128, 64, 0, 1);
-                constexpr uint32_t ID_1B = idesc_bf16(128, 64, 0, 0);
-                constexpr uint32_t ID_2 = idesc_bf16(128, 128, 0, 1);
-                constexpr uint32_t ID_3 = idesc_bf16(128, 64, 0, 0);
+                constexpr uint32_t ID_G = idesc_f16kind(128, 64, 0, 0, !F16);
+                constexpr uint32_t ID_W = idesc_f16kind(128, 64, 1, 0, !F16);
+                constexpr uint32_t ID_U = idesc_f16kind(128, 64, 1, 0, !F16);
+                constexpr uint32_t ID_1A = idesc_f16kind(128, 64, 0, 1, !F16);
+                constexpr uint32_t ID_1B = idesc_f16kind(128, 64, 0, 0, !F16);
+                constexpr uint32_t ID_2 = idesc_f16kind(128, 128, 0, 1, !F16);
+                constexpr uint32_t ID_3 = idesc_f16kind(128, 64, 0, 0, !F16);
                 // descriptor bases; a byte offset `o` inside a tile is added as (o >> 4)
                 // KQ stage ks starts (ks * KQ_STAGE) >> 4 descriptor units after stage 0
                 const uint64_t dKQk = sdesc_sw128(sbase + OFF_KQ0, 16, 1024);      // K-major
@@ -891,7 +929,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) gdn_prefill_chunk_kernel(const __
                                     const uint32_t off = sw128(tp, c);
                                     const uint4 va = *reinterpret_cast<const uint4 *>(kq + off);
                                     const uint4 vb = *reinterpret_cast<const uint4 *>(kq + KQ_KB + off);
-                                    ss += sumsq8_bf16(va) + sumsq8_bf16(vb);
+                                    ss += sumsq8_bf16<F16>(va) + sumsq8_bf16<F16>(vb);
                                 }
                                 rn = 1.0f / sqrtf(ss + 1e-12f);
                             }
@@ -958,7 +996,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) gdn_prefill_chunk_kernel(const __
                         ok = ok && cx.wait(B_G_DONE, p_g & 1);
                         ++p_g;
                         tc_fence_after();
-                        build_row(tl + TM_G, pw, ga, solve, smem + OFF_P + ks * P_STAGE, has_retrieval);
+                        build_row<F16>(tl + TM_G, pw, ga, solve, smem + OFF_P + ks * P_STAGE, has_retrieval);
                         if (pw >= 2) fence_proxy_async_smem();
                         // W = T diag(beta Gamma rk) K carries the retrieval term: zero without it
                         if (lt < 64)
@@ -1007,8 +1045,8 @@ __global__ void __launch_bounds__(NTHREADS, 1) gdn_prefill_chunk_kernel(const __
 #pragma unroll
                             for (int r = 0; r < 16; ++r) {
                                 const uint32_t off = sw128(16 * I + r, j >> 3) + cw;
-                                *reinterpret_cast<__nv_bfloat16 *>(smem + OFF_TB + off) = __float2bfloat16_rn(x[r] * bj);
-                                *reinterpret_cast<__nv_bfloat16 *>(smem + OFF_TBG + off) = __float2bfloat16_rn(x[r] * sj);
+                                *reinterpret_cast<uint16_t *>(smem + OFF_TB + off) = elem16<F16>(x[r] * bj);
+                                *reinterpret_cast<uint16_t *>(smem + OFF_TBG + off) = elem16<F16>(x[r] * sj);
                             }
                         }
                         named_sync(3, 128);
@@ -1026,7 +1064,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) gdn_prefill_chunk_kernel(const __
                             blk_mma(acc2, solve + (pw ? 13 : 11) * SOLVE_BLK, tmp);
                             __syncwarp();
                             blk_store(tmp, acc2, -1.f);
-                            blk_store_tiles(acc2, -1.f, pw ? 3 : 1, pw ? 2 : 0, ga, smem + OFF_TB, smem + OFF_TBG);
+                            blk_store_tiles<F16>(acc2, -1.f, pw ? 3 : 1, pw ? 2 : 0, ga, smem + OFF_TB, smem + OFF_TBG);
                         }
                         named_sync(3, 128);
 #pragma unroll 1
@@ -1058,7 +1096,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) gdn_prefill_chunk_kernel(const __
 #pragma unroll 1
                                 for (int t = 0; t < np; ++t) blk_mma(acc, t ? X1 : X0, t ? Y1 : Y0);
                                 if (ph == 0) blk_store(solve + dst * SOLVE_BLK, acc, sgn);
-                                else blk_store_tiles(acc, sgn, 2 + pp, q, ga, smem + OFF_TB, smem + OFF_TBG);
+                                else blk_store_tiles<F16>(acc, sgn, 2 + pp, q, ga, smem + OFF_TB, smem + OFF_TBG);
                             }
                             if (ph == 1) fence_proxy_async_smem();   // T tiles -> UMMA operands
                             named_sync(3, 128);
@@ -1092,7 +1130,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) gdn_prefill_chunk_kernel(const __
                     for (int e = 0; e < 32; ++e) t[e] = -t[e];
 #pragma unroll
                     for (int c = 0; c < 4; ++c)
-                        *reinterpret_cast<uint4 *>(smem + OFF_WNEG + sw128(dv, 4 * q + c)) = pack8_bf16(t + 8 * c);
+                        *reinterpret_cast<uint4 *>(smem + OFF_WNEG + sw128(dv, 4 * q + c)) = pack8_bf16<F16>(t + 8 * c);
                 }
                 fence_proxy_async_smem();
                 tc_fence_before();
@@ -1127,7 +1165,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) gdn_prefill_chunk_kernel(const __
                     ok = cx.wait(B_GATE_FULL + gs, s_gate[gs] & 1);
                     ++s_gate[gs];
                     const float gC = reinterpret_cast<const float *>(smem + OFF_GATE + gs * GATE_BYTES)[GA_GC];
-                    load_state_tmem<GENERAL>(init, Dk, tl, gC);
+                    load_state_tmem<GENERAL, F16>(init, Dk, tl, gC);
                     tmem_wait_st();
                     tc_fence_before();
                     ok = !named_sync_or(2, 128, !ok || cx.aborted());
@@ -1175,8 +1213,8 @@ __global__ void __launch_bounds__(NTHREADS, 1) gdn_prefill_chunk_kernel(const __
                             uint32_t w[16];
 #pragma unroll
                             for (int e = 0; e < 8; ++e) {
-                                w[e] = gdn::pack_bf16x2(u[16 * h + 2 * e], u[16 * h + 2 * e + 1]);
-                                w[8 + e] = gdn::pack_bf16x2(u[16 * h + 2 * e] * d[2 * e], u[16 * h + 2 * e + 1] * d[2 * e + 1]);
+                                w[e] = pack2<F16>(u[16 * h + 2 * e], u[16 * h + 2 * e + 1]);
+                                w[8 + e] = pack2<F16>(u[16 * h + 2 * e] * d[2 * e], u[16 * h + 2 * e + 1] * d[2 * e + 1]);
                             }
                             tmem_st16u(tl + TM_U + t0, w);
                         }
@@ -1209,7 +1247,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) gdn_prefill_chunk_kernel(const __
                         if (more) {
                             uint32_t w[16];
 #pragma unroll
-                            for (int e = 0; e < 16; ++e) w[e] = gdn::pack_bf16x2(x[2 * e], x[2 * e + 1]);
+                            for (int e = 0; e < 16; ++e) w[e] = pack2<F16>(x[2 * e], x[2 * e + 1]);
                             tmem_st16u(tl + TM_SB + 16 * q, w);
 #pragma unroll
                             for (int e = 0; e < 32; ++e) x[e] *= gC1;
@@ -1224,7 +1262,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) gdn_prefill_chunk_kernel(const __
                             }
                         }
                     }
-                    if (!more && has_next) load_state_tmem<GENERAL>(next_init, Dk, tl, gC1);
+                    if (!more && has_next) load_state_tmem<GENERAL, F16>(next_init, Dk, tl, gC1);
                     if (chain) {
                         tmem_wait_st();
                         tc_fence_before();
@@ -1245,7 +1283,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) gdn_prefill_chunk_kernel(const __
                         uint8_t *ost = smem + OFF_OST + 512 * warp;
                         const int tt = lane >> 2;   // token of this lane's 16-byte store
                         const int ocol = 32 * warp + 8 * (lane & 3);   // this lane's 8 dv
-                        __nv_bfloat16 *obase = p.out + ((int64_t)(un.start + n * C + tt) * p.Hv + un.h) * Dv + ocol;
+                        uint16_t *obase = p.out + ((int64_t)(un.start + n * C + tt) * p.Hv + un.h) * Dv + ocol;
                         const int64_t ostride8 = (int64_t)8 * p.Hv * Dv;
 #pragma unroll 1
                         for (int q = 0; q < 4; ++q) {
@@ -1259,8 +1297,8 @@ __global__ void __launch_bounds__(NTHREADS, 1) gdn_prefill_chunk_kernel(const __
                                 const float gg[8] = {g0.x, g0.y, g0.z, g0.w, g1.x, g1.y, g1.z, g1.w};
 #pragma unroll
                                 for (int e = 0; e < 8; ++e)
-                                    *reinterpret_cast<__nv_bfloat16 *>(ost + e * 64 + lane * 2) =
-                                        __float2bfloat16_rn(sc * fmaf(gg[e], y[8 * hb + e], z[8 * hb + e]));
+                                    *reinterpret_cast<uint16_t *>(ost + e * 64 + lane * 2) =
+                                        elem16<F16>(sc * fmaf(gg[e], y[8 * hb + e], z[8 * hb + e]));
                                 __syncwarp();
                                 const uint4 v = *reinterpret_cast<const uint4 *>(ost + lane * 16);
                                 __syncwarp();
@@ -1322,7 +1360,8 @@ PFN_cuTensorMapEncodeTiled_v12000 get_encode()
     return fn;
 }
 
-bool make_map_3d_bf16(CUtensorMap *m, const void *base, uint64_t d0, uint64_t d1, uint64_t d2)
+bool make_map_3d_16(CUtensorMap *m, const void *base, uint64_t d0, uint64_t d1, uint64_t d2,
+                    bool f16)
 {
     auto enc = get_encode();
     if (!enc) return false;
@@ -1330,7 +1369,8 @@ bool make_map_3d_bf16(CUtensorMap *m, const void *base, uint64_t d0, uint64_t d1
     cuuint64_t strides[2] = {d0 * 2, d0 * d1 * 2};
     cuuint32_t box[3] = {64, 1, 64};
     cuuint32_t estr[3] = {1, 1, 1};
-    return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(base), dims, strides,
+    return enc(m, f16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3,
+               const_cast<void *>(base), dims, strides,
                box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
@@ -1360,7 +1400,8 @@ int num_sms()
 
 bool prefill_chunked_supported(const GdnPrefillArgs &a)
 {
-    return a.dtype == GDN_BF16 && a.Dk >= 8 && a.Dk <= 128 && a.Dk % 8 == 0 && a.Dv >= 8 &&
+    return (a.dtype == GDN_BF16 || a.dtype == GDN_F16) && a.Dk >= 8 && a.Dk <= 128 &&
+           a.Dk % 8 == 0 && a.Dv >= 8 &&
            a.Dv <= 128 && a.Dv % 8 == 0 && (a.Hv % 4) == 0 && get_encode() != nullptr;
 }
 
@@ -1370,11 +1411,14 @@ cudaError_t launch_prefill_chunked(const GdnPrefillArgs &a, cudaStream_t stream)
     if (a.B == 0) return cudaSuccess;
     static bool attr_set = false;
     if (!attr_set) {
-        cudaError_t e = cudaFuncSetAttribute(gdn_prefill_chunk_kernel<false>,
+        cudaError_t e = cudaFuncSetAttribute(gdn_prefill_chunk_kernel<false, false>,
                                              cudaFuncAttributeMaxDynamicSharedMemorySize,
                                              (int)SMEM_BYTES);
         if (e == cudaSuccess)
-            e = cudaFuncSetAttribute(gdn_prefill_chunk_kernel<true>,
+            e = cudaFuncSetAttribute(gdn_prefill_chunk_kernel<true, false>,
+                                     cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SMEM_BYTES);
+        if (e == cudaSuccess)
+            e = cudaFuncSetAttribute(gdn_prefill_chunk_kernel<true, true>,
                                      cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SMEM_BYTES);
         if (e != cudaSuccess) return e;
         attr_set = true;
@@ -1386,9 +1430,10 @@ cudaError_t launch_prefill_chunked(const GdnPrefillArgs &a, cudaStream_t stream)
     if (a.N > 0) {
         // head dims below 128 read zeros past their end (TMA fill), so every tile is a
         // zero-padded 128-wide tile and the products are unchanged
-        if (!make_map_3d_bf16(&p.tm_q, a.q, a.Dk, a.Hq, N) ||
-            !make_map_3d_bf16(&p.tm_k, a.k, a.Dk, a.Hq, N) ||
-            !make_map_3d_bf16(&p.tm_v, a.v, a.Dv, a.Hv, N) ||
+        const bool f16 = a.dtype == GDN_F16;
+        if (!make_map_3d_16(&p.tm_q, a.q, a.Dk, a.Hq, N, f16) ||
+            !make_map_3d_16(&p.tm_k, a.k, a.Dk, a.Hq, N, f16) ||
+            !make_map_3d_16(&p.tm_v, a.v, a.Dv, a.Hv, N, f16) ||
             (a.has_decay && !make_map_2d_f32(&p.tm_g, a.g, a.Hv, N)) ||
             (a.has_retrieval && !make_map_2d_f32(&p.tm_beta, a.beta, a.Hv, N)))
             return cudaErrorInvalidValue;
@@ -1396,7 +1441,7 @@ cudaError_t launch_prefill_chunked(const GdnPrefillArgs &a, cudaStream_t stream)
     p.cu_seqlens = a.cu_seqlens;
     p.initial_state = a.initial_state;
     p.final_state = a.final_state;
-    p.out = static_cast<__nv_bfloat16 *>(a.out);
+    p.out = static_cast<uint16_t *>(a.out);
     p.dev_status = a.dev_status;
     p.N = a.N;
     p.B = a.B;
@@ -1415,9 +1460,12 @@ cudaError_t launch_prefill_chunked(const GdnPrefillArgs &a, cudaStream_t stream)
     const int grid = units < num_sms() ? units : num_sms();
     const bool general = !a.has_decay || !a.has_retrieval || a.beta_sigmoid || a.a_log != nullptr ||
                          a.Dk != D || a.Dv != D;
-    if (general)
-        gdn_prefill_chunk_kernel<true><<<grid, NTHREADS, SMEM_BYTES, stream>>>(p);
+    // fp16 activations run the general instantiation with fp16 operand tiles
+    if (a.dtype == GDN_F16)
+        gdn_prefill_chunk_kernel<true, true><<<grid, NTHREADS, SMEM_BYTES, stream>>>(p);
+    else if (general)
+        gdn_prefill_chunk_kernel<true, false><<<grid, NTHREADS, SMEM_BYTES, stream>>>(p);
     else
-        gdn_prefill_chunk_kernel<false><<<grid, NTHREADS, SMEM_BYTES, stream>>>(p);
+        gdn_prefill_chunk_kernel<false, false><<<grid, NTHREADS, SMEM_BYTES, stream>>>(p);
     return cudaGetLastError();
 }

@@ -316,13 +316,13 @@ __device__ __forceinline__ uint64_t sdesc_sw128(uint32_t saddr, uint32_t lbo, ui
     return d;
 }
 
-// Instruction descriptor for kind::f16 with bf16 A/B and fp32 D.
+// Instruction descriptor for kind::f16 with bf16 (bf16 = true) or fp16 A/B and fp32 D.
 // a_mn / b_mn: operand is MN-major (1) or K-major (0).
-__host__ __device__ constexpr uint32_t idesc_bf16(int M, int N, int a_mn, int b_mn)
+__host__ __device__ constexpr uint32_t idesc_f16kind(int M, int N, int a_mn, int b_mn, bool bf16)
 {
-    return (1u << 4)                       // D format: f32
-           | (1u << 7)                     // A format: bf16
-           | (1u << 10)                    // B format: bf16
+    return (1u << 4)                              // D format: f32
+           | ((bf16 ? 1u : 0u) << 7)              // A format: bf16 (1) or f16 (0)
+           | ((bf16 ? 1u : 0u) << 10)             // B format: the same
            | ((uint32_t)a_mn << 15) | ((uint32_t)b_mn << 16) |
            ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
 }

@@ -55,7 +55,7 @@ typedef enum {
 typedef enum {
     GDN_F32 = 0,   /* float32 activations */
     GDN_BF16 = 1,  /* bfloat16 activations */
-    GDN_F16 = 2    /* float16 activations (prefill per-token kernel, conv1d) */
+    GDN_F16 = 2    /* float16 activations (prefill, conv1d) */
 } gdn_dtype;
 
 /* flags */
@@ -125,10 +125,11 @@ enum {
  *                  bound (the call's outputs are then invalid).
  * Requirements: 1 <= Dk, Dv <= 256; Hv % Hq == 0; q, k, v, out,
  * initial_state and final_state 16-byte aligned; out must not overlap any
- * input.  bf16 with Dk, Dv in {8, 16, ..., 128} and Hv % 4 == 0 runs the chunked
- * tensor-core kernel (unless GDN_PREFILL_SEQUENTIAL); everything else (fp32,
- * fp16, heads wider than 128 or not a multiple of 8) runs the per-token kernel,
- * which computes in fp32.  The chunked kernel floors each g at -30
+ * input.  bf16 or fp16 with Dk, Dv in {8, 16, ..., 128} and Hv % 4 == 0 runs the
+ * chunked tensor-core kernel (unless GDN_PREFILL_SEQUENTIAL; its operand tiles
+ * take the activations' type, fp32 accumulation and state); everything else
+ * (fp32, heads wider than 128 or not a multiple of 8) runs the per-token
+ * kernel, which computes in fp32.  The chunked kernel floors each g at -30
  * (exp(-30) ~ 9e-14) so that in-chunk decay differences stay finite.
  * Overlapping request ranges are not supported (their outputs are undefined).
  */
@@ -235,7 +236,7 @@ GDN_API gdn_status gdn_conv1d(const void *x, const void *weight, void *conv_stat
 
 /* 1 when gdn_prefill with these arguments runs the chunked tensor-core
  * kernel, 0 when it runs the per-token kernel (host-only query, no launch).
- * The chunked kernel takes bf16 with Dk and Dv multiples of 8 up to 128 (smaller heads
+ * The chunked kernel takes bf16 or fp16 with Dk and Dv multiples of 8 up to 128 (smaller heads
  * run as zero-padded 128-wide tiles) and Hv % 4 == 0. */
 GDN_API int32_t gdn_prefill_uses_chunked(gdn_dtype dtype, int32_t Hv, int32_t Dk, int32_t Dv,
                                          uint32_t flags);

@@ -3,9 +3,11 @@ the update rules of "com.microsoft.GatedDeltaNet" (Attributes table: linear, gat
 gated_delta), its qwen gate and sigmoid beta activations, and float16 activations.
 
 Tolerances (relative L2 over the whole tensor): 2e-2 for bf16 activations with the fp32
-state (as for the default rule); 2e-3 for fp16 activations, whose only rounding against the
-oracle is the fp16 cast of the outputs (unit roundoff 2^-11 ~ 4.9e-4) on top of the fp32
-state arithmetic.
+state (as for the default rule). For fp16 activations on the per-token kernel 2e-3: its only
+rounding against the oracle is the fp16 cast of the outputs (unit roundoff 2^-11 ~ 4.9e-4) on
+top of the fp32 state arithmetic. For fp16 on the tensor-core kernel 2.5e-3: every MMA operand
+(q, k, v and the T, P, -W, U and state tiles) is rounded to fp16, and the bf16 bound 2e-2 is about
+five bf16 unit roundoffs (2^-8), so the same five fp16 unit roundoffs give 2.5e-3.
 """
 import numpy as np
 import pytest
@@ -16,6 +18,7 @@ from _util import TOL_BF16, dev, f64, rel_l2
 pytestmark = pytest.mark.gpu
 
 TOL_F16 = 2e-3
+TOL_F16_CHUNKED = 2.5e-3
 RULES = {"gated_delta": (True, True), "gated": (True, False), "delta": (False, True),
          "linear": (False, False)}
 LENGTHS = [1, 64, 65, 200, 0, 130]
@@ -82,16 +85,30 @@ def test_qwen_gate_and_sigmoid_beta(gdn, W, oracle_mod, rule, sequential):
     assert rel_l2(f, rf) <= TOL_BF16, rule
 
 
+@pytest.mark.parametrize("sequential", [True, False])
 @pytest.mark.parametrize("Dk,Dv", [(128, 128), (64, 32)])
-def test_fp16_activations(gdn, W, oracle_mod, Dk, Dv):
-    """float16 q/k/v/out run the per-token kernel (fp32 arithmetic); the oracle reads the same
-    fp16-rounded inputs."""
-    assert not gdn.prefill_uses_chunked(torch.float16, 4, Dk, Dv)
+def test_fp16_activations(gdn, W, oracle_mod, Dk, Dv, sequential):
+    """float16 q/k/v/out on the per-token kernel (fp32 arithmetic) and on the tensor-core kernel
+    (fp16 operand tiles); the oracle reads the same fp16-rounded inputs."""
+    assert gdn.prefill_uses_chunked(torch.float16, 4, Dk, Dv)
     c = W.make_prefill(34, LENGTHS, 2, 4, Dk, Dv, dtype=torch.float16, init_std=0.02,
                        qk_l2norm=True)
-    o, f, ro, rf = _run_both(gdn, oracle_mod, c, c.g, c.beta, False)
-    assert o.dtype == np.float64 and rel_l2(o, ro) <= TOL_F16
-    assert rel_l2(f, rf) <= TOL_F16
+    o, f, ro, rf = _run_both(gdn, oracle_mod, c, c.g, c.beta, sequential)
+    tol = TOL_F16 if sequential else TOL_F16_CHUNKED
+    assert o.dtype == np.float64 and rel_l2(o, ro) <= tol
+    assert rel_l2(f, rf) <= tol
+
+
+@pytest.mark.parametrize("rule", ["delta", "linear"])
+def test_fp16_rules_on_tensor_cores(gdn, W, oracle_mod, rule):
+    """The fp16 tensor-core kernel with the rule switches (general instantiation)."""
+    has_decay, has_beta = RULES[rule]
+    c = W.make_prefill(36, LENGTHS, 2, 4, 128, 128, dtype=torch.float16, init_std=0.02,
+                       qk_l2norm=True)
+    o, f, ro, rf = _run_both(gdn, oracle_mod, c, c.g if has_decay else None,
+                             c.beta if has_beta else None, False, update_rule=rule)
+    assert rel_l2(o, ro) <= TOL_F16_CHUNKED, rule
+    assert rel_l2(f, rf) <= TOL_F16_CHUNKED, rule
 
 
 def test_linear_rule_long_sequence_matches_oracle(gdn, W, oracle_mod):
