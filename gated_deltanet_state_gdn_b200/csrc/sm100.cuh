@@ -1,5 +1,5 @@
-// sm100.cuh -- thin inline-PTX wrappers for the sm_100a features the chunked
-// prefill kernel uses: mbarriers, TMA tensor loads, tcgen05 (TMEM allocation,
+// sm100.cuh -- thin inline-PTX wrappers for the sm_100a features the kernels
+// use: mbarriers, bulk and TMA tensor loads, cp.async, tcgen05 (TMEM allocation,
 // UMMA issue/commit, TMEM load/store, fences) and warp-level tf32 mma.
 //
 // Descriptor formats (shared-memory matrix descriptor and the instruction
@@ -76,6 +76,19 @@ __device__ __forceinline__ void bulk_load_1d(uint32_t dst, const void *src, uint
         "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(dst),
         "l"(src), "r"(bytes), "r"(bar)
         : "memory");
+}
+
+// 8-byte global -> shared asynchronous copy (dst and src 8-byte aligned)
+__device__ __forceinline__ void cp_async8(uint32_t dst, const void *src)
+{
+    asm volatile("cp.async.ca.shared.global [%0], [%1], 8;" ::"r"(dst), "l"(src) : "memory");
+}
+
+// one arrival on `bar` once every cp.async this thread issued so far has landed; the arrival
+// counts toward the barrier's expected count (.noinc)
+__device__ __forceinline__ void cp_async_arrive(uint32_t bar)
+{
+    asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(bar) : "memory");
 }
 
 // pull the 128-byte line holding p into L2

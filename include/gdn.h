@@ -173,7 +173,9 @@ GDN_API gdn_status gdn_prefill(const void *q, const void *k, const void *v,
  *   scale  applied as given (the Python binding maps None to 1/sqrt(Dk))
  *   flags  GDN_DISABLE_STATE_UPDATE | GDN_DECODE_QK_L2NORM | GDN_DECODE_IDX64, or 0
  *   dev_status  optional device int32; GDN_DEV_BAD_SLOT is OR-ed in when a
- *               slot index >= pool_size is met (that read/write is skipped).
+ *               slot index >= pool_size is met (that read/write is skipped);
+ *               GDN_DEV_TIMEOUT if a copy into shared memory did not complete
+ *               within its bound (the CTA stops; outputs invalid).
  * Requirements: H == HV; Dk == 128; Dv in {64, 128}; 1 <= T <= 16;
  * 1 <= nh <= 4; scatter_idx requires the update enabled; state_pool 16-byte
  * aligned with slot_stride and head_stride multiples of 4 elements,

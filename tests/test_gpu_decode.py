@@ -236,3 +236,86 @@ def test_int64_slot_indices(gdn, W):
     assert int(status.item()) == gdn.GDN_DEV_BAD_SLOT
     keep = [r for r in range(c.read_idx.shape[0]) if r != live]
     assert torch.equal(ob[keep], o32[keep])
+
+
+# ---------------------------------------------------------------- launch forms
+def sub_case(c, rows):
+    """The rows `rows` of decode case c as a case of their own (same pool)."""
+    s = copy.copy(c)
+    for name in ("q", "k", "v", "a", "b", "read_idx", "write_idx", "scatter_idx"):
+        t = getattr(c, name)
+        if t is not None:
+            setattr(s, name, t[rows].contiguous())
+    return s
+
+
+@pytest.mark.parametrize("Dv", [64, 128])
+def test_launch_forms_agree(gdn, W, oracle_mod, Dv):
+    """Single-token rows that fill many waves of CTAs take the one-CTA-per-(row, head) form; the
+    same rows called 8 at a time take the persistent form.  Both run the same per-unit
+    arithmetic, so outputs and the pool agree bit for bit, padding rows, a read slot beyond the
+    pool and a write slot beyond the pool included; sampled rows match the oracle."""
+    B, P = 160, 352
+    c = W.make_decode(900 + Dv, P=P, B=B, T=1, nh=1, H=32, Dv=Dv, pad_frac=0.1,
+                      write_mode="distinct")
+    reads = c.read_idx.numpy()
+    live = np.nonzero(reads >= 0)[0]
+    c.read_idx[int(live[3])] = P + 5
+    c.write_idx[int(live[7])] = P + 7
+    sentinel = torch.full((B, 1, 32, Dv), 3.0, dtype=torch.bfloat16)
+
+    status_all = torch.zeros(1, dtype=torch.int32, device="cuda")
+    pool_all = dev(c.pool)
+    o_all, _ = run_gpu(gdn, c, pool_dev=pool_all, out=sentinel, dev_status=status_all)
+
+    status_8 = torch.zeros(1, dtype=torch.int32, device="cuda")
+    pool_8 = dev(c.pool)
+    o_8 = []
+    for r0 in range(0, B, 8):
+        sc = sub_case(c, slice(r0, r0 + 8))
+        o, _ = run_gpu(gdn, sc, pool_dev=pool_8, out=sentinel[r0:r0 + 8], dev_status=status_8)
+        o_8.append(o)
+    o_8 = torch.cat(o_8)
+    assert int(status_all.item()) == gdn.GDN_DEV_BAD_SLOT == int(status_8.item())
+    assert torch.equal(o_all, o_8)
+    assert torch.equal(pool_all, pool_8)
+
+    ok = [int(r) for r in live if r not in (live[3], live[7])]
+    rows = np.sort(np.random.default_rng(1).choice(ok, 12, replace=False))
+    ro, rp = run_oracle(oracle_mod, c, rows=rows)
+    oc = o_all.cpu()
+    assert rel_l2(f64(oc[torch.from_numpy(rows)]), ro) <= TOL_BF16
+    for i, r in enumerate(rows):
+        assert rel_l2(f64(pool_all[int(c.write_idx[r])].cpu()), rp[i]) <= TOL_BF16
+    skipped = np.nonzero(c.read_idx.numpy() < 0)[0].tolist() + [int(live[3])]
+    assert torch.equal(oc[skipped], sentinel[skipped])
+
+
+def test_stream_form_walks_many_units(gdn, W, oracle_mod):
+    """Persistent form with several (row, head) units per CTA: padding rows, a read slot beyond
+    the pool and scatter entries of -1 interleaved with live units; every output and pool slot
+    against the oracle."""
+    B, P = 64, 200
+    c = W.make_decode(950, P=P, B=B, T=2, nh=2, H=32, Dv=64, pad_frac=0.2,
+                      write_mode="none", scatter=True)
+    live = np.nonzero(c.read_idx.numpy() >= 0)[0]
+    c.scatter_idx[int(live[0]), 1] = -1
+    c.scatter_idx[int(live[5]), 0] = -1
+    bad = int(live[9])
+    c.read_idx[bad] = P + 1
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    sentinel = torch.full((B, 2, 32, 64), -4.0, dtype=torch.bfloat16)
+    o, pool = run_gpu(gdn, c, out=sentinel, dev_status=status)
+    assert int(status.item()) == gdn.GDN_DEV_BAD_SLOT
+    ok = [r for r in range(B) if r != bad]
+    good = sub_case(c, ok)
+    ro, rp = run_oracle(oracle_mod, good, out=sentinel[ok])
+    assert rel_l2(f64(o.cpu()[ok]), ro) <= TOL_BF16
+    pc = pool.cpu()
+    sc = set(int(x) for r in ok if c.read_idx[r] >= 0 for x in c.scatter_idx[r].tolist() if x >= 0)
+    for s in range(P):
+        if s in sc:
+            assert rel_l2(f64(pc[s]), rp[s]) <= TOL_BF16, s
+        else:
+            assert torch.equal(pc[s], c.pool[s]), s
+    assert torch.equal(o.cpu()[bad], sentinel[bad])
