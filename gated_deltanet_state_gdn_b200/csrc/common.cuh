@@ -5,6 +5,8 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <atomic>
+
 #include "gdn.h"
 
 namespace gdn {
@@ -130,6 +132,25 @@ struct GdnConv1dArgs {
     int64_t N;
     int32_t dtype, write_state;
     int32_t *dev_status;
+};
+
+// Host-side setup done once per device (kernel attribute opt-ins): run() calls f() unless it
+// already succeeded on the current device.  Threads that race may both call f, which must
+// therefore be idempotent; devices numbered 32 and up call it every time.
+struct DeviceOnce {
+    std::atomic<uint32_t> done{0};
+    template <class F>
+    cudaError_t run(F &&f)
+    {
+        int dev = 0;
+        cudaError_t e = cudaGetDevice(&dev);
+        if (e != cudaSuccess) return e;
+        const uint32_t bit = dev < 32 ? (1u << dev) : 0u;
+        if (bit && (done.load(std::memory_order_acquire) & bit)) return cudaSuccess;
+        e = f();
+        if (e == cudaSuccess && bit) done.fetch_or(bit, std::memory_order_release);
+        return e;
+    }
 };
 
 cudaError_t launch_decode(const GdnDecodeArgs &a, cudaStream_t stream);

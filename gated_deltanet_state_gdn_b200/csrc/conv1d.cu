@@ -502,14 +502,13 @@ cudaError_t launch_staged_k(const GdnConv1dArgs &a, int L, int tiles, int64_t ch
                             cudaStream_t stream)
 {
     const size_t smem = (size_t)(L + K - 1) * kRowBytes;
-    static bool attr = false;  // opt in once to the largest stage any call uses
-    if (!attr) {
-        const cudaError_t e = cudaFuncSetAttribute(conv1d_staged_kernel<T, K>,
-                                                   cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                                   (kStagedMaxL + K - 1) * kRowBytes);
-        if (e != cudaSuccess) return e;
-        attr = true;
-    }
+    static DeviceOnce smem_opt_in;   // the largest stage any call uses
+    const cudaError_t e = smem_opt_in.run([] {
+        return cudaFuncSetAttribute(conv1d_staged_kernel<T, K>,
+                                    cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                    (kStagedMaxL + K - 1) * kRowBytes);
+    });
+    if (e != cudaSuccess) return e;
     conv1d_staged_kernel<T, K><<<(unsigned)(chunks * tiles), kThreads, smem, stream>>>(a, L, tiles);
     return cudaGetLastError();
 }

@@ -1346,17 +1346,18 @@ __global__ void __launch_bounds__(NTHREADS, 1) gdn_prefill_chunk_kernel(const __
 // ============================================================================ host side
 namespace {
 
+// the driver's tensor-map encoder, looked up once (thread-safe static initialisation)
 PFN_cuTensorMapEncodeTiled_v12000 get_encode()
 {
-    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
-    if (!fn) {
+    static const PFN_cuTensorMapEncodeTiled_v12000 fn = [] {
         cudaDriverEntryPointQueryResult q;
         void *ptr = nullptr;
         if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) ==
                 cudaSuccess &&
             q == cudaDriverEntryPointSuccess)
-            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
-    }
+            return reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
+        return static_cast<PFN_cuTensorMapEncodeTiled_v12000>(nullptr);
+    }();
     return fn;
 }
 
@@ -1409,8 +1410,8 @@ cudaError_t launch_prefill_chunked(const GdnPrefillArgs &a, cudaStream_t stream)
 {
     using namespace gdn_chunk;
     if (a.B == 0) return cudaSuccess;
-    static bool attr_set = false;
-    if (!attr_set) {
+    static DeviceOnce smem_opt_in;
+    cudaError_t attr_err = smem_opt_in.run([] {
         cudaError_t e = cudaFuncSetAttribute(gdn_prefill_chunk_kernel<false, false>,
                                              cudaFuncAttributeMaxDynamicSharedMemorySize,
                                              (int)SMEM_BYTES);
@@ -1420,9 +1421,9 @@ cudaError_t launch_prefill_chunked(const GdnPrefillArgs &a, cudaStream_t stream)
         if (e == cudaSuccess)
             e = cudaFuncSetAttribute(gdn_prefill_chunk_kernel<true, true>,
                                      cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SMEM_BYTES);
-        if (e != cudaSuccess) return e;
-        attr_set = true;
-    }
+        return e;
+    });
+    if (attr_err != cudaSuccess) return attr_err;
     Params p;
     memset(&p, 0, sizeof(p));
     const uint64_t N = (uint64_t)(a.N > 0 ? a.N : 1);
