@@ -17,6 +17,8 @@ import torch
 
 _PKG = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_PKG, "libgdn.so")
+# test build compiled with GDN_CHECKS (bounds-checked accesses, GDN_DEV_BOUNDS)
+CHECKED_LIB_PATH = os.path.join(_PKG, "libgdn_checked.so")
 
 GDN_OK = 0
 GDN_ERR_NULL = 1
@@ -52,6 +54,8 @@ UPDATE_RULES = {
 GDN_DEV_BAD_SLOT = 1
 GDN_DEV_TIMEOUT = 2
 GDN_DEV_INTERNAL = 4
+GDN_DEV_BOUNDS = 8            # checked builds only
+GDN_DEV_TEST_STALL = 1 << 30  # checked builds only, set by the caller (decode timeout path)
 
 EXPORTED = ("gdn_prefill", "gdn_decode", "gdn_conv1d", "gdn_status_string", "gdn_last_error",
             "gdn_abi_version", "gdn_prefill_uses_chunked")
@@ -67,6 +71,16 @@ class GdnError(RuntimeError):
         if status == GDN_ERR_CUDA:
             detail = ": " + lib().gdn_last_error().decode()
         super().__init__(f"{where} failed with {name}{detail}")
+
+
+def use_library(path: str) -> str:
+    """Route the calls that follow through the library at `path` (for instance the checked test
+    build CHECKED_LIB_PATH); returns the path in use before."""
+    global _lib, LIB_PATH
+    prev = LIB_PATH
+    LIB_PATH = path
+    _lib = None
+    return prev
 
 
 def lib():

@@ -77,6 +77,47 @@ __device__ __forceinline__ float softplus20(float x)
 
 __device__ __forceinline__ float sigmoidf_(float x) { return 1.0f / (1.0f + expf(-x)); }
 
+// ---------------------------------------------------------------- checked builds
+// Compiled with GDN_CHECKS, every global access and every data-dependent shared-memory access
+// is first tested against its buffer; one outside it is skipped (a load yields zero) and
+// GDN_DEV_BOUNDS is OR-ed into the status word.  Without GDN_CHECKS the tests are constant
+// true and vanish.
+#ifdef GDN_CHECKS
+constexpr bool kChecked = true;
+#else
+constexpr bool kChecked = false;
+#endif
+
+// elements [i, i + len) inside [0, n)
+__device__ __forceinline__ bool in_range(int64_t i, int64_t len, int64_t n, int32_t *status)
+{
+    if constexpr (!kChecked) return true;
+    if (i >= 0 && len >= 0 && i + len <= n) return true;
+    if (status) atomicOr(status, GDN_DEV_BOUNDS);
+    return false;
+}
+
+// bytes [p, p + len) inside the block's dynamic shared memory
+__device__ __forceinline__ bool in_smem(const void *p, uint32_t len, int32_t *status)
+{
+    if constexpr (!kChecked) return true;
+    extern __shared__ unsigned char gdn_dynamic_smem[];
+    uint32_t dyn;
+    asm("mov.u32 %0, %%dynamic_smem_size;" : "=r"(dyn));
+    const int64_t off = (int64_t)__cvta_generic_to_shared(p) -
+                        (int64_t)__cvta_generic_to_shared(gdn_dynamic_smem);
+    if (off >= 0 && off + len <= dyn) return true;
+    if (status) atomicOr(status, GDN_DEV_BOUNDS);
+    return false;
+}
+
+// checked builds: the caller asked for the timeout path to be exercised (GDN_DEV_TEST_STALL)
+__device__ __forceinline__ bool test_stall_requested(const int32_t *status)
+{
+    if constexpr (!kChecked) return false;
+    return status && (*reinterpret_cast<const volatile int32_t *>(status) & GDN_DEV_TEST_STALL);
+}
+
 }  // namespace gdn
 
 // Launchers implemented by the kernel translation units.

@@ -35,6 +35,8 @@
 namespace gdn_conv {
 
 using namespace sm100;
+using gdn::in_range;
+using gdn::in_smem;
 
 constexpr int kThreads = 128;
 constexpr int kVecBytes = 16;  // bytes of a row per thread on the vector path
@@ -169,6 +171,27 @@ __device__ __forceinline__ bool wait_copies(uint32_t bar, int32_t *dev_status)
     return true;
 }
 
+// Checked builds: the rows a block touches (its chunk [t0, t1), the K-1 look-back rows of a later
+// chunk, the last K-1 rows of the request for a first chunk that does not reach its end), its
+// channels [c, c + nc) and its window slot r all lie inside their buffers.  Every access of the
+// block is inside these ranges.  Always true in other builds.
+template <int W>
+__device__ __forceinline__ bool rows_in_range(const GdnConv1dArgs &a, int ci, int t0, int t1, int e,
+                                              int c, int nc, uint32_t r)
+{
+    if constexpr (!gdn::kChecked) return true;
+    int lo = ci > 0 ? t0 - W : t0;
+    int hi = t1;
+    if (W > 0 && ci == 0 && t1 < e) {
+        lo = min(lo, e - W);
+        hi = e;
+    }
+    const int64_t cd = a.conv_dim;
+    return in_range(lo, hi - lo, a.N, a.dev_status) && in_range(c, nc, cd, a.dev_status) &&
+           (W == 0 || in_range(((int64_t)r * cd + c) * W, (int64_t)nc * W, (int64_t)a.max_slots * cd * W,
+                               a.dev_status));
+}
+
 // Element path (rows not 16-byte aligned): every access goes through registers.
 template <typename T, int K, bool VEC, int kBatch>
 __global__ void __launch_bounds__(kThreads) conv1d_kernel(const GdnConv1dArgs a, const int L, const int tiles)
@@ -184,7 +207,8 @@ __global__ void __launch_bounds__(kThreads) conv1d_kernel(const GdnConv1dArgs a,
     const int tile = (int)(blockIdx.x % (unsigned)tiles);
     const int chunk = (int)(blockIdx.x / (unsigned)tiles);
     const int c0 = (tile * kThreads + threadIdx.x) * V;
-    const bool has_ch = c0 < a.conv_dim;
+    const bool has_ch = c0 < a.conv_dim &&
+                        in_range((int64_t)c0 * K, V * K, (int64_t)a.conv_dim * K, a.dev_status);
     Flat<T, V * K, VEC> fw;
     if (has_ch) fw.load(static_cast<const T *>(a.weight) + (int64_t)c0 * K);
 
@@ -209,6 +233,7 @@ __global__ void __launch_bounds__(kThreads) conv1d_kernel(const GdnConv1dArgs a,
     const int64_t ld = a.conv_dim;
     const int t0 = s + ci * L;
     const int t1 = min(e, t0 + L);
+    if (!rows_in_range<W>(a, ci, t0, t1, e, c0, V, r)) return;
 
     float wf[K][V];
     {
@@ -341,7 +366,8 @@ __global__ void __launch_bounds__(kThreads) conv1d_staged_kernel(const GdnConv1d
     const int chunk = (int)(blockIdx.x / (unsigned)tiles);
     const int tc0 = tile * kThreads * V;  // first channel of the tile
     const int c0 = tc0 + threadIdx.x * V;
-    const bool has_ch = c0 < a.conv_dim;
+    const bool has_ch = c0 < a.conv_dim &&
+                        in_range((int64_t)c0 * K, V * K, (int64_t)a.conv_dim * K, a.dev_status);
     const uint32_t bar = smem_u32(&s_bar);
     if (threadIdx.x == 0) {
         mbar_init(bar, 1);
@@ -369,6 +395,11 @@ __global__ void __launch_bounds__(kThreads) conv1d_staged_kernel(const GdnConv1d
             atomicOr(a.dev_status, GDN_DEV_BAD_SLOT);
         return;
     }
+    // (checked builds) the tile's rows, channels, window slot and stage, tested block-wide
+    // before any copy is issued
+    if (!rows_in_range<W>(a, ci, t0, t1, e, tc0, (int)(row_bytes / sizeof(T)), r) ||
+        !in_smem(stage, (uint32_t)(t1 - r0) * kRowBytes, a.dev_status))
+        return;
     if (threadIdx.x == 0) {
         const int nrows = t1 - r0;
         mbar_arrive_expect_tx(bar, (uint32_t)nrows * row_bytes);

@@ -71,28 +71,59 @@ __device__ __forceinline__ Stage stage_at(unsigned char *base, int T, int nh)
 }
 
 // Input piece i of unit (b, h): an 8-byte global source and its shared-memory destination.
-// Pieces run over the k rows, then the q rows, then the v rows of every token.
+// Pieces run over the k rows, then the q rows, then the v rows of every token.  Returns false
+// (checked builds only) when either side lies outside its buffer.
 template <int DV>
-__device__ __forceinline__ void input_piece(const GdnDecodeArgs &p, const Stage &st, int b, int h,
+__device__ __forceinline__ bool input_piece(const GdnDecodeArgs &p, const Stage &st, int b, int h,
                                             int i, const void *&src, void *&dst)
 {
     constexpr int RW = kDecodeDk / 4;   // 8-byte pieces of a k or q row
     constexpr int VW = DV / 4;
     const int T = p.T, nh = p.nh, H = p.H;
     const int nk = T * nh * RW, nq = T * RW;
+    int64_t e_src, n_src;
     if (i < nk) {
         const int row = i / RW, c = i - row * RW;   // row = t * nh + j
-        src = static_cast<const __nv_bfloat16 *>(p.k) + (((int64_t)b * T * nh + row) * H + h) * kDecodeDk + 4 * c;
+        e_src = (((int64_t)b * T * nh + row) * H + h) * kDecodeDk + 4 * c;
+        n_src = (int64_t)p.B * T * nh * H * kDecodeDk;
+        src = static_cast<const __nv_bfloat16 *>(p.k) + e_src;
         dst = st.k + 4 * i;
     } else if (i < nk + nq) {
         const int e = i - nk, t = e / RW, c = e - t * RW;
-        src = static_cast<const __nv_bfloat16 *>(p.q) + (((int64_t)b * T + t) * H + h) * kDecodeDk + 4 * c;
+        e_src = (((int64_t)b * T + t) * H + h) * kDecodeDk + 4 * c;
+        n_src = (int64_t)p.B * T * H * kDecodeDk;
+        src = static_cast<const __nv_bfloat16 *>(p.q) + e_src;
         dst = st.q + 4 * e;
     } else {
         const int e = i - nk - nq, row = e / VW, c = e - row * VW;
-        src = static_cast<const __nv_bfloat16 *>(p.v) + (((int64_t)b * T * nh + row) * p.HV + h) * DV + 4 * c;
+        e_src = (((int64_t)b * T * nh + row) * p.HV + h) * DV + 4 * c;
+        n_src = (int64_t)p.B * T * nh * p.HV * DV;
+        src = static_cast<const __nv_bfloat16 *>(p.v) + e_src;
         dst = st.v + 4 * e;
     }
+    return in_range(e_src, 4, n_src, p.dev_status) && in_smem(dst, 8, p.dev_status);
+}
+
+// elements of the pool the strides can reach
+template <int DV>
+__device__ __forceinline__ int64_t pool_elems(const GdnDecodeArgs &p)
+{
+    return (int64_t)(p.pool_size - 1) * p.slot_stride + (int64_t)(p.HV - 1) * p.head_stride +
+           (int64_t)DV * kDecodeDk;
+}
+
+// a lane's R x 4 float4 of state rows at pool element `base` (row stride 128), evict-first
+template <int DV, int R>
+__device__ __forceinline__ void store_state(const GdnDecodeArgs &p, int64_t base, const float4 (&s)[R][4])
+{
+    const int64_t n = pool_elems<DV>(p);
+#pragma unroll
+    for (int i = 0; i < R; ++i)
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            const int64_t e = base + i * kDecodeDk + 32 * j;
+            if (in_range(e, 4, n, p.dev_status)) st_stream(p.pool + e, s[i][j]);
+        }
 }
 
 template <int DV>
@@ -107,8 +138,12 @@ __device__ __forceinline__ unsigned short gate_raw(const GdnDecodeArgs &p, int b
     const int T = p.T;
     const unsigned short *ag = static_cast<const unsigned short *>(p.a);
     const unsigned short *bg = static_cast<const unsigned short *>(p.b);
-    return i < T ? __ldg(ag + ((int64_t)b * T + i) * p.HV + h)
-                 : __ldg(bg + ((int64_t)b * T * p.nh + (i - T)) * p.HV + h);
+    if (i < T) {
+        const int64_t e = ((int64_t)b * T + i) * p.HV + h;
+        return in_range(e, 1, (int64_t)p.B * T * p.HV, p.dev_status) ? __ldg(ag + e) : (unsigned short)0;
+    }
+    const int64_t e = ((int64_t)b * T * p.nh + (i - T)) * p.HV + h;
+    return in_range(e, 1, (int64_t)p.B * T * p.nh * p.HV, p.dev_status) ? __ldg(bg + e) : (unsigned short)0;
 }
 
 // alpha = exp(-exp(A_log) softplus20(a + dt_bias)), beta = sigmoid(b)
@@ -222,7 +257,7 @@ __device__ __forceinline__ void update_unit(float4 (&s)[R][4], const GdnDecodeAr
             }
 #pragma unroll
             for (int i = 0; i < R; ++i) o[i] = group_sum<8>(o[i]) * qs;
-            if (sub == 0) {
+            if (sub == 0 && in_range((bt * HV + h) * DV + row0, R, (int64_t)p.B * T * HV * DV, p.dev_status)) {
                 __nv_bfloat16 *op = og + (bt * HV + h) * DV + row0;
                 if constexpr (R == 4) {
                     uint2 wv;
@@ -244,11 +279,7 @@ __device__ __forceinline__ void update_unit(float4 (&s)[R][4], const GdnDecodeAr
             if (sidx >= p.pool_size) {
                 if (p.dev_status && threadIdx.x == 0) atomicOr(p.dev_status, GDN_DEV_BAD_SLOT);
             } else if (sidx >= 0) {
-                float *dst = p.pool + (int64_t)sidx * p.slot_stride + head_off;
-#pragma unroll
-                for (int i = 0; i < R; ++i)
-#pragma unroll
-                    for (int j = 0; j < 4; ++j) st_stream(dst + i * DK + 32 * j, s[i][j]);
+                store_state<DV, R>(p, (int64_t)sidx * p.slot_stride + head_off, s);
             }
         }
     }
@@ -258,11 +289,7 @@ __device__ __forceinline__ void update_unit(float4 (&s)[R][4], const GdnDecodeAr
         if (w >= p.pool_size) {
             if (p.dev_status && threadIdx.x == 0) atomicOr(p.dev_status, GDN_DEV_BAD_SLOT);
         } else if (w >= 0) {
-            float *dst = p.pool + w * p.slot_stride + head_off;
-#pragma unroll
-            for (int i = 0; i < R; ++i)
-#pragma unroll
-                for (int j = 0; j < 4; ++j) st_stream(dst + i * DK + 32 * j, s[i][j]);
+            store_state<DV, R>(p, w * p.slot_stride + head_off, s);
         }
     }
 }
@@ -280,7 +307,8 @@ __device__ __forceinline__ uint32_t side_raw(const GdnDecodeArgs &p, int b, int 
 {
     const int ng = p.T * (1 + p.nh);
     if (i < ng) return gate_raw(p, b, h, i);
-    return (uint32_t)__ldg(p.scatter_idx + (int64_t)b * p.T + (i - ng));
+    const int64_t e = (int64_t)b * p.T + (i - ng);
+    return in_range(e, 1, (int64_t)p.B * p.T, p.dev_status) ? (uint32_t)__ldg(p.scatter_idx + e) : 0xffffffffu;
 }
 
 __device__ __forceinline__ void side_store(const GdnDecodeArgs &p, const Stage &st, int h, int i,
@@ -322,11 +350,14 @@ decode_kernel(const GdnDecodeArgs p)
     // the state streams in (all loads in flight before any use)
     float4 s[R][4];
     {
-        const float *src = p.pool + r * p.slot_stride + head_off;
+        const int64_t n = pool_elems<DV>(p);
 #pragma unroll
         for (int i = 0; i < R; ++i)
 #pragma unroll
-            for (int j = 0; j < 4; ++j) s[i][j] = ld_stream(src + i * DK + 32 * j);
+            for (int j = 0; j < 4; ++j) {
+                const int64_t e = r * p.slot_stride + head_off + i * DK + 32 * j;
+                s[i][j] = in_range(e, 4, n, p.dev_status) ? ld_stream(p.pool + e) : make_float4(0.f, 0.f, 0.f, 0.f);
+            }
     }
     const int64_t w = write_slot(p, b, r);
 
@@ -338,8 +369,8 @@ decode_kernel(const GdnDecodeArgs p)
         for (int i = threadIdx.x; i < n; i += blockDim.x) {
             const void *src;
             void *dst;
-            input_piece<DV>(p, st, b, h, i, src, dst);
-            *static_cast<uint2 *>(dst) = __ldg(static_cast<const uint2 *>(src));
+            if (input_piece<DV>(p, st, b, h, i, src, dst))
+                *static_cast<uint2 *>(dst) = __ldg(static_cast<const uint2 *>(src));
         }
         const int ns = side_count(p);
         for (int i = threadIdx.x; i < ns; i += blockDim.x) side_store(p, st, h, i, side_raw(p, b, h, i));
@@ -397,24 +428,27 @@ decode_stream_kernel(const GdnDecodeArgs p)
 
     // copies of unit uu (read slot rr) into the state buffer and stage `buf`; every thread
     // arrives once, thread 0 also posts the state's byte count (0 for a skipped unit)
+    // (checked builds: a caller-requested stall makes the first wait run out)
+    bool stall = threadIdx.x == 0 && test_stall_requested(p.dev_status);
     auto issue = [&](int uu, int64_t rr, int buf) {
         const int bb = uu / HV, hh = uu - bb * HV;
         const bool live = rr >= 0 && rr < p.pool_size;
         if (threadIdx.x == 0) {
             if (rr >= p.pool_size && p.dev_status) atomicOr(p.dev_status, GDN_DEV_BAD_SLOT);
+            const int64_t e = rr * p.slot_stride + (int64_t)hh * p.head_stride;
+            const bool copy = live && in_range(e, DV * DK, pool_elems<DV>(p), p.dev_status) &&
+                              in_smem(sstate, kStateBytes, p.dev_status);
             fence_proxy_async_smem();
-            mbar_arrive_expect_tx(bar, live ? kStateBytes : 0u);
-            if (live)
-                bulk_load_1d(smem_u32(sstate), p.pool + rr * p.slot_stride + (int64_t)hh * p.head_stride,
-                             kStateBytes, bar);
+            mbar_arrive_expect_tx(bar, (copy ? kStateBytes : 0u) + (stall ? 16u : 0u));
+            stall = false;
+            if (copy) bulk_load_1d(smem_u32(sstate), p.pool + e, kStateBytes, bar);
         }
-        if (live) {
+        if (live && in_smem(stage0 + buf * sbytes, (uint32_t)sbytes, p.dev_status)) {
             const Stage st = stage_at<DV>(stage0 + buf * sbytes, T, nh);
             for (int i = threadIdx.x; i < npieces; i += NT) {
                 const void *src;
                 void *dst;
-                input_piece<DV>(p, st, bb, hh, i, src, dst);
-                cp_async8(smem_u32(dst), src);
+                if (input_piece<DV>(p, st, bb, hh, i, src, dst)) cp_async8(smem_u32(dst), src);
             }
         }
         cp_async_arrive(bar);

@@ -62,6 +62,9 @@ using namespace sm100;
 
 namespace gdn_chunk {
 
+using gdn::in_range;
+using gdn::kChecked;
+
 constexpr int C = 64;       // chunk length (tokens)
 constexpr int D = 128;      // Dk = Dv
 constexpr int NTHREADS = 480;
@@ -1145,7 +1148,12 @@ __global__ void __launch_bounds__(NTHREADS, 1) gdn_prefill_chunk_kernel(const __
                 const int nc = (un.len + C - 1) / C;
                 // this lane's state row (dv < Dv; lanes past Dv carry zero rows)
                 const int64_t st_off = (((int64_t)un.b * p.Hv + un.h) * Dv + dv) * Dk;
+#ifdef GDN_CHECKS
+                const int64_t st_n = (int64_t)p.B * p.Hv * Dv * Dk;
+                const bool row_ok = (!GENERAL || dv < Dv) && in_range(st_off, Dk, st_n, p.dev_status);
+#else
                 const bool row_ok = !GENERAL || dv < Dv;
+#endif
                 const float *init = p.initial_state && row_ok ? p.initial_state + st_off : nullptr;
                 float *fin = row_ok ? p.final_state + st_off : nullptr;
                 if (nc == 0) {
@@ -1176,10 +1184,18 @@ __global__ void __launch_bounds__(NTHREADS, 1) gdn_prefill_chunk_kernel(const __
                 // pulled into L2 now
                 const Unit nx = load_unit(smem, min(k + 1, nunits - 1));
                 const bool has_next = k + 1 < nunits && nx.len > 0;
+#ifdef GDN_CHECKS
+                const int64_t nx_off = (((int64_t)nx.b * p.Hv + nx.h) * Dv + dv) * Dk;
+                const float *next_init =
+                    has_next && p.initial_state && row_ok && in_range(nx_off, Dk, st_n, p.dev_status)
+                        ? p.initial_state + nx_off
+                        : nullptr;
+#else
                 const float *next_init =
                     has_next && p.initial_state && row_ok
                         ? p.initial_state + (((int64_t)nx.b * p.Hv + nx.h) * Dv + dv) * Dk
                         : nullptr;
+#endif
                 if (next_init) {
                     for (int c = 0; c < Dk; c += 32) prefetch_l2(next_init + c);
                 }
@@ -1253,7 +1269,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) gdn_prefill_chunk_kernel(const __
                             for (int e = 0; e < 32; ++e) x[e] *= gC1;
                             tmem_st32(tl + TM_S + 32 * q, x);
                         } else {
-                            if (!GENERAL) {
+                            if (!GENERAL && (!kChecked || row_ok)) {
 #pragma unroll
                                 for (int c = 0; c < 32; c += 4) st4(fin + 32 * q + c, x[c], x[c + 1], x[c + 2], x[c + 3]);
                             } else if (row_ok) {
@@ -1303,7 +1319,9 @@ __global__ void __launch_bounds__(NTHREADS, 1) gdn_prefill_chunk_kernel(const __
                                 const uint4 v = *reinterpret_cast<const uint4 *>(ost + lane * 16);
                                 __syncwarp();
                                 const int i0 = 16 * q + 8 * hb;   // first token of this group
-                                if (i0 + tt < len_n && (!GENERAL || ocol < Dv))
+                                if (i0 + tt < len_n && (!GENERAL || ocol < Dv) &&
+                                    in_range(((int64_t)(un.start + n * C + tt + i0) * p.Hv + un.h) * Dv + ocol,
+                                             8, (int64_t)p.N * p.Hv * Dv, p.dev_status))
                                     *reinterpret_cast<uint4 *>(obase + (i0 / 8) * ostride8) = v;
                             }
                         }

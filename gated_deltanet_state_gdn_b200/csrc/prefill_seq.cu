@@ -88,6 +88,14 @@ prefill_seq_kernel(const GdnPrefillArgs p)
 
     float S[R][EPL];
     const int64_t state_off = ((int64_t)b * Hv + h) * Dv * (int64_t)Dk;
+    // (checked builds) every access below lies in the tokens [start, end), query head qh and
+    // this head's state slice: test those ranges once
+    if constexpr (kChecked) {
+        if (!in_range(start, end > start ? end - start : 0, p.N, p.dev_status) ||
+            !in_range(qh, 1, Hq, p.dev_status) ||
+            !in_range(state_off, (int64_t)Dv * Dk, (int64_t)p.B * Hv * Dv * Dk, p.dev_status))
+            return;
+    }
 #pragma unroll
     for (int i = 0; i < R; ++i)
 #pragma unroll

@@ -77,7 +77,16 @@ enum {
 enum {
     GDN_DEV_BAD_SLOT = 1,  /* a slot index >= the pool size was skipped (decode, conv1d) */
     GDN_DEV_TIMEOUT = 2,   /* a kernel-internal wait exceeded its bound; outputs invalid */
-    GDN_DEV_INTERNAL = 4   /* a kernel's layout self-check failed; nothing was computed */
+    GDN_DEV_INTERNAL = 4,  /* a kernel's layout self-check failed; nothing was computed */
+    /* Checked builds only (libgdn_checked.so, compiled with GDN_CHECKS): every global and
+     * data-dependent shared-memory access is tested against its buffer first; one outside it
+     * is skipped (a load reads zero) and this bit is set.  Ordinary builds never set it. */
+    GDN_DEV_BOUNDS = 8,
+    /* Checked builds only, set by the CALLER in *dev_status before a gdn_decode call: the
+     * persistent decode kernel posts 16 bytes more than its first copy delivers, so that
+     * wait runs out after its bound (about a second), GDN_DEV_TIMEOUT is set and the kernel
+     * returns.  Exercises the timeout path without a fault; ignored by ordinary builds. */
+    GDN_DEV_TEST_STALL = 1 << 30
 };
 
 /*

@@ -178,3 +178,14 @@ def test_binding_fails_loudly_without_library(monkeypatch, tmp_path):
     monkeypatch.setattr(b, "LIB_PATH", str(tmp_path / "missing.so"))
     with pytest.raises(RuntimeError, match="no fallback"):
         b.lib()
+
+
+def test_checked_build_exports_the_same_entry_points():
+    """The bounds-checked test build (compiled with GDN_CHECKS) loads without a GPU and exports
+    the same C ABI as the product library."""
+    from gated_deltanet_state_gdn_b200 import build
+    C = ctypes.CDLL(build.build(checked=True))
+    for name in declared_symbols():
+        assert hasattr(C, name), name
+    C.gdn_abi_version.restype = ctypes.c_int32
+    assert C.gdn_abi_version() == 2
