@@ -365,7 +365,7 @@ __device__ __noinline__ void build_unit_list(const Params &p, uint8_t *smem, int
         // CTAs kept in order of (work so far, index), as packed 64-bit keys: a request's heads
         // go to the first Hv of the order; the order is then rebuilt by merging the untouched
         // tail with the updated head (both stay sorted), each thread placing one CTA with a
-        // binary search.
+        // binary search into the other of two buffers (one barrier per step).
         long long *key = reinterpret_cast<long long *>(ord + 128);   // two buffers of G keys
         for (int i = tid; i < G; i += NTHREADS) key[i] = i;
         if (tid == 0) *count_out = 0;
@@ -408,9 +408,10 @@ __device__ __noinline__ void build_unit_list(const Params &p, uint8_t *smem, int
                         }
                         npos = (tid - m) + lo;
                     }
+                    // nd is not od, and every read of nd's previous contents (as the old order
+                    // of the step before) finished before that step's closing barrier
+                    nd[npos] = kx;
                 }
-                __syncthreads();
-                if (tid < G) nd[npos] = kx;
                 __syncthreads();
                 cur ^= 1;
             }
