@@ -20,18 +20,25 @@
 // without the delta retrieval A = 0 (T = I) and W = 0, so U = diag(beta) V with
 // beta = 1 (the rule has no beta input).  The qwen gate and the sigmoid beta
 // are applied to the per-token gate values before the prefix sum.
-// The norms rk, rq are never applied to the bf16 tiles: they fold into A, P,
-// the columns of T (for W), the decayed copy of U (for S_C) and the output
-// scale, so the tensor cores always read the caller's q/k bytes.
+// The norms rk, rq are never applied to the bf16 q/k tiles, so the tensor cores
+// always read the caller's bytes.  With D = diag(rk), A = diag(beta rk) B D for
+// the raw key products B = (K K^T) * decay, and (I + A)^-1 = D^-1 (I + A')^-1 D
+// with A' = diag(beta rk^2) B: every row of A' needs only its own norm, rk_i^2 =
+// 1 / (k_i . k_i + eps), read from the Gram diagonal.  Carrying U' = D U instead
+// of U, the column norms land in the T' tiles and cancel elsewhere:
+//   T'  = (I + A')^-1,  Tb = T' diag(beta rk),  Tbg = T' diag(beta Gamma rk^2)
+//   U'  = Tb V - Tbg K S0                       (= D U)
+//   S_C = Gamma_C S0 + (diag(exp(G_C - G)) K)^T U'
+//   O   = scale (diag(Gamma rq) Q S0 + P' U'),  P'_ij = rq_i (q_i . k_j) exp(G_i - G_j)
 // All state-dependent products are evaluated transposed (rows = value index
 // dv), so every tcgen05 MMA here has M = 128:
 //   (G)  [K; Q] K^T                         -> TMEM  (Gram, 128 x 64)
-//   (W)  W^T  = K^T . Tbg^T                 -> TMEM  (Tbg = T diag(beta Gamma rk))
-//   (U~) U^T  = V^T . Tb^T                  -> TMEM  (Tb  = T diag(beta))
+//   (W)  W^T  = K^T . Tbg^T                 -> TMEM
+//   (U~) U^T  = V^T . Tb^T                  -> TMEM
 //   (1a) U^T += S^T . (-W)^T                 (bf16 copy of S^T from TMEM)
 //   (1b) Y    = S^T . Q^T
-//   (2)  S^T += (U^T diag(exp(G_C - G) rk)) . K   (fp32 accumulator stays in TMEM)
-//   (3)  Z    = U^T . P^T
+//   (2)  S^T += (U^T diag(exp(G_C - G))) . K  (fp32 accumulator stays in TMEM)
+//   (3)  Z    = U^T . P'^T
 //   O^T = scale (Y diag(Gamma rq) + Z)
 // TMEM (512 columns): S^T [0,128) | U^T [128,192) | Y [192,256) | Z [256,320) |
 // Gram [320,384) | W^T [384,448) | bf16 S^T [448,512) (A of 1a/1b, 8 columns per
@@ -41,8 +48,8 @@
 // CTA = 15 warps, one (request, value head) unit at a time, persistent over a
 // longest-first unit list:
 //   warps 0-3   state warpgroup: TMEM <-> bf16 operand tiles, outputs, state I/O
-//   warps 4-7   prep front: row norms, gates, Gram -> A and P
-//   warps 8-11  prep back: the 64x64 unit-triangular solve and the bf16 T tiles
+//   warps 4-7   prep front: gates, query norms, Gram -> A' (with the key norms) and P'
+//   warps 8-11  prep back: the 64x64 unit-triangular solve and the bf16 T' tiles
 //               (front and back work on consecutive chunks, ahead of the state chain)
 //   warp  12    TMA producers (lane 0: q/k/g/beta tiles in three stages; lane 1: v tiles)
 //   warp  13    TMEM owner; UMMA issuer of the state chain (1a, 1b, 2, 3)
@@ -112,12 +119,12 @@ constexpr int GA_CF = 64;      // exp(Gend_J(i) - G_i): factor to the end of i's
 constexpr int GA_BETA = 128;   // beta_i (0 beyond the request)
 constexpr int GA_GAM = 192;    // exp(G_i)
 constexpr int GA_DEC = 256;    // exp(G_C - G_i)
-constexpr int GA_RK = 320;     // key norm factor rk_i (1 without qk_l2norm)
-constexpr int GA_RQ = 384;     // query norm factor rq_i
+constexpr int GA_RQ = 384;     // query norm factor rq_i (1 without qk_l2norm)
 constexpr int GA_GEND = 448;   // G_end of each 16-block * log2(e)  [4]
 constexpr int GA_GC = 452;     // exp(G_C)
-constexpr int GA_BG = 456;     // beta_i Gamma_i rk_i (column scale of Tbg)
-static_assert((GA_BG + 64) * 4 <= (int)GATE_BYTES, "gate stage size");
+constexpr int GA_BG = 456;     // beta_i Gamma_i rk_i^2 (column scale of Tbg)
+constexpr int GA_TB = 520;     // beta_i rk_i (column scale of Tb)
+static_assert((GA_TB + 64) * 4 <= (int)GATE_BYTES, "gate stage size");
 
 // barrier indices
 enum {
@@ -475,8 +482,8 @@ __device__ __forceinline__ void blk_store(float *Z, const float (&acc)[2][4], fl
     }
 }
 
-// Block (I, J) of T from an mma fragment (times sgn), written to the bf16 operand
-// tiles Tb = T diag(beta) and Tbg = T diag(beta Gamma rk) (K-major, 128B-swizzled)
+// Block (I, J) of T' from an mma fragment (times sgn), written to the bf16 operand
+// tiles Tb = T' diag(beta rk) and Tbg = T' diag(beta Gamma rk^2) (K-major, 128B-swizzled)
 template <bool F16>
 __device__ __forceinline__ void blk_store_tiles(const float (&acc)[2][4], float sgn, int I, int J,
                                                 const float *ga, uint8_t *tb, uint8_t *tbg)
@@ -486,7 +493,7 @@ __device__ __forceinline__ void blk_store_tiles(const float (&acc)[2][4], float 
 #pragma unroll
     for (int nh = 0; nh < 2; ++nh) {
         const int j = 16 * J + 8 * nh + 2 * t;
-        const float2 b = *reinterpret_cast<const float2 *>(ga + GA_BETA + j);
+        const float2 b = *reinterpret_cast<const float2 *>(ga + GA_TB + j);
         const float2 bg = *reinterpret_cast<const float2 *>(ga + GA_BG + j);
 #pragma unroll
         for (int h = 0; h < 2; ++h) {
@@ -515,15 +522,18 @@ __device__ __forceinline__ int t_slot(int I, int J)
     return 8 + J;
 }
 
-// Row i of A (TMEM quadrants 0-1: beta_i (k^_i . k^_j) exp(G_i - G_j) for j < i, fp32
-// into the solve blocks) or of P (quadrants 2-3: (q^_i . k^_j) exp(G_i - G_j) for
-// j <= i, bf16 tile), read 16 Gram columns at a time from TMEM.  Blocks right of the
-// row's diagonal block are zero: never stored for A, zero from the start in P.  The
-// exponent of an earlier block J is split as exp(G_i - Gend_J) exp(Gend_J - G_j),
-// both <= 1.
+// Row i of A' (TMEM quadrants 0-1: beta_i rk_i^2 (k_i . k_j) exp(G_i - G_j) for j < i, fp32
+// into the solve blocks) or of P' (quadrants 2-3: rq_i (q_i . k_j) exp(G_i - G_j) for
+// j <= i, bf16 tile), read 16 Gram columns at a time from TMEM.  Only the row's own norm
+// enters: the key norms of the columns move into the T' tiles (see the kernel notes), and
+// a key row takes its own norm from the Gram diagonal k_i . k_i, element r of its diagonal
+// block.  Blocks right of the
+// row's diagonal block are zero: never stored for A', zero from the start in P'.  The
+// exponent of an earlier block J is split as exp(G_i - Gend_J) exp(Gend_J - G_j), both
+// <= 1.  Returns rk_i for key rows (1 without the norm or for query rows).
 template <bool F16>
-__device__ __forceinline__ void build_row(uint32_t tl_gram, int qd, const float *ga, float *solve,
-                                          uint8_t *ptile, bool retrieval)
+__device__ __forceinline__ float build_row(uint32_t tl_gram, int qd, const float *ga, float *solve,
+                                           uint8_t *ptile, bool retrieval, bool knorm)
 {
     const int lane = threadIdx.x & 31;
     const bool isP = qd >= 2;
@@ -532,38 +542,45 @@ __device__ __forceinline__ void build_row(uint32_t tl_gram, int qd, const float 
     const int i = 16 * I + r;
     const int jmax = 2 * (qd & 1) + 1;   // last diagonal block among the warp's rows
     const float G2i = ga[GA_G2 + i];
-    // without the delta retrieval A = 0, so T = I
-    const float rowscale = isP ? ga[GA_RQ + i] : (retrieval ? ga[GA_BETA + i] * ga[GA_RK + i] : 0.f);
+    // without the delta retrieval A' = 0, so T' = I; key rows take rk_i^2 at their diagonal
+    // block, which the descending block order reaches first
+    float rk = 1.f;
+    float rowscale = isP ? ga[GA_RQ + i] : (retrieval ? ga[GA_BETA + i] : 0.f);
     float gend[3];
 #pragma unroll
     for (int J = 0; J < 3; ++J) gend[J] = ga[GA_GEND + J];
 #pragma unroll 1
-    for (int J = 0; J <= jmax; ++J) {
+    for (int J = jmax; J >= 0; --J) {
         // ---- loads (TMEM Gram columns, gate factors) before any store of this block
-        float x[16], cf[16], g2[16], rk[16];
+        float x[16], cf[16], g2[16];
         tmem_ld16(tl_gram + 16 * J, x);
 #pragma unroll
         for (int q = 0; q < 4; ++q) {
             const float4 a = ld4(ga + GA_CF + 16 * J + 4 * q);
             const float4 b = ld4(ga + GA_G2 + 16 * J + 4 * q);
-            const float4 c = ld4(ga + GA_RK + 16 * J + 4 * q);
             cf[4 * q] = a.x; cf[4 * q + 1] = a.y; cf[4 * q + 2] = a.z; cf[4 * q + 3] = a.w;
             g2[4 * q] = b.x; g2[4 * q + 1] = b.y; g2[4 * q + 2] = b.z; g2[4 * q + 3] = b.w;
-            rk[4 * q] = c.x; rk[4 * q + 1] = c.y; rk[4 * q + 2] = c.z; rk[4 * q + 3] = c.w;
         }
         tmem_wait_ld();
         if (J > I) continue;
+        if (J == I && knorm && !isP) {
+            float kk = 0.f;
+#pragma unroll
+            for (int e = 0; e < 16; ++e) kk = e == r ? x[e] : kk;
+            rk = 1.0f / sqrtf(kk + 1e-12f);
+            rowscale *= rk * rk;
+        }
         // ---- compute
         if (J < I) {
             const float f = ex2_approx(G2i - (J == 0 ? gend[0] : (J == 1 ? gend[1] : gend[2]))) * rowscale;
 #pragma unroll
-            for (int jj = 0; jj < 16; ++jj) x[jj] *= f * cf[jj] * rk[jj];
+            for (int jj = 0; jj < 16; ++jj) x[jj] *= f * cf[jj];
         } else {
             // branch-free: every lane evaluates all 16 factors, then masks
             const int lim = isP ? r + 1 : r;
 #pragma unroll
             for (int jj = 0; jj < 16; ++jj) {
-                const float e = ex2_approx(fminf(G2i - g2[jj], 0.f)) * rk[jj] * rowscale;
+                const float e = ex2_approx(fminf(G2i - g2[jj], 0.f)) * rowscale;
                 x[jj] = (jj < lim) ? x[jj] * e : 0.f;
             }
         }
@@ -577,6 +594,7 @@ __device__ __forceinline__ void build_row(uint32_t tl_gram, int qd, const float 
             for (int q = 0; q < 4; ++q) st4(row + 4 * q, x[4 * q], x[4 * q + 1], x[4 * q + 2], x[4 * q + 3]);
         }
     }
+    return rk;
 }
 
 // ========================================================================== kernel
@@ -895,13 +913,12 @@ __global__ void __launch_bounds__(NTHREADS, 1) gdn_prefill_chunk_kernel(const __
         } else if (warp >= 4) {
             // ------------------------------------------------------------ prep warpgroups
             // Two groups of four warps form a two-stage pipeline over consecutive chunks:
-            //   front (warps 4-7):  row norms, gates, A and P from the Gram (TMEM)
-            //   back  (warps 8-11): 16x16 diagonal inverses, block merges, bf16 T tiles
+            //   front (warps 4-7):  gates, query norms, A' and P' from the Gram (TMEM)
+            //   back  (warps 8-11): 16x16 diagonal inverses, block merges, bf16 T' tiles
             // A crosses in one of two solve areas (A_READY / SOLVE_FREE per area).
             const int pg = (warp - 4) >> 2;          // 0 front, 1 back
             const int lt = tid - 128 - 128 * pg;     // thread in the group, 0..127
             const int pw = lt >> 5;                  // warp in the group == TMEM lane quadrant
-            const int tp = 32 * pw + lane;           // TMEM lane == row handled by this thread
             const uint32_t tl = tmem + ((uint32_t)(32 * pw) << 16);
             const int nbar = pg ? 3 : 1;             // the group's named barrier
             bool ok = true;
@@ -923,24 +940,8 @@ __global__ void __launch_bounds__(NTHREADS, 1) gdn_prefill_chunk_kernel(const __
                         ++p_gate_empty[ks];
                         if (p_sf[s] > 0) ok = ok && cx.wait(B_SOLVE_FREE + s, (p_sf[s] - 1) & 1);
                         ++p_sf[s];
-                        // --- row norms (K rows 0..63, Q rows 64..127), conflict-free chunk order
-                        {
-                            float rn = 1.f;
-                            if (p.qk_l2norm) {
-                                float ss = 0.f;
-#pragma unroll
-                                for (int c = 0; c < 8; ++c) {
-                                    const uint32_t off = sw128(tp, c);
-                                    const uint4 va = *reinterpret_cast<const uint4 *>(kq + off);
-                                    const uint4 vb = *reinterpret_cast<const uint4 *>(kq + KQ_KB + off);
-                                    ss += sumsq8_bf16<F16>(va) + sumsq8_bf16<F16>(vb);
-                                }
-                                rn = 1.0f / sqrtf(ss + 1e-12f);
-                            }
-                            ga[GA_RK + tp] = rn;   // GA_RQ = GA_RK + 64
-                        }
-                        // --- gates (front warp 0, tokens 2l and 2l+1 per lane): floored, masked
-                        //     log-decay, inclusive prefix sum, exponentials
+                        // --- gates first (front warp 0, tokens 2l and 2l+1 per lane): floored,
+                        //     masked log-decay, inclusive prefix sum, exponentials
                         if (pw == 0) {
                             const int i0 = 2 * lane, i1 = i0 + 1;
                             const int hc = un.h & 3;
@@ -991,20 +992,49 @@ __global__ void __launch_bounds__(NTHREADS, 1) gdn_prefill_chunk_kernel(const __
                                 make_float2(ex2_approx(gcl - G2a), ex2_approx(gcl - G2b));
                             if ((lane & 7) == 7) ga[GA_GEND + (lane >> 3)] = G2b;
                             if (lane == 31) ga[GA_GC] = ex2_approx(G2b);
+                            // published at once: the state chain waits for exp(G_C) of the next
+                            // chunk, and nothing here depends on the norms
+                            __syncwarp();
+                            if (lane == 0) mbar_arrive(cx.bar(B_GATE_FULL + ks));
+                        }
+                        // --- query row norms (Q rows 64..127 of the stage): two threads per row,
+                        //     chunks c and 4 + c of each k-block (distinct swizzled 16-byte
+                        //     positions within every four rows: conflict-free).  Key row norms
+                        //     come from the Gram diagonal inside build_row; without qk_l2norm
+                        //     every factor is 1.
+                        if (p.qk_l2norm) {
+                            const int qrow = 64 + (lt >> 1);
+                            const int hf = lt & 1;
+                            float ss = 0.f;
+#pragma unroll
+                            for (int c = 0; c < 4; ++c) {
+                                const uint32_t off = sw128(qrow, 4 * hf + c);
+                                const uint4 va = *reinterpret_cast<const uint4 *>(kq + off);
+                                const uint4 vb = *reinterpret_cast<const uint4 *>(kq + KQ_KB + off);
+                                ss += sumsq8_bf16<F16>(va) + sumsq8_bf16<F16>(vb);
+                            }
+                            ss += __shfl_xor_sync(0xffffffffu, ss, 1);
+                            if (hf == 0) ga[GA_RQ + (qrow - 64)] = 1.0f / sqrtf(ss + 1e-12f);
+                        } else if (lt < 64) {
+                            ga[GA_RQ + lt] = 1.f;
                         }
                         named_sync(1, 128);
-                        if (lt == 0) mbar_arrive(cx.bar(B_GATE_FULL + ks));
                         // --- Gram -> A (rows 0..63, fp32 blocks) and P (rows 64..127, bf16 tile); P
                         //     shares the KQ stage, so the (3) product that last read it completed
                         //     before this stage was reloaded (KQ_EMPTY is committed after it)
                         ok = ok && cx.wait(B_G_DONE, p_g & 1);
                         ++p_g;
                         tc_fence_after();
-                        build_row<F16>(tl + TM_G, pw, ga, solve, smem + OFF_P + ks * P_STAGE, has_retrieval);
+                        const float rk = build_row<F16>(tl + TM_G, pw, ga, solve, smem + OFF_P + ks * P_STAGE,
+                                                        has_retrieval, p.qk_l2norm != 0);
                         if (pw >= 2) fence_proxy_async_smem();
-                        // W = T diag(beta Gamma rk) K carries the retrieval term: zero without it
-                        if (lt < 64)
-                            ga[GA_BG + lt] = has_retrieval ? ga[GA_BETA + lt] * ga[GA_GAM + lt] * ga[GA_RK + lt] : 0.f;
+                        // column scales of the T' tiles (thread lt < 64 built key row lt): W = Tbg K
+                        // carries the retrieval term (zero without it), U~ = Tb V
+                        if (lt < 64) {
+                            const float b = ga[GA_BETA + lt];
+                            ga[GA_BG + lt] = has_retrieval ? b * ga[GA_GAM + lt] * rk * rk : 0.f;
+                            ga[GA_TB + lt] = b * rk;
+                        }
                         tc_fence_before();
                         named_sync(1, 128);
                         if (lt == 0) {
@@ -1044,7 +1074,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) gdn_prefill_chunk_kernel(const __
 #pragma unroll
                             for (int r = 0; r < 16; ++r) Db[r * SOLVE_LD + c] = x[r];
                             const int j = 16 * I + c;
-                            const float bj = ga[GA_BETA + j], sj = ga[GA_BG + j];
+                            const float bj = ga[GA_TB + j], sj = ga[GA_BG + j];
                             const uint32_t cw = (uint32_t)(j & 7) * 2u;
 #pragma unroll
                             for (int r = 0; r < 16; ++r) {
@@ -1224,8 +1254,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) gdn_prefill_chunk_kernel(const __
 #pragma unroll
                             for (int e = 0; e < 16; e += 4) {
                                 const float4 d4 = ld4(ga + GA_DEC + t0 + e);
-                                const float4 k4 = ld4(ga + GA_RK + t0 + e);
-                                d[e] = d4.x * k4.x; d[e + 1] = d4.y * k4.y; d[e + 2] = d4.z * k4.z; d[e + 3] = d4.w * k4.w;
+                                d[e] = d4.x; d[e + 1] = d4.y; d[e + 2] = d4.z; d[e + 3] = d4.w;
                             }
                             uint32_t w[16];
 #pragma unroll
