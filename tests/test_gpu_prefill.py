@@ -230,6 +230,36 @@ def test_chunked_equals_sequential(gdn, W, lengths):
     assert rel_l2(f64(fc), f64(fs_)) <= TOL_BF16
 
 
+def test_norm_extremes_on_tensor_cores(gdn, W, oracle_mod):
+    """In-kernel q/k normalisation with all-zero, tiny (x 1e-3) and large (x 100) rows.  A key
+    row's norm comes from the Gram diagonal and its column scale rides in the T' tiles, so a zero
+    key row puts a factor of about 1e6 on a column that only ever meets exact zeros; a zero query
+    row reads out zero."""
+    c = W.make_prefill(97, [150, 64, 33], 2, 4, 128, 128, init_std=0.02, qk_l2norm=True)
+    assert gdn.prefill_uses_chunked(c.q.dtype, 4, 128, 128)
+    k = c.k.float()
+    q = c.q.float()
+    idx = torch.from_numpy(np.random.default_rng(5).permutation(k.shape[0]))
+    k[idx[:12]] = 0.0
+    k[idx[12:24]] *= 1e-3
+    k[idx[24:36]] *= 100.0
+    q[idx[36:48]] = 0.0
+    q[idx[48:60]] *= 1e-3
+    c.k = k.to(c.k.dtype)
+    c.q = q.to(c.q.dtype)
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    out, fs = gdn.gdn_prefill(dev(c.q), dev(c.k), dev(c.v), dev(c.g), dev(c.beta),
+                              dev(c.cu_seqlens), dev(c.initial_state), scale=c.scale,
+                              qk_l2norm=True, dev_status=status)
+    torch.cuda.synchronize()
+    assert int(status.item()) == 0
+    assert torch.isfinite(out.float()).all() and torch.isfinite(fs).all()
+    ro, rf = oracle_prefill_case(oracle_mod, c)
+    assert rel_l2(f64(out), ro) <= TOL_BF16
+    assert rel_l2(f64(fs), rf) <= TOL_BF16
+    assert (out[idx[36:48].cuda()] == 0).all()
+
+
 # ---------------------------------------------------------------- full sizes
 def _sampled_heads_parity(oracle_mod, c, out, fs, heads):
     o = f64(out)
