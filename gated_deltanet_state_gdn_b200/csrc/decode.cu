@@ -203,9 +203,12 @@ __device__ __forceinline__ void update_unit(float4 (&s)[R][4], const GdnDecodeAr
             const float beta = st.beta[tj];
             float vr[R];
             const __nv_bfloat16 *vp = st.v + tj * DV + row0;
-            if constexpr (R == 4) {
-                float4 v4 = lds_bf16x4(vp);
-                vr[0] = v4.x; vr[1] = v4.y; vr[2] = v4.z; vr[3] = v4.w;
+            if constexpr (R == 4 || R == 8) {
+#pragma unroll
+                for (int h = 0; h < R / 4; ++h) {
+                    const float4 v4 = lds_bf16x4(vp + 4 * h);
+                    vr[4 * h] = v4.x; vr[4 * h + 1] = v4.y; vr[4 * h + 2] = v4.z; vr[4 * h + 3] = v4.w;
+                }
             } else {
 #pragma unroll
                 for (int i = 0; i < R; ++i) vr[i] = bf16_to_f32(vp[i]);
@@ -259,7 +262,14 @@ __device__ __forceinline__ void update_unit(float4 (&s)[R][4], const GdnDecodeAr
             for (int i = 0; i < R; ++i) o[i] = group_sum<8>(o[i]) * qs;
             if (sub == 0 && in_range((bt * HV + h) * DV + row0, R, (int64_t)p.B * T * HV * DV, p.dev_status)) {
                 __nv_bfloat16 *op = og + (bt * HV + h) * DV + row0;
-                if constexpr (R == 4) {
+                if constexpr (R == 8) {
+                    uint4 wv;
+                    wv.x = pack_bf16x2(o[0], o[1]);
+                    wv.y = pack_bf16x2(o[2], o[3]);
+                    wv.z = pack_bf16x2(o[4], o[5]);
+                    wv.w = pack_bf16x2(o[6], o[7]);
+                    *reinterpret_cast<uint4 *>(op) = wv;
+                } else if constexpr (R == 4) {
                     uint2 wv;
                     wv.x = pack_bf16x2(o[0], o[1]);
                     wv.y = pack_bf16x2(o[2], o[3]);
@@ -326,7 +336,7 @@ __device__ __forceinline__ int side_count(const GdnDecodeArgs &p)
 
 // ---------------------------------------------------------------- one CTA per (row, head)
 template <int DV, int R>
-__global__ void __launch_bounds__(DV / (4 * R) * 32)
+__global__ void __launch_bounds__(DV / (4 * R) * 32, R == 8 ? 3 : 1)
 decode_kernel(const GdnDecodeArgs p)
 {
     constexpr int DK = kDecodeDk;
@@ -515,6 +525,7 @@ decode_stream_kernel(const GdnDecodeArgs p)
 namespace {
 
 constexpr int kMaxDevices = 16;
+constexpr long long kPerUnitWaves = 4;   // waves of resident one-CTA-per-unit CTAs
 
 int sm_count()
 {
@@ -589,16 +600,18 @@ int per_unit_occupancy()
     return nb;
 }
 
-template <int DV, int R, int MINB>
+template <int DV, int R, int MINB, int RU>
 cudaError_t launch_form(const GdnDecodeArgs &a, cudaStream_t stream)
 {
     // One CTA per unit keeps every state load of its resident CTAs in flight at once and wins
-    // once the units fill many waves of them; with fewer waves, or several tokens per unit
+    // once the units fill several waves of them; with fewer waves, or several tokens per unit
     // (scatter stores, longer arithmetic), the persistent form's overlap of the next unit's
-    // loads with this unit's arithmetic and stores wins (8 waves from a sweep of shapes).
+    // loads with this unit's arithmetic and stores wins.  RU rows per lane for the one-CTA
+    // form (8 at Dv = 128: 128 threads, three CTAs and 192 KB of state loads per SM).
     const long long units = (long long)a.B * a.HV;
-    const long long resident = (long long)sm_count() * per_unit_occupancy<DV, R>();
-    if (a.T == 1 && resident > 0 && units >= 8 * resident) return launch_per_unit<DV, R>(a, stream);
+    const long long resident = (long long)sm_count() * per_unit_occupancy<DV, RU>();
+    if (a.T == 1 && resident > 0 && units >= kPerUnitWaves * resident)
+        return launch_per_unit<DV, RU>(a, stream);
     return launch_stream<DV, R, MINB>(a, stream);
 }
 
@@ -608,6 +621,6 @@ cudaError_t launch_decode(const GdnDecodeArgs &a, cudaStream_t stream)
 {
     if ((long long)a.B * a.HV == 0) return cudaSuccess;
     constexpr int R = 4;
-    if (a.Dv == 128) return launch_form<128, R, 2>(a, stream);
-    return launch_form<64, R, 4>(a, stream);
+    if (a.Dv == 128) return launch_form<128, R, 2, 8>(a, stream);
+    return launch_form<64, R, 4, 4>(a, stream);
 }
