@@ -18,8 +18,9 @@
 //
 // Two launch forms share that per-unit code:
 //   decode_kernel         one CTA per unit; the state is loaded straight into
-//                         registers.  Used for single-token units that fill
-//                         many waves of resident CTAs.
+//                         registers (8 rows per lane at Dv = 128: 128 threads,
+//                         three CTAs per SM).  Used for single-token units that
+//                         fill several waves of resident CTAs.
 //   decode_stream_kernel  persistent: one CTA per resident slot walks the units
 //                         blockIdx.x + i * gridDim.x.  While it updates and
 //                         stores unit i, one bulk copy brings unit i+1's state
