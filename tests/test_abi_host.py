@@ -189,3 +189,17 @@ def test_checked_build_exports_the_same_entry_points():
         assert hasattr(C, name), name
     C.gdn_abi_version.restype = ctypes.c_int32
     assert C.gdn_abi_version() == 2
+
+
+def test_use_library_switches_and_fails_loudly(tmp_path):
+    """use_library routes later calls through another build and returns the previous path; a
+    missing library still raises instead of falling back."""
+    import gated_deltanet_state_gdn_b200 as g
+    import gated_deltanet_state_gdn_b200._binding as b
+    prev = g.use_library(str(tmp_path / "missing.so"))
+    try:
+        with pytest.raises(RuntimeError, match="no fallback"):
+            b.lib()
+    finally:
+        assert g.use_library(prev) == str(tmp_path / "missing.so")
+    assert b.LIB_PATH == prev
