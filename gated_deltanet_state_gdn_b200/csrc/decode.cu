@@ -264,12 +264,14 @@ __device__ __forceinline__ void update_unit(float4 (&s)[R][4], const GdnDecodeAr
             if (sub == 0 && in_range((bt * HV + h) * DV + row0, R, (int64_t)p.B * T * HV * DV, p.dev_status)) {
                 __nv_bfloat16 *op = og + (bt * HV + h) * DV + row0;
                 if constexpr (R == 8) {
-                    uint4 wv;
-                    wv.x = pack_bf16x2(o[0], o[1]);
-                    wv.y = pack_bf16x2(o[2], o[3]);
-                    wv.z = pack_bf16x2(o[4], o[5]);
-                    wv.w = pack_bf16x2(o[6], o[7]);
-                    *reinterpret_cast<uint4 *>(op) = wv;
+                    // two 8-byte stores: `out` is only required to be 8-byte aligned
+                    uint2 w0, w1;
+                    w0.x = pack_bf16x2(o[0], o[1]);
+                    w0.y = pack_bf16x2(o[2], o[3]);
+                    w1.x = pack_bf16x2(o[4], o[5]);
+                    w1.y = pack_bf16x2(o[6], o[7]);
+                    reinterpret_cast<uint2 *>(op)[0] = w0;
+                    reinterpret_cast<uint2 *>(op)[1] = w1;
                 } else if constexpr (R == 4) {
                     uint2 wv;
                     wv.x = pack_bf16x2(o[0], o[1]);

@@ -319,3 +319,26 @@ def test_stream_form_walks_many_units(gdn, W, oracle_mod):
         else:
             assert torch.equal(pc[s], c.pool[s]), s
     assert torch.equal(o.cpu()[bad], sentinel[bad])
+
+
+@pytest.mark.parametrize("B", [12, 96])   # persistent form; one-CTA form (8 rows per lane)
+def test_output_only_8_byte_aligned(gdn, W, oracle_mod, B):
+    """The ABI asks for an 8-byte aligned `out`: an output that starts 8 bytes past a 16-byte
+    boundary gets the same bytes as an aligned one, from both launch forms."""
+    c = W.make_decode(1000 + B, P=2 * B + 16, B=B, T=1, nh=1, H=32, Dv=128, pad_frac=0.1,
+                      write_mode="distinct")
+    aligned, _ = run_gpu(gdn, c)
+    buf = torch.full((B * 32 * 128 + 4,), 7.0, dtype=torch.bfloat16, device="cuda")
+    out = buf[4:].view(B, 1, 32, 128)
+    assert out.data_ptr() % 16 == 8
+    pool = dev(c.pool)
+    o, _ = gdn.gdn_decode(dev(c.q), dev(c.k), dev(c.v), pool, dev(c.read_idx), dev(c.A_log),
+                          dev(c.a), dev(c.dt_bias), dev(c.b), scale=c.scale, out=out,
+                          use_qk_l2norm=c.use_qk_l2norm, write_idx=dev(c.write_idx))
+    torch.cuda.synchronize()
+    live = (c.read_idx >= 0).cuda()
+    assert torch.equal(o[live], aligned.cuda()[live])
+    assert (buf[:4] == 7.0).all()
+    rows = np.nonzero(c.read_idx.numpy() >= 0)[0][:6]
+    ro, _ = run_oracle(oracle_mod, c, rows=rows)
+    assert rel_l2(f64(o.cpu()[torch.from_numpy(rows)]), ro) <= TOL_BF16
