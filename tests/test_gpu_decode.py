@@ -342,3 +342,31 @@ def test_output_only_8_byte_aligned(gdn, W, oracle_mod, B):
     rows = np.nonzero(c.read_idx.numpy() >= 0)[0][:6]
     ro, _ = run_oracle(oracle_mod, c, rows=rows)
     assert rel_l2(f64(o.cpu()[torch.from_numpy(rows)]), ro) <= TOL_BF16
+
+
+def test_decode_equals_prefill_with_host_gate(gdn, W):
+    """nh = 1 decode over 16 tokens equals the tensor-core prefill of the same tokens with
+    g = -exp(A_log) softplus20(a + dt_bias) and beta = sigmoid(b) evaluated on the host; q and k
+    are unit rows and both in-kernel norms are off (their epsilons differ)."""
+    B, T, H, Dv = 4, 16, 4, 128
+    c = W.make_decode(1200, P=8, B=B, T=T, nh=1, H=H, Dv=Dv, write_mode="none",
+                      host_norm_qk=True, use_qk_l2norm=False)
+    reads = c.read_idx.to(torch.int64)
+    init = c.pool[reads].clone()   # the prefill's initial states, before the pool is updated
+    pool = dev(c.pool)
+    od, _ = gdn.gdn_decode(dev(c.q), dev(c.k), dev(c.v), pool, dev(c.read_idx), dev(c.A_log),
+                           dev(c.a), dev(c.dt_bias), dev(c.b), scale=c.scale,
+                           use_qk_l2norm=False)
+    torch.cuda.synchronize()
+    x = c.a.double() + c.dt_bias.double()[None, None, :]
+    sp = torch.where(x > 20, x, torch.log1p(torch.exp(x)))
+    g = (-torch.exp(c.A_log.double())[None, None, :] * sp).float().reshape(B * T, H)
+    beta = torch.sigmoid(c.b[:, :, 0].double()).float().reshape(B * T, H)
+    op, fp = gdn.gdn_prefill(dev(c.q.reshape(B * T, H, 128)), dev(c.k[:, :, 0].reshape(B * T, H, 128)),
+                             dev(c.v[:, :, 0].reshape(B * T, H, Dv)), dev(g), dev(beta),
+                             dev(torch.arange(0, B * T + 1, T, dtype=torch.int32)),
+                             dev(init), scale=c.scale, qk_l2norm=False)
+    torch.cuda.synchronize()
+    assert gdn.prefill_uses_chunked(torch.bfloat16, H, 128, Dv)
+    assert rel_l2(f64(od.reshape(B * T, H, Dv)), f64(op)) <= TOL_BF16
+    assert rel_l2(f64(pool[reads.cuda()]), f64(fp)) <= TOL_BF16

@@ -286,3 +286,26 @@ def test_full_long_prefill_sampled_heads(gdn, W, oracle_mod):
     out, fs = run_gpu_prefill(c)
     assert torch.isfinite(out.float()).all() and torch.isfinite(fs).all()
     _sampled_heads_parity(oracle_mod, c, out, fs, [0, 31])
+
+
+@pytest.mark.parametrize("n", [64, 100])
+def test_split_and_resume_on_tensor_cores(gdn, W, n):
+    """A request run as two calls, the second starting from the first's final state, equals one
+    call (split on a chunk boundary and inside a chunk)."""
+    import copy
+    L = 230
+    c = W.make_prefill(124, [L], 2, 4, 128, 128, init_std=0.02, qk_l2norm=True)
+    assert gdn.prefill_uses_chunked(c.q.dtype, 4, 128, 128)
+    o_full, f_full = run_gpu_prefill(c)
+    parts, init = [], c.initial_state
+    for lo, hi in ((0, n), (n, L)):
+        s = copy.copy(c)
+        for name in ("q", "k", "v", "g", "beta"):
+            setattr(s, name, getattr(c, name)[lo:hi].contiguous())
+        s.cu_seqlens = torch.tensor([0, hi - lo], dtype=torch.int32)
+        s.initial_state = init
+        o, f = run_gpu_prefill(s)
+        parts.append(o.cpu())
+        init = f.cpu()
+    assert rel_l2(f64(torch.cat(parts)), f64(o_full)) <= TOL_BF16
+    assert rel_l2(f64(init), f64(f_full)) <= TOL_BF16
