@@ -5,7 +5,14 @@
 
 One step = one gdn_prefill call over the whole prefill workload (default: 8
 ragged requests with lengths U[1,4096], Hq=16, Hv=32, Dk=Dv=128, bf16), inputs
-resident in HBM.  `value` is prefill tokens/s over all ranks.  The same run
+resident in HBM, consecutive launches alternating between two independent input
+sets.  `value` is prefill tokens/s over all ranks.  After the K timed steps the
+same K-launch window is repeated until a quarter second of launches has been
+timed, so that the clock record covers a few dozen samples; the repeats are
+reported beside the measurement.  The long-context workload (B=1, S=32768) is
+timed the same way through the same call and reported under "long_prefill".
+`roofline.bound` is the roof (tensor cores or HBM) whose ideal time is longer;
+both fractions are reported.  The same run
 then times gdn_decode over the state-pool workload (pool [1024,32,128,128]
 fp32, 256 rows with 13 padding rows) for K steps and reports its state-pool
 GB/s under "decode", and gdn_conv1d (the causal conv feeding q, k, v: conv_dim
@@ -245,39 +252,77 @@ def to_dev(t):
     return None if t is None else t.cuda(non_blocking=False)
 
 
-def time_prefill(gdn, case, steps, warmup, world):
-    q, k, v, g, beta = map(to_dev, (case.q, case.k, case.v, case.g, case.beta))
-    cu, init = to_dev(case.cu_seqlens), to_dev(case.initial_state)
+def prefill_sets(case, nsets):
+    """`nsets` independent device copies of the prefill inputs and outputs, used in turn by
+    consecutive launches: by the time a set comes round again the other sets (each larger than
+    L2) have streamed through L2, so no launch re-reads its initial states, gates or q/k/v from
+    L2 (the rotation stands in for an L2 flush between launches)."""
     Hq, Hv, Dk, Dv = case.dims
-    out = torch.empty((case.N, Hv, Dv), dtype=case.q.dtype, device="cuda")
-    fs = torch.empty((case.B, Hv, Dv, Dk), dtype=torch.float32, device="cuda")
+    sets = []
+    for _ in range(nsets):
+        q, k, v, g, beta = map(to_dev, (case.q, case.k, case.v, case.g, case.beta))
+        cu, init = to_dev(case.cu_seqlens), to_dev(case.initial_state)
+        out = torch.empty((case.N, Hv, Dv), dtype=case.q.dtype, device="cuda")
+        fs = torch.empty((case.B, Hv, Dv, Dk), dtype=torch.float32, device="cuda")
+        sets.append((q, k, v, g, beta, cu, init, fs, out))
+    return sets
 
-    def step():
+
+def time_prefill(gdn, case, steps, warmup, world, nsets=2, min_window_s=0.25):
+    """K timed gdn_prefill launches (one per step, rotating over `nsets` input sets), then
+    further windows of K launches until at least `min_window_s` of launches have been timed, so
+    that the clock record of the prefill covers a few dozen samples.  The first window is the
+    reported measurement; the repeats are reported beside it.  Every window is bracketed by a
+    barrier and a device synchronisation; per-launch CUDA events on the launching stream."""
+    sets = prefill_sets(case, nsets)
+
+    def step(i):
+        q, k, v, g, beta, cu, init, fs, out = sets[i % nsets]
         gdn.gdn_prefill(q, k, v, g, beta, cu, init, fs, out, num_requests=case.B,
                         scale=case.scale, qk_l2norm=case.qk_l2norm)
 
-    for _ in range(warmup):
-        step()
+    for i in range(warmup):
+        step(i)
     stream = torch.cuda.current_stream()
-    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-          for _ in range(steps)]
-    barrier(world)
-    torch.cuda.synchronize()
-    t0 = torch.cuda.Event(enable_timing=True)
-    t1 = torch.cuda.Event(enable_timing=True)
-    host0 = time.time()
-    t0.record(stream)
-    for s, e in ev:
-        s.record(stream)
-        step()
-        e.record(stream)
-    t1.record(stream)
-    torch.cuda.synchronize()
-    host1 = time.time()
-    barrier(world)
-    total_ms = t0.elapsed_time(t1)
-    launch_ms = [s.elapsed_time(e) for s, e in ev]
-    time_prefill.window = (host0, host1)
+
+    def window(base):
+        ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+              for _ in range(steps)]
+        barrier(world)
+        torch.cuda.synchronize()
+        t0 = torch.cuda.Event(enable_timing=True)
+        t1 = torch.cuda.Event(enable_timing=True)
+        host0 = time.time()
+        t0.record(stream)
+        for i, (s, e) in enumerate(ev):
+            s.record(stream)
+            step(base + i)
+            e.record(stream)
+        t1.record(stream)
+        torch.cuda.synchronize()
+        host1 = time.time()
+        barrier(world)
+        return t0.elapsed_time(t1), [s.elapsed_time(e) for s, e in ev], (host0, host1)
+
+    total_ms, launch_ms, (h0, h1) = window(warmup)
+    repeats = []
+    timed_s = total_ms / 1e3
+    n = 1
+    # every rank takes the same number of windows: the count follows rank 0's first window
+    want = max(0, math.ceil(min_window_s / max(timed_s, 1e-6)) - 1)
+    if world > 1:
+        import torch.distributed as dist
+        t = torch.tensor([want], dtype=torch.int64, device="cuda")
+        dist.broadcast(t, 0)
+        want = int(t.item())
+    for _ in range(want):
+        w_ms, w_launch, (_, h1) = window(warmup + n * steps)
+        repeats.append(w_ms / steps)
+        n += 1
+    del sets
+    time_prefill.window = (h0, h1)
+    time_prefill.repeats = repeats
+    time_prefill.launches = n * steps
     return total_ms, launch_ms
 
 
@@ -358,26 +403,31 @@ def time_prefill_e2e(gdn, case, steps, warmup, world):
     return t0.elapsed_time(t1), h2d, d2h
 
 
-def time_decode(gdn, case, steps, warmup, world, graph=False):
+def time_decode(gdn, case, steps, warmup, world, graph=False, npools=1):
     """Per-launch CUDA events around back-to-back launches; with graph=True the `steps` launches
     are captured in one CUDA graph (for launches short enough that the Python call would
     otherwise show in the events), replayed once untimed and once timed, and the mean per launch
-    is returned for every step."""
-    q, k, v, a, b = map(to_dev, (case.q, case.k, case.v, case.a, case.b))
-    A_log, dt_bias = to_dev(case.A_log), to_dev(case.dt_bias)
-    ri, wi, si = to_dev(case.read_idx), to_dev(case.write_idx), to_dev(case.scatter_idx)
-    pool = to_dev(case.pool)
+    is returned for every step.  With npools > 1 consecutive launches use `npools` independent
+    copies of the pool (and of the inputs), so that one lap of the rotation moves more bytes than
+    L2 holds and no launch finds its slots still in L2 from an earlier launch."""
     B, T, H, Dk = case.q.shape
     HV, Dv = case.v.shape[3], case.v.shape[4]
-    out = torch.zeros((B, T, HV, Dv), dtype=torch.bfloat16, device="cuda")
+    sets = []
+    for _ in range(npools):
+        q, k, v, a, b = map(to_dev, (case.q, case.k, case.v, case.a, case.b))
+        out = torch.zeros((B, T, HV, Dv), dtype=torch.bfloat16, device="cuda")
+        sets.append((q, k, v, a, b, to_dev(case.pool), out))
+    A_log, dt_bias = to_dev(case.A_log), to_dev(case.dt_bias)
+    ri, wi, si = to_dev(case.read_idx), to_dev(case.write_idx), to_dev(case.scatter_idx)
 
-    def step(stream=None):
+    def step(i, stream=None):
+        q, k, v, a, b, pool, out = sets[i % npools]
         gdn.gdn_decode(q, k, v, pool, ri, A_log, a, dt_bias, b, scale=case.scale, out=out,
                        scatter_idx=si, use_qk_l2norm=case.use_qk_l2norm, write_idx=wi,
                        stream=stream)
 
-    for _ in range(warmup):
-        step()
+    for i in range(warmup):
+        step(i)
     stream = torch.cuda.current_stream()
     barrier(world)
     torch.cuda.synchronize()
@@ -386,8 +436,8 @@ def time_decode(gdn, case, steps, warmup, world, graph=False):
         g = torch.cuda.CUDAGraph()
         with torch.cuda.stream(side):
             with torch.cuda.graph(g, stream=side):
-                for _ in range(steps):
-                    step(side)
+                for i in range(steps):
+                    step(i, side)
         torch.cuda.synchronize()
         g.replay()   # first replay uploads the graph: untimed
         torch.cuda.synchronize()
@@ -398,17 +448,17 @@ def time_decode(gdn, case, steps, warmup, world, graph=False):
         torch.cuda.synchronize()
         barrier(world)
         per = e0.elapsed_time(e1) / steps
-        del g, pool
+        del g, sets
         return [per] * steps
     ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
           for _ in range(steps)]
-    for s, e in ev:
+    for i, (s, e) in enumerate(ev):
         s.record(stream)
-        step()
+        step(i)
         e.record(stream)
     torch.cuda.synchronize()
     barrier(world)
-    del pool
+    del sets
     return [s.elapsed_time(e) for s, e in ev]
 
 
@@ -423,19 +473,24 @@ def conv_bytes(case):
     return 2 * N * C * esz + 2 * live * C * (K - 1) * esz + C * K * esz
 
 
-def time_conv(gdn, case, steps, warmup, world, graph=False):
+def time_conv(gdn, case, steps, warmup, world, graph=False, nsets=1):
     """Per-launch CUDA events around back-to-back launches; with graph=True the `steps`
     launches are captured in one CUDA graph (host launch cost out of the way for small calls)
-    and the mean per launch is returned for every step."""
-    x, w, st, si, ro = map(to_dev, (case.x, case.weight, case.conv_state, case.slot_idx,
-                                    case.row_offsets))
-    out = torch.empty_like(x)
+    and the mean per launch is returned for every step.  With nsets > 1 consecutive launches
+    use `nsets` independent copies of x, the window pool and out, so that one lap of the
+    rotation moves more bytes than L2 holds."""
+    w, si, ro = map(to_dev, (case.weight, case.slot_idx, case.row_offsets))
+    sets = []
+    for _ in range(nsets):
+        x, st = to_dev(case.x), to_dev(case.conv_state)
+        sets.append((x, st, torch.empty_like(x)))
 
-    def step(stream=None):
+    def step(i, stream=None):
+        x, st, out = sets[i % nsets]
         gdn.gdn_conv1d(x, w, st, si, ro, out, stream=stream)
 
-    for _ in range(warmup):
-        step()
+    for i in range(warmup):
+        step(i)
     stream = torch.cuda.current_stream()
     barrier(world)
     torch.cuda.synchronize()
@@ -444,8 +499,8 @@ def time_conv(gdn, case, steps, warmup, world, graph=False):
         g = torch.cuda.CUDAGraph()
         with torch.cuda.stream(side):
             with torch.cuda.graph(g, stream=side):
-                for _ in range(steps):
-                    step(side)
+                for i in range(steps):
+                    step(i, side)
         torch.cuda.synchronize()
         g.replay()
         torch.cuda.synchronize()
@@ -460,12 +515,13 @@ def time_conv(gdn, case, steps, warmup, world, graph=False):
         return [per] * steps
     ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
           for _ in range(steps)]
-    for s, e in ev:
+    for i, (s, e) in enumerate(ev):
         s.record(stream)
-        step()
+        step(i)
         e.record(stream)
     torch.cuda.synchronize()
     barrier(world)
+    del sets
     return [s.elapsed_time(e) for s, e in ev]
 
 
@@ -511,6 +567,41 @@ def cpu_oracle_sample(case, target_s=10.0, repeats=1):
             "runs": len(times)}
 
 
+def prefill_roofline(gdn, case, launch_ms, peaks, sm_mhz, traffic):
+    """Roofline of one prefill workload from its per-launch CUDA-event times.
+
+    The kernel is held to both of its roofs: the tensor cores (algorithmic FLOPs of the chunk
+    form against the measured bf16 peak) and HBM (algorithmic bytes against the measured copy
+    bandwidth).  `bound` is the roof whose ideal time is the longer one, and `frac` is taken
+    against it; both fractions are reported."""
+    Hq, Hv, Dk, Dv = case.dims
+    avg_s = statistics.mean(launch_ms) / 1e3
+    if not gdn.prefill_uses_chunked(case.q.dtype, Hv, Dk, Dv):
+        byts = prefill_bytes(case)
+        ach = byts / avg_s / 1e9
+        return {"kernel": "gdn_prefill_seq", "bound": "hbm", "achieved": ach,
+                "peak": peaks["hbm_gbs"], "unit": "GB/s", "frac": ach / peaks["hbm_gbs"],
+                "traffic": None, "peak_source": peaks["source"]}
+    flops = case.N * Hv * prefill_flops_per_token_head(Dk, Dv)
+    byts = prefill_bytes(case)
+    tc_peak, hbm_peak = peaks["bf16_tflops"], peaks["hbm_gbs"]
+    t_tc = flops / (tc_peak * 1e12)
+    t_hbm = byts / (hbm_peak * 1e9)
+    tc = {"achieved": flops / avg_s / 1e12, "peak": tc_peak, "unit": "TFLOP/s",
+          "frac": flops / avg_s / 1e12 / tc_peak, "ideal_us": t_tc * 1e6,
+          "algorithmic_flops": flops}
+    hbm = {"achieved": byts / avg_s / 1e9, "peak": hbm_peak, "unit": "GB/s",
+           "frac": byts / avg_s / 1e9 / hbm_peak, "ideal_us": t_hbm * 1e6,
+           "algorithmic_bytes": byts}
+    b = tc if t_tc >= t_hbm else hbm
+    return {"kernel": "gdn_prefill_chunk", "bound": "tensor" if t_tc >= t_hbm else "hbm",
+            "achieved": b["achieved"], "peak": b["peak"], "unit": b["unit"], "frac": b["frac"],
+            "traffic": traffic, "tensor": tc, "hbm": hbm,
+            "ms_per_launch": avg_s * 1e3,
+            "kcycles_per_launch": None if sm_mhz is None else avg_s * 1e3 * sm_mhz,
+            "peak_source": peaks["source"] + " (burst bf16; copy bandwidth)"}
+
+
 def profile_phase(gdn, workloads, args):
     """Run one phase for `--steps` steps after `--warmup` (under a profiler); prints timings."""
     if args.phase == "prefill":
@@ -546,7 +637,9 @@ def workload_config(case, name):
     return {"workload": case.name, "requests": case.B, "tokens": case.N,
             "lengths": "U[1,4096] seeded" if name == "ragged" else str(case.N),
             "Hq": Hq, "Hv": Hv, "Dk": Dk, "Dv": Dv, "chunk": CHUNK,
-            "l2": "inputs larger than L2 (q+k+v+out > 126 MB), no flush"}
+            "l2": "inputs larger than L2 (q+k+v+out > 126 MB), and consecutive launches "
+                  "alternate between two independent input sets, so no launch re-reads "
+                  "initial states, gates or q/k/v left in L2 by the previous one"}
 
 
 def main():
@@ -559,6 +652,7 @@ def main():
     ap.add_argument("--no-decode", action="store_true")
     ap.add_argument("--no-conv", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-long", action="store_true", help="skip the long-context prefill line")
     ap.add_argument("--no-cpu", action="store_true", help="skip the CPU oracle baseline")
     ap.add_argument("--phase", default="all", choices=["all", "prefill", "decode", "conv"],
                     help="prefill or decode alone (for profiling); 'all' for the JSON line")
@@ -606,31 +700,32 @@ def main():
     clocks.start()
     total_ms, launch_ms = time_prefill(gdn, case, args.steps, args.warmup, world)
     prefill_window = time_prefill.window
+    prefill_repeats = time_prefill.repeats
+    launches = time_prefill.launches
     max_ms = max_over_ranks(total_ms, world)
     ms_per_step = max_ms / args.steps
     tokens = case.N * world
     value = job_throughput(case.N, world, ms_per_step)
-    launches = args.steps
+    prefill_clocks = clocks.summary(prefill_window, "prefill timed windows")
+    traffic = ncu_traffic("prefill_chunk_ragged_prefill.md", "prefill_chunk.cu") \
+        if args.workload == "ragged" else None
+    roof = prefill_roofline(gdn, case, launch_ms, peaks, prefill_clocks["sm_mhz"], traffic)
+    roof["repeat_windows_ms_per_launch"] = prefill_repeats
 
-    chunked = gdn.prefill_uses_chunked(case.q.dtype, Hv, Dk, Dv)
-    avg_launch_s = statistics.mean(launch_ms) / 1e3
-    if chunked:
-        flops = case.N * Hv * prefill_flops_per_token_head(Dk, Dv)
-        ach = flops / avg_launch_s / 1e12
-        traffic = ncu_traffic("prefill_chunk_ragged_prefill.md", "prefill_chunk.cu") \
-            if args.workload == "ragged" else None
-        roof = {"kernel": "gdn_prefill_chunk", "bound": "tensor", "achieved": ach,
-                "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
-                "frac": ach / peaks["bf16_tflops"], "traffic": traffic,
-                "algorithmic_bytes": prefill_bytes(case),
-                "hbm_frac": prefill_bytes(case) / avg_launch_s / 1e9 / peaks["hbm_gbs"],
-                "peak_source": peaks["source"] + " (burst bf16)"}
-    else:
-        byts = prefill_bytes(case)
-        ach = byts / avg_launch_s / 1e9
-        roof = {"kernel": "gdn_prefill_seq", "bound": "hbm", "achieved": ach,
-                "peak": peaks["hbm_gbs"], "unit": "GB/s", "frac": ach / peaks["hbm_gbs"],
-                "traffic": None, "peak_source": peaks["source"]}
+    # the long-context workload (B = 1, S = 32768) through the same call, in the same run
+    long_prefill = None
+    if args.workload == "ragged" and not args.no_long:
+        lcase = make_case("long")
+        l_total, l_launch = time_prefill(gdn, lcase, args.steps, args.warmup, world)
+        l_clocks = clocks.summary(time_prefill.window, "long-context prefill timed windows")
+        l_max = max_over_ranks(l_total, world) / args.steps
+        long_prefill = {
+            "workload": lcase.name, "tokens": lcase.N, "ms_per_step": l_max,
+            "value": job_throughput(lcase.N, world, l_max), "unit": "tokens/s",
+            "roofline": prefill_roofline(gdn, lcase, l_launch, peaks, l_clocks["sm_mhz"], None),
+            "repeat_windows_ms_per_launch": time_prefill.repeats, "clocks": l_clocks}
+        launches += time_prefill.launches
+        del lcase
 
     decode = decode_mtp = None
     if not args.no_decode:
@@ -648,14 +743,16 @@ def main():
         del dcase
         # MTP / Gated DeltaProduct: T = 4 tokens, 2 Householder sub-steps, per-token scatter
         mcase = workloads.mtp_case()
-        mms = time_decode(gdn, mcase, args.steps, args.warmup, world, graph=True)
+        mms = time_decode(gdn, mcase, args.steps, args.warmup, world, graph=True, npools=4)
         mmax = max_over_ranks(sum(mms), world) / args.steps
         mbytes = decode_bytes(mcase)
         decode_mtp = {"workload": mcase.name, "value": mbytes * world / (mmax / 1e3) / 1e9,
                       "unit": "GB/s", "bytes_per_step": mbytes, "ms_per_step": mmax,
                       "frac": mbytes / (statistics.mean(mms) / 1e3) / 1e9 / peaks["hbm_gbs"],
                       "peak": peaks["hbm_gbs"], "peak_source": peaks["source"],
-                      "timing": "one CUDA graph of K launches (pool 256 MB)"}
+                      "timing": "one CUDA graph of K launches rotating over 4 independent "
+                                "256 MB pools (690 MB moved per lap > L2): no slot is "
+                                "rewritten while an earlier write of it can still sit in L2"}
         launches += args.steps
         del mcase
 
@@ -665,8 +762,10 @@ def main():
                 ("conv1d", workloads.conv_ragged_case(), False,
                  "back-to-back launches, working set > L2 (steady-state HBM traffic)"),
                 ("conv1d_decode", workloads.conv_decode_case(), True,
-                 "one CUDA graph of K launches; 33.6 MB working set stays in L2")):
-            cms = time_conv(gdn, ccase, args.steps, args.warmup, world, graph=graph)
+                 "one CUDA graph of K launches rotating over 6 independent copies of x, the "
+                 "window pool and out (202 MB moved per lap > L2)")):
+            cms = time_conv(gdn, ccase, args.steps, args.warmup, world, graph=graph,
+                            nsets=6 if graph else 1)
             cmax = max_over_ranks(sum(cms), world) / args.steps
             cbytes = conv_bytes(ccase)
             per_gpu = cbytes / (statistics.mean(cms) / 1e3) / 1e9
@@ -703,10 +802,10 @@ def main():
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
             "data": "synthetic", "config": dict(workload_config(case, args.workload),
                                                 parallelism=f"replicas{world}"),
-            "roofline": roof, "decode": decode, "decode_mtp": decode_mtp, "conv1d": conv,
+            "roofline": roof, "long_prefill": long_prefill, "decode": decode, "decode_mtp": decode_mtp, "conv1d": conv,
             "conv1d_decode": conv_dec,
             "e2e": e2e, "cpu_baseline": cpu,
-            "clocks": clocks.summary(prefill_window, "prefill timed region"),
+            "clocks": prefill_clocks,
             "clocks_all_phases": clocks.summary(),
             "gpu_launches": launches,
         }

@@ -149,6 +149,15 @@ def _check_cuda(name, t, dtype=None):
     return t.contiguous()
 
 
+def _align16(t):
+    """A contiguous input whose data does not start on a 16-byte boundary (a view such as
+    g[1:]) is copied into a fresh allocation, which the caching allocator aligns; gdn_prefill
+    requires 16-byte aligned inputs."""
+    if t is not None and t.data_ptr() % 16 != 0:
+        t = t.clone()
+    return t
+
+
 def gdn_prefill(q, k, v, g, beta, cu_seqlens=None, initial_state=None, final_state=None,
                 out=None, *, num_requests: Optional[int] = None, scale: Optional[float] = None,
                 qk_l2norm: bool = False, sequential: bool = False, update_rule: str = "gated_delta",
@@ -199,6 +208,7 @@ def gdn_prefill(q, k, v, g, beta, cu_seqlens=None, initial_state=None, final_sta
     dt_bias = _check_cuda("dt_bias", dt_bias, torch.float32)
     cu_seqlens = _check_cuda("cu_seqlens", cu_seqlens, torch.int32)
     initial_state = _check_cuda("initial_state", initial_state, torch.float32)
+    q, k, v, g, beta, initial_state = map(_align16, (q, k, v, g, beta, initial_state))
     N, Hq, Dk = q.shape
     Hv, Dv = v.shape[1], v.shape[2]
     if k.shape != q.shape or v.shape[0] != N or (g is not None and g.shape != (N, Hv)) or \

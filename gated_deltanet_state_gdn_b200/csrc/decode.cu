@@ -393,13 +393,14 @@ decode_kernel(const GdnDecodeArgs p)
 }
 
 // ---------------------------------------------------------------- persistent, prefetching
-// bounded wait on an mbarrier phase: false when it does not complete within ~2^31 cycles
-__device__ __forceinline__ bool wait_phase(uint32_t bar, uint32_t parity)
+// bounded wait on an mbarrier phase: false when it does not complete within `limit` cycles
+// (2^31, about a second, for a wait on the pipeline)
+__device__ __forceinline__ bool wait_phase(uint32_t bar, uint32_t parity, long long limit = 1ll << 31)
 {
     if (sm100::mbar_try_wait(bar, parity)) return true;
     const long long start = clock64();
     while (!sm100::mbar_try_wait(bar, parity))
-        if (clock64() - start > (1ll << 31)) return false;
+        if (clock64() - start > limit) return false;
     return true;
 }
 
@@ -504,7 +505,10 @@ decode_stream_kernel(const GdnDecodeArgs p)
         if (__syncthreads_or(timed_out)) {
             if (threadIdx.x == 0) {
                 if (p.dev_status) atomicOr(p.dev_status, GDN_DEV_TIMEOUT);
-                wait_phase(bar, (uint32_t)(it & 1));   // let copies still in flight land
+                // let copies still in flight land before the CTA's shared memory goes away;
+                // one that is on its way lands within microseconds, so this wait is short
+                // (2^24 cycles, ~8 ms) rather than a second bound on bytes that never come
+                wait_phase(bar, (uint32_t)(it & 1), 1ll << 24);
             }
             return;
         }

@@ -99,8 +99,8 @@ gdn_status gdn_prefill(const void *q, const void *k, const void *v, const float 
     const size_t gb_bytes = (size_t)N * Hv * 4;
     const size_t st_bytes = (size_t)B * Hv * Dv * Dk * 4;
     if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(out, 16) ||
-        !aligned(initial_state, 16) || !aligned(final_state, 16) || !aligned(g, 4) ||
-        !aligned(beta, 4) || !aligned(cu_seqlens, 4) || !aligned(a_log, 4) || !aligned(dt_bias, 4))
+        !aligned(initial_state, 16) || !aligned(final_state, 16) || !aligned(g, 16) ||
+        !aligned(beta, 16) || !aligned(cu_seqlens, 4) || !aligned(a_log, 4) || !aligned(dt_bias, 4))
         return GDN_ERR_ALIGN;
     if (overlaps(initial_state, st_bytes, final_state, st_bytes)) return GDN_ERR_ALIAS;
     if (overlaps(out, v_bytes, q, qk_bytes) || overlaps(out, v_bytes, k, qk_bytes) ||

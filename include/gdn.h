@@ -132,9 +132,12 @@ enum {
  *   dev_status     optional device int32; GDN_DEV_TIMEOUT is OR-ed in if an
  *                  internal pipeline wait of the chunked kernel exceeds its
  *                  bound (the call's outputs are then invalid).
- * Requirements: 1 <= Dk, Dv <= 256; Hv % Hq == 0; q, k, v, out,
- * initial_state and final_state 16-byte aligned; out must not overlap any
- * input.  bf16 or fp16 with Dk, Dv in {8, 16, ..., 128} and Hv % 4 == 0 runs the
+ * Requirements: 1 <= Dk, Dv <= 256; Hv % Hq == 0; q, k, v, g, beta, out,
+ * initial_state and final_state 16-byte aligned (the chunked kernel reads g
+ * and beta through tensor maps, whose base must be 16-byte aligned; the rule
+ * holds for every call, so a view such as g[1:] of a 4-byte aligned buffer is
+ * GDN_ERR_ALIGN, not a launch failure); out must not overlap any input.
+ * bf16 or fp16 with Dk, Dv in {8, 16, ..., 128} and Hv % 4 == 0 runs the
  * chunked tensor-core kernel (unless GDN_PREFILL_SEQUENTIAL; its operand tiles
  * take the activations' type, fp32 accumulation and state); everything else
  * (fp32, heads wider than 128 or not a multiple of 8) runs the per-token

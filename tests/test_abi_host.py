@@ -78,6 +78,9 @@ def test_prefill_host_validation(L):
     assert prefill(L, final=None) == 1
     assert prefill(L, beta=None) == 1
     assert prefill(L, v=P(3, 8)) == 4                     # 16-byte alignment
+    assert prefill(L, g=P(4, 4)) == 4                     # g, beta: tensor-map bases
+    assert prefill(L, beta=P(5, 8)) == 4
+    assert prefill(L, g=P(4, 4), dtype=1, Hv=4, Dk=128, Dv=128) == 4
     assert prefill(L, g=P(4, 2)) == 4
     assert prefill(L, flags=1 << 9) == 6                  # unknown flag
     assert prefill(L, init=P(7, 256), final=P(7)) == 5    # initial/final overlap
