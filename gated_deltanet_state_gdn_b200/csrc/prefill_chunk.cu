@@ -3,9 +3,10 @@
 // Operation: the recurrence of "com.microsoft.GatedDeltaNet" (Description),
 //   S_t = exp(g_t) S_{t-1} + k_t (beta_t (v_t - exp(g_t) S_{t-1}^T k_t))^T,
 //   o_t = scale * S_t^T q_t,
-// for bf16 q/k/v with Dk, Dv <= 128 (multiples of 8; smaller heads are read as
-// 128-wide tiles zero-filled past their end by the TMA, which leaves every
-// product unchanged), computed 64 tokens at a time.  The
+// for bf16 or fp16 q/k/v with Dk, Dv <= 128 (smaller heads are read as 128-wide
+// tiles zero-filled past their end, by the TMA when Dk and Dv are multiples of 8 and
+// Hv % 4 == 0, else by plain loads of the TMA warp; zero padding leaves every product
+// unchanged), computed 64 tokens at a time.  The
 // chunk form (derived from the recurrence; the op page names a chunk-parallel
 // prefill with chunk_size 64 and states that the chunk size does not change
 // the result) is, for a chunk with incoming state S0 (Dk x Dv), cumulative
@@ -54,8 +55,16 @@
 //   warp  12    TMA producers (lane 0: q/k/g/beta tiles in three stages; lane 1: v tiles)
 //   warp  13    TMEM owner; UMMA issuer of the state chain (1a, 1b, 2, 3)
 //   warp  14    UMMA issuer of the prep stream (G, W, U~)
-// Every wait on an mbarrier is bounded; on timeout the kernel sets
-// GDN_DEV_TIMEOUT in the status word, drains and exits.
+// Every wait on an mbarrier is bounded (2^31 cycles) and also ends as soon as another
+// role has raised the CTA's abort flag; a wait that runs out raises the flag and sets
+// GDN_DEV_TIMEOUT in the status word.  After an abort every thread still reaches the same
+// barriers: each of the three 128-thread groups (state, prep front, prep back) runs one
+// control flow in which a failed wait only clears `ok` (named barriers and warp-collective
+// tcgen05.ld/st are reached on every path) and leaves its chunk loop through the per-chunk
+// OR vote; the single-thread roles (TMA lanes, UMMA issuers) leave their loops on the flag;
+// all threads then meet the CTA barrier that ends the batch and see the flag alike.  The
+// teardown drains copies and MMAs still in flight (bounded) and frees TMEM.  Checked builds
+// can force this path from the host (GDN_DEV_TEST_STALL).
 #include <cudaTypedefs.h>
 #include <stdio.h>
 #include <string.h>
@@ -102,7 +111,7 @@ constexpr uint32_t GATE_BYTES = 2560;
 constexpr uint32_t OFF_GATE = OFF_GB0 + KQ_STAGES * 2048;      // KQ_STAGES x processed gates
 constexpr uint32_t OFF_UNITS = OFF_GATE + KQ_STAGES * GATE_BYTES;   // int4 x MAX_UNITS
 constexpr uint32_t OFF_BARS = OFF_UNITS + MAX_UNITS * 16;
-constexpr uint32_t NUM_BARS = 30;
+constexpr uint32_t NUM_BARS = 32;
 static_assert(NUM_BARS * 8 <= 256, "barrier area");
 constexpr uint32_t OFF_MISC = OFF_BARS + 256;                  // tmem base, abort flag, count
 constexpr uint32_t OFF_OGR = OFF_MISC + 64;                    // Gamma_i rq_i for the outputs, 64 floats
@@ -131,7 +140,9 @@ enum {
     B_KQ_FULL = 0, B_KQ_EMPTY = 3, B_V_FULL = 6, B_V_EMPTY = 7, B_GATE_FULL = 8,
     B_GATE_EMPTY = 11, B_G_DONE = 14, B_T_READY = 15, B_W_DONE = 16, B_WNEG = 17,
     B_S_READY = 18, B_U_DONE = 19, B_E1 = 20, B_S_DONE = 21, B_Z_DONE = 22, B_Y_FREE = 23,
-    B_G_FREE = 24, B_A_READY = 25, B_SOLVE_FREE = 27, B_UT_DONE = 29, B_COUNT = 30
+    B_G_FREE = 24, B_A_READY = 25, B_SOLVE_FREE = 27, B_UT_DONE = 29,
+    B_DRAIN_CHAIN = 30, B_DRAIN_PREP = 31,   // abort teardown: each UMMA issuer's last commit
+    B_COUNT = 32
 };
 static_assert(B_COUNT == (int)NUM_BARS, "barrier count");
 
@@ -154,8 +165,13 @@ struct __align__(64) Params {
     float scale;
     int32_t qk_l2norm;
     int32_t has_decay, has_retrieval, beta_sigmoid;   // update rule and activations
-    int32_t Dk, Dv;   // head sizes (multiples of 8, <= 128; the tiles are zero-padded to 128)
+    int32_t Dk, Dv;   // head sizes (<= 128; the tiles are zero-padded to 128)
     const float *a_log, *dt_bias;                     // qwen gate when non-NULL
+    // plain staging (head sizes that are not multiples of 8, or Hv % 4 != 0: rows whose
+    // strides the tensor maps cannot describe): the TMA warp copies rows with ordinary loads
+    int32_t stage_plain;
+    const uint16_t *q, *k, *v;
+    const float *g, *beta;
 };
 
 // --------------------------------------------------------------------------
@@ -283,11 +299,17 @@ __device__ __noinline__ void load_state_tmem(const float *init, int Dk, uint32_t
 #pragma unroll 1
     for (int hq = 0; hq < 2; ++hq) {
         float x[64];
+        if (!GENERAL || (Dk & 3) == 0) {
 #pragma unroll
-        for (int c = 0; c < 64; c += 4) {
-            const float4 v = init && (!GENERAL || 64 * hq + c < Dk) ? ld4(init + 64 * hq + c)
-                                                                    : make_float4(0.f, 0.f, 0.f, 0.f);
-            x[c] = v.x; x[c + 1] = v.y; x[c + 2] = v.z; x[c + 3] = v.w;
+            for (int c = 0; c < 64; c += 4) {
+                const float4 v = init && (!GENERAL || 64 * hq + c < Dk) ? ld4(init + 64 * hq + c)
+                                                                        : make_float4(0.f, 0.f, 0.f, 0.f);
+                x[c] = v.x; x[c + 1] = v.y; x[c + 2] = v.z; x[c + 3] = v.w;
+            }
+        } else {
+            // rows of Dk floats with Dk % 4 != 0 are only 4-byte aligned
+#pragma unroll
+            for (int c = 0; c < 64; ++c) x[c] = init && 64 * hq + c < Dk ? init[64 * hq + c] : 0.f;
         }
 #pragma unroll
         for (int q = 0; q < 4; ++q) {
@@ -597,6 +619,47 @@ __device__ __forceinline__ float build_row(uint32_t tl_gram, int qd, const float
     return rk;
 }
 
+// Plain staging of one chunk's q/k (and g/beta) or v rows into the swizzled operand tiles, for
+// head sizes the tensor maps cannot describe (row strides that are not multiples of 16 bytes).
+// The 32 lanes of the TMA warp copy element by element; the tiles were zeroed at kernel start
+// and positions past the head size are never written, so the padding stays zero exactly as
+// the TMA's fill would leave it.  Tokens at or past N read as zero, as with the TMA.
+__device__ __noinline__ void stage_plain_kq(const Params &p, uint8_t *kq, float *gtile, int qh, int h,
+                                            int64_t t0, bool has_decay, bool has_retrieval)
+{
+    const int lane = threadIdx.x & 31;
+    const int Dk = p.Dk;
+    const int n = C * Dk;
+    for (int idx = lane; idx < 2 * n; idx += 32) {
+        const int which = idx >= n;              // 0: k rows, 1: q rows
+        const int r = idx - which * n;
+        const int i = r / Dk, e = r - i * Dk;
+        const int64_t t = t0 + i;
+        uint16_t x = 0;
+        if (t < p.N) x = (which ? p.q : p.k)[(t * p.Hq + qh) * Dk + e];
+        const uint32_t off = (e >> 6) * KQ_KB + which * 8192u + sw128(i, (e & 63) >> 3) + (uint32_t)(e & 7) * 2u;
+        *reinterpret_cast<uint16_t *>(kq + off) = x;
+    }
+    for (int i = lane; i < C; i += 32) {
+        const int64_t t = t0 + i;
+        const bool in = t < p.N;
+        if (has_decay) gtile[i * 4 + (h & 3)] = in ? p.g[t * p.Hv + h] : 0.f;
+        if (has_retrieval) gtile[256 + i * 4 + (h & 3)] = in ? p.beta[t * p.Hv + h] : 0.f;
+    }
+}
+
+__device__ __noinline__ void stage_plain_v(const Params &p, uint8_t *vt, int h, int64_t t0)
+{
+    const int lane = threadIdx.x & 31;
+    const int Dv = p.Dv;
+    for (int idx = lane; idx < C * Dv; idx += 32) {
+        const int j = idx / Dv, e = idx - j * Dv;
+        const int64_t t = t0 + j;
+        const uint16_t x = t < p.N ? p.v[(t * p.Hv + h) * Dv + e] : (uint16_t)0;
+        *reinterpret_cast<uint16_t *>(vt + (e >> 6) * V_HALF + sw128(j, (e & 63) >> 3) + (uint32_t)(e & 7) * 2u) = x;
+    }
+}
+
 // ========================================================================== kernel
 // GENERAL = false: the default rule (gated_delta, no gate or beta activation), with the
 // variant switches folded at compile time; GENERAL = true reads them from p.
@@ -635,7 +698,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) gdn_prefill_chunk_kernel(const __
         for (int i = 0; i < (int)NUM_BARS; ++i) mbar_init(cx.bar(i), 1);
         fence_mbar_init();
     }
-    if (warp == TMA_WARP && lane == 0) {
+    if (warp == TMA_WARP && lane == 0 && !(GENERAL && p.stage_plain)) {
         prefetch_tmap(&p.tm_q);
         prefetch_tmap(&p.tm_k);
         prefetch_tmap(&p.tm_v);
@@ -650,6 +713,12 @@ __global__ void __launch_bounds__(NTHREADS, 1) gdn_prefill_chunk_kernel(const __
     static_assert(OFF_TB == OFF_P + KQ_STAGES * P_STAGE && OFF_TBG == OFF_TB + 8192, "tile order");
     for (int i = tid; i < (int)((OFF_TBG + 8192 - OFF_P) / 16); i += NTHREADS)
         reinterpret_cast<uint4 *>(smem + OFF_P)[i] = make_uint4(0u, 0u, 0u, 0u);
+    // plain staging writes only the head's own columns: the q/k stages and the v tile start
+    // zeroed, so their padding is zero as the TMA would fill it
+    static_assert(OFF_KQ0 == 0 && OFF_V == KQ_STAGES * KQ_STAGE, "staging tiles are contiguous");
+    if (GENERAL && p.stage_plain)
+        for (int i = tid; i < (int)((OFF_V + 16384) / 16); i += NTHREADS)
+            reinterpret_cast<uint4 *>(smem)[i] = make_uint4(0u, 0u, 0u, 0u);
     fence_proxy_async_smem();
     tc_fence_before();
     __syncthreads();
@@ -688,13 +757,50 @@ __global__ void __launch_bounds__(NTHREADS, 1) gdn_prefill_chunk_kernel(const __
             }
         }
 
-        if (warp == TMA_WARP) {
+        if (warp == TMA_WARP && GENERAL && p.stage_plain) {
+            // ------------------------------------------------------------ plain staging
+            // the whole warp stages each chunk's q/k/g/beta stage, then its v tile, in chunk
+            // order (the two streams are not independent here, which costs overlap but no
+            // progress: a v tile waits only on products of earlier chunks)
+            bool ok = true;
+            for (int k = 0; k < nunits && ok; ++k) {
+                const Unit un = load_unit(smem, k);
+                const int qh = (int)(((int64_t)un.h * p.Hq) / p.Hv);
+                const int nc = (un.len + C - 1) / C;
+                for (int n = 0; n < nc && ok; ++n) {
+                    const uint32_t ks = (gc + n) % KQ_STAGES;
+                    const int64_t t0 = (int64_t)un.start + (int64_t)n * C;
+                    if (kq_use[ks] > 0) ok = cx.wait(B_KQ_EMPTY + ks, (kq_use[ks] - 1) & 1);
+                    ok = __all_sync(0xffffffffu, ok);
+                    if (!ok) break;
+                    ++kq_use[ks];
+                    stage_plain_kq(p, smem + OFF_KQ0 + ks * KQ_STAGE,
+                                   reinterpret_cast<float *>(smem + OFF_GB0 + ks * 2048), qh, un.h, t0,
+                                   has_decay, has_retrieval);
+                    fence_proxy_async_smem();
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(cx.bar(B_KQ_FULL + ks));
+                    if (v_use > 0) ok = cx.wait(B_V_EMPTY, (v_use - 1) & 1);
+                    ok = __all_sync(0xffffffffu, ok);
+                    if (!ok) break;
+                    ++v_use;
+                    stage_plain_v(p, smem + OFF_V, un.h, t0);
+                    fence_proxy_async_smem();
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(cx.bar(B_V_FULL));
+                }
+                gc += nc;
+            }
+        } else if (warp == TMA_WARP) {
             // ------------------------------------------------------------ TMA producers
             // lane 0: q/k/g/beta tiles (KQ_STAGES stages); lane 1: v tiles (one stage).  The
             // two streams are released by different consumers (the state chain, the W/U~
             // products), so neither waits behind the other.  Each also pulls a later chunk
             // of its stream into L2, so that a reload does not start cold.
             if (lane == 0) {
+                // checked builds: a caller-requested stall makes the first q/k stage expect 16
+                // bytes more than its copies deliver, so every wait on it runs out
+                bool stall = batch0 == 0 && gdn::test_stall_requested(p.dev_status);
                 for (int k = 0; k < nunits && !cx.aborted(); ++k) {
                     const Unit un = load_unit(smem, k);
                     const int qh = (int)(((int64_t)un.h * p.Hq) / p.Hv);
@@ -707,7 +813,9 @@ __global__ void __launch_bounds__(NTHREADS, 1) gdn_prefill_chunk_kernel(const __
                         const uint32_t gb = sbase + OFF_GB0 + ks * 2048;
                         const int t0 = un.start + n * C;
                         const uint32_t kb = cx.bar(B_KQ_FULL + ks);
-                        mbar_arrive_expect_tx(kb, 32768 + (has_decay ? 1024 : 0) + (has_retrieval ? 1024 : 0));
+                        mbar_arrive_expect_tx(kb, 32768 + (has_decay ? 1024 : 0) + (has_retrieval ? 1024 : 0) +
+                                                      (stall ? 16 : 0));
+                        stall = false;
                         tma_load_3d(kq, &p.tm_k, kb, 0, qh, t0);
                         tma_load_3d(kq + KQ_KB, &p.tm_k, kb, 64, qh, t0);
                         tma_load_3d(kq + 8192, &p.tm_q, kb, 0, qh, t0);
@@ -1188,11 +1296,13 @@ __global__ void __launch_bounds__(NTHREADS, 1) gdn_prefill_chunk_kernel(const __
                 const float *init = p.initial_state && row_ok ? p.initial_state + st_off : nullptr;
                 float *fin = row_ok ? p.final_state + st_off : nullptr;
                 if (nc == 0) {
-                    if (row_ok) {
+                    if (row_ok && (!GENERAL || (Dk & 3) == 0)) {
                         for (int c = 0; c < Dk; c += 4) {
                             float4 v = init ? ld4(init + c) : make_float4(0.f, 0.f, 0.f, 0.f);
                             *reinterpret_cast<float4 *>(fin + c) = v;
                         }
+                    } else if (row_ok) {
+                        for (int c = 0; c < Dk; ++c) fin[c] = init ? init[c] : 0.f;
                     }
                     continue;
                 }
@@ -1302,9 +1412,13 @@ __global__ void __launch_bounds__(NTHREADS, 1) gdn_prefill_chunk_kernel(const __
                             if (!GENERAL && (!kChecked || row_ok)) {
 #pragma unroll
                                 for (int c = 0; c < 32; c += 4) st4(fin + 32 * q + c, x[c], x[c + 1], x[c + 2], x[c + 3]);
-                            } else if (row_ok) {
+                            } else if (row_ok && (Dk & 3) == 0) {
                                 for (int c = 0; c < 32 && 32 * q + c < Dk; c += 4)
                                     st4(fin + 32 * q + c, x[c], x[c + 1], x[c + 2], x[c + 3]);
+                            } else if (row_ok) {
+#pragma unroll
+                                for (int c = 0; c < 32; ++c)
+                                    if (32 * q + c < Dk) fin[32 * q + c] = x[c];
                             }
                         }
                     }
@@ -1349,10 +1463,20 @@ __global__ void __launch_bounds__(NTHREADS, 1) gdn_prefill_chunk_kernel(const __
                                 const uint4 v = *reinterpret_cast<const uint4 *>(ost + lane * 16);
                                 __syncwarp();
                                 const int i0 = 16 * q + 8 * hb;   // first token of this group
-                                if (i0 + tt < len_n && (!GENERAL || ocol < Dv) &&
-                                    in_range(((int64_t)(un.start + n * C + tt + i0) * p.Hv + un.h) * Dv + ocol,
-                                             8, (int64_t)p.N * p.Hv * Dv, p.dev_status))
-                                    *reinterpret_cast<uint4 *>(obase + (i0 / 8) * ostride8) = v;
+                                if (!GENERAL || (Dv & 7) == 0) {
+                                    if (i0 + tt < len_n && (!GENERAL || ocol < Dv) &&
+                                        in_range(((int64_t)(un.start + n * C + tt + i0) * p.Hv + un.h) * Dv + ocol,
+                                                 8, (int64_t)p.N * p.Hv * Dv, p.dev_status))
+                                        *reinterpret_cast<uint4 *>(obase + (i0 / 8) * ostride8) = v;
+                                } else if (i0 + tt < len_n && ocol < Dv) {
+                                    // rows of Dv elements with Dv % 8 != 0: element stores, only
+                                    // the head's own columns
+                                    const int ne = min(8, Dv - ocol);
+                                    const uint16_t *ve = reinterpret_cast<const uint16_t *>(&v);
+                                    if (in_range(((int64_t)(un.start + n * C + tt + i0) * p.Hv + un.h) * Dv + ocol,
+                                                 ne, (int64_t)p.N * p.Hv * Dv, p.dev_status))
+                                        for (int e = 0; e < ne; ++e) obase[(i0 / 8) * ostride8 + e] = ve[e];
+                                }
                             }
                         }
                         tc_fence_before();
@@ -1371,17 +1495,32 @@ __global__ void __launch_bounds__(NTHREADS, 1) gdn_prefill_chunk_kernel(const __
         batch0 += wcover;
     }
 
-    // teardown: drain outstanding TMA stages on abort, then free TMEM
-    if (cx.aborted() && warp == TMA_WARP && lane < 2) {
-        // each producer lane waits for the copies it issued
-        for (int s = 0; s < KQ_STAGES; ++s) {
+    // teardown after an abort: every role has left its loop (each wait ends on the abort flag
+    // or its own bound, each group leaves through its vote) and met the barrier above.  Copies
+    // and MMAs still in flight land before the shared memory and TMEM go away: each TMA lane
+    // waits for the last copy of every stage it filled, each UMMA issuer commits once more and
+    // waits for that commit (it arrives when all of the thread's earlier MMAs completed).  An
+    // operation on its way completes within microseconds, so these waits are short (2^24
+    // cycles, ~8 ms) rather than a second bound on bytes that may never come.
+    if (cx.aborted()) {
+        constexpr long long kDrain = 1ll << 24;
+        if (warp == TMA_WARP && lane < 2) {
+            for (int s = 0; s < KQ_STAGES; ++s) {
+                const long long t0 = clock64();
+                while (kq_use[s] > 0 && !mbar_try_wait(cx.bar(B_KQ_FULL + s), (kq_use[s] - 1) & 1))
+                    if (clock64() - t0 > kDrain) break;
+            }
             const long long t0 = clock64();
-            while (kq_use[s] > 0 && !mbar_try_wait(cx.bar(B_KQ_FULL + s), (kq_use[s] - 1) & 1))
-                if (clock64() - t0 > (1ll << 31)) break;
+            while (v_use > 0 && !mbar_try_wait(cx.bar(B_V_FULL), (v_use - 1) & 1))
+                if (clock64() - t0 > kDrain) break;
         }
-        const long long t0 = clock64();
-        while (v_use > 0 && !mbar_try_wait(cx.bar(B_V_FULL), (v_use - 1) & 1))
-            if (clock64() - t0 > (1ll << 31)) break;
+        if ((warp == MMA_WARP || warp == ISSUE_WARP) && lane == 0) {
+            const uint32_t db = cx.bar(warp == MMA_WARP ? B_DRAIN_CHAIN : B_DRAIN_PREP);
+            umma_commit(db);
+            const long long t0 = clock64();
+            while (!mbar_try_wait(db, 0))
+                if (clock64() - t0 > kDrain) break;
+        }
     }
     tc_fence_before();
     __syncthreads();
@@ -1447,11 +1586,18 @@ int num_sms()
 
 }  // namespace
 
+// Head sizes up to 128 of bf16 or fp16 run on the tensor cores.  Rows the tensor maps can
+// describe (Dk, Dv multiples of 8, Hv % 4 == 0) are loaded by the TMA; any other size is
+// staged with plain loads into the same zero-padded tiles.
 bool prefill_chunked_supported(const GdnPrefillArgs &a)
 {
-    return (a.dtype == GDN_BF16 || a.dtype == GDN_F16) && a.Dk >= 8 && a.Dk <= 128 &&
-           a.Dk % 8 == 0 && a.Dv >= 8 &&
-           a.Dv <= 128 && a.Dv % 8 == 0 && (a.Hv % 4) == 0 && get_encode() != nullptr;
+    return (a.dtype == GDN_BF16 || a.dtype == GDN_F16) && a.Dk >= 1 && a.Dk <= 128 &&
+           a.Dv >= 1 && a.Dv <= 128 && get_encode() != nullptr;
+}
+
+static bool prefill_needs_plain_staging(const GdnPrefillArgs &a)
+{
+    return a.Dk % 8 != 0 || a.Dv % 8 != 0 || a.Hv % 4 != 0;
 }
 
 cudaError_t launch_prefill_chunked(const GdnPrefillArgs &a, cudaStream_t stream)
@@ -1475,8 +1621,9 @@ cudaError_t launch_prefill_chunked(const GdnPrefillArgs &a, cudaStream_t stream)
     Params p;
     memset(&p, 0, sizeof(p));
     const uint64_t N = (uint64_t)(a.N > 0 ? a.N : 1);
+    const bool plain = prefill_needs_plain_staging(a);
     // TMA maps need a valid base even when N == 0 (no chunk is loaded then)
-    if (a.N > 0) {
+    if (a.N > 0 && !plain) {
         // head dims below 128 read zeros past their end (TMA fill), so every tile is a
         // zero-padded 128-wide tile and the products are unchanged
         const bool f16 = a.dtype == GDN_F16;
@@ -1505,10 +1652,16 @@ cudaError_t launch_prefill_chunked(const GdnPrefillArgs &a, cudaStream_t stream)
     p.Dv = a.Dv;
     p.a_log = a.a_log;
     p.dt_bias = a.dt_bias;
+    p.stage_plain = plain ? 1 : 0;
+    p.q = static_cast<const uint16_t *>(a.q);
+    p.k = static_cast<const uint16_t *>(a.k);
+    p.v = static_cast<const uint16_t *>(a.v);
+    p.g = a.g;
+    p.beta = a.beta;
     const int units = a.B * a.Hv;
     const int grid = units < num_sms() ? units : num_sms();
     const bool general = !a.has_decay || !a.has_retrieval || a.beta_sigmoid || a.a_log != nullptr ||
-                         a.Dk != D || a.Dv != D;
+                         a.Dk != D || a.Dv != D || plain;
     // fp16 activations run the general instantiation with fp16 operand tiles
     if (a.dtype == GDN_F16)
         gdn_prefill_chunk_kernel<true, true><<<grid, NTHREADS, SMEM_BYTES, stream>>>(p);

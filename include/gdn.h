@@ -82,9 +82,10 @@ enum {
      * data-dependent shared-memory access is tested against its buffer first; one outside it
      * is skipped (a load reads zero) and this bit is set.  Ordinary builds never set it. */
     GDN_DEV_BOUNDS = 8,
-    /* Checked builds only, set by the CALLER in *dev_status before a gdn_decode call: the
-     * persistent decode kernel posts 16 bytes more than its first copy delivers, so that
-     * wait runs out after its bound (about a second), GDN_DEV_TIMEOUT is set and the kernel
+    /* Checked builds only, set by the CALLER in *dev_status before a gdn_decode or a
+     * chunked gdn_prefill call: the persistent decode kernel, or the chunked prefill
+     * kernel's first q/k stage, posts 16 bytes more than its copies deliver, so the waits on
+     * it run out after their bound (about a second), GDN_DEV_TIMEOUT is set and the kernel
      * returns.  Exercises the timeout path without a fault; ignored by ordinary builds. */
     GDN_DEV_TEST_STALL = 1 << 30
 };
@@ -137,11 +138,12 @@ enum {
  * and beta through tensor maps, whose base must be 16-byte aligned; the rule
  * holds for every call, so a view such as g[1:] of a 4-byte aligned buffer is
  * GDN_ERR_ALIGN, not a launch failure); out must not overlap any input.
- * bf16 or fp16 with Dk, Dv in {8, 16, ..., 128} and Hv % 4 == 0 runs the
- * chunked tensor-core kernel (unless GDN_PREFILL_SEQUENTIAL; its operand tiles
- * take the activations' type, fp32 accumulation and state); everything else
- * (fp32, heads wider than 128 or not a multiple of 8) runs the per-token
- * kernel, which computes in fp32.  The chunked kernel floors each g at -30
+ * bf16 or fp16 with Dk, Dv <= 128 runs the chunked tensor-core kernel (unless
+ * GDN_PREFILL_SEQUENTIAL; its operand tiles take the activations' type, fp32
+ * accumulation and state; rows that a tensor map cannot describe -- Dk or Dv
+ * not a multiple of 8, or Hv % 4 != 0 -- are copied into its zero-padded tiles
+ * with plain loads); everything else (fp32, heads wider than 128) runs the
+ * per-token kernel, which computes in fp32.  The chunked kernel floors each g at -30
  * (exp(-30) ~ 9e-14) so that in-chunk decay differences stay finite.
  * Overlapping request ranges are not supported (their outputs are undefined).
  */
@@ -250,8 +252,8 @@ GDN_API gdn_status gdn_conv1d(const void *x, const void *weight, void *conv_stat
 
 /* 1 when gdn_prefill with these arguments runs the chunked tensor-core
  * kernel, 0 when it runs the per-token kernel (host-only query, no launch).
- * The chunked kernel takes bf16 or fp16 with Dk and Dv multiples of 8 up to 128 (smaller heads
- * run as zero-padded 128-wide tiles) and Hv % 4 == 0. */
+ * The chunked kernel takes bf16 or fp16 with Dk, Dv up to 128 (smaller heads run as
+ * zero-padded 128-wide tiles) and any Hv. */
 GDN_API int32_t gdn_prefill_uses_chunked(gdn_dtype dtype, int32_t Hv, int32_t Dk, int32_t Dv,
                                          uint32_t flags);
 

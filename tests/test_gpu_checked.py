@@ -6,8 +6,11 @@ reach every kernel and launch form.
 * The checks change no arithmetic: outputs, final states and pools equal the product
   library's bit for bit.
 * The persistent decode kernel's bounded wait, made to run out on request
-  (GDN_DEV_TEST_STALL), ends with GDN_DEV_TIMEOUT after about two seconds, and the next call
+  (GDN_DEV_TEST_STALL), ends with GDN_DEV_TIMEOUT after about a second, and the next call
   on the same context is correct.
+* The chunked prefill kernel's abort path, forced the same way (its first q/k stage expects
+  16 bytes more than arrive), ends every role through its waits' bounds, the abort flag and
+  the per-chunk votes: GDN_DEV_TIMEOUT, a return within seconds, and a correct next call.
 """
 import copy
 import time
@@ -73,6 +76,7 @@ def prefill_fn(gdn, c):
     ("chunked default", [70, 1, 130, 0, 64], 2, 4, 128, 128, torch.bfloat16),
     ("chunked head sizes", [33, 100], 2, 4, 64, 40, torch.bfloat16),
     ("chunked fp16", [90, 5], 2, 4, 128, 128, torch.float16),
+    ("chunked plain-staged odd heads", [33, 70, 0, 5], 1, 2, 12, 9, torch.bfloat16),
     ("per-token fp32", [20, 7], 1, 2, 12, 9, torch.float32),
 ])
 def test_prefill_in_bounds(gdn, W, name, lengths, Hq, Hv, Dk, Dv, dtype):
@@ -82,6 +86,36 @@ def test_prefill_in_bounds(gdn, W, name, lengths, Hq, Hv, Dk, Dv, dtype):
     assert chunked == name.startswith("chunked")
     r0, r1, st = both(gdn, prefill_fn(gdn, c))
     assert st == 0
+    assert_same(r0, r1)
+
+
+def test_chunked_prefill_wait_runs_out_on_request(gdn, W):
+    """GDN_DEV_TEST_STALL in the status word makes the chunked kernel's first q/k stage expect
+    16 bytes more than its copies deliver (one request of one chunk, four value heads: four
+    CTAs).  The prep front's wait on that stage runs out; the UMMA issuers, the prep back and
+    the state warpgroup end their waits on the abort flag; every group leaves through its
+    per-chunk vote; the teardown drains and frees TMEM.  GDN_DEV_TIMEOUT is reported, no
+    bounds bit, the call returns within seconds, and a normal call on the same context then
+    matches the product library bit for bit."""
+    c = W.make_prefill(77, [40], 1, 4, 128, 128, init_std=0.05, qk_l2norm=True)
+    assert gdn.prefill_uses_chunked(c.q.dtype, 4, 128, 128)
+    product = gdn._binding.LIB_PATH
+    gdn.use_library(gdn.CHECKED_LIB_PATH)
+    try:
+        st = torch.full((1,), gdn.GDN_DEV_TEST_STALL, dtype=torch.int32, device="cuda")
+        t0 = time.time()
+        prefill_fn(gdn, c)(st)
+        took = time.time() - t0
+        s = int(st.item())
+        assert s & gdn.GDN_DEV_TIMEOUT
+        assert not s & gdn.GDN_DEV_BOUNDS
+        assert took < 60
+        st2 = torch.zeros(1, dtype=torch.int32, device="cuda")
+        r1 = prefill_fn(gdn, c)(st2)
+        assert int(st2.item()) == 0
+    finally:
+        gdn.use_library(product)
+    r0 = prefill_fn(gdn, c)(None)
     assert_same(r0, r1)
 
 

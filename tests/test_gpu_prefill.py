@@ -62,7 +62,10 @@ def test_tiny_oracle_case_fp32(gdn, W, oracle_mod):
 
 @pytest.mark.parametrize("dtype,tol", [(torch.float32, TOL_F32), (torch.bfloat16, TOL_BF16)])
 def test_odd_head_sizes_gqa(gdn, W, oracle_mod, dtype, tol):
-    """The op page's example call shape: T=4, Hq=1, Hv=2, Dk=12, Dv=9, with an initial state."""
+    """The op page's example call shape: T=4, Hq=1, Hv=2, Dk=12, Dv=9, with an initial state;
+    bf16 runs it on the tensor cores (plain-staged zero-padded tiles), fp32 on the per-token
+    kernel."""
+    assert gdn.prefill_uses_chunked(dtype, 2, 12, 9) == (dtype == torch.bfloat16)
     c = W.make_prefill(11, [4], 1, 2, 12, 9, dtype=dtype, uniform=True, init_std=0.5,
                        qk_l2norm=True)
     out, fs = run_gpu_prefill(c)
@@ -179,12 +182,39 @@ def test_chunked_path_is_selected(gdn):
     assert gdn.prefill_uses_chunked(torch.bfloat16, 32, 128, 128)
     assert not gdn.prefill_uses_chunked(torch.bfloat16, 32, 128, 128, sequential=True)
     assert not gdn.prefill_uses_chunked(torch.float32, 32, 128, 128)
-    assert not gdn.prefill_uses_chunked(torch.bfloat16, 2, 128, 128)
+    assert gdn.prefill_uses_chunked(torch.bfloat16, 2, 128, 128)       # plain-staged gates
     assert gdn.prefill_uses_chunked(torch.bfloat16, 32, 64, 128)
     assert gdn.prefill_uses_chunked(torch.bfloat16, 32, 8, 8)
-    assert not gdn.prefill_uses_chunked(torch.bfloat16, 32, 60, 128)   # not a multiple of 8
+    assert gdn.prefill_uses_chunked(torch.bfloat16, 32, 60, 128)       # plain-staged rows
+    assert gdn.prefill_uses_chunked(torch.bfloat16, 2, 12, 9)          # the op page's example
+    assert gdn.prefill_uses_chunked(torch.float16, 3, 1, 1)
     assert not gdn.prefill_uses_chunked(torch.bfloat16, 32, 128, 136)  # wider than 128
     assert not gdn.prefill_uses_chunked(torch.bfloat16, 32, 256, 256)
+
+
+@pytest.mark.parametrize("Hq,Hv,Dk,Dv", [(1, 2, 12, 9), (1, 3, 1, 1), (2, 6, 33, 7),
+                                         (1, 2, 127, 100), (2, 4, 60, 128), (1, 1, 128, 128)])
+def test_chunked_plain_staged_shapes(gdn, W, oracle_mod, Hq, Hv, Dk, Dv):
+    """Head sizes that are not multiples of 8, and value-head counts that are not multiples of
+    4, on the tensor-core kernel: their rows are copied into the zero-padded tiles by plain
+    loads instead of tensor maps.  Ragged requests with an empty one, initial states, the
+    in-kernel norm, tokens no request covers; every output and final state against the oracle,
+    uncovered outputs untouched, no pipeline wait timed out."""
+    assert gdn.prefill_uses_chunked(torch.bfloat16, Hv, Dk, Dv)
+    c = W.make_prefill(700 + Dk + Dv + Hv, [70, 0, 1, 130, 64], Hq, Hv, Dk, Dv, init_std=0.1,
+                       qk_l2norm=True)
+    c.cu_seqlens = torch.tensor([0, 70, 70, 71, 201, c.N - 5], dtype=torch.int32)
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    keep = torch.full((c.N, Hv, Dv), 7.0, dtype=torch.bfloat16)
+    out, fs = gdn.gdn_prefill(dev(c.q), dev(c.k), dev(c.v), dev(c.g), dev(c.beta),
+                              dev(c.cu_seqlens), dev(c.initial_state), None, dev(keep),
+                              scale=c.scale, qk_l2norm=True, dev_status=status)
+    torch.cuda.synchronize()
+    assert int(status.item()) == 0
+    ro, rf = oracle_prefill_case(oracle_mod, c, out=f64(keep))
+    assert_prefill_parity(out, fs, ro, rf, request_ranges(c.cu_seqlens, c.B, c.N), TOL_BF16)
+    assert torch.equal(out[c.N - 5:].cpu(), keep[c.N - 5:])
+    assert torch.equal(fs[1].cpu(), c.initial_state[1])
 
 
 @pytest.mark.parametrize("Dk,Dv", [(64, 64), (128, 64), (64, 128), (96, 32), (8, 8), (120, 128)])
