@@ -57,8 +57,9 @@ GDN_DEV_INTERNAL = 4
 GDN_DEV_BOUNDS = 8            # checked builds only
 GDN_DEV_TEST_STALL = 1 << 30  # checked builds only, set by the caller (decode timeout path)
 
-EXPORTED = ("gdn_prefill", "gdn_decode", "gdn_conv1d", "gdn_status_string", "gdn_last_error",
-            "gdn_abi_version", "gdn_prefill_uses_chunked")
+EXPORTED = ("gdn_prefill", "gdn_prefill_ws", "gdn_prefill_workspace_size", "gdn_decode",
+            "gdn_conv1d", "gdn_status_string", "gdn_last_error", "gdn_abi_version",
+            "gdn_prefill_uses_chunked")
 
 _lib = None
 
@@ -98,6 +99,12 @@ def lib():
         L.gdn_prefill.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp,
                                   i32, i64, i32, i32, i32, i32, ctypes.c_int, f32, i32, u32,
                                   vp, vp]
+        L.gdn_prefill_ws.restype = ctypes.c_int
+        L.gdn_prefill_ws.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp,
+                                     i32, i64, i32, i32, i32, i32, ctypes.c_int, f32, i32, u32,
+                                     vp, ctypes.c_uint64, vp, vp]
+        L.gdn_prefill_workspace_size.restype = ctypes.c_uint64
+        L.gdn_prefill_workspace_size.argtypes = [i32, i64, i32, i32, i32, i32, ctypes.c_int, u32]
         L.gdn_decode.restype = ctypes.c_int
         L.gdn_decode.argtypes = [vp, vp, vp, vp, i32, i64, i64, vp, vp, vp,
                                  vp, vp, vp, vp, f32, vp,
@@ -162,7 +169,7 @@ def gdn_prefill(q, k, v, g, beta, cu_seqlens=None, initial_state=None, final_sta
                 out=None, *, num_requests: Optional[int] = None, scale: Optional[float] = None,
                 qk_l2norm: bool = False, sequential: bool = False, update_rule: str = "gated_delta",
                 gate_activation: str = "none", a_log=None, dt_bias=None,
-                beta_activation: str = "none", dev_status=None, stream=None):
+                beta_activation: str = "none", split: bool = True, dev_status=None, stream=None):
     """Gated DeltaNet prefill (log-space form) over ragged requests.
 
     q, k: [N, Hq, Dk] or [B, S, Hq, Dk]; v: [N, Hv, Dv] (same leading axes);
@@ -171,7 +178,10 @@ def gdn_prefill(q, k, v, g, beta, cu_seqlens=None, initial_state=None, final_sta
     int32 (rank-3 form) or None; initial_state: [B, Hv, Dv, Dk] fp32 or None.
     update_rule: gated_delta | gated | delta | linear; gate_activation: none |
     qwen (a_log, dt_bias: [Hv] fp32); beta_activation: none | sigmoid.
-    ``scale`` None or 0 selects 1/sqrt(Dk).  Returns (out, final_state).
+    ``scale`` None or 0 selects 1/sqrt(Dk).  With ``split`` (the default) a call that
+    gdn_prefill_workspace_size says can cut long requests into parallel segments gets a
+    workspace from torch's allocator and runs through gdn_prefill_ws; ``split=False`` always
+    calls gdn_prefill.  Returns (out, final_state).
     """
     if update_rule not in UPDATE_RULES:
         raise ValueError(f"unknown update_rule {update_rule!r}")
@@ -236,11 +246,23 @@ def gdn_prefill(q, k, v, g, beta, cu_seqlens=None, initial_state=None, final_sta
         scale = 1.0 / math.sqrt(Dk)
     flags = (GDN_PREFILL_SEQUENTIAL if sequential else 0) | rule_flags
     flags |= (GDN_GATE_QWEN if qwen else 0) | (GDN_BETA_SIGMOID if beta_activation == "sigmoid" else 0)
-    st = lib().gdn_prefill(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(a_log),
-                           _ptr(dt_bias), _ptr(cu_seqlens),
-                           _ptr(initial_state), _ptr(final_state), _ptr(out), B, N, Hq, Hv, Dk,
-                           Dv, dt, float(scale), int(bool(qk_l2norm)), flags, _ptr(dev_status),
-                           _stream(stream))
+    ws_bytes = int(lib().gdn_prefill_workspace_size(B, N, Hq, Hv, Dk, Dv, dt, flags)) \
+        if split else 0
+    if ws_bytes > 0:
+        ws = torch.empty(ws_bytes, dtype=torch.uint8, device=q.device)
+        if stream is not None:
+            ws.record_stream(stream)   # released to the allocator only after the call
+        st = lib().gdn_prefill_ws(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(a_log),
+                                  _ptr(dt_bias), _ptr(cu_seqlens), _ptr(initial_state),
+                                  _ptr(final_state), _ptr(out), B, N, Hq, Hv, Dk, Dv, dt,
+                                  float(scale), int(bool(qk_l2norm)), flags, _ptr(ws), ws_bytes,
+                                  _ptr(dev_status), _stream(stream))
+    else:
+        st = lib().gdn_prefill(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(a_log),
+                               _ptr(dt_bias), _ptr(cu_seqlens),
+                               _ptr(initial_state), _ptr(final_state), _ptr(out), B, N, Hq, Hv,
+                               Dk, Dv, dt, float(scale), int(bool(qk_l2norm)), flags,
+                               _ptr(dev_status), _stream(stream))
     if st != GDN_OK:
         raise GdnError(st, "gdn_prefill")
     return out, final_state

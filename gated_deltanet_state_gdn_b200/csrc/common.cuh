@@ -140,6 +140,9 @@ struct GdnPrefillArgs {
     int32_t has_decay, has_retrieval;
     const float *a_log, *dt_bias;   // non-NULL: qwen gate on g
     int32_t beta_sigmoid;
+    // caller-owned device workspace for the sequence-parallel split (NULL: no split)
+    void *workspace;
+    uint64_t workspace_bytes;
 };
 
 struct GdnDecodeArgs {
@@ -199,3 +202,6 @@ cudaError_t launch_conv1d(const GdnConv1dArgs &a, cudaStream_t stream);
 cudaError_t launch_prefill_sequential(const GdnPrefillArgs &a, cudaStream_t stream);
 cudaError_t launch_prefill_chunked(const GdnPrefillArgs &a, cudaStream_t stream);
 bool prefill_chunked_supported(const GdnPrefillArgs &a);
+// bytes of workspace with which gdn_prefill may split long requests (0: never splits)
+uint64_t prefill_split_workspace_bytes(const GdnPrefillArgs &a);
+cudaError_t launch_seq_compose(const GdnPrefillArgs &a, void *workspace, int G, cudaStream_t stream);

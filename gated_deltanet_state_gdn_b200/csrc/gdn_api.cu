@@ -63,12 +63,31 @@ int32_t gdn_prefill_uses_chunked(gdn_dtype dtype, int32_t Hv, int32_t Dk, int32_
     return prefill_chunked_supported(a) ? 1 : 0;
 }
 
-gdn_status gdn_prefill(const void *q, const void *k, const void *v, const float *g,
-                       const float *beta, const float *a_log, const float *dt_bias,
-                       const int32_t *cu_seqlens, const float *initial_state,
-                       float *final_state, void *out, int32_t B, int64_t N, int32_t Hq,
-                       int32_t Hv, int32_t Dk, int32_t Dv, gdn_dtype dtype, float scale,
-                       int32_t qk_l2norm, uint32_t flags, int32_t *dev_status, void *stream)
+}  // extern "C"
+
+namespace {
+
+// scalar part of the prefill arguments (enough for host-only queries)
+GdnPrefillArgs prefill_shape(int32_t B, int64_t N, int32_t Hq, int32_t Hv, int32_t Dk, int32_t Dv,
+                             gdn_dtype dtype, uint32_t flags)
+{
+    GdnPrefillArgs a;
+    memset(&a, 0, sizeof(a));
+    const uint32_t rule = flags & GDN_RULE_MASK;
+    a.B = B; a.N = N; a.Hq = Hq; a.Hv = Hv; a.Dk = Dk; a.Dv = Dv; a.dtype = dtype;
+    a.has_decay = rule == 0 || rule == GDN_RULE_GATED;
+    a.has_retrieval = rule == 0 || rule == GDN_RULE_DELTA;
+    a.beta_sigmoid = (flags & GDN_BETA_SIGMOID) ? 1 : 0;
+    return a;
+}
+
+gdn_status prefill_impl(const void *q, const void *k, const void *v, const float *g,
+                        const float *beta, const float *a_log, const float *dt_bias,
+                        const int32_t *cu_seqlens, const float *initial_state,
+                        float *final_state, void *out, int32_t B, int64_t N, int32_t Hq,
+                        int32_t Hv, int32_t Dk, int32_t Dv, gdn_dtype dtype, float scale,
+                        int32_t qk_l2norm, uint32_t flags, void *workspace,
+                        uint64_t workspace_bytes, int32_t *dev_status, void *stream)
 {
     if (dtype != GDN_F32 && dtype != GDN_BF16 && dtype != GDN_F16) return GDN_ERR_DTYPE;
     if (B < 0 || N < 0 || Hq < 1 || Hv < 1 || Dk < 1 || Dv < 1) return GDN_ERR_SHAPE;
@@ -125,6 +144,28 @@ gdn_status gdn_prefill(const void *q, const void *k, const void *v, const float 
     a.scale = scale; a.qk_l2norm = qk_l2norm ? 1 : 0; a.dev_status = dev_status;
     a.has_decay = has_decay; a.has_retrieval = has_retrieval;
     a.a_log = a_log; a.dt_bias = dt_bias; a.beta_sigmoid = (flags & GDN_BETA_SIGMOID) ? 1 : 0;
+    a.workspace = nullptr;
+    a.workspace_bytes = 0;
+
+    // workspace of the sequence-parallel split: used only when the call can split and the
+    // chunked kernel runs; then it must be large enough, aligned, and overlap nothing
+    if (workspace && !(flags & GDN_PREFILL_SEQUENTIAL) && prefill_chunked_supported(a)) {
+        const uint64_t need = prefill_split_workspace_bytes(a);
+        if (need > 0) {
+            if (workspace_bytes < need) return GDN_ERR_SHAPE;
+            if (!aligned(workspace, 16)) return GDN_ERR_ALIGN;
+            const size_t wb = (size_t)need;
+            if (overlaps(workspace, wb, q, qk_bytes) || overlaps(workspace, wb, k, qk_bytes) ||
+                overlaps(workspace, wb, v, v_bytes) || overlaps(workspace, wb, g, gb_bytes) ||
+                overlaps(workspace, wb, beta, gb_bytes) || overlaps(workspace, wb, out, v_bytes) ||
+                overlaps(workspace, wb, initial_state, st_bytes) ||
+                overlaps(workspace, wb, final_state, st_bytes) ||
+                overlaps(workspace, wb, cu_seqlens, (size_t)(B + 1) * 4))
+                return GDN_ERR_ALIAS;
+            a.workspace = workspace;
+            a.workspace_bytes = workspace_bytes;
+        }
+    }
 
     cudaStream_t s = (cudaStream_t)stream;
     cudaError_t e;
@@ -134,6 +175,45 @@ gdn_status gdn_prefill(const void *q, const void *k, const void *v, const float 
         e = launch_prefill_sequential(a, s);
     if (e != cudaSuccess) return cuda_fail(e, "gdn_prefill launch");
     return GDN_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+gdn_status gdn_prefill(const void *q, const void *k, const void *v, const float *g,
+                       const float *beta, const float *a_log, const float *dt_bias,
+                       const int32_t *cu_seqlens, const float *initial_state,
+                       float *final_state, void *out, int32_t B, int64_t N, int32_t Hq,
+                       int32_t Hv, int32_t Dk, int32_t Dv, gdn_dtype dtype, float scale,
+                       int32_t qk_l2norm, uint32_t flags, int32_t *dev_status, void *stream)
+{
+    return prefill_impl(q, k, v, g, beta, a_log, dt_bias, cu_seqlens, initial_state, final_state,
+                        out, B, N, Hq, Hv, Dk, Dv, dtype, scale, qk_l2norm, flags, nullptr, 0,
+                        dev_status, stream);
+}
+
+gdn_status gdn_prefill_ws(const void *q, const void *k, const void *v, const float *g,
+                          const float *beta, const float *a_log, const float *dt_bias,
+                          const int32_t *cu_seqlens, const float *initial_state,
+                          float *final_state, void *out, int32_t B, int64_t N, int32_t Hq,
+                          int32_t Hv, int32_t Dk, int32_t Dv, gdn_dtype dtype, float scale,
+                          int32_t qk_l2norm, uint32_t flags, void *workspace,
+                          uint64_t workspace_bytes, int32_t *dev_status, void *stream)
+{
+    return prefill_impl(q, k, v, g, beta, a_log, dt_bias, cu_seqlens, initial_state, final_state,
+                        out, B, N, Hq, Hv, Dk, Dv, dtype, scale, qk_l2norm, flags, workspace,
+                        workspace_bytes, dev_status, stream);
+}
+
+uint64_t gdn_prefill_workspace_size(int32_t B, int64_t N, int32_t Hq, int32_t Hv, int32_t Dk,
+                                    int32_t Dv, gdn_dtype dtype, uint32_t flags)
+{
+    if ((flags & GDN_PREFILL_SEQUENTIAL) || B < 1 || Hq < 1 || Hv < 1 || Hv % Hq != 0 || N < 0)
+        return 0;
+    const GdnPrefillArgs a = prefill_shape(B, N, Hq, Hv, Dk, Dv, dtype, flags);
+    if ((flags & GDN_GATE_QWEN) || !prefill_chunked_supported(a)) return 0;
+    return prefill_split_workspace_bytes(a);
 }
 
 gdn_status gdn_decode(const void *q, const void *k, const void *v, float *state_pool,

@@ -72,6 +72,7 @@
 #include <cuda_fp16.h>
 
 #include "common.cuh"
+#include "seqpar.cuh"
 #include "sm100.cuh"
 
 using namespace sm100;
@@ -172,6 +173,9 @@ struct __align__(64) Params {
     int32_t stage_plain;
     const uint16_t *q, *k, *v;
     const float *g, *beta;
+    // sequence-parallel split (seqpar.cuh): pass 1 or 3, the split rule's CTA count, workspace
+    int32_t seq_pass, seq_G;
+    float *seq_ws;
 };
 
 // --------------------------------------------------------------------------
@@ -293,8 +297,9 @@ __device__ __forceinline__ void st4(float *p, float a, float b, float c, float d
 // its bf16 copy
 // into the (1a)/(1b) A-operand columns and gC * S0 into the fp32 state columns.  Runs once per
 // unit, out of line so that the per-chunk code stays compact.
-template <bool GENERAL, bool F16>
-__device__ __noinline__ void load_state_tmem(const float *init, int Dk, uint32_t tl, float gC)
+template <bool GENERAL, bool F16, bool IDENT = false>
+__device__ __noinline__ void load_state_tmem(const float *init, int Dk, uint32_t tl, float gC,
+                                             int ident = -1)
 {
 #pragma unroll 1
     for (int hq = 0; hq < 2; ++hq) {
@@ -310,6 +315,11 @@ __device__ __noinline__ void load_state_tmem(const float *init, int Dk, uint32_t
             // rows of Dk floats with Dk % 4 != 0 are only 4-byte aligned
 #pragma unroll
             for (int c = 0; c < 64; ++c) x[c] = init && 64 * hq + c < Dk ? init[64 * hq + c] : 0.f;
+        }
+        // the identity's row `ident` (sequence-parallel transition runs; init is NULL then)
+        if (IDENT && ident >= 0) {
+#pragma unroll
+            for (int c = 0; c < 64; ++c) x[c] = 64 * hq + c == ident ? 1.f : x[c];
         }
 #pragma unroll
         for (int q = 0; q < 4; ++q) {
@@ -332,6 +342,65 @@ __device__ __noinline__ void load_state_tmem(const float *init, int Dk, uint32_t
 __device__ __forceinline__ bool greedy_schedule(const Params &p, int G)
 {
     return p.B <= 32 && G <= 256 && p.B * ((p.Hv + G - 1) / G) <= MAX_UNITS;
+}
+
+// Units of a sequence-parallel pass (seqpar.cuh), one per CTA at most: every request in
+// index order, its pseudo-requests in a fixed order, Hv heads each; CTA c takes unit c.  The
+// unit's b field carries the request in bits 0-7, the segment in bits 8-11, the mode in bits
+// 12-14 and whether the request is split in bit 15.
+__device__ __noinline__ void build_seq_unit(const Params &p, uint8_t *smem, int *count_out)
+{
+    if (threadIdx.x == 0) {
+        int rs[gdn_seq::MAX_REQ], rl[gdn_seq::MAX_REQ], nc[gdn_seq::MAX_REQ];
+        for (int b = 0; b < p.B; ++b) {
+            int64_t st, en;
+            if (p.cu_seqlens) {
+                st = clampi(p.cu_seqlens[b], 0, p.N);
+                en = clampi(p.cu_seqlens[b + 1], 0, p.N);
+            } else {
+                const int64_t S = p.N / p.B;
+                st = (int64_t)b * S;
+                en = st + S;
+            }
+            rs[b] = (int)st;
+            rl[b] = en > st ? (int)(en - st) : 0;
+            nc[b] = (rl[b] + C - 1) / C;
+        }
+        const uint32_t mask = gdn_seq::split_mask(nc, p.B, p.Hv, p.seq_G);
+        int4 *list = reinterpret_cast<int4 *>(smem + OFF_UNITS);
+        int idx = 0, found = 0;
+        for (int b = 0; b < p.B && !found; ++b) {
+            const bool split = (mask >> b) & 1u;
+            int s0 = 0, s1 = 0, s2 = 0;
+            if (split) gdn_seq::segments(nc[b], s0, s1, s2);
+            // pseudo-requests of this pass: (mode, segment, first token, tokens)
+            int4 ps[3];
+            int nps = 0;
+            if (p.seq_pass == 1) {
+                if (split) {
+                    ps[nps++] = make_int4(gdn_seq::MODE_TRUE, 0, rs[b], s0 * C);
+                    ps[nps++] = make_int4(gdn_seq::MODE_IDENT, 1, rs[b] + s0 * C, s1 * C);
+                    ps[nps++] = make_int4(gdn_seq::MODE_ZERO, 1, rs[b] + s0 * C, s1 * C);
+                } else {
+                    ps[nps++] = make_int4(gdn_seq::MODE_TRUE, 0, rs[b], rl[b]);
+                }
+            } else if (split) {
+                ps[nps++] = make_int4(gdn_seq::MODE_TRUE, 1, rs[b] + s0 * C, s1 * C);
+                ps[nps++] = make_int4(gdn_seq::MODE_TRUE, 2, rs[b] + (s0 + s1) * C, rl[b] - (s0 + s1) * C);
+            }
+            for (int i = 0; i < nps && !found; ++i) {
+                if ((int)blockIdx.x < idx + p.Hv) {
+                    const int h = blockIdx.x - idx;
+                    list[0] = make_int4(b | (ps[i].y << 8) | (ps[i].x << 12) | ((split ? 1 : 0) << 15), h,
+                                        ps[i].z, ps[i].w);
+                    found = 1;
+                }
+                idx += p.Hv;
+            }
+        }
+        *count_out = found;
+    }
+    __syncthreads();
 }
 
 __device__ __noinline__ void build_unit_list(const Params &p, uint8_t *smem, int batch0,
@@ -660,12 +729,47 @@ __device__ __noinline__ void stage_plain_v(const Params &p, uint8_t *vt, int h, 
     }
 }
 
+// Start state, final-state destination and outputs of a unit of a split pass (seqpar.cuh):
+// segment 0 runs from the true initial state, its final state the start of segment 1;
+// segment 1 runs from the identity (final state A1^T) and from zero (B1^T), without outputs;
+// in pass 3 segments 1 and 2 run from their composed start states, segment 2's final state the
+// request's.  `bfield` is the unit's b field (request, segment, mode, split bit).
+__device__ __noinline__ void seq_unit_io(const Params &p, int bfield, int h, int dv, const float *&init,
+                                         float *&fin, int &ident, bool &outputs_on)
+{
+    const gdn_seq::Workspace ws{p.seq_ws, p.B, p.Hv, D, D};
+    const int ub = bfield & 255, useg = (bfield >> 8) & 15, umode = (bfield >> 12) & 7;
+    const bool usplit = (bfield >> 15) & 1;
+    const int64_t ro = (int64_t)dv * D;
+    if (umode == gdn_seq::MODE_IDENT) {
+        init = nullptr;
+        ident = dv;
+        fin = ws.A1(ub, h) + ro;
+        outputs_on = false;
+    } else if (umode == gdn_seq::MODE_ZERO) {
+        init = nullptr;
+        fin = ws.B1(ub, h) + ro;
+        outputs_on = false;
+    } else if (useg == 1) {
+        init = ws.S1(ub, h) + ro;
+        fin = nullptr;
+    } else if (useg == 2) {
+        init = ws.S2(ub, h) + ro;
+    } else if (usplit) {
+        fin = ws.S1(ub, h) + ro;
+    }
+}
+
 // ========================================================================== kernel
 // GENERAL = false: the default rule (gated_delta, no gate or beta activation), with the
 // variant switches folded at compile time; GENERAL = true reads them from p.
-template <bool GENERAL, bool F16>
+// SEQ = true: a pass of the sequence-parallel split (default rule, bf16, 128-wide heads), one
+// unit per CTA, whose mode picks its start state, where its final state goes and whether it
+// writes outputs (seqpar.cuh).
+template <bool GENERAL, bool F16, bool SEQ = false>
 __global__ void __launch_bounds__(NTHREADS, 1) gdn_prefill_chunk_kernel(const __grid_constant__ Params p)
 {
+    static_assert(!SEQ || (!GENERAL && !F16), "the split runs the default bf16 instantiation");
     const bool has_decay = GENERAL ? p.has_decay != 0 : true;
     const bool has_retrieval = GENERAL ? p.has_retrieval != 0 : true;
     const bool beta_sigmoid = GENERAL ? p.beta_sigmoid != 0 : false;
@@ -736,14 +840,17 @@ __global__ void __launch_bounds__(NTHREADS, 1) gdn_prefill_chunk_kernel(const __
 
     const int G = gridDim.x;
     const int U = p.B * p.Hv;
-    const int waves = (U + G - 1) / G;
+    const int waves = SEQ ? 1 : (U + G - 1) / G;
 
     for (int batch0 = 0; batch0 < waves;) {
-        build_unit_list(p, smem, batch0, count_slot);
+        if constexpr (SEQ)
+            build_seq_unit(p, smem, count_slot);
+        else
+            build_unit_list(p, smem, batch0, count_slot);
         __syncthreads();
         const int nunits = *count_slot;
         int wcover = 0;
-        if (greedy_schedule(p, G)) {
+        if (SEQ || greedy_schedule(p, G)) {
             wcover = waves;   // one list holds every unit of this CTA
         } else {
             int cnt = 0;
@@ -838,10 +945,23 @@ __global__ void __launch_bounds__(NTHREADS, 1) gdn_prefill_chunk_kernel(const __
                 for (int k = 0; k < nunits && !cx.aborted(); ++k) {
                     const Unit un = load_unit(smem, k);
                     const int nc = (un.len + C - 1) / C;
+                    // a transition run from the identity takes v = 0: the tile is zeroed once
+                    // and every chunk's stage completes without a copy (SEQ passes hold one unit
+                    // per CTA, so nothing reloads the tile in between)
+                    const bool vzero = SEQ && ((un.b >> 12) & 7) == gdn_seq::MODE_IDENT;
                     for (int n = 0; n < nc; ++n) {
                         const int t0 = un.start + n * C;
                         if (v_use > 0 && !cx.wait(B_V_EMPTY, (v_use - 1) & 1)) break;
                         ++v_use;
+                        if (vzero) {
+                            if (n == 0) {
+                                for (int i = 0; i < 16384 / 16; ++i)
+                                    reinterpret_cast<uint4 *>(smem + OFF_V)[i] = make_uint4(0u, 0u, 0u, 0u);
+                                fence_proxy_async_smem();
+                            }
+                            mbar_arrive(cx.bar(B_V_FULL));
+                            continue;
+                        }
                         mbar_arrive_expect_tx(cx.bar(B_V_FULL), 16384);
                         tma_load_3d(sbase + OFF_V, &p.tm_v, cx.bar(B_V_FULL), 0, un.h, t0);
                         tma_load_3d(sbase + OFF_V + V_HALF, &p.tm_v, cx.bar(B_V_FULL), 64, un.h, t0);
@@ -1285,8 +1405,10 @@ __global__ void __launch_bounds__(NTHREADS, 1) gdn_prefill_chunk_kernel(const __
             for (int k = 0; k < nunits; ++k) {
                 const Unit un = load_unit(smem, k);
                 const int nc = (un.len + C - 1) / C;
+                // SEQ units carry their request, segment, mode and split bit in the b field
+                const int ub = SEQ ? (un.b & 255) : un.b;
                 // this lane's state row (dv < Dv; lanes past Dv carry zero rows)
-                const int64_t st_off = (((int64_t)un.b * p.Hv + un.h) * Dv + dv) * Dk;
+                const int64_t st_off = (((int64_t)ub * p.Hv + un.h) * Dv + dv) * Dk;
 #ifdef GDN_CHECKS
                 const int64_t st_n = (int64_t)p.B * p.Hv * Dv * Dk;
                 const bool row_ok = (!GENERAL || dv < Dv) && in_range(st_off, Dk, st_n, p.dev_status);
@@ -1295,6 +1417,9 @@ __global__ void __launch_bounds__(NTHREADS, 1) gdn_prefill_chunk_kernel(const __
 #endif
                 const float *init = p.initial_state && row_ok ? p.initial_state + st_off : nullptr;
                 float *fin = row_ok ? p.final_state + st_off : nullptr;
+                int ident = -1;            // start from the identity's row dv instead of init
+                bool outputs_on = true;
+                if constexpr (SEQ) seq_unit_io(p, un.b, un.h, dv, init, fin, ident, outputs_on);
                 if (nc == 0) {
                     if (row_ok && (!GENERAL || (Dk & 3) == 0)) {
                         for (int c = 0; c < Dk; c += 4) {
@@ -1314,7 +1439,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) gdn_prefill_chunk_kernel(const __
                     ok = cx.wait(B_GATE_FULL + gs, s_gate[gs] & 1);
                     ++s_gate[gs];
                     const float gC = reinterpret_cast<const float *>(smem + OFF_GATE + gs * GATE_BYTES)[GA_GC];
-                    load_state_tmem<GENERAL, F16>(init, Dk, tl, gC);
+                    load_state_tmem<GENERAL, F16, SEQ>(init, Dk, tl, gC, ident);
                     tmem_wait_st();
                     tc_fence_before();
                     ok = !named_sync_or(2, 128, !ok || cx.aborted());
@@ -1409,7 +1534,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) gdn_prefill_chunk_kernel(const __
                             for (int e = 0; e < 32; ++e) x[e] *= gC1;
                             tmem_st32(tl + TM_S + 32 * q, x);
                         } else {
-                            if (!GENERAL && (!kChecked || row_ok)) {
+                            if (!GENERAL && fin && (!kChecked || row_ok)) {
 #pragma unroll
                                 for (int c = 0; c < 32; c += 4) st4(fin + 32 * q + c, x[c], x[c + 1], x[c + 2], x[c + 3]);
                             } else if (row_ok && (Dk & 3) == 0) {
@@ -1464,7 +1589,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) gdn_prefill_chunk_kernel(const __
                                 __syncwarp();
                                 const int i0 = 16 * q + 8 * hb;   // first token of this group
                                 if (!GENERAL || (Dv & 7) == 0) {
-                                    if (i0 + tt < len_n && (!GENERAL || ocol < Dv) &&
+                                    if (outputs_on && i0 + tt < len_n && (!GENERAL || ocol < Dv) &&
                                         in_range(((int64_t)(un.start + n * C + tt + i0) * p.Hv + un.h) * Dv + ocol,
                                                  8, (int64_t)p.N * p.Hv * Dv, p.dev_status))
                                         *reinterpret_cast<uint4 *>(obase + (i0 / 8) * ostride8) = v;
@@ -1600,6 +1725,18 @@ static bool prefill_needs_plain_staging(const GdnPrefillArgs &a)
     return a.Dk % 8 != 0 || a.Dv % 8 != 0 || a.Hv % 4 != 0;
 }
 
+// The split (seqpar.cuh) runs the default bf16 instantiation on 128-wide heads, for calls with
+// few requests whose units fit one per SM; the device decides per request whether to split.
+uint64_t prefill_split_workspace_bytes(const GdnPrefillArgs &a)
+{
+    if (!prefill_chunked_supported(a) || prefill_needs_plain_staging(a)) return 0;
+    if (a.dtype != GDN_BF16 || a.Dk != 128 || a.Dv != 128) return 0;
+    if (!a.has_decay || !a.has_retrieval || a.beta_sigmoid || a.a_log) return 0;
+    if (a.B < 1 || a.B > gdn_seq::MAX_REQ || a.B * a.Hv > gdn_seq::MAX_UNITS_PER_CALL) return 0;
+    if (a.B * a.Hv > num_sms()) return 0;
+    return gdn_seq::workspace_bytes(a.B, a.Hv, a.Dk, a.Dv);
+}
+
 cudaError_t launch_prefill_chunked(const GdnPrefillArgs &a, cudaStream_t stream)
 {
     using namespace gdn_chunk;
@@ -1614,6 +1751,9 @@ cudaError_t launch_prefill_chunked(const GdnPrefillArgs &a, cudaStream_t stream)
                                      cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SMEM_BYTES);
         if (e == cudaSuccess)
             e = cudaFuncSetAttribute(gdn_prefill_chunk_kernel<true, true>,
+                                     cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SMEM_BYTES);
+        if (e == cudaSuccess)
+            e = cudaFuncSetAttribute(gdn_prefill_chunk_kernel<false, false, true>,
                                      cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SMEM_BYTES);
         return e;
     });
@@ -1659,7 +1799,26 @@ cudaError_t launch_prefill_chunked(const GdnPrefillArgs &a, cudaStream_t stream)
     p.g = a.g;
     p.beta = a.beta;
     const int units = a.B * a.Hv;
-    const int grid = units < num_sms() ? units : num_sms();
+    const int nsm = num_sms();
+    const int grid = units < nsm ? units : nsm;
+    const uint64_t ws_need = prefill_split_workspace_bytes(a);
+    if (ws_need > 0 && a.workspace && a.workspace_bytes >= ws_need) {
+        // pass 1, composition, pass 3 (seqpar.cuh); every launch sees the same CTA count, on
+        // which the split rule depends
+        // (grids: at most three units per (request, head) in pass 1 and two in pass 3)
+        p.seq_ws = static_cast<float *>(a.workspace);
+        p.seq_G = nsm;
+        p.seq_pass = 1;
+        const int g1 = 3 * units < nsm ? 3 * units : nsm, g3 = 2 * units < nsm ? 2 * units : nsm;
+        gdn_prefill_chunk_kernel<false, false, true><<<g1, NTHREADS, SMEM_BYTES, stream>>>(p);
+        cudaError_t e = cudaGetLastError();
+        if (e != cudaSuccess) return e;
+        e = launch_seq_compose(a, a.workspace, nsm, stream);
+        if (e != cudaSuccess) return e;
+        p.seq_pass = 3;
+        gdn_prefill_chunk_kernel<false, false, true><<<g3, NTHREADS, SMEM_BYTES, stream>>>(p);
+        return cudaGetLastError();
+    }
     const bool general = !a.has_decay || !a.has_retrieval || a.beta_sigmoid || a.a_log != nullptr ||
                          a.Dk != D || a.Dv != D || plain;
     // fp16 activations run the general instantiation with fp16 operand tiles

@@ -11,7 +11,9 @@
  * Conventions shared by every call
  *   - Every tensor argument is a DEVICE pointer owned by the caller.  The
  *     library allocates no device memory and keeps no pointer after the call
- *     returns (device-side it only holds read-only constant tables).
+ *     returns (device-side it only holds read-only constant tables).  Scratch
+ *     memory, where a call can use some (gdn_prefill_ws), is passed in by the
+ *     caller.
  *   - Calls are asynchronous on `stream` (a cudaStream_t; NULL means the
  *     legacy default stream).  The library never reads tensor contents on the
  *     host and never synchronises, so a call may be captured in a CUDA graph.
@@ -157,6 +159,58 @@ GDN_API gdn_status gdn_prefill(const void *q, const void *k, const void *v,
                        int32_t Dk, int32_t Dv, gdn_dtype dtype,
                        float scale, int32_t qk_l2norm, uint32_t flags,
                        int32_t *dev_status, void *stream);
+
+/*
+ * gdn_prefill_ws -- gdn_prefill with a caller-owned device workspace, which lets
+ * the call cut long requests into segments that run in parallel.
+ *
+ * Defined by the same operation as gdn_prefill ("com.microsoft.GatedDeltaNet",
+ * Description); the op's Attributes table states that how the sequence is cut
+ * into chunks does not change the result.  The recurrence is affine in the
+ * state: over a run of tokens S_end = A S_start + B.  When a call holds too few
+ * (request, value head) units to fill the GPU, a long request is cut into three
+ * segments of whole 64-token chunks: segment 0 runs from the true initial state;
+ * segment 1 runs twice in parallel with it, from the identity with v = 0 (giving
+ * A_1) and from zero (giving B_1); a small kernel composes the start state of
+ * segment 2; then segments 1 and 2 run from their true start states.  Results
+ * equal gdn_prefill's within the same tolerance (every product still goes
+ * through bf16 operands with fp32 state).
+ *
+ * Arguments: those of gdn_prefill, plus
+ *   workspace        device buffer of at least gdn_prefill_workspace_size(...)
+ *                    bytes, 16-byte aligned, overlapping no other argument; it
+ *                    holds per (request, value head) the start states of
+ *                    segments 1 and 2 and segment 1's A and B (fp32).  Owned
+ *                    by the caller, written and read by the call on `stream`
+ *                    (calls sharing one workspace must be ordered).  NULL: no
+ *                    split (exactly gdn_prefill).
+ *   workspace_bytes  its size.
+ * Whether a request is split is decided on the device from cu_seqlens (the host
+ * reads no tensor): a request of fewer than 24 chunks never is, nor any request
+ * of a call whose split would not shorten its longest chain.  The split applies
+ * to the default rule (gated_delta, no gate or beta activation), bf16,
+ * Dk = Dv = 128, at most 8 requests and at most one (request, head) unit per SM;
+ * any other call ignores the workspace.  Errors: GDN_ERR_SHAPE if a non-NULL
+ * workspace is smaller than the size the call needs, GDN_ERR_ALIGN, GDN_ERR_ALIAS;
+ * otherwise as gdn_prefill.
+ */
+GDN_API gdn_status gdn_prefill_ws(const void *q, const void *k, const void *v,
+                          const float *g, const float *beta,
+                          const float *a_log, const float *dt_bias,
+                          const int32_t *cu_seqlens,
+                          const float *initial_state, float *final_state,
+                          void *out,
+                          int32_t B, int64_t N, int32_t Hq, int32_t Hv,
+                          int32_t Dk, int32_t Dv, gdn_dtype dtype,
+                          float scale, int32_t qk_l2norm, uint32_t flags,
+                          void *workspace, uint64_t workspace_bytes,
+                          int32_t *dev_status, void *stream);
+
+/* Workspace bytes gdn_prefill_ws needs for these sizes (0: the call never splits,
+ * pass NULL).  Host-only: reads the current device's SM count, launches nothing. */
+GDN_API uint64_t gdn_prefill_workspace_size(int32_t B, int64_t N, int32_t Hq, int32_t Hv,
+                                            int32_t Dk, int32_t Dv, gdn_dtype dtype,
+                                            uint32_t flags);
 
 /*
  * gdn_decode -- Gated DeltaProduct decode / MTP over an fp32 state pool.

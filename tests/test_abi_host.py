@@ -206,3 +206,19 @@ def test_use_library_switches_and_fails_loudly(tmp_path):
     finally:
         assert g.use_library(prev) == str(tmp_path / "missing.so")
     assert b.LIB_PATH == prev
+
+
+def test_split_workspace_query_needs_a_device(L):
+    """gdn_prefill_workspace_size is a host-only query; without a device (or for calls that
+    never split) it is 0, and gdn_prefill_ws with a NULL workspace validates like gdn_prefill."""
+    import gated_deltanet_state_gdn_b200 as g
+    ws = L.gdn_prefill_workspace_size
+    assert ws(1, 32768, 16, 32, 128, 128, g.GDN_F32, 0) == 0          # fp32: per-token kernel
+    assert ws(1, 32768, 16, 32, 128, 128, g.GDN_BF16, g.GDN_PREFILL_SEQUENTIAL) == 0
+    assert ws(1, 32768, 16, 32, 64, 64, g.GDN_BF16, 0) == 0           # only 128-wide heads
+    assert ws(16, 32768, 16, 32, 128, 128, g.GDN_BF16, 0) == 0        # more than 8 requests
+    assert ws(1, 32768, 3, 32, 128, 128, g.GDN_BF16, 0) == 0          # Hv % Hq != 0
+    st = L.gdn_prefill_ws(P(1), P(2), P(3), P(4), P(5), None, None, None, None, P(7), P(8),
+                          2, 64, 1, 1, 16, 16, 0, 1.0, 0, 0, None, 0, None, None)
+    assert st == L.gdn_prefill(P(1), P(2), P(3), P(4), P(5), None, None, None, None, P(7), P(8),
+                               2, 64, 1, 1, 16, 16, 0, 1.0, 0, 0, None, None)
