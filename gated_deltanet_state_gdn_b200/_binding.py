@@ -57,9 +57,9 @@ GDN_DEV_INTERNAL = 4
 GDN_DEV_BOUNDS = 8            # checked builds only
 GDN_DEV_TEST_STALL = 1 << 30  # checked builds only, set by the caller (decode timeout path)
 
-EXPORTED = ("gdn_prefill", "gdn_prefill_ws", "gdn_prefill_workspace_size", "gdn_decode",
-            "gdn_conv1d", "gdn_status_string", "gdn_last_error", "gdn_abi_version",
-            "gdn_prefill_uses_chunked")
+EXPORTED = ("gdn_prefill", "gdn_prefill_ws", "gdn_prefill_workspace_size",
+            "gdn_prefill_noalloc", "gdn_decode", "gdn_conv1d", "gdn_status_string",
+            "gdn_last_error", "gdn_abi_version", "gdn_prefill_uses_chunked")
 
 _lib = None
 
@@ -103,6 +103,8 @@ def lib():
         L.gdn_prefill_ws.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp,
                                      i32, i64, i32, i32, i32, i32, ctypes.c_int, f32, i32, u32,
                                      vp, ctypes.c_uint64, vp, vp]
+        L.gdn_prefill_noalloc.restype = ctypes.c_int
+        L.gdn_prefill_noalloc.argtypes = L.gdn_prefill.argtypes
         L.gdn_prefill_workspace_size.restype = ctypes.c_uint64
         L.gdn_prefill_workspace_size.argtypes = [i32, i64, i32, i32, i32, i32, ctypes.c_int, u32]
         L.gdn_decode.restype = ctypes.c_int

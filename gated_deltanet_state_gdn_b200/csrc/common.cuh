@@ -205,3 +205,5 @@ bool prefill_chunked_supported(const GdnPrefillArgs &a);
 // bytes of workspace with which gdn_prefill may split long requests (0: never splits)
 uint64_t prefill_split_workspace_bytes(const GdnPrefillArgs &a);
 cudaError_t launch_seq_compose(const GdnPrefillArgs &a, void *workspace, int G, cudaStream_t stream);
+// records a CUDA failure for gdn_last_error() and returns GDN_ERR_CUDA
+gdn_status gdn_report_cuda_failure(cudaError_t e, const char *where);

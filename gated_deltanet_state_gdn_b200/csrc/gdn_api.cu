@@ -32,6 +32,8 @@ bool overlaps(const void *p, size_t bytes, const void *q, size_t qbytes)
 
 }  // namespace
 
+gdn_status gdn_report_cuda_failure(cudaError_t e, const char *where) { return cuda_fail(e, where); }
+
 extern "C" {
 
 int32_t gdn_abi_version(void) { return GDN_ABI_VERSION; }

@@ -213,6 +213,38 @@ GDN_API uint64_t gdn_prefill_workspace_size(int32_t B, int64_t N, int32_t Hq, in
                                             uint32_t flags);
 
 /*
+ * gdn_prefill_noalloc -- gdn_prefill_ws whose workspace is a fixed array inside the
+ * library, so the call allocates nothing and needs no workspace from the caller.
+ *
+ * No passage of the pages corresponds to this entry point: it serves callers that cannot
+ * allocate device memory for a call -- a host runtime that owns all device memory
+ * through its own pool, a C caller without a memory manager, a serving path that must
+ * never allocate -- and still want the sequence-parallel split of gdn_prefill_ws.
+ *
+ * Arguments and results: exactly those of gdn_prefill (inputs and outputs are the
+ * caller's).  The workspace is a static device array of 8 MiB (8388608 bytes) that every
+ * GPU loading the library holds until the process exits; 8 MiB covers 32 (request, value
+ * head) units of 128 x 128 heads, e.g. one request with 32 value heads.  A call whose split
+ * would need more (gdn_prefill_workspace_size > 8 MiB) returns GDN_ERR_UNSUPPORTED before
+ * launching anything; a call that cannot split runs as gdn_prefill.
+ * The array's device address is looked up (cudaGetSymbolAddress) on the first call made on
+ * each device, with that device current; make that first call before any stream capture.
+ * All calls on a device share the one array: calls that overlap on the GPU (on different
+ * streams, without ordering) race on it and must not be issued.  Nothing in the array needs
+ * to start at zero: every byte a call reads was written earlier by the same call.
+ */
+GDN_API gdn_status gdn_prefill_noalloc(const void *q, const void *k, const void *v,
+                               const float *g, const float *beta,
+                               const float *a_log, const float *dt_bias,
+                               const int32_t *cu_seqlens,
+                               const float *initial_state, float *final_state,
+                               void *out,
+                               int32_t B, int64_t N, int32_t Hq, int32_t Hv,
+                               int32_t Dk, int32_t Dv, gdn_dtype dtype,
+                               float scale, int32_t qk_l2norm, uint32_t flags,
+                               int32_t *dev_status, void *stream);
+
+/*
  * gdn_decode -- Gated DeltaProduct decode / MTP over an fp32 state pool.
  *
  * Defined by "flashinfer.cake_gdp.cake_gated_delta_product_mtp" (description,
