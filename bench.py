@@ -606,7 +606,8 @@ def profile_phase(gdn, workloads, args):
     """Run one phase for `--steps` steps after `--warmup` (under a profiler); prints timings."""
     if args.phase == "prefill":
         case = make_case(args.workload)
-        total_ms, launch_ms = time_prefill(gdn, case, args.steps, args.warmup, 1)
+        # no repeat windows: under a profiler every launch counts
+        total_ms, launch_ms = time_prefill(gdn, case, args.steps, args.warmup, 1, min_window_s=0.0)
         print(json.dumps({"phase": "prefill", "workload": case.name,
                           "ms_per_launch": statistics.mean(launch_ms)}), flush=True)
     elif args.phase == "conv":
