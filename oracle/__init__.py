@@ -45,6 +45,7 @@ def _load():
             D, D, D, D, D, I32, D, D, D,
             ctypes.c_int, ctypes.c_int64, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int,
             ctypes.c_double, ctypes.c_int, ctypes.c_int, D, D, ctypes.c_int, ctypes.c_int,
+            ctypes.c_int,
         ]
         lib.oracle_decode.restype = None
         lib.oracle_decode.argtypes = [
@@ -90,7 +91,8 @@ RULES = {"gated_delta": 0, "gated": 1, "delta": 2, "linear": 3}
 
 def prefill(q, k, v, g, beta, cu_seqlens=None, initial_state=None, *, B=None,
             scale=1.0, qk_l2norm=False, out=None, threads=None, update_rule="gated_delta",
-            gate_activation="none", a_log=None, dt_bias=None, beta_activation="none"):
+            gate_activation="none", a_log=None, dt_bias=None, beta_activation="none",
+            decay_per_key=False):
     """Sequential recurrence of the log-space form, float64.
 
     q, k: [N, Hq, Dk]; v: [N, Hv, Dv]; g, beta: [N, Hv] (None where the update
@@ -98,6 +100,9 @@ def prefill(q, k, v, g, beta, cu_seqlens=None, initial_state=None, *, B=None,
     packing, needs ``B``); initial_state: [B, Hv, Dv, Dk] or None.
     update_rule: gated_delta | gated | delta | linear; gate_activation: none |
     qwen (needs a_log, dt_bias [Hv]); beta_activation: none | sigmoid.
+    decay_per_key: g is [N, Hv, Dk], one log-space decay per key dimension (the op's
+    per-key-dimension spelling of ``decay``; the scalar exp(g_t) becomes diag(exp(g_t))
+    on the key axis of the state).
     ``out`` (optional, [N, Hv, Dv] float64) supplies the values kept for
     tokens that no request covers.
     Returns (out [N, Hv, Dv], final_state [B, Hv, Dv, Dk]) as float64.
@@ -121,6 +126,9 @@ def prefill(q, k, v, g, beta, cu_seqlens=None, initial_state=None, *, B=None,
     else:
         cu = None
         assert B is not None and N % B == 0
+    if g is not None:
+        assert g.shape == ((N, Hv, Dk) if decay_per_key else (N, Hv)), g.shape
+    assert not decay_per_key or has_decay
     s0 = None if initial_state is None else _f64(initial_state)
     fs = np.zeros((B, Hv, Dv, Dk), np.float64)
     o = np.zeros((N, Hv, Dv), np.float64) if out is None else _f64(out).copy()
@@ -128,7 +136,8 @@ def prefill(q, k, v, g, beta, cu_seqlens=None, initial_state=None, *, B=None,
     _load().oracle_prefill(_dp(q), _dp(k), _dp(v), _dp(g), _dp(beta), _ip(cu), _dp(s0),
                            _dp(fs), _dp(o), B, N, Hq, Hv, Dk, Dv, float(scale),
                            int(bool(qk_l2norm)), rule, _dp(al), _dp(dtb),
-                           int(beta_activation == "sigmoid"), int(nt))
+                           int(beta_activation == "sigmoid"), int(bool(decay_per_key)),
+                           int(nt))
     return o, fs
 
 

@@ -85,6 +85,9 @@ static double softplus20(double x) { return x > 20.0 ? x : log1p(exp(x)); }
  *   g, beta       [N, Hv]            (log-space decay, update rate); g is NULL
  *                                    for rules without decay, beta for rules
  *                                    without retrieval
+ *   g_per_key     non-zero: g is [N, Hv, Dk], one log-space decay per key
+ *                                    dimension (the op's per-key-dimension
+ *                                    spelling of `decay`)
  *   rule          0 gated_delta, 1 gated, 2 delta, 3 linear
  *   a_log, dt_bias [Hv] or NULL      (non-NULL: qwen gate on g)
  *   beta_sigmoid  non-zero: beta <- sigmoid(beta)
@@ -103,7 +106,7 @@ void oracle_prefill(const double *q, const double *k, const double *v,
                     int B, int64_t N, int Hq, int Hv, int Dk, int Dv,
                     double scale, int qk_l2norm, int rule,
                     const double *a_log, const double *dt_bias, int beta_sigmoid,
-                    int nthreads)
+                    int g_per_key, int nthreads)
 {
     int nunits = B * Hv;
     const int has_decay = rule == 0 || rule == 1;
@@ -159,6 +162,44 @@ void oracle_prefill(const double *q, const double *k, const double *v,
                     xq[i] *= rq;
                     xk[i] *= rk;
                 }
+            }
+            if (g_per_key) {
+                /* Per-key-dimension decay: the scalar exp(g_t) of the recurrence becomes
+                 * D_t = diag(exp(g_t[0..Dk))) acting on the key axis of S, in both of its
+                 * places: S_t = D_t S_{t-1} + k_t (beta_t (v_t - (D_t S_{t-1})^T k_t))^T. */
+                double bt = 1.0;
+                if (has_retrieval) {
+                    bt = beta[t * Hv + h];
+                    if (beta_sigmoid) bt = 1.0 / (1.0 + exp(-bt));
+                }
+                const double *gt = g + (t * Hv + h) * Dk;
+                /* S <- D_t S_{t-1} */
+                for (int i = 0; i < Dk; ++i) {
+                    double li = gt[i];
+                    if (a_log) li = -exp(a_log[h]) * softplus20(li + dt_bias[h]);
+                    const double gi = exp(li);
+                    for (int j = 0; j < Dv; ++j) S[(int64_t)i * Dv + j] *= gi;
+                }
+                /* p = (D_t S_{t-1})^T k_t */
+                for (int j = 0; j < Dv; ++j) {
+                    double acc = 0.0;
+                    for (int i = 0; i < Dk; ++i) acc += S[(int64_t)i * Dv + j] * xk[i];
+                    p[j] = acc;
+                }
+                /* S_t = D_t S_{t-1} + k_t (beta (v_t - p))^T; without the retrieval the
+                 * written value is beta v_t */
+                for (int i = 0; i < Dk; ++i)
+                    for (int j = 0; j < Dv; ++j) {
+                        double u = bt * (vt[j] - (has_retrieval ? p[j] : 0.0));
+                        S[(int64_t)i * Dv + j] += xk[i] * u;
+                    }
+                double *ot = out + (t * Hv + h) * Dv;
+                for (int j = 0; j < Dv; ++j) {
+                    double acc = 0.0;
+                    for (int i = 0; i < Dk; ++i) acc += S[(int64_t)i * Dv + j] * xq[i];
+                    ot[j] = scale * acc;
+                }
+                continue;
             }
             /* gate: log-space decay (qwen form if requested), update rate */
             double lg = 0.0;

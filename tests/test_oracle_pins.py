@@ -468,3 +468,132 @@ def test_rule_inputs_are_checked(oracle_mod):
         oracle_mod.prefill(q, k, v, z, z, None, None, B=1, update_rule="linear")
     with pytest.raises(AssertionError):
         oracle_mod.prefill(q, k, v, None, z, None, None, B=1, update_rule="gated_delta")
+
+
+# ---------------------------------------------------------------- per-key-dimension decay
+# "com.microsoft.GatedDeltaNet", Inputs table (`decay`, the per-key-dimension spelling
+# (..., num_heads_v, head_size_qk)): the scalar exp(g_t) of the Description's recurrence is
+# read as D_t = diag(exp(g_t)) on the key axis of the K-major state, in both places,
+#   S_t = D_t S_{t-1} + k_t (beta_t (v_t - (D_t S_{t-1})^T k_t))^T,
+# i.e. the gamma form S_t = (I - beta_t k_t k_t^T) D_t S_{t-1} + beta_t k_t v_t^T.
+def brute_prefill_per_key(q, k, v, g, beta, lengths, init, scale, l2norm, Hq, Hv,
+                          a_log=None, dt_bias=None):
+    """The gamma form with a diagonal decay, as literal Dk x Dk matrix products (K-major)."""
+    N = q.shape[0]
+    Dk, Dv = q.shape[2], v.shape[2]
+    out = np.zeros((N, Hv, Dv))
+    final = np.zeros((len(lengths), Hv, Dv, Dk))
+    off = 0
+    for b, L in enumerate(lengths):
+        for h in range(Hv):
+            qh = (h * Hq) // Hv
+            S = np.zeros((Dk, Dv)) if init is None else init[b, h].T.copy()
+            for t in range(off, off + L):
+                kt, qt = k[t, qh].copy(), q[t, qh].copy()
+                if l2norm:
+                    kt = kt / np.sqrt(kt @ kt + 1e-12)
+                    qt = qt / np.sqrt(qt @ qt + 1e-12)
+                lg = g[t, h]
+                if a_log is not None:
+                    lg = -np.exp(a_log[h]) * np_softplus20(lg + dt_bias[h])
+                Dt = np.diag(np.exp(lg))
+                bt = beta[t, h]
+                S = (np.eye(Dk) - bt * np.outer(kt, kt)) @ Dt @ S + bt * np.outer(kt, v[t, h])
+                out[t, h] = scale * (qt @ S)
+            final[b, h] = S.T
+        off += L
+    return out, final
+
+
+@pytest.mark.parametrize("l2norm", [False, True])
+@pytest.mark.parametrize("Hq,Hv", [(1, 1), (1, 2), (2, 4)])
+def test_per_key_decay_matches_diagonal_gamma_form(oracle_mod, l2norm, Hq, Hv):
+    rng = np.random.default_rng(300 + Hq * 10 + Hv + int(l2norm))
+    lengths = [6, 1, 8, 0, 3]
+    N, Dk, Dv = sum(lengths), 5, 4
+    q = rng.standard_normal((N, Hq, Dk))
+    k = rng.standard_normal((N, Hq, Dk))
+    if not l2norm:
+        k /= np.linalg.norm(k, axis=-1, keepdims=True)
+    v = rng.standard_normal((N, Hv, Dv))
+    g = -rng.uniform(0.0, 2.0, (N, Hv, Dk))
+    beta = rng.uniform(0.0, 1.0, (N, Hv))
+    init = rng.standard_normal((len(lengths), Hv, Dv, Dk))
+    cu = np.concatenate([[0], np.cumsum(lengths)]).astype(np.int32)
+    out, fs = oracle_mod.prefill(q, k, v, g, beta, cu, init, scale=0.8, qk_l2norm=l2norm,
+                                 decay_per_key=True)
+    bo, bf = brute_prefill_per_key(q, k, v, g, beta, lengths, init, 0.8, l2norm, Hq, Hv)
+    np.testing.assert_allclose(out, bo, rtol=1e-10, atol=1e-12)
+    np.testing.assert_allclose(fs, bf, rtol=1e-10, atol=1e-12)
+    # the empty request copies its state through
+    np.testing.assert_array_equal(fs[3], init[3])
+
+
+def test_per_key_decay_qwen_gate_and_sigmoid_beta(oracle_mod):
+    """The qwen gate maps every key dimension's decay input with the head's a_log and
+    dt_bias; beta_activation sigmoid as in the scalar case."""
+    rng = np.random.default_rng(310)
+    N, Hv, Dk, Dv = 9, 2, 4, 3
+    q, k = rng.standard_normal((2, N, 1, Dk))
+    v = rng.standard_normal((N, Hv, Dv))
+    graw = rng.standard_normal((N, Hv, Dk))
+    braw = rng.standard_normal((N, Hv))
+    a_log, dtb = rng.uniform(-1, 1, Hv), rng.uniform(-1, 1, Hv)
+    init = rng.standard_normal((1, Hv, Dv, Dk))
+    out, fs = oracle_mod.prefill(q, k, v, graw, braw, None, init, B=1, scale=0.9,
+                                 qk_l2norm=True, gate_activation="qwen", a_log=a_log,
+                                 dt_bias=dtb, beta_activation="sigmoid", decay_per_key=True)
+    bo, bf = brute_prefill_per_key(q, k, v, graw, 1.0 / (1.0 + np.exp(-braw)), [N], init, 0.9,
+                                   True, 1, Hv, a_log=a_log, dt_bias=dtb)
+    np.testing.assert_allclose(out, bo, rtol=1e-10, atol=1e-12)
+    np.testing.assert_allclose(fs, bf, rtol=1e-10, atol=1e-12)
+
+
+def test_per_key_gated_rule_is_decayed_linear_attention(oracle_mod):
+    """update_rule gated with a per-key decay: the causal sum with per-dimension decay
+    ratios, out_t = scale (sum_i q_t[i] e^{G_t[i]} S0[i, :] + sum_{j<=t} (sum_i q_t[i] k_j[i]
+    e^{G_t[i] - G_j[i]}) v_j), and final state diag(e^{G_T}) S0 + sum_j (k_j e^{G_T - G_j}) v_j^T,
+    with G the inclusive prefix sums of g over the tokens."""
+    rng, q, k, v, init = _rand_case(311, 12, 5, 3, unit_keys=False)
+    g = -rng.uniform(0.0, 1.0, (12, 1, 5))
+    out, fs = oracle_mod.prefill(q, k, v, g, None, None, init, B=1, scale=1.1,
+                                 update_rule="gated", decay_per_key=True)
+    Q, K, V, G = q[:, 0], k[:, 0], v[:, 0], np.cumsum(g[:, 0], axis=0)
+    S0k = init[0, 0].T
+    mask = np.tril(np.ones((12, 12)))
+    scores = np.einsum("ti,ji,tji->tj", Q, K, np.exp(G[:, None, :] - G[None, :, :])) * mask
+    ro = 1.1 * ((Q * np.exp(G)) @ S0k + scores @ V)
+    rf = np.exp(G[-1])[:, None] * S0k + (K * np.exp(G[-1] - G)).T @ V
+    np.testing.assert_allclose(out[:, 0], ro, rtol=1e-10, atol=1e-12)
+    np.testing.assert_allclose(fs[0, 0], rf.T, rtol=1e-10, atol=1e-12)
+
+
+def test_per_key_beta0_scales_state_columns(oracle_mod):
+    """beta = 0 leaves only the decay: the V-major final state's column i is the initial one
+    times exp(sum_t g_t[i]), and o_t = scale S0 (e^{G_t} * q_t)."""
+    rng, q, k, v, init = _rand_case(312, 7, 6, 4)
+    g = -rng.uniform(0.0, 0.7, (7, 1, 6))
+    out, fs = oracle_mod.prefill(q, k, v, g, np.zeros((7, 1)), None, init, B=1, scale=0.6,
+                                 decay_per_key=True)
+    np.testing.assert_allclose(fs[0, 0], init[0, 0] * np.exp(g[:, 0].sum(0))[None, :],
+                               rtol=1e-12)
+    G = np.cumsum(g[:, 0], axis=0)
+    np.testing.assert_allclose(out[:, 0], 0.6 * (q[:, 0] * np.exp(G)) @ init[0, 0].T,
+                               rtol=1e-12, atol=1e-14)
+
+
+def test_per_key_decay_with_equal_dimensions_is_the_scalar_gate(oracle_mod):
+    """A per-key decay that is the same in every key dimension is the scalar decay, whose
+    oracle is pinned to the page's worked examples and its own brute force above."""
+    rng = np.random.default_rng(313)
+    N, Hv, Dk, Dv = 10, 2, 4, 5
+    q, k = rng.standard_normal((2, N, 1, Dk))
+    v = rng.standard_normal((N, Hv, Dv))
+    g = -rng.uniform(0.0, 1.5, (N, Hv))
+    beta = rng.uniform(0.0, 1.0, (N, Hv))
+    init = rng.standard_normal((1, Hv, Dv, Dk))
+    o1, f1 = oracle_mod.prefill(q, k, v, g, beta, None, init, B=1, qk_l2norm=True)
+    o2, f2 = oracle_mod.prefill(q, k, v, np.repeat(g[:, :, None], Dk, axis=2), beta, None, init,
+                                B=1, qk_l2norm=True, decay_per_key=True)
+    np.testing.assert_allclose(o2, o1, rtol=1e-12, atol=1e-14)
+    np.testing.assert_allclose(f2, f1, rtol=1e-12, atol=1e-14)
