@@ -11,6 +11,7 @@ from ._binding import (  # noqa: F401
     GDN_ERR_UNSUPPORTED, GDN_F32, GDN_OK, GDN_PREFILL_SEQUENTIAL, EXPORTED, LIB_PATH, GdnError,
     GDN_F16, gdn_conv1d, gdn_decode, gdn_prefill, lib, prefill_uses_chunked, status_string,
     CHECKED_LIB_PATH, GDN_DEV_BOUNDS, GDN_DEV_TEST_STALL, GDN_DEV_TIMEOUT, use_library,
+    GDN_DECAY_PER_KEY,
 )
 
 __all__ = ["gdn_prefill", "gdn_decode", "gdn_conv1d", "GdnError", "lib", "status_string"]

@@ -42,6 +42,7 @@ GDN_RULE_DELTA = 2 << 3
 GDN_RULE_LINEAR = 3 << 3
 GDN_GATE_QWEN = 1 << 5
 GDN_BETA_SIGMOID = 1 << 6
+GDN_DECAY_PER_KEY = 1 << 8
 
 # update_rule of the op -> (flag bits, has decay input, has beta input)
 UPDATE_RULES = {
@@ -127,11 +128,12 @@ def lib():
 
 
 def prefill_uses_chunked(dtype: torch.dtype, Hv: int, Dk: int, Dv: int,
-                         sequential: bool = False) -> bool:
+                         sequential: bool = False, decay_per_key: bool = False) -> bool:
     """True when gdn_prefill would run the chunked tensor-core kernel for these sizes."""
     code = {torch.bfloat16: GDN_BF16, torch.float16: GDN_F16}.get(dtype, GDN_F32)
-    return bool(lib().gdn_prefill_uses_chunked(code, Hv, Dk, Dv,
-                                               GDN_PREFILL_SEQUENTIAL if sequential else 0))
+    flags = (GDN_PREFILL_SEQUENTIAL if sequential else 0) | \
+        (GDN_DECAY_PER_KEY if decay_per_key else 0)
+    return bool(lib().gdn_prefill_uses_chunked(code, Hv, Dk, Dv, flags))
 
 
 def status_string(status: int) -> str:
@@ -176,7 +178,8 @@ def gdn_prefill(q, k, v, g, beta, cu_seqlens=None, initial_state=None, final_sta
 
     q, k: [N, Hq, Dk] or [B, S, Hq, Dk]; v: [N, Hv, Dv] (same leading axes);
     activations fp32, bf16 or fp16; g, beta: [N, Hv] fp32 (g None for the rules
-    without decay, beta None for those without retrieval); cu_seqlens: [B+1]
+    without decay, beta None for those without retrieval); g may instead be
+    [N, Hv, Dk] (one decay per key dimension, GDN_DECAY_PER_KEY); cu_seqlens: [B+1]
     int32 (rank-3 form) or None; initial_state: [B, Hv, Dv, Dk] fp32 or None.
     update_rule: gated_delta | gated | delta | linear; gate_activation: none |
     qwen (a_log, dt_bias: [Hv] fp32); beta_activation: none | sigmoid.
@@ -196,6 +199,8 @@ def gdn_prefill(q, k, v, g, beta, cu_seqlens=None, initial_state=None, final_sta
     qwen = gate_activation == "qwen"
     if qwen != (a_log is not None and dt_bias is not None):
         raise ValueError("gate_activation 'qwen' requires a_log and dt_bias (and only it takes them)")
+    # the per-key-dimension spelling of the decay has one more axis than [..., Hv]
+    per_key = g is not None and g.dim() == q.dim()
     if q.dim() == 4:
         Bq, S = q.shape[0], q.shape[1]
         if cu_seqlens is not None:
@@ -204,7 +209,8 @@ def gdn_prefill(q, k, v, g, beta, cu_seqlens=None, initial_state=None, final_sta
         q = q.reshape(Bq * S, *q.shape[2:])
         k = k.reshape(Bq * S, *k.shape[2:])
         v = v.reshape(Bq * S, *v.shape[2:])
-        g = None if g is None else g.reshape(Bq * S, -1)
+        g = None if g is None else (g.reshape(Bq * S, *g.shape[2:]) if per_key
+                                    else g.reshape(Bq * S, -1))
         beta = None if beta is None else beta.reshape(Bq * S, -1)
         if out is not None:
             out = out.view(Bq * S, *out.shape[2:])
@@ -223,7 +229,8 @@ def gdn_prefill(q, k, v, g, beta, cu_seqlens=None, initial_state=None, final_sta
     q, k, v, g, beta, initial_state = map(_align16, (q, k, v, g, beta, initial_state))
     N, Hq, Dk = q.shape
     Hv, Dv = v.shape[1], v.shape[2]
-    if k.shape != q.shape or v.shape[0] != N or (g is not None and g.shape != (N, Hv)) or \
+    g_shape = (N, Hv, Dk) if per_key else (N, Hv)
+    if k.shape != q.shape or v.shape[0] != N or (g is not None and g.shape != g_shape) or \
             (beta is not None and beta.shape != (N, Hv)):
         raise ValueError("inconsistent q/k/v/g/beta shapes")
     if qwen and (a_log.shape != (Hv,) or dt_bias.shape != (Hv,)):
@@ -248,6 +255,7 @@ def gdn_prefill(q, k, v, g, beta, cu_seqlens=None, initial_state=None, final_sta
         scale = 1.0 / math.sqrt(Dk)
     flags = (GDN_PREFILL_SEQUENTIAL if sequential else 0) | rule_flags
     flags |= (GDN_GATE_QWEN if qwen else 0) | (GDN_BETA_SIGMOID if beta_activation == "sigmoid" else 0)
+    flags |= GDN_DECAY_PER_KEY if per_key else 0
     ws_bytes = int(lib().gdn_prefill_workspace_size(B, N, Hq, Hv, Dk, Dv, dt, flags)) \
         if split else 0
     if ws_bytes > 0:

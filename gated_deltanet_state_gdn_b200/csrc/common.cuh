@@ -140,6 +140,7 @@ struct GdnPrefillArgs {
     int32_t has_decay, has_retrieval;
     const float *a_log, *dt_bias;   // non-NULL: qwen gate on g
     int32_t beta_sigmoid;
+    int32_t g_per_key;              // g is [N, Hv, Dk]: one decay per key dimension
     // caller-owned device workspace for the sequence-parallel split (NULL: no split)
     void *workspace;
     uint64_t workspace_bytes;

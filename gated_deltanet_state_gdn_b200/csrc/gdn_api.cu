@@ -62,6 +62,7 @@ int32_t gdn_prefill_uses_chunked(gdn_dtype dtype, int32_t Hv, int32_t Dk, int32_
     GdnPrefillArgs a;
     memset(&a, 0, sizeof(a));
     a.dtype = dtype; a.Dk = Dk; a.Dv = Dv; a.Hq = 1; a.Hv = Hv;
+    a.g_per_key = (flags & GDN_DECAY_PER_KEY) ? 1 : 0;
     return prefill_chunked_supported(a) ? 1 : 0;
 }
 
@@ -80,6 +81,7 @@ GdnPrefillArgs prefill_shape(int32_t B, int64_t N, int32_t Hq, int32_t Hv, int32
     a.has_decay = rule == 0 || rule == GDN_RULE_GATED;
     a.has_retrieval = rule == 0 || rule == GDN_RULE_DELTA;
     a.beta_sigmoid = (flags & GDN_BETA_SIGMOID) ? 1 : 0;
+    a.g_per_key = (flags & GDN_DECAY_PER_KEY) ? 1 : 0;
     return a;
 }
 
@@ -95,7 +97,8 @@ gdn_status prefill_impl(const void *q, const void *k, const void *v, const float
     if (B < 0 || N < 0 || Hq < 1 || Hv < 1 || Dk < 1 || Dv < 1) return GDN_ERR_SHAPE;
     if (Hv % Hq != 0) return GDN_ERR_SHAPE;
     if (Dk > 256 || Dv > 256) return GDN_ERR_UNSUPPORTED;
-    const uint32_t known = GDN_PREFILL_SEQUENTIAL | GDN_RULE_MASK | GDN_GATE_QWEN | GDN_BETA_SIGMOID;
+    const uint32_t known = GDN_PREFILL_SEQUENTIAL | GDN_RULE_MASK | GDN_GATE_QWEN |
+                           GDN_BETA_SIGMOID | GDN_DECAY_PER_KEY;
     if (flags & ~known) return GDN_ERR_UNSUPPORTED;
     // update_rule: decay input exactly for gated / gated_delta, beta exactly for delta /
     // gated_delta, qwen parameters exactly with the qwen gate (which needs a decay)
@@ -103,7 +106,8 @@ gdn_status prefill_impl(const void *q, const void *k, const void *v, const float
     const bool has_decay = rule == 0 || rule == GDN_RULE_GATED;
     const bool has_retrieval = rule == 0 || rule == GDN_RULE_DELTA;
     const bool qwen = (flags & GDN_GATE_QWEN) != 0;
-    if (qwen && !has_decay) return GDN_ERR_SHAPE;
+    const bool per_key = (flags & GDN_DECAY_PER_KEY) != 0;
+    if ((qwen || per_key) && !has_decay) return GDN_ERR_SHAPE;
     if ((flags & GDN_BETA_SIGMOID) && !has_retrieval) return GDN_ERR_SHAPE;
     if (B == 0) return N == 0 ? GDN_OK : GDN_ERR_SHAPE;
     if (!cu_seqlens && N % B != 0) return GDN_ERR_SHAPE;
@@ -118,6 +122,7 @@ gdn_status prefill_impl(const void *q, const void *k, const void *v, const float
     const size_t qk_bytes = (size_t)N * Hq * Dk * esz;
     const size_t v_bytes = (size_t)N * Hv * Dv * esz;
     const size_t gb_bytes = (size_t)N * Hv * 4;
+    const size_t g_bytes = per_key ? gb_bytes * Dk : gb_bytes;
     const size_t st_bytes = (size_t)B * Hv * Dv * Dk * 4;
     if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(out, 16) ||
         !aligned(initial_state, 16) || !aligned(final_state, 16) || !aligned(g, 16) ||
@@ -125,13 +130,13 @@ gdn_status prefill_impl(const void *q, const void *k, const void *v, const float
         return GDN_ERR_ALIGN;
     if (overlaps(initial_state, st_bytes, final_state, st_bytes)) return GDN_ERR_ALIAS;
     if (overlaps(out, v_bytes, q, qk_bytes) || overlaps(out, v_bytes, k, qk_bytes) ||
-        overlaps(out, v_bytes, v, v_bytes) || overlaps(out, v_bytes, g, gb_bytes) ||
+        overlaps(out, v_bytes, v, v_bytes) || overlaps(out, v_bytes, g, g_bytes) ||
         overlaps(out, v_bytes, beta, gb_bytes) || overlaps(out, v_bytes, final_state, st_bytes) ||
         overlaps(out, v_bytes, initial_state, st_bytes) ||
         overlaps(final_state, st_bytes, q, qk_bytes) ||
         overlaps(final_state, st_bytes, k, qk_bytes) ||
         overlaps(final_state, st_bytes, v, v_bytes) ||
-        overlaps(final_state, st_bytes, g, gb_bytes) ||
+        overlaps(final_state, st_bytes, g, g_bytes) ||
         overlaps(final_state, st_bytes, beta, gb_bytes) ||
         overlaps(final_state, st_bytes, cu_seqlens, (size_t)(B + 1) * 4) ||
         overlaps(out, v_bytes, a_log, (size_t)Hv * 4) || overlaps(out, v_bytes, dt_bias, (size_t)Hv * 4) ||
@@ -146,6 +151,7 @@ gdn_status prefill_impl(const void *q, const void *k, const void *v, const float
     a.scale = scale; a.qk_l2norm = qk_l2norm ? 1 : 0; a.dev_status = dev_status;
     a.has_decay = has_decay; a.has_retrieval = has_retrieval;
     a.a_log = a_log; a.dt_bias = dt_bias; a.beta_sigmoid = (flags & GDN_BETA_SIGMOID) ? 1 : 0;
+    a.g_per_key = per_key ? 1 : 0;
     a.workspace = nullptr;
     a.workspace_bytes = 0;
 
@@ -158,7 +164,7 @@ gdn_status prefill_impl(const void *q, const void *k, const void *v, const float
             if (!aligned(workspace, 16)) return GDN_ERR_ALIGN;
             const size_t wb = (size_t)need;
             if (overlaps(workspace, wb, q, qk_bytes) || overlaps(workspace, wb, k, qk_bytes) ||
-                overlaps(workspace, wb, v, v_bytes) || overlaps(workspace, wb, g, gb_bytes) ||
+                overlaps(workspace, wb, v, v_bytes) || overlaps(workspace, wb, g, g_bytes) ||
                 overlaps(workspace, wb, beta, gb_bytes) || overlaps(workspace, wb, out, v_bytes) ||
                 overlaps(workspace, wb, initial_state, st_bytes) ||
                 overlaps(workspace, wb, final_state, st_bytes) ||

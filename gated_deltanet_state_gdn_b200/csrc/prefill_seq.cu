@@ -12,6 +12,11 @@
 // its qwen gate maps g to -exp(a_log[h]) softplus(g + dt_bias[h]) and its
 // sigmoid activation maps beta to sigmoid(beta), both in fp32.
 //
+// With the per-key-dimension decay (the op's Inputs table, `decay` of shape
+// (..., num_heads_v, head_size_qk)) exp(g_t) becomes diag(exp(g_t)) on the key
+// axis: each lane scales its own key columns of S by their decay before the
+// retrieval and the write, S_t = D_t S_{t-1} + k_t (beta_t (v_t - (D_t S_{t-1})^T k_t))^T.
+//
 // This is the general path: fp32, bf16 or fp16 activations, any Dk, Dv in
 // [1, 256], any Hq | Hv.  It is also the sequential counterpart the chunked
 // tensor-core kernel is checked against.  Layout: grid (B * Hv, Dv tiles of
@@ -57,7 +62,7 @@ __device__ __forceinline__ void store_act<__half>(__half *p, float x)
     *p = __float2half_rn(x);
 }
 
-template <typename Tin, int EPL>
+template <typename Tin, int EPL, bool PER_KEY>
 __global__ void __launch_bounds__(kSeqWarps * 32)
 prefill_seq_kernel(const GdnPrefillArgs p)
 {
@@ -133,6 +138,46 @@ prefill_seq_kernel(const GdnPrefillArgs p)
                 qx[j] *= rq;
             }
         }
+        if constexpr (PER_KEY) {
+            // gamma_j for this lane's key columns (p.has_decay holds on this path)
+            float gam[EPL], kd[EPL];
+            const float *gt = p.g + (t * Hv + h) * (int64_t)Dk;
+#pragma unroll
+            for (int j = 0; j < EPL; ++j) {
+                const int e = lane + 32 * j;
+                float lg = e < Dk ? __ldg(gt + e) : 0.f;
+                if (p.a_log) lg = -expf(__ldg(p.a_log + h)) * softplus20(lg + __ldg(p.dt_bias + h));
+                gam[j] = expf(lg);
+                kd[j] = p.has_retrieval ? gam[j] * kx[j] : 0.f;   // D_t k_t: the retrieval
+            }
+            float bt = 1.f;
+            if (p.has_retrieval) {
+                bt = __ldg(p.beta + t * Hv + h);
+                if (p.beta_sigmoid) bt = sigmoidf_(bt);
+            }
+            const int64_t vo = (t * Hv + h) * (int64_t)Dv;
+#pragma unroll
+            for (int i = 0; i < R; ++i) {
+                const int row = row_base + i;
+                if (row >= Dv) break;  // uniform across the warp
+                const float vi = load_act<Tin>(vg + vo + row);
+                // row `row` of (D_t S_{t-1})^T k_t (V-major: sum over the key columns)
+                float pd = 0.f;
+#pragma unroll
+                for (int j = 0; j < EPL; ++j) pd += S[i][j] * kd[j];
+                pd = warp_sum(pd);
+                const float u = bt * (vi - pd);
+                float o = 0.f;
+#pragma unroll
+                for (int j = 0; j < EPL; ++j) {
+                    S[i][j] = fmaf(kx[j], u, gam[j] * S[i][j]);
+                    o += S[i][j] * qx[j];
+                }
+                o = warp_sum(o);
+                if (lane == 0) store_act<Tin>(og + vo + row, p.scale * o);
+            }
+            continue;
+        }
         float lg = 0.f, bt = 1.f;
         if (p.has_decay) {
             lg = __ldg(p.g + t * Hv + h);
@@ -176,21 +221,27 @@ prefill_seq_kernel(const GdnPrefillArgs p)
         }
 }
 
-template <typename Tin>
+template <typename Tin, bool PER_KEY>
 static cudaError_t launch_seq_t(const GdnPrefillArgs &a, cudaStream_t stream)
 {
     dim3 grid((unsigned)a.B * (unsigned)a.Hv, (unsigned)((a.Dv + kSeqWarps * kSeqRows - 1) /
                                                          (kSeqWarps * kSeqRows)));
     dim3 block(kSeqWarps * 32);
     if (a.Dk <= 32)
-        prefill_seq_kernel<Tin, 1><<<grid, block, 0, stream>>>(a);
+        prefill_seq_kernel<Tin, 1, PER_KEY><<<grid, block, 0, stream>>>(a);
     else if (a.Dk <= 64)
-        prefill_seq_kernel<Tin, 2><<<grid, block, 0, stream>>>(a);
+        prefill_seq_kernel<Tin, 2, PER_KEY><<<grid, block, 0, stream>>>(a);
     else if (a.Dk <= 128)
-        prefill_seq_kernel<Tin, 4><<<grid, block, 0, stream>>>(a);
+        prefill_seq_kernel<Tin, 4, PER_KEY><<<grid, block, 0, stream>>>(a);
     else
-        prefill_seq_kernel<Tin, 8><<<grid, block, 0, stream>>>(a);
+        prefill_seq_kernel<Tin, 8, PER_KEY><<<grid, block, 0, stream>>>(a);
     return cudaGetLastError();
+}
+
+template <typename Tin>
+static cudaError_t launch_seq_t(const GdnPrefillArgs &a, cudaStream_t stream)
+{
+    return a.g_per_key ? launch_seq_t<Tin, true>(a, stream) : launch_seq_t<Tin, false>(a, stream);
 }
 
 }  // namespace gdn

@@ -94,14 +94,18 @@ class DecodeCase:
 def make_prefill(seed: int, lengths, Hq: int, Hv: int, Dk: int, Dv: int, *,
                  dtype=torch.bfloat16, uniform: bool = False, init_std: Optional[float] = 0.02,
                  qk_l2norm: bool = True, host_norm_qk: bool = False, scale: Optional[float] = None,
-                 gate: str = "softplus", name: str = "prefill") -> PrefillCase:
+                 gate: str = "softplus", name: str = "prefill",
+                 decay_per_key: bool = False) -> PrefillCase:
     """Generic ragged prefill case.
 
     gate="softplus": g = -softplus(N(0,1)), beta = sigmoid(N(0,1)).
     gate="uniform":  gamma ~ U[0.8, 1] passed as g = ln(gamma), beta ~ U[0, 1].
+    decay_per_key: g has one value per key dimension, [N, Hv, Dk], drawn the same way
+    element by element.
     host_norm_qk: q and k are unit-normalised in fp32 before the cast.
     uniform=True: every length must be equal and cu_seqlens is None.
     """
+    gshape = lambda: (N, Hv, Dk) if decay_per_key else (N, Hv)
     rng = np.random.default_rng(seed)
     lengths = [int(x) for x in lengths]
     B = len(lengths)
@@ -113,10 +117,10 @@ def make_prefill(seed: int, lengths, Hq: int, Hv: int, Dk: int, Dv: int, *,
         q = _unit_rows(q)
         k = _unit_rows(k)
     if gate == "softplus":
-        g = _neg_softplus(rng.standard_normal((N, Hv), dtype=np.float32))
+        g = _neg_softplus(rng.standard_normal(gshape(), dtype=np.float32))
         beta = _sigmoid(rng.standard_normal((N, Hv), dtype=np.float32))
     elif gate == "uniform":
-        gamma = rng.uniform(0.8, 1.0, (N, Hv))
+        gamma = rng.uniform(0.8, 1.0, gshape())
         g = np.log(gamma).astype(np.float32)
         beta = rng.uniform(0.0, 1.0, (N, Hv)).astype(np.float32)
     else:
@@ -152,13 +156,17 @@ def tiny_oracle_case(seed: int = 1) -> PrefillCase:
                        scale=1.0, qk_l2norm=False, meta={"S": S})
 
 
-def ragged_prefill_case(seed: int = 2, n_req: int = 8, max_len: int = 4096) -> PrefillCase:
+def ragged_prefill_case(seed: int = 2, n_req: int = 8, max_len: int = 4096,
+                        decay_per_key: bool = False) -> PrefillCase:
     """8 requests, lengths U[1, 4096] packed by cu_seqlens; Hq=16, Hv=32, D=128, bf16,
-    qk_l2_norm=1, g=-softplus(N(0,1)), beta=sigmoid(N(0,1)), initial state N(0, 0.02^2)."""
+    qk_l2_norm=1, g=-softplus(N(0,1)), beta=sigmoid(N(0,1)), initial state N(0, 0.02^2).
+    decay_per_key: g is [N, 32, 128], -softplus(N(0,1)) in every key dimension."""
     rng = np.random.default_rng(seed)
     lengths = rng.integers(1, max_len + 1, n_req).tolist()
+    tag = "_per_key_decay" if decay_per_key else ""
     c = make_prefill(seed + 1000, lengths, 16, 32, 128, 128, init_std=0.02, qk_l2norm=True,
-                     name=f"ragged_prefill_{n_req}req_U1-{max_len}_Hq16_Hv32_D128_bf16")
+                     name=f"ragged_prefill_{n_req}req_U1-{max_len}_Hq16_Hv32_D128_bf16{tag}",
+                     decay_per_key=decay_per_key)
     return c
 
 

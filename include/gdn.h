@@ -72,7 +72,8 @@ enum {
     GDN_RULE_LINEAR = 3u << 3,          /* neither: S_t = S_{t-1} + k_t v_t^T */
     GDN_RULE_MASK = 3u << 3,
     GDN_GATE_QWEN = 1u << 5,            /* prefill: g <- -exp(a_log[h]) softplus(g + dt_bias[h]) */
-    GDN_BETA_SIGMOID = 1u << 6          /* prefill: beta <- sigmoid(beta) */
+    GDN_BETA_SIGMOID = 1u << 6,         /* prefill: beta <- sigmoid(beta) */
+    GDN_DECAY_PER_KEY = 1u << 8         /* prefill: g is [N, Hv, Dk], one decay per key dimension */
 };
 
 /* bits OR-ed into *dev_status by the kernels */
@@ -111,6 +112,15 @@ enum {
  *                  `decay` input and the kernels use
  *                  -exp(a_log[h]) * softplus(g + dt_bias[h]) (softplus(x) = x
  *                  for x > 20), in float32.
+ *                  With GDN_DECAY_PER_KEY, g is [N, Hv, Dk] float32, the op's
+ *                  per-key-dimension spelling of `decay` (Inputs table): exp(g_t)
+ *                  becomes diag(exp(g_t[0..Dk))) on the key axis of the state,
+ *                  in both places of the recurrence,
+ *                    S_t = D_t S_{t-1} + k_t (beta_t (v_t - (D_t S_{t-1})^T k_t))^T
+ *                  (V-major: column i of S scales by exp(g_t[i])); the qwen gate
+ *                  maps every element with its head's a_log and dt_bias.  The
+ *                  page lists this spelling as not implemented by its own kernels;
+ *                  here it runs the per-token kernel.
  *   beta           [N, Hv] float32, update rate; required exactly for the rules
  *                  with the delta retrieval (gated_delta, delta), NULL
  *                  otherwise (the write is then k_t v_t^T).  With
@@ -131,7 +141,8 @@ enum {
  *                  (sum x^2 + 1e-12)^(-1/2) before use.
  *   flags          GDN_PREFILL_SEQUENTIAL, one GDN_RULE_* (update_rule of the
  *                  op's Attributes table: which of the decay and the delta
- *                  retrieval survive), GDN_GATE_QWEN, GDN_BETA_SIGMOID.
+ *                  retrieval survive), GDN_GATE_QWEN, GDN_BETA_SIGMOID,
+ *                  GDN_DECAY_PER_KEY (needs a rule with decay, else GDN_ERR_SHAPE).
  *   dev_status     optional device int32; GDN_DEV_TIMEOUT is OR-ed in if an
  *                  internal pipeline wait of the chunked kernel exceeds its
  *                  bound (the call's outputs are then invalid).

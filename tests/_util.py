@@ -29,7 +29,8 @@ def oracle_prefill_case(oracle, c, out=None):
     return oracle.prefill(f64(c.q), f64(c.k), f64(c.v), f64(c.g), f64(c.beta),
                           None if c.cu_seqlens is None else c.cu_seqlens.numpy(),
                           None if c.initial_state is None else f64(c.initial_state),
-                          B=c.B, scale=c.scale, qk_l2norm=c.qk_l2norm, out=out)
+                          B=c.B, scale=c.scale, qk_l2norm=c.qk_l2norm, out=out,
+                          decay_per_key=c.g.dim() == 3)
 
 
 def run_gpu_prefill(c, sequential=False, out=None):

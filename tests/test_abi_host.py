@@ -108,6 +108,22 @@ def test_prefill_rule_and_gate_validation(L):
     assert prefill(L, dtype=2, flags=1 << 7) == 6         # unknown flag bit
 
 
+def test_prefill_per_key_decay_validation(L):
+    """GDN_DECAY_PER_KEY: g is [N, Hv, Dk]; it needs a rule with decay, and the overlap
+    checks use the larger g."""
+    import gated_deltanet_state_gdn_b200 as g
+    PK, DELTA, LINEAR = g.GDN_DECAY_PER_KEY, 2 << 3, 3 << 3
+    assert PK == 1 << 8
+    assert prefill(L, flags=PK | DELTA, g=None) == 2      # no decay to spell per key
+    assert prefill(L, flags=PK | LINEAR, g=None, beta=None) == 2
+    # N * Hv * Dk floats of g = 64 * 16 * 4 bytes: out 4 KiB - 64 past g's start overlaps it
+    assert prefill(L, flags=PK, out=P(4, 64 * 16 * 4 - 64)) == 5
+    assert prefill(L, flags=PK, final=P(4, 64 * 16 * 4 - 64)) == 5
+    assert prefill(L, flags=PK, g=P(4, 8)) == 4
+    assert L.gdn_prefill_uses_chunked(g.GDN_BF16, 32, 128, 128, PK) == 0
+    assert L.gdn_prefill_workspace_size(1, 32768, 16, 32, 128, 128, g.GDN_BF16, PK) == 0
+
+
 def decode(L, **kw):
     args = dict(q=P(1), k=P(2), v=P(3), pool=P(4), P=16, ss=32 * 128 * 128, hs=128 * 128,
                 ri=P(5), wi=None, si=None, A=P(6), a=P(7), dtb=P(8), b=P(9), scale=0.1,

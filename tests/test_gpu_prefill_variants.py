@@ -39,10 +39,12 @@ def W():
 
 
 def _run_both(gdn, oracle_mod, c, g, beta, sequential, **kw):
+    # the binding reads the per-key spelling from g's rank; the oracle takes it as a flag
     o, f = gdn.gdn_prefill(dev(c.q), dev(c.k), dev(c.v), dev(g), dev(beta), dev(c.cu_seqlens),
                            dev(c.initial_state), scale=c.scale, qk_l2norm=c.qk_l2norm,
                            sequential=sequential,
-                           **{k: (dev(v) if torch.is_tensor(v) else v) for k, v in kw.items()})
+                           **{k: (dev(v) if torch.is_tensor(v) else v) for k, v in kw.items()
+                              if k != "decay_per_key"})
     torch.cuda.synchronize()
     okw = {k: (f64(v) if torch.is_tensor(v) else v) for k, v in kw.items()}
     ro, rf = oracle_mod.prefill(f64(c.q), f64(c.k), f64(c.v), None if g is None else f64(g),
@@ -117,4 +119,87 @@ def test_linear_rule_long_sequence_matches_oracle(gdn, W, oracle_mod):
     """Without decay the state is a plain causal sum; a 1000-token request keeps growing it."""
     c = W.make_prefill(35, [1000], 1, 4, 128, 128, init_std=None, qk_l2norm=True)
     o, f, ro, rf = _run_both(gdn, oracle_mod, c, None, None, False, update_rule="linear")
+    _parity(c, o, f, ro, rf, TOL_BF16)
+
+
+# ------------------------------------------------------- per-key-dimension decay
+# "com.microsoft.GatedDeltaNet", Inputs table: `decay` spelled (..., num_heads_v,
+# head_size_qk), exp(g_t) read as diag(exp(g_t)) on the key axis of the state (the oracle's
+# reading, pinned in test_oracle_pins).  It runs the per-token kernel (fp32 arithmetic).
+TOL_BY_DTYPE = {torch.bfloat16: TOL_BF16, torch.float16: TOL_F16, torch.float32: 1e-4}
+
+
+@pytest.mark.parametrize("dtype,Dk,Dv,Hq,Hv", [
+    (torch.bfloat16, 128, 128, 2, 4), (torch.float16, 64, 32, 1, 2), (torch.float32, 12, 9, 1, 2),
+    (torch.float32, 256, 256, 1, 1), (torch.bfloat16, 160, 96, 2, 2), (torch.bfloat16, 1, 1, 1, 3)])
+def test_per_key_decay_matches_oracle(gdn, W, oracle_mod, dtype, Dk, Dv, Hq, Hv):
+    assert not gdn.prefill_uses_chunked(dtype, Hv, Dk, Dv, decay_per_key=True)
+    c = W.make_prefill(41, LENGTHS, Hq, Hv, Dk, Dv, dtype=dtype, init_std=0.02,
+                       qk_l2norm=True, decay_per_key=True)
+    assert tuple(c.g.shape) == (c.N, Hv, Dk)
+    o, f, ro, rf = _run_both(gdn, oracle_mod, c, c.g, c.beta, False, decay_per_key=True)
+    _parity(c, o, f, ro, rf, TOL_BY_DTYPE[dtype])
+
+
+@pytest.mark.parametrize("rule,qwen", [("gated", False), ("gated", True), ("gated_delta", True)])
+def test_per_key_decay_rules_and_gates(gdn, W, oracle_mod, rule, qwen):
+    """The gated rule (no retrieval, beta = 1) and the qwen gate applied to every key
+    dimension with its head's a_log and dt_bias (raw decay N(0,1)), with the sigmoid beta."""
+    c = W.make_prefill(42, LENGTHS, 2, 4, 128, 64, init_std=0.02, qk_l2norm=True,
+                       decay_per_key=True)
+    has_decay, has_beta = RULES[rule]
+    rng = np.random.default_rng(43)
+    g = c.g
+    kw = {"update_rule": rule, "decay_per_key": True}
+    if qwen:
+        g = torch.from_numpy(rng.standard_normal(c.g.shape).astype(np.float32))
+        kw.update(gate_activation="qwen",
+                  a_log=torch.from_numpy(rng.uniform(-2, 1, 4).astype(np.float32)),
+                  dt_bias=torch.from_numpy((0.5 * rng.standard_normal(4)).astype(np.float32)))
+    beta = None
+    if has_beta:
+        beta = torch.from_numpy(rng.standard_normal(c.beta.shape).astype(np.float32))
+        kw["beta_activation"] = "sigmoid"
+    o, f, ro, rf = _run_both(gdn, oracle_mod, c, g, beta, False, **kw)
+    _parity(c, o, f, ro, rf, TOL_BF16)
+
+
+def test_per_key_decay_equal_dimensions_match_scalar_gate(gdn, W):
+    """The same decay in every key dimension is the scalar gate: the per-key and the scalar
+    instantiations of the per-token kernel (fp32) agree to fp32 rounding."""
+    c = W.make_prefill(44, LENGTHS, 2, 4, 64, 64, dtype=torch.float32, init_std=0.02,
+                       qk_l2norm=True)
+    gk = c.g[:, :, None].expand(-1, -1, 64).contiguous()
+    args = (dev(c.q), dev(c.k), dev(c.v))
+    o1, f1 = gdn.gdn_prefill(*args, dev(c.g), dev(c.beta), dev(c.cu_seqlens),
+                             dev(c.initial_state), scale=c.scale, qk_l2norm=True)
+    o2, f2 = gdn.gdn_prefill(*args, dev(gk), dev(c.beta), dev(c.cu_seqlens),
+                             dev(c.initial_state), scale=c.scale, qk_l2norm=True)
+    torch.cuda.synchronize()
+    assert_prefill_parity(f64(o2), f64(f2), f64(o1), f64(f1),
+                          request_ranges(c.cu_seqlens, c.B, c.N), 1e-5)
+
+
+def test_per_key_decay_rank4_spelling(gdn, W, oracle_mod):
+    """(batch, sequence, heads, dim) activations with the decay as (batch, sequence, Hv, Dk)."""
+    B, S, Hq, Hv, D = 3, 70, 1, 2, 32
+    c = W.make_prefill(45, [S] * B, Hq, Hv, D, D, uniform=True, init_std=0.02, qk_l2norm=True,
+                       decay_per_key=True)
+    o, f = gdn.gdn_prefill(dev(c.q).view(B, S, Hq, D), dev(c.k).view(B, S, Hq, D),
+                           dev(c.v).view(B, S, Hv, D), dev(c.g).view(B, S, Hv, D),
+                           dev(c.beta).view(B, S, Hv), None, dev(c.initial_state),
+                           scale=c.scale, qk_l2norm=True)
+    torch.cuda.synchronize()
+    ro, rf = oracle_mod.prefill(f64(c.q), f64(c.k), f64(c.v), f64(c.g), f64(c.beta), None,
+                                f64(c.initial_state), B=B, scale=c.scale, qk_l2norm=True,
+                                decay_per_key=True)
+    assert_prefill_parity(f64(o), f64(f), ro, rf, [(b * S, (b + 1) * S) for b in range(B)],
+                          TOL_BF16)
+
+
+def test_full_ragged_prefill_per_key_decay_all_heads(gdn, W, oracle_mod):
+    """The ragged workload's shapes (8 requests, U[1, 4096], Hq=16, Hv=32, D=128, bf16) with a
+    per-key decay -softplus(N(0,1)) in every key dimension: every head and row."""
+    c = W.ragged_prefill_case(decay_per_key=True)
+    o, f, ro, rf = _run_both(gdn, oracle_mod, c, c.g, c.beta, False, decay_per_key=True)
     _parity(c, o, f, ro, rf, TOL_BF16)
