@@ -112,15 +112,52 @@ prefill_seq_kernel(const GdnPrefillArgs p)
                           : 0.f;
         }
 
-    for (int64_t t = start; t < end; ++t) {
-        float kx[EPL], qx[EPL];
+    // The raw inputs of token t + 1 (k, q, the decay, beta and this warp's R values) are
+    // loaded while token t is computed, so the loop waits on no global load; the R rows'
+    // warp reductions run interleaved (same butterfly order as warp_sum, so every value is
+    // the one a row-by-row loop computes).
+    constexpr int NG = PER_KEY ? EPL : 1;
+    float nk[EPL], nq[EPL], nlg[NG], nbt = 1.f, nv[R];
+    auto load_token = [&](int64_t t) {
         const int64_t qk_off = (t * Hq + qh) * (int64_t)Dk;
 #pragma unroll
         for (int j = 0; j < EPL; ++j) {
             const int e = lane + 32 * j;
-            kx[j] = e < Dk ? load_act<Tin>(kg + qk_off + e) : 0.f;
-            qx[j] = e < Dk ? load_act<Tin>(qg + qk_off + e) : 0.f;
+            nk[j] = e < Dk ? load_act<Tin>(kg + qk_off + e) : 0.f;
+            nq[j] = e < Dk ? load_act<Tin>(qg + qk_off + e) : 0.f;
         }
+        if constexpr (PER_KEY) {
+            const float *gt = p.g + (t * Hv + h) * (int64_t)Dk;
+#pragma unroll
+            for (int j = 0; j < EPL; ++j) {
+                const int e = lane + 32 * j;
+                nlg[j] = e < Dk ? __ldg(gt + e) : 0.f;
+            }
+        } else {
+            nlg[0] = p.has_decay ? __ldg(p.g + t * Hv + h) : 0.f;
+        }
+        nbt = p.has_retrieval ? __ldg(p.beta + t * Hv + h) : 1.f;
+        const int64_t vo = (t * Hv + h) * (int64_t)Dv;
+#pragma unroll
+        for (int i = 0; i < R; ++i)
+            nv[i] = row_base + i < Dv ? load_act<Tin>(vg + vo + row_base + i) : 0.f;
+    };
+    if (start < end) load_token(start);
+
+    for (int64_t t = start; t < end; ++t) {
+        float kx[EPL], qx[EPL], lgv[NG], vv[R];
+        float bt = nbt;
+#pragma unroll
+        for (int j = 0; j < EPL; ++j) {
+            kx[j] = nk[j];
+            qx[j] = nq[j];
+        }
+#pragma unroll
+        for (int j = 0; j < NG; ++j) lgv[j] = nlg[j];
+#pragma unroll
+        for (int i = 0; i < R; ++i) vv[i] = nv[i];
+        if (t + 1 < end) load_token(t + 1);
+
         if (p.qk_l2norm) {
             float sk = 0.f, sq = 0.f;
 #pragma unroll
@@ -138,77 +175,55 @@ prefill_seq_kernel(const GdnPrefillArgs p)
                 qx[j] *= rq;
             }
         }
-        if constexpr (PER_KEY) {
-            // gamma_j for this lane's key columns (p.has_decay holds on this path)
-            float gam[EPL], kd[EPL];
-            const float *gt = p.g + (t * Hv + h) * (int64_t)Dk;
+        if (p.has_retrieval && p.beta_sigmoid) bt = sigmoidf_(bt);
+        // gam: the decay of each of this lane's key columns (one value without PER_KEY);
+        // kr: the key as the retrieval sees it -- D_t k_t per key, k_t (scaled by gamma
+        // after the sum) for the scalar decay
+        float gam[NG], kr[EPL];
 #pragma unroll
-            for (int j = 0; j < EPL; ++j) {
-                const int e = lane + 32 * j;
-                float lg = e < Dk ? __ldg(gt + e) : 0.f;
-                if (p.a_log) lg = -expf(__ldg(p.a_log + h)) * softplus20(lg + __ldg(p.dt_bias + h));
-                gam[j] = expf(lg);
-                kd[j] = p.has_retrieval ? gam[j] * kx[j] : 0.f;   // D_t k_t: the retrieval
-            }
-            float bt = 1.f;
-            if (p.has_retrieval) {
-                bt = __ldg(p.beta + t * Hv + h);
-                if (p.beta_sigmoid) bt = sigmoidf_(bt);
-            }
-            const int64_t vo = (t * Hv + h) * (int64_t)Dv;
-#pragma unroll
-            for (int i = 0; i < R; ++i) {
-                const int row = row_base + i;
-                if (row >= Dv) break;  // uniform across the warp
-                const float vi = load_act<Tin>(vg + vo + row);
-                // row `row` of (D_t S_{t-1})^T k_t (V-major: sum over the key columns)
-                float pd = 0.f;
-#pragma unroll
-                for (int j = 0; j < EPL; ++j) pd += S[i][j] * kd[j];
-                pd = warp_sum(pd);
-                const float u = bt * (vi - pd);
-                float o = 0.f;
-#pragma unroll
-                for (int j = 0; j < EPL; ++j) {
-                    S[i][j] = fmaf(kx[j], u, gam[j] * S[i][j]);
-                    o += S[i][j] * qx[j];
-                }
-                o = warp_sum(o);
-                if (lane == 0) store_act<Tin>(og + vo + row, p.scale * o);
-            }
-            continue;
+        for (int j = 0; j < NG; ++j) {
+            float lg = lgv[j];
+            if (p.has_decay && p.a_log)
+                lg = -expf(__ldg(p.a_log + h)) * softplus20(lg + __ldg(p.dt_bias + h));
+            gam[j] = expf(lg);
         }
-        float lg = 0.f, bt = 1.f;
-        if (p.has_decay) {
-            lg = __ldg(p.g + t * Hv + h);
-            if (p.a_log) lg = -expf(__ldg(p.a_log + h)) * softplus20(lg + __ldg(p.dt_bias + h));
-        }
-        if (p.has_retrieval) {
-            bt = __ldg(p.beta + t * Hv + h);
-            if (p.beta_sigmoid) bt = sigmoidf_(bt);
-        }
-        const float gamma = expf(lg);
-        const float rg = p.has_retrieval ? gamma : 0.f;   // weight of the retrieval term
-        const int64_t vo = (t * Hv + h) * (int64_t)Dv;
+#pragma unroll
+        for (int j = 0; j < EPL; ++j)
+            kr[j] = PER_KEY ? (p.has_retrieval ? gam[j] * kx[j] : 0.f) : kx[j];
+        // weight of the retrieval term (per key it sits in kr)
+        const float rg = PER_KEY ? 1.f : (p.has_retrieval ? gam[0] : 0.f);
+
+        float pd[R], o[R];
 #pragma unroll
         for (int i = 0; i < R; ++i) {
-            const int row = row_base + i;
-            if (row >= Dv) break;  // uniform across the warp
-            const float vi = load_act<Tin>(vg + vo + row);
-            float pd = 0.f;
+            pd[i] = 0.f;
 #pragma unroll
-            for (int j = 0; j < EPL; ++j) pd += S[i][j] * kx[j];
-            pd = warp_sum(pd);
-            const float u = bt * (vi - rg * pd);
-            float o = 0.f;
+            for (int j = 0; j < EPL; ++j) pd[i] += S[i][j] * kr[j];
+        }
+#pragma unroll
+        for (int m = 1; m < 32; m <<= 1)
+#pragma unroll
+            for (int i = 0; i < R; ++i) pd[i] += __shfl_xor_sync(0xffffffffu, pd[i], m);
+#pragma unroll
+        for (int i = 0; i < R; ++i) {
+            const float u = PER_KEY ? bt * (vv[i] - pd[i]) : bt * (vv[i] - rg * pd[i]);
+            o[i] = 0.f;
 #pragma unroll
             for (int j = 0; j < EPL; ++j) {
-                S[i][j] = fmaf(kx[j], u, gamma * S[i][j]);
-                o += S[i][j] * qx[j];
+                S[i][j] = fmaf(kx[j], u, gam[PER_KEY ? j : 0] * S[i][j]);
+                o[i] += S[i][j] * qx[j];
             }
-            o = warp_sum(o);
-            if (lane == 0) store_act<Tin>(og + vo + row, p.scale * o);
         }
+#pragma unroll
+        for (int m = 1; m < 32; m <<= 1)
+#pragma unroll
+            for (int i = 0; i < R; ++i) o[i] += __shfl_xor_sync(0xffffffffu, o[i], m);
+        // lane i stores row row_base + i
+        float oi = o[0];
+#pragma unroll
+        for (int i = 1; i < R; ++i) oi = lane == i ? o[i] : oi;
+        if (lane < R && row_base + lane < Dv)
+            store_act<Tin>(og + (t * Hv + h) * (int64_t)Dv + row_base + lane, p.scale * oi);
     }
 
 #pragma unroll
