@@ -10,7 +10,9 @@ sets.  `value` is prefill tokens/s over all ranks.  After the K timed steps the
 same K-launch window is repeated until a quarter second of launches has been
 timed, so that the clock record covers a few dozen samples; the repeats are
 reported beside the measurement.  The long-context workload (B=1, S=32768) is
-timed the same way through the same call and reported under "long_prefill".
+timed the same way through the same call and reported under "long_prefill", and the
+ragged workload with a per-key-dimension decay (g of shape [N, Hv, Dk], the per-token
+kernel) under "prefill_per_key_decay".
 `roofline.bound` is the roof (tensor cores or HBM) whose ideal time is longer;
 both fractions are reported.  The same run
 then times gdn_decode over the state-pool workload (pool [1024,32,128,128]
@@ -89,7 +91,8 @@ def prefill_bytes(case):
     N = case.N
     Hq, Hv, Dk, Dv = case.dims
     esz = case.q.element_size()
-    b = N * (2 * Hq * Dk + 2 * Hv * Dv) * esz + N * Hv * 8  # q, k, v, out, g, beta
+    g_per_token = Hv * (Dk if case.g is not None and case.g.dim() == 3 else 1)
+    b = N * (2 * Hq * Dk + 2 * Hv * Dv) * esz + N * (g_per_token + Hv) * 4  # q, k, v, out, g, beta
     st = case.B * Hv * Dv * Dk * 4
     b += st * (2 if case.initial_state is not None else 1)
     if case.cu_seqlens is not None:
@@ -576,12 +579,16 @@ def prefill_roofline(gdn, case, launch_ms, peaks, sm_mhz, traffic):
     against it; both fractions are reported."""
     Hq, Hv, Dk, Dv = case.dims
     avg_s = statistics.mean(launch_ms) / 1e3
-    if not gdn.prefill_uses_chunked(case.q.dtype, Hv, Dk, Dv):
+    per_key = case.g is not None and case.g.dim() == 3
+    if not gdn.prefill_uses_chunked(case.q.dtype, Hv, Dk, Dv, decay_per_key=per_key):
         byts = prefill_bytes(case)
         ach = byts / avg_s / 1e9
         return {"kernel": "gdn_prefill_seq", "bound": "hbm", "achieved": ach,
                 "peak": peaks["hbm_gbs"], "unit": "GB/s", "frac": ach / peaks["hbm_gbs"],
-                "traffic": None, "peak_source": peaks["source"]}
+                "traffic": None, "algorithmic_bytes": byts, "ms_per_launch": avg_s * 1e3,
+                "peak_source": peaks["source"],
+                "note": "per-token recurrence: one dependent step per token per head, so its "
+                        "time follows the longest request, not the bytes"}
     flops = case.N * Hv * prefill_flops_per_token_head(Dk, Dv)
     byts = prefill_bytes(case)
     tc_peak, hbm_peak = peaks["bf16_tflops"], peaks["hbm_gbs"]
@@ -654,6 +661,8 @@ def main():
     ap.add_argument("--no-conv", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-long", action="store_true", help="skip the long-context prefill line")
+    ap.add_argument("--no-per-key", action="store_true",
+                    help="skip the per-key-dimension decay prefill line")
     ap.add_argument("--no-cpu", action="store_true", help="skip the CPU oracle baseline")
     ap.add_argument("--phase", default="all", choices=["all", "prefill", "decode", "conv"],
                     help="prefill or decode alone (for profiling); 'all' for the JSON line")
@@ -727,6 +736,21 @@ def main():
             "repeat_windows_ms_per_launch": time_prefill.repeats, "clocks": l_clocks}
         launches += time_prefill.launches
         del lcase
+
+    # the per-key-dimension decay over the ragged workload's shapes (per-token kernel)
+    per_key = None
+    if args.workload == "ragged" and not args.no_per_key:
+        pcase = workloads.ragged_prefill_case(decay_per_key=True)
+        p_steps = max(3, args.steps // 10)
+        p_total, p_launch = time_prefill(gdn, pcase, p_steps, args.warmup, world,
+                                         min_window_s=0.0)
+        p_max = max_over_ranks(p_total, world) / p_steps
+        per_key = {
+            "workload": pcase.name, "tokens": pcase.N, "steps": p_steps, "ms_per_step": p_max,
+            "value": job_throughput(pcase.N, world, p_max), "unit": "tokens/s",
+            "roofline": prefill_roofline(gdn, pcase, p_launch, peaks, None, None)}
+        launches += time_prefill.launches
+        del pcase
 
     decode = decode_mtp = None
     if not args.no_decode:
@@ -803,7 +827,8 @@ def main():
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
             "data": "synthetic", "config": dict(workload_config(case, args.workload),
                                                 parallelism=f"replicas{world}"),
-            "roofline": roof, "long_prefill": long_prefill, "decode": decode, "decode_mtp": decode_mtp, "conv1d": conv,
+            "roofline": roof, "long_prefill": long_prefill, "prefill_per_key_decay": per_key,
+            "decode": decode, "decode_mtp": decode_mtp, "conv1d": conv,
             "conv1d_decode": conv_dec,
             "e2e": e2e, "cpu_baseline": cpu,
             "clocks": prefill_clocks,
