@@ -55,6 +55,21 @@ const char *gdn_status_string(int32_t s)
     }
 }
 
+}  // extern "C"
+
+namespace {
+
+// the chunked tensor-core kernel takes the call: its own size/dtype rule, and a scalar decay
+// (the per-key-dimension spelling runs the per-token kernel)
+bool chunked_path(const GdnPrefillArgs &a)
+{
+    return !a.g_per_key && prefill_chunked_supported(a);
+}
+
+}  // namespace
+
+extern "C" {
+
 int32_t gdn_prefill_uses_chunked(gdn_dtype dtype, int32_t Hv, int32_t Dk, int32_t Dv,
                                  uint32_t flags)
 {
@@ -63,7 +78,7 @@ int32_t gdn_prefill_uses_chunked(gdn_dtype dtype, int32_t Hv, int32_t Dk, int32_
     memset(&a, 0, sizeof(a));
     a.dtype = dtype; a.Dk = Dk; a.Dv = Dv; a.Hq = 1; a.Hv = Hv;
     a.g_per_key = (flags & GDN_DECAY_PER_KEY) ? 1 : 0;
-    return prefill_chunked_supported(a) ? 1 : 0;
+    return chunked_path(a) ? 1 : 0;
 }
 
 }  // extern "C"
@@ -157,7 +172,7 @@ gdn_status prefill_impl(const void *q, const void *k, const void *v, const float
 
     // workspace of the sequence-parallel split: used only when the call can split and the
     // chunked kernel runs; then it must be large enough, aligned, and overlap nothing
-    if (workspace && !(flags & GDN_PREFILL_SEQUENTIAL) && prefill_chunked_supported(a)) {
+    if (workspace && !(flags & GDN_PREFILL_SEQUENTIAL) && chunked_path(a)) {
         const uint64_t need = prefill_split_workspace_bytes(a);
         if (need > 0) {
             if (workspace_bytes < need) return GDN_ERR_SHAPE;
@@ -177,7 +192,7 @@ gdn_status prefill_impl(const void *q, const void *k, const void *v, const float
 
     cudaStream_t s = (cudaStream_t)stream;
     cudaError_t e;
-    if (!(flags & GDN_PREFILL_SEQUENTIAL) && prefill_chunked_supported(a))
+    if (!(flags & GDN_PREFILL_SEQUENTIAL) && chunked_path(a))
         e = launch_prefill_chunked(a, s);
     else
         e = launch_prefill_sequential(a, s);
@@ -220,7 +235,7 @@ uint64_t gdn_prefill_workspace_size(int32_t B, int64_t N, int32_t Hq, int32_t Hv
     if ((flags & GDN_PREFILL_SEQUENTIAL) || B < 1 || Hq < 1 || Hv < 1 || Hv % Hq != 0 || N < 0)
         return 0;
     const GdnPrefillArgs a = prefill_shape(B, N, Hq, Hv, Dk, Dv, dtype, flags);
-    if ((flags & GDN_GATE_QWEN) || !prefill_chunked_supported(a)) return 0;
+    if ((flags & GDN_GATE_QWEN) || !chunked_path(a)) return 0;
     return prefill_split_workspace_bytes(a);
 }
 

@@ -1717,7 +1717,7 @@ int num_sms()
 bool prefill_chunked_supported(const GdnPrefillArgs &a)
 {
     return (a.dtype == GDN_BF16 || a.dtype == GDN_F16) && a.Dk >= 1 && a.Dk <= 128 &&
-           a.Dv >= 1 && a.Dv <= 128 && !a.g_per_key && get_encode() != nullptr;
+           a.Dv >= 1 && a.Dv <= 128 && get_encode() != nullptr;
 }
 
 static bool prefill_needs_plain_staging(const GdnPrefillArgs &a)
