@@ -206,5 +206,8 @@ bool prefill_chunked_supported(const GdnPrefillArgs &a);
 // bytes of workspace with which gdn_prefill may split long requests (0: never splits)
 uint64_t prefill_split_workspace_bytes(const GdnPrefillArgs &a);
 cudaError_t launch_seq_compose(const GdnPrefillArgs &a, void *workspace, int G, cudaStream_t stream);
+// the chunked tensor-core kernel for the per-key-dimension decay (prefill_kd.cu)
+bool prefill_kd_supported(const GdnPrefillArgs &a);
+cudaError_t launch_prefill_kd(const GdnPrefillArgs &a, cudaStream_t stream);
 // records a CUDA failure for gdn_last_error() and returns GDN_ERR_CUDA
 gdn_status gdn_report_cuda_failure(cudaError_t e, const char *where);

@@ -60,7 +60,7 @@ const char *gdn_status_string(int32_t s)
 namespace {
 
 // the chunked tensor-core kernel takes the call: its own size/dtype rule, and a scalar decay
-// (the per-key-dimension spelling runs the per-token kernel)
+// (the per-key-dimension spelling has a tensor-core kernel of its own, prefill_kd.cu)
 bool chunked_path(const GdnPrefillArgs &a)
 {
     return !a.g_per_key && prefill_chunked_supported(a);
@@ -78,7 +78,8 @@ int32_t gdn_prefill_uses_chunked(gdn_dtype dtype, int32_t Hv, int32_t Dk, int32_
     memset(&a, 0, sizeof(a));
     a.dtype = dtype; a.Dk = Dk; a.Dv = Dv; a.Hq = 1; a.Hv = Hv;
     a.g_per_key = (flags & GDN_DECAY_PER_KEY) ? 1 : 0;
-    return chunked_path(a) ? 1 : 0;
+    a.has_decay = 1;   // the per-key spelling always comes with a decay input
+    return (chunked_path(a) || prefill_kd_supported(a)) ? 1 : 0;
 }
 
 }  // extern "C"
@@ -194,6 +195,8 @@ gdn_status prefill_impl(const void *q, const void *k, const void *v, const float
     cudaError_t e;
     if (!(flags & GDN_PREFILL_SEQUENTIAL) && chunked_path(a))
         e = launch_prefill_chunked(a, s);
+    else if (!(flags & GDN_PREFILL_SEQUENTIAL) && prefill_kd_supported(a))
+        e = launch_prefill_kd(a, s);
     else
         e = launch_prefill_sequential(a, s);
     if (e != cudaSuccess) return cuda_fail(e, "gdn_prefill launch");

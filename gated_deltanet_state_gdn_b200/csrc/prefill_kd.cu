@@ -1,0 +1,883 @@
+// prefill_kd.cu -- chunked prefill with a per-key-dimension decay on sm_100a tensor cores.
+//
+// Operation: the recurrence of "com.microsoft.GatedDeltaNet" (Description) with `decay`
+// in its per-key-dimension spelling (Inputs table, shape (..., num_heads_v, head_size_qk)),
+// read as D_t = diag(exp(g_t)) on the key axis of the state:
+//   S_t = D_t S_{t-1} + k_t (beta_t (v_t - (D_t S_{t-1})^T k_t))^T,   o_t = scale S_t^T q_t.
+// bf16 q/k/v with 8 <= Dk, Dv <= 128 (zero-padded to 128-wide tiles), 64 tokens a chunk.
+// The scaled operands below reach 2^104, beyond fp16's exponent range (2^15), so fp16
+// activations take the per-token kernel; bf16 has fp32's exponent range.  Every operand
+// here carries one bf16 rounding of a decayed product (the scalar-decay kernel feeds the raw
+// bytes and decays in fp32 after the MMA); heads narrower than 8 have no rows to average that
+// over and no tensor-core work worth the rounding, so they take the per-token fp32 kernel.
+//
+// Chunk form (derived from the recurrence as for the scalar decay, with every decay factor
+// now a vector over the key dimensions).  For a chunk with incoming state S0 (Dk x Dv),
+// per-dimension cumulative log-decay G_i = sum_{l<=i} g_l, normalised rows k^_i, q^_i:
+//   A_ij = beta_i sum_d k^_i[d] k^_j[d] e^{G_i[d] - G_j[d]}  (j < i),   T = (I + A)^-1
+//   P_ij = sum_d q^_i[d] k^_j[d] e^{G_i[d] - G_j[d]}          (j <= i)
+//   W = T diag(beta) (K^ * e^G),   U~ = T diag(beta) V,   U = U~ - W S0
+//   O = scale ((Q^ * e^G) S0 + P U)
+//   S_C = diag(e^{G_C}) S0 + (K^ * e^{G_C - G})^T U
+// The decay sits inside the contractions of A and P, so it is split between the two
+// operands relative to a reference.  Each 16-token block I of the chunk takes as reference
+// M_I = G at its eighth token: the row operand is x_i * e^{G_i - M_I} (one tile for all
+// rows), the key operand of block I is k^_j * e^{M_I - G_j} for every j up to the block's
+// end, and the four key operands are stacked into one 160-row tile, so a single MMA
+// (N = 160) gives every block's products at once.  Every factor stays within 2^104 once
+// each per-dimension log-decay is floored at -9 (at most 8 tokens lie between a token and
+// its reference, 8 * 9 * log2(e) < 104): the products that are used are <= 1, the others
+// (j > i) are masked out by selection.  The floor changes a per-token decay factor below
+// e^-9 ~ 1.2e-4 into 1.2e-4, far below the bf16 operand rounding.
+// All state-dependent products are evaluated transposed (rows = value index dv, M = 128):
+//   (G)  [K^;Q^]*e^{G-M} x Bcat^T  -> TMEM (128 x 160)
+//   (W)  W^T = (K^ e^G)^T Tb^T      (U~) U~^T = V^T Tb^T,   Tb = T diag(beta)
+//   (1a) U^T += S^T (-W)^T          (1b) Y = S^T (Q^ e^G)^T
+//   (2)  S^T = S^T diag(e^{G_C}) + U^T (K^ e^{G_C - G})
+//   (3)  Z = U^T P^T                O^T = scale (Y + Z)
+//
+// One CTA of 128 threads per (request, value head); thread t owns TMEM lane t (the state
+// row dv = t).  The phases of a chunk run one after another (plain loads stage and scale the
+// operand tiles, thread 0 issues the MMAs, a bounded wait on one mbarrier ends each group).
+// The triangular solve works on 16 x 16 blocks: fp32 forward substitution inside the four
+// diagonal blocks, then tf32 warp MMAs merge the blocks below the diagonal.
+#include <cuda_fp16.h>
+
+#include "common.cuh"
+#include "sm100.cuh"
+
+using namespace sm100;
+
+namespace gdn_kd {
+
+constexpr int C = 64;            // chunk length (tokens)
+constexpr int NT = 128;          // threads per CTA
+constexpr float G_FLOOR = -9.f;  // per-dimension log-decay floor
+constexpr float LOG2E = 1.4426950408889634f;
+
+// ---- shared memory (bytes from a 1024-aligned base) ----
+// region Y: the Gram operands, then (after the Gram) P, -W and the bf16 U
+constexpr uint32_t OFF_ASIDE = 0;        // [kb 2][128 rows: K^ 0-63, Q^ 64-127][128 B], kb 16384
+constexpr uint32_t ASIDE_KB = 16384;
+constexpr uint32_t OFF_BCAT = 32768;     // [kb 2][160 rows][128 B], kb 20480
+constexpr uint32_t BCAT_KB = 20480;
+constexpr uint32_t OFF_P = 0;            // [64 rows i][64 j], K-major
+constexpr uint32_t OFF_WNEG = 8192;      // [128 rows dk][64 i], MN-major B of (1a)
+constexpr uint32_t OFF_UB = 24576;       // [128 rows dv][64 j], K-major A of (2), (3)
+// region Z: decayed operands and v
+constexpr uint32_t OFF_KG = 73728;       // K^ e^G        [kb 2][64 rows j][128 B], kb 8192
+constexpr uint32_t OFF_QG = 90112;       // Q^ e^G
+constexpr uint32_t OFF_KD = 106496;      // K^ e^{G_C-G}
+constexpr uint32_t OFF_VT = 122880;      // v             [dv half 2][64 rows j][128 B]
+constexpr uint32_t TILE_KB = 8192;
+constexpr uint32_t OFF_SB = 139264;      // bf16 S^T      [kb 2][128 rows dv][128 B], kb 16384
+// region X: log-decays, then (after the operands are built) A and Tb
+constexpr uint32_t OFF_G2 = 172032;      // fp32 [64][128]: G * log2(e)
+constexpr uint32_t OFF_A = 172032;       // solve area: 16 fp32 blocks of 16 x SOLVE_LD
+constexpr uint32_t SOLVE_LD = 20;        // padded row stride (floats)
+constexpr uint32_t SOLVE_BLK = 16 * SOLVE_LD;
+constexpr uint32_t OFF_TB = 192512;      // [64 rows i][64 j], K-major B of (W), (U~)
+constexpr uint32_t OFF_VEC = 204800;     // per-dimension vectors, fp32
+constexpr int VEC_EM = 0;        // e^{M_I}                 [4][128]
+constexpr int VEC_CM = 512;      // e^{M_I' - M_I}, I' > I  [6][128]
+constexpr int VEC_EC3 = 1280;    // e^{G_C - M_3}           [128]
+constexpr int VEC_GC = 1408;     // e^{G_C}                 [128]
+constexpr int VEC_M2 = 1536;     // M_I * log2(e)           [4][128]
+constexpr uint32_t OFF_ROW = OFF_VEC + 2048 * 4;   // per-token values, fp32
+constexpr int ROW_BETA = 0, ROW_QK = 64;   // beta_j; rq_j rk_j (q_j . k_j)
+constexpr uint32_t OFF_BAR = OFF_ROW + 1024;       // mbarrier, TMEM base, flag
+constexpr uint32_t SMEM_USED = OFF_BAR + 64;
+constexpr uint32_t SMEM_BYTES = SMEM_USED + 1024;  // + alignment slack
+static_assert(SMEM_BYTES <= 232448, "shared memory budget");
+static_assert(OFF_BCAT + 2 * BCAT_KB <= OFF_KG && OFF_UB + 16384 <= OFF_KG, "region Y");
+static_assert(OFF_A + 16 * SOLVE_BLK * 4 <= OFF_TB && OFF_TB + 8192 <= OFF_VEC &&
+              OFF_G2 + 64 * 128 * 4 <= OFF_VEC, "region X");
+static_assert(OFF_TB % 1024 == 0 && OFF_SB % 1024 == 0 && OFF_VT % 1024 == 0 &&
+              OFF_BCAT % 1024 == 0 && OFF_KD % 1024 == 0, "swizzled tiles need 1024 alignment");
+
+// TMEM columns: the Gram's 160 columns are reused by W and U once A and P are read
+constexpr uint32_t TM_S = 0, TM_G = 128, TM_W = 128, TM_U = 192, TM_Y = 288, TM_Z = 352;
+
+__device__ __forceinline__ uint32_t sw128(uint32_t row, uint32_t c)
+{
+    return row * 128u + ((c ^ (row & 7u)) << 4);
+}
+
+template <bool F16>
+__device__ __forceinline__ uint32_t pack2(float lo, float hi)
+{
+    if constexpr (F16) {
+        const __half2 v = __floats2half2_rn(lo, hi);
+        return *reinterpret_cast<const uint32_t *>(&v);
+    } else {
+        return gdn::pack_bf16x2(lo, hi);
+    }
+}
+
+template <bool F16>
+__device__ __forceinline__ uint4 pack8(const float *x)
+{
+    return make_uint4(pack2<F16>(x[0], x[1]), pack2<F16>(x[2], x[3]), pack2<F16>(x[4], x[5]),
+                      pack2<F16>(x[6], x[7]));
+}
+
+template <bool F16>
+__device__ __forceinline__ float to_f(uint16_t b)
+{
+    if constexpr (F16) return __half2float(*reinterpret_cast<const __half *>(&b));
+    else return __uint_as_float((uint32_t)b << 16);
+}
+
+template <bool F16>
+__device__ __forceinline__ uint16_t elem16(float x)
+{
+    if constexpr (F16) {
+        const __half v = __float2half_rn(x);
+        return *reinterpret_cast<const uint16_t *>(&v);
+    } else {
+        const __nv_bfloat16 v = __float2bfloat16_rn(x);
+        return *reinterpret_cast<const uint16_t *>(&v);
+    }
+}
+
+// 16-byte global -> shared asynchronous copy (both addresses 16-byte aligned)
+__device__ __forceinline__ void cp_async16(uint32_t dst, const void *src)
+{
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
+}
+
+__device__ __forceinline__ void cp_async_wait_all()
+{
+    asm volatile("cp.async.wait_all;" ::: "memory");
+}
+
+// elements [8c, 8c + 8) of a row of `n` 16-bit values (zero past n); `vec`: the row start is
+// 16-byte aligned and n % 8 == 0
+template <bool F16>
+__device__ __forceinline__ void load8(const uint16_t *row, int c, int n, bool vec, float (&x)[8])
+{
+    if (vec) {
+        if (8 * c < n) {
+            const uint4 r = __ldg(reinterpret_cast<const uint4 *>(row) + c);
+            const uint32_t w[4] = {r.x, r.y, r.z, r.w};
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                x[2 * e] = to_f<F16>((uint16_t)(w[e] & 0xffffu));
+                x[2 * e + 1] = to_f<F16>((uint16_t)(w[e] >> 16));
+            }
+            return;
+        }
+#pragma unroll
+        for (int e = 0; e < 8; ++e) x[e] = 0.f;
+        return;
+    }
+#pragma unroll
+    for (int e = 0; e < 8; ++e) x[e] = (8 * c + e < n) ? to_f<F16>(row[8 * c + e]) : 0.f;
+}
+
+// the bits of elements [8c, 8c + 8) of a row of `n` 16-bit values (zero past n)
+__device__ __forceinline__ uint4 load_raw8(const uint16_t *row, int c, int n, bool vec)
+{
+    if (vec) return 8 * c < n ? __ldg(reinterpret_cast<const uint4 *>(row) + c) : make_uint4(0u, 0u, 0u, 0u);
+    uint32_t w[4];
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+        const int d = 8 * c + 2 * e;
+        const uint32_t lo = d < n ? row[d] : 0u, hi = d + 1 < n ? row[d + 1] : 0u;
+        w[e] = lo | (hi << 16);
+    }
+    return make_uint4(w[0], w[1], w[2], w[3]);
+}
+
+template <bool F16>
+__device__ __forceinline__ void unpack8(uint4 r, float (&x)[8])
+{
+    const uint32_t w[4] = {r.x, r.y, r.z, r.w};
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+        x[2 * e] = to_f<F16>((uint16_t)(w[e] & 0xffffu));
+        x[2 * e + 1] = to_f<F16>((uint16_t)(w[e] >> 16));
+    }
+}
+
+// one state row (32 fp32 columns of block `blk`) into the bf16 S^T tile (K-major, dk across)
+template <bool F16>
+__device__ __forceinline__ void store_sb(uint8_t *sb, int dv, int blk, const float (&x)[32])
+{
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+        const int ch = 4 * (blk & 1) + q;   // 16-byte chunk within the 64-dk k-block
+        *reinterpret_cast<uint4 *>(sb + (blk >> 1) * 16384 + sw128(dv, ch)) = pack8<F16>(x + 8 * q);
+    }
+}
+
+// ---- blocked solve of T = (I + A)^-1 (A strictly lower, 4 x 4 blocks of 16)
+// slots of the solve area: 0-3 A_II, 4 A_10, 5 A_32, 6-9 A_20 A_21 A_30 A_31 (later the
+// products X), 10-13 D_I = (I + A_II)^-1, 14 T_10, 15 T_32
+__host__ __device__ constexpr int a_slot(int I, int J)
+{
+    return I == 1 ? 4 : (I == 2 ? 6 + J : (J == 2 ? 5 : 8 + J));
+}
+
+// acc[nh][.] += X(16x16) * Y(16x16) on padded fp32 blocks, tf32 inputs (mma.m16n8k8 fragments)
+__device__ __forceinline__ void blk_mma(float (&acc)[2][4], const float *X, const float *Y)
+{
+    const int lane = threadIdx.x & 31;
+    const int g = lane >> 2, t = lane & 3;
+#pragma unroll
+    for (int kh = 0; kh < 2; ++kh) {
+        uint32_t a[4];
+        a[0] = __float_as_uint(X[g * SOLVE_LD + 8 * kh + t]);
+        a[1] = __float_as_uint(X[(g + 8) * SOLVE_LD + 8 * kh + t]);
+        a[2] = __float_as_uint(X[g * SOLVE_LD + 8 * kh + t + 4]);
+        a[3] = __float_as_uint(X[(g + 8) * SOLVE_LD + 8 * kh + t + 4]);
+#pragma unroll
+        for (int nh = 0; nh < 2; ++nh) {
+            uint32_t b[2];
+            b[0] = __float_as_uint(Y[(8 * kh + t) * SOLVE_LD + 8 * nh + g]);
+            b[1] = __float_as_uint(Y[(8 * kh + t + 4) * SOLVE_LD + 8 * nh + g]);
+            mma_tf32_16x8x8(acc[nh], a, b);
+        }
+    }
+}
+
+__device__ __forceinline__ void blk_store(float *Z, const float (&acc)[2][4], float sgn)
+{
+    const int lane = threadIdx.x & 31;
+    const int g = lane >> 2, t = lane & 3;
+#pragma unroll
+    for (int nh = 0; nh < 2; ++nh) {
+        *reinterpret_cast<float2 *>(Z + g * SOLVE_LD + 8 * nh + 2 * t) =
+            make_float2(sgn * acc[nh][0], sgn * acc[nh][1]);
+        *reinterpret_cast<float2 *>(Z + (g + 8) * SOLVE_LD + 8 * nh + 2 * t) =
+            make_float2(sgn * acc[nh][2], sgn * acc[nh][3]);
+    }
+}
+
+// block (I, J) of T (times sgn) into Tb = T diag(beta) (bf16, K-major, 128B-swizzled)
+template <bool F16>
+__device__ __forceinline__ void blk_store_tb(const float (&acc)[2][4], float sgn, int I, int J,
+                                             const float *beta, uint8_t *tb)
+{
+    const int lane = threadIdx.x & 31;
+    const int g = lane >> 2, t = lane & 3;
+#pragma unroll
+    for (int nh = 0; nh < 2; ++nh) {
+        const int j = 16 * J + 8 * nh + 2 * t;
+        const float b0 = beta[j], b1 = beta[j + 1];
+#pragma unroll
+        for (int hh = 0; hh < 2; ++hh) {
+            const uint32_t off = sw128(16 * I + g + 8 * hh, j >> 3) + (uint32_t)(j & 7) * 2u;
+            *reinterpret_cast<uint32_t *>(tb + off) =
+                pack2<F16>(sgn * acc[nh][2 * hh] * b0, sgn * acc[nh][2 * hh + 1] * b1);
+        }
+    }
+}
+
+// thread 0 waits (bounded) for the MMA group committed to `bar`; every thread gets the outcome
+__device__ __forceinline__ bool cta_wait_mma(uint32_t bar, uint32_t &phase, volatile int *flag,
+                                             int32_t *status)
+{
+    if (threadIdx.x == 0) {
+        bool good = mbar_try_wait(bar, phase & 1);
+        if (!good) {
+            const long long t0 = clock64();
+            while (!(good = mbar_try_wait(bar, phase & 1)))
+                if (clock64() - t0 > (1ll << 31)) break;
+        }
+        if (!good && status) atomicOr(status, GDN_DEV_TIMEOUT);
+        *flag = good ? 1 : 0;
+    }
+    ++phase;
+    __syncthreads();
+    const bool good = *flag != 0;
+    tc_fence_after();
+    return good;
+}
+
+template <bool F16>
+__global__ void __launch_bounds__(NT, 1) gdn_prefill_kd_kernel(const __grid_constant__ GdnPrefillArgs p)
+{
+    extern __shared__ uint8_t smem_raw[];
+    const uint32_t raw_base = smem_u32(smem_raw);
+    uint8_t *smem = smem_raw + ((1024u - (raw_base & 1023u)) & 1023u);
+    const uint32_t sbase = smem_u32(smem);
+    const int tid = threadIdx.x, warp = tid >> 5;
+    const int Hv = p.Hv, Hq = p.Hq, Dk = p.Dk, Dv = p.Dv;
+    const int b = blockIdx.x / Hv, h = blockIdx.x - b * Hv;
+    const int qh = (int)(((int64_t)h * Hq) / Hv);
+    const bool retrieval = p.has_retrieval != 0;
+
+    int64_t start, end;
+    if (p.cu_seqlens) {
+        start = gdn::clamp_i64(p.cu_seqlens[b], 0, p.N);
+        end = gdn::clamp_i64(p.cu_seqlens[b + 1], 0, p.N);
+    } else {
+        const int64_t S = p.N / p.B;
+        start = (int64_t)b * S;
+        end = start + S;
+    }
+    const int len = end > start ? (int)(end - start) : 0;
+    const int nc = (len + C - 1) / C;
+    const int64_t soff = ((int64_t)b * Hv + h) * Dv * (int64_t)Dk;
+    if constexpr (gdn::kChecked) {
+        if (!gdn::in_range(start, len, p.N, p.dev_status) || !gdn::in_range(qh, 1, Hq, p.dev_status) ||
+            !gdn::in_range(soff, (int64_t)Dv * Dk, (int64_t)p.B * Hv * Dv * Dk, p.dev_status))
+            return;
+    }
+
+    const uint16_t *kg = static_cast<const uint16_t *>(p.k);
+    const uint16_t *qg = static_cast<const uint16_t *>(p.q);
+    const uint16_t *vg = static_cast<const uint16_t *>(p.v);
+    uint16_t *og = static_cast<uint16_t *>(p.out);
+    const bool kvec = (Dk & 7) == 0, vvec = (Dv & 7) == 0;
+
+    const uint32_t bar = sbase + OFF_BAR;
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + OFF_BAR + 8);
+    volatile int *flag = reinterpret_cast<volatile int *>(smem + OFF_BAR + 12);
+    float *G2 = reinterpret_cast<float *>(smem + OFF_G2);
+    float *solve = reinterpret_cast<float *>(smem + OFF_A);
+    float *vec = reinterpret_cast<float *>(smem + OFF_VEC);
+    float *rowv = reinterpret_cast<float *>(smem + OFF_ROW);
+
+    if (tid == 0) {
+        mbar_init(bar, 1);
+        fence_mbar_init();
+        *flag = 1;
+    }
+    if (warp == 0) {
+        tmem_alloc(sbase + OFF_BAR + 8, 512);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+    const uint32_t tl = tmem + ((uint32_t)(32 * warp) << 16);   // this warp's TMEM lanes
+    uint32_t phase = 0;
+
+    // state S^T (row dv = tid) into TMEM, and its bf16 copy
+    {
+        float x[32];
+#pragma unroll 1
+        for (int blk = 0; blk < 4; ++blk) {
+#pragma unroll
+            for (int e = 0; e < 32; ++e) {
+                const int dk = 32 * blk + e;
+                x[e] = (p.initial_state && tid < Dv && dk < Dk) ? p.initial_state[soff + (int64_t)tid * Dk + dk] : 0.f;
+            }
+            tmem_st32(tl + TM_S + 32 * blk, x);
+            store_sb<F16>(smem + OFF_SB, tid, blk, x);
+        }
+        tmem_wait_st();
+    }
+    fence_proxy_async_smem();
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+
+    constexpr uint32_t ID_G = idesc_f16kind(128, 160, 0, 0, !F16);
+    constexpr uint32_t ID_WU = idesc_f16kind(128, 64, 1, 0, !F16);
+    constexpr uint32_t ID_1A = idesc_f16kind(128, 64, 0, 1, !F16);
+    constexpr uint32_t ID_1B = idesc_f16kind(128, 64, 0, 0, !F16);
+    constexpr uint32_t ID_2 = idesc_f16kind(128, 128, 0, 1, !F16);
+    constexpr uint32_t ID_3 = idesc_f16kind(128, 64, 0, 0, !F16);
+
+    bool ok = true;
+    for (int n = 0; n < nc && ok; ++n) {
+        const int64_t t0 = start + (int64_t)n * C;
+        const int ln = min(C, len - n * C);
+
+        // ---- raw rows of the chunk, unit (token j, 8 dimensions 8c..8c+7), 8 units per thread,
+        //      all requested at once so that their latency overlaps the decay staging below
+        uint4 rk8[8], rq8[8], rv8[8];
+#pragma unroll
+        for (int it = 0; it < 8; ++it) {
+            const int u = tid + NT * it, j = u >> 4, c = u & 15;
+            if (j < ln) {
+                const int64_t qk = ((t0 + j) * Hq + qh) * (int64_t)Dk;
+                rk8[it] = load_raw8(kg + qk, c, Dk, kvec);
+                rq8[it] = load_raw8(qg + qk, c, Dk, kvec);
+                rv8[it] = load_raw8(vg + ((t0 + j) * Hv + h) * (int64_t)Dv, c, Dv, vvec);
+            } else {
+                rk8[it] = rq8[it] = rv8[it] = make_uint4(0u, 0u, 0u, 0u);
+            }
+        }
+        // ---- the chunk's raw log-decays into G2 (rows of Dk floats; asynchronous 16-byte
+        //      copies when rows are 16-byte multiples), zero past the request and past Dk
+        if ((Dk & 3) == 0) {
+            const int pieces = Dk >> 2;   // 16-byte pieces per row
+            for (int u = tid; u < C * 32; u += NT) {
+                const int i = u >> 5, c4 = u & 31;
+                float *dst = G2 + i * 128 + 4 * c4;
+                if (i < ln && c4 < pieces)
+                    cp_async16(smem_u32(dst), p.g + ((t0 + i) * Hv + h) * (int64_t)Dk + 4 * c4);
+                else
+                    *reinterpret_cast<float4 *>(dst) = make_float4(0.f, 0.f, 0.f, 0.f);
+            }
+            cp_async_wait_all();
+        } else {
+            for (int u = tid; u < C * 128; u += NT) {
+                const int i = u >> 7, d = u & 127;
+                G2[u] = (i < ln && d < Dk) ? __ldg(p.g + ((t0 + i) * Hv + h) * (int64_t)Dk + d) : 0.f;
+            }
+        }
+        __syncthreads();
+        // ---- per-dimension cumulative log-decay (thread = key dimension), in place
+        {
+            const int d = tid;
+            const float ea = p.a_log ? expf(__ldg(p.a_log + h)) : 0.f;
+            const float dtb = p.a_log ? __ldg(p.dt_bias + h) : 0.f;
+            float acc = 0.f;
+#pragma unroll 8
+            for (int i = 0; i < C; ++i) {
+                float g = G2[i * 128 + d];
+                if (i < ln && d < Dk) {
+                    if (p.a_log) g = -ea * gdn::softplus20(g + dtb);
+                    g = fmaxf(g, G_FLOOR);
+                }
+                acc += g;
+                G2[i * 128 + d] = acc * LOG2E;
+            }
+        }
+        if (tid < C) {
+            float bt = 0.f;
+            if (tid < ln) {
+                bt = retrieval ? __ldg(p.beta + (t0 + tid) * Hv + h) : 1.f;
+                if (retrieval && p.beta_sigmoid) bt = gdn::sigmoidf_(bt);
+            }
+            rowv[ROW_BETA + tid] = bt;
+        }
+        __syncthreads();
+        {
+            const int d = tid;
+            float m2[4];
+#pragma unroll
+            for (int I = 0; I < 4; ++I) m2[I] = G2[(16 * I + 7) * 128 + d];
+            const float gc = G2[63 * 128 + d];
+#pragma unroll
+            for (int I = 0; I < 4; ++I) {
+                vec[VEC_EM + I * 128 + d] = ex2_approx(m2[I]);
+                vec[VEC_M2 + I * 128 + d] = m2[I];
+            }
+#pragma unroll
+            for (int I2 = 1; I2 < 4; ++I2)
+#pragma unroll
+                for (int I = 0; I < I2; ++I)
+                    vec[VEC_CM + (I2 * (I2 - 1) / 2 + I) * 128 + d] = ex2_approx(m2[I2] - m2[I]);
+            vec[VEC_EC3 + d] = ex2_approx(gc - m2[3]);
+            vec[VEC_GC + d] = ex2_approx(gc);
+        }
+        __syncthreads();
+
+        // ---- operand tiles from the raw rows; a row's 16 units sit on 16 consecutive lanes,
+        //      so its norms come from a 16-lane reduction.  q_j . k_j (from the raw bytes) is
+        //      kept for the diagonal of P: its decay factor is 1, and taken from the
+        //      bf16-rounded decayed operands its value would carry their rounding relative to
+        //      |q^||k^| rather than to the product, which near-orthogonal q and k make small.
+#pragma unroll
+        for (int it = 0; it < 8; ++it) {
+            const int u = tid + NT * it, j = u >> 4, c = u & 15;
+            const int I = j >> 4;
+            float kx[8], qx[8], vx[8];
+            unpack8<F16>(rk8[it], kx);
+            unpack8<F16>(rq8[it], qx);
+            unpack8<F16>(rv8[it], vx);
+            float ssk = 0.f, ssq = 0.f, sqk = 0.f;
+#pragma unroll
+            for (int e = 0; e < 8; ++e) {
+                ssk = fmaf(kx[e], kx[e], ssk);
+                ssq = fmaf(qx[e], qx[e], ssq);
+                sqk = fmaf(qx[e], kx[e], sqk);
+            }
+#pragma unroll
+            for (int m = 1; m < 16; m <<= 1) {
+                ssk += __shfl_xor_sync(0xffffffffu, ssk, m);
+                ssq += __shfl_xor_sync(0xffffffffu, ssq, m);
+                sqk += __shfl_xor_sync(0xffffffffu, sqk, m);
+            }
+            const float rk = p.qk_l2norm ? 1.0f / sqrtf(ssk + 1e-12f) : 1.f;
+            const float rq = p.qk_l2norm ? 1.0f / sqrtf(ssq + 1e-12f) : 1.f;
+            if (c == 0) rowv[ROW_QK + j] = rq * rk * sqk;
+
+            float g2[8], mI[8], em[8];
+            {
+                const float4 a0 = *reinterpret_cast<const float4 *>(G2 + j * 128 + 8 * c);
+                const float4 a1 = *reinterpret_cast<const float4 *>(G2 + j * 128 + 8 * c + 4);
+                g2[0] = a0.x; g2[1] = a0.y; g2[2] = a0.z; g2[3] = a0.w;
+                g2[4] = a1.x; g2[5] = a1.y; g2[6] = a1.z; g2[7] = a1.w;
+            }
+#pragma unroll
+            for (int e = 0; e < 8; ++e) {
+                mI[e] = vec[VEC_M2 + I * 128 + 8 * c + e];
+                em[e] = vec[VEC_EM + I * 128 + 8 * c + e];
+            }
+            float ak[8], aq[8], kgm[8], qgm[8], bk[8];
+#pragma unroll
+            for (int e = 0; e < 8; ++e) {
+                const float f = ex2_approx(g2[e] - mI[e]);    // e^{G_j - M_I}
+                const float kh = kx[e] * rk;
+                ak[e] = kh * f;
+                aq[e] = qx[e] * rq * f;
+                kgm[e] = ak[e] * em[e];                        // k^ e^{G_j}
+                qgm[e] = aq[e] * em[e];
+                bk[e] = kh * ex2_approx(mI[e] - g2[e]);        // k^ e^{M_I - G_j}
+            }
+            const uint32_t kb = (uint32_t)(c >> 3) , ch = (uint32_t)(c & 7);
+            *reinterpret_cast<uint4 *>(smem + OFF_ASIDE + kb * ASIDE_KB + sw128(j, ch)) = pack8<F16>(ak);
+            *reinterpret_cast<uint4 *>(smem + OFF_ASIDE + kb * ASIDE_KB + sw128(64 + j, ch)) = pack8<F16>(aq);
+            *reinterpret_cast<uint4 *>(smem + OFF_KG + kb * TILE_KB + sw128(j, ch)) = pack8<F16>(kgm);
+            *reinterpret_cast<uint4 *>(smem + OFF_QG + kb * TILE_KB + sw128(j, ch)) = pack8<F16>(qgm);
+            *reinterpret_cast<uint4 *>(smem + OFF_VT + kb * TILE_KB + sw128(j, ch)) = pack8<F16>(vx);
+            // key operand of every block I2 >= I: k^ e^{M_I2 - G_j} = bk e^{M_I2 - M_I}; the
+            // last one also gives k^ e^{G_C - G_j} = k^ e^{M_3 - G_j} e^{G_C - M_3}
+#pragma unroll 1
+            for (int I2 = I; I2 < 4; ++I2) {
+                float bb[8];
+#pragma unroll
+                for (int e = 0; e < 8; ++e)
+                    bb[e] = I2 == I ? bk[e] : bk[e] * vec[VEC_CM + (I2 * (I2 - 1) / 2 + I) * 128 + 8 * c + e];
+                const int row = 8 * I2 * (I2 + 1) + j;   // 16 * I2 (I2 + 1) / 2 + j
+                *reinterpret_cast<uint4 *>(smem + OFF_BCAT + kb * BCAT_KB + sw128(row, ch)) = pack8<F16>(bb);
+                if (I2 == 3) {
+                    float kd[8];
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) kd[e] = bb[e] * vec[VEC_EC3 + 8 * c + e];
+                    *reinterpret_cast<uint4 *>(smem + OFF_KD + kb * TILE_KB + sw128(j, ch)) = pack8<F16>(kd);
+                }
+            }
+        }
+        fence_proxy_async_smem();
+        __syncthreads();
+
+        // ---- (G): all blocks' products in one MMA
+        if (tid == 0) {
+            tc_fence_after();
+            const uint64_t dA = sdesc_sw128(sbase + OFF_ASIDE, 16, 1024);
+            const uint64_t dB = sdesc_sw128(sbase + OFF_BCAT, 16, 1024);
+#pragma unroll 1
+            for (int kk = 0; kk < 8; ++kk)
+                umma_bf16(tmem + TM_G, dA + (((kk >> 2) * ASIDE_KB + (kk & 3) * 32) >> 4),
+                          dB + (((kk >> 2) * BCAT_KB + (kk & 3) * 32) >> 4), ID_G, kk > 0);
+            umma_commit(bar);
+        }
+        ok = cta_wait_mma(bar, phase, flag, p.dev_status);
+        if (!ok) break;
+
+        // ---- A (key rows, fp32) and P (query rows, bf16 tile) from the Gram; thread = TMEM
+        //      lane = row; a warp's lanes 0-15 and 16-31 hold two consecutive 16-blocks
+        {
+            const bool isq = warp >= 2;
+            const int i = tid & 63;
+            const int myI = i >> 4;
+            const int Ia = 2 * (warp & 1);
+            const float bi = rowv[ROW_BETA + i];
+            uint8_t *P = smem + OFF_P;
+#pragma unroll 1
+            for (int w2 = 0; w2 < 2; ++w2) {
+                const int I = Ia + w2;
+                const int off = 8 * I * (I + 1);
+#pragma unroll 1
+                for (int blk = 0; blk <= I; ++blk) {
+                    float x[16];
+                    tmem_ld16(tl + TM_G + off + 16 * blk, x);
+                    tmem_wait_ld();
+                    if (myI != I) continue;
+                    const int j0 = 16 * blk;
+                    if (!isq) {
+                        float *row = solve + (blk == I ? I : a_slot(I, blk)) * SOLVE_BLK + (i & 15) * SOLVE_LD;
+#pragma unroll
+                        for (int q4 = 0; q4 < 4; ++q4) {
+                            float y[4];
+#pragma unroll
+                            for (int e = 0; e < 4; ++e) {
+                                const int j = j0 + 4 * q4 + e;
+                                y[e] = (retrieval && j < i) ? bi * x[4 * q4 + e] : 0.f;
+                            }
+                            *reinterpret_cast<float4 *>(row + 4 * q4) = make_float4(y[0], y[1], y[2], y[3]);
+                        }
+                    } else {
+                        // the diagonal from the raw bytes in fp32: rq_i rk_i (q_i . k_i)
+                        const float pii = rowv[ROW_QK + i];
+                        float y[16];
+#pragma unroll
+                        for (int e = 0; e < 16; ++e) y[e] = (j0 + e < i) ? x[e] : (j0 + e == i ? pii : 0.f);
+                        *reinterpret_cast<uint4 *>(P + sw128(i, 2 * blk)) = pack8<F16>(y);
+                        *reinterpret_cast<uint4 *>(P + sw128(i, 2 * blk + 1)) = pack8<F16>(y + 8);
+                    }
+                }
+            }
+            // P blocks right of the row's own block are zero (the solve reads no A block there)
+            if (isq)
+                for (int blk = myI + 1; blk < 4; ++blk) {
+                    *reinterpret_cast<uint4 *>(P + sw128(i, 2 * blk)) = make_uint4(0u, 0u, 0u, 0u);
+                    *reinterpret_cast<uint4 *>(P + sw128(i, 2 * blk + 1)) = make_uint4(0u, 0u, 0u, 0u);
+                }
+        }
+        tc_fence_before();
+        __syncthreads();
+
+        // ---- T = (I + A)^-1 by blocks, written as Tb = T diag(beta) (bf16 B operand of (W),
+        //      (U~)); the blocks above the diagonal of Tb are zero
+        {
+            const float *beta = rowv + ROW_BETA;
+            uint8_t *tb = smem + OFF_TB;
+            if (tid < 64) {
+                // diagonal inverses D_I = (I + A_II)^-1, thread = column c of block I
+                const int I = tid >> 4, c = tid & 15;
+                const float *Ab = solve + I * SOLVE_BLK;
+                float x[16];
+#pragma unroll
+                for (int r = 0; r < 16; ++r) {
+                    float acc0 = (r == c) ? 1.f : 0.f, acc1 = 0.f;
+#pragma unroll
+                    for (int m = 0; m < r; ++m) {
+                        if (m & 1) acc1 = fmaf(-Ab[r * SOLVE_LD + m], x[m], acc1);
+                        else acc0 = fmaf(-Ab[r * SOLVE_LD + m], x[m], acc0);
+                    }
+                    x[r] = acc0 + acc1;
+                }
+                float *Db = solve + (10 + I) * SOLVE_BLK;
+#pragma unroll
+                for (int r = 0; r < 16; ++r) Db[r * SOLVE_LD + c] = x[r];
+                const int j = 16 * I + c;
+                const float bj = beta[j];
+#pragma unroll
+                for (int r = 0; r < 16; ++r)
+                    *reinterpret_cast<uint16_t *>(tb + sw128(16 * I + r, j >> 3) + (j & 7) * 2) = elem16<F16>(x[r] * bj);
+            } else {
+                // zero blocks above the diagonal: (I, J) with J > I, 16 rows x 32 bytes each
+                for (int u = tid - 64; u < 6 * 16 * 2; u += 64) {
+                    const int pr = u >> 5, rr = (u >> 1) & 15, hf = u & 1;
+                    const int I = pr < 3 ? 0 : (pr < 5 ? 1 : 2);
+                    const int J = pr < 3 ? 1 + pr : (pr < 5 ? pr - 1 : 3);
+                    *reinterpret_cast<uint4 *>(tb + sw128(16 * I + rr, 2 * J + hf)) = make_uint4(0u, 0u, 0u, 0u);
+                }
+            }
+            __syncthreads();
+            // T_10 = -D_1 (A_10 D_0) (warp 0), T_32 = -D_3 (A_32 D_2) (warp 1)
+            if (warp < 2) {
+                float *tmp = solve + (warp ? 15 : 14) * SOLVE_BLK;
+                float acc[2][4] = {};
+                blk_mma(acc, solve + (warp ? 5 : 4) * SOLVE_BLK, solve + (warp ? 12 : 10) * SOLVE_BLK);
+                blk_store(tmp, acc, 1.f);
+                __syncwarp();
+                float acc2[2][4] = {};
+                blk_mma(acc2, solve + (warp ? 13 : 11) * SOLVE_BLK, tmp);
+                __syncwarp();
+                blk_store(tmp, acc2, -1.f);
+                blk_store_tb<F16>(acc2, -1.f, warp ? 3 : 1, warp ? 2 : 0, beta, tb);
+            }
+            __syncthreads();
+            // lower-left 2 x 2 of blocks: X = A_BA T_AA (slots 2p+q), then T_BA = -T_BB X
+#pragma unroll 1
+            for (int ph = 0; ph < 2; ++ph) {
+                const int pp = (warp >> 1) & 1, q = warp & 1;
+                const float *X0, *Y0, *X1 = nullptr, *Y1 = nullptr;
+                if (ph == 0) {
+                    if (q == 0) {
+                        X0 = solve + a_slot(2 + pp, 0) * SOLVE_BLK; Y0 = solve + 10 * SOLVE_BLK;
+                        X1 = solve + a_slot(2 + pp, 1) * SOLVE_BLK; Y1 = solve + 14 * SOLVE_BLK;
+                    } else {
+                        X0 = solve + a_slot(2 + pp, 1) * SOLVE_BLK; Y0 = solve + 11 * SOLVE_BLK;
+                    }
+                } else {
+                    if (pp == 0) {
+                        X0 = solve + 12 * SOLVE_BLK; Y0 = solve + q * SOLVE_BLK;
+                    } else {
+                        X0 = solve + 15 * SOLVE_BLK; Y0 = solve + q * SOLVE_BLK;
+                        X1 = solve + 13 * SOLVE_BLK; Y1 = solve + (2 + q) * SOLVE_BLK;
+                    }
+                }
+                float acc[2][4] = {};
+                const int np = X1 ? 2 : 1;
+#pragma unroll 1
+                for (int t = 0; t < np; ++t) blk_mma(acc, t ? X1 : X0, t ? Y1 : Y0);
+                if (ph == 0) blk_store(solve + (2 * pp + q) * SOLVE_BLK, acc, 1.f);
+                else blk_store_tb<F16>(acc, -1.f, 2 + pp, q, beta, tb);
+                __syncthreads();
+            }
+        }
+        fence_proxy_async_smem();
+        __syncthreads();
+
+        // ---- (W), (U~)
+        if (tid == 0) {
+            tc_fence_after();
+            const uint64_t dKG = sdesc_sw128(sbase + OFF_KG, TILE_KB, 1024);
+            const uint64_t dVT = sdesc_sw128(sbase + OFF_VT, TILE_KB, 1024);
+            const uint64_t dTB = sdesc_sw128(sbase + OFF_TB, 16, 1024);
+            if (retrieval) {
+#pragma unroll 1
+                for (int kk = 0; kk < 4; ++kk)
+                    umma_bf16(tmem + TM_W, dKG + ((kk * 2048) >> 4), dTB + ((kk * 32) >> 4), ID_WU, kk > 0);
+            }
+#pragma unroll 1
+            for (int kk = 0; kk < 4; ++kk)
+                umma_bf16(tmem + TM_U, dVT + ((kk * 2048) >> 4), dTB + ((kk * 32) >> 4), ID_WU, kk > 0);
+            umma_commit(bar);
+        }
+        ok = cta_wait_mma(bar, phase, flag, p.dev_status);
+        if (!ok) break;
+
+        // ---- -W as the MN-major B operand of (1a): thread = dk row, 64 tokens i across
+        if (retrieval) {
+            uint8_t *wn = smem + OFF_WNEG;
+#pragma unroll 1
+            for (int half = 0; half < 2; ++half) {
+                float x[32];
+                tmem_ld32(tl + TM_W + 32 * half, x);
+                tmem_wait_ld();
+#pragma unroll
+                for (int e = 0; e < 32; ++e) x[e] = -x[e];
+#pragma unroll
+                for (int q = 0; q < 4; ++q)
+                    *reinterpret_cast<uint4 *>(wn + sw128(tid, 4 * half + q)) = pack8<F16>(x + 8 * q);
+            }
+        }
+        fence_proxy_async_smem();
+        tc_fence_before();
+        __syncthreads();
+
+        // ---- (1a) U^T += S^T (-W)^T, (1b) Y = S^T (Q^ e^G)^T
+        if (tid == 0) {
+            tc_fence_after();
+            const uint64_t dSB = sdesc_sw128(sbase + OFF_SB, 16, 1024);
+            const uint64_t dWN = sdesc_sw128(sbase + OFF_WNEG, 8192, 1024);
+            const uint64_t dQG = sdesc_sw128(sbase + OFF_QG, 16, 1024);
+            if (retrieval) {
+#pragma unroll 1
+                for (int kk = 0; kk < 8; ++kk)
+                    umma_bf16(tmem + TM_U, dSB + (((kk >> 2) * 16384 + (kk & 3) * 32) >> 4),
+                              dWN + ((kk * 2048) >> 4), ID_1A, 1);
+            }
+#pragma unroll 1
+            for (int kk = 0; kk < 8; ++kk)
+                umma_bf16(tmem + TM_Y, dSB + (((kk >> 2) * 16384 + (kk & 3) * 32) >> 4),
+                          dQG + (((kk >> 2) * TILE_KB + (kk & 3) * 32) >> 4), ID_1B, kk > 0);
+            umma_commit(bar);
+        }
+        ok = cta_wait_mma(bar, phase, flag, p.dev_status);
+        if (!ok) break;
+
+        // ---- U^T -> bf16 A operand of (2), (3); the state's decay diag(e^{G_C}) on its columns
+        {
+            uint8_t *ub = smem + OFF_UB;
+            float x[32];
+#pragma unroll 1
+            for (int half = 0; half < 2; ++half) {
+                tmem_ld32(tl + TM_U + 32 * half, x);
+                tmem_wait_ld();
+#pragma unroll
+                for (int q = 0; q < 4; ++q)
+                    *reinterpret_cast<uint4 *>(ub + sw128(tid, 4 * half + q)) = pack8<F16>(x + 8 * q);
+            }
+#pragma unroll 1
+            for (int blk = 0; blk < 4; ++blk) {
+                tmem_ld32(tl + TM_S + 32 * blk, x);
+                tmem_wait_ld();
+#pragma unroll
+                for (int e = 0; e < 32; ++e) x[e] *= vec[VEC_GC + 32 * blk + e];
+                tmem_st32(tl + TM_S + 32 * blk, x);
+            }
+            tmem_wait_st();
+        }
+        fence_proxy_async_smem();
+        tc_fence_before();
+        __syncthreads();
+
+        // ---- (2) S^T += U^T (K^ e^{G_C - G}), (3) Z = U^T P^T
+        if (tid == 0) {
+            tc_fence_after();
+            const uint64_t dUB = sdesc_sw128(sbase + OFF_UB, 16, 1024);
+            const uint64_t dKD = sdesc_sw128(sbase + OFF_KD, TILE_KB, 1024);
+            const uint64_t dP = sdesc_sw128(sbase + OFF_P, 16, 1024);
+#pragma unroll 1
+            for (int kk = 0; kk < 4; ++kk)
+                umma_bf16(tmem + TM_S, dUB + ((kk * 32) >> 4), dKD + ((kk * 2048) >> 4), ID_2, 1);
+#pragma unroll 1
+            for (int kk = 0; kk < 4; ++kk)
+                umma_bf16(tmem + TM_Z, dUB + ((kk * 32) >> 4), dP + ((kk * 32) >> 4), ID_3, kk > 0);
+            umma_commit(bar);
+        }
+        ok = cta_wait_mma(bar, phase, flag, p.dev_status);
+        if (!ok) break;
+
+        // ---- outputs O^T = scale (Y + Z) (thread = dv), then the new state's bf16 copy
+        {
+            float y[32], z[32];
+#pragma unroll 1
+            for (int half = 0; half < 2; ++half) {
+                tmem_ld32(tl + TM_Y + 32 * half, y);
+                tmem_ld32(tl + TM_Z + 32 * half, z);
+                tmem_wait_ld();
+                if (tid < Dv) {
+#pragma unroll
+                    for (int e = 0; e < 32; ++e) {
+                        const int i = 32 * half + e;
+                        if (i < ln)
+                            og[((t0 + i) * Hv + h) * (int64_t)Dv + tid] = elem16<F16>(p.scale * (y[e] + z[e]));
+                    }
+                }
+            }
+#pragma unroll 1
+            for (int blk = 0; blk < 4; ++blk) {
+                tmem_ld32(tl + TM_S + 32 * blk, y);
+                tmem_wait_ld();
+                store_sb<F16>(smem + OFF_SB, tid, blk, y);
+            }
+        }
+        fence_proxy_async_smem();
+        tc_fence_before();
+        __syncthreads();
+        tc_fence_after();
+    }
+
+    if (ok) {
+        // final state (V-major, fp32); an empty request copies its initial state through
+        float x[32];
+#pragma unroll 1
+        for (int blk = 0; blk < 4; ++blk) {
+            tmem_ld32(tl + TM_S + 32 * blk, x);
+            tmem_wait_ld();
+            if (tid < Dv)
+#pragma unroll
+                for (int e = 0; e < 32; ++e) {
+                    const int dk = 32 * blk + e;
+                    if (dk < Dk) p.final_state[soff + (int64_t)tid * Dk + dk] = x[e];
+                }
+        }
+    } else if (tid == 0) {
+        // a wait ran out: give the MMAs in flight a last bounded chance before TMEM is freed
+        const long long t0 = clock64();
+        while (!mbar_try_wait(bar, (phase - 1) & 1))
+            if (clock64() - t0 > (1ll << 24)) break;
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    if (warp == 0) tmem_dealloc(tmem, 512);
+}
+
+}  // namespace gdn_kd
+
+bool prefill_kd_supported(const GdnPrefillArgs &a)
+{
+    return a.g_per_key && a.has_decay && a.dtype == GDN_BF16 && a.Dk >= 8 && a.Dk <= 128 &&
+           a.Dv >= 8 && a.Dv <= 128;
+}
+
+cudaError_t launch_prefill_kd(const GdnPrefillArgs &a, cudaStream_t stream)
+{
+    using namespace gdn_kd;
+    if (a.B == 0 || a.Hv == 0) return cudaSuccess;
+    static DeviceOnce smem_opt_in;
+    cudaError_t e = smem_opt_in.run([] {
+        return cudaFuncSetAttribute(gdn_prefill_kd_kernel<false>,
+                                    cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SMEM_BYTES);
+    });
+    if (e != cudaSuccess) return e;
+    const unsigned grid = (unsigned)a.B * (unsigned)a.Hv;
+    gdn_prefill_kd_kernel<false><<<grid, NT, SMEM_BYTES, stream>>>(a);
+    return cudaGetLastError();
+}

@@ -120,7 +120,14 @@ def test_prefill_per_key_decay_validation(L):
     assert prefill(L, flags=PK, out=P(4, 64 * 16 * 4 - 64)) == 5
     assert prefill(L, flags=PK, final=P(4, 64 * 16 * 4 - 64)) == 5
     assert prefill(L, flags=PK, g=P(4, 8)) == 4
-    assert L.gdn_prefill_uses_chunked(g.GDN_BF16, 32, 128, 128, PK) == 0
+    # bf16 heads of 8 to 128 run the per-key tensor-core kernel; fp16, fp32 and other heads the
+    # per-token kernel; the sequence split never takes the per-key decay
+    assert L.gdn_prefill_uses_chunked(g.GDN_BF16, 32, 128, 128, PK) == 1
+    assert L.gdn_prefill_uses_chunked(g.GDN_BF16, 3, 12, 9, PK) == 1
+    assert L.gdn_prefill_uses_chunked(g.GDN_F16, 3, 12, 9, PK) == 0
+    assert L.gdn_prefill_uses_chunked(g.GDN_BF16, 3, 4, 128, PK) == 0   # narrower than 8
+    assert L.gdn_prefill_uses_chunked(g.GDN_F32, 32, 128, 128, PK) == 0
+    assert L.gdn_prefill_uses_chunked(g.GDN_BF16, 32, 160, 128, PK) == 0
     assert L.gdn_prefill_workspace_size(1, 32768, 16, 32, 128, 128, g.GDN_BF16, PK) == 0
 
 

@@ -125,24 +125,31 @@ def test_linear_rule_long_sequence_matches_oracle(gdn, W, oracle_mod):
 # ------------------------------------------------------- per-key-dimension decay
 # "com.microsoft.GatedDeltaNet", Inputs table: `decay` spelled (..., num_heads_v,
 # head_size_qk), exp(g_t) read as diag(exp(g_t)) on the key axis of the state (the oracle's
-# reading, pinned in test_oracle_pins).  It runs the per-token kernel (fp32 arithmetic).
+# reading, pinned in test_oracle_pins).  bf16 heads of 8 to 128 run the per-key tensor-core
+# kernel (bf16 operand tiles, as the scalar-decay chunked kernel, so the same 2e-2 bound);
+# fp16 (whose exponent range cannot hold the kernel's scaled operands), fp32, other head
+# sizes and `sequential` run the per-token kernel (fp32 arithmetic).
 TOL_BY_DTYPE = {torch.bfloat16: TOL_BF16, torch.float16: TOL_F16, torch.float32: 1e-4}
 
 
+@pytest.mark.parametrize("sequential", [False, True])
 @pytest.mark.parametrize("dtype,Dk,Dv,Hq,Hv", [
     (torch.bfloat16, 128, 128, 2, 4), (torch.float16, 64, 32, 1, 2), (torch.float32, 12, 9, 1, 2),
-    (torch.float32, 256, 256, 1, 1), (torch.bfloat16, 160, 96, 2, 2), (torch.bfloat16, 1, 1, 1, 3)])
-def test_per_key_decay_matches_oracle(gdn, W, oracle_mod, dtype, Dk, Dv, Hq, Hv):
-    assert not gdn.prefill_uses_chunked(dtype, Hv, Dk, Dv, decay_per_key=True)
+    (torch.float32, 256, 256, 1, 1), (torch.bfloat16, 160, 96, 2, 2), (torch.bfloat16, 1, 1, 1, 3),
+    (torch.bfloat16, 12, 9, 1, 2), (torch.float16, 128, 128, 2, 2), (torch.bfloat16, 100, 72, 3, 6)])
+def test_per_key_decay_matches_oracle(gdn, W, oracle_mod, dtype, Dk, Dv, Hq, Hv, sequential):
+    tc = dtype == torch.bfloat16 and 8 <= min(Dk, Dv) and max(Dk, Dv) <= 128 and not sequential
+    assert gdn.prefill_uses_chunked(dtype, Hv, Dk, Dv, sequential, decay_per_key=True) == tc
     c = W.make_prefill(41, LENGTHS, Hq, Hv, Dk, Dv, dtype=dtype, init_std=0.02,
                        qk_l2norm=True, decay_per_key=True)
     assert tuple(c.g.shape) == (c.N, Hv, Dk)
-    o, f, ro, rf = _run_both(gdn, oracle_mod, c, c.g, c.beta, False, decay_per_key=True)
+    o, f, ro, rf = _run_both(gdn, oracle_mod, c, c.g, c.beta, sequential, decay_per_key=True)
     _parity(c, o, f, ro, rf, TOL_BY_DTYPE[dtype])
 
 
+@pytest.mark.parametrize("sequential", [False, True])
 @pytest.mark.parametrize("rule,qwen", [("gated", False), ("gated", True), ("gated_delta", True)])
-def test_per_key_decay_rules_and_gates(gdn, W, oracle_mod, rule, qwen):
+def test_per_key_decay_rules_and_gates(gdn, W, oracle_mod, rule, qwen, sequential):
     """The gated rule (no retrieval, beta = 1) and the qwen gate applied to every key
     dimension with its head's a_log and dt_bias (raw decay N(0,1)), with the sigmoid beta."""
     c = W.make_prefill(42, LENGTHS, 2, 4, 128, 64, init_std=0.02, qk_l2norm=True,
@@ -160,8 +167,40 @@ def test_per_key_decay_rules_and_gates(gdn, W, oracle_mod, rule, qwen):
     if has_beta:
         beta = torch.from_numpy(rng.standard_normal(c.beta.shape).astype(np.float32))
         kw["beta_activation"] = "sigmoid"
-    o, f, ro, rf = _run_both(gdn, oracle_mod, c, g, beta, False, **kw)
+    o, f, ro, rf = _run_both(gdn, oracle_mod, c, g, beta, sequential, **kw)
     _parity(c, o, f, ro, rf, TOL_BF16)
+
+
+def test_per_key_decay_strong_and_infinite_decays(gdn, W, oracle_mod):
+    """Per-dimension decays down to -40 and -inf in some dimensions (a dimension that forgets
+    at once) on the tensor-core kernel: it floors every per-dimension log-decay at -9 so that
+    its scaled operands stay finite; a decay factor below e^-9 ~ 1.2e-4 then weighs the old
+    column at 1.2e-4 instead of less, far inside the bf16 bound (the oracle keeps the raw g)."""
+    c = W.make_prefill(46, LENGTHS, 2, 4, 128, 128, init_std=0.02, qk_l2norm=True,
+                       decay_per_key=True)
+    rng = np.random.default_rng(47)
+    g = c.g.numpy().copy()
+    strong = rng.random(g.shape) < 0.05
+    g[strong] = -rng.uniform(9.0, 40.0, int(strong.sum()))
+    g[:, :, 5] = -np.inf
+    g[:, 1, :8] = -np.inf
+    g = torch.from_numpy(g.astype(np.float32))
+    assert gdn.prefill_uses_chunked(torch.bfloat16, 4, 128, 128, decay_per_key=True)
+    o, f, ro, rf = _run_both(gdn, oracle_mod, c, g, c.beta, False, decay_per_key=True)
+    _parity(c, o, f, ro, rf, TOL_BF16)
+
+
+def test_per_key_decay_tensor_cores_match_per_token_kernel(gdn, W):
+    """The two per-key kernels on the same bf16 bytes (requests of 1 to 200 tokens, an empty
+    one, GQA): outputs and states agree within the bf16 bound."""
+    c = W.make_prefill(48, LENGTHS, 2, 4, 128, 128, init_std=0.02, qk_l2norm=True,
+                       decay_per_key=True)
+    args = [dev(t) for t in (c.q, c.k, c.v, c.g, c.beta, c.cu_seqlens, c.initial_state)]
+    o1, f1 = gdn.gdn_prefill(*args, scale=c.scale, qk_l2norm=True)
+    o2, f2 = gdn.gdn_prefill(*args, scale=c.scale, qk_l2norm=True, sequential=True)
+    torch.cuda.synchronize()
+    assert_prefill_parity(f64(o1), f64(f1), f64(o2), f64(f2),
+                          request_ranges(c.cu_seqlens, c.B, c.N), TOL_BF16)
 
 
 def test_per_key_decay_equal_dimensions_match_scalar_gate(gdn, W):
@@ -178,6 +217,28 @@ def test_per_key_decay_equal_dimensions_match_scalar_gate(gdn, W):
     torch.cuda.synchronize()
     assert_prefill_parity(f64(o2), f64(f2), f64(o1), f64(f1),
                           request_ranges(c.cu_seqlens, c.B, c.N), 1e-5)
+
+
+def test_per_key_tensor_cores_with_equal_dimensions_match_scalar_chunked(gdn, W, oracle_mod):
+    """bf16: the per-key tensor-core kernel with the same decay in every key dimension and the
+    scalar-decay chunked kernel (two different chunk factorings of one recurrence) are each
+    held to the oracle of the scalar gate.  (Against each other the bound would be twice the
+    bound each meets against the oracle.)"""
+    c = W.make_prefill(49, LENGTHS, 2, 4, 128, 128, init_std=0.02, qk_l2norm=True)
+    gk = c.g[:, :, None].expand(-1, -1, 128).contiguous()
+    args = (dev(c.q), dev(c.k), dev(c.v))
+    assert gdn.prefill_uses_chunked(torch.bfloat16, 4, 128, 128, decay_per_key=True)
+    o1, f1 = gdn.gdn_prefill(*args, dev(c.g), dev(c.beta), dev(c.cu_seqlens),
+                             dev(c.initial_state), scale=c.scale, qk_l2norm=True, split=False)
+    o2, f2 = gdn.gdn_prefill(*args, dev(gk), dev(c.beta), dev(c.cu_seqlens),
+                             dev(c.initial_state), scale=c.scale, qk_l2norm=True)
+    torch.cuda.synchronize()
+    ro, rf = oracle_mod.prefill(f64(c.q), f64(c.k), f64(c.v), f64(c.g), f64(c.beta),
+                                c.cu_seqlens.numpy(), f64(c.initial_state), scale=c.scale,
+                                qk_l2norm=True)
+    ranges = request_ranges(c.cu_seqlens, c.B, c.N)
+    assert_prefill_parity(f64(o1), f64(f1), ro, rf, ranges, TOL_BF16)
+    assert_prefill_parity(f64(o2), f64(f2), ro, rf, ranges, TOL_BF16)
 
 
 def test_per_key_decay_rank4_spelling(gdn, W, oracle_mod):
