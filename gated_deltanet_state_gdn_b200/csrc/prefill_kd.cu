@@ -36,8 +36,8 @@
 //   (2)  S^T = S^T diag(e^{G_C}) + U^T (K^ e^{G_C - G})
 //   (3)  Z = U^T P^T                O^T = scale (Y + Z)
 //
-// One CTA of 128 threads per (request, value head); thread t owns TMEM lane t (the state
-// row dv = t).  The phases of a chunk run one after another (plain loads stage and scale the
+// One CTA of 256 threads per (request, value head): two warpgroups, whose thread t owns TMEM
+// lane t (the state row dv = t) and which split each row's columns between them.  The phases of a chunk run one after another (plain loads stage and scale the
 // operand tiles, thread 0 issues the MMAs, a bounded wait on one mbarrier ends each group).
 // The triangular solve works on 16 x 16 blocks: fp32 forward substitution inside the four
 // diagonal blocks, then tf32 warp MMAs merge the blocks below the diagonal.
@@ -51,7 +51,7 @@ using namespace sm100;
 namespace gdn_kd {
 
 constexpr int C = 64;            // chunk length (tokens)
-constexpr int NT = 128;          // threads per CTA
+constexpr int NT = 256;          // threads per CTA: two warpgroups over the 128 TMEM lanes
 constexpr float G_FLOOR = -9.f;  // per-dimension log-decay floor
 constexpr float LOG2E = 1.4426950408889634f;
 
@@ -303,6 +303,7 @@ __global__ void __launch_bounds__(NT, 1) gdn_prefill_kd_kernel(const __grid_cons
     uint8_t *smem = smem_raw + ((1024u - (raw_base & 1023u)) & 1023u);
     const uint32_t sbase = smem_u32(smem);
     const int tid = threadIdx.x, warp = tid >> 5;
+    const int wg = tid >> 7, lt = tid & 127;   // warpgroup; TMEM lane = state row
     const int Hv = p.Hv, Hq = p.Hq, Dk = p.Dk, Dv = p.Dv;
     const int b = blockIdx.x / Hv, h = blockIdx.x - b * Hv;
     const int qh = (int)(((int64_t)h * Hq) / Hv);
@@ -353,21 +354,21 @@ __global__ void __launch_bounds__(NT, 1) gdn_prefill_kd_kernel(const __grid_cons
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
-    const uint32_t tl = tmem + ((uint32_t)(32 * warp) << 16);   // this warp's TMEM lanes
+    const uint32_t tl = tmem + ((uint32_t)(32 * (warp & 3)) << 16);   // this warp's TMEM lanes
     uint32_t phase = 0;
 
-    // state S^T (row dv = tid) into TMEM, and its bf16 copy
+    // state S^T (row dv = lt, column blocks 2 wg and 2 wg + 1) into TMEM, and its bf16 copy
     {
         float x[32];
 #pragma unroll 1
-        for (int blk = 0; blk < 4; ++blk) {
+        for (int blk = 2 * wg; blk < 2 * wg + 2; ++blk) {
 #pragma unroll
             for (int e = 0; e < 32; ++e) {
                 const int dk = 32 * blk + e;
-                x[e] = (p.initial_state && tid < Dv && dk < Dk) ? p.initial_state[soff + (int64_t)tid * Dk + dk] : 0.f;
+                x[e] = (p.initial_state && lt < Dv && dk < Dk) ? p.initial_state[soff + (int64_t)lt * Dk + dk] : 0.f;
             }
             tmem_st32(tl + TM_S + 32 * blk, x);
-            store_sb<F16>(smem + OFF_SB, tid, blk, x);
+            store_sb<F16>(smem + OFF_SB, lt, blk, x);
         }
         tmem_wait_st();
     }
@@ -388,11 +389,13 @@ __global__ void __launch_bounds__(NT, 1) gdn_prefill_kd_kernel(const __grid_cons
         const int64_t t0 = start + (int64_t)n * C;
         const int ln = min(C, len - n * C);
 
-        // ---- raw rows of the chunk, unit (token j, 8 dimensions 8c..8c+7), 8 units per thread,
+        // ---- raw rows of the chunk, unit (token j, 8 dimensions 8c..8c+7),
         //      all requested at once so that their latency overlaps the decay staging below
-        uint4 rk8[8], rq8[8], rv8[8];
+        //      (UNITS units per thread)
+        constexpr int UNITS = C * 16 / NT;   // units per thread
+        uint4 rk8[UNITS], rq8[UNITS], rv8[UNITS];
 #pragma unroll
-        for (int it = 0; it < 8; ++it) {
+        for (int it = 0; it < UNITS; ++it) {
             const int u = tid + NT * it, j = u >> 4, c = u & 15;
             if (j < ln) {
                 const int64_t qk = ((t0 + j) * Hq + qh) * (int64_t)Dk;
@@ -423,22 +426,31 @@ __global__ void __launch_bounds__(NT, 1) gdn_prefill_kd_kernel(const __grid_cons
             }
         }
         __syncthreads();
-        // ---- per-dimension cumulative log-decay (thread = key dimension), in place
+        // ---- per-dimension cumulative log-decay, in place: thread = key dimension, warpgroup
+        //      wg scans tokens [32 wg, 32 wg + 32); the second half then adds the first's total
+        float acc = 0.f;
         {
-            const int d = tid;
+            const int d = lt;
             const float ea = p.a_log ? expf(__ldg(p.a_log + h)) : 0.f;
             const float dtb = p.a_log ? __ldg(p.dt_bias + h) : 0.f;
-            float acc = 0.f;
 #pragma unroll 8
-            for (int i = 0; i < C; ++i) {
+            for (int i = 32 * wg; i < 32 * wg + 32; ++i) {
                 float g = G2[i * 128 + d];
                 if (i < ln && d < Dk) {
                     if (p.a_log) g = -ea * gdn::softplus20(g + dtb);
                     g = fmaxf(g, G_FLOOR);
                 }
                 acc += g;
-                G2[i * 128 + d] = acc * LOG2E;
+                G2[i * 128 + d] = acc;
             }
+        }
+        __syncthreads();
+        {
+            const int d = lt;
+            const float base = wg ? G2[31 * 128 + d] : 0.f;
+            __syncthreads();
+#pragma unroll 8
+            for (int i = 32 * wg; i < 32 * wg + 32; ++i) G2[i * 128 + d] = (G2[i * 128 + d] + base) * LOG2E;
         }
         if (tid < C) {
             float bt = 0.f;
@@ -449,7 +461,7 @@ __global__ void __launch_bounds__(NT, 1) gdn_prefill_kd_kernel(const __grid_cons
             rowv[ROW_BETA + tid] = bt;
         }
         __syncthreads();
-        {
+        if (tid < 128) {
             const int d = tid;
             float m2[4];
 #pragma unroll
@@ -476,7 +488,7 @@ __global__ void __launch_bounds__(NT, 1) gdn_prefill_kd_kernel(const __grid_cons
         //      bf16-rounded decayed operands its value would carry their rounding relative to
         //      |q^||k^| rather than to the product, which near-orthogonal q and k make small.
 #pragma unroll
-        for (int it = 0; it < 8; ++it) {
+        for (int it = 0; it < UNITS; ++it) {
             const int u = tid + NT * it, j = u >> 4, c = u & 15;
             const int I = j >> 4;
             float kx[8], qx[8], vx[8];
@@ -564,18 +576,17 @@ __global__ void __launch_bounds__(NT, 1) gdn_prefill_kd_kernel(const __grid_cons
         ok = cta_wait_mma(bar, phase, flag, p.dev_status);
         if (!ok) break;
 
-        // ---- A (key rows, fp32) and P (query rows, bf16 tile) from the Gram; thread = TMEM
-        //      lane = row; a warp's lanes 0-15 and 16-31 hold two consecutive 16-blocks
+        // ---- A (key rows, fp32) and P (query rows, bf16 tile) from the Gram; TMEM lane = row;
+        //      a warp's lanes 0-15 and 16-31 hold two consecutive 16-blocks, of which warpgroup
+        //      wg takes the (wg)th
         {
-            const bool isq = warp >= 2;
-            const int i = tid & 63;
+            const bool isq = (warp & 3) >= 2;
+            const int i = lt & 63;
             const int myI = i >> 4;
-            const int Ia = 2 * (warp & 1);
             const float bi = rowv[ROW_BETA + i];
             uint8_t *P = smem + OFF_P;
-#pragma unroll 1
-            for (int w2 = 0; w2 < 2; ++w2) {
-                const int I = Ia + w2;
+            {
+                const int I = 2 * (warp & 1) + wg;
                 const int off = 8 * I * (I + 1);
 #pragma unroll 1
                 for (int blk = 0; blk <= I; ++blk) {
@@ -608,7 +619,7 @@ __global__ void __launch_bounds__(NT, 1) gdn_prefill_kd_kernel(const __grid_cons
                 }
             }
             // P blocks right of the row's own block are zero (the solve reads no A block there)
-            if (isq)
+            if (isq && myI == 2 * (warp & 1) + wg)
                 for (int blk = myI + 1; blk < 4; ++blk) {
                     *reinterpret_cast<uint4 *>(P + sw128(i, 2 * blk)) = make_uint4(0u, 0u, 0u, 0u);
                     *reinterpret_cast<uint4 *>(P + sw128(i, 2 * blk + 1)) = make_uint4(0u, 0u, 0u, 0u);
@@ -645,7 +656,7 @@ __global__ void __launch_bounds__(NT, 1) gdn_prefill_kd_kernel(const __grid_cons
 #pragma unroll
                 for (int r = 0; r < 16; ++r)
                     *reinterpret_cast<uint16_t *>(tb + sw128(16 * I + r, j >> 3) + (j & 7) * 2) = elem16<F16>(x[r] * bj);
-            } else {
+            } else if (tid < 128) {
                 // zero blocks above the diagonal: (I, J) with J > I, 16 rows x 32 bytes each
                 for (int u = tid - 64; u < 6 * 16 * 2; u += 64) {
                     const int pr = u >> 5, rr = (u >> 1) & 15, hf = u & 1;
@@ -689,12 +700,14 @@ __global__ void __launch_bounds__(NT, 1) gdn_prefill_kd_kernel(const __grid_cons
                         X1 = solve + 13 * SOLVE_BLK; Y1 = solve + (2 + q) * SOLVE_BLK;
                     }
                 }
-                float acc[2][4] = {};
-                const int np = X1 ? 2 : 1;
+                if (warp < 4) {
+                    float acc[2][4] = {};
+                    const int np = X1 ? 2 : 1;
 #pragma unroll 1
-                for (int t = 0; t < np; ++t) blk_mma(acc, t ? X1 : X0, t ? Y1 : Y0);
-                if (ph == 0) blk_store(solve + (2 * pp + q) * SOLVE_BLK, acc, 1.f);
-                else blk_store_tb<F16>(acc, -1.f, 2 + pp, q, beta, tb);
+                    for (int t = 0; t < np; ++t) blk_mma(acc, t ? X1 : X0, t ? Y1 : Y0);
+                    if (ph == 0) blk_store(solve + (2 * pp + q) * SOLVE_BLK, acc, 1.f);
+                    else blk_store_tb<F16>(acc, -1.f, 2 + pp, q, beta, tb);
+                }
                 __syncthreads();
             }
         }
@@ -720,20 +733,18 @@ __global__ void __launch_bounds__(NT, 1) gdn_prefill_kd_kernel(const __grid_cons
         ok = cta_wait_mma(bar, phase, flag, p.dev_status);
         if (!ok) break;
 
-        // ---- -W as the MN-major B operand of (1a): thread = dk row, 64 tokens i across
+        // ---- -W as the MN-major B operand of (1a): lane = dk row, tokens 32 wg .. 32 wg + 31
         if (retrieval) {
             uint8_t *wn = smem + OFF_WNEG;
-#pragma unroll 1
-            for (int half = 0; half < 2; ++half) {
-                float x[32];
-                tmem_ld32(tl + TM_W + 32 * half, x);
-                tmem_wait_ld();
+            const int half = wg;
+            float x[32];
+            tmem_ld32(tl + TM_W + 32 * half, x);
+            tmem_wait_ld();
 #pragma unroll
-                for (int e = 0; e < 32; ++e) x[e] = -x[e];
+            for (int e = 0; e < 32; ++e) x[e] = -x[e];
 #pragma unroll
-                for (int q = 0; q < 4; ++q)
-                    *reinterpret_cast<uint4 *>(wn + sw128(tid, 4 * half + q)) = pack8<F16>(x + 8 * q);
-            }
+            for (int q = 0; q < 4; ++q)
+                *reinterpret_cast<uint4 *>(wn + sw128(lt, 4 * half + q)) = pack8<F16>(x + 8 * q);
         }
         fence_proxy_async_smem();
         tc_fence_before();
@@ -764,16 +775,16 @@ __global__ void __launch_bounds__(NT, 1) gdn_prefill_kd_kernel(const __grid_cons
         {
             uint8_t *ub = smem + OFF_UB;
             float x[32];
-#pragma unroll 1
-            for (int half = 0; half < 2; ++half) {
+            {
+                const int half = wg;
                 tmem_ld32(tl + TM_U + 32 * half, x);
                 tmem_wait_ld();
 #pragma unroll
                 for (int q = 0; q < 4; ++q)
-                    *reinterpret_cast<uint4 *>(ub + sw128(tid, 4 * half + q)) = pack8<F16>(x + 8 * q);
+                    *reinterpret_cast<uint4 *>(ub + sw128(lt, 4 * half + q)) = pack8<F16>(x + 8 * q);
             }
 #pragma unroll 1
-            for (int blk = 0; blk < 4; ++blk) {
+            for (int blk = 2 * wg; blk < 2 * wg + 2; ++blk) {
                 tmem_ld32(tl + TM_S + 32 * blk, x);
                 tmem_wait_ld();
 #pragma unroll
@@ -803,28 +814,29 @@ __global__ void __launch_bounds__(NT, 1) gdn_prefill_kd_kernel(const __grid_cons
         ok = cta_wait_mma(bar, phase, flag, p.dev_status);
         if (!ok) break;
 
-        // ---- outputs O^T = scale (Y + Z) (thread = dv), then the new state's bf16 copy
+        // ---- outputs O^T = scale (Y + Z) (lane = dv, tokens 32 wg .. 32 wg + 31), then the new
+        //      state's bf16 copy (column blocks 2 wg, 2 wg + 1)
         {
             float y[32], z[32];
-#pragma unroll 1
-            for (int half = 0; half < 2; ++half) {
+            {
+                const int half = wg;
                 tmem_ld32(tl + TM_Y + 32 * half, y);
                 tmem_ld32(tl + TM_Z + 32 * half, z);
                 tmem_wait_ld();
-                if (tid < Dv) {
+                if (lt < Dv) {
 #pragma unroll
                     for (int e = 0; e < 32; ++e) {
                         const int i = 32 * half + e;
                         if (i < ln)
-                            og[((t0 + i) * Hv + h) * (int64_t)Dv + tid] = elem16<F16>(p.scale * (y[e] + z[e]));
+                            og[((t0 + i) * Hv + h) * (int64_t)Dv + lt] = elem16<F16>(p.scale * (y[e] + z[e]));
                     }
                 }
             }
 #pragma unroll 1
-            for (int blk = 0; blk < 4; ++blk) {
+            for (int blk = 2 * wg; blk < 2 * wg + 2; ++blk) {
                 tmem_ld32(tl + TM_S + 32 * blk, y);
                 tmem_wait_ld();
-                store_sb<F16>(smem + OFF_SB, tid, blk, y);
+                store_sb<F16>(smem + OFF_SB, lt, blk, y);
             }
         }
         fence_proxy_async_smem();
@@ -837,14 +849,14 @@ __global__ void __launch_bounds__(NT, 1) gdn_prefill_kd_kernel(const __grid_cons
         // final state (V-major, fp32); an empty request copies its initial state through
         float x[32];
 #pragma unroll 1
-        for (int blk = 0; blk < 4; ++blk) {
+        for (int blk = 2 * wg; blk < 2 * wg + 2; ++blk) {
             tmem_ld32(tl + TM_S + 32 * blk, x);
             tmem_wait_ld();
-            if (tid < Dv)
+            if (lt < Dv)
 #pragma unroll
                 for (int e = 0; e < 32; ++e) {
                     const int dk = 32 * blk + e;
-                    if (dk < Dk) p.final_state[soff + (int64_t)tid * Dk + dk] = x[e];
+                    if (dk < Dk) p.final_state[soff + (int64_t)lt * Dk + dk] = x[e];
                 }
         }
     } else if (tid == 0) {
