@@ -64,6 +64,8 @@ constexpr uint32_t BCAT_KB = 20480;
 constexpr uint32_t OFF_P = 0;            // [64 rows i][64 j], K-major
 constexpr uint32_t OFF_WNEG = 8192;      // [128 rows dk][64 i], MN-major B of (1a)
 constexpr uint32_t OFF_UB = 24576;       // [128 rows dv][64 j], K-major A of (2), (3)
+constexpr uint32_t OFF_GN = 40960;       // raw log-decays of the next chunk, fp32 [64][128]:
+                                         // staged once the Gram has read the key operands
 // region Z: decayed operands and v
 constexpr uint32_t OFF_KG = 73728;       // K^ e^G        [kb 2][64 rows j][128 B], kb 8192
 constexpr uint32_t OFF_QG = 90112;       // Q^ e^G
@@ -89,7 +91,8 @@ constexpr uint32_t OFF_BAR = OFF_ROW + 1024;       // mbarrier, TMEM base, flag
 constexpr uint32_t SMEM_USED = OFF_BAR + 64;
 constexpr uint32_t SMEM_BYTES = SMEM_USED + 1024;  // + alignment slack
 static_assert(SMEM_BYTES <= 232448, "shared memory budget");
-static_assert(OFF_BCAT + 2 * BCAT_KB <= OFF_KG && OFF_UB + 16384 <= OFF_KG, "region Y");
+static_assert(OFF_BCAT + 2 * BCAT_KB <= OFF_KG && OFF_UB + 16384 <= OFF_GN &&
+              OFF_GN + 64 * 128 * 4 <= OFF_KG, "region Y");
 static_assert(OFF_A + 16 * SOLVE_BLK * 4 <= OFF_TB && OFF_TB + 8192 <= OFF_VEC &&
               OFF_G2 + 64 * 128 * 4 <= OFF_VEC, "region X");
 static_assert(OFF_TB % 1024 == 0 && OFF_SB % 1024 == 0 && OFF_VT % 1024 == 0 &&
@@ -274,6 +277,29 @@ __device__ __forceinline__ void blk_store_tb(const float (&acc)[2][4], float sgn
     }
 }
 
+// a chunk's raw log-decays (rows of Dk floats, zero past the request's ln tokens and past Dk)
+// into dst fp32 [64][128]: asynchronous 16-byte copies when rows are 16-byte multiples
+__device__ __forceinline__ void stage_g(float *dst, const GdnPrefillArgs &p, int64_t t0, int ln, int h)
+{
+    const int Dk = p.Dk, Hv = p.Hv;
+    if ((Dk & 3) == 0) {
+        const int pieces = Dk >> 2;
+        for (int u = threadIdx.x; u < C * 32; u += NT) {
+            const int i = u >> 5, c4 = u & 31;
+            float *d = dst + i * 128 + 4 * c4;
+            if (i < ln && c4 < pieces)
+                cp_async16(smem_u32(d), p.g + ((t0 + i) * Hv + h) * (int64_t)Dk + 4 * c4);
+            else
+                *reinterpret_cast<float4 *>(d) = make_float4(0.f, 0.f, 0.f, 0.f);
+        }
+    } else {
+        for (int u = threadIdx.x; u < C * 128; u += NT) {
+            const int i = u >> 7, d = u & 127;
+            dst[u] = (i < ln && d < Dk) ? __ldg(p.g + ((t0 + i) * Hv + h) * (int64_t)Dk + d) : 0.f;
+        }
+    }
+}
+
 // thread 0 waits (bounded) for the MMA group committed to `bar`; every thread gets the outcome
 __device__ __forceinline__ bool cta_wait_mma(uint32_t bar, uint32_t &phase, volatile int *flag,
                                              int32_t *status)
@@ -384,16 +410,13 @@ __global__ void __launch_bounds__(NT, 1) gdn_prefill_kd_kernel(const __grid_cons
     constexpr uint32_t ID_2 = idesc_f16kind(128, 128, 0, 1, !F16);
     constexpr uint32_t ID_3 = idesc_f16kind(128, 64, 0, 0, !F16);
 
-    bool ok = true;
-    for (int n = 0; n < nc && ok; ++n) {
+    // the raw rows of chunk n (unit (token j, 8 dimensions 8c..8c+7), UNITS units per thread),
+    // requested one chunk ahead: they travel while the previous chunk's products run
+    constexpr int UNITS = C * 16 / NT;
+    uint4 rk8[UNITS], rq8[UNITS], rv8[UNITS];
+    auto load_rows = [&](int n) {
         const int64_t t0 = start + (int64_t)n * C;
         const int ln = min(C, len - n * C);
-
-        // ---- raw rows of the chunk, unit (token j, 8 dimensions 8c..8c+7),
-        //      all requested at once so that their latency overlaps the decay staging below
-        //      (UNITS units per thread)
-        constexpr int UNITS = C * 16 / NT;   // units per thread
-        uint4 rk8[UNITS], rq8[UNITS], rv8[UNITS];
 #pragma unroll
         for (int it = 0; it < UNITS; ++it) {
             const int u = tid + NT * it, j = u >> 4, c = u & 15;
@@ -406,25 +429,20 @@ __global__ void __launch_bounds__(NT, 1) gdn_prefill_kd_kernel(const __grid_cons
                 rk8[it] = rq8[it] = rv8[it] = make_uint4(0u, 0u, 0u, 0u);
             }
         }
-        // ---- the chunk's raw log-decays into G2 (rows of Dk floats; asynchronous 16-byte
-        //      copies when rows are 16-byte multiples), zero past the request and past Dk
-        if ((Dk & 3) == 0) {
-            const int pieces = Dk >> 2;   // 16-byte pieces per row
-            for (int u = tid; u < C * 32; u += NT) {
-                const int i = u >> 5, c4 = u & 31;
-                float *dst = G2 + i * 128 + 4 * c4;
-                if (i < ln && c4 < pieces)
-                    cp_async16(smem_u32(dst), p.g + ((t0 + i) * Hv + h) * (int64_t)Dk + 4 * c4);
-                else
-                    *reinterpret_cast<float4 *>(dst) = make_float4(0.f, 0.f, 0.f, 0.f);
-            }
-            cp_async_wait_all();
-        } else {
-            for (int u = tid; u < C * 128; u += NT) {
-                const int i = u >> 7, d = u & 127;
-                G2[u] = (i < ln && d < Dk) ? __ldg(p.g + ((t0 + i) * Hv + h) * (int64_t)Dk + d) : 0.f;
-            }
-        }
+    };
+    float *gn = reinterpret_cast<float *>(smem + OFF_GN);
+    if (nc > 0) {
+        load_rows(0);
+        stage_g(gn, p, start, min(C, len), h);
+    }
+
+    bool ok = true;
+    for (int n = 0; n < nc && ok; ++n) {
+        const int64_t t0 = start + (int64_t)n * C;
+        const int ln = min(C, len - n * C);
+
+        // ---- this chunk's raw log-decays (staged during the previous chunk) are in gn
+        cp_async_wait_all();
         __syncthreads();
         // ---- per-dimension cumulative log-decay, in place: thread = key dimension, warpgroup
         //      wg scans tokens [32 wg, 32 wg + 32); the second half then adds the first's total
@@ -435,7 +453,7 @@ __global__ void __launch_bounds__(NT, 1) gdn_prefill_kd_kernel(const __grid_cons
             const float dtb = p.a_log ? __ldg(p.dt_bias + h) : 0.f;
 #pragma unroll 8
             for (int i = 32 * wg; i < 32 * wg + 32; ++i) {
-                float g = G2[i * 128 + d];
+                float g = gn[i * 128 + d];
                 if (i < ln && d < Dk) {
                     if (p.a_log) g = -ea * gdn::softplus20(g + dtb);
                     g = fmaxf(g, G_FLOOR);
@@ -561,6 +579,7 @@ __global__ void __launch_bounds__(NT, 1) gdn_prefill_kd_kernel(const __grid_cons
         }
         fence_proxy_async_smem();
         __syncthreads();
+        if (n + 1 < nc) load_rows(n + 1);
 
         // ---- (G): all blocks' products in one MMA
         if (tid == 0) {
@@ -575,6 +594,7 @@ __global__ void __launch_bounds__(NT, 1) gdn_prefill_kd_kernel(const __grid_cons
         }
         ok = cta_wait_mma(bar, phase, flag, p.dev_status);
         if (!ok) break;
+        if (n + 1 < nc) stage_g(gn, p, t0 + C, min(C, len - (n + 1) * C), h);
 
         // ---- A (key rows, fp32) and P (query rows, bf16 tile) from the Gram; TMEM lane = row;
         //      a warp's lanes 0-15 and 16-31 hold two consecutive 16-blocks, of which warpgroup
