@@ -637,13 +637,15 @@ def make_case(name):
         return workloads.ragged_prefill_case()
     if name == "long":
         return workloads.long_prefill_case()
+    if name == "ragged_per_key":
+        return workloads.ragged_prefill_case(decay_per_key=True)
     raise ValueError(name)
 
 
 def workload_config(case, name):
     Hq, Hv, Dk, Dv = case.dims
     return {"workload": case.name, "requests": case.B, "tokens": case.N,
-            "lengths": "U[1,4096] seeded" if name == "ragged" else str(case.N),
+            "lengths": "U[1,4096] seeded" if name.startswith("ragged") else str(case.N),
             "Hq": Hq, "Hv": Hv, "Dk": Dk, "Dv": Dv, "chunk": CHUNK,
             "l2": "inputs larger than L2 (q+k+v+out > 126 MB), and consecutive launches "
                   "alternate between two independent input sets, so no launch re-reads "
@@ -656,7 +658,7 @@ def main():
     ap.add_argument("--steps", type=int, default=100)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="gdn", choices=["gdn", "reference"])
-    ap.add_argument("--workload", default="ragged", choices=["ragged", "long"])
+    ap.add_argument("--workload", default="ragged", choices=["ragged", "long", "ragged_per_key"])
     ap.add_argument("--no-decode", action="store_true")
     ap.add_argument("--no-conv", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")

@@ -119,8 +119,12 @@ enum {
  *                    S_t = D_t S_{t-1} + k_t (beta_t (v_t - (D_t S_{t-1})^T k_t))^T
  *                  (V-major: column i of S scales by exp(g_t[i])); the qwen gate
  *                  maps every element with its head's a_log and dt_bias.  The
- *                  page lists this spelling as not implemented by its own kernels;
- *                  here it runs the per-token kernel.
+ *                  page lists this spelling as not implemented by its own kernels.
+ *                  bf16 heads of 8 to 128 run a chunked tensor-core kernel of
+ *                  their own, which floors each per-dimension log-decay at -9
+ *                  (a decay factor below e^-9 ~ 1.2e-4 counts as 1.2e-4) so that
+ *                  its decay-scaled operands stay in range; fp16, fp32 and other
+ *                  head sizes run the per-token kernel (no floor).
  *   beta           [N, Hv] float32, update rate; required exactly for the rules
  *                  with the delta retrieval (gated_delta, delta), NULL
  *                  otherwise (the write is then k_t v_t^T).  With
@@ -347,10 +351,11 @@ GDN_API gdn_status gdn_conv1d(const void *x, const void *weight, void *conv_stat
                               int32_t kernel_size, int32_t max_slots, gdn_dtype dtype,
                               int32_t write_state, int32_t *dev_status, void *stream);
 
-/* 1 when gdn_prefill with these arguments runs the chunked tensor-core
- * kernel, 0 when it runs the per-token kernel (host-only query, no launch).
- * The chunked kernel takes bf16 or fp16 with Dk, Dv up to 128 (smaller heads run as
- * zero-padded 128-wide tiles) and any Hv. */
+/* 1 when gdn_prefill with these arguments runs a chunked tensor-core kernel,
+ * 0 when it runs the per-token kernel (host-only query, no launch).  The chunked
+ * kernel takes bf16 or fp16 with Dk, Dv up to 128 (smaller heads run as
+ * zero-padded 128-wide tiles) and any Hv; with GDN_DECAY_PER_KEY, bf16 with Dk,
+ * Dv from 8 to 128. */
 GDN_API int32_t gdn_prefill_uses_chunked(gdn_dtype dtype, int32_t Hv, int32_t Dk, int32_t Dv,
                                          uint32_t flags);
 
