@@ -601,7 +601,8 @@ def prefill_roofline(gdn, case, launch_ms, peaks, sm_mhz, traffic):
            "frac": byts / avg_s / 1e9 / hbm_peak, "ideal_us": t_hbm * 1e6,
            "algorithmic_bytes": byts}
     b = tc if t_tc >= t_hbm else hbm
-    return {"kernel": "gdn_prefill_chunk", "bound": "tensor" if t_tc >= t_hbm else "hbm",
+    return {"kernel": "gdn_prefill_kd" if per_key else "gdn_prefill_chunk",
+            "bound": "tensor" if t_tc >= t_hbm else "hbm",
             "achieved": b["achieved"], "peak": b["peak"], "unit": b["unit"], "frac": b["frac"],
             "traffic": traffic, "tensor": tc, "hbm": hbm,
             "ms_per_launch": avg_s * 1e3,
@@ -750,7 +751,8 @@ def main():
         per_key = {
             "workload": pcase.name, "tokens": pcase.N, "steps": p_steps, "ms_per_step": p_max,
             "value": job_throughput(pcase.N, world, p_max), "unit": "tokens/s",
-            "roofline": prefill_roofline(gdn, pcase, p_launch, peaks, None, None)}
+            "roofline": prefill_roofline(gdn, pcase, p_launch, peaks, None,
+                                         ncu_traffic("prefill_kd_ragged_per_key.md", "prefill_kd.cu"))}
         launches += time_prefill.launches
         del pcase
 
