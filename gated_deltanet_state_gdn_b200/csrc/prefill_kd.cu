@@ -36,8 +36,9 @@
 //   (2)  S^T = S^T diag(e^{G_C}) + U^T (K^ e^{G_C - G})
 //   (3)  Z = U^T P^T                O^T = scale (Y + Z)
 //
-// One CTA of 256 threads per (request, value head): two warpgroups, whose thread t owns TMEM
-// lane t (the state row dv = t) and which split each row's columns between them.  The phases of a chunk run one after another (plain loads stage and scale the
+// One CTA of 256 threads per (request, value head), longest requests first: two
+// warpgroups, whose thread t owns TMEM lane t (the state row dv = t) and which split each
+// row's columns between them.  The phases of a chunk run one after another (plain loads stage and scale the
 // operand tiles, thread 0 issues the MMAs, a bounded wait on one mbarrier ends each group).
 // The triangular solve works on 16 x 16 blocks: fp32 forward substitution inside the four
 // diagonal blocks, then tf32 warp MMAs merge the blocks below the diagonal.
@@ -300,15 +301,18 @@ __device__ __forceinline__ void stage_g(float *dst, const GdnPrefillArgs &p, int
     }
 }
 
-// thread 0 waits (bounded) for the MMA group committed to `bar`; every thread gets the outcome
-__device__ __forceinline__ bool cta_wait_mma(uint32_t bar, uint32_t &phase, volatile int *flag,
-                                             int32_t *status)
+// thread 0 waits (bounded) for the MMA group committed to `bar`; every thread gets the outcome.
+// `wbar` is the barrier actually waited on: `bar`, or (checked builds, GDN_DEV_TEST_STALL) a
+// barrier that nothing arrives on, so that the wait runs out
+__device__ __forceinline__ bool cta_wait_mma(uint32_t bar, uint32_t wbar, uint32_t &phase,
+                                             volatile int *flag, int32_t *status)
 {
+    (void)bar;
     if (threadIdx.x == 0) {
-        bool good = mbar_try_wait(bar, phase & 1);
+        bool good = mbar_try_wait(wbar, phase & 1);
         if (!good) {
             const long long t0 = clock64();
-            while (!(good = mbar_try_wait(bar, phase & 1)))
+            while (!(good = mbar_try_wait(wbar, phase & 1)))
                 if (clock64() - t0 > (1ll << 31)) break;
         }
         if (!good && status) atomicOr(status, GDN_DEV_TIMEOUT);
@@ -331,7 +335,31 @@ __global__ void __launch_bounds__(NT, 1) gdn_prefill_kd_kernel(const __grid_cons
     const int tid = threadIdx.x, warp = tid >> 5;
     const int wg = tid >> 7, lt = tid & 127;   // warpgroup; TMEM lane = state row
     const int Hv = p.Hv, Hq = p.Hq, Dk = p.Dk, Dv = p.Dv;
-    const int b = blockIdx.x / Hv, h = blockIdx.x - b * Hv;
+    // CTAs take the (request, head) units longest request first (ties by request index), so
+    // that the chains of the longest requests start in the first wave of CTAs
+    int b = blockIdx.x / Hv;
+    const int h = blockIdx.x - b * Hv;
+    if (p.cu_seqlens && p.B > 1 && p.B <= NT) {
+        int *lens = reinterpret_cast<int *>(smem + OFF_KG);     // scratch before the first chunk
+        int *pick = reinterpret_cast<int *>(smem + OFF_BAR + 32);
+        if (tid < p.B) {
+            const int64_t st = gdn::clamp_i64(p.cu_seqlens[tid], 0, p.N);
+            const int64_t en = gdn::clamp_i64(p.cu_seqlens[tid + 1], 0, p.N);
+            lens[tid] = en > st ? (int)(en - st) : 0;
+        }
+        __syncthreads();
+        if (tid < p.B) {
+            const int li = lens[tid];
+            int rank = 0;
+            for (int j2 = 0; j2 < p.B; ++j2) {
+                const int lj = lens[j2];
+                rank += (lj > li) || (lj == li && j2 < tid);
+            }
+            if (rank == b) *pick = tid;
+        }
+        __syncthreads();
+        b = *pick;
+    }
     const int qh = (int)(((int64_t)h * Hq) / Hv);
     const bool retrieval = p.has_retrieval != 0;
 
@@ -362,6 +390,9 @@ __global__ void __launch_bounds__(NT, 1) gdn_prefill_kd_kernel(const __grid_cons
     const uint32_t bar = sbase + OFF_BAR;
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + OFF_BAR + 8);
     volatile int *flag = reinterpret_cast<volatile int *>(smem + OFF_BAR + 12);
+    // checked builds, GDN_DEV_TEST_STALL: the first MMA wait of CTA 0 runs on a barrier that
+    // nothing arrives on, so it runs out and the CTA leaves through the timeout path
+    uint32_t stall_bar = (blockIdx.x == 0 && gdn::test_stall_requested(p.dev_status)) ? sbase + OFF_BAR + 16 : 0u;
     float *G2 = reinterpret_cast<float *>(smem + OFF_G2);
     float *solve = reinterpret_cast<float *>(smem + OFF_A);
     float *vec = reinterpret_cast<float *>(smem + OFF_VEC);
@@ -369,6 +400,7 @@ __global__ void __launch_bounds__(NT, 1) gdn_prefill_kd_kernel(const __grid_cons
 
     if (tid == 0) {
         mbar_init(bar, 1);
+        mbar_init(sbase + OFF_BAR + 16, 1);
         fence_mbar_init();
         *flag = 1;
     }
@@ -592,7 +624,8 @@ __global__ void __launch_bounds__(NT, 1) gdn_prefill_kd_kernel(const __grid_cons
                           dB + (((kk >> 2) * BCAT_KB + (kk & 3) * 32) >> 4), ID_G, kk > 0);
             umma_commit(bar);
         }
-        ok = cta_wait_mma(bar, phase, flag, p.dev_status);
+        ok = cta_wait_mma(bar, stall_bar ? stall_bar : bar, phase, flag, p.dev_status);
+        stall_bar = 0;
         if (!ok) break;
         if (n + 1 < nc) stage_g(gn, p, t0 + C, min(C, len - (n + 1) * C), h);
 
@@ -750,7 +783,8 @@ __global__ void __launch_bounds__(NT, 1) gdn_prefill_kd_kernel(const __grid_cons
                 umma_bf16(tmem + TM_U, dVT + ((kk * 2048) >> 4), dTB + ((kk * 32) >> 4), ID_WU, kk > 0);
             umma_commit(bar);
         }
-        ok = cta_wait_mma(bar, phase, flag, p.dev_status);
+        ok = cta_wait_mma(bar, stall_bar ? stall_bar : bar, phase, flag, p.dev_status);
+        stall_bar = 0;
         if (!ok) break;
 
         // ---- -W as the MN-major B operand of (1a): lane = dk row, tokens 32 wg .. 32 wg + 31
@@ -788,7 +822,8 @@ __global__ void __launch_bounds__(NT, 1) gdn_prefill_kd_kernel(const __grid_cons
                           dQG + (((kk >> 2) * TILE_KB + (kk & 3) * 32) >> 4), ID_1B, kk > 0);
             umma_commit(bar);
         }
-        ok = cta_wait_mma(bar, phase, flag, p.dev_status);
+        ok = cta_wait_mma(bar, stall_bar ? stall_bar : bar, phase, flag, p.dev_status);
+        stall_bar = 0;
         if (!ok) break;
 
         // ---- U^T -> bf16 A operand of (2), (3); the state's decay diag(e^{G_C}) on its columns
@@ -831,7 +866,8 @@ __global__ void __launch_bounds__(NT, 1) gdn_prefill_kd_kernel(const __grid_cons
                 umma_bf16(tmem + TM_Z, dUB + ((kk * 32) >> 4), dP + ((kk * 32) >> 4), ID_3, kk > 0);
             umma_commit(bar);
         }
-        ok = cta_wait_mma(bar, phase, flag, p.dev_status);
+        ok = cta_wait_mma(bar, stall_bar ? stall_bar : bar, phase, flag, p.dev_status);
+        stall_bar = 0;
         if (!ok) break;
 
         // ---- outputs O^T = scale (Y + Z) (lane = dv, tokens 32 wg .. 32 wg + 31), then the new

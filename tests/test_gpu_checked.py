@@ -62,6 +62,7 @@ def assert_same(r0, r1):
 
 # ---------------------------------------------------------------- prefill
 def prefill_fn(gdn, c):
+    # the per-key spelling of the decay is read from g's rank
     def fn(st):
         o, f = gdn.gdn_prefill(dev(c.q), dev(c.k), dev(c.v), dev(c.g), dev(c.beta),
                                dev(c.cu_seqlens), dev(c.initial_state), None, None,
@@ -72,17 +73,20 @@ def prefill_fn(gdn, c):
     return fn
 
 
-@pytest.mark.parametrize("name,lengths,Hq,Hv,Dk,Dv,dtype", [
-    ("chunked default", [70, 1, 130, 0, 64], 2, 4, 128, 128, torch.bfloat16),
-    ("chunked head sizes", [33, 100], 2, 4, 64, 40, torch.bfloat16),
-    ("chunked fp16", [90, 5], 2, 4, 128, 128, torch.float16),
-    ("chunked plain-staged odd heads", [33, 70, 0, 5], 1, 2, 12, 9, torch.bfloat16),
-    ("per-token fp32", [20, 7], 1, 2, 12, 9, torch.float32),
+@pytest.mark.parametrize("name,lengths,Hq,Hv,Dk,Dv,dtype,per_key", [
+    ("chunked default", [70, 1, 130, 0, 64], 2, 4, 128, 128, torch.bfloat16, False),
+    ("chunked head sizes", [33, 100], 2, 4, 64, 40, torch.bfloat16, False),
+    ("chunked fp16", [90, 5], 2, 4, 128, 128, torch.float16, False),
+    ("chunked plain-staged odd heads", [33, 70, 0, 5], 1, 2, 12, 9, torch.bfloat16, False),
+    ("chunked per-key decay", [70, 1, 130, 0, 64], 2, 4, 128, 128, torch.bfloat16, True),
+    ("chunked per-key decay odd heads", [33, 70, 0, 5], 1, 2, 10, 9, torch.bfloat16, True),
+    ("per-token fp32", [20, 7], 1, 2, 12, 9, torch.float32, False),
+    ("per-token per-key fp16", [20, 7], 1, 2, 12, 9, torch.float16, True),
 ])
-def test_prefill_in_bounds(gdn, W, name, lengths, Hq, Hv, Dk, Dv, dtype):
+def test_prefill_in_bounds(gdn, W, name, lengths, Hq, Hv, Dk, Dv, dtype, per_key):
     c = W.make_prefill(11 + len(name), lengths, Hq, Hv, Dk, Dv, dtype=dtype, init_std=0.02,
-                       qk_l2norm=True)
-    chunked = gdn.prefill_uses_chunked(dtype, Hv, Dk, Dv)
+                       qk_l2norm=True, decay_per_key=per_key)
+    chunked = gdn.prefill_uses_chunked(dtype, Hv, Dk, Dv, decay_per_key=per_key)
     assert chunked == name.startswith("chunked")
     r0, r1, st = both(gdn, prefill_fn(gdn, c))
     assert st == 0
@@ -99,6 +103,34 @@ def test_chunked_prefill_wait_runs_out_on_request(gdn, W):
     matches the product library bit for bit."""
     c = W.make_prefill(77, [40], 1, 4, 128, 128, init_std=0.05, qk_l2norm=True)
     assert gdn.prefill_uses_chunked(c.q.dtype, 4, 128, 128)
+    product = gdn._binding.LIB_PATH
+    gdn.use_library(gdn.CHECKED_LIB_PATH)
+    try:
+        st = torch.full((1,), gdn.GDN_DEV_TEST_STALL, dtype=torch.int32, device="cuda")
+        t0 = time.time()
+        prefill_fn(gdn, c)(st)
+        took = time.time() - t0
+        s = int(st.item())
+        assert s & gdn.GDN_DEV_TIMEOUT
+        assert not s & gdn.GDN_DEV_BOUNDS
+        assert took < 60
+        st2 = torch.zeros(1, dtype=torch.int32, device="cuda")
+        r1 = prefill_fn(gdn, c)(st2)
+        assert int(st2.item()) == 0
+    finally:
+        gdn.use_library(product)
+    r0 = prefill_fn(gdn, c)(None)
+    assert_same(r0, r1)
+
+
+def test_per_key_prefill_wait_runs_out_on_request(gdn, W):
+    """The per-key tensor-core kernel: GDN_DEV_TEST_STALL makes CTA 0 wait for its first MMA
+    group on a barrier that nothing arrives on.  The wait runs out, GDN_DEV_TIMEOUT is set, the
+    CTA drains the group it issued, frees TMEM and returns; the other CTAs finish normally.  A
+    normal call on the same context then matches the product library bit for bit."""
+    c = W.make_prefill(78, [40, 90], 1, 4, 128, 128, init_std=0.05, qk_l2norm=True,
+                       decay_per_key=True)
+    assert gdn.prefill_uses_chunked(c.q.dtype, 4, 128, 128, decay_per_key=True)
     product = gdn._binding.LIB_PATH
     gdn.use_library(gdn.CHECKED_LIB_PATH)
     try:
