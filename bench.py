@@ -529,14 +529,15 @@ def time_conv(gdn, case, steps, warmup, world, graph=False, nsets=1):
 
 
 # ---------------------------------------------------------------- CPU oracle
-def cpu_oracle_sample(case, target_s=10.0, repeats=1):
+def cpu_oracle_sample(case, target_s=10.0, repeats=1, threads=None):
     """Time the float64 oracle on a bounded sample of the prefill workload: the first L
     tokens of the packed stream with every head; L is grown until one run takes ~target_s/8,
     then scaled so that one run is ~target_s (at most the whole stream).  With repeats > 1
-    the calibrated sample is run that many times and the median rate is reported."""
+    the calibrated sample is run that many times and the median rate is reported.  threads:
+    host threads for the oracle's (request, head) units (default: all cores)."""
     import oracle
     oracle.build()
-    threads = oracle.max_threads()
+    threads = oracle.max_threads() if threads is None else int(threads)
     Hq, Hv, Dk, Dv = case.dims
     start = 0 if case.cu_seqlens is None else int(case.cu_seqlens[0])
     total = case.N - start
@@ -823,6 +824,10 @@ def main():
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu:
         cpu = cpu_oracle_sample(case, target_s=args.cpu_seconds)
+        # the same oracle on one host thread, a shorter sample
+        one = cpu_oracle_sample(case, target_s=max(1.0, args.cpu_seconds / 3), threads=1)
+        cpu["single_thread"] = {"value": one["value"], "unit": one["unit"], "cores": 1,
+                                "sample": one["sample"]}
 
     if rank == 0:
         line = {
