@@ -446,9 +446,11 @@ __global__ void __launch_bounds__(NT, 1) gdn_prefill_kd_kernel(const __grid_cons
     // requested one chunk ahead: they travel while the previous chunk's products run
     constexpr int UNITS = C * 16 / NT;
     uint4 rk8[UNITS], rq8[UNITS], rv8[UNITS];
+    float rbeta = 0.f;   // beta of token tid (threads < 64), raw
     auto load_rows = [&](int n) {
         const int64_t t0 = start + (int64_t)n * C;
         const int ln = min(C, len - n * C);
+        if (tid < C) rbeta = (tid < ln && retrieval) ? __ldg(p.beta + (t0 + tid) * Hv + h) : 0.f;
 #pragma unroll
         for (int it = 0; it < UNITS; ++it) {
             const int u = tid + NT * it, j = u >> 4, c = u & 15;
@@ -490,22 +492,21 @@ __global__ void __launch_bounds__(NT, 1) gdn_prefill_kd_kernel(const __grid_cons
                     if (p.a_log) g = -ea * gdn::softplus20(g + dtb);
                     g = fmaxf(g, G_FLOOR);
                 }
-                acc += g;
+                acc += g * LOG2E;
                 G2[i * 128 + d] = acc;
             }
         }
         __syncthreads();
-        {
+        if (wg == 1) {
             const int d = lt;
-            const float base = wg ? G2[31 * 128 + d] : 0.f;
-            __syncthreads();
+            const float base = G2[31 * 128 + d];
 #pragma unroll 8
-            for (int i = 32 * wg; i < 32 * wg + 32; ++i) G2[i * 128 + d] = (G2[i * 128 + d] + base) * LOG2E;
+            for (int i = 32; i < 64; ++i) G2[i * 128 + d] += base;
         }
         if (tid < C) {
             float bt = 0.f;
             if (tid < ln) {
-                bt = retrieval ? __ldg(p.beta + (t0 + tid) * Hv + h) : 1.f;
+                bt = retrieval ? rbeta : 1.f;
                 if (retrieval && p.beta_sigmoid) bt = gdn::sigmoidf_(bt);
             }
             rowv[ROW_BETA + tid] = bt;
@@ -593,7 +594,7 @@ __global__ void __launch_bounds__(NT, 1) gdn_prefill_kd_kernel(const __grid_cons
             *reinterpret_cast<uint4 *>(smem + OFF_VT + kb * TILE_KB + sw128(j, ch)) = pack8<F16>(vx);
             // key operand of every block I2 >= I: k^ e^{M_I2 - G_j} = bk e^{M_I2 - M_I}; the
             // last one also gives k^ e^{G_C - G_j} = k^ e^{M_3 - G_j} e^{G_C - M_3}
-#pragma unroll 1
+#pragma unroll
             for (int I2 = I; I2 < 4; ++I2) {
                 float bb[8];
 #pragma unroll
@@ -611,9 +612,8 @@ __global__ void __launch_bounds__(NT, 1) gdn_prefill_kd_kernel(const __grid_cons
         }
         fence_proxy_async_smem();
         __syncthreads();
-        if (n + 1 < nc) load_rows(n + 1);
 
-        // ---- (G): all blocks' products in one MMA
+        // ---- (G): all blocks' products in one MMA; then the next chunk's rows are requested
         if (tid == 0) {
             tc_fence_after();
             const uint64_t dA = sdesc_sw128(sbase + OFF_ASIDE, 16, 1024);
@@ -624,6 +624,7 @@ __global__ void __launch_bounds__(NT, 1) gdn_prefill_kd_kernel(const __grid_cons
                           dB + (((kk >> 2) * BCAT_KB + (kk & 3) * 32) >> 4), ID_G, kk > 0);
             umma_commit(bar);
         }
+        if (n + 1 < nc) load_rows(n + 1);
         ok = cta_wait_mma(bar, stall_bar ? stall_bar : bar, phase, flag, p.dev_status);
         stall_bar = 0;
         if (!ok) break;
