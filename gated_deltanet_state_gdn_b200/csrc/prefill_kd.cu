@@ -301,13 +301,12 @@ __device__ __forceinline__ void stage_g(float *dst, const GdnPrefillArgs &p, int
     }
 }
 
-// thread 0 waits (bounded) for the MMA group committed to `bar`; every thread gets the outcome.
-// `wbar` is the barrier actually waited on: `bar`, or (checked builds, GDN_DEV_TEST_STALL) a
-// barrier that nothing arrives on, so that the wait runs out
-__device__ __forceinline__ bool cta_wait_mma(uint32_t bar, uint32_t wbar, uint32_t &phase,
-                                             volatile int *flag, int32_t *status)
+// thread 0 waits (bounded) on `wbar` for the MMA group committed to it; every thread gets the
+// outcome.  (Checked builds with GDN_DEV_TEST_STALL pass, once, a barrier that nothing arrives
+// on instead of the commit barrier, so that the wait runs out.)
+__device__ __forceinline__ bool cta_wait_mma(uint32_t wbar, uint32_t &phase, volatile int *flag,
+                                             int32_t *status)
 {
-    (void)bar;
     if (threadIdx.x == 0) {
         bool good = mbar_try_wait(wbar, phase & 1);
         if (!good) {
@@ -475,14 +474,16 @@ __global__ void __launch_bounds__(NT, 1) gdn_prefill_kd_kernel(const __grid_cons
         const int64_t t0 = start + (int64_t)n * C;
         const int ln = min(C, len - n * C);
 
-        // ---- this chunk's raw log-decays (staged during the previous chunk) are in gn
+        // ---- this chunk's raw log-decays (staged during the previous chunk or before the loop)
+        //      are in gn
         cp_async_wait_all();
         __syncthreads();
-        // ---- per-dimension cumulative log-decay, in place: thread = key dimension, warpgroup
-        //      wg scans tokens [32 wg, 32 wg + 32); the second half then adds the first's total
-        float acc = 0.f;
+        // ---- per-dimension cumulative log-decay (log2 units) into G2: thread = key dimension,
+        //      warpgroup wg scans tokens [32 wg, 32 wg + 32); the second half then adds the
+        //      first's total
         {
             const int d = lt;
+            float acc = 0.f;
             const float ea = p.a_log ? expf(__ldg(p.a_log + h)) : 0.f;
             const float dtb = p.a_log ? __ldg(p.dt_bias + h) : 0.f;
 #pragma unroll 8
@@ -625,7 +626,7 @@ __global__ void __launch_bounds__(NT, 1) gdn_prefill_kd_kernel(const __grid_cons
             umma_commit(bar);
         }
         if (n + 1 < nc) load_rows(n + 1);
-        ok = cta_wait_mma(bar, stall_bar ? stall_bar : bar, phase, flag, p.dev_status);
+        ok = cta_wait_mma(stall_bar ? stall_bar : bar, phase, flag, p.dev_status);
         stall_bar = 0;
         if (!ok) break;
         if (n + 1 < nc) stage_g(gn, p, t0 + C, min(C, len - (n + 1) * C), h);
@@ -784,7 +785,7 @@ __global__ void __launch_bounds__(NT, 1) gdn_prefill_kd_kernel(const __grid_cons
                 umma_bf16(tmem + TM_U, dVT + ((kk * 2048) >> 4), dTB + ((kk * 32) >> 4), ID_WU, kk > 0);
             umma_commit(bar);
         }
-        ok = cta_wait_mma(bar, stall_bar ? stall_bar : bar, phase, flag, p.dev_status);
+        ok = cta_wait_mma(stall_bar ? stall_bar : bar, phase, flag, p.dev_status);
         stall_bar = 0;
         if (!ok) break;
 
@@ -823,7 +824,7 @@ __global__ void __launch_bounds__(NT, 1) gdn_prefill_kd_kernel(const __grid_cons
                           dQG + (((kk >> 2) * TILE_KB + (kk & 3) * 32) >> 4), ID_1B, kk > 0);
             umma_commit(bar);
         }
-        ok = cta_wait_mma(bar, stall_bar ? stall_bar : bar, phase, flag, p.dev_status);
+        ok = cta_wait_mma(stall_bar ? stall_bar : bar, phase, flag, p.dev_status);
         stall_bar = 0;
         if (!ok) break;
 
@@ -867,7 +868,7 @@ __global__ void __launch_bounds__(NT, 1) gdn_prefill_kd_kernel(const __grid_cons
                 umma_bf16(tmem + TM_Z, dUB + ((kk * 32) >> 4), dP + ((kk * 32) >> 4), ID_3, kk > 0);
             umma_commit(bar);
         }
-        ok = cta_wait_mma(bar, stall_bar ? stall_bar : bar, phase, flag, p.dev_status);
+        ok = cta_wait_mma(stall_bar ? stall_bar : bar, phase, flag, p.dev_status);
         stall_bar = 0;
         if (!ok) break;
 
