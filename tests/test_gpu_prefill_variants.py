@@ -264,3 +264,15 @@ def test_full_ragged_prefill_per_key_decay_all_heads(gdn, W, oracle_mod):
     c = W.ragged_prefill_case(decay_per_key=True)
     o, f, ro, rf = _run_both(gdn, oracle_mod, c, c.g, c.beta, False, decay_per_key=True)
     _parity(c, o, f, ro, rf, TOL_BF16)
+
+
+def test_per_key_decay_many_requests(gdn, W, oracle_mod):
+    """300 requests of 0 to 70 tokens: more requests than the per-key kernel orders by length
+    (it then takes them in index order), every request and head against the oracle."""
+    rng = np.random.default_rng(50)
+    lengths = rng.integers(0, 71, 300).tolist()
+    c = W.make_prefill(51, lengths, 1, 2, 32, 16, init_std=0.02, qk_l2norm=True,
+                       decay_per_key=True)
+    assert gdn.prefill_uses_chunked(torch.bfloat16, 2, 32, 16, decay_per_key=True)
+    o, f, ro, rf = _run_both(gdn, oracle_mod, c, c.g, c.beta, False, decay_per_key=True)
+    _parity(c, o, f, ro, rf, TOL_BF16)
