@@ -155,9 +155,13 @@ def test_noncontiguous_inputs_and_inputs_unchanged(gdn, W, oracle_mod):
     assert_prefill_parity(out, fs, ro, rf, request_ranges(c.cu_seqlens, c.B, c.N), TOL_BF16)
 
 
+@pytest.mark.parametrize("per_key", [False, True])
 @pytest.mark.parametrize("sequential", [True, False])
-def test_deterministic(gdn, W, sequential):
-    c = W.make_prefill(61, [300, 77], 2, 4, 128, 128, init_std=0.02, qk_l2norm=True)
+def test_deterministic(gdn, W, sequential, per_key):
+    """Three calls on the same bytes give the same bytes (a race would show as a difference):
+    the scalar-decay chunked kernel, the per-key-decay chunked kernel and the per-token kernel."""
+    c = W.make_prefill(61, [300, 77], 2, 4, 128, 128, init_std=0.02, qk_l2norm=True,
+                       decay_per_key=per_key)
     runs = [run_gpu_prefill(c, sequential=sequential) for _ in range(3)]
     for o, f in runs[1:]:
         assert torch.equal(o, runs[0][0]) and torch.equal(f, runs[0][1])
