@@ -309,13 +309,16 @@ def test_full_long_prefill_all_heads(gdn, W, oracle_mod):
 
 
 @pytest.mark.parametrize("n", [64, 100])
-def test_split_and_resume_on_tensor_cores(gdn, W, n):
+@pytest.mark.parametrize("per_key", [False, True])
+def test_split_and_resume_on_tensor_cores(gdn, W, n, per_key):
     """A request run as two calls, the second starting from the first's final state, equals one
-    call (split on a chunk boundary and inside a chunk)."""
+    call (split on a chunk boundary and inside a chunk), on the scalar-decay and the
+    per-key-decay chunked kernels."""
     import copy
     L = 230
-    c = W.make_prefill(124, [L], 2, 4, 128, 128, init_std=0.02, qk_l2norm=True)
-    assert gdn.prefill_uses_chunked(c.q.dtype, 4, 128, 128)
+    c = W.make_prefill(124, [L], 2, 4, 128, 128, init_std=0.02, qk_l2norm=True,
+                       decay_per_key=per_key)
+    assert gdn.prefill_uses_chunked(c.q.dtype, 4, 128, 128, decay_per_key=per_key)
     o_full, f_full = run_gpu_prefill(c)
     parts, init = [], c.initial_state
     for lo, hi in ((0, n), (n, L)):
