@@ -738,10 +738,16 @@ def main():
             "value": job_throughput(lcase.N, world, l_max), "unit": "tokens/s",
             "roofline": prefill_roofline(gdn, lcase, l_launch, peaks, l_clocks["sm_mhz"], None),
             "repeat_windows_ms_per_launch": time_prefill.repeats, "clocks": l_clocks}
-        launches += time_prefill.launches
+        # a call that takes the sequence split launches three kernels: two passes and the
+        # composition of the segment maps
+        Hq_l, Hv_l, Dk_l, Dv_l = lcase.dims
+        splits = gdn.lib().gdn_prefill_workspace_size(lcase.B, lcase.N, Hq_l, Hv_l, Dk_l, Dv_l,
+                                                      gdn.GDN_BF16, 0) > 0
+        long_prefill["kernels_per_call"] = 3 if splits else 1
+        launches += time_prefill.launches * long_prefill["kernels_per_call"]
         del lcase
 
-    # the per-key-dimension decay over the ragged workload's shapes (per-token kernel)
+    # the per-key-dimension decay over the ragged workload's shapes (its tensor-core kernel)
     per_key = None
     if args.workload == "ragged" and not args.no_per_key:
         pcase = workloads.ragged_prefill_case(decay_per_key=True)
