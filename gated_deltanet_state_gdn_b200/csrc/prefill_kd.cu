@@ -179,6 +179,15 @@ __device__ __forceinline__ void load8(const uint16_t *row, int c, int n, bool ve
     for (int e = 0; e < 8; ++e) x[e] = (8 * c + e < n) ? to_f<F16>(row[8 * c + e]) : 0.f;
 }
 
+// 8 consecutive floats from 32-byte aligned shared memory
+__device__ __forceinline__ void lds8(const float *src, float (&x)[8])
+{
+    const float4 a = *reinterpret_cast<const float4 *>(src);
+    const float4 b = *reinterpret_cast<const float4 *>(src + 4);
+    x[0] = a.x; x[1] = a.y; x[2] = a.z; x[3] = a.w;
+    x[4] = b.x; x[5] = b.y; x[6] = b.z; x[7] = b.w;
+}
+
 // the bits of elements [8c, 8c + 8) of a row of `n` 16-bit values (zero past n)
 __device__ __forceinline__ uint4 load_raw8(const uint16_t *row, int c, int n, bool vec)
 {
@@ -565,17 +574,9 @@ __global__ void __launch_bounds__(NT, 1) gdn_prefill_kd_kernel(const __grid_cons
             if (c == 0) rowv[ROW_QK + j] = rq * rk * sqk;
 
             float g2[8], mI[8], em[8];
-            {
-                const float4 a0 = *reinterpret_cast<const float4 *>(G2 + j * 128 + 8 * c);
-                const float4 a1 = *reinterpret_cast<const float4 *>(G2 + j * 128 + 8 * c + 4);
-                g2[0] = a0.x; g2[1] = a0.y; g2[2] = a0.z; g2[3] = a0.w;
-                g2[4] = a1.x; g2[5] = a1.y; g2[6] = a1.z; g2[7] = a1.w;
-            }
-#pragma unroll
-            for (int e = 0; e < 8; ++e) {
-                mI[e] = vec[VEC_M2 + I * 128 + 8 * c + e];
-                em[e] = vec[VEC_EM + I * 128 + 8 * c + e];
-            }
+            lds8(G2 + j * 128 + 8 * c, g2);
+            lds8(vec + VEC_M2 + I * 128 + 8 * c, mI);
+            lds8(vec + VEC_EM + I * 128 + 8 * c, em);
             float ak[8], aq[8], kgm[8], qgm[8], bk[8];
 #pragma unroll
             for (int e = 0; e < 8; ++e) {
@@ -598,15 +599,22 @@ __global__ void __launch_bounds__(NT, 1) gdn_prefill_kd_kernel(const __grid_cons
 #pragma unroll
             for (int I2 = I; I2 < 4; ++I2) {
                 float bb[8];
+                if (I2 == I) {
 #pragma unroll
-                for (int e = 0; e < 8; ++e)
-                    bb[e] = I2 == I ? bk[e] : bk[e] * vec[VEC_CM + (I2 * (I2 - 1) / 2 + I) * 128 + 8 * c + e];
+                    for (int e = 0; e < 8; ++e) bb[e] = bk[e];
+                } else {
+                    float cm[8];
+                    lds8(vec + VEC_CM + (I2 * (I2 - 1) / 2 + I) * 128 + 8 * c, cm);
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) bb[e] = bk[e] * cm[e];
+                }
                 const int row = 8 * I2 * (I2 + 1) + j;   // 16 * I2 (I2 + 1) / 2 + j
                 *reinterpret_cast<uint4 *>(smem + OFF_BCAT + kb * BCAT_KB + sw128(row, ch)) = pack8<F16>(bb);
                 if (I2 == 3) {
-                    float kd[8];
+                    float kd[8], ec[8];
+                    lds8(vec + VEC_EC3 + 8 * c, ec);
 #pragma unroll
-                    for (int e = 0; e < 8; ++e) kd[e] = bb[e] * vec[VEC_EC3 + 8 * c + e];
+                    for (int e = 0; e < 8; ++e) kd[e] = bb[e] * ec[e];
                     *reinterpret_cast<uint4 *>(smem + OFF_KD + kb * TILE_KB + sw128(j, ch)) = pack8<F16>(kd);
                 }
             }
@@ -877,16 +885,34 @@ __global__ void __launch_bounds__(NT, 1) gdn_prefill_kd_kernel(const __grid_cons
         {
             float y[32], z[32];
             {
+                // 8 tokens at a time through a warp-private [8 tokens][32 dv] scratch (the solve
+                // area is free by now), then one 16-byte store per lane: lanes 4t..4t+3 write
+                // token t's 64 bytes of this warp's dv
                 const int half = wg;
                 tmem_ld32(tl + TM_Y + 32 * half, y);
                 tmem_ld32(tl + TM_Z + 32 * half, z);
                 tmem_wait_ld();
-                if (lt < Dv) {
+                const int lane = tid & 31;
+                uint8_t *ost = smem + OFF_A + 512 * warp;
+                const int tt = lane >> 2, dvc = 32 * (warp & 3) + 8 * (lane & 3);
 #pragma unroll
-                    for (int e = 0; e < 32; ++e) {
-                        const int i = 32 * half + e;
-                        if (i < ln)
-                            og[((t0 + i) * Hv + h) * (int64_t)Dv + lt] = elem16<F16>(p.scale * (y[e] + z[e]));
+                for (int g8 = 0; g8 < 4; ++g8) {
+#pragma unroll
+                    for (int e = 0; e < 8; ++e)
+                        *reinterpret_cast<uint16_t *>(ost + e * 64 + lane * 2) =
+                            elem16<F16>(p.scale * (y[8 * g8 + e] + z[8 * g8 + e]));
+                    __syncwarp();
+                    const uint4 v = *reinterpret_cast<const uint4 *>(ost + lane * 16);
+                    __syncwarp();
+                    const int i = 32 * half + 8 * g8 + tt;
+                    if (i < ln && dvc < Dv) {
+                        uint16_t *dst = og + ((t0 + i) * Hv + h) * (int64_t)Dv + dvc;
+                        if (vvec) {
+                            *reinterpret_cast<uint4 *>(dst) = v;
+                        } else {
+                            const uint16_t *ve = reinterpret_cast<const uint16_t *>(&v);
+                            for (int e = 0; e < 8 && dvc + e < Dv; ++e) dst[e] = ve[e];
+                        }
                     }
                 }
             }
