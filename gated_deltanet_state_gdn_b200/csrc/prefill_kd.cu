@@ -36,7 +36,7 @@
 //   (2)  S^T = S^T diag(e^{G_C}) + U^T (K^ e^{G_C - G})
 //   (3)  Z = U^T P^T                O^T = scale (Y + Z)
 //
-// One CTA of 256 threads per (request, value head), longest requests first: two
+// One CTA of 512 threads per (request, value head), longest requests first: four
 // warpgroups, whose thread t owns TMEM lane t (the state row dv = t) and which split each
 // row's columns between them.  The phases of a chunk run one after another (plain loads stage and scale the
 // operand tiles, thread 0 issues the MMAs, a bounded wait on one mbarrier ends each group).
@@ -52,7 +52,10 @@ using namespace sm100;
 namespace gdn_kd {
 
 constexpr int C = 64;            // chunk length (tokens)
-constexpr int NT = 256;          // threads per CTA: two warpgroups over the 128 TMEM lanes
+constexpr int NT = 512;          // threads per CTA: four warpgroups over the 128 TMEM lanes
+constexpr int NWG = NT / 128;    // warpgroups
+constexpr int BPW = 4 / NWG;     // 32-column state blocks per warpgroup
+constexpr int CPW = 64 / NWG;    // chunk columns (tokens) per warpgroup
 constexpr float G_FLOOR = -9.f;  // per-dimension log-decay floor
 constexpr float LOG2E = 1.4426950408889634f;
 
@@ -423,11 +426,12 @@ __global__ void __launch_bounds__(NT, 1) gdn_prefill_kd_kernel(const __grid_cons
     const uint32_t tl = tmem + ((uint32_t)(32 * (warp & 3)) << 16);   // this warp's TMEM lanes
     uint32_t phase = 0;
 
-    // state S^T (row dv = lt, column blocks 2 wg and 2 wg + 1) into TMEM, and its bf16 copy
+    // state S^T (row dv = lt, column blocks BPW wg .. BPW wg + BPW - 1) into TMEM, and its bf16
+    // copy
     {
         float x[32];
 #pragma unroll 1
-        for (int blk = 2 * wg; blk < 2 * wg + 2; ++blk) {
+        for (int blk = BPW * wg; blk < BPW * (wg + 1); ++blk) {
 #pragma unroll
             for (int e = 0; e < 32; ++e) {
                 const int dk = 32 * blk + e;
@@ -488,15 +492,15 @@ __global__ void __launch_bounds__(NT, 1) gdn_prefill_kd_kernel(const __grid_cons
         cp_async_wait_all();
         __syncthreads();
         // ---- per-dimension cumulative log-decay (log2 units) into G2: thread = key dimension,
-        //      warpgroup wg scans tokens [32 wg, 32 wg + 32); the second half then adds the
-        //      first's total
+        //      warpgroup wg scans tokens [CPW wg, CPW wg + CPW); each later segment then adds
+        //      the totals of the segments before it
         {
             const int d = lt;
             float acc = 0.f;
             const float ea = p.a_log ? expf(__ldg(p.a_log + h)) : 0.f;
             const float dtb = p.a_log ? __ldg(p.dt_bias + h) : 0.f;
 #pragma unroll 8
-            for (int i = 32 * wg; i < 32 * wg + 32; ++i) {
+            for (int i = CPW * wg; i < CPW * wg + CPW; ++i) {
                 float g = gn[i * 128 + d];
                 if (i < ln && d < Dk) {
                     if (p.a_log) g = -ea * gdn::softplus20(g + dtb);
@@ -507,11 +511,15 @@ __global__ void __launch_bounds__(NT, 1) gdn_prefill_kd_kernel(const __grid_cons
             }
         }
         __syncthreads();
-        if (wg == 1) {
+        {
             const int d = lt;
-            const float base = G2[31 * 128 + d];
+            float base = 0.f;
+            for (int m = 0; m < wg; ++m) base += G2[(CPW * m + CPW - 1) * 128 + d];
+            __syncthreads();
+            if (wg > 0) {
 #pragma unroll 8
-            for (int i = 32; i < 64; ++i) G2[i * 128 + d] += base;
+                for (int i = CPW * wg; i < CPW * wg + CPW; ++i) G2[i * 128 + d] += base;
+            }
         }
         if (tid < C) {
             float bt = 0.f;
@@ -641,8 +649,8 @@ __global__ void __launch_bounds__(NT, 1) gdn_prefill_kd_kernel(const __grid_cons
 
         // ---- A (key rows, fp32) and P (query rows, bf16 tile) from the Gram; TMEM lane = row;
         //      a warp's lanes 0-15 and 16-31 hold two consecutive 16-blocks, of which warpgroup
-        //      wg takes the (wg)th
-        {
+        //      wg (0 or 1) takes the (wg)th
+        if (wg < 2) {
             const bool isq = (warp & 3) >= 2;
             const int i = lt & 63;
             const int myI = i >> 4;
@@ -797,18 +805,20 @@ __global__ void __launch_bounds__(NT, 1) gdn_prefill_kd_kernel(const __grid_cons
         stall_bar = 0;
         if (!ok) break;
 
-        // ---- -W as the MN-major B operand of (1a): lane = dk row, tokens 32 wg .. 32 wg + 31
+        // ---- -W as the MN-major B operand of (1a): lane = dk row, tokens CPW wg .. + CPW - 1
         if (retrieval) {
             uint8_t *wn = smem + OFF_WNEG;
-            const int half = wg;
-            float x[32];
-            tmem_ld32(tl + TM_W + 32 * half, x);
-            tmem_wait_ld();
 #pragma unroll
-            for (int e = 0; e < 32; ++e) x[e] = -x[e];
+            for (int c16 = 0; c16 < CPW / 16; ++c16) {
+                const int col = CPW * wg + 16 * c16;
+                float x[16];
+                tmem_ld16(tl + TM_W + col, x);
+                tmem_wait_ld();
 #pragma unroll
-            for (int q = 0; q < 4; ++q)
-                *reinterpret_cast<uint4 *>(wn + sw128(lt, 4 * half + q)) = pack8<F16>(x + 8 * q);
+                for (int e = 0; e < 16; ++e) x[e] = -x[e];
+                *reinterpret_cast<uint4 *>(wn + sw128(lt, col / 8)) = pack8<F16>(x);
+                *reinterpret_cast<uint4 *>(wn + sw128(lt, col / 8 + 1)) = pack8<F16>(x + 8);
+            }
         }
         fence_proxy_async_smem();
         tc_fence_before();
@@ -840,16 +850,17 @@ __global__ void __launch_bounds__(NT, 1) gdn_prefill_kd_kernel(const __grid_cons
         {
             uint8_t *ub = smem + OFF_UB;
             float x[32];
-            {
-                const int half = wg;
-                tmem_ld32(tl + TM_U + 32 * half, x);
-                tmem_wait_ld();
 #pragma unroll
-                for (int q = 0; q < 4; ++q)
-                    *reinterpret_cast<uint4 *>(ub + sw128(lt, 4 * half + q)) = pack8<F16>(x + 8 * q);
+            for (int c16 = 0; c16 < CPW / 16; ++c16) {
+                const int col = CPW * wg + 16 * c16;
+                float u16[16];
+                tmem_ld16(tl + TM_U + col, u16);
+                tmem_wait_ld();
+                *reinterpret_cast<uint4 *>(ub + sw128(lt, col / 8)) = pack8<F16>(u16);
+                *reinterpret_cast<uint4 *>(ub + sw128(lt, col / 8 + 1)) = pack8<F16>(u16 + 8);
             }
 #pragma unroll 1
-            for (int blk = 2 * wg; blk < 2 * wg + 2; ++blk) {
+            for (int blk = BPW * wg; blk < BPW * (wg + 1); ++blk) {
                 tmem_ld32(tl + TM_S + 32 * blk, x);
                 tmem_wait_ld();
 #pragma unroll
@@ -880,23 +891,31 @@ __global__ void __launch_bounds__(NT, 1) gdn_prefill_kd_kernel(const __grid_cons
         stall_bar = 0;
         if (!ok) break;
 
-        // ---- outputs O^T = scale (Y + Z) (lane = dv, tokens 32 wg .. 32 wg + 31), then the new
-        //      state's bf16 copy (column blocks 2 wg, 2 wg + 1)
+        // ---- outputs O^T = scale (Y + Z) (lane = dv, tokens CPW wg .. CPW wg + CPW - 1), then
+        //      the new state's bf16 copy (column blocks BPW wg .. BPW wg + BPW - 1)
         {
-            float y[32], z[32];
+            float y[CPW], z[CPW];
             {
                 // 8 tokens at a time through a warp-private [8 tokens][32 dv] scratch (the solve
                 // area is free by now), then one 16-byte store per lane: lanes 4t..4t+3 write
                 // token t's 64 bytes of this warp's dv
-                const int half = wg;
-                tmem_ld32(tl + TM_Y + 32 * half, y);
-                tmem_ld32(tl + TM_Z + 32 * half, z);
-                tmem_wait_ld();
+#pragma unroll
+                for (int c16 = 0; c16 < CPW / 16; ++c16) {
+                    float y16[16], z16[16];
+                    tmem_ld16(tl + TM_Y + CPW * wg + 16 * c16, y16);
+                    tmem_ld16(tl + TM_Z + CPW * wg + 16 * c16, z16);
+                    tmem_wait_ld();
+#pragma unroll
+                    for (int e = 0; e < 16; ++e) {
+                        y[16 * c16 + e] = y16[e];
+                        z[16 * c16 + e] = z16[e];
+                    }
+                }
                 const int lane = tid & 31;
                 uint8_t *ost = smem + OFF_A + 512 * warp;
                 const int tt = lane >> 2, dvc = 32 * (warp & 3) + 8 * (lane & 3);
 #pragma unroll
-                for (int g8 = 0; g8 < 4; ++g8) {
+                for (int g8 = 0; g8 < CPW / 8; ++g8) {
 #pragma unroll
                     for (int e = 0; e < 8; ++e)
                         *reinterpret_cast<uint16_t *>(ost + e * 64 + lane * 2) =
@@ -904,7 +923,7 @@ __global__ void __launch_bounds__(NT, 1) gdn_prefill_kd_kernel(const __grid_cons
                     __syncwarp();
                     const uint4 v = *reinterpret_cast<const uint4 *>(ost + lane * 16);
                     __syncwarp();
-                    const int i = 32 * half + 8 * g8 + tt;
+                    const int i = CPW * wg + 8 * g8 + tt;
                     if (i < ln && dvc < Dv) {
                         uint16_t *dst = og + ((t0 + i) * Hv + h) * (int64_t)Dv + dvc;
                         if (vvec) {
@@ -917,10 +936,11 @@ __global__ void __launch_bounds__(NT, 1) gdn_prefill_kd_kernel(const __grid_cons
                 }
             }
 #pragma unroll 1
-            for (int blk = 2 * wg; blk < 2 * wg + 2; ++blk) {
-                tmem_ld32(tl + TM_S + 32 * blk, y);
+            for (int blk = BPW * wg; blk < BPW * (wg + 1); ++blk) {
+                float x[32];
+                tmem_ld32(tl + TM_S + 32 * blk, x);
                 tmem_wait_ld();
-                store_sb<F16>(smem + OFF_SB, lt, blk, y);
+                store_sb<F16>(smem + OFF_SB, lt, blk, x);
             }
         }
         fence_proxy_async_smem();
@@ -933,7 +953,7 @@ __global__ void __launch_bounds__(NT, 1) gdn_prefill_kd_kernel(const __grid_cons
         // final state (V-major, fp32); an empty request copies its initial state through
         float x[32];
 #pragma unroll 1
-        for (int blk = 2 * wg; blk < 2 * wg + 2; ++blk) {
+        for (int blk = BPW * wg; blk < BPW * (wg + 1); ++blk) {
             tmem_ld32(tl + TM_S + 32 * blk, x);
             tmem_wait_ld();
             if (lt < Dv)

@@ -267,10 +267,10 @@ def test_full_ragged_prefill_per_key_decay_all_heads(gdn, W, oracle_mod):
 
 
 def test_per_key_decay_many_requests(gdn, W, oracle_mod):
-    """300 requests of 0 to 70 tokens: more requests than the per-key kernel orders by length
+    """600 requests of 0 to 40 tokens: more requests than the per-key kernel orders by length
     (it then takes them in index order), every request and head against the oracle."""
     rng = np.random.default_rng(50)
-    lengths = rng.integers(0, 71, 300).tolist()
+    lengths = rng.integers(0, 41, 600).tolist()
     c = W.make_prefill(51, lengths, 1, 2, 32, 16, init_std=0.02, qk_l2norm=True,
                        decay_per_key=True)
     assert gdn.prefill_uses_chunked(torch.bfloat16, 2, 32, 16, decay_per_key=True)
