@@ -276,3 +276,14 @@ def test_per_key_decay_many_requests(gdn, W, oracle_mod):
     assert gdn.prefill_uses_chunked(torch.bfloat16, 2, 32, 16, decay_per_key=True)
     o, f, ro, rf = _run_both(gdn, oracle_mod, c, c.g, c.beta, False, decay_per_key=True)
     _parity(c, o, f, ro, rf, TOL_BF16)
+
+
+@pytest.mark.parametrize("sequential", [False, True])
+def test_per_key_decay_without_in_kernel_norm(gdn, W, oracle_mod, sequential):
+    """q and k unit-normalised on the host in fp32 before the bf16 cast, qk_l2norm off (the
+    long-context workload's convention), with a per-key decay: both per-key kernels against
+    the oracle."""
+    c = W.make_prefill(52, LENGTHS, 2, 4, 128, 128, init_std=0.02, qk_l2norm=False,
+                       host_norm_qk=True, decay_per_key=True)
+    o, f, ro, rf = _run_both(gdn, oracle_mod, c, c.g, c.beta, sequential, decay_per_key=True)
+    _parity(c, o, f, ro, rf, TOL_BF16)
