@@ -19,9 +19,12 @@
 //
 // This is the general path: fp32, bf16 or fp16 activations, any Dk, Dv in
 // [1, 256], any Hq | Hv.  It is also the sequential counterpart the chunked
-// tensor-core kernel is checked against.  Layout: grid (B * Hv, Dv tiles of
-// 32 rows); a warp owns 4 V-rows of S (V-major, one row = Dk floats), lane l
-// owns elements l + 32 j of each row; row dot products are warp reductions.
+// tensor-core kernel is checked against.  Layout: a 1-D grid of (request, value
+// head, tile of 32 V-rows) blocks, the tile index fastest and the requests
+// longest first (for up to 256 requests), so that the longest chains start in
+// the first wave of blocks; a warp owns 4 V-rows of S (V-major, one row = Dk
+// floats), lane l owns elements l + 32 j of each row; row dot products are warp
+// reductions.
 #include <cuda_fp16.h>
 
 #include "common.cuh"
@@ -67,13 +70,37 @@ __global__ void __launch_bounds__(kSeqWarps * 32)
 prefill_seq_kernel(const GdnPrefillArgs p)
 {
     constexpr int R = kSeqRows;
+    constexpr int NT = kSeqWarps * 32;
     const int lane = threadIdx.x & 31;
     const int warp = threadIdx.x >> 5;
     const int Hv = p.Hv, Hq = p.Hq, Dk = p.Dk, Dv = p.Dv;
-    const int b = blockIdx.x / Hv;
-    const int h = blockIdx.x - b * Hv;
+    const int tiles = (Dv + kSeqWarps * R - 1) / (kSeqWarps * R);
+    const int unit = (int)(blockIdx.x / (unsigned)tiles);
+    const int tile = (int)blockIdx.x - unit * tiles;
+    int b = unit / Hv;
+    const int h = unit - b * Hv;
+    // request of rank b in decreasing length (ties by index)
+    if (p.cu_seqlens && p.B > 1 && p.B <= NT) {
+        __shared__ int lens[NT];
+        __shared__ int pick;
+        const int t = threadIdx.x;
+        if (t < p.B) {
+            const int64_t st = clamp_i64(p.cu_seqlens[t], 0, p.N);
+            const int64_t en = clamp_i64(p.cu_seqlens[t + 1], 0, p.N);
+            lens[t] = en > st ? (int)(en - st) : 0;
+        }
+        __syncthreads();
+        if (t < p.B) {
+            const int li = lens[t];
+            int rank = 0;
+            for (int j2 = 0; j2 < p.B; ++j2) rank += (lens[j2] > li) || (lens[j2] == li && j2 < t);
+            if (rank == b) pick = t;
+        }
+        __syncthreads();
+        b = pick;
+    }
     const int qh = (int)(((int64_t)h * Hq) / Hv);
-    const int row_base = blockIdx.y * (kSeqWarps * R) + warp * R;
+    const int row_base = tile * (kSeqWarps * R) + warp * R;
     if (row_base >= Dv) return;  // whole warp idle (uniform)
 
     int64_t start, end;
@@ -239,8 +266,9 @@ prefill_seq_kernel(const GdnPrefillArgs p)
 template <typename Tin, bool PER_KEY>
 static cudaError_t launch_seq_t(const GdnPrefillArgs &a, cudaStream_t stream)
 {
-    dim3 grid((unsigned)a.B * (unsigned)a.Hv, (unsigned)((a.Dv + kSeqWarps * kSeqRows - 1) /
-                                                         (kSeqWarps * kSeqRows)));
+    const unsigned tiles = (unsigned)((a.Dv + kSeqWarps * kSeqRows - 1) / (kSeqWarps * kSeqRows));
+    if ((uint64_t)a.B * a.Hv * tiles > 0x7fffffffull) return cudaErrorInvalidConfiguration;
+    dim3 grid((unsigned)a.B * (unsigned)a.Hv * tiles);
     dim3 block(kSeqWarps * 32);
     if (a.Dk <= 32)
         prefill_seq_kernel<Tin, 1, PER_KEY><<<grid, block, 0, stream>>>(a);
