@@ -630,7 +630,10 @@ __global__ void __launch_bounds__(NT, 1) gdn_prefill_kd_kernel(const __grid_cons
         fence_proxy_async_smem();
         __syncthreads();
 
-        // ---- (G): all blocks' products in one MMA; then the next chunk's rows are requested
+        // ---- (G): all blocks' products in one MMA; then (1b) Y = S^T (Q^ e^G)^T, which needs
+        //      only the state's bf16 copy and this tile: it runs under the A/P build and the
+        //      solve, outside the commit that is waited for next (the later commits cover it);
+        //      then the next chunk's rows are requested
         if (tid == 0) {
             tc_fence_after();
             const uint64_t dA = sdesc_sw128(sbase + OFF_ASIDE, 16, 1024);
@@ -640,6 +643,12 @@ __global__ void __launch_bounds__(NT, 1) gdn_prefill_kd_kernel(const __grid_cons
                 umma_bf16(tmem + TM_G, dA + (((kk >> 2) * ASIDE_KB + (kk & 3) * 32) >> 4),
                           dB + (((kk >> 2) * BCAT_KB + (kk & 3) * 32) >> 4), ID_G, kk > 0);
             umma_commit(bar);
+            const uint64_t dSB = sdesc_sw128(sbase + OFF_SB, 16, 1024);
+            const uint64_t dQG = sdesc_sw128(sbase + OFF_QG, 16, 1024);
+#pragma unroll 1
+            for (int kk = 0; kk < 8; ++kk)
+                umma_bf16(tmem + TM_Y, dSB + (((kk >> 2) * 16384 + (kk & 3) * 32) >> 4),
+                          dQG + (((kk >> 2) * TILE_KB + (kk & 3) * 32) >> 4), ID_1B, kk > 0);
         }
         if (n + 1 < nc) load_rows(n + 1);
         ok = cta_wait_mma(stall_bar ? stall_bar : bar, phase, flag, p.dev_status);
@@ -824,22 +833,17 @@ __global__ void __launch_bounds__(NT, 1) gdn_prefill_kd_kernel(const __grid_cons
         tc_fence_before();
         __syncthreads();
 
-        // ---- (1a) U^T += S^T (-W)^T, (1b) Y = S^T (Q^ e^G)^T
+        // ---- (1a) U^T += S^T (-W)^T
         if (tid == 0) {
             tc_fence_after();
             const uint64_t dSB = sdesc_sw128(sbase + OFF_SB, 16, 1024);
             const uint64_t dWN = sdesc_sw128(sbase + OFF_WNEG, 8192, 1024);
-            const uint64_t dQG = sdesc_sw128(sbase + OFF_QG, 16, 1024);
             if (retrieval) {
 #pragma unroll 1
                 for (int kk = 0; kk < 8; ++kk)
                     umma_bf16(tmem + TM_U, dSB + (((kk >> 2) * 16384 + (kk & 3) * 32) >> 4),
                               dWN + ((kk * 2048) >> 4), ID_1A, 1);
             }
-#pragma unroll 1
-            for (int kk = 0; kk < 8; ++kk)
-                umma_bf16(tmem + TM_Y, dSB + (((kk >> 2) * 16384 + (kk & 3) * 32) >> 4),
-                          dQG + (((kk >> 2) * TILE_KB + (kk & 3) * 32) >> 4), ID_1B, kk > 0);
             umma_commit(bar);
         }
         ok = cta_wait_mma(stall_bar ? stall_bar : bar, phase, flag, p.dev_status);
