@@ -74,6 +74,7 @@
 #include "common.cuh"
 #include "seqpar.cuh"
 #include "sm100.cuh"
+#include "tile16.cuh"
 
 using namespace sm100;
 
@@ -81,6 +82,15 @@ namespace gdn_chunk {
 
 using gdn::in_range;
 using gdn::kChecked;
+using gdn_tile::a_slot;
+using gdn_tile::blk_mma;
+using gdn_tile::blk_store;
+using gdn_tile::elem16;
+using gdn_tile::pack2;
+using gdn_tile::pack8;
+using gdn_tile::SOLVE_BLK;
+using gdn_tile::SOLVE_LD;
+using gdn_tile::sw128;
 
 constexpr int C = 64;       // chunk length (tokens)
 constexpr int D = 128;      // Dk = Dv
@@ -102,9 +112,7 @@ constexpr uint32_t OFF_P = 131072;       // KQ_STAGES x [64 rows i][64 j], 8 KB 
 constexpr uint32_t P_STAGE = 8192;
 constexpr uint32_t OFF_TB = OFF_P + KQ_STAGES * P_STAGE;   // [64 rows i][64 j], 8 KB
 constexpr uint32_t OFF_TBG = OFF_TB + 8192;
-constexpr uint32_t SOLVE_LD = 20;        // padded row stride (floats)
-constexpr uint32_t SOLVE_BLK = 16 * SOLVE_LD;  // floats per block
-constexpr uint32_t SOLVE_BYTES = 16 * SOLVE_BLK * 4;
+constexpr uint32_t SOLVE_BYTES = 16 * SOLVE_BLK * 4;   // 16 padded 16 x 16 fp32 blocks
 constexpr uint32_t OFF_SOLVE0 = OFF_TBG + 8192;   // two areas of 16 blocks of 16 x 20 fp32
 constexpr uint32_t OFF_SOLVE1 = OFF_SOLVE0 + SOLVE_BYTES;
 constexpr uint32_t OFF_GB0 = OFF_SOLVE1 + SOLVE_BYTES;         // KQ_STAGES x (g tile 1 KB + beta tile 1 KB)
@@ -218,48 +226,6 @@ __device__ __forceinline__ Unit load_unit(const uint8_t *smem, int k)
 __device__ __forceinline__ int64_t clampi(int64_t x, int64_t lo, int64_t hi)
 {
     return x < lo ? lo : (x > hi ? hi : x);
-}
-
-// 16-byte chunk `c` of row `r` in a 128B-swizzled tile whose base is 1024-aligned
-__device__ __forceinline__ uint32_t sw128(uint32_t row, uint32_t c)
-{
-    return row * 128u + ((c ^ (row & 7u)) << 4);
-}
-
-// 16-bit operand element: bf16, or fp16 (F16) for fp16 activations; every tile the tensor
-// cores read has the activations' type, since an MMA takes A and B of one type
-template <bool F16>
-__device__ __forceinline__ uint32_t pack2(float lo, float hi)
-{
-    if constexpr (F16) {
-        const __half2 v = __floats2half2_rn(lo, hi);
-        return *reinterpret_cast<const uint32_t *>(&v);
-    } else {
-        return gdn::pack_bf16x2(lo, hi);
-    }
-}
-
-template <bool F16>
-__device__ __forceinline__ uint16_t elem16(float x)
-{
-    if constexpr (F16) {
-        const __half v = __float2half_rn(x);
-        return *reinterpret_cast<const uint16_t *>(&v);
-    } else {
-        const __nv_bfloat16 v = __float2bfloat16_rn(x);
-        return *reinterpret_cast<const uint16_t *>(&v);
-    }
-}
-
-template <bool F16 = false>
-__device__ __forceinline__ uint4 pack8_bf16(const float *x)
-{
-    uint4 r;
-    r.x = pack2<F16>(x[0], x[1]);
-    r.y = pack2<F16>(x[2], x[3]);
-    r.z = pack2<F16>(x[4], x[5]);
-    r.w = pack2<F16>(x[6], x[7]);
-    return r;
 }
 
 template <bool F16 = false>
@@ -535,44 +501,6 @@ __device__ __noinline__ void build_unit_list(const Params &p, uint8_t *smem, int
     *count_out = total;
 }
 
-// --------------------------------------------------------------------------
-// warp-level 16x16x16 tf32 products on padded fp32 blocks (row stride SOLVE_LD); the
-// fp32 bits are passed as they are and the tensor core reads them as tf32
-// acc[nh][.] += X(16x16) * Y(16x16), fragments of mma.m16n8k8
-__device__ __forceinline__ void blk_mma(float (&acc)[2][4], const float *X, const float *Y)
-{
-    const int lane = threadIdx.x & 31;
-    const int g = lane >> 2, t = lane & 3;
-#pragma unroll
-    for (int kh = 0; kh < 2; ++kh) {
-        uint32_t a[4];
-        a[0] = __float_as_uint(X[g * SOLVE_LD + 8 * kh + t]);
-        a[1] = __float_as_uint(X[(g + 8) * SOLVE_LD + 8 * kh + t]);
-        a[2] = __float_as_uint(X[g * SOLVE_LD + 8 * kh + t + 4]);
-        a[3] = __float_as_uint(X[(g + 8) * SOLVE_LD + 8 * kh + t + 4]);
-#pragma unroll
-        for (int nh = 0; nh < 2; ++nh) {
-            uint32_t b[2];
-            b[0] = __float_as_uint(Y[(8 * kh + t) * SOLVE_LD + 8 * nh + g]);
-            b[1] = __float_as_uint(Y[(8 * kh + t + 4) * SOLVE_LD + 8 * nh + g]);
-            mma_tf32_16x8x8(acc[nh], a, b);
-        }
-    }
-}
-
-__device__ __forceinline__ void blk_store(float *Z, const float (&acc)[2][4], float sgn)
-{
-    const int lane = threadIdx.x & 31;
-    const int g = lane >> 2, t = lane & 3;
-#pragma unroll
-    for (int nh = 0; nh < 2; ++nh) {
-        *reinterpret_cast<float2 *>(Z + g * SOLVE_LD + 8 * nh + 2 * t) =
-            make_float2(sgn * acc[nh][0], sgn * acc[nh][1]);
-        *reinterpret_cast<float2 *>(Z + (g + 8) * SOLVE_LD + 8 * nh + 2 * t) =
-            make_float2(sgn * acc[nh][2], sgn * acc[nh][3]);
-    }
-}
-
 // Block (I, J) of T' from an mma fragment (times sgn), written to the bf16 operand
 // tiles Tb = T' diag(beta rk) and Tbg = T' diag(beta Gamma rk^2) (K-major, 128B-swizzled)
 template <bool F16>
@@ -596,12 +524,7 @@ __device__ __forceinline__ void blk_store_tiles(const float (&acc)[2][4], float 
     }
 }
 
-// SOLVE slots: 0-3 A_II (strictly lower), 4 A_10, 5 A_32, 6-9 A_20 A_21 A_30 A_31
-// (later X, later T_20 T_21 T_30 T_31), 10-13 D_I = (I + A_II)^-1, 14 T_10, 15 T_32.
-__host__ __device__ constexpr int a_slot(int I, int J)
-{
-    return I == 1 ? 4 : (I == 2 ? 6 + J : (J == 2 ? 5 : 8 + J));
-}
+// SOLVE slots (see tile16.cuh): the X products later hold T_20 T_21 T_30 T_31.
 
 __device__ __forceinline__ int t_slot(int I, int J)
 {
@@ -677,8 +600,8 @@ __device__ __forceinline__ float build_row(uint32_t tl_gram, int qd, const float
         }
         // ---- stores
         if (isP) {
-            *reinterpret_cast<uint4 *>(ptile + sw128(i, 2 * J)) = pack8_bf16<F16>(x);
-            *reinterpret_cast<uint4 *>(ptile + sw128(i, 2 * J + 1)) = pack8_bf16<F16>(x + 8);
+            *reinterpret_cast<uint4 *>(ptile + sw128(i, 2 * J)) = pack8<F16>(x);
+            *reinterpret_cast<uint4 *>(ptile + sw128(i, 2 * J + 1)) = pack8<F16>(x + 8);
         } else {
             float *row = solve + (J == I ? I : a_slot(I, J)) * SOLVE_BLK + r * SOLVE_LD;
 #pragma unroll
@@ -1392,7 +1315,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) gdn_prefill_chunk_kernel(const __
                     for (int e = 0; e < 32; ++e) t[e] = -t[e];
 #pragma unroll
                     for (int c = 0; c < 4; ++c)
-                        *reinterpret_cast<uint4 *>(smem + OFF_WNEG + sw128(dv, 4 * q + c)) = pack8_bf16<F16>(t + 8 * c);
+                        *reinterpret_cast<uint4 *>(smem + OFF_WNEG + sw128(dv, 4 * q + c)) = pack8<F16>(t + 8 * c);
                 }
                 fence_proxy_async_smem();
                 tc_fence_before();

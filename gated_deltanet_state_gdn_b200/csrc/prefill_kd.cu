@@ -46,10 +46,21 @@
 
 #include "common.cuh"
 #include "sm100.cuh"
+#include "tile16.cuh"
 
 using namespace sm100;
 
 namespace gdn_kd {
+
+using gdn_tile::a_slot;
+using gdn_tile::blk_mma;
+using gdn_tile::blk_store;
+using gdn_tile::elem16;
+using gdn_tile::pack2;
+using gdn_tile::pack8;
+using gdn_tile::SOLVE_BLK;
+using gdn_tile::SOLVE_LD;
+using gdn_tile::sw128;
 
 constexpr int C = 64;            // chunk length (tokens)
 constexpr int NT = 512;          // threads per CTA: four warpgroups over the 128 TMEM lanes
@@ -80,8 +91,6 @@ constexpr uint32_t OFF_SB = 139264;      // bf16 S^T      [kb 2][128 rows dv][12
 // region X: log-decays, then (after the operands are built) A and Tb
 constexpr uint32_t OFF_G2 = 172032;      // fp32 [64][128]: G * log2(e)
 constexpr uint32_t OFF_A = 172032;       // solve area: 16 fp32 blocks of 16 x SOLVE_LD
-constexpr uint32_t SOLVE_LD = 20;        // padded row stride (floats)
-constexpr uint32_t SOLVE_BLK = 16 * SOLVE_LD;
 constexpr uint32_t OFF_TB = 192512;      // [64 rows i][64 j], K-major B of (W), (U~)
 constexpr uint32_t OFF_VEC = 204800;     // per-dimension vectors, fp32
 constexpr int VEC_EM = 0;        // e^{M_I}                 [4][128]
@@ -105,46 +114,11 @@ static_assert(OFF_TB % 1024 == 0 && OFF_SB % 1024 == 0 && OFF_VT % 1024 == 0 &&
 // TMEM columns: the Gram's 160 columns are reused by W and U once A and P are read
 constexpr uint32_t TM_S = 0, TM_G = 128, TM_W = 128, TM_U = 192, TM_Y = 288, TM_Z = 352;
 
-__device__ __forceinline__ uint32_t sw128(uint32_t row, uint32_t c)
-{
-    return row * 128u + ((c ^ (row & 7u)) << 4);
-}
-
-template <bool F16>
-__device__ __forceinline__ uint32_t pack2(float lo, float hi)
-{
-    if constexpr (F16) {
-        const __half2 v = __floats2half2_rn(lo, hi);
-        return *reinterpret_cast<const uint32_t *>(&v);
-    } else {
-        return gdn::pack_bf16x2(lo, hi);
-    }
-}
-
-template <bool F16>
-__device__ __forceinline__ uint4 pack8(const float *x)
-{
-    return make_uint4(pack2<F16>(x[0], x[1]), pack2<F16>(x[2], x[3]), pack2<F16>(x[4], x[5]),
-                      pack2<F16>(x[6], x[7]));
-}
-
 template <bool F16>
 __device__ __forceinline__ float to_f(uint16_t b)
 {
     if constexpr (F16) return __half2float(*reinterpret_cast<const __half *>(&b));
     else return __uint_as_float((uint32_t)b << 16);
-}
-
-template <bool F16>
-__device__ __forceinline__ uint16_t elem16(float x)
-{
-    if constexpr (F16) {
-        const __half v = __float2half_rn(x);
-        return *reinterpret_cast<const uint16_t *>(&v);
-    } else {
-        const __nv_bfloat16 v = __float2bfloat16_rn(x);
-        return *reinterpret_cast<const uint16_t *>(&v);
-    }
 }
 
 // 16-byte global -> shared asynchronous copy (both addresses 16-byte aligned)
@@ -156,30 +130,6 @@ __device__ __forceinline__ void cp_async16(uint32_t dst, const void *src)
 __device__ __forceinline__ void cp_async_wait_all()
 {
     asm volatile("cp.async.wait_all;" ::: "memory");
-}
-
-// elements [8c, 8c + 8) of a row of `n` 16-bit values (zero past n); `vec`: the row start is
-// 16-byte aligned and n % 8 == 0
-template <bool F16>
-__device__ __forceinline__ void load8(const uint16_t *row, int c, int n, bool vec, float (&x)[8])
-{
-    if (vec) {
-        if (8 * c < n) {
-            const uint4 r = __ldg(reinterpret_cast<const uint4 *>(row) + c);
-            const uint32_t w[4] = {r.x, r.y, r.z, r.w};
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-                x[2 * e] = to_f<F16>((uint16_t)(w[e] & 0xffffu));
-                x[2 * e + 1] = to_f<F16>((uint16_t)(w[e] >> 16));
-            }
-            return;
-        }
-#pragma unroll
-        for (int e = 0; e < 8; ++e) x[e] = 0.f;
-        return;
-    }
-#pragma unroll
-    for (int e = 0; e < 8; ++e) x[e] = (8 * c + e < n) ? to_f<F16>(row[8 * c + e]) : 0.f;
 }
 
 // 8 consecutive floats from 32-byte aligned shared memory
@@ -224,49 +174,6 @@ __device__ __forceinline__ void store_sb(uint8_t *sb, int dv, int blk, const flo
     for (int q = 0; q < 4; ++q) {
         const int ch = 4 * (blk & 1) + q;   // 16-byte chunk within the 64-dk k-block
         *reinterpret_cast<uint4 *>(sb + (blk >> 1) * 16384 + sw128(dv, ch)) = pack8<F16>(x + 8 * q);
-    }
-}
-
-// ---- blocked solve of T = (I + A)^-1 (A strictly lower, 4 x 4 blocks of 16)
-// slots of the solve area: 0-3 A_II, 4 A_10, 5 A_32, 6-9 A_20 A_21 A_30 A_31 (later the
-// products X), 10-13 D_I = (I + A_II)^-1, 14 T_10, 15 T_32
-__host__ __device__ constexpr int a_slot(int I, int J)
-{
-    return I == 1 ? 4 : (I == 2 ? 6 + J : (J == 2 ? 5 : 8 + J));
-}
-
-// acc[nh][.] += X(16x16) * Y(16x16) on padded fp32 blocks, tf32 inputs (mma.m16n8k8 fragments)
-__device__ __forceinline__ void blk_mma(float (&acc)[2][4], const float *X, const float *Y)
-{
-    const int lane = threadIdx.x & 31;
-    const int g = lane >> 2, t = lane & 3;
-#pragma unroll
-    for (int kh = 0; kh < 2; ++kh) {
-        uint32_t a[4];
-        a[0] = __float_as_uint(X[g * SOLVE_LD + 8 * kh + t]);
-        a[1] = __float_as_uint(X[(g + 8) * SOLVE_LD + 8 * kh + t]);
-        a[2] = __float_as_uint(X[g * SOLVE_LD + 8 * kh + t + 4]);
-        a[3] = __float_as_uint(X[(g + 8) * SOLVE_LD + 8 * kh + t + 4]);
-#pragma unroll
-        for (int nh = 0; nh < 2; ++nh) {
-            uint32_t b[2];
-            b[0] = __float_as_uint(Y[(8 * kh + t) * SOLVE_LD + 8 * nh + g]);
-            b[1] = __float_as_uint(Y[(8 * kh + t + 4) * SOLVE_LD + 8 * nh + g]);
-            mma_tf32_16x8x8(acc[nh], a, b);
-        }
-    }
-}
-
-__device__ __forceinline__ void blk_store(float *Z, const float (&acc)[2][4], float sgn)
-{
-    const int lane = threadIdx.x & 31;
-    const int g = lane >> 2, t = lane & 3;
-#pragma unroll
-    for (int nh = 0; nh < 2; ++nh) {
-        *reinterpret_cast<float2 *>(Z + g * SOLVE_LD + 8 * nh + 2 * t) =
-            make_float2(sgn * acc[nh][0], sgn * acc[nh][1]);
-        *reinterpret_cast<float2 *>(Z + (g + 8) * SOLVE_LD + 8 * nh + 2 * t) =
-            make_float2(sgn * acc[nh][2], sgn * acc[nh][3]);
     }
 }
 
