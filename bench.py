@@ -62,22 +62,47 @@ def load_peaks():
             "source": "fallback"}
 
 
-def ncu_traffic(profile_name: str, source: str):
-    """DRAM bytes per launch recorded in profiles/<profile_name> by an ncu capture, or None when
-    the kernel source changed since (the summary stores the first 16 hex of its sha256)."""
+def source_digest(source: str):
+    """First 16 hex of the sha256 over a kernel file and, depth first, every header of csrc/ that
+    it includes with quotes (each counted once), or None when the file is missing.  A change to a
+    shared device header therefore counts as a change of every kernel that includes it."""
     import hashlib
     import re
+    csrc = os.path.join(ROOT, "gated_deltanet_state_gdn_b200", "csrc")
+    h = hashlib.sha256()
+    seen = set()
+
+    def visit(name):
+        path = os.path.join(csrc, name)
+        if name in seen or not os.path.exists(path):
+            return
+        seen.add(name)
+        data = open(path, "rb").read()
+        h.update(data)
+        for inc in re.findall(rb'^\s*#\s*include\s*"([^"]+)"', data, re.M):
+            visit(inc.decode())
+
+    if not os.path.exists(os.path.join(csrc, source)):
+        return None
+    visit(source)
+    return h.hexdigest()[:16]
+
+
+def ncu_traffic(profile_name: str, source: str, key: str = "traffic_bytes_per_launch"):
+    """DRAM bytes recorded under `key` (per launch, or per call for a call of several launches)
+    in profiles/<profile_name> by an ncu capture, or None when the kernel source changed since
+    (the summary stores source_digest of the sources it was captured on)."""
+    import re
     path = os.path.join(ROOT, "profiles", profile_name)
-    src = os.path.join(ROOT, "gated_deltanet_state_gdn_b200", "csrc", source)
-    if not (os.path.exists(path) and os.path.exists(src)):
+    digest = source_digest(source)
+    if not (os.path.exists(path) and digest):
         return None
     text = open(path).read()
-    m_t = re.search(r"^traffic_bytes_per_launch:\s*(\d+)", text, re.M)
+    m_t = re.search(r"^" + re.escape(key) + r":\s*(\d+)", text, re.M)
     m_h = re.search(r"^source_sha256_16:\s*([0-9a-f]+)", text, re.M)
     if not (m_t and m_h):
         return None
-    sha = hashlib.sha256(open(src, "rb").read()).hexdigest()[:16]
-    return int(m_t.group(1)) if sha == m_h.group(1) else None
+    return int(m_t.group(1)) if digest == m_h.group(1) else None
 
 
 def prefill_flops_per_token_head(Dk, Dv, C=CHUNK):
@@ -736,7 +761,10 @@ def main():
         long_prefill = {
             "workload": lcase.name, "tokens": lcase.N, "ms_per_step": l_max,
             "value": job_throughput(lcase.N, world, l_max), "unit": "tokens/s",
-            "roofline": prefill_roofline(gdn, lcase, l_launch, peaks, l_clocks["sm_mhz"], None),
+            "roofline": prefill_roofline(
+                gdn, lcase, l_launch, peaks, l_clocks["sm_mhz"],
+                ncu_traffic("prefill_chunk_long_split.md", "prefill_chunk.cu",
+                            "traffic_bytes_per_call")),
             "repeat_windows_ms_per_launch": time_prefill.repeats, "clocks": l_clocks}
         # a call that takes the sequence split launches three kernels: two passes and the
         # composition of the segment maps
@@ -744,6 +772,9 @@ def main():
         splits = gdn.lib().gdn_prefill_workspace_size(lcase.B, lcase.N, Hq_l, Hv_l, Dk_l, Dv_l,
                                                       gdn.GDN_BF16, 0) > 0
         long_prefill["kernels_per_call"] = 3 if splits else 1
+        if long_prefill["roofline"].get("traffic") is not None:
+            long_prefill["roofline"]["traffic_scope"] = \
+                "one call: both passes and the composition of the segment maps"
         launches += time_prefill.launches * long_prefill["kernels_per_call"]
         del lcase
 

@@ -5,8 +5,8 @@
 * the prefill's algorithmic HBM bytes, counted term by term here (q, k, v, out in the
   activations' type, g and beta in fp32 -- g with Dk values per token and head in the
   per-key-dimension spelling --, states in fp32, cu_seqlens);
-* the DRAM traffic read from a committed ncu summary only while the kernel source still has the
-  hash the summary records.
+* the DRAM traffic read from a committed ncu summary only while the kernel source, with the csrc
+  headers it includes, still has the digest the summary records.
 """
 import os
 import sys
@@ -52,3 +52,26 @@ def test_profile_traffic_follows_the_source_hash(bench):
     # a different source file never matches a summary's hash
     assert bench.ncu_traffic("prefill_kd_ragged_per_key.md", "decode.cu") is None
     assert bench.ncu_traffic("no_such_profile.md", "prefill_kd.cu") is None
+
+
+def test_source_digest_covers_included_headers(bench):
+    import hashlib
+    csrc = os.path.join(ROOT, "gated_deltanet_state_gdn_b200", "csrc")
+
+    def raw(name):
+        return open(os.path.join(csrc, name), "rb").read()
+
+    # prefill_kd.cu includes common.cuh, sm100.cuh and tile16.cuh (which includes the first two
+    # again); each header enters the digest once, depth first, after the file that includes it
+    want = hashlib.sha256(raw("prefill_kd.cu") + raw("common.cuh") + raw("sm100.cuh")
+                          + raw("tile16.cuh")).hexdigest()[:16]
+    assert bench.source_digest("prefill_kd.cu") == want
+    assert bench.source_digest("prefill_kd.cu") != hashlib.sha256(raw("prefill_kd.cu")).hexdigest()[:16]
+    assert bench.source_digest("no_such_kernel.cu") is None
+
+
+def test_profile_traffic_keys(bench):
+    # the long-context summary records DRAM bytes per call (three launches), not per launch
+    assert bench.ncu_traffic("prefill_chunk_long_split.md", "prefill_chunk.cu") is None
+    t = bench.ncu_traffic("prefill_chunk_long_split.md", "prefill_chunk.cu", "traffic_bytes_per_call")
+    assert t is None or t > 0
