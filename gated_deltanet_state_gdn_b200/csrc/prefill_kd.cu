@@ -38,8 +38,10 @@
 //
 // One CTA of 512 threads per (request, value head), longest requests first: four
 // warpgroups, whose thread t owns TMEM lane t (the state row dv = t) and which split each
-// row's columns between them.  The phases of a chunk run one after another (plain loads stage and scale the
-// operand tiles, thread 0 issues the MMAs, a bounded wait on one mbarrier ends each group).
+// row's columns between them.  The phases of a chunk run one after another: plain loads stage
+// and scale the operand tiles, thread 0 issues the MMAs and a bounded wait on an mbarrier ends
+// each group.  (1b) alone is issued by another thread, with its own mbarrier, while the tensor
+// pipe is idle, and the output phase waits for it.
 // The triangular solve works on 16 x 16 blocks: fp32 forward substitution inside the four
 // diagonal blocks, then tf32 warp MMAs merge the blocks below the diagonal.
 #include <cuda_fp16.h>
@@ -67,6 +69,7 @@ constexpr int NT = 512;          // threads per CTA: four warpgroups over the 12
 constexpr int NWG = NT / 128;    // warpgroups
 constexpr int BPW = 4 / NWG;     // 32-column state blocks per warpgroup
 constexpr int CPW = 64 / NWG;    // chunk columns (tokens) per warpgroup
+static_assert(NWG == 4 && CPW == 16, "the decay scan gives warpgroup I the tokens of block I");
 constexpr float G_FLOOR = -9.f;  // per-dimension log-decay floor
 constexpr float LOG2E = 1.4426950408889634f;
 
@@ -98,6 +101,7 @@ constexpr int VEC_CM = 512;      // e^{M_I' - M_I}, I' > I  [6][128]
 constexpr int VEC_EC3 = 1280;    // e^{G_C - M_3}           [128]
 constexpr int VEC_GC = 1408;     // e^{G_C}                 [128]
 constexpr int VEC_M2 = 1536;     // M_I * log2(e)           [4][128]
+constexpr int VEC_TOT = VEC_CM;  // segment totals of the scan [3][128], before e^{M_I' - M_I}
 constexpr uint32_t OFF_ROW = OFF_VEC + 2048 * 4;   // per-token values, fp32
 constexpr int ROW_BETA = 0, ROW_QK = 64;   // beta_j; rq_j rk_j (q_j . k_j)
 constexpr uint32_t OFF_BAR = OFF_ROW + 1024;       // mbarrier, TMEM base, flag
@@ -113,6 +117,10 @@ static_assert(OFF_TB % 1024 == 0 && OFF_SB % 1024 == 0 && OFF_VT % 1024 == 0 &&
 
 // TMEM columns: the Gram's 160 columns are reused by W and U once A and P are read
 constexpr uint32_t TM_S = 0, TM_G = 128, TM_W = 128, TM_U = 192, TM_Y = 288, TM_Z = 352;
+
+// the thread that issues (1b): lane 0 of warp 12, whose lane quarter (key rows of blocks 0-1)
+// needs only three A/P loads, dealt to warpgroups 0-2
+constexpr int Y_ISSUER = 384;
 
 template <bool F16>
 __device__ __forceinline__ float to_f(uint16_t b)
@@ -220,23 +228,34 @@ __device__ __forceinline__ void stage_g(float *dst, const GdnPrefillArgs &p, int
     }
 }
 
-// thread 0 waits (bounded) on `wbar` for the MMA group committed to it; every thread gets the
-// outcome.  (Checked builds with GDN_DEV_TEST_STALL pass, once, a barrier that nothing arrives
-// on instead of the commit barrier, so that the wait runs out.)
+// bounded wait for the phase of `wbar` with parity `parity`
+__device__ __forceinline__ bool mbar_wait_bounded(uint32_t wbar, uint32_t parity)
+{
+    bool good = mbar_try_wait(wbar, parity);
+    if (!good) {
+        const long long t0 = clock64();
+        while (!(good = mbar_try_wait(wbar, parity)))
+            if (clock64() - t0 > (1ll << 31)) break;
+    }
+    return good;
+}
+
+// thread 0 waits (bounded) on `wbar` for the MMA group committed to it, and also on `wbar2`
+// when given; every thread gets the outcome.  (Checked builds with GDN_DEV_TEST_STALL pass,
+// once, a barrier that nothing arrives on instead of the commit barrier, so that the wait runs
+// out.)
 __device__ __forceinline__ bool cta_wait_mma(uint32_t wbar, uint32_t &phase, volatile int *flag,
-                                             int32_t *status)
+                                             int32_t *status, uint32_t wbar2 = 0,
+                                             uint32_t *phase2 = nullptr)
 {
     if (threadIdx.x == 0) {
-        bool good = mbar_try_wait(wbar, phase & 1);
-        if (!good) {
-            const long long t0 = clock64();
-            while (!(good = mbar_try_wait(wbar, phase & 1)))
-                if (clock64() - t0 > (1ll << 31)) break;
-        }
+        bool good = mbar_wait_bounded(wbar, phase & 1);
+        if (good && wbar2) good = mbar_wait_bounded(wbar2, *phase2 & 1);
         if (!good && status) atomicOr(status, GDN_DEV_TIMEOUT);
         *flag = good ? 1 : 0;
     }
     ++phase;
+    if (wbar2) ++*phase2;
     __syncthreads();
     const bool good = *flag != 0;
     tc_fence_after();
@@ -306,6 +325,7 @@ __global__ void __launch_bounds__(NT, 1) gdn_prefill_kd_kernel(const __grid_cons
     const bool kvec = (Dk & 7) == 0, vvec = (Dv & 7) == 0;
 
     const uint32_t bar = sbase + OFF_BAR;
+    const uint32_t bar_y = sbase + OFF_BAR + 40;   // commits of (1b), issued by Y_ISSUER
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + OFF_BAR + 8);
     volatile int *flag = reinterpret_cast<volatile int *>(smem + OFF_BAR + 12);
     // checked builds, GDN_DEV_TEST_STALL: the first MMA wait of CTA 0 runs on a barrier that
@@ -319,6 +339,7 @@ __global__ void __launch_bounds__(NT, 1) gdn_prefill_kd_kernel(const __grid_cons
     if (tid == 0) {
         mbar_init(bar, 1);
         mbar_init(sbase + OFF_BAR + 16, 1);
+        mbar_init(bar_y, 1);
         fence_mbar_init();
         *flag = 1;
     }
@@ -331,7 +352,11 @@ __global__ void __launch_bounds__(NT, 1) gdn_prefill_kd_kernel(const __grid_cons
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
     const uint32_t tl = tmem + ((uint32_t)(32 * (warp & 3)) << 16);   // this warp's TMEM lanes
-    uint32_t phase = 0;
+    uint32_t phase = 0, phase_y = 0;
+    // a (1b) group was committed to bar_y (completing the phase of parity y_parity) and its
+    // completion has not been seen yet
+    bool y_pending = false;
+    uint32_t y_parity = 0;
 
     // state S^T (row dv = lt, column blocks BPW wg .. BPW wg + BPW - 1) into TMEM, and its bf16
     // copy
@@ -362,30 +387,38 @@ __global__ void __launch_bounds__(NT, 1) gdn_prefill_kd_kernel(const __grid_cons
     constexpr uint32_t ID_3 = idesc_f16kind(128, 64, 0, 0, !F16);
 
     // the raw rows of chunk n (unit (token j, 8 dimensions 8c..8c+7), UNITS units per thread),
-    // requested one chunk ahead: they travel while the previous chunk's products run
+    // requested one chunk ahead, while the Gram runs: they travel while the rest of the chunk
+    // runs.  A row's 16 units sit on 16 consecutive lanes; the first unit of a thread lies in
+    // blocks 0-1 and the second, counted from the end, in blocks 3-2, so that every warp stores
+    // the same number of stacked key rows (block I writes 4 - I of them).
     constexpr int UNITS = C * 16 / NT;
+    static_assert(UNITS == 2, "unit map");
     uint4 rk8[UNITS], rq8[UNITS], rv8[UNITS];
     float rbeta = 0.f;   // beta of token tid (threads < 64), raw
-    auto load_rows = [&](int n) {
+    auto unit_of = [&](int it) { return it == 0 ? tid : 2 * NT - 1 - tid; };
+    auto load_unit = [&](int n, int it) {
+        const int64_t t0 = start + (int64_t)n * C;
+        const int ln = min(C, len - n * C);
+        const int u = unit_of(it), j = u >> 4, c = u & 15;
+        if (j < ln) {
+            const int64_t qk = ((t0 + j) * Hq + qh) * (int64_t)Dk;
+            rk8[it] = load_raw8(kg + qk, c, Dk, kvec);
+            rq8[it] = load_raw8(qg + qk, c, Dk, kvec);
+            rv8[it] = load_raw8(vg + ((t0 + j) * Hv + h) * (int64_t)Dv, c, Dv, vvec);
+        } else {
+            rk8[it] = rq8[it] = rv8[it] = make_uint4(0u, 0u, 0u, 0u);
+        }
+    };
+    auto load_beta = [&](int n) {
         const int64_t t0 = start + (int64_t)n * C;
         const int ln = min(C, len - n * C);
         if (tid < C) rbeta = (tid < ln && retrieval) ? __ldg(p.beta + (t0 + tid) * Hv + h) : 0.f;
-#pragma unroll
-        for (int it = 0; it < UNITS; ++it) {
-            const int u = tid + NT * it, j = u >> 4, c = u & 15;
-            if (j < ln) {
-                const int64_t qk = ((t0 + j) * Hq + qh) * (int64_t)Dk;
-                rk8[it] = load_raw8(kg + qk, c, Dk, kvec);
-                rq8[it] = load_raw8(qg + qk, c, Dk, kvec);
-                rv8[it] = load_raw8(vg + ((t0 + j) * Hv + h) * (int64_t)Dv, c, Dv, vvec);
-            } else {
-                rk8[it] = rq8[it] = rv8[it] = make_uint4(0u, 0u, 0u, 0u);
-            }
-        }
     };
     float *gn = reinterpret_cast<float *>(smem + OFF_GN);
     if (nc > 0) {
-        load_rows(0);
+        load_beta(0);
+#pragma unroll
+        for (int it = 0; it < UNITS; ++it) load_unit(0, it);
         stage_g(gn, p, start, min(C, len), h);
     }
 
@@ -399,33 +432,45 @@ __global__ void __launch_bounds__(NT, 1) gdn_prefill_kd_kernel(const __grid_cons
         cp_async_wait_all();
         __syncthreads();
         // ---- per-dimension cumulative log-decay (log2 units) into G2: thread = key dimension,
-        //      warpgroup wg scans tokens [CPW wg, CPW wg + CPW); each later segment then adds
-        //      the totals of the segments before it
+        //      warpgroup wg holds tokens [16 wg, 16 wg + 16) in registers, publishes their
+        //      total, and scans from the totals of the segments before it.  Segment wg is block
+        //      I = wg, so the same thread has the block's reference M_I (its eighth token) and,
+        //      in the last block, G_C.
         {
             const int d = lt;
-            float acc = 0.f;
-            const float ea = p.a_log ? expf(__ldg(p.a_log + h)) : 0.f;
-            const float dtb = p.a_log ? __ldg(p.dt_bias + h) : 0.f;
-#pragma unroll 8
-            for (int i = CPW * wg; i < CPW * wg + CPW; ++i) {
-                float g = gn[i * 128 + d];
-                if (i < ln && d < Dk) {
-                    if (p.a_log) g = -ea * gdn::softplus20(g + dtb);
-                    g = fmaxf(g, G_FLOOR);
-                }
-                acc += g * LOG2E;
-                G2[i * 128 + d] = acc;
+            float gv[CPW];
+#pragma unroll
+            for (int e = 0; e < CPW; ++e) gv[e] = gn[(CPW * wg + e) * 128 + d];
+            if (p.a_log) {
+                const float ea = expf(__ldg(p.a_log + h)), dtb = __ldg(p.dt_bias + h);
+#pragma unroll
+                for (int e = 0; e < CPW; ++e)
+                    if (CPW * wg + e < ln && d < Dk) gv[e] = -ea * gdn::softplus20(gv[e] + dtb);
             }
-        }
-        __syncthreads();
-        {
-            const int d = lt;
-            float base = 0.f;
-            for (int m = 0; m < wg; ++m) base += G2[(CPW * m + CPW - 1) * 128 + d];
+            float tot = 0.f;
+#pragma unroll
+            for (int e = 0; e < CPW; ++e) {
+                // positions past the request or past Dk hold the zeros staged for them
+                if (CPW * wg + e < ln && d < Dk) gv[e] = fmaxf(gv[e], G_FLOOR);
+                gv[e] *= LOG2E;
+                tot += gv[e];
+            }
+            if (wg < NWG - 1) vec[VEC_TOT + wg * 128 + d] = tot;
             __syncthreads();
-            if (wg > 0) {
-#pragma unroll 8
-                for (int i = CPW * wg; i < CPW * wg + CPW; ++i) G2[i * 128 + d] += base;
+            float acc = 0.f;
+            for (int m = 0; m < wg; ++m) acc += vec[VEC_TOT + m * 128 + d];
+            float mref = 0.f;
+#pragma unroll
+            for (int e = 0; e < CPW; ++e) {
+                acc += gv[e];
+                G2[(CPW * wg + e) * 128 + d] = acc;
+                if (e == 7) mref = acc;
+            }
+            vec[VEC_M2 + wg * 128 + d] = mref;
+            vec[VEC_EM + wg * 128 + d] = ex2_approx(mref);
+            if (wg == NWG - 1) {
+                vec[VEC_EC3 + d] = ex2_approx(acc - mref);
+                vec[VEC_GC + d] = ex2_approx(acc);
             }
         }
         if (tid < C) {
@@ -437,24 +482,13 @@ __global__ void __launch_bounds__(NT, 1) gdn_prefill_kd_kernel(const __grid_cons
             rowv[ROW_BETA + tid] = bt;
         }
         __syncthreads();
-        if (tid < 128) {
-            const int d = tid;
-            float m2[4];
-#pragma unroll
-            for (int I = 0; I < 4; ++I) m2[I] = G2[(16 * I + 7) * 128 + d];
-            const float gc = G2[63 * 128 + d];
-#pragma unroll
-            for (int I = 0; I < 4; ++I) {
-                vec[VEC_EM + I * 128 + d] = ex2_approx(m2[I]);
-                vec[VEC_M2 + I * 128 + d] = m2[I];
-            }
-#pragma unroll
-            for (int I2 = 1; I2 < 4; ++I2)
-#pragma unroll
-                for (int I = 0; I < I2; ++I)
-                    vec[VEC_CM + (I2 * (I2 - 1) / 2 + I) * 128 + d] = ex2_approx(m2[I2] - m2[I]);
-            vec[VEC_EC3 + d] = ex2_approx(gc - m2[3]);
-            vec[VEC_GC + d] = ex2_approx(gc);
+        // e^{M_I2 - M_I} for I < I2 (pair index I2 (I2 - 1) / 2 + I), per key dimension; the
+        // segment totals above are read by now
+        for (int u = tid; u < 6 * 128; u += NT) {
+            const int pr = u >> 7, d = u & 127;
+            const int I2 = pr < 1 ? 1 : (pr < 3 ? 2 : 3);
+            const int I = pr - I2 * (I2 - 1) / 2;
+            vec[VEC_CM + pr * 128 + d] = ex2_approx(vec[VEC_M2 + I2 * 128 + d] - vec[VEC_M2 + I * 128 + d]);
         }
         __syncthreads();
 
@@ -465,12 +499,12 @@ __global__ void __launch_bounds__(NT, 1) gdn_prefill_kd_kernel(const __grid_cons
         //      |q^||k^| rather than to the product, which near-orthogonal q and k make small.
 #pragma unroll
         for (int it = 0; it < UNITS; ++it) {
-            const int u = tid + NT * it, j = u >> 4, c = u & 15;
+            const int u = unit_of(it), j = u >> 4, c = u & 15;
             const int I = j >> 4;
-            float kx[8], qx[8], vx[8];
+            float kx[8], qx[8];
             unpack8<F16>(rk8[it], kx);
             unpack8<F16>(rq8[it], qx);
-            unpack8<F16>(rv8[it], vx);
+            const uint4 v8 = rv8[it];   // v enters its tile as it is (the tile has v's type)
             float ssk = 0.f, ssq = 0.f, sqk = 0.f;
 #pragma unroll
             for (int e = 0; e < 8; ++e) {
@@ -508,7 +542,7 @@ __global__ void __launch_bounds__(NT, 1) gdn_prefill_kd_kernel(const __grid_cons
             *reinterpret_cast<uint4 *>(smem + OFF_ASIDE + kb * ASIDE_KB + sw128(64 + j, ch)) = pack8<F16>(aq);
             *reinterpret_cast<uint4 *>(smem + OFF_KG + kb * TILE_KB + sw128(j, ch)) = pack8<F16>(kgm);
             *reinterpret_cast<uint4 *>(smem + OFF_QG + kb * TILE_KB + sw128(j, ch)) = pack8<F16>(qgm);
-            *reinterpret_cast<uint4 *>(smem + OFF_VT + kb * TILE_KB + sw128(j, ch)) = pack8<F16>(vx);
+            *reinterpret_cast<uint4 *>(smem + OFF_VT + kb * TILE_KB + sw128(j, ch)) = v8;
             // key operand of every block I2 >= I: k^ e^{M_I2 - G_j} = bk e^{M_I2 - M_I}; the
             // last one also gives k^ e^{G_C - G_j} = k^ e^{M_3 - G_j} e^{G_C - M_3}
 #pragma unroll
@@ -537,10 +571,7 @@ __global__ void __launch_bounds__(NT, 1) gdn_prefill_kd_kernel(const __grid_cons
         fence_proxy_async_smem();
         __syncthreads();
 
-        // ---- (G): all blocks' products in one MMA; then (1b) Y = S^T (Q^ e^G)^T, which needs
-        //      only the state's bf16 copy and this tile: it runs under the A/P build and the
-        //      solve, outside the commit that is waited for next (the later commits cover it);
-        //      then the next chunk's rows are requested
+        // ---- (G): all blocks' products in one MMA
         if (tid == 0) {
             tc_fence_after();
             const uint64_t dA = sdesc_sw128(sbase + OFF_ASIDE, 16, 1024);
@@ -550,63 +581,86 @@ __global__ void __launch_bounds__(NT, 1) gdn_prefill_kd_kernel(const __grid_cons
                 umma_bf16(tmem + TM_G, dA + (((kk >> 2) * ASIDE_KB + (kk & 3) * 32) >> 4),
                           dB + (((kk >> 2) * BCAT_KB + (kk & 3) * 32) >> 4), ID_G, kk > 0);
             umma_commit(bar);
+        }
+        // the next chunk's rows are requested while the Gram runs; the issuing thread's warp
+        // requests its own after the wait, when the others' requests have left the queue
+        auto load_next = [&] {
+            if (n + 1 < nc) {
+                load_beta(n + 1);
+#pragma unroll
+                for (int it = 0; it < UNITS; ++it) load_unit(n + 1, it);
+            }
+        };
+        if (warp != 0) load_next();
+        ok = cta_wait_mma(stall_bar ? stall_bar : bar, phase, flag, p.dev_status);
+        stall_bar = 0;
+        if (!ok) break;
+        if (warp == 0) load_next();
+        if (n + 1 < nc) stage_g(gn, p, t0 + C, min(C, len - (n + 1) * C), h);
+
+        // ---- (1b) Y = S^T (Q^ e^G)^T needs only the state's bf16 copy and this chunk's tile:
+        //      a thread of a warp that has no A/P load issues it while the tensor pipe is idle,
+        //      with a commit to its own barrier, which the output phase waits for
+        if (tid == Y_ISSUER) {
             const uint64_t dSB = sdesc_sw128(sbase + OFF_SB, 16, 1024);
             const uint64_t dQG = sdesc_sw128(sbase + OFF_QG, 16, 1024);
 #pragma unroll 1
             for (int kk = 0; kk < 8; ++kk)
                 umma_bf16(tmem + TM_Y, dSB + (((kk >> 2) * 16384 + (kk & 3) * 32) >> 4),
                           dQG + (((kk >> 2) * TILE_KB + (kk & 3) * 32) >> 4), ID_1B, kk > 0);
+            umma_commit(bar_y);
         }
-        if (n + 1 < nc) load_rows(n + 1);
-        ok = cta_wait_mma(stall_bar ? stall_bar : bar, phase, flag, p.dev_status);
-        stall_bar = 0;
-        if (!ok) break;
-        if (n + 1 < nc) stage_g(gn, p, t0 + C, min(C, len - (n + 1) * C), h);
+        y_pending = true;
+        y_parity = phase_y & 1;
 
-        // ---- A (key rows, fp32) and P (query rows, bf16 tile) from the Gram; TMEM lane = row;
-        //      a warp's lanes 0-15 and 16-31 hold two consecutive 16-blocks, of which warpgroup
-        //      wg (0 or 1) takes the (wg)th
-        if (wg < 2) {
-            const bool isq = (warp & 3) >= 2;
+        // ---- A (key rows, fp32) and P (query rows, bf16 tile) from the Gram; TMEM lane = row.
+        //      The lanes of warp quarter g4 hold the key (g4 < 2) or query rows of blocks 2h and
+        //      2h + 1 (h = g4 & 1), whose key columns are contiguous in the Gram: 3 loads of 16
+        //      columns from column 0 (h = 0) or 7 from column 48 (h = 1), dealt to the four
+        //      warpgroups; each load belongs to one block and serves that block's 16 lanes
+        {
+            const int g4 = warp & 3, hb = g4 & 1;
+            const bool isq = g4 >= 2;
             const int i = lt & 63;
             const int myI = i >> 4;
             const float bi = rowv[ROW_BETA + i];
             uint8_t *P = smem + OFF_P;
-            {
-                const int I = 2 * (warp & 1) + wg;
-                const int off = 8 * I * (I + 1);
+            const int nld = hb ? 7 : 3;
 #pragma unroll 1
-                for (int blk = 0; blk <= I; ++blk) {
-                    float x[16];
-                    tmem_ld16(tl + TM_G + off + 16 * blk, x);
-                    tmem_wait_ld();
-                    if (myI != I) continue;
-                    const int j0 = 16 * blk;
-                    if (!isq) {
-                        float *row = solve + (blk == I ? I : a_slot(I, blk)) * SOLVE_BLK + (i & 15) * SOLVE_LD;
+            for (int ld = wg; ld < nld; ld += NWG) {
+                const int col = (hb ? 48 : 0) + 16 * ld;
+                float x[16];
+                tmem_ld16(tl + TM_G + col, x);
+                tmem_wait_ld();
+                const int I = hb ? (ld < 3 ? 2 : 3) : (ld < 1 ? 0 : 1);
+                if (myI != I) continue;
+                const int blk = (col - 8 * I * (I + 1)) >> 4;   // key block of these columns
+                const int j0 = 16 * blk;
+                if (!isq) {
+                    float *row = solve + (blk == I ? I : a_slot(I, blk)) * SOLVE_BLK + (i & 15) * SOLVE_LD;
 #pragma unroll
-                        for (int q4 = 0; q4 < 4; ++q4) {
-                            float y[4];
+                    for (int q4 = 0; q4 < 4; ++q4) {
+                        float y[4];
 #pragma unroll
-                            for (int e = 0; e < 4; ++e) {
-                                const int j = j0 + 4 * q4 + e;
-                                y[e] = (retrieval && j < i) ? bi * x[4 * q4 + e] : 0.f;
-                            }
-                            *reinterpret_cast<float4 *>(row + 4 * q4) = make_float4(y[0], y[1], y[2], y[3]);
+                        for (int e = 0; e < 4; ++e) {
+                            const int j = j0 + 4 * q4 + e;
+                            y[e] = (retrieval && j < i) ? bi * x[4 * q4 + e] : 0.f;
                         }
-                    } else {
-                        // the diagonal from the raw bytes in fp32: rq_i rk_i (q_i . k_i)
-                        const float pii = rowv[ROW_QK + i];
-                        float y[16];
-#pragma unroll
-                        for (int e = 0; e < 16; ++e) y[e] = (j0 + e < i) ? x[e] : (j0 + e == i ? pii : 0.f);
-                        *reinterpret_cast<uint4 *>(P + sw128(i, 2 * blk)) = pack8<F16>(y);
-                        *reinterpret_cast<uint4 *>(P + sw128(i, 2 * blk + 1)) = pack8<F16>(y + 8);
+                        *reinterpret_cast<float4 *>(row + 4 * q4) = make_float4(y[0], y[1], y[2], y[3]);
                     }
+                } else {
+                    // the diagonal from the raw bytes in fp32: rq_i rk_i (q_i . k_i)
+                    const float pii = rowv[ROW_QK + i];
+                    float y[16];
+#pragma unroll
+                    for (int e = 0; e < 16; ++e) y[e] = (j0 + e < i) ? x[e] : (j0 + e == i ? pii : 0.f);
+                    *reinterpret_cast<uint4 *>(P + sw128(i, 2 * blk)) = pack8<F16>(y);
+                    *reinterpret_cast<uint4 *>(P + sw128(i, 2 * blk + 1)) = pack8<F16>(y + 8);
                 }
             }
-            // P blocks right of the row's own block are zero (the solve reads no A block there)
-            if (isq && myI == 2 * (warp & 1) + wg)
+            // P blocks right of the row's own block are zero (the solve reads no A block there);
+            // the last warpgroup writes them for the query rows
+            if (isq && wg == NWG - 1)
                 for (int blk = myI + 1; blk < 4; ++blk) {
                     *reinterpret_cast<uint4 *>(P + sw128(i, 2 * blk)) = make_uint4(0u, 0u, 0u, 0u);
                     *reinterpret_cast<uint4 *>(P + sw128(i, 2 * blk + 1)) = make_uint4(0u, 0u, 0u, 0u);
@@ -620,36 +674,45 @@ __global__ void __launch_bounds__(NT, 1) gdn_prefill_kd_kernel(const __grid_cons
         {
             const float *beta = rowv + ROW_BETA;
             uint8_t *tb = smem + OFF_TB;
-            if (tid < 64) {
-                // diagonal inverses D_I = (I + A_II)^-1, thread = column c of block I
-                const int I = tid >> 4, c = tid & 15;
-                const float *Ab = solve + I * SOLVE_BLK;
-                float x[16];
+            {
+                // diagonal inverses D_I = (I + A_II)^-1 by a column sweep: warps 4I .. 4I + 3
+                // take block I, and lane (row r, half) holds row r of columns c0 and c0 + 1
+                // (c0 = 4 (warp & 3) + 2 half).  At step m the lanes of row m, final by then,
+                // broadcast their entries and every later row subtracts A_rm times them.
+                const int lane = tid & 31;
+                const int I = warp >> 2, r = lane & 15;
+                const int c0 = 4 * (warp & 3) + 2 * (lane >> 4);
+                const float *Ar = solve + I * SOLVE_BLK + r * SOLVE_LD;
+                float a[16];
 #pragma unroll
-                for (int r = 0; r < 16; ++r) {
-                    float acc0 = (r == c) ? 1.f : 0.f, acc1 = 0.f;
+                for (int q4 = 0; q4 < 4; ++q4) {
+                    const float4 v = *reinterpret_cast<const float4 *>(Ar + 4 * q4);
+                    a[4 * q4] = v.x;
+                    a[4 * q4 + 1] = v.y;
+                    a[4 * q4 + 2] = v.z;
+                    a[4 * q4 + 3] = v.w;
+                }
+                float x0 = (r == c0) ? 1.f : 0.f, x1 = (r == c0 + 1) ? 1.f : 0.f;
 #pragma unroll
-                    for (int m = 0; m < r; ++m) {
-                        if (m & 1) acc1 = fmaf(-Ab[r * SOLVE_LD + m], x[m], acc1);
-                        else acc0 = fmaf(-Ab[r * SOLVE_LD + m], x[m], acc0);
+                for (int m = 0; m < 15; ++m) {
+                    const float y0 = __shfl_sync(0xffffffffu, x0, (lane & 16) | m);
+                    const float y1 = __shfl_sync(0xffffffffu, x1, (lane & 16) | m);
+                    if (m < r) {
+                        x0 = fmaf(-a[m], y0, x0);
+                        x1 = fmaf(-a[m], y1, x1);
                     }
-                    x[r] = acc0 + acc1;
                 }
                 float *Db = solve + (10 + I) * SOLVE_BLK;
-#pragma unroll
-                for (int r = 0; r < 16; ++r) Db[r * SOLVE_LD + c] = x[r];
-                const int j = 16 * I + c;
-                const float bj = beta[j];
-#pragma unroll
-                for (int r = 0; r < 16; ++r)
-                    *reinterpret_cast<uint16_t *>(tb + sw128(16 * I + r, j >> 3) + (j & 7) * 2) = elem16<F16>(x[r] * bj);
-            } else if (tid < 128) {
+                *reinterpret_cast<float2 *>(Db + r * SOLVE_LD + c0) = make_float2(x0, x1);
+                const int j = 16 * I + c0;
+                *reinterpret_cast<uint32_t *>(tb + sw128(16 * I + r, j >> 3) + (j & 7) * 2) =
+                    pack2<F16>(x0 * beta[j], x1 * beta[j + 1]);
                 // zero blocks above the diagonal: (I, J) with J > I, 16 rows x 32 bytes each
-                for (int u = tid - 64; u < 6 * 16 * 2; u += 64) {
+                for (int u = tid; u < 6 * 16 * 2; u += NT) {
                     const int pr = u >> 5, rr = (u >> 1) & 15, hf = u & 1;
-                    const int I = pr < 3 ? 0 : (pr < 5 ? 1 : 2);
-                    const int J = pr < 3 ? 1 + pr : (pr < 5 ? pr - 1 : 3);
-                    *reinterpret_cast<uint4 *>(tb + sw128(16 * I + rr, 2 * J + hf)) = make_uint4(0u, 0u, 0u, 0u);
+                    const int Iz = pr < 3 ? 0 : (pr < 5 ? 1 : 2);
+                    const int Jz = pr < 3 ? 1 + pr : (pr < 5 ? pr - 1 : 3);
+                    *reinterpret_cast<uint4 *>(tb + sw128(16 * Iz + rr, 2 * Jz + hf)) = make_uint4(0u, 0u, 0u, 0u);
                 }
             }
             __syncthreads();
@@ -798,7 +861,8 @@ __global__ void __launch_bounds__(NT, 1) gdn_prefill_kd_kernel(const __grid_cons
                 umma_bf16(tmem + TM_Z, dUB + ((kk * 32) >> 4), dP + ((kk * 32) >> 4), ID_3, kk > 0);
             umma_commit(bar);
         }
-        ok = cta_wait_mma(stall_bar ? stall_bar : bar, phase, flag, p.dev_status);
+        ok = cta_wait_mma(stall_bar ? stall_bar : bar, phase, flag, p.dev_status, bar_y, &phase_y);
+        if (ok) y_pending = false;
         stall_bar = 0;
         if (!ok) break;
 
@@ -879,6 +943,11 @@ __global__ void __launch_bounds__(NT, 1) gdn_prefill_kd_kernel(const __grid_cons
         const long long t0 = clock64();
         while (!mbar_try_wait(bar, (phase - 1) & 1))
             if (clock64() - t0 > (1ll << 24)) break;
+        if (y_pending) {
+            const long long t1 = clock64();
+            while (!mbar_try_wait(bar_y, y_parity))
+                if (clock64() - t1 > (1ll << 24)) break;
+        }
     }
     tc_fence_before();
     __syncthreads();
