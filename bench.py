@@ -554,12 +554,13 @@ def time_conv(gdn, case, steps, warmup, world, graph=False, nsets=1):
 
 
 # ---------------------------------------------------------------- CPU oracle
-def cpu_oracle_sample(case, target_s=10.0, repeats=1, threads=None):
+def cpu_oracle_sample(case, target_s=10.0, repeats=1, threads=None, warmup=0):
     """Time the float64 oracle on a bounded sample of the prefill workload: the first L
     tokens of the packed stream with every head; L is grown until one run takes ~target_s/8,
-    then scaled so that one run is ~target_s (at most the whole stream).  With repeats > 1
-    the calibrated sample is run that many times and the median rate is reported.  threads:
-    host threads for the oracle's (request, head) units (default: all cores)."""
+    then scaled so that one run is ~target_s (at most the whole stream).  The calibrated
+    sample then runs `warmup` times untimed and `repeats` times timed, and the median rate of
+    the timed runs is reported.  threads: host threads for the oracle's (request, head) units
+    (default: all cores)."""
     import oracle
     oracle.build()
     threads = oracle.max_threads() if threads is None else int(threads)
@@ -587,13 +588,15 @@ def cpu_oracle_sample(case, target_s=10.0, repeats=1, threads=None):
         L *= 2
         dt = run(L)
     L_final = max(1, min(total, int(L * (target_s / max(dt, 1e-6)))))
+    for _ in range(max(0, warmup)):
+        run(L_final)
     times = [run(L_final) for _ in range(max(1, repeats))]
     dt = statistics.median(times)
     return {"value": L_final / dt, "unit": "tokens/s", "cores": threads, "kind": "oracle",
             "sample": f"first {L_final} tokens of the packed stream run as one request, "
                       f"all {Hv} value heads ({Hq} query/key heads), float64, {dt:.2f} s per run"
                       + (f", median of {len(times)} runs" if len(times) > 1 else ""),
-            "runs": len(times)}
+            "runs": len(times), "warmup_runs": max(0, warmup)}
 
 
 def prefill_roofline(gdn, case, launch_ms, peaks, sm_mhz, traffic):
@@ -707,13 +710,14 @@ def main():
         if rank != 0:
             return 0
         case = make_case(args.workload)
-        # K steps of one calibrated sample each, sized so that the run stays near 90 s
-        per_step = min(2.5, max(0.2, 90.0 / max(1, args.steps)))
-        base = cpu_oracle_sample(case, target_s=per_step, repeats=args.steps)
+        # W untimed and K timed steps of one calibrated sample each, sized so that the run
+        # stays near 90 s
+        per_step = min(2.5, max(0.2, 90.0 / max(1, args.steps + args.warmup)))
+        base = cpu_oracle_sample(case, target_s=per_step, repeats=args.steps, warmup=args.warmup)
         val = base["value"]
         print(json.dumps({
             "impl": "reference", "metric": METRIC, "value": val, "unit": "tokens/s",
-            "n_gpus": args.gpus, "steps": args.steps, "warmup": 0,
+            "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": case.N / val * 1e3, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "f64", "data": "synthetic",
             "config": workload_config(case, args.workload), "cpu_baseline": base,
