@@ -242,14 +242,15 @@ __device__ __forceinline__ bool mbar_wait_bounded(uint32_t wbar, uint32_t parity
 
 // thread 0 waits (bounded) on `wbar` for the MMA group committed to it, and also on `wbar2`
 // when given; every thread gets the outcome.  (Checked builds with GDN_DEV_TEST_STALL pass,
-// once, a barrier that nothing arrives on instead of the commit barrier, so that the wait runs
-// out.)
+// once, a barrier that nothing arrives on instead of the commit barrier, with `fresh` set: a
+// barrier that has completed no phase is waited on with parity 0, since parity 1 would name
+// the phase before its first, which counts as complete.)
 __device__ __forceinline__ bool cta_wait_mma(uint32_t wbar, uint32_t &phase, volatile int *flag,
                                              int32_t *status, uint32_t wbar2 = 0,
-                                             uint32_t *phase2 = nullptr)
+                                             uint32_t *phase2 = nullptr, bool fresh = false)
 {
     if (threadIdx.x == 0) {
-        bool good = mbar_wait_bounded(wbar, phase & 1);
+        bool good = mbar_wait_bounded(wbar, fresh ? 0u : (phase & 1));
         if (good && wbar2) good = mbar_wait_bounded(wbar2, *phase2 & 1);
         if (!good && status) atomicOr(status, GDN_DEV_TIMEOUT);
         *flag = good ? 1 : 0;
@@ -328,8 +329,10 @@ __global__ void __launch_bounds__(NT, 1) gdn_prefill_kd_kernel(const __grid_cons
     const uint32_t bar_y = sbase + OFF_BAR + 40;   // commits of (1b), issued by Y_ISSUER
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + OFF_BAR + 8);
     volatile int *flag = reinterpret_cast<volatile int *>(smem + OFF_BAR + 12);
-    // checked builds, GDN_DEV_TEST_STALL: the first MMA wait of CTA 0 runs on a barrier that
-    // nothing arrives on, so it runs out and the CTA leaves through the timeout path
+    // checked builds, GDN_DEV_TEST_STALL: CTA 0's wait for its first (W, U~) group runs on a
+    // barrier that nothing arrives on, so it runs out and the CTA leaves through the timeout
+    // path while (1b) and, in a request of more than one chunk, the next decay tile's copies
+    // are in flight
     uint32_t stall_bar = (blockIdx.x == 0 && gdn::test_stall_requested(p.dev_status)) ? sbase + OFF_BAR + 16 : 0u;
     float *G2 = reinterpret_cast<float *>(smem + OFF_G2);
     float *solve = reinterpret_cast<float *>(smem + OFF_A);
@@ -592,8 +595,7 @@ __global__ void __launch_bounds__(NT, 1) gdn_prefill_kd_kernel(const __grid_cons
             }
         };
         if (warp != 0) load_next();
-        ok = cta_wait_mma(stall_bar ? stall_bar : bar, phase, flag, p.dev_status);
-        stall_bar = 0;
+        ok = cta_wait_mma(bar, phase, flag, p.dev_status);
         if (!ok) break;
         if (warp == 0) load_next();
         if (n + 1 < nc) stage_g(gn, p, t0 + C, min(C, len - (n + 1) * C), h);
@@ -780,7 +782,8 @@ __global__ void __launch_bounds__(NT, 1) gdn_prefill_kd_kernel(const __grid_cons
                 umma_bf16(tmem + TM_U, dVT + ((kk * 2048) >> 4), dTB + ((kk * 32) >> 4), ID_WU, kk > 0);
             umma_commit(bar);
         }
-        ok = cta_wait_mma(stall_bar ? stall_bar : bar, phase, flag, p.dev_status);
+        ok = cta_wait_mma(stall_bar ? stall_bar : bar, phase, flag, p.dev_status, 0, nullptr,
+                          stall_bar != 0);
         stall_bar = 0;
         if (!ok) break;
 
@@ -816,8 +819,7 @@ __global__ void __launch_bounds__(NT, 1) gdn_prefill_kd_kernel(const __grid_cons
             }
             umma_commit(bar);
         }
-        ok = cta_wait_mma(stall_bar ? stall_bar : bar, phase, flag, p.dev_status);
-        stall_bar = 0;
+        ok = cta_wait_mma(bar, phase, flag, p.dev_status);
         if (!ok) break;
 
         // ---- U^T -> bf16 A operand of (2), (3); the state's decay diag(e^{G_C}) on its columns
@@ -861,9 +863,8 @@ __global__ void __launch_bounds__(NT, 1) gdn_prefill_kd_kernel(const __grid_cons
                 umma_bf16(tmem + TM_Z, dUB + ((kk * 32) >> 4), dP + ((kk * 32) >> 4), ID_3, kk > 0);
             umma_commit(bar);
         }
-        ok = cta_wait_mma(stall_bar ? stall_bar : bar, phase, flag, p.dev_status, bar_y, &phase_y);
+        ok = cta_wait_mma(bar, phase, flag, p.dev_status, bar_y, &phase_y);
         if (ok) y_pending = false;
-        stall_bar = 0;
         if (!ok) break;
 
         // ---- outputs O^T = scale (Y + Z) (lane = dv, tokens CPW wg .. CPW wg + CPW - 1), then
@@ -949,6 +950,8 @@ __global__ void __launch_bounds__(NT, 1) gdn_prefill_kd_kernel(const __grid_cons
                 if (clock64() - t1 > (1ll << 24)) break;
         }
     }
+    // a CTA that left mid-chunk may still have the next decay tile's copies in flight
+    cp_async_wait_all();
     tc_fence_before();
     __syncthreads();
     tc_fence_after();

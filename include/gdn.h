@@ -88,7 +88,7 @@ enum {
     /* Checked builds only, set by the CALLER in *dev_status before a gdn_decode or a
      * chunked gdn_prefill call: the persistent decode kernel, or the chunked prefill
      * kernel's first q/k stage, posts 16 bytes more than its copies deliver (the per-key
-     * decay kernel's first CTA waits for its first MMA group on a barrier that nothing
+     * decay kernel's first CTA waits for its first W/U~ MMA group on a barrier that nothing
      * arrives on), so the waits run out after their bound (about a second), GDN_DEV_TIMEOUT
      * is set and the kernel returns.  Exercises the timeout path without a fault; ignored by
      * ordinary builds. */

@@ -124,10 +124,12 @@ def test_chunked_prefill_wait_runs_out_on_request(gdn, W):
 
 
 def test_per_key_prefill_wait_runs_out_on_request(gdn, W):
-    """The per-key tensor-core kernel: GDN_DEV_TEST_STALL makes CTA 0 wait for its first MMA
-    group on a barrier that nothing arrives on.  The wait runs out, GDN_DEV_TIMEOUT is set, the
-    CTA drains the group it issued, frees TMEM and returns; the other CTAs finish normally.  A
-    normal call on the same context then matches the product library bit for bit."""
+    """The per-key tensor-core kernel: GDN_DEV_TEST_STALL makes CTA 0 wait for its first W/U~
+    MMA group on a barrier that nothing arrives on.  By then (1b) is in flight on its own
+    barrier and, CTA 0's request having two chunks, so are the copies of the next chunk's decay
+    tile.  The wait runs out, GDN_DEV_TIMEOUT is set, the CTA drains both barriers and its
+    copies, frees TMEM and returns; the other CTAs finish normally.  A normal call on the same
+    context then matches the product library bit for bit."""
     c = W.make_prefill(78, [40, 90], 1, 4, 128, 128, init_std=0.05, qk_l2norm=True,
                        decay_per_key=True)
     assert gdn.prefill_uses_chunked(c.q.dtype, 4, 128, 128, decay_per_key=True)
