@@ -6,7 +6,9 @@
   activations' type, g and beta in fp32 -- g with Dk values per token and head in the
   per-key-dimension spelling --, states in fp32, cu_seqlens);
 * the DRAM traffic read from a committed ncu summary only while the kernel source, with the csrc
-  headers it includes, still has the digest the summary records.
+  headers it includes, still has the digest the summary records;
+* the oracle arm (`--impl reference`) printing one line with the contract's keys, its warm-up
+  steps run untimed.
 """
 import os
 import sys
@@ -75,3 +77,25 @@ def test_profile_traffic_keys(bench):
     assert bench.ncu_traffic("prefill_chunk_long_split.md", "prefill_chunk.cu") is None
     t = bench.ncu_traffic("prefill_chunk_long_split.md", "prefill_chunk.cu", "traffic_bytes_per_call")
     assert t is None or t > 0
+
+
+def test_reference_arm_prints_one_contract_line():
+    # the oracle arm runs on the host cores alone: W untimed and K timed steps, one JSON line
+    import json
+    import subprocess
+    r = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference",
+                        "--steps", "2", "--warmup", "3"], cwd=ROOT, capture_output=True,
+                       text=True, timeout=300)
+    assert r.returncode == 0, r.stderr[-2000:]
+    lines = [l for l in r.stdout.splitlines() if l.startswith("{")]
+    assert len(lines) == 1
+    d = json.loads(lines[0])
+    for key in ("impl", "metric", "value", "unit", "n_gpus", "steps", "warmup", "ms_per_step",
+                "higher_is_better", "scaling", "vs_baseline", "dtype", "data", "config",
+                "cpu_baseline", "e2e"):
+        assert key in d, key
+    assert d["impl"] == "reference" and d["steps"] == 2 and d["warmup"] == 3
+    assert d["value"] > 0 and d["e2e"]["value"] == d["value"]
+    assert d["e2e"]["h2d_bytes_per_step"] == 0 and d["e2e"]["d2h_bytes_per_step"] == 0
+    assert d["cpu_baseline"]["kind"] == "oracle" and d["cpu_baseline"]["cores"] >= 1
+    assert d["cpu_baseline"]["runs"] == 2 and d["cpu_baseline"]["warmup_runs"] == 3
